@@ -1,0 +1,222 @@
+"""CPU oracle for group-wise weight quantisation and the weight-only matmul.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` are the only callers.  The CUDA library
+never imports, links or calls anything here, and nothing here imports the
+CUDA library.  The arithmetic lives in ``wq_oracle.c`` (plain C, built with
+gcc, binary32 quantisation with round-half-to-even, binary64 dequantisation
+and matmul); this module only marshals numpy arrays in and out of it.
+
+Sources, by page title and section:
+  * "Quantization for LLM inference: FP8, INT4 (GPTQ, AWQ) and GGUF" --
+    "The minimum maths: scale and zero-point" (s, z, encode, decode) and
+    "Numerical example" (the 8-weight table and the storage count).
+  * "Quantization Methods Compared: INT8, GPTQ, AWQ, FP8, FP4 and KV-Cache
+    Quantization" -- "What quantisation does" (symmetric absmax INT8, the
+    outlier example, granularity and bits per weight).
+  * "Test-time quantization: quantising on the fly with no calibration
+    dataset" -- "The error of quantising an outlier with the wrong scale"
+    (rounding error at most half a scale).
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(page values, closed forms, brute force, invariants, an independent binary64
+matmul); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+from .accounting import bits_per_weight, model_gigabytes, example_bytes  # noqa: F401
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+EXACT = 0   # s and z kept in binary32 (the pages' arithmetic)
+STORED = 1  # s and z rounded to bf16 before encoding (the library's format)
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile wq_oracle.c into liboracle.so with gcc (no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-fno-fast-math", "-Wall", "-Wextra", "-o", _LIB + ".tmp", _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _bind(path: str):
+    """Open a compiled oracle library and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.oracle_quantize_int4.argtypes = [P, I64, I64, I64, I64, I, P, P, P]
+    lib.oracle_quantize_int8.argtypes = [P, I64, I64, I64, I64, I, P, P]
+    lib.oracle_pack_int4.argtypes = [P, I64, I64, P]
+    lib.oracle_unpack_int4.argtypes = [P, I64, I64, P]
+    lib.oracle_dequant_int4.argtypes = [P, P, P, I64, I64, I64, P]
+    lib.oracle_dequant_int8.argtypes = [P, P, I64, I64, I64, P]
+    lib.oracle_matmul.argtypes = [P, P, I64, I64, I64, P, P]
+    lib.oracle_f32_to_bf16_array.argtypes = [P, I64, P]
+    lib.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
+    lib.oracle_f32_to_bf16.restype = ctypes.c_uint16
+    lib.oracle_set_threads.argtypes = [I]
+    lib.oracle_max_threads.restype = I
+    for name in ("oracle_quantize_int4", "oracle_quantize_int8", "oracle_pack_int4",
+                 "oracle_unpack_int4", "oracle_dequant_int4", "oracle_dequant_int8",
+                 "oracle_matmul"):
+        getattr(lib, name).restype = I
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(build())
+    return _lib
+
+
+def swap_library(path):
+    """Make the wrappers call the oracle compiled at ``path`` (None: the default build).
+
+    Returns the previously bound library handle.  Used only by the mutation
+    tests, which compile deliberately broken copies of wq_oracle.c and check
+    that the pins reject them.
+    """
+    global _lib
+    old = _lib
+    _lib = _bind(path) if path is not None else None
+    return old
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle: {what} rejected its arguments")
+
+
+def set_threads(n: int) -> None:
+    """Number of OpenMP threads the oracle's outer loops use (rows / outputs)."""
+    _load().oracle_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def bf16_bits(values) -> np.ndarray:
+    """binary32 -> bf16 bit patterns (uint16), round to nearest, ties to even."""
+    v = np.ascontiguousarray(values, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint16)
+    _load().oracle_f32_to_bf16_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def bf16_value(bits) -> np.ndarray:
+    """bf16 bit patterns -> binary32 values (exact widening)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def quantize_int4(w, g: int, mode: int = STORED):
+    """Asymmetric INT4 per group of ``g`` consecutive weights along a row.
+
+    w: [N][K] binary32 values (bf16 weights widened exactly).
+    Returns (codes uint8 [N][K] in 0..15, s float32 [N][K/g], z float32 [N][K/g]);
+    s and z are the values the codes were encoded against (bf16-representable in
+    STORED mode).
+    """
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.empty((N, K), dtype=np.uint8)
+    s = np.empty((N, K // g), dtype=np.float32)
+    z = np.empty((N, K // g), dtype=np.float32)
+    _check(_load().oracle_quantize_int4(_ptr(w), N, K, K, g, mode, _ptr(codes), _ptr(s), _ptr(z)),
+           "quantize_int4")
+    return codes, s, z
+
+
+def pack_int4(codes) -> np.ndarray:
+    """[N][K] codes -> [N][K/2] bytes, code 2j in the low nibble of byte j."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    N, K = c.shape
+    out = np.empty((N, K // 2), dtype=np.uint8)
+    _check(_load().oracle_pack_int4(_ptr(c), N, K, _ptr(out)), "pack_int4")
+    return out
+
+
+def unpack_int4(packed, K: int) -> np.ndarray:
+    p = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = p.shape[0]
+    out = np.empty((N, K), dtype=np.uint8)
+    _check(_load().oracle_unpack_int4(_ptr(p), N, K, _ptr(out)), "unpack_int4")
+    return out
+
+
+def quantize_int8(w, g: int, mode: int = STORED):
+    """Symmetric absmax INT8 per group of ``g`` weights (g = K: per output channel).
+
+    Returns (codes int8 [N][K] in -127..127, s float32 [N][K/g]).
+    """
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.empty((N, K), dtype=np.int8)
+    s = np.empty((N, K // g), dtype=np.float32)
+    _check(_load().oracle_quantize_int8(_ptr(w), N, K, K, g, mode, _ptr(codes), _ptr(s)),
+           "quantize_int8")
+    return codes, s
+
+
+def dequant_int4(codes, s, z, g: int) -> np.ndarray:
+    """w_hat = s * (q - z) in binary64, [N][K]."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    N, K = c.shape
+    out = np.empty((N, K), dtype=np.float64)
+    _check(_load().oracle_dequant_int4(_ptr(c), _ptr(s), _ptr(z), N, K, g, _ptr(out)),
+           "dequant_int4")
+    return out
+
+
+def dequant_int8(codes, s, g: int) -> np.ndarray:
+    """w_hat = q * s in binary64, [N][K]."""
+    c = np.ascontiguousarray(codes, dtype=np.int8)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    N, K = c.shape
+    out = np.empty((N, K), dtype=np.float64)
+    _check(_load().oracle_dequant_int8(_ptr(c), _ptr(s), N, K, g, _ptr(out)), "dequant_int8")
+    return out
+
+
+def matmul(x, w_hat):
+    """y[m][n] = sum_k x[m][k] * w_hat[n][k] and a[m][n] = sum_k |x[m][k] * w_hat[n][k]|, binary64."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    w_hat = np.ascontiguousarray(w_hat, dtype=np.float64)
+    M, K = x.shape
+    N = w_hat.shape[0]
+    if w_hat.shape[1] != K:
+        raise ValueError("oracle.matmul: K mismatch")
+    y = np.empty((M, N), dtype=np.float64)
+    a = np.empty((M, N), dtype=np.float64)
+    _check(_load().oracle_matmul(_ptr(x), _ptr(w_hat), M, N, K, _ptr(y), _ptr(a)), "matmul")
+    return y, a
+
+
+def gemm_w4a16(x, codes, s, z, g: int):
+    """Reference for the W4A16 matmul: dequantise, then the binary64 matmul. Returns (y, a)."""
+    return matmul(x, dequant_int4(codes, s, z, g))
+
+
+def gemm_w8a16(x, codes, s, g: int):
+    """Reference for the W8A16 matmul: dequantise, then the binary64 matmul. Returns (y, a)."""
+    return matmul(x, dequant_int8(codes, s, g))

@@ -1,0 +1,76 @@
+"""Planted mistakes in the oracle must fail its pins.
+
+Each case compiles a copy of oracle/wq_oracle.c with one plausible mistake
+(a dropped term, a wrong sign, a wrong constant, a transposed index, another
+rounding rule), binds the wrappers to it, runs the pin tests and expects at
+least one of them to fail.  CPU only; the real oracle is rebound afterwards.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+MUTANTS = {
+    "zero_point_sign": ("nearbyintf(-mn / s)", "nearbyintf(mn / s)"),
+    "range_over_16": ("(mx - mn) / 15.0f", "(mx - mn) / 16.0f"),
+    "encode_minus_z": ("nearbyintf(wg[i] / s + z)", "nearbyintf(wg[i] / s - z)"),
+    "truncate_not_round": ("nearbyintf(wg[i] / s + z)", "floorf(wg[i] / s + z)"),
+    "ties_away_from_zero": ("nearbyintf(wg[i] / s + z)", "roundf(wg[i] / s + z)"),
+    "no_upper_clip": ("if (t > 15.0f) t = 15.0f;", ";"),
+    "z_not_rounded": ("float z = store_param(nearbyintf(-mn / s) + 0.0f, mode);",
+                      "float z = store_param(-mn / s, mode);"),
+    "int8_qmax_128": ("amax / 127.0f", "amax / 128.0f"),
+    "int8_no_round": ("float t = nearbyintf(wg[i] / s);", "float t = truncf(wg[i] / s);"),
+    "dequant_plus_z": ("((double)codes[n * K + k] - (double)z[n * G + k / g])",
+                       "((double)codes[n * K + k] + (double)z[n * G + k / g])"),
+    "dequant_group_index": ("s[n * G + k / g] * ((double)codes", "s[n * G + k % G] * ((double)codes"),
+    "matmul_transposed": ("x[m * K + k] * w_hat[n * K + k]", "x[m * K + k] * w_hat[k * N + n]"),
+    "matmul_drops_abs": ("aacc += fabs(p);", "aacc += p;"),
+    "pack_nibbles_swapped": ("(codes[n * K + 2 * j] & 0xf) | ((codes[n * K + 2 * j + 1] & 0xf) << 4)",
+                             "(codes[n * K + 2 * j + 1] & 0xf) | ((codes[n * K + 2 * j] & 0xf) << 4)"),
+    "bf16_truncates": ("if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u))) kept += 1u;", ";"),
+}
+
+PINS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+
+
+def _call_pin(fn):
+    import inspect
+    params = inspect.signature(fn).parameters
+    if not params:
+        fn()
+        return
+    # parametrised pins: run every parameter value the test module declares
+    marks = [m for m in getattr(fn, "pytestmark", []) if m.name == "parametrize"]
+    assert len(marks) == 1
+    name, values = marks[0].args
+    for v in values:
+        fn(**{name: v})
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_pins_reject_mutant(mutant, tmp_path):
+    src = open(oracle._SRC).read()
+    old, new = MUTANTS[mutant]
+    assert src.count(old) >= 1, f"mutation site for {mutant} not found"
+    path_c = os.path.join(tmp_path, "mutant.c")
+    path_so = os.path.join(tmp_path, "libmutant.so")
+    with open(path_c, "w") as f:
+        f.write(src.replace(old, new, 1))
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+                    "-o", path_so, path_c, "-lm"], check=True)
+    saved = oracle.swap_library(path_so)
+    failures = 0
+    try:
+        for fn in PINS:
+            try:
+                _call_pin(fn)
+            except Exception:
+                failures += 1
+    finally:
+        oracle.swap_library(None)
+        oracle._lib = saved
+    assert failures > 0, f"no pin caught mutant {mutant}"

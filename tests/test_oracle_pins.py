@@ -1,0 +1,350 @@
+"""Pins for the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: values the
+pages print (tests/golden/, cited there), closed forms, brute force over all
+codes on small groups, invariants that hold for any input, and independent
+library routines (numpy's binary64 matmul, torch's bf16 rounding).  These are
+CPU-only.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import wq_inputs
+from golden import read, scalar
+
+U_BF16 = 2.0 ** -8  # unit roundoff of bf16 (8 significant bits: half an ulp of 2^-7)
+
+
+# --------------------------------------------------------------------------
+# "Quantization for LLM inference ...", "Numerical example"
+# --------------------------------------------------------------------------
+
+def _worked():
+    sc, rows = read("int4_worked_example.txt")
+    w = np.array([[float(r[0]) for r in rows]], dtype=np.float32)
+    return sc, rows, w
+
+
+@pytest.mark.parametrize("mode", [oracle.EXACT, oracle.STORED])
+def test_worked_example_codes_scale_zero(mode):
+    sc, rows, w = _worked()
+    g = int(scalar(sc, "group"))
+    codes, s, z = oracle.quantize_int4(w, g, mode)
+    assert codes[0].tolist() == [int(r[3]) for r in rows]
+    assert [int(r[2]) for r in rows] == [int(r[3]) for r in rows]  # no code was clipped except 15.14
+    assert z[0, 0] == scalar(sc, "z_printed")
+    # s printed to 4 decimals: 0.1553.  Both the binary32 and the bf16 value round to it.
+    assert abs(float(s[0, 0]) - scalar(sc, "s_printed")) < 5e-5
+    # range and the unrounded zero-point as printed
+    assert abs((w.max() - w.min()) - scalar(sc, "range")) < 1e-6
+    assert abs(-w.min() / float(s[0, 0]) - scalar(sc, "z_unrounded_printed")) < 5e-3
+
+
+@pytest.mark.parametrize("mode", [oracle.EXACT, oracle.STORED])
+def test_worked_example_t_column(mode):
+    """t = w/s + z, printed to 2 decimals; the garbled -0.91 row uses the recomputed value."""
+    sc, rows, w = _worked()
+    codes, s, z = oracle.quantize_int4(w, 8, mode)
+    t = w[0].astype(np.float64) / float(s[0, 0]) + float(z[0, 0])
+    want = np.array([float(r[6]) for r in rows])
+    assert np.all(np.abs(t - want) < 0.006), (t, want)
+    # the printed value of the garbled row is not what the formula gives
+    printed = np.array([float(r[1]) for r in rows])
+    assert abs(t[5] - printed[5]) > 0.1 and abs(t[5] - 0.14) < 0.006
+
+
+@pytest.mark.parametrize("mode", [oracle.EXACT, oracle.STORED])
+def test_worked_example_reconstruction_and_mse(mode):
+    sc, rows, w = _worked()
+    codes, s, z = oracle.quantize_int4(w, 8, mode)
+    w_hat = oracle.dequant_int4(codes, s, z, 8)[0]
+    printed_hat = np.array([float(r[4]) for r in rows])
+    printed_err = np.array([float(r[5]) for r in rows])
+    # printed to 3 decimals from s ~ 0.1553; our s differs by < 3e-5, |q - z| <= 9
+    assert np.all(np.abs(w_hat - printed_hat) < 1e-3)
+    err = w_hat - w[0].astype(np.float64)
+    assert np.all(np.abs(err - printed_err) < 1e-3)
+    mse = float(np.mean(err ** 2))
+    assert abs(mse - scalar(sc, "mse_printed")) < 5e-5  # "MSE ~ 0.0015"
+
+
+def test_worked_example_storage():
+    sc, rows, w = _worked()
+    codes, s, z = oracle.quantize_int4(w, 8, oracle.STORED)
+    packed = oracle.pack_int4(codes)
+    assert packed.nbytes == 4  # 8 x 4 bits
+    assert oracle.example_bytes(8, 4, 16, 4) == scalar(sc, "storage_bytes_printed")
+
+
+# --------------------------------------------------------------------------
+# "Quantization Methods Compared ...", "What quantisation does"
+# --------------------------------------------------------------------------
+
+def _int8_fixture():
+    sc, _ = read("int8_absmax_example.txt")
+    w = np.array([[float(v) for v in sc["weights"][0]]], dtype=np.float32)
+    return sc, w
+
+
+@pytest.mark.parametrize("mode", [oracle.EXACT, oracle.STORED])
+def test_absmax_int8_example_sub_one_percent(mode):
+    sc, w = _int8_fixture()
+    codes, s = oracle.quantize_int8(w, w.shape[1], mode)
+    # s = max|w| / 127 (bf16-rounded in STORED mode)
+    assert abs(float(s[0, 0]) - 0.90 / 127) <= (U_BF16 if mode else 1e-7) * 0.90 / 127
+    w_hat = oracle.dequant_int8(codes, s, w.shape[1])[0]
+    rel = np.abs(w_hat - w[0]) / np.abs(w[0])
+    assert rel.max() * 100 < scalar(sc, "max_rel_error_before_percent_below")
+    assert codes[0].tolist() == [17, -71, 47, 127]
+
+
+@pytest.mark.parametrize("mode", [oracle.EXACT, oracle.STORED])
+def test_absmax_int8_outlier_31_percent(mode):
+    sc, w = _int8_fixture()
+    w5 = np.concatenate([w, [[scalar(sc, "outlier")]]], axis=1).astype(np.float32)
+    codes, s = oracle.quantize_int8(w5, w5.shape[1], mode)
+    if mode == oracle.EXACT:
+        assert abs(float(s[0, 0]) - scalar(sc, "step_with_outlier_printed")) < 5e-5
+    else:
+        assert abs(float(s[0, 0]) - 20.0 / 127) <= U_BF16 * 20.0 / 127
+    w_hat = oracle.dequant_int8(codes, s, w5.shape[1])[0]
+    rel = abs(w_hat[0] - 0.12) / 0.12
+    assert round(rel * 100) == scalar(sc, "rel_error_after_percent_printed")
+    assert codes[0, -1] == 127
+
+
+def test_storage_accounting():
+    sc, _ = read("storage_accounting.txt")
+    for b, g, sb, zb, v in sc["bits_per_weight"]:
+        assert oracle.bits_per_weight(int(b), int(g), int(sb), int(zb)) == float(v)
+    for b, g, sb, zb, v in sc["model_gb_70b"]:
+        assert round(oracle.model_gigabytes(70e9, int(b), int(g), int(sb), int(zb)), 1) == float(v)
+    for b, g, sb, zb, v in sc["fp16_gb_70b"]:
+        assert oracle.model_gigabytes(70e9, int(b), int(g), int(sb), int(zb)) == float(v)
+    fp16 = oracle.model_gigabytes(70e9, 16, 1, 0, 0)
+    assert round(fp16 / oracle.model_gigabytes(70e9, 4, 16, 8, 0), 2) == 3.56
+    for b, n, sb, zb, v in sc["example_bytes"]:
+        assert oracle.example_bytes(int(n), int(b), int(sb), int(zb)) == float(v)
+    # the library's format carries a bf16 zero-point as well
+    assert oracle.bits_per_weight(4, 128, 16, 16) == 4.25
+    assert oracle.bits_per_weight(4, 32, 16, 16) == 5.0
+
+
+@pytest.mark.parametrize("g", [32, 64, 128])
+def test_storage_matches_array_bytes(g):
+    w = wq_inputs.tiny_weight()
+    codes, s, z = oracle.quantize_int4(w.numpy(), g)
+    packed = oracle.pack_int4(codes)
+    nbytes = packed.nbytes + 2 * s.size + 2 * z.size  # bf16 s and z
+    N, K = w.shape
+    assert nbytes * 8 == N * K * oracle.bits_per_weight(4, g, 16, 16)
+
+
+# --------------------------------------------------------------------------
+# Error bound: "Test-time quantization ...", "The error of quantising an
+# outlier with the wrong scale" -- the rounding error is at most half a scale.
+# --------------------------------------------------------------------------
+
+def _groups(seed, n_groups, g):
+    gens = [
+        wq_inputs.uniform_weight(n_groups, g, seed),
+        wq_inputs.heavy_tail_weight(n_groups, g, seed + 1),
+        wq_inputs.tiny_weight(seed + 2, N=n_groups, K=g),
+        wq_inputs.llm_weight(n_groups, g, seed + 3, outlier_frac=0.01, outlier_mult=20,
+                             dtype=torch.float32),
+        wq_inputs.uniform_weight(n_groups, g, seed + 4, lo=-1e-3, hi=5.0),
+    ]
+    return np.concatenate([t.numpy() for t in gens], axis=0)
+
+
+@pytest.mark.parametrize("g", [8, 32, 128])
+def test_int4_error_at_most_half_scale_exact(g):
+    w = _groups(11, 2000 // g * 8, g)
+    codes, s, z = oracle.quantize_int4(w, g, oracle.EXACT)
+    err = np.abs(oracle.dequant_int4(codes, s, z, g) - w.astype(np.float64))
+    bound = 0.5 * np.repeat(s.astype(np.float64), g, axis=1) * (1 + 1e-5)
+    assert np.all(err <= bound)
+    # the bound is tight: some element reaches at least 0.45 s
+    assert np.max(err / bound) > 0.9
+
+
+@pytest.mark.parametrize("g", [8, 32, 128])
+def test_int4_error_bound_stored(g):
+    """bf16 s can be up to u below the binary32 s, so the clipped top element may exceed s/2 by 15u/(1-u) s."""
+    w = _groups(21, 2000 // g * 8, g)
+    codes, s, z = oracle.quantize_int4(w, g, oracle.STORED)
+    err = np.abs(oracle.dequant_int4(codes, s, z, g) - w.astype(np.float64))
+    k = 0.5 + 15 * U_BF16 / (1 - U_BF16)
+    bound = k * np.repeat(s.astype(np.float64), g, axis=1) * (1 + 1e-5)
+    assert np.all(err <= bound)
+    # non-clipped codes are still within half a scale
+    inner = (codes > 0) & (codes < 15)
+    assert np.all(err[inner] <= 0.5 * np.repeat(s.astype(np.float64), g, axis=1)[inner] * (1 + 1e-5))
+
+
+def test_int8_error_at_most_half_scale_exact():
+    w = _groups(31, 256, 64)
+    codes, s = oracle.quantize_int8(w, 64, oracle.EXACT)
+    err = np.abs(oracle.dequant_int8(codes, s, 64) - w.astype(np.float64))
+    assert np.all(err <= 0.5 * np.repeat(s.astype(np.float64), 64, axis=1) * (1 + 1e-5))
+
+
+# --------------------------------------------------------------------------
+# Brute force on small groups: every code is the nearest level (ties to even).
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [oracle.EXACT, oracle.STORED])
+def test_int4_codes_are_nearest_levels(mode):
+    w = _groups(41, 400, 8)
+    codes, s, z = oracle.quantize_int4(w, 8, mode)
+    # the scale and zero-point themselves, by the page's formulas
+    mn, mx = w.min(1).astype(np.float64), w.max(1).astype(np.float64)
+    s64 = s[:, 0].astype(np.float64)
+    rel = 1e-6 if mode == oracle.EXACT else U_BF16 * 1.0001
+    assert np.all(np.abs(s64 - (mx - mn) / 15) <= rel * (mx - mn) / 15)
+    assert np.all(np.abs(z[:, 0] - np.round(-mn / s64)) <= 1)  # round of binary32 vs binary64 quotient
+    assert np.all(z == np.round(z))
+    levels = np.arange(16, dtype=np.float64)
+    for i in range(w.shape[0]):
+        t = w[i].astype(np.float64) / s64[i] + float(z[i, 0])
+        d = np.abs(t[:, None] - levels[None, :])
+        best = d.min(axis=1)
+        chosen = d[np.arange(8), codes[i]]
+        assert np.all(chosen <= best + 1e-5), (i, t, codes[i])
+
+
+def test_int4_ties_round_to_even():
+    # min 0, max 15 -> s = 1 and z = 0 exactly; the other values sit on half-integers
+    w = np.array([[0.0, 15.0, 2.5, 3.5, 0.5, 1.5, 14.5, 7.5]], dtype=np.float32)
+    for mode in (oracle.EXACT, oracle.STORED):
+        codes, s, z = oracle.quantize_int4(w, 8, mode)
+        assert s[0, 0] == 1.0 and z[0, 0] == 0.0
+        assert codes[0].tolist() == [0, 15, 2, 4, 0, 2, 14, 8]
+
+
+def test_int8_codes_are_nearest_levels():
+    w = _groups(51, 200, 8)
+    codes, s = oracle.quantize_int8(w, 8, oracle.EXACT)
+    levels = np.arange(-127, 128, dtype=np.float64)
+    for i in range(w.shape[0]):
+        t = w[i].astype(np.float64) / float(s[i, 0])
+        d = np.abs(t[:, None] - levels[None, :])
+        chosen = d[np.arange(8), codes[i].astype(np.int64) + 127]
+        assert np.all(chosen <= d.min(axis=1) + 1e-5)
+    # the largest magnitude maps to +-127
+    amax_idx = np.abs(w).argmax(axis=1)
+    assert np.all(np.abs(codes[np.arange(w.shape[0]), amax_idx]) == 127)
+
+
+# --------------------------------------------------------------------------
+# Degenerate groups (the pages are silent; readings in the design notes)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", [oracle.EXACT, oracle.STORED])
+def test_degenerate_groups(mode):
+    w = np.zeros((4, 32), dtype=np.float32)
+    w[1, :] = 0.25
+    w[2, :] = -3.0
+    w[3, :] = 1.0e-30  # below bf16's smallest normal step for s
+    codes, s, z = oracle.quantize_int4(w, 32, mode)
+    w_hat = oracle.dequant_int4(codes, s, z, 32)
+    assert s[0, 0] == 1.0 and z[0, 0] == 0.0 and np.all(codes[0] == 0)
+    assert np.all(w_hat[0] == 0.0)
+    assert np.all(w_hat[1] == 0.25) and np.all(w_hat[2] == -3.0)
+    assert np.all(np.abs(w_hat[3] - 1e-30) <= 1e-30 * U_BF16)
+    c8, s8 = oracle.quantize_int8(w, 32, mode)
+    assert s8[0, 0] == 1.0 and np.all(c8[0] == 0)
+    assert np.all(c8[1] == 127) and np.all(c8[2] == -127)
+    assert np.all(np.abs(oracle.dequant_int8(c8, s8, 32)[1] - 0.25) <= 0.5 * s8[1, 0])
+
+
+def test_one_signed_groups_keep_codes_in_range():
+    w = wq_inputs.one_signed_weight(64, 128, 7).numpy()
+    codes, s, z = oracle.quantize_int4(w, 128, oracle.EXACT)
+    assert codes.min() >= 0 and codes.max() <= 15
+    assert np.all(z < 0)  # min > 0 puts the zero-point below code 0
+    err = np.abs(oracle.dequant_int4(codes, s, z, 128) - w.astype(np.float64))
+    assert np.all(err <= 0.5 * np.repeat(s.astype(np.float64), 128, axis=1) * (1 + 1e-5))
+
+
+# --------------------------------------------------------------------------
+# Stored parameters, packing and bf16 rounding
+# --------------------------------------------------------------------------
+
+def test_stored_params_are_bf16_values():
+    w = wq_inputs.llm_weight(64, 512, 3, dtype=torch.float32).numpy()
+    codes, s, z = oracle.quantize_int4(w, 128, oracle.STORED)
+    for p in (s, z):
+        assert np.array_equal(oracle.bf16_value(oracle.bf16_bits(p)), p)
+    c8, s8 = oracle.quantize_int8(w, 512, oracle.STORED)
+    assert np.array_equal(oracle.bf16_value(oracle.bf16_bits(s8)), s8)
+
+
+def test_bf16_rounding_matches_torch():
+    g = torch.Generator().manual_seed(5)
+    v = torch.randn(200000, generator=g) * torch.exp2(torch.randint(-60, 60, (200000,), generator=g).float())
+    # exact ties: a kept value plus half a bf16 ulp
+    # finite patterns only (inputs are finite by contract); both signs
+    base = torch.randint(0, 0x7f7f, (4096,), generator=g).to(torch.int32) << 16
+    base[::2] |= torch.tensor(-(1 << 31), dtype=torch.int32)
+    ties = (base | 0x8000).view(torch.float32)
+    denorm = torch.tensor([1e-40, -3e-39, 1.2e-38, 0.0, -0.0], dtype=torch.float32)
+    allv = torch.cat([v, ties, denorm])
+    ours = oracle.bf16_bits(allv.numpy())
+    theirs = allv.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, theirs)
+
+
+def test_pack_unpack_roundtrip_and_order():
+    g = torch.Generator().manual_seed(9)
+    codes = torch.randint(0, 16, (33, 64), generator=g).to(torch.uint8).numpy()
+    packed = oracle.pack_int4(codes)
+    assert packed.shape == (33, 32)
+    assert np.array_equal(oracle.unpack_int4(packed, 64), codes)
+    # code 2j in the low nibble, code 2j+1 in the high nibble
+    assert np.array_equal(packed & 0xF, codes[:, 0::2]) and np.array_equal(packed >> 4, codes[:, 1::2])
+
+
+# --------------------------------------------------------------------------
+# The binary64 matmul against numpy, and its closed forms
+# --------------------------------------------------------------------------
+
+def test_matmul_against_numpy():
+    g = torch.Generator().manual_seed(13)
+    M, N, K = 5, 37, 96
+    x = torch.randn(M, K, generator=g).double().numpy()
+    wh = torch.randn(N, K, generator=g).double().numpy()
+    y, a = oracle.matmul(x, wh)
+    assert y.shape == (M, N)
+    ref = x @ wh.T
+    aref = np.abs(x) @ np.abs(wh).T
+    assert np.all(np.abs(y - ref) <= 1e-12 * aref)
+    assert np.allclose(a, aref, rtol=1e-12, atol=0)
+
+
+def test_matmul_closed_forms():
+    K, N = 64, 9
+    g = torch.Generator().manual_seed(17)
+    wh = torch.randn(N, K, generator=g).double().numpy()
+    x = np.zeros((K, K))
+    x[np.arange(K), np.arange(K)] = 1.0  # unit vectors pick out columns of w_hat^T
+    y, a = oracle.matmul(x, wh)
+    assert np.array_equal(y, wh.T) and np.array_equal(a, np.abs(wh).T)
+
+
+def test_gemm_w4a16_reference_tiny():
+    w = wq_inputs.tiny_weight()
+    x = wq_inputs.plain_activations(1, 256, 0)
+    codes, s, z = oracle.quantize_int4(w.numpy(), 128)
+    y, a = oracle.gemm_w4a16(x.double().numpy(), codes, s, z, 128)
+    # independent evaluation: group-wise sum of s * sum x * (q - z), binary64, numpy
+    xs = x.double().numpy()[0]
+    ref = np.zeros(w.shape[0])
+    for gi in range(2):
+        sl = slice(gi * 128, (gi + 1) * 128)
+        ref += s[:, gi].astype(np.float64) * ((codes[:, sl].astype(np.float64) - z[:, gi:gi + 1]) @ xs[sl])
+    assert np.all(np.abs(y[0] - ref) <= 1e-12 * a[0])
