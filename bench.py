@@ -1,0 +1,492 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 decode path on a 70B-shaped model (synthetic weights).
+
+Workload ("full70b"): 80 layers x {qkv 8192->10240, o 8192->8192, gate+up
+8192->57344, down 28672->8192} = 68.45 G weights, bf16 ~ N(0, 0.02) drawn
+on the GPU from fixed seeds, quantised to INT4 with groups of 128 (bf16 s and
+z: 4.25 bits per weight, 36.4 GB), the bf16 weights then discarded.  A step is
+one decode step: every one of the 320 linears at M = 1 (one bf16 activation
+vector ~ N(0, 1) each), i.e. the whole packed model is streamed from HBM
+once; the weights (36.4 GB) exceed L2 (126 MB) by ~290x, so no L2 flush is
+needed between steps.
+
+The line printed carries
+  value      weight GB/s of the M = 1 decode step (algorithmic bytes: packed
+             codes, scales, zero-points, activations and outputs) over the
+             timed steps, CUDA events on the launch stream, max over ranks;
+  m128       the same 320 linears at M = 128 (TFLOP/s, fraction of the bf16
+             dense tensor peak);
+  rows       each hot-path step measured in the same run: INT4 quantisation of
+             the whole model, INT8 per-channel quantisation and the W8A16
+             matmul at K = N = 8192, the W4A16 matmul per linear shape;
+  e2e        the M = 1 step through the C ABI with the activations copied in
+             from pinned host memory and the outputs read back every step;
+  roofline   the dominant kernel (the W4A16 M = 1 matmul) against the
+             measured HBM copy bandwidth;
+  cpu_baseline  the CPU oracle on a bounded sample of the same workload.
+`--impl reference` times the CPU oracle alone on the same metric.  Several
+GPUs run independent replicas (weak scaling; no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import wq_inputs  # noqa: E402
+
+METRIC = "W4A16 weight GB/s and % HBM peak at M=1; TFLOP/s and % tensor peak at M=128"
+G = 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; only scalars cross ranks)
+# ---------------------------------------------------------------------------
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        self.index = vis.split(",")[local_rank] if vis else str(local_rank)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.index, f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append((float(p[1]), float(p[2]), float(p[3]), p[4], p[5], p[6], p[7], p[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        load = [r for r in rows if r[2] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for name, v in (("hw_slowdown", r[4]), ("hw_thermal_slowdown", r[5]),
+                            ("sw_thermal_slowdown", r[6]), ("sw_power_cap", r[7])):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in load),
+                "power_w_max": max(r[2] for r in load), "reasons": sorted(reasons), "samples": len(load)}
+
+
+# ---------------------------------------------------------------------------
+# the model
+# ---------------------------------------------------------------------------
+
+def linear_bytes(M, N, K, g=G):
+    """Algorithmic bytes of one W4A16 call: packed codes, bf16 s and z, bf16 x and y."""
+    return N * K // 2 + 2 * 2 * N * (K // g) + 2 * M * K + 2 * M * N
+
+
+class Model:
+    def __init__(self, layers: int, wq, device):
+        self.wq = wq
+        self.linears = []  # (name, K, N, q, s, z)
+        quant_ms = 0.0
+        quant_bytes = 0
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for layer in range(layers):
+            for j, (name, K, N) in enumerate(wq_inputs.FULL70B_LINEARS):
+                w = wq_inputs.llm_weight(N, K, wq_inputs.full70b_seed(layer, j), outlier_frac=0.0, device=device)
+                q = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
+                s = torch.empty((N, K // G), dtype=torch.bfloat16, device=device)
+                z = torch.empty((N, K // G), dtype=torch.bfloat16, device=device)
+                ev0.record()
+                wq.wq_quantize_int4(w, G, q, s, z)
+                ev1.record()
+                ev1.synchronize()
+                quant_ms += ev0.elapsed_time(ev1)
+                quant_bytes += N * K * 2 + N * K // 2 + 4 * N * (K // G)
+                del w
+                self.linears.append((name, K, N, q, s, z))
+        torch.cuda.empty_cache()
+        self.quant_ms, self.quant_bytes = quant_ms, quant_bytes
+        self.weights = sum(K * N for _, K, N, *_ in self.linears)
+
+    def buffers(self, M, device, seed=0):
+        xs, ys = [], []
+        for i, (name, K, N, *_) in enumerate(self.linears):
+            xs.append(wq_inputs.plain_activations(M, K, seed + i, device=device))
+            ys.append(torch.empty((M, N), dtype=torch.bfloat16, device=device))
+        return xs, ys
+
+    def step(self, xs, ys):
+        f = self.wq.wq_gemm_w4a16
+        for (name, K, N, q, s, z), x, y in zip(self.linears, xs, ys):
+            f(x, q, s, z, G, y=y)
+
+    def step_bytes(self, M):
+        return sum(linear_bytes(M, N, K) for _, K, N, *_ in self.linears)
+
+
+def time_steps(fn, steps, warmup, world):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def graph_of(fn):
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm the path once outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+# ---------------------------------------------------------------------------
+# rows measured beside the step
+# ---------------------------------------------------------------------------
+
+def int8_rows(wq, device, copies=8, reps=5):
+    """a2 + a6: INT8 per-channel quantise and W8A16 at K = N = 8192, rotating over copies (> 3x L2)."""
+    K = N = 8192
+    ws = [wq_inputs.block_outlier_weight(N, K, wq_inputs.SEEDS["gran"] + c, device=device) for c in range(copies)]
+    qs = [torch.empty((N, K), dtype=torch.int8, device=device) for _ in range(copies)]
+    ss = [torch.empty((N, 1), dtype=torch.bfloat16, device=device) for _ in range(copies)]
+    x = wq_inputs.activations(1, K, 4, device=device)
+    y = torch.empty((1, N), dtype=torch.bfloat16, device=device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for c in range(copies):
+        wq.wq_quantize_int8(ws[c], None, qs[c], ss[c])
+    torch.cuda.synchronize()
+    e0.record()
+    for r in range(reps):
+        for c in range(copies):
+            wq.wq_quantize_int8(ws[c], None, qs[c], ss[c])
+    e1.record()
+    e1.synchronize()
+    qms = e0.elapsed_time(e1) / (reps * copies)
+    del ws
+    torch.cuda.empty_cache()
+    for c in range(copies):
+        wq.wq_gemm_w8a16(x, qs[c], ss[c], None, y=y)
+    torch.cuda.synchronize()
+    e0.record()
+    for r in range(reps * 4):
+        for c in range(copies):
+            wq.wq_gemm_w8a16(x, qs[c], ss[c], None, y=y)
+    e1.record()
+    e1.synchronize()
+    gms = e0.elapsed_time(e1) / (reps * 4 * copies)
+    qbytes = N * K * 2 + N * K + 2 * N
+    gbytes = N * K + 2 * N + 2 * K + 2 * N
+    return ({"us": qms * 1e3, "GB_s": qbytes / (qms * 1e-3) / 1e9, "shape": "K=N=8192 bf16->int8 per-channel"},
+            {"us": gms * 1e3, "GB_s": gbytes / (gms * 1e-3) / 1e9, "shape": "K=N=8192 per-channel, M=1"})
+
+
+def per_linear_us(model, xs, ys, reps=3):
+    """Average device time of each linear shape at M = 1 (events around each call)."""
+    out = {}
+    for name, K, N in wq_inputs.FULL70B_LINEARS:
+        idx = [i for i, l in enumerate(model.linears) if l[0] == name]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            for i in idx:
+                _, K_, N_, q, s, z = model.linears[i]
+                model.wq.wq_gemm_w4a16(xs[i], q, s, z, G, y=ys[i])
+        e1.record()
+        e1.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (reps * len(idx))
+        out[name] = {"us": round(us, 2), "GB_s": round(linear_bytes(1, N, K) / (us * 1e-6) / 1e9, 1)}
+    return out
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(budget_s: float, model=None, seed=0):
+    """Time the CPU oracle's W4A16 path (unpack, dequantise, binary64 matmul) at M = 1 on
+    row blocks of the 70B-shaped linears until about budget_s seconds of CPU work.
+    Returns (GB/s of algorithmic bytes, cores used, sample description)."""
+    import oracle
+    oracle.set_threads(os.cpu_count() or 1)
+    cores = oracle.max_threads()
+    rows_per_block = 512
+    done_bytes, done_s, blocks = 0, 0.0, 0
+    li = 0
+    while done_s < budget_s:
+        name, K, N = wq_inputs.FULL70B_LINEARS[li % 4]
+        li += 1
+        r0 = (blocks * 997) % max(1, N - rows_per_block)
+        if model is not None:
+            _, K_, N_, q, s, z = [l for l in model.linears if l[0] == name][0]
+            packed = q[r0:r0 + rows_per_block].cpu().numpy()
+            sv = s[r0:r0 + rows_per_block].float().cpu().numpy()
+            zv = z[r0:r0 + rows_per_block].float().cpu().numpy()
+        else:
+            w = wq_inputs.llm_weight(rows_per_block, K, 7000 + blocks, outlier_frac=0.0).float().numpy()
+            codes, sv, zv = oracle.quantize_int4(w, G)
+            packed = oracle.pack_int4(codes)
+        x = wq_inputs.plain_activations(1, K, seed + blocks).double().numpy()
+        t0 = time.perf_counter()
+        codes = oracle.unpack_int4(packed, K)
+        oracle.gemm_w4a16(x, codes, sv, zv, G)
+        done_s += time.perf_counter() - t0
+        done_bytes += linear_bytes(1, rows_per_block, K)
+        blocks += 1
+    desc = (f"{blocks} blocks of {rows_per_block} rows of the 70B-shaped linears at M=1 "
+            f"({done_bytes / 1e9:.2f} GB of algorithmic bytes, {done_s:.1f} s)")
+    return done_bytes / done_s / 1e9, cores, desc
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    total_s, total_b = 0.0, 0.0
+    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup):
+        oracle_sample(per_step / 4, seed=100 + i)
+    gbs = []
+    for i in range(args.steps):
+        v, cores, desc = oracle_sample(per_step, seed=i)
+        gbs.append(v)
+    value = statistics.mean(gbs)
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "full70b decode step, W4A16 g128, M=1 (bounded CPU sample per step)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": desc + " per step"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["wq", "reference"], default="wq")
+    ap.add_argument("--layers", type=int, default=wq_inputs.FULL70B_LAYERS)
+    ap.add_argument("--m128-steps", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-graph", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, local = dist_init()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    import group_wise_weight_b200 as wq
+    wq.lib()  # fails loudly if the CUDA library is missing
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+
+    model = Model(args.layers, wq, device)
+    weights_total = model.weights
+    xs1, ys1 = model.buffers(1, device)
+    bytes1 = model.step_bytes(1)
+    launches_per_step = len(model.linears)
+
+    step1 = (lambda: model.step(xs1, ys1))
+    g1 = None if args.no_graph else graph_of(step1)
+    run1 = (lambda: g1.replay()) if g1 is not None else step1
+
+    with Clocks(local) as clk:
+        ms1 = time_steps(run1, args.steps, args.warmup, world)
+    clocks = clk.summary()
+    ms1 = reduce_max(ms1, world)
+    t_step = ms1 / args.steps
+    value = reduce_sum(bytes1 * args.steps, world) / (ms1 * 1e-3) / 1e9
+
+    # the same step through the C ABI with host buffers: pinned H2D of every activation, D2H of every output
+    x_host = torch.cat([x.reshape(-1) for x in xs1]).cpu().pin_memory()
+    y_host = torch.empty(sum(y.numel() for y in ys1), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x_host, device=device)
+    y_dev = torch.empty_like(y_host, device=device)
+    xs_view, ys_view, o1, o2 = [], [], 0, 0
+    for x, y in zip(xs1, ys1):
+        xs_view.append(x_dev[o1:o1 + x.numel()].view_as(x))
+        ys_view.append(y_dev[o2:o2 + y.numel()].view_as(y))
+        o1 += x.numel()
+        o2 += y.numel()
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        model.step(xs_view, ys_view)
+        y_host.copy_(y_dev, non_blocking=True)
+
+    ms_e2e = reduce_max(time_steps(e2e_step, args.steps, args.warmup, world), world)
+    e2e_value = reduce_sum(bytes1 * args.steps, world) / (ms_e2e * 1e-3) / 1e9
+
+    lin = per_linear_us(model, xs1, ys1)
+
+    # M = 128 over the same model
+    m128_steps = args.m128_steps if args.m128_steps is not None else max(3, args.steps // 4)
+    xs128, ys128 = model.buffers(128, device, seed=10_000)
+    step128 = (lambda: model.step(xs128, ys128))
+    g128 = None if args.no_graph else graph_of(step128)
+    run128 = (lambda: g128.replay()) if g128 is not None else step128
+    ms128 = reduce_max(time_steps(run128, m128_steps, 3, world), world)
+    flops128 = 2.0 * 128 * weights_total
+    tflops128 = reduce_sum(flops128 * m128_steps, world) / (ms128 * 1e-3) / 1e12
+    del xs128, ys128, g128
+    torch.cuda.empty_cache()
+
+    q8_row, g8_row = int8_rows(wq, device)
+
+    quant_gbs = model.quant_bytes / (model.quant_ms * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1:
+        v, cores, desc = oracle_sample(args.cpu_seconds, model=model)
+        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    per_gpu_gbs = bytes1 / (t_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 x int4 -> f32 accumulate", "data": "synthetic",
+        "config": {"workload": "full70b decode step: 80 layers x (qkv 8192->10240, o 8192->8192, "
+                               "gate+up 8192->57344, down 28672->8192), W4A16 g128 bf16 s/z, M=1",
+                   "layers": args.layers, "linears_per_step": launches_per_step, "weights": weights_total,
+                   "bytes_per_step": bytes1, "cuda_graph": g1 is not None,
+                   "l2": "inputs larger than L2 (%.1f GB of packed weights per step vs 126 MB L2)" % (bytes1 / 1e9),
+                   "parallelism": f"replicas x{world}"},
+        "pct_hbm_peak": round(100 * per_gpu_gbs / peaks["hbm_gbs"], 1),
+        "m128": {"tflops": round(tflops128, 1), "ms_per_step": round(ms128 / m128_steps, 3),
+                 "pct_bf16_peak": round(100 * tflops128 / world / peaks["bf16_tflops_sustained"], 1),
+                 "peak_tflops": peaks["bf16_tflops_sustained"], "peak_kind": "sustained (kernel inside a long step)",
+                 "steps": m128_steps},
+        "rows": {
+            "a1_quantize_int4": {"GB_s": round(quant_gbs, 1), "ms_total": round(model.quant_ms, 2),
+                                 "shape": "all 320 linears, bf16 -> int4 g128"},
+            "a2_quantize_int8": {k: (round(v, 2) if isinstance(v, float) else v) for k, v in q8_row.items()},
+            "a4_w4a16_m1_per_linear": lin,
+            "a5_w4a16_m128": {"tflops": round(tflops128 / world, 1)},
+            "a6_w8a16_m1": {k: (round(v, 2) if isinstance(v, float) else v) for k, v in g8_row.items()},
+        },
+        "roofline": {"bound": "hbm", "kernel": "gemv_w4a16 (M=1)", "achieved": round(per_gpu_gbs, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(per_gpu_gbs / peaks["hbm_gbs"], 4),
+                     "peak_source": peaks["source"], "traffic": None,
+                     "bytes_per_launch_avg": bytes1 // launches_per_step},
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": x_host.numel() * 2,
+                "d2h_bytes_per_step": y_host.numel() * 2, "ms_per_step": round(ms_e2e / args.steps, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g1
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,214 @@
+"""Python binding of libwq (include/wq.h): group-wise weight quantisation and the
+dequant-fused weight-only matmul on NVIDIA B200.
+
+Argument marshalling only.  Every step runs in the CUDA kernels of
+``libwq.so``; this module passes device pointers, sizes and the current CUDA
+stream through ctypes and allocates output tensors with torch when the
+caller does not pass them.  There is no CPU path: the functions require CUDA
+tensors and raise if ``libwq.so`` is missing.
+
+bf16 scales and zero-points are returned as ``torch.bfloat16`` tensors (the
+C ABI's uint16 bit patterns).  Function names are those of the C ABI.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwq.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "wq.h")
+
+WQ_OK = 0
+WQ_ERR_ARG = -1
+WQ_ERR_SHAPE = -2
+WQ_ERR_ALIGN = -3
+WQ_ERR_UNSUPPORTED = -4
+WQ_ERR_CUDA = -5
+WQ_ERR_WORKSPACE = -6
+WQ_ERR_DEVICE_TIMEOUT = -7
+WQ_F32 = 0
+WQ_BF16 = 1
+
+_lib = None
+
+
+class WQError(RuntimeError):
+    """A libwq call returned a status other than WQ_OK."""
+
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{wq_status_str(status)} ({detail})" if detail else wq_status_str(status))
+        self.status = status
+
+
+def lib():
+    """The loaded libwq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libwq.so not found at {LIB_PATH}: build it with "
+                               "`python -m group_wise_weight_b200.build` (or __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.wq_status_str.argtypes = [I]
+        L.wq_status_str.restype = ctypes.c_char_p
+        L.wq_last_error.argtypes = []
+        L.wq_last_error.restype = ctypes.c_char_p
+        L.wq_version.restype = I
+        L.wq_quantize_int4.argtypes = [P, I, I64, I64, I64, I, P, P, P, P]
+        L.wq_quantize_int4.restype = I
+        L.wq_quantize_int8.argtypes = [P, I, I64, I64, I64, I, P, P, P]
+        L.wq_quantize_int8.restype = I
+        L.wq_gemm_workspace_bytes.argtypes = [I64, I64, I64, I, I]
+        L.wq_gemm_workspace_bytes.restype = SZ
+        L.wq_gemm_w4a16.argtypes = [P, I64, I64, I64, P, P, P, I, P, P, SZ, P]
+        L.wq_gemm_w4a16.restype = I
+        L.wq_gemm_w8a16.argtypes = [P, I64, I64, I64, P, P, I, P, P, SZ, P]
+        L.wq_gemm_w8a16.restype = I
+        L.wq_device_status.argtypes = [P]
+        L.wq_device_status.restype = I
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/wq.h declares."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wq_[a-z0-9_]+)\s*\(", text)))
+
+
+def wq_status_str(status: int) -> str:
+    return lib().wq_status_str(int(status)).decode()
+
+
+def wq_last_error() -> str:
+    return lib().wq_last_error().decode()
+
+
+def wq_version() -> int:
+    return int(lib().wq_version())
+
+
+def _check(rc: int):
+    if rc != WQ_OK:
+        raise WQError(rc, wq_last_error())
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (libwq has no CPU path)")
+    return t.data_ptr()
+
+
+def _dense(t: torch.Tensor, name: str):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def wq_quantize_int4(w: torch.Tensor, g: int = 128, qweight=None, scales=None, zeros=None, stream=None):
+    """Asymmetric INT4 per group of g weights along K.  w: [N][K] (row stride >= K) fp32 or bf16 on CUDA.
+
+    Returns (qweight uint8 [N][K/2], scales bf16 [N][K/g], zeros bf16 [N][K/g]).
+    """
+    if w.dim() != 2 or w.stride(1) != 1:
+        raise ValueError("w must be a 2-D tensor with unit stride along K")
+    wtype = {torch.float32: WQ_F32, torch.bfloat16: WQ_BF16}.get(w.dtype)
+    if wtype is None:
+        raise TypeError("w must be float32 or bfloat16")
+    N, K = w.shape
+    dev = w.device
+    qweight = torch.empty((N, K // 2), dtype=torch.uint8, device=dev) if qweight is None else qweight
+    scales = torch.empty((N, K // g), dtype=torch.bfloat16, device=dev) if scales is None else scales
+    zeros = torch.empty((N, K // g), dtype=torch.bfloat16, device=dev) if zeros is None else zeros
+    for t, n in ((qweight, "qweight"), (scales, "scales"), (zeros, "zeros")):
+        _dense(t, n)
+    _check(lib().wq_quantize_int4(_dev(w, "w"), wtype, N, K, w.stride(0), int(g), _dev(qweight, "qweight"),
+                                  _dev(scales, "scales"), _dev(zeros, "zeros"), _stream_handle(stream)))
+    return qweight, scales, zeros
+
+
+def wq_quantize_int8(w: torch.Tensor, g: int | None = None, qweight=None, scales=None, stream=None):
+    """Symmetric absmax INT8 per group of g weights (g=None or K: per output channel).
+
+    Returns (qweight int8 [N][K], scales bf16 [N][K/g]).
+    """
+    if w.dim() != 2 or w.stride(1) != 1:
+        raise ValueError("w must be a 2-D tensor with unit stride along K")
+    wtype = {torch.float32: WQ_F32, torch.bfloat16: WQ_BF16}.get(w.dtype)
+    if wtype is None:
+        raise TypeError("w must be float32 or bfloat16")
+    N, K = w.shape
+    g = K if g is None else int(g)
+    dev = w.device
+    qweight = torch.empty((N, K), dtype=torch.int8, device=dev) if qweight is None else qweight
+    scales = torch.empty((N, K // g), dtype=torch.bfloat16, device=dev) if scales is None else scales
+    _dense(qweight, "qweight")
+    _dense(scales, "scales")
+    _check(lib().wq_quantize_int8(_dev(w, "w"), wtype, N, K, w.stride(0), g, _dev(qweight, "qweight"),
+                                  _dev(scales, "scales"), _stream_handle(stream)))
+    return qweight, scales
+
+
+def wq_gemm_workspace_bytes(M: int, N: int, K: int, g: int, wbits: int) -> int:
+    return int(lib().wq_gemm_workspace_bytes(int(M), int(N), int(K), int(g), int(wbits)))
+
+
+def _workspace(workspace, need: int, dev):
+    if need == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def wq_gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, g: int = 128,
+                  y=None, workspace=None, stream=None) -> torch.Tensor:
+    """y[M][N] = x[M][K] @ w_hat^T with w_hat = s * (q - z) dequantised in-kernel.  bf16 in, bf16 out."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    _dense(x, "x")
+    M, K = x.shape
+    N = qweight.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dense(y, "y")
+    need = wq_gemm_workspace_bytes(M, N, K, g, 4)
+    workspace, ws_bytes = _workspace(workspace, need, x.device)
+    _check(lib().wq_gemm_w4a16(_dev(x, "x"), M, N, K, _dev(qweight, "qweight"), _dev(scales, "scales"),
+                               _dev(zeros, "zeros"), int(g), _dev(y, "y"),
+                               workspace.data_ptr() if workspace is not None else None, ws_bytes,
+                               _stream_handle(stream)))
+    return y
+
+
+def wq_gemm_w8a16(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, g: int | None = None, y=None,
+                  workspace=None, stream=None) -> torch.Tensor:
+    """y[M][N] = x[M][K] @ w_hat^T with w_hat = q * s dequantised in-kernel.  g=None: per output channel."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    _dense(x, "x")
+    M, K = x.shape
+    N = qweight.shape[0]
+    g = K if g is None else int(g)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dense(y, "y")
+    need = wq_gemm_workspace_bytes(M, N, K, g, 8)
+    workspace, ws_bytes = _workspace(workspace, need, x.device)
+    _check(lib().wq_gemm_w8a16(_dev(x, "x"), M, N, K, _dev(qweight, "qweight"), _dev(scales, "scales"), g,
+                               _dev(y, "y"), workspace.data_ptr() if workspace is not None else None, ws_bytes,
+                               _stream_handle(stream)))
+    return y
+
+
+def wq_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word as a WQ_* code."""
+    return int(lib().wq_device_status(_stream_handle(stream)))

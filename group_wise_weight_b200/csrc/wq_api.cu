@@ -1,0 +1,170 @@
+// wq_api.cu -- the C ABI of libwq (declared in include/wq.h): argument
+// checks, kernel choice and launch.  Kernel choice is a pure function of
+// (M, N, K, g); nothing is cached between calls except the per-device status
+// word used by bounded waits.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "wq_common.cuh"
+#include "wq_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int status, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+
+int fail(int status, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return status;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_launch(const char *what)
+{
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+    return WQ_OK;
+}
+
+// Shared checks of the quantisers.
+int check_quantize(const char *what, const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g,
+                   const void *q, const void *s, const void *z, bool int8)
+{
+    if (!w || !q || !s || (!int8 && !z)) return fail(WQ_ERR_ARG, "%s: null pointer", what);
+    if (N <= 0 || K <= 0 || ldw <= 0) return fail(WQ_ERR_ARG, "%s: N, K and ldw must be positive", what);
+    if (wtype != WQ_F32 && wtype != WQ_BF16) return fail(WQ_ERR_UNSUPPORTED, "%s: wtype %d", what, wtype);
+    const bool g_ok = g == 32 || g == 64 || g == 128 || (int8 && (int64_t)g == K);
+    if (!g_ok) return fail(WQ_ERR_UNSUPPORTED, "%s: group size %d", what, g);
+    if (K % 32 != 0 || K % g != 0 || ldw < K)
+        return fail(WQ_ERR_SHAPE, "%s: need K %% 32 == 0, K %% g == 0, ldw >= K (K=%lld g=%d ldw=%lld)", what,
+                    (long long)K, g, (long long)ldw);
+    if (N > 0x7fffffffLL) return fail(WQ_ERR_SHAPE, "%s: N too large", what);
+    if (ldw % 8 != 0 || !aligned16(w) || !aligned16(q) || !aligned16(s) || (z && !aligned16(z)))
+        return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned and ldw a multiple of 8", what);
+    return WQ_OK;
+}
+
+int check_gemm(const char *what, const void *x, int64_t M, int64_t N, int64_t K, const void *q, const void *s,
+               const void *z, int g, const void *y, bool int8)
+{
+    if (!x || !q || !s || (!int8 && !z) || !y) return fail(WQ_ERR_ARG, "%s: null pointer", what);
+    if (M <= 0 || N <= 0 || K <= 0) return fail(WQ_ERR_ARG, "%s: M, N and K must be positive", what);
+    const bool g_ok = g == 32 || g == 64 || g == 128 || (int8 && (int64_t)g == K);
+    if (!g_ok) return fail(WQ_ERR_UNSUPPORTED, "%s: group size %d", what, g);
+    if (K % 32 != 0 || K % g != 0)
+        return fail(WQ_ERR_SHAPE, "%s: need K %% 32 == 0 and K %% g == 0 (K=%lld g=%d)", what, (long long)K, g);
+    if (N > 0x7fffffffLL * 8 || M > 0x7fffffffLL) return fail(WQ_ERR_SHAPE, "%s: M or N too large", what);
+    if (!aligned16(x) || !aligned16(q) || !aligned16(s) || (z && !aligned16(z)) || !aligned16(y))
+        return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned", what);
+    return WQ_OK;
+}
+
+}  // namespace
+
+// Per-device status word written by kernels whose waits ran out.
+__device__ int g_wq_device_status = 0;
+
+extern "C" {
+
+const char *wq_status_str(int status)
+{
+    switch (status) {
+    case WQ_OK: return "WQ_OK";
+    case WQ_ERR_ARG: return "WQ_ERR_ARG: null pointer or non-positive size";
+    case WQ_ERR_SHAPE: return "WQ_ERR_SHAPE: K, g or ldw do not fit the layout";
+    case WQ_ERR_ALIGN: return "WQ_ERR_ALIGN: pointer or leading dimension misaligned";
+    case WQ_ERR_UNSUPPORTED: return "WQ_ERR_UNSUPPORTED: group size or dtype not supported";
+    case WQ_ERR_CUDA: return "WQ_ERR_CUDA: CUDA error";
+    case WQ_ERR_WORKSPACE: return "WQ_ERR_WORKSPACE: workspace missing or too small";
+    case WQ_ERR_DEVICE_TIMEOUT: return "WQ_ERR_DEVICE_TIMEOUT: a kernel gave up on a bounded wait";
+    default: return "unknown status";
+    }
+}
+
+const char *wq_last_error(void) { return g_last_error.c_str(); }
+
+int wq_version(void) { return 100; }
+
+int wq_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *qweight,
+                     uint16_t *scales, uint16_t *zeros, void *stream)
+{
+    g_last_error.clear();
+    int rc = check_quantize("wq_quantize_int4", w, wtype, N, K, ldw, g, qweight, scales, zeros, false);
+    if (rc != WQ_OK) return rc;
+    wq::launch_quantize_int4(w, wtype, N, K, ldw, g, qweight, scales, zeros, static_cast<cudaStream_t>(stream));
+    return check_launch("wq_quantize_int4");
+}
+
+int wq_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, int8_t *qweight,
+                     uint16_t *scales, void *stream)
+{
+    g_last_error.clear();
+    int rc = check_quantize("wq_quantize_int8", w, wtype, N, K, ldw, g, qweight, scales, nullptr, true);
+    if (rc != WQ_OK) return rc;
+    wq::launch_quantize_int8(w, wtype, N, K, ldw, g, qweight, scales, static_cast<cudaStream_t>(stream));
+    return check_launch("wq_quantize_int8");
+}
+
+size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits)
+{
+    (void)M; (void)N; (void)K; (void)g; (void)wbits;
+    return 0;
+}
+
+int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *qweight,
+                  const uint16_t *scales, const uint16_t *zeros, int g, uint16_t *y, void *workspace,
+                  size_t ws_bytes, void *stream)
+{
+    g_last_error.clear();
+    int rc = check_gemm("wq_gemm_w4a16", x, M, N, K, qweight, scales, zeros, g, y, false);
+    if (rc != WQ_OK) return rc;
+    const size_t need = wq_gemm_workspace_bytes(M, N, K, g, 4);
+    if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+        return fail(WQ_ERR_WORKSPACE, "wq_gemm_w4a16: need %zu workspace bytes", need);
+    wq::launch_gemv_w4a16(x, M, N, K, qweight, scales, zeros, g, y, static_cast<cudaStream_t>(stream));
+    return check_launch("wq_gemm_w4a16");
+}
+
+int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *qweight,
+                  const uint16_t *scales, int g, uint16_t *y, void *workspace, size_t ws_bytes, void *stream)
+{
+    g_last_error.clear();
+    int rc = check_gemm("wq_gemm_w8a16", x, M, N, K, qweight, scales, nullptr, g, y, true);
+    if (rc != WQ_OK) return rc;
+    const size_t need = wq_gemm_workspace_bytes(M, N, K, g, 8);
+    if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+        return fail(WQ_ERR_WORKSPACE, "wq_gemm_w8a16: need %zu workspace bytes", need);
+    wq::launch_gemv_w8a16(x, M, N, K, qweight, scales, g, y, static_cast<cudaStream_t>(stream));
+    return check_launch("wq_gemm_w8a16");
+}
+
+int wq_device_status(void *stream)
+{
+    g_last_error.clear();
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int host = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&host, g_wq_device_status, sizeof(int), 0,
+                                              cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_device_status: %s", cudaGetErrorString(e));
+    if (host != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_wq_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_device_status: %s", cudaGetErrorString(e));
+        return fail(WQ_ERR_DEVICE_TIMEOUT, "a kernel recorded a bounded-wait timeout (code %d)", host);
+    }
+    return WQ_OK;
+}
+
+}  // extern "C"

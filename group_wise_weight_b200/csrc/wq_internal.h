@@ -1,0 +1,22 @@
+// wq_internal.h -- host-side launchers behind the C ABI (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace wq {
+
+// Quantisers (wq_quant.cu).  Arguments are validated by the caller.
+void launch_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *q,
+                          uint16_t *s, uint16_t *z, cudaStream_t st);
+void launch_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, int8_t *q,
+                          uint16_t *s, cudaStream_t st);
+
+// CUDA-core matmul for small M (wq_gemv.cu).  Any M >= 1 is accepted; rows of
+// x are processed in tiles of up to 16.
+void launch_gemv_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
+                       const uint16_t *z, int g, uint16_t *y, cudaStream_t st);
+void launch_gemv_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *q, const uint16_t *s,
+                       int g, uint16_t *y, cudaStream_t st);
+
+}  // namespace wq

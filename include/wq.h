@@ -1,0 +1,168 @@
+/*
+ * wq.h -- C ABI of libwq, group-wise weight quantisation and the
+ * dequant-fused weight-only matmul for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow these web pages (cited by title and section):
+ *  [P2] "Quantization for LLM inference: FP8, INT4 (GPTQ, AWQ) and GGUF --
+ *       the model's accounting zoom", section "The minimum maths: scale and
+ *       zero-point": asymmetric b-bit quantisation of a block of weights,
+ *       s = (max - min) / (2^b - 1), z = round(-min / s),
+ *       q = clip(round(w / s + z), 0, 2^b - 1), decode w_hat = s * (q - z);
+ *       section "Numerical example": 4-bit codes, two per byte, a bf16 scale.
+ *  [P3] "Quantization Methods Compared: INT8, GPTQ, AWQ, FP8, FP4 and
+ *       KV-Cache Quantization", section "What quantisation does": symmetric
+ *       absmax INT8, s = max|w| / 127, q = round(w / s), w_hat = q * s;
+ *       one scale per tensor, per output channel or per group of 128 (or 32)
+ *       consecutive weights.  Section "Hardware, formats and the roofline":
+ *       decode reads every weight once per step and real 4-bit kernels
+ *       dequantise inside the matmul.
+ *
+ * Conventions shared by every call
+ *  - Weights are stored one row per output channel: W is [N][K] with K (the
+ *    reduction axis) contiguous; groups are g consecutive weights of a row.
+ *    y[m][n] = sum_k x[m][k] * w_hat[n][k].
+ *  - bf16 values travel as uint16_t bit patterns (the top half of an IEEE
+ *    binary32).  Row-major, densely packed unless a leading dimension is given.
+ *  - Every pointer is a DEVICE pointer to memory the caller owns; the library
+ *    never allocates or frees device memory.  Pointers must be 16-byte
+ *    aligned.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) and never synchronises.  Argument errors are
+ *    detected on the host before anything is launched and leave every output
+ *    untouched.
+ *  - Inputs are finite; non-finite inputs give unspecified (but in-bounds)
+ *    results.
+ *  - Quantisation is bit-exact against the arithmetic stated below: binary32
+ *    with round-to-nearest-even for every operation, "round" = round half to
+ *    even, bf16 rounding = round to nearest even.
+ *
+ * Return value of every int-returning call: one of the WQ_* status codes.
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WQ_OK 0
+#define WQ_ERR_ARG (-1)            /* null pointer, or a size <= 0                      */
+#define WQ_ERR_SHAPE (-2)          /* K not a multiple of 32, g does not divide K, ldw < K */
+#define WQ_ERR_ALIGN (-3)          /* a pointer not 16-byte aligned, or ldw % 8 != 0      */
+#define WQ_ERR_UNSUPPORTED (-4)    /* group size or dtype outside the supported set       */
+#define WQ_ERR_CUDA (-5)           /* a CUDA call or launch failed; see wq_last_error()   */
+#define WQ_ERR_WORKSPACE (-6)      /* workspace null or smaller than wq_gemm_workspace_bytes */
+#define WQ_ERR_DEVICE_TIMEOUT (-7) /* a kernel gave up on a bounded wait (see wq_device_status) */
+
+/* Element type of the unquantised weight given to the quantisers. */
+#define WQ_F32 0
+#define WQ_BF16 1
+
+/* Text for a status code (static storage; never NULL). */
+const char *wq_status_str(int status);
+
+/* Detail of the last error raised by a call on this host thread ("" if none). */
+const char *wq_last_error(void);
+
+/* Library ABI version: 100 * major + minor. */
+int wq_version(void);
+
+/*
+ * Asymmetric INT4 quantisation, one (scale, zero-point) per group of g
+ * consecutive weights along K  ([P2] "The minimum maths", b = 4).
+ *
+ *   w       [N][ldw] of WQ_F32 or WQ_BF16 (wtype); only the first K columns are read
+ *   qweight [N][K/2] bytes: byte j of a row holds q[2j] in bits 0-3 and
+ *           q[2j+1] in bits 4-7
+ *   scales  [N][K/g] bf16;  zeros [N][K/g] bf16
+ *
+ * Per group, in binary32 (widening a bf16 w is exact):
+ *   mn, mx = min, max of the group
+ *   s  = bf16((mx - mn) / 15)                 one subtraction, one division
+ *   if s == 0: s = bf16(max(|mn|, |mx|)); if still 0: s = 1
+ *   z  = bf16(round(-mn / s) + 0)             (+0 turns -0 into +0)
+ *   q  = clip(round(w / s + z), 0, 15)        with the stored s and z
+ * Requirements: N >= 1; K >= 32, K % 32 == 0; g in {32, 64, 128}, K % g == 0;
+ * ldw >= K, ldw % 8 == 0; all pointers 16-byte aligned.
+ */
+int wq_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g,
+                     uint8_t *qweight, uint16_t *scales, uint16_t *zeros, void *stream);
+
+/*
+ * Symmetric absmax INT8 quantisation  ([P3] "What quantisation does").
+ * One scale per group of g weights; g == K gives one scale per output
+ * channel (row).
+ *
+ *   w       [N][ldw] of WQ_F32 or WQ_BF16
+ *   qweight [N][K] int8 in -127..127
+ *   scales  [N][K/g] bf16
+ *
+ * Per group, in binary32:
+ *   s = bf16(max|w| / 127); if s == 0: s = 1
+ *   q = clip(round(w / s), -127, 127)   (the clip matters when the bf16 s
+ *                                        rounded below max|w| / 127)
+ * Requirements: as wq_quantize_int4, with g in {32, 64, 128, K}.
+ */
+int wq_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g,
+                     int8_t *qweight, uint16_t *scales, void *stream);
+
+/*
+ * Bytes of device workspace wq_gemm_w4a16 (wbits = 4) or wq_gemm_w8a16
+ * (wbits = 8) needs for this shape; 0 when the chosen kernel needs none.
+ * The workspace holds binary32 partial sums of a K-split and per-tile
+ * arrival counters; the library leaves the counters zeroed on return, so
+ * a workspace must be zero-filled once before its first use and may then be
+ * reused by later calls on the same stream.
+ */
+size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits);
+
+/*
+ * W4A16 weight-only matmul with in-kernel dequantisation
+ * ([P2] decode w_hat = s * (q - z); [P3] "real 4-bit kernels dequantise ...
+ * inside the kernel").
+ *
+ *   x       [M][K] bf16 activations
+ *   qweight, scales, zeros: as produced by wq_quantize_int4 with group g
+ *   y       [M][N] bf16, y[m][n] = sum_k x[m][k] * s[n][k/g] * (q[n][k] - z[n][k/g])
+ *
+ * Arithmetic: binary32 accumulation, one final rounding to bf16.  M <= 16
+ * runs a CUDA-core kernel that keeps (q - z) exact and applies s per group in
+ * binary32.  Larger M runs a tcgen05 tensor-core kernel whose operand is
+ * w_hat rounded once to bf16.  Either way |y - y_exact| stays within
+ * 4e-3 * sum_k |x[m][k] * w_hat[n][k]| on the inputs this library is tested on.
+ * Requirements: M, N >= 1; K % 32 == 0; g in {32, 64, 128}, K % g == 0;
+ * pointers 16-byte aligned; workspace of wq_gemm_workspace_bytes(M, N, K, g, 4)
+ * bytes (may be NULL when that is 0).  x and y must not overlap.
+ */
+int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *qweight,
+                  const uint16_t *scales, const uint16_t *zeros, int g, uint16_t *y,
+                  void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * W8A16 weight-only matmul: y[m][n] = sum_k x[m][k] * s[n][k/g] * q[n][k]
+ * ([P3] dequantised value q * s).  qweight [N][K] int8, scales [N][K/g]
+ * bf16, g in {32, 64, 128, K}.  Other arguments and guarantees as
+ * wq_gemm_w4a16.
+ */
+int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *qweight,
+                  const uint16_t *scales, int g, uint16_t *y, void *workspace, size_t ws_bytes,
+                  void *stream);
+
+/*
+ * Device status word.  Kernels with waits on barriers bound every wait; a
+ * wait that runs out records a code on the device and the kernel returns
+ * early instead of hanging.  This call synchronises `stream`, returns
+ * WQ_ERR_DEVICE_TIMEOUT if any kernel of this library recorded a timeout on
+ * the current device since the last call (and clears it), WQ_ERR_CUDA if the
+ * stream reports an error, else WQ_OK.
+ */
+int wq_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H */

@@ -1,0 +1,115 @@
+"""The C ABI library: it builds for sm_100a, loads, exports every function
+include/wq.h declares, and rejects bad arguments on the host before any
+launch.  CPU only: no call here reaches a kernel launch (every call fails
+validation, or is a pure host query)."""
+import ctypes
+import subprocess
+
+import pytest
+
+import group_wise_weight_b200 as wq
+from group_wise_weight_b200 import build as wqbuild
+
+
+@pytest.fixture(scope="module")
+def L():
+    wqbuild.build()
+    return wq.lib()
+
+
+def test_exports_every_declared_function(L):
+    names = wq.header_functions()
+    assert len(names) >= 9
+    out = subprocess.run(["nm", "-D", "--defined-only", wq.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(L, n)
+
+
+def test_status_strings(L):
+    for code in range(0, -8, -1):
+        s = wq.wq_status_str(code)
+        assert s.startswith("WQ_")
+    assert wq.wq_status_str(12345) == "unknown status"
+    assert wq.wq_version() >= 100
+
+
+# Fake, never-dereferenced device addresses: validation must reject the call first.
+A = 1 << 20          # 16-byte aligned
+MIS = (1 << 20) + 2  # misaligned
+
+
+def _q4(L, w=A, wt=wq.WQ_BF16, N=4, K=256, ldw=256, g=128, q=A, s=A, z=A):
+    return L.wq_quantize_int4(w, wt, N, K, ldw, g, q, s, z, None)
+
+
+def _q8(L, w=A, wt=wq.WQ_BF16, N=4, K=256, ldw=256, g=128, q=A, s=A):
+    return L.wq_quantize_int8(w, wt, N, K, ldw, g, q, s, None)
+
+
+def _g4(L, x=A, M=1, N=4, K=256, q=A, s=A, z=A, g=128, y=A, ws=None, wsb=0):
+    return L.wq_gemm_w4a16(x, M, N, K, q, s, z, g, y, ws, wsb, None)
+
+
+def _g8(L, x=A, M=1, N=4, K=256, q=A, s=A, g=128, y=A, ws=None, wsb=0):
+    return L.wq_gemm_w8a16(x, M, N, K, q, s, g, y, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(w=None), wq.WQ_ERR_ARG), (dict(q=None), wq.WQ_ERR_ARG), (dict(z=None), wq.WQ_ERR_ARG),
+    (dict(N=0), wq.WQ_ERR_ARG), (dict(K=-32), wq.WQ_ERR_ARG),
+    (dict(wt=7), wq.WQ_ERR_UNSUPPORTED), (dict(g=16), wq.WQ_ERR_UNSUPPORTED),
+    (dict(g=256), wq.WQ_ERR_UNSUPPORTED),
+    (dict(K=96, ldw=96), wq.WQ_ERR_SHAPE), (dict(K=48, ldw=48, g=32), wq.WQ_ERR_SHAPE),
+    (dict(ldw=128), wq.WQ_ERR_SHAPE),
+    (dict(w=MIS), wq.WQ_ERR_ALIGN), (dict(s=MIS), wq.WQ_ERR_ALIGN), (dict(ldw=260), wq.WQ_ERR_ALIGN),
+])
+def test_quantize_int4_rejects(L, kw, code):
+    assert _q4(L, **kw) == code
+    assert wq.wq_last_error() != ""
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(s=None), wq.WQ_ERR_ARG), (dict(g=100), wq.WQ_ERR_UNSUPPORTED),
+    (dict(K=160, ldw=160, g=128), wq.WQ_ERR_SHAPE), (dict(q=MIS), wq.WQ_ERR_ALIGN),
+])
+def test_quantize_int8_rejects(L, kw, code):
+    assert _q8(L, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=None), wq.WQ_ERR_ARG), (dict(y=None), wq.WQ_ERR_ARG), (dict(M=0), wq.WQ_ERR_ARG),
+    (dict(N=-1), wq.WQ_ERR_ARG), (dict(g=256), wq.WQ_ERR_UNSUPPORTED),
+    (dict(K=200), wq.WQ_ERR_SHAPE), (dict(K=320, g=128), wq.WQ_ERR_SHAPE),
+    (dict(x=MIS), wq.WQ_ERR_ALIGN), (dict(y=MIS), wq.WQ_ERR_ALIGN), (dict(z=MIS), wq.WQ_ERR_ALIGN),
+])
+def test_gemm_w4a16_rejects(L, kw, code):
+    assert _g4(L, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(s=None), wq.WQ_ERR_ARG), (dict(g=96), wq.WQ_ERR_UNSUPPORTED), (dict(K=224, g=64), wq.WQ_ERR_SHAPE),
+    (dict(q=MIS), wq.WQ_ERR_ALIGN),
+])
+def test_gemm_w8a16_rejects(L, kw, code):
+    assert _g8(L, **kw) == code
+
+
+def test_workspace_query_is_pure(L):
+    for M in (1, 16, 17, 128, 4096):
+        for wb in (4, 8):
+            a = wq.wq_gemm_workspace_bytes(M, 28672, 8192, 128, wb)
+            b = wq.wq_gemm_workspace_bytes(M, 28672, 8192, 128, wb)
+            assert a == b and a >= 0
+
+
+def test_python_binding_refuses_cpu_tensors(L):
+    import torch
+    with pytest.raises(TypeError):
+        wq.wq_quantize_int4(torch.zeros(4, 256, dtype=torch.bfloat16), 128)
+    with pytest.raises(TypeError):
+        wq.wq_gemm_w4a16(torch.zeros(1, 256, dtype=torch.bfloat16), torch.zeros(4, 128, dtype=torch.uint8),
+                         torch.zeros(4, 2, dtype=torch.bfloat16), torch.zeros(4, 2, dtype=torch.bfloat16), 128)

@@ -1,0 +1,328 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Quantisation outputs (packed codes, bf16 scales, bf16 zero-points) must be
+bit-exact.  Matmul outputs must satisfy, element by element,
+    |y - y_ref| <= 4e-3 * sum_k |x[m][k] * w_hat[n][k]|
+with y_ref and the sum computed by the oracle in binary64.  Inputs come from
+the seeded generators in wq_inputs; small cases are compared in full, the
+full-size workloads on sampled output rows the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import group_wise_weight_b200 as wq
+import oracle
+import wq_inputs
+from group_wise_weight_b200 import build as wqbuild
+
+pytestmark = pytest.mark.gpu
+TOL = 4e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    wqbuild.build()
+    wq.lib()
+    torch.cuda.init()
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def w_f32(w: torch.Tensor) -> np.ndarray:
+    return w.float().numpy()
+
+
+def oracle_q4(w: torch.Tensor, g: int):
+    codes, s, z = oracle.quantize_int4(w_f32(w), g)
+    return codes, s, z, oracle.pack_int4(codes), oracle.bf16_bits(s), oracle.bf16_bits(z)
+
+
+def oracle_q8(w: torch.Tensor, g: int):
+    codes, s = oracle.quantize_int8(w_f32(w), g)
+    return codes, s, oracle.bf16_bits(s)
+
+
+def check_q4(w: torch.Tensor, g: int, rows=None):
+    wd = w.cuda()
+    q, s, z = wq.wq_quantize_int4(wd, g)
+    torch.cuda.synchronize()
+    sel = slice(None) if rows is None else rows
+    codes, so, zo, packed, sb, zb = oracle_q4(w[sel], g)
+    assert np.array_equal(q.cpu().numpy()[sel], packed), "packed codes differ"
+    assert np.array_equal(bits(s)[sel], sb), "scales differ"
+    assert np.array_equal(bits(z)[sel], zb), "zero-points differ"
+    return q, s, z, (codes, so, zo)
+
+
+def check_y(y: torch.Tensor, y_ref: np.ndarray, a_ref: np.ndarray) -> float:
+    yg = y.double().cpu().numpy()
+    err = np.abs(yg - y_ref)
+    bound = TOL * a_ref
+    bad = err > bound
+    ratio = float(np.max(err / np.where(a_ref > 0, a_ref, 1.0)))
+    assert not bad.any(), f"{bad.sum()} outputs outside 4e-3*sum|x*w_hat|; max ratio {ratio:.3e}"
+    return ratio
+
+
+def sample_rows(N: int, n: int, seed: int) -> np.ndarray:
+    g = torch.Generator().manual_seed(seed)
+    r = torch.randperm(N, generator=g)[:n].numpy()
+    return np.unique(np.concatenate([r, [0, N - 1]]))
+
+
+# ---------------------------------------------------------------------------
+# Quantisation, bit-exact
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("g", [32, 64, 128])
+def test_quantize_int4_tiny(g):
+    check_q4(wq_inputs.tiny_weight(), g)
+
+
+def test_quantize_int4_tiny_bf16_input():
+    check_q4(wq_inputs.tiny_weight().to(torch.bfloat16), 128)
+
+
+def test_quantize_int4_decode_up():
+    w = wq_inputs.llm_weight(14336, 4096, wq_inputs.SEEDS["decode_up"])
+    check_q4(w, 128)
+
+
+def test_quantize_int4_gran_g32():
+    w = wq_inputs.block_outlier_weight(8192, 8192, wq_inputs.SEEDS["gran"])
+    check_q4(w, 32)
+
+
+def test_quantize_int4_sweep_sampled_rows():
+    w = wq_inputs.llm_weight(28672, 8192, wq_inputs.SEEDS["sweep"])
+    check_q4(w, 128, rows=sample_rows(28672, 512, 1))
+
+
+@pytest.mark.parametrize("g", [32, 128, None])
+def test_quantize_int8(g):
+    w = wq_inputs.block_outlier_weight(1024, 2048, 40)
+    gg = 2048 if g is None else g
+    wd = w.cuda()
+    q, s = wq.wq_quantize_int8(wd, g)
+    torch.cuda.synchronize()
+    codes, so, sb = oracle_q8(w, gg)
+    assert np.array_equal(q.cpu().numpy(), codes)
+    assert np.array_equal(bits(s), sb)
+
+
+def test_quantize_int8_gran_per_channel_fp32():
+    w = wq_inputs.block_outlier_weight(8192, 8192, wq_inputs.SEEDS["gran"], dtype=torch.float32)
+    q, s = wq.wq_quantize_int8(w.cuda())
+    torch.cuda.synchronize()
+    codes, so, sb = oracle_q8(w, 8192)
+    assert np.array_equal(q.cpu().numpy(), codes)
+    assert np.array_equal(bits(s), sb)
+
+
+def test_quantize_padded_rows_and_odd_sizes():
+    # ldw > K (a column slice of a wider matrix), N = 1 and N not a multiple of anything
+    for N, K, ldw in ((1, 32, 32), (7, 96, 104), (129, 4096 + 128, 4352), (3, 288, 296)):
+        base = wq_inputs.llm_weight(N, ldw, 70 + N, dtype=torch.float32)
+        wd = base.cuda()[:, :K]
+        g = 32
+        q, s, z = wq.wq_quantize_int4(wd, g)
+        q8, s8 = wq.wq_quantize_int8(wd, g)
+        torch.cuda.synchronize()
+        _, _, _, packed, sb, zb = oracle_q4(base[:, :K].contiguous(), g)
+        assert np.array_equal(q.cpu().numpy(), packed) and np.array_equal(bits(s), sb) and np.array_equal(bits(z), zb)
+        c8, _, s8b = oracle_q8(base[:, :K].contiguous(), g)
+        assert np.array_equal(q8.cpu().numpy(), c8) and np.array_equal(bits(s8), s8b)
+
+
+def test_quantize_degenerate_and_one_signed_groups():
+    w = wq_inputs.llm_weight(64, 512, 81, dtype=torch.float32)
+    w[0] = 0.0                    # all-zero row
+    w[1, :128] = 0.25             # constant group
+    w[2, 128:256] = -3.0
+    w[3] = w[3].abs() + 0.01      # one-signed row
+    w[4, :128] = 1e-30            # tiny constant group
+    w[5, :32] = torch.tensor([0.0, 15.0, 2.5, 3.5, 0.5, 1.5, 14.5, 7.5] * 4)  # exact ties
+    w[6] = -w[6].abs() - 5.0      # one-signed, far from zero
+    for g in (32, 128):
+        check_q4(w, g)
+        q8, s8 = wq.wq_quantize_int8(w.cuda(), g)
+        torch.cuda.synchronize()
+        c8, _, s8b = oracle_q8(w, g)
+        assert np.array_equal(q8.cpu().numpy(), c8) and np.array_equal(bits(s8), s8b)
+
+
+def test_quantize_worked_example_on_gpu():
+    # the page's 8-weight group, replicated into one 32-wide group of a row
+    v = torch.tensor([0.31, -0.12, 0.78, -0.05, 1.42, -0.91, 0.23, 0.66], dtype=torch.float32)
+    w = v.repeat(1, 4)
+    q, s, z = wq.wq_quantize_int4(w.cuda(), 32)
+    torch.cuda.synchronize()
+    codes = oracle.unpack_int4(q.cpu().numpy(), 32)[0]
+    assert codes[:8].tolist() == [8, 5, 11, 6, 15, 0, 7, 10]
+    assert bits(z)[0, 0] == oracle.bf16_bits(np.float32(6.0))
+
+
+def test_quantize_does_not_write_outside_outputs():
+    N, K, g = 37, 256, 64
+    w = wq_inputs.llm_weight(N, K, 91).cuda()
+    pad = 4096
+    canary = 0x5A
+    qb = torch.full((N * K // 2 + 2 * pad,), canary, dtype=torch.uint8, device="cuda")
+    sb = torch.full((N * K // g + 2 * pad,), 12345, dtype=torch.int16, device="cuda")
+    zb = torch.full((N * K // g + 2 * pad,), 12345, dtype=torch.int16, device="cuda")
+    q = qb[pad:pad + N * K // 2].view(N, K // 2)
+    s = sb[pad:pad + N * K // g].view(torch.bfloat16).view(N, K // g)
+    z = zb[pad:pad + N * K // g].view(torch.bfloat16).view(N, K // g)
+    wq.wq_quantize_int4(w, g, q, s, z)
+    torch.cuda.synchronize()
+    assert bool((qb[:pad] == canary).all()) and bool((qb[-pad:] == canary).all())
+    assert bool((sb[:pad] == 12345).all()) and bool((sb[-pad:] == 12345).all())
+    assert bool((zb[:pad] == 12345).all()) and bool((zb[-pad:] == 12345).all())
+
+
+def test_errors_with_real_tensors():
+    w = torch.zeros(4, 256, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_quantize_int4(w, 48)
+    assert e.value.status == wq.WQ_ERR_UNSUPPORTED
+    buf = torch.zeros(4 * 256 + 8, dtype=torch.bfloat16, device="cuda")
+    wmis = buf[1:1 + 4 * 256].view(4, 256)  # 2-byte offset
+    with pytest.raises(wq.WQError) as e:
+        wq.wq_quantize_int4(wmis, 128)
+    assert e.value.status == wq.WQ_ERR_ALIGN
+
+
+# ---------------------------------------------------------------------------
+# Matmul, within 4e-3 * sum|x * w_hat|
+# ---------------------------------------------------------------------------
+
+def _w4_case(N, K, g, M, seed, wgen=None, xgen=None):
+    w = wq_inputs.llm_weight(N, K, seed) if wgen is None else wgen
+    x = wq_inputs.activations(M, K, seed) if xgen is None else xgen
+    q, s, z, (codes, so, zo) = check_q4(w, g)
+    y = wq.wq_gemm_w4a16(x.cuda(), q, s, z, g)
+    torch.cuda.synchronize()
+    y_ref, a_ref = oracle.gemm_w4a16(x.double().numpy(), codes, so, zo, g)
+    return check_y(y.cpu(), y_ref, a_ref)
+
+
+def test_gemm_w4a16_tiny():
+    w = wq_inputs.tiny_weight()
+    x = wq_inputs.plain_activations(1, 256, 0)
+    _w4_case(512, 256, 128, 1, 0, wgen=w, xgen=x)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 7, 8, 9, 15, 16, 17, 31, 32, 33, 64, 127, 128, 129])
+def test_gemm_w4a16_batch_sizes(M):
+    _w4_case(1000, 512, 128, M, 100 + M)
+
+
+@pytest.mark.parametrize("N,K,g", [(1, 32, 32), (7, 64, 32), (129, 128, 64), (300, 1024, 128), (33, 4096, 32)])
+@pytest.mark.parametrize("M", [1, 4, 16, 40])
+def test_gemm_w4a16_shapes(N, K, g, M):
+    _w4_case(N, K, g, M, 7 * N + K + M)
+
+
+def test_gemm_w4a16_degenerate_groups():
+    w = wq_inputs.llm_weight(64, 512, 81, dtype=torch.float32)
+    w[0] = 0.0
+    w[1, :128] = 0.25
+    w[3] = w[3].abs() + 0.01
+    w[6] = -w[6].abs() - 5.0
+    for M in (1, 8, 48):
+        _w4_case(64, 512, 128, M, 5, wgen=w)
+
+
+def _sampled_w4(N, K, g, Ms, seed, wgen, rows):
+    q, s, z, (codes, so, zo) = check_q4(wgen, g, rows=rows)
+    ratios = []
+    for M in Ms:
+        x = wq_inputs.activations(M, K, seed + M)
+        y = wq.wq_gemm_w4a16(x.cuda(), q, s, z, g)
+        torch.cuda.synchronize()
+        y_ref, a_ref = oracle.gemm_w4a16(x.double().numpy(), codes, so, zo, g)
+        ratios.append(check_y(y.cpu()[:, rows], y_ref, a_ref))
+    return ratios
+
+
+def test_gemm_w4a16_decode_up_m1():
+    w = wq_inputs.llm_weight(14336, 4096, wq_inputs.SEEDS["decode_up"])
+    _sampled_w4(14336, 4096, 128, [1], 2, w, sample_rows(14336, 256, 2))
+
+
+def test_gemm_w4a16_sweep_sampled():
+    w = wq_inputs.llm_weight(28672, 8192, wq_inputs.SEEDS["sweep"])
+    _sampled_w4(28672, 8192, 128, [1, 8, 32, 128], 3, w, sample_rows(28672, 192, 3))
+
+
+def test_gemm_w4a16_gran_g32():
+    w = wq_inputs.block_outlier_weight(8192, 8192, wq_inputs.SEEDS["gran"])
+    _sampled_w4(8192, 8192, 32, [1, 16], 4, w, sample_rows(8192, 192, 4))
+
+
+def _w8_case(w, x, g, rows=None):
+    K = w.shape[1]
+    gg = K if g is None else g
+    q, s = wq.wq_quantize_int8(w.cuda(), g)
+    y = wq.wq_gemm_w8a16(x.cuda(), q, s, g)
+    torch.cuda.synchronize()
+    sel = slice(None) if rows is None else rows
+    codes, so, sb = oracle_q8(w[sel], gg)
+    assert np.array_equal(q.cpu().numpy()[sel], codes) and np.array_equal(bits(s)[sel], sb)
+    y_ref, a_ref = oracle.gemm_w8a16(x.double().numpy(), codes, so, gg)
+    return check_y(y.cpu()[:, sel], y_ref, a_ref)
+
+
+@pytest.mark.parametrize("M", [1, 2, 5, 16, 17, 64, 128])
+@pytest.mark.parametrize("g", [None, 32, 128])
+def test_gemm_w8a16(M, g):
+    w = wq_inputs.block_outlier_weight(600, 1024, 200 + M)
+    x = wq_inputs.activations(M, 1024, 300 + M)
+    _w8_case(w, x, g)
+
+
+def test_gemm_w8a16_gran_per_channel():
+    w = wq_inputs.block_outlier_weight(8192, 8192, wq_inputs.SEEDS["gran"])
+    rows = sample_rows(8192, 192, 5)
+    for M in (1, 16):
+        _w8_case(w, wq_inputs.activations(M, 8192, 4 + M), None, rows=rows)
+
+
+def test_full70b_layer_shapes_sampled():
+    """One layer of the 70B-shaped step, generated on the GPU like the benchmark, sampled rows checked."""
+    layer = 0
+    for j, (name, K, N) in enumerate(wq_inputs.FULL70B_LINEARS):
+        seed = wq_inputs.full70b_seed(layer, j)
+        wd = wq_inputs.llm_weight(N, K, seed, outlier_frac=0.0, device="cuda")
+        rows = sample_rows(N, 64, seed)
+        q, s, z = wq.wq_quantize_int4(wd, 128)
+        wrows = wd[torch.as_tensor(rows, device="cuda")].cpu()
+        codes, so, zo, packed, sb, zb = oracle_q4(wrows, 128)
+        assert np.array_equal(q.cpu().numpy()[rows], packed)
+        assert np.array_equal(bits(s)[rows], sb) and np.array_equal(bits(z)[rows], zb)
+        for M in (1, 128):
+            x = wq_inputs.plain_activations(M, K, seed, device="cuda")
+            y = wq.wq_gemm_w4a16(x, q, s, z, 128)
+            torch.cuda.synchronize()
+            y_ref, a_ref = oracle.gemm_w4a16(x.double().cpu().numpy(), codes, so, zo, 128)
+            check_y(y.cpu()[:, rows], y_ref, a_ref)
+        del wd, q, s, z
+        torch.cuda.empty_cache()
+
+
+def test_gemm_output_offsets_and_canaries():
+    N, K, M = 100, 256, 3
+    w = wq_inputs.llm_weight(N, K, 11)
+    q, s, z, (codes, so, zo) = check_q4(w, 64)
+    x = wq_inputs.activations(M, K, 12).cuda()
+    pad = 2048
+    yb = torch.full((M * N + 2 * pad,), -7, dtype=torch.int16, device="cuda")
+    y = yb[pad:pad + M * N].view(torch.bfloat16).view(M, N)
+    wq.wq_gemm_w4a16(x, q, s, z, 64, y=y)
+    torch.cuda.synchronize()
+    assert bool((yb[:pad] == -7).all()) and bool((yb[-pad:] == -7).all())
+    y_ref, a_ref = oracle.gemm_w4a16(x.double().cpu().numpy(), codes, so, zo, 64)
+    check_y(y.cpu(), y_ref, a_ref)
