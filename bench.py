@@ -190,6 +190,9 @@ class Model:
         torch.cuda.empty_cache()
         self.quant_ms, self.quant_bytes = quant_ms, quant_bytes
         self.weights = sum(K * N for _, K, N, *_ in self.linears)
+        # one workspace serves every call: calls run in order on one stream and each leaves it zeroed
+        need = max(wq.wq_gemm_workspace_bytes(M, N, K, G, 4) for M in (1, 128) for _, K, N, *_ in self.linears)
+        self.ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=device)
 
     def buffers(self, M, device, seed=0):
         xs, ys = [], []
@@ -201,7 +204,7 @@ class Model:
     def step(self, xs, ys):
         f = self.wq.wq_gemm_w4a16
         for (name, K, N, q, s, z), x, y in zip(self.linears, xs, ys):
-            f(x, q, s, z, G, y=y)
+            f(x, q, s, z, G, y=y, workspace=self.ws)
 
     def step_bytes(self, M):
         return sum(linear_bytes(M, N, K) for _, K, N, *_ in self.linears)
@@ -289,7 +292,7 @@ def per_linear_us(model, xs, ys, reps=3):
         for _ in range(reps):
             for i in idx:
                 _, K_, N_, q, s, z = model.linears[i]
-                model.wq.wq_gemm_w4a16(xs[i], q, s, z, G, y=ys[i])
+                model.wq.wq_gemm_w4a16(xs[i], q, s, z, G, y=ys[i], workspace=model.ws)
         e1.record()
         e1.synchronize()
         us = e0.elapsed_time(e1) * 1e3 / (reps * len(idx))

@@ -74,6 +74,24 @@ int check_gemm(const char *what, const void *x, int64_t M, int64_t N, int64_t K,
 // Per-device status word written by kernels whose waits ran out.
 __device__ int g_wq_device_status = 0;
 
+namespace {
+
+// Device address of the status word on the current device (looked up once per device).
+int *status_word()
+{
+    static int *addr[128] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_wq_device_status) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int *>(p);
+    }
+    return addr[dev];
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *wq_status_str(int status)
@@ -117,7 +135,8 @@ int wq_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw
 
 size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits)
 {
-    (void)M; (void)N; (void)K; (void)g; (void)wbits;
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    if (wbits == 4) return wq::gemv_tma_workspace_bytes(M, N, K, g);
     return 0;
 }
 
@@ -131,7 +150,15 @@ int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint
     const size_t need = wq_gemm_workspace_bytes(M, N, K, g, 4);
     if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
         return fail(WQ_ERR_WORKSPACE, "wq_gemm_w4a16: need %zu workspace bytes", need);
-    wq::launch_gemv_w4a16(x, M, N, K, qweight, scales, zeros, g, y, static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (wq::gemv_tma_eligible(M, N, K, g)) {
+        int *status = status_word();
+        if (!status) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: no device status word");
+        if (wq::launch_gemv_w4a16_tma(x, M, N, K, qweight, scales, zeros, y, workspace, status, st) != 0)
+            return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: tensor map encoding failed");
+        return check_launch("wq_gemm_w4a16");
+    }
+    wq::launch_gemv_w4a16(x, M, N, K, qweight, scales, zeros, g, y, st);
     return check_launch("wq_gemm_w4a16");
 }
 

@@ -40,6 +40,13 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void *p)
     return r;
 }
 
+__device__ __forceinline__ uint32_t ld_nc_u32(const uint32_t *p)
+{
+    uint32_t r;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(r) : "l"(p));
+    return r;
+}
+
 __device__ __forceinline__ uint16_t ld_nc_u16(const uint16_t *p)
 {
     uint16_t r;
