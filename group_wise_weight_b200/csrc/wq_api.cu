@@ -136,7 +136,10 @@ int wq_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw
 size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits)
 {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
-    if (wbits == 4) return wq::gemv_tma_workspace_bytes(M, N, K, g);
+    if (wbits == 4) {
+        if (wq::gemm_tc_eligible(M, N, K, g)) return wq::gemm_tc_workspace_bytes(M, N, K, g);
+        return wq::gemv_tma_workspace_bytes(M, N, K, g);
+    }
     return 0;
 }
 
@@ -151,6 +154,13 @@ int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint
     if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
         return fail(WQ_ERR_WORKSPACE, "wq_gemm_w4a16: need %zu workspace bytes", need);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (wq::gemm_tc_eligible(M, N, K, g)) {
+        int *status = status_word();
+        if (!status) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: no device status word");
+        if (wq::launch_gemm_w4a16_tc(x, M, N, K, qweight, scales, zeros, g, y, workspace, status, st) != 0)
+            return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: tensor map encoding failed");
+        return check_launch("wq_gemm_w4a16");
+    }
     if (wq::gemv_tma_eligible(M, N, K, g)) {
         int *status = status_word();
         if (!status) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: no device status word");

@@ -1,0 +1,468 @@
+// wq_gemm_tc.cu -- W4A16 matmul for batches of activations (M > 16) on the
+// 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// At batch sizes like 128 the matmul is a dense contraction and the pages'
+// roofline argument ("Quantization Methods Compared: INT8, GPTQ, AWQ, FP8,
+// FP4 and KV-Cache Quantization", section "Hardware, formats and the
+// roofline") puts it near or past the ridge point, so the tensor cores do
+// the work.  The 4-bit weights are dequantised inside the kernel
+// ("... real 4-bit kernels dequantise to fp16 inside the kernel"), with the
+// decode w_hat = s (q - z) of "Quantization for LLM inference: FP8, INT4
+// (GPTQ, AWQ) and GGUF", section "The minimum maths".
+//
+// Formulation: D[n][m] = sum_k w_hat[n][k] * x[m][k], a 128 x BN tile per
+// CTA at a time (MMA M = 128 weight rows, N = BN activation rows, K = 16 per
+// instruction).  The weight operand A lives in tensor memory: dequant warps
+// write bf16 w_hat there with tcgen05.st, so the dequantised tile never
+// touches shared memory.  The activation operand B is loaded by TMA into
+// shared memory with the 128-byte swizzle.  The accumulator D lives in
+// tensor memory and is read back by the same warps for the epilogue.
+//
+// Warp roles (320 threads): warp 0 issues TMA loads (weights box
+// [128 rows x 64 B] with the 64-byte swizzle, two activation boxes
+// [BN rows x 64 elements] with the 128-byte swizzle per 128-k stage); warp 1
+// allocates tensor memory and one of its lanes issues the MMAs; warps 2..9
+// dequantise (two warps per 32-lane quarter of tensor memory, each taking
+// half of the stage's 128 k) and run the epilogue.
+//
+// Dequantisation: natural k order.  A code word v (8 codes, k .. k+7) and
+// v >> 4 give, with one byte permute and one LOP3 per pair, the bf16x2 pair
+// (128 + q[2j], 128 + q[2j+1]); subtracting (128 + z) is exact, so the MMA
+// operand is the exact integer q - z.  Each group of g consecutive k gets its
+// own accumulator region in tensor memory, and the dequant warps, one stage
+// behind the MMAs, add s * D_group into binary32 registers ("promotion"):
+// (q - z) is never rounded and s is applied in binary32, as in the decode
+// kernels.  Tensor memory: A 2 x 64 columns, D 2 stages x (128/g) groups x BN
+// columns (BN = 128 for g = 128, 64 for g = 64, 32 for g = 32).
+//
+// Scheduling: stream-K over (tile, stage) units so every SM gets the same
+// number of stages.  A tile split between CTAs leaves one binary32 partial
+// per segment in the workspace; the CTA whose stages complete the tile sums
+// the partials of the others and writes y.  Every barrier wait is bounded.
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "wq_internal.h"
+#include "wq_sm100.cuh"
+
+namespace wq {
+
+namespace {
+
+constexpr int kTileN = 128;         // weight rows per tile (MMA M)
+constexpr int kStageK = 128;        // k per stage
+constexpr int kStages = 4;
+constexpr int kDequantWarps = 8;
+constexpr int kThreads = (2 + kDequantWarps) * 32;
+constexpr int kWeightStageBytes = kTileN * (kStageK / 2);  // 8 KB
+constexpr uint32_t kTmemCols = 512;  // A: 2 x 64 columns, D: 2 x 128/g x BN = 256 columns
+
+template <int BN>
+struct Cfg {
+    static constexpr int kXAtomBytes = BN * 128;  // BN rows x 64 bf16
+    static constexpr int kStageBytes = 2 * kXAtomBytes + kWeightStageBytes;
+    static constexpr size_t kBarOff = (size_t)kStages * kStageBytes;
+    // full[S], empty[S], a_full[2], a_empty[2], d_full[2], d_empty[2], done, then flags
+    static constexpr size_t kFlagOff = kBarOff + (2 * kStages + 4 + 4 + 1) * 8;
+    static constexpr size_t kBytes = kFlagOff + 64;
+};
+
+struct Sched {
+    int64_t n_tiles, tiles, spt, total, per, extra;
+    __host__ __device__ int64_t cta_of(int64_t u) const
+    {
+        const int64_t big = extra * (per + 1);
+        return u < big ? u / (per + 1) : extra + (u - big) / per;
+    }
+    __host__ __device__ int64_t begin_of(int64_t b) const { return b * per + (b < extra ? b : extra); }
+};
+
+__device__ __forceinline__ uint32_t word_of4(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// (128 + q) - (128 + z) in bf16: exact for the integers involved (|q - z| <= 256).
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t q128, uint32_t zc)
+{
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&q128);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162 *>(&zc);
+    a = __hsub2(a, b);
+    return *reinterpret_cast<uint32_t *>(&a);
+}
+
+template <int BN, int GROUP>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, int64_t M,
+                     int64_t N, int64_t K, const uint16_t *__restrict__ sc, const uint16_t *__restrict__ zp,
+                     uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ counters, int max_segs,
+                     int *__restrict__ status)
+{
+    using C = Cfg<BN>;
+    constexpr int NG = kStageK / GROUP;     // groups per stage
+    constexpr int kDCols = NG * BN;         // accumulator columns per stage
+    static_assert(128 + 2 * kDCols <= (int)kTmemCols, "tensor memory budget");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *empty = full + kStages;
+    uint64_t *a_full = empty + kStages;
+    uint64_t *a_empty = a_full + 2;
+    uint64_t *d_full = a_empty + 2;
+    uint64_t *d_empty = d_full + 2;
+    uint64_t *done = d_empty + 2;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kFlagOff);
+    volatile int *last_flag = abort_flag + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kFlagOff + 16);
+
+    const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
+    Sched S;
+    S.n_tiles = (N + kTileN - 1) / kTileN;
+    S.tiles = S.n_tiles * ((M + BN - 1) / BN);
+    S.spt = K / kStageK;
+    S.total = S.tiles * S.spt;
+    S.per = S.total / gridDim.x;
+    S.extra = S.total % gridDim.x;
+    const int64_t beg = S.begin_of(blockIdx.x);
+    const int64_t end = beg + S.per + ((int64_t)blockIdx.x < S.extra ? 1 : 0);
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kDequantWarps + 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&a_full[a], kDequantWarps);
+            mbar_init(&a_empty[a], 1);
+            mbar_init(&d_full[a], 1);
+            mbar_init(&d_empty[a], kDequantWarps);
+        }
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        *last_flag = 0;
+        fence_mbar_init();
+    }
+    if (wid == 1) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t d_tmem = tmem + 128;  // accumulators: stage buffer b, group gi at 128 + (b * NG + gi) * BN
+
+    if (wid == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            int64_t it = 0;
+            for (int64_t u = beg; u < end; ++u, ++it) {
+                const int s = (int)(it % kStages);
+                const uint32_t use = (uint32_t)(it / kStages);
+                if (it >= kStages && !mbar_wait_fast(&empty[s], (use & 1u) ^ 1u, status, abort_flag)) break;
+                const int64_t tile = u / S.spt, ks = u - tile * S.spt;
+                const int64_t nt = tile % S.n_tiles, mt = tile / S.n_tiles;
+                uint8_t *st = smem + (size_t)s * C::kStageBytes;
+                mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+                tma_load_2d(st, &xmap, &full[s], (int)(ks * kStageK), (int)(mt * BN));
+                tma_load_2d(st + C::kXAtomBytes, &xmap, &full[s], (int)(ks * kStageK + 64), (int)(mt * BN));
+                tma_load_2d(st + 2 * C::kXAtomBytes, &wmap, &full[s], (int)(ks * (kStageK / 2)), (int)(nt * kTileN));
+            }
+            const int64_t first = it > kStages ? it - kStages : 0;
+            for (int64_t j = first; j < it; ++j) {
+                // drain: wait (bounded, ignoring the abort flag) until every issued copy landed
+                const uint64_t t0 = global_ns();
+                while (!mbar_try_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1)))
+                    if (global_ns() - t0 > kWaitLimitNs) { record_timeout(status); break; }
+            }
+        }
+    } else if (wid == 1) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+            int64_t it = 0;
+            for (int64_t u = beg; u < end;) {
+                const int64_t tile = u / S.spt;
+                const int64_t ks0 = u - tile * S.spt;
+                const int64_t ks1 = std::min<int64_t>(S.spt, ks0 + (end - u));
+                for (int64_t ks = ks0; ks < ks1; ++ks, ++it) {
+                    const int s = (int)(it % kStages);
+                    const int a = (int)(it & 1);
+                    mbar_wait_fast(&full[s], (uint32_t)((it / kStages) & 1), status, abort_flag);
+                    mbar_wait_fast(&a_full[a], (uint32_t)((it >> 1) & 1), status, abort_flag);
+                    if (it >= 2) mbar_wait_fast(&d_empty[a], (uint32_t)(((it >> 1) & 1) ^ 1), status, abort_flag);
+                    tc_fence_after();
+                    const uint32_t xs = smem_u32(smem + (size_t)s * C::kStageBytes);
+#pragma unroll
+                    for (int j = 0; j < kStageK / 16; ++j) {
+                        constexpr int kStepsPerGroup = GROUP / 16;
+                        const int gi = j / kStepsPerGroup;
+                        const uint32_t baddr = xs + (uint32_t)(j >> 2) * C::kXAtomBytes + (uint32_t)(j & 3) * 32u;
+                        const uint64_t bdesc = smem_desc(baddr, 16, 1024, 2);
+                        tc_mma_ts(d_tmem + (uint32_t)((a * NG + gi) * BN), tmem + (uint32_t)a * 64u + (uint32_t)j * 8u,
+                                  bdesc, idesc, (j % kStepsPerGroup) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty[s]);
+                    tc_commit(&a_empty[a]);
+                    tc_commit(&d_full[a]);
+                }
+                u += ks1 - ks0;
+            }
+            tc_commit(done);
+            // every MMA must have completed before tensor memory is released
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait(done, 0))
+                if (global_ns() - t0 > kWaitLimitNs) { record_timeout(status); break; }
+        }
+    } else {
+        // ------------------------------ dequant + promotion + epilogue ------------------------------
+        const int dw = wid - 2;            // 0..7
+        const int quarter = wid & 3;       // tensor-memory lanes 32*quarter .. +31
+        const int half = dw >> 2;          // k half of each stage, column half of the accumulators
+        const int r = quarter * 32 + lane; // row of the tile
+        const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
+        constexpr int kCols = BN / 2;      // accumulator columns this warp promotes
+        const int G = (int)(K / GROUP);
+        int64_t it = 0;
+        float acc[kCols];
+        float sprev[NG];                   // scales of the previous stage's groups (for its promotion)
+
+        // add s * D of stage `pit` (buffer pit & 1) to acc, then hand the buffer back to the MMA warp
+        auto promote = [&](int64_t pit) {
+            const int b = (int)(pit & 1);
+            mbar_wait_fast(&d_full[b], (uint32_t)((pit >> 1) & 1), status, abort_flag);
+            tc_fence_after();
+#pragma unroll
+            for (int gi = 0; gi < NG; ++gi) {
+#pragma unroll
+                for (int c0 = 0; c0 < kCols; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(d_tmem + lane_bits + (uint32_t)((b * NG + gi) * BN + half * kCols + c0), v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c0 + i < kCols) acc[c0 + i] = fmaf(sprev[gi], __uint_as_float(v[i]), acc[c0 + i]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&d_empty[b]);
+        };
+
+        for (int64_t u = beg; u < end;) {
+            const int64_t tile = u / S.spt;
+            const int64_t ks0 = u - tile * S.spt;
+            const int64_t ks1 = std::min<int64_t>(S.spt, ks0 + (end - u));
+            const int64_t nt = tile % S.n_tiles, mt = tile / S.n_tiles;
+            const int64_t n = nt * kTileN + r;
+            const int64_t nrow = n < N ? n : N - 1;
+            const uint16_t *srow = sc + nrow * G, *zrow = zp + nrow * G;
+#pragma unroll
+            for (int c = 0; c < kCols; ++c) acc[c] = 0.0f;
+
+            for (int64_t ks = ks0; ks < ks1; ++ks, ++it) {
+                const int s = (int)(it % kStages);
+                const int a = (int)(it & 1);
+                mbar_wait_fast(&full[s], (uint32_t)((it / kStages) & 1), status, abort_flag);
+                if (it >= 2) mbar_wait_fast(&a_empty[a], (uint32_t)(((it >> 1) & 1) ^ 1), status, abort_flag);
+                // this thread's 64 codes: row r, bytes [32*half, 32*half + 32) of the 64-byte row,
+                // stored with the 64-byte swizzle (16-byte chunk index ^= (row >> 1) & 3)
+                const uint32_t wbase = smem_u32(smem + (size_t)s * C::kStageBytes + 2 * C::kXAtomBytes) + r * 64;
+                const uint32_t sw = (uint32_t)((r >> 1) & 3);
+                uint4 wv[2];
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(wv[0].x), "=r"(wv[0].y), "=r"(wv[0].z), "=r"(wv[0].w)
+                             : "r"(wbase + 16u * ((2u * half) ^ sw)));
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(wv[1].x), "=r"(wv[1].y), "=r"(wv[1].z), "=r"(wv[1].w)
+                             : "r"(wbase + 16u * ((2u * half + 1u) ^ sw)));
+                // zero-points of this thread's 64 k (one or two groups), scales of the stage's groups
+                const int64_t k0 = ks * kStageK + half * 64;
+                const int gA = (int)(k0 / GROUP), gB = (int)((k0 + 32) / GROUP);
+                const float zA = 128.0f + bf16_to_f32(zrow[gA]), zB = 128.0f + bf16_to_f32(zrow[gB]);
+                const uint32_t zA2 = pack_bf16x2(zA, zA), zB2 = pack_bf16x2(zB, zB);
+                float scur[NG];
+#pragma unroll
+                for (int gi = 0; gi < NG; ++gi) scur[gi] = bf16_to_f32(srow[ks * NG + gi]);
+                uint32_t A[32];
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    const uint32_t v = w < 4 ? word_of4(wv[0], w) : word_of4(wv[1], w - 4);
+                    const uint32_t v4 = v >> 4;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t t = __byte_perm(v, v4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
+                        const uint32_t q128 = (t & 0x000F000Fu) | 0x43004300u;
+                        A[w * 4 + j] = bf2_sub(q128, w < 4 ? zA2 : zB2);
+                    }
+                }
+                // the codes are consumed: give the shared-memory slot back
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                tmem_st32(tmem + lane_bits + (uint32_t)a * 64u + (uint32_t)half * 32u, A);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[a]);
+                // promote the previous stage of this segment while this one is multiplied
+                if (ks > ks0) promote(it - 1);
+#pragma unroll
+                for (int gi = 0; gi < NG; ++gi) sprev[gi] = scur[gi];
+            }
+            promote(it - 1);  // the segment's last stage
+
+            // ---- segment output ----
+            const int64_t mbase = mt * BN + half * kCols;
+            const bool whole = (ks0 == 0 && ks1 == S.spt);
+            if (whole) {
+                if (n < N) {
+#pragma unroll
+                    for (int c = 0; c < kCols; ++c)
+                        if (mbase + c < M) y[(mbase + c) * N + n] = f32_to_bf16(acc[c]);
+                }
+            } else {
+                // partial of this segment -> workspace slot; the CTA that completes the tile sums them
+                const int64_t cta_first = S.cta_of(tile * S.spt);
+                const int64_t my_seg = (int64_t)blockIdx.x - cta_first;
+                const int64_t cta_last = S.cta_of(tile * S.spt + S.spt - 1);
+                float *slot = ws + ((tile * max_segs + my_seg) * BN) * kTileN;
+#pragma unroll
+                for (int c = 0; c < kCols; ++c) slot[(int64_t)(half * kCols + c) * kTileN + r] = acc[c];
+                __threadfence();
+                named_bar_sync(1, kDequantWarps * 32);
+                if (tid == 64) {
+                    const int add = (int)(ks1 - ks0);
+                    const int prev = atomicAdd(counters + tile, add);
+                    *last_flag = (prev + add == (int)S.spt) ? 1 : 0;
+                }
+                named_bar_sync(1, kDequantWarps * 32);
+                if (*last_flag) {
+                    __threadfence();
+                    for (int64_t o = 0; o <= cta_last - cta_first; ++o) {
+                        if (o == my_seg) continue;
+                        const float *other = ws + ((tile * max_segs + o) * BN) * kTileN;
+#pragma unroll
+                        for (int c = 0; c < kCols; ++c) acc[c] += __ldcg(other + (int64_t)(half * kCols + c) * kTileN + r);
+                    }
+                    if (n < N) {
+#pragma unroll
+                        for (int c = 0; c < kCols; ++c)
+                            if (mbase + c < M) y[(mbase + c) * N + n] = f32_to_bf16(acc[c]);
+                    }
+                    named_bar_sync(1, kDequantWarps * 32);
+                    if (tid == 64) atomicExch(counters + tile, 0);
+                }
+            }
+            u += ks1 - ks0;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (wid == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+template <int BN, int GROUP>
+int run(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s, const uint16_t *z,
+        uint16_t *y, void *workspace, int *status, cudaStream_t st)
+{
+    CUtensorMap wmap, xmap;
+    if (!encode_tmap_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, (uint64_t)(K / 2), (uint64_t)N, (uint64_t)(K / 2),
+                        kStageK / 2, kTileN, CU_TENSOR_MAP_SWIZZLE_64B))
+        return -1;
+    if (!encode_tmap_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, BN,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return -1;
+    auto kern = gemm_w4a16_tc_kernel<BN, GROUP>;
+    // at least 120 KB so that one CTA owns each SM (and its tensor memory)
+    const size_t smem = std::max<size_t>(Cfg<BN>::kBytes + 1024, 120 * 1024);
+    static std::mutex mu;
+    static std::map<int, int> sms_of;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int sms;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = sms_of.find(dev);
+        if (it == sms_of.end()) {
+            int v = 148, optin = 0;
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<32, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<32, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<32, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<64, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+            it = sms_of.emplace(dev, v).first;
+        }
+        sms = it->second;
+    }
+    const int64_t tiles = ((N + kTileN - 1) / kTileN) * ((M + BN - 1) / BN);
+    const int64_t total = tiles * (K / kStageK);
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(total, sms));
+    const int max_segs = (int)gemm_tc_max_segments(total, grid, K / kStageK);
+    uint8_t *w8 = static_cast<uint8_t *>(workspace);
+    float *ws = reinterpret_cast<float *>(w8);
+    int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, GROUP));
+    kern<<<(unsigned)grid, kThreads, smem, st>>>(wmap, xmap, M, N, K, s, z, y, ws, counters, max_segs, status);
+    return 0;
+}
+
+}  // namespace
+
+int gemm_tc_bn(int64_t M, int g)
+{
+    const int by_m = M <= 32 ? 32 : (M <= 64 ? 64 : 128);
+    const int by_g = g; // tensor-memory budget: 2 stages x (128 / g) groups x BN <= 256 columns
+    return by_m < by_g ? by_m : by_g;
+}
+
+int64_t gemm_tc_max_segments(int64_t total, int64_t grid, int64_t spt)
+{
+    const int64_t per = total / grid;  // >= 1
+    return (spt + per - 1) / per + 1;
+}
+
+size_t gemm_tc_partials_bytes(int64_t M, int64_t N, int64_t K, int g)
+{
+    const int BN = gemm_tc_bn(M, g);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t tiles = ((N + kTileN - 1) / kTileN) * ((M + BN - 1) / BN);
+    const int64_t spt = K / kStageK;
+    const int64_t total = tiles * spt;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(total, sms));
+    const int64_t segs = gemm_tc_max_segments(total, grid, spt);
+    const size_t b = sizeof(float) * (size_t)(tiles * segs * BN * kTileN);
+    return (b + 255) / 256 * 256;
+}
+
+bool gemm_tc_eligible(int64_t M, int64_t N, int64_t K, int g)
+{
+    return M > 16 && N >= kTileN && K >= kStageK && K % kStageK == 0 && (g == 32 || g == 64 || g == 128) &&
+           K / 2 <= 0xffffffffLL && M <= 0x7fffffffLL;
+}
+
+size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
+{
+    if (!gemm_tc_eligible(M, N, K, g)) return 0;
+    const int BN = gemm_tc_bn(M, g);
+    const int64_t tiles = ((N + kTileN - 1) / kTileN) * ((M + BN - 1) / BN);
+    return gemm_tc_partials_bytes(M, N, K, g) + (sizeof(int) * (size_t)tiles + 255) / 256 * 256;
+}
+
+int launch_gemm_w4a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
+                         const uint16_t *z, int g, uint16_t *y, void *workspace, int *status, cudaStream_t st)
+{
+    const int bn = gemm_tc_bn(M, g);
+    if (g == 32) return run<32, 32>(x, M, N, K, q, s, z, y, workspace, status, st);
+    if (g == 64) return bn == 32 ? run<32, 64>(x, M, N, K, q, s, z, y, workspace, status, st)
+                                 : run<64, 64>(x, M, N, K, q, s, z, y, workspace, status, st);
+    if (bn == 32) return run<32, 128>(x, M, N, K, q, s, z, y, workspace, status, st);
+    if (bn == 64) return run<64, 128>(x, M, N, K, q, s, z, y, workspace, status, st);
+    return run<128, 128>(x, M, N, K, q, s, z, y, workspace, status, st);
+}
+
+}  // namespace wq

@@ -125,17 +125,6 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity, int *
     }
 }
 
-__device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, int *status, volatile int *abort)
-{
-    return mbar_wait(bar, parity, status, abort);
-}
-
-// Common case inline (one try), the bounded loop out of line.
-__device__ __forceinline__ bool mbar_wait_fast(uint64_t *bar, uint32_t parity, int *status, volatile int *abort)
-{
-    return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, status, abort);
-}
-
 __device__ __forceinline__ uint4 lds128(uint32_t addr)
 {
     uint4 v;

@@ -27,6 +27,13 @@ def _lib():
     torch.cuda.init()
 
 
+@pytest.fixture(autouse=True)
+def _no_device_timeouts():
+    """Every test must leave the device status word clean (no bounded wait ran out)."""
+    yield
+    assert wq.wq_device_status() == wq.WQ_OK, "a kernel recorded a bounded-wait timeout"
+
+
 def bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
@@ -218,6 +225,13 @@ def test_gemm_w4a16_tiny():
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 7, 8, 9, 15, 16, 17, 31, 32, 33, 64, 127, 128, 129])
 def test_gemm_w4a16_batch_sizes(M):
     _w4_case(1000, 512, 128, M, 100 + M)
+
+
+@pytest.mark.parametrize("M,N,K,g", [(32, 128, 128, 128), (17, 256, 256, 64), (64, 384, 1024, 32),
+                                     (128, 130, 384, 128), (200, 512, 640, 128), (256, 128, 128, 32)])
+def test_gemm_w4a16_tensor_core_tiles(M, N, K, g):
+    """Shapes around the tcgen05 kernel's tile edges: one tile, ragged N, several M tiles, split K."""
+    _w4_case(N, K, g, M, 17 * M + N)
 
 
 @pytest.mark.parametrize("N,K,g", [(1, 32, 32), (7, 64, 32), (129, 128, 64), (300, 1024, 128), (33, 4096, 32)])
