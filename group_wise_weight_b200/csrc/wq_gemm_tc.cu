@@ -18,12 +18,13 @@
 // shared memory with the 128-byte swizzle.  The accumulator D lives in
 // tensor memory and is read back by the same warps for the epilogue.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads (weights box
-// [128 rows x 64 B] with the 64-byte swizzle, two activation boxes
-// [BN rows x 64 elements] with the 128-byte swizzle per 128-k stage); warp 1
-// allocates tensor memory and one of its lanes issues the MMAs; warps 2..9
-// dequantise (two warps per 32-lane quarter of tensor memory, each taking
-// half of the stage's 128 k) and run the epilogue.
+// Warp roles (352 threads): warp 0 issues TMA loads of weight boxes
+// [128 rows x 64 B] (64-byte swizzle) into a weight ring; warp 2 issues the
+// activation boxes [BN rows x 64 elements] (128-byte swizzle) into an
+// activation ring; warp 1 allocates tensor memory and one of its lanes issues
+// the MMAs; warps 3..10 dequantise (two warps per 32-lane quarter of tensor
+// memory, each taking half of the stage's 128 k), promote half of the
+// accumulator columns and write the output.
 //
 // Dequantisation: natural k order.  A code word v (8 codes, k .. k+7) and
 // v >> 4 give, with one byte permute and one LOP3 per pair, the bf16x2 pair
@@ -53,19 +54,26 @@ namespace {
 
 constexpr int kTileN = 128;         // weight rows per tile (MMA M)
 constexpr int kStageK = 128;        // k per stage
-constexpr int kStages = 4;
+constexpr int kWStages = 8;          // weight boxes in flight (released by the dequant warps)
 constexpr int kDequantWarps = 8;
-constexpr int kThreads = (2 + kDequantWarps) * 32;
+constexpr int kWPQ = kDequantWarps / 4;     // dequant warps per 32-lane quarter of tensor memory
+constexpr int kKPerWarp = 128 / kWPQ;       // k of a stage each dequant warp handles
+constexpr int kChunksPerWarp = kKPerWarp / 32;  // 16-byte code chunks per thread and stage
+constexpr int kFirstDequantWarp = 3;  // warps 0, 1, 2: weight producer, MMA issuer, activation producer
+constexpr int kThreads = (kFirstDequantWarp + kDequantWarps) * 32;
 constexpr int kWeightStageBytes = kTileN * (kStageK / 2);  // 8 KB
-constexpr uint32_t kTmemCols = 512;  // A: 2 x 64 columns, D: 2 x 128/g x BN = 256 columns
+constexpr uint32_t kTmemCols = 512;  // A: kABufs x 64 columns, D: 2 x 128/g x BN = 256 columns
+constexpr uint32_t kABufs = 4;       // dequantised weight tiles in tensor memory
 
 template <int BN>
 struct Cfg {
-    static constexpr int kXAtomBytes = BN * 128;  // BN rows x 64 bf16
-    static constexpr int kStageBytes = 2 * kXAtomBytes + kWeightStageBytes;
-    static constexpr size_t kBarOff = (size_t)kStages * kStageBytes;
-    // full[S], empty[S], a_full[2], a_empty[2], d_full[2], d_empty[2], done, then flags
-    static constexpr size_t kFlagOff = kBarOff + (2 * kStages + 4 + 4 + 1) * 8;
+    static constexpr int kXAtomBytes = BN * 128;             // BN rows x 64 bf16
+    static constexpr int kXStageBytes = 2 * kXAtomBytes;     // 128 k of activations
+    static constexpr int kXStages = BN == 128 ? 3 : (BN == 64 ? 4 : 6);
+    static constexpr size_t kWOff = (size_t)kXStages * kXStageBytes;
+    static constexpr size_t kBarOff = kWOff + (size_t)kWStages * kWeightStageBytes;
+    // x_full[XS], x_empty[XS], w_full[WS], w_empty[WS], a_full[A], a_empty[A], d_full[2], d_empty[2], done
+    static constexpr size_t kFlagOff = kBarOff + (2 * kXStages + 2 * kWStages + 2 * kABufs + 4 + 1) * 8;
     static constexpr size_t kBytes = kFlagOff + 64;
 };
 
@@ -93,6 +101,15 @@ __device__ __forceinline__ uint32_t bf2_sub(uint32_t q128, uint32_t zc)
     return *reinterpret_cast<uint32_t *>(&a);
 }
 
+// Slot and phase of a ring of `n` buffers, advanced one use at a time.
+struct Ring {
+    uint32_t slot = 0, phase = 0;
+    __device__ __forceinline__ void next(uint32_t n)
+    {
+        if (++slot == n) { slot = 0; phase ^= 1u; }
+    }
+};
+
 template <int BN, int GROUP>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, int64_t M,
@@ -103,14 +120,17 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     using C = Cfg<BN>;
     constexpr int NG = kStageK / GROUP;     // groups per stage
     constexpr int kDCols = NG * BN;         // accumulator columns per stage
-    static_assert(128 + 2 * kDCols <= (int)kTmemCols, "tensor memory budget");
+    constexpr uint32_t XS = (uint32_t)C::kXStages;
+    static_assert((int)kABufs * 64 + 2 * kDCols <= (int)kTmemCols, "tensor memory budget");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
-    uint64_t *empty = full + kStages;
-    uint64_t *a_full = empty + kStages;
-    uint64_t *a_empty = a_full + 2;
-    uint64_t *d_full = a_empty + 2;
+    uint64_t *x_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *x_empty = x_full + XS;
+    uint64_t *w_full = x_empty + XS;
+    uint64_t *w_empty = w_full + kWStages;
+    uint64_t *a_full = w_empty + kWStages;
+    uint64_t *a_empty = a_full + kABufs;
+    uint64_t *d_full = a_empty + kABufs;
     uint64_t *d_empty = d_full + 2;
     uint64_t *done = d_empty + 2;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kFlagOff);
@@ -127,17 +147,24 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     S.extra = S.total % gridDim.x;
     const int64_t beg = S.begin_of(blockIdx.x);
     const int64_t end = beg + S.per + ((int64_t)blockIdx.x < S.extra ? 1 : 0);
+    const int spt = (int)S.spt;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kDequantWarps + 1);
+        for (uint32_t i = 0; i < XS; ++i) {
+            mbar_init(&x_full[i], 1);
+            mbar_init(&x_empty[i], 1);
         }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(&a_full[a], kDequantWarps);
-            mbar_init(&a_empty[a], 1);
-            mbar_init(&d_full[a], 1);
-            mbar_init(&d_empty[a], kDequantWarps);
+        for (int i = 0; i < kWStages; ++i) {
+            mbar_init(&w_full[i], 1);
+            mbar_init(&w_empty[i], kDequantWarps);
+        }
+        for (uint32_t i = 0; i < kABufs; ++i) {
+            mbar_init(&a_full[i], kDequantWarps);
+            mbar_init(&a_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&d_full[i], 1);
+            mbar_init(&d_empty[i], kDequantWarps);
         }
         mbar_init(done, 1);
         *abort_flag = 0;
@@ -149,29 +176,41 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t d_tmem = tmem + 128;  // accumulators: stage buffer b, group gi at 128 + (b * NG + gi) * BN
+    const uint32_t d_tmem = tmem + kABufs * 64u;  // accumulators: stage buffer b, group gi at (b * NG + gi) * BN
 
-    if (wid == 0) {
-        // ------------------------------ TMA producer ------------------------------
-        if (lane == 0) {
-            int64_t it = 0;
-            for (int64_t u = beg; u < end; ++u, ++it) {
-                const int s = (int)(it % kStages);
-                const uint32_t use = (uint32_t)(it / kStages);
-                if (it >= kStages && !mbar_wait_fast(&empty[s], (use & 1u) ^ 1u, status, abort_flag)) break;
-                const int64_t tile = u / S.spt, ks = u - tile * S.spt;
-                const int64_t nt = tile % S.n_tiles, mt = tile / S.n_tiles;
-                uint8_t *st = smem + (size_t)s * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-                tma_load_2d(st, &xmap, &full[s], (int)(ks * kStageK), (int)(mt * BN));
-                tma_load_2d(st + C::kXAtomBytes, &xmap, &full[s], (int)(ks * kStageK + 64), (int)(mt * BN));
-                tma_load_2d(st + 2 * C::kXAtomBytes, &wmap, &full[s], (int)(ks * (kStageK / 2)), (int)(nt * kTileN));
+    if (wid == 0 || wid == 2) {
+        // ------------------------------ TMA producers ------------------------------
+        // warp 0: weight boxes into the weight ring; warp 2: activation boxes into the activation ring
+        const bool weights = wid == 0;
+        const uint32_t nst = weights ? (uint32_t)kWStages : XS;
+        uint64_t *fullb = weights ? w_full : x_full;
+        uint64_t *emptyb = weights ? w_empty : x_empty;
+        if (lane == 0 && beg < end) {
+            Ring rg;
+            uint32_t issued = 0;
+            int64_t tile = beg / spt;
+            int ks = (int)(beg - tile * spt);
+            for (int64_t u = beg; u < end; ++u) {
+                if (issued >= nst && !mbar_wait_fast(&emptyb[rg.slot], rg.phase ^ 1u, status, abort_flag)) break;
+                const int nt = (int)(tile % S.n_tiles), mt = (int)(tile / S.n_tiles);
+                if (weights) {
+                    mbar_arrive_expect_tx(&fullb[rg.slot], kWeightStageBytes);
+                    tma_load_2d(smem + C::kWOff + rg.slot * kWeightStageBytes, &wmap, &fullb[rg.slot],
+                                ks * (kStageK / 2), nt * kTileN);
+                } else {
+                    uint8_t *st = smem + rg.slot * C::kXStageBytes;
+                    mbar_arrive_expect_tx(&fullb[rg.slot], C::kXStageBytes);
+                    tma_load_2d(st, &xmap, &fullb[rg.slot], ks * kStageK, mt * BN);
+                    tma_load_2d(st + C::kXAtomBytes, &xmap, &fullb[rg.slot], ks * kStageK + 64, mt * BN);
+                }
+                ++issued;
+                rg.next(nst);
+                if (++ks == spt) { ks = 0; ++tile; }
             }
-            const int64_t first = it > kStages ? it - kStages : 0;
-            for (int64_t j = first; j < it; ++j) {
-                // drain: wait (bounded, ignoring the abort flag) until every issued copy landed
+            // drain: every issued copy must land before the CTA may exit (bounded, ignoring abort)
+            for (uint32_t j = issued > nst ? issued - nst : 0; j < issued; ++j) {
                 const uint64_t t0 = global_ns();
-                while (!mbar_try_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1)))
+                while (!mbar_try_wait(&fullb[j % nst], (j / nst) & 1u))
                     if (global_ns() - t0 > kWaitLimitNs) { record_timeout(status); break; }
             }
         }
@@ -179,31 +218,34 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
-            int64_t it = 0;
+            constexpr int kStepsPerGroup = GROUP / 16;
+            Ring xr, ar, dr;  // activation ring, A buffers, D double buffers
+            uint32_t it = 0;
+            const uint32_t xbase = smem_u32(smem);
             for (int64_t u = beg; u < end;) {
-                const int64_t tile = u / S.spt;
-                const int64_t ks0 = u - tile * S.spt;
-                const int64_t ks1 = std::min<int64_t>(S.spt, ks0 + (end - u));
-                for (int64_t ks = ks0; ks < ks1; ++ks, ++it) {
-                    const int s = (int)(it % kStages);
-                    const int a = (int)(it & 1);
-                    mbar_wait_fast(&full[s], (uint32_t)((it / kStages) & 1), status, abort_flag);
-                    mbar_wait_fast(&a_full[a], (uint32_t)((it >> 1) & 1), status, abort_flag);
-                    if (it >= 2) mbar_wait_fast(&d_empty[a], (uint32_t)(((it >> 1) & 1) ^ 1), status, abort_flag);
+                const int64_t tile = u / spt;
+                const int ks0 = (int)(u - tile * spt);
+                const int ks1 = (int)std::min<int64_t>(spt, ks0 + (end - u));
+                for (int ks = ks0; ks < ks1; ++ks, ++it) {
+                    mbar_wait_fast(&x_full[xr.slot], xr.phase, status, abort_flag);
+                    mbar_wait_fast(&a_full[ar.slot], ar.phase, status, abort_flag);
+                    if (it >= 2) mbar_wait_fast(&d_empty[dr.slot], dr.phase ^ 1u, status, abort_flag);
                     tc_fence_after();
-                    const uint32_t xs = smem_u32(smem + (size_t)s * C::kStageBytes);
+                    const uint32_t xs = xbase + xr.slot * (uint32_t)C::kXStageBytes;
+                    const uint32_t a_col = tmem + ar.slot * 64u;
+                    const uint32_t d_col = d_tmem + dr.slot * (uint32_t)kDCols;
 #pragma unroll
                     for (int j = 0; j < kStageK / 16; ++j) {
-                        constexpr int kStepsPerGroup = GROUP / 16;
-                        const int gi = j / kStepsPerGroup;
                         const uint32_t baddr = xs + (uint32_t)(j >> 2) * C::kXAtomBytes + (uint32_t)(j & 3) * 32u;
-                        const uint64_t bdesc = smem_desc(baddr, 16, 1024, 2);
-                        tc_mma_ts(d_tmem + (uint32_t)((a * NG + gi) * BN), tmem + (uint32_t)a * 64u + (uint32_t)j * 8u,
-                                  bdesc, idesc, (j % kStepsPerGroup) != 0 ? 1u : 0u);
+                        tc_mma_ts(d_col + (uint32_t)((j / kStepsPerGroup) * BN), a_col + (uint32_t)j * 8u,
+                                  smem_desc(baddr, 16, 1024, 2), idesc, (j % kStepsPerGroup) != 0 ? 1u : 0u);
                     }
-                    tc_commit(&empty[s]);
-                    tc_commit(&a_empty[a]);
-                    tc_commit(&d_full[a]);
+                    tc_commit(&x_empty[xr.slot]);
+                    tc_commit(&a_empty[ar.slot]);
+                    tc_commit(&d_full[dr.slot]);
+                    xr.next(XS);
+                    ar.next(kABufs);
+                    dr.next(2);
                 }
                 u += ks1 - ks0;
             }
@@ -215,104 +257,125 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         }
     } else {
         // ------------------------------ dequant + promotion + epilogue ------------------------------
-        const int dw = wid - 2;            // 0..7
-        const int quarter = wid & 3;       // tensor-memory lanes 32*quarter .. +31
-        const int half = dw >> 2;          // k half of each stage, column half of the accumulators
-        const int r = quarter * 32 + lane; // row of the tile
+        const int dw = wid - kFirstDequantWarp;  // 0 .. kDequantWarps-1
+        const int quarter = wid & 3;             // tensor-memory lanes 32*quarter .. +31
+        const int kq = dw >> 2;                  // k part of each stage, column part of the accumulators
+        const int r = quarter * 32 + lane;       // row of the tile
         const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
-        constexpr int kCols = BN / 2;      // accumulator columns this warp promotes
+        constexpr int kCols = BN / kWPQ;         // accumulator columns this warp promotes
         const int G = (int)(K / GROUP);
-        int64_t it = 0;
+        // this thread's code chunks in a weight slot: row r, chunks kq*kChunksPerWarp + i, 64-byte swizzle
+        uint32_t w_addr[kChunksPerWarp];
+#pragma unroll
+        for (int i = 0; i < kChunksPerWarp; ++i)
+            w_addr[i] = smem_u32(smem + C::kWOff) + (uint32_t)r * 64u +
+                        16u * ((uint32_t)(kq * kChunksPerWarp + i) ^ (uint32_t)((r >> 1) & 3));
+        const uint32_t a_addr = tmem + lane_bits + (uint32_t)(kq * kKPerWarp / 2);
+        const uint32_t dq_addr = d_tmem + lane_bits + (uint32_t)(kq * kCols);
+        Ring wr, ar, pr;  // weight ring, A buffers, D buffers being promoted
+        uint32_t it = 0;
         float acc[kCols];
-        float sprev[NG];                   // scales of the previous stage's groups (for its promotion)
+        float sprev[NG];
 
-        // add s * D of stage `pit` (buffer pit & 1) to acc, then hand the buffer back to the MMA warp
-        auto promote = [&](int64_t pit) {
-            const int b = (int)(pit & 1);
-            mbar_wait_fast(&d_full[b], (uint32_t)((pit >> 1) & 1), status, abort_flag);
+        // add s * D of the oldest unpromoted stage to acc, then hand its buffer back to the MMA warp
+        auto promote = [&]() {
+            mbar_wait_fast(&d_full[pr.slot], pr.phase, status, abort_flag);
             tc_fence_after();
 #pragma unroll
             for (int gi = 0; gi < NG; ++gi) {
+                const f32x2 s2{sprev[gi], sprev[gi]};
+                constexpr int kChunk = kCols < 16 ? kCols : 16;
 #pragma unroll
-                for (int c0 = 0; c0 < kCols; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(d_tmem + lane_bits + (uint32_t)((b * NG + gi) * BN + half * kCols + c0), v);
+                for (int c0 = 0; c0 < kCols; c0 += kChunk) {
+                    uint32_t v[kChunk];
+                    const uint32_t col = dq_addr + pr.slot * (uint32_t)kDCols + (uint32_t)(gi * BN + c0);
+                    if (kChunk == 16) tmem_ld16(col, v);
+                    else tmem_ld8(col, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (c0 + i < kCols) acc[c0 + i] = fmaf(sprev[gi], __uint_as_float(v[i]), acc[c0 + i]);
+                    for (int i = 0; i < kChunk; i += 2) {
+                        const f32x2 r2 = fma2(s2, f32x2{__uint_as_float(v[i]), __uint_as_float(v[i + 1])},
+                                              f32x2{acc[c0 + i], acc[c0 + i + 1]});
+                        acc[c0 + i] = r2.x;
+                        acc[c0 + i + 1] = r2.y;
+                    }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&d_empty[b]);
+            if (lane == 0) mbar_arrive(&d_empty[pr.slot]);
+            pr.next(2);
         };
 
         for (int64_t u = beg; u < end;) {
-            const int64_t tile = u / S.spt;
-            const int64_t ks0 = u - tile * S.spt;
-            const int64_t ks1 = std::min<int64_t>(S.spt, ks0 + (end - u));
+            const int64_t tile = u / spt;
+            const int ks0 = (int)(u - tile * spt);
+            const int ks1 = (int)std::min<int64_t>(spt, ks0 + (end - u));
             const int64_t nt = tile % S.n_tiles, mt = tile / S.n_tiles;
             const int64_t n = nt * kTileN + r;
             const int64_t nrow = n < N ? n : N - 1;
-            const uint16_t *srow = sc + nrow * G, *zrow = zp + nrow * G;
+            const uint16_t *sp = sc + nrow * G + (int64_t)ks0 * NG;  // scales of the stage's groups
+            const uint16_t *zbase = zp + nrow * G;                    // zero-points of the row
 #pragma unroll
             for (int c = 0; c < kCols; ++c) acc[c] = 0.0f;
 
-            for (int64_t ks = ks0; ks < ks1; ++ks, ++it) {
-                const int s = (int)(it % kStages);
-                const int a = (int)(it & 1);
-                mbar_wait_fast(&full[s], (uint32_t)((it / kStages) & 1), status, abort_flag);
-                if (it >= 2) mbar_wait_fast(&a_empty[a], (uint32_t)(((it >> 1) & 1) ^ 1), status, abort_flag);
-                // this thread's 64 codes: row r, bytes [32*half, 32*half + 32) of the 64-byte row,
-                // stored with the 64-byte swizzle (16-byte chunk index ^= (row >> 1) & 3)
-                const uint32_t wbase = smem_u32(smem + (size_t)s * C::kStageBytes + 2 * C::kXAtomBytes) + r * 64;
-                const uint32_t sw = (uint32_t)((r >> 1) & 3);
-                uint4 wv[2];
-                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(wv[0].x), "=r"(wv[0].y), "=r"(wv[0].z), "=r"(wv[0].w)
-                             : "r"(wbase + 16u * ((2u * half) ^ sw)));
-                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(wv[1].x), "=r"(wv[1].y), "=r"(wv[1].z), "=r"(wv[1].w)
-                             : "r"(wbase + 16u * ((2u * half + 1u) ^ sw)));
-                // zero-points of this thread's 64 k (one or two groups), scales of the stage's groups
-                const int64_t k0 = ks * kStageK + half * 64;
-                const int gA = (int)(k0 / GROUP), gB = (int)((k0 + 32) / GROUP);
-                const float zA = 128.0f + bf16_to_f32(zrow[gA]), zB = 128.0f + bf16_to_f32(zrow[gB]);
-                const uint32_t zA2 = pack_bf16x2(zA, zA), zB2 = pack_bf16x2(zB, zB);
+            for (int ks = ks0; ks < ks1; ++ks, ++it) {
+                mbar_wait_fast(&w_full[wr.slot], wr.phase, status, abort_flag);
+                if (it >= kABufs) {
+                    mbar_wait_fast(&a_empty[ar.slot], ar.phase ^ 1u, status, abort_flag);
+                    tc_fence_after();  // the tcgen05.st below must not move ahead of this wait
+                }
+                uint4 wv[kChunksPerWarp];
+#pragma unroll
+                for (int i = 0; i < kChunksPerWarp; ++i)
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(wv[i].x), "=r"(wv[i].y), "=r"(wv[i].z), "=r"(wv[i].w)
+                                 : "r"(w_addr[i] + wr.slot * (uint32_t)kWeightStageBytes));
                 float scur[NG];
 #pragma unroll
-                for (int gi = 0; gi < NG; ++gi) scur[gi] = bf16_to_f32(srow[ks * NG + gi]);
-                uint32_t A[32];
+                for (int gi = 0; gi < NG; ++gi) scur[gi] = bf16_to_f32(sp[gi]);
+                sp += NG;
+                uint32_t A[kKPerWarp / 2];
 #pragma unroll
-                for (int w = 0; w < 8; ++w) {
-                    const uint32_t v = w < 4 ? word_of4(wv[0], w) : word_of4(wv[1], w - 4);
-                    const uint32_t v4 = v >> 4;
+                for (int i = 0; i < kChunksPerWarp; ++i) {
+                    // zero-point of this 32-k chunk (a chunk never straddles a group: g >= 32)
+                    const int kc = ks * kStageK + (kq * kChunksPerWarp + i) * 32;
+                    const float zf = 128.0f + bf16_to_f32(zbase[kc / GROUP]);
+                    const uint32_t z2 = pack_bf16x2(zf, zf);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t t = __byte_perm(v, v4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
-                        const uint32_t q128 = (t & 0x000F000Fu) | 0x43004300u;
-                        A[w * 4 + j] = bf2_sub(q128, w < 4 ? zA2 : zB2);
+                    for (int w = 0; w < 4; ++w) {
+                        const uint32_t v = word_of4(wv[i], w);
+                        const uint32_t v4 = v >> 4;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t t = __byte_perm(v, v4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
+                            A[i * 16 + w * 4 + j] = bf2_sub((t & 0x000F000Fu) | 0x43004300u, z2);
+                        }
                     }
                 }
-                // the codes are consumed: give the shared-memory slot back
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-                tmem_st32(tmem + lane_bits + (uint32_t)a * 64u + (uint32_t)half * 32u, A);
+                if (kKPerWarp / 2 == 32) tmem_st32(a_addr + ar.slot * 64u, A);
+                else tmem_st16(a_addr + ar.slot * 64u, A);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[a]);
+                // tcgen05.st consumed the registers computed from the loaded codes, so no read of the
+                // weight slot can still be pending: hand both the slot and the A buffer over
+                if (lane == 0) {
+                    mbar_arrive(&w_empty[wr.slot]);
+                    mbar_arrive(&a_full[ar.slot]);
+                }
+                wr.next(kWStages);
+                ar.next(kABufs);
                 // promote the previous stage of this segment while this one is multiplied
-                if (ks > ks0) promote(it - 1);
+                if (ks > ks0) promote();
 #pragma unroll
                 for (int gi = 0; gi < NG; ++gi) sprev[gi] = scur[gi];
             }
-            promote(it - 1);  // the segment's last stage
+            promote();  // the segment's last stage
 
             // ---- segment output ----
-            const int64_t mbase = mt * BN + half * kCols;
-            const bool whole = (ks0 == 0 && ks1 == S.spt);
+            const int64_t mbase = mt * BN + kq * kCols;
+            const bool whole = (ks0 == 0 && ks1 == spt);
             if (whole) {
                 if (n < N) {
 #pragma unroll
@@ -321,18 +384,18 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 }
             } else {
                 // partial of this segment -> workspace slot; the CTA that completes the tile sums them
-                const int64_t cta_first = S.cta_of(tile * S.spt);
+                const int64_t cta_first = S.cta_of(tile * spt);
                 const int64_t my_seg = (int64_t)blockIdx.x - cta_first;
-                const int64_t cta_last = S.cta_of(tile * S.spt + S.spt - 1);
+                const int64_t cta_last = S.cta_of(tile * spt + spt - 1);
                 float *slot = ws + ((tile * max_segs + my_seg) * BN) * kTileN;
 #pragma unroll
-                for (int c = 0; c < kCols; ++c) slot[(int64_t)(half * kCols + c) * kTileN + r] = acc[c];
+                for (int c = 0; c < kCols; ++c) slot[(int64_t)(kq * kCols + c) * kTileN + r] = acc[c];
                 __threadfence();
                 named_bar_sync(1, kDequantWarps * 32);
-                if (tid == 64) {
-                    const int add = (int)(ks1 - ks0);
+                if (tid == kFirstDequantWarp * 32) {
+                    const int add = ks1 - ks0;
                     const int prev = atomicAdd(counters + tile, add);
-                    *last_flag = (prev + add == (int)S.spt) ? 1 : 0;
+                    *last_flag = (prev + add == spt) ? 1 : 0;
                 }
                 named_bar_sync(1, kDequantWarps * 32);
                 if (*last_flag) {
@@ -341,7 +404,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                         if (o == my_seg) continue;
                         const float *other = ws + ((tile * max_segs + o) * BN) * kTileN;
 #pragma unroll
-                        for (int c = 0; c < kCols; ++c) acc[c] += __ldcg(other + (int64_t)(half * kCols + c) * kTileN + r);
+                        for (int c = 0; c < kCols; ++c) acc[c] += __ldcg(other + (int64_t)(kq * kCols + c) * kTileN + r);
                     }
                     if (n < N) {
 #pragma unroll
@@ -349,7 +412,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                             if (mbase + c < M) y[(mbase + c) * N + n] = f32_to_bf16(acc[c]);
                     }
                     named_bar_sync(1, kDequantWarps * 32);
-                    if (tid == 64) atomicExch(counters + tile, 0);
+                    if (tid == kFirstDequantWarp * 32) atomicExch(counters + tile, 0);
                 }
             }
             u += ks1 - ks0;
