@@ -561,7 +561,9 @@ void run_w4_mma(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_
 void launch_gemv_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
                        const uint16_t *z, int g, uint16_t *y, cudaStream_t st)
 {
-    if (g == 128 && M <= 16) {
+    // M = 1: the CUDA-core form below measured fastest.  2 <= M <= 16 normally takes the TMA
+    // pipeline (wq_gemv_tma.cu); shapes it does not take (N < 128, K < 256) come here.
+    if (g == 128 && M >= 2 && M <= 16) {
         if (M <= 8) run_w4_mma<1, 1, 4, 2>(x, M, N, K, q, s, z, y, st);
         else run_w4_mma<2, 1, 4, 2>(x, M, N, K, q, s, z, y, st);
         return;
