@@ -68,6 +68,8 @@ def lib():
         L.wq_gemm_w4a16.restype = I
         L.wq_gemm_w8a16.argtypes = [P, I64, I64, I64, P, P, I, P, P, SZ, P]
         L.wq_gemm_w8a16.restype = I
+        L.wq_gemm_w4a16_noalloc.argtypes = [P, I64, I64, I64, P, P, P, I, P, P]
+        L.wq_gemm_w4a16_noalloc.restype = I
         L.wq_device_status.argtypes = [P]
         L.wq_device_status.restype = I
         _lib = L
@@ -206,6 +208,23 @@ def wq_gemm_w8a16(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, 
     _check(lib().wq_gemm_w8a16(_dev(x, "x"), M, N, K, _dev(qweight, "qweight"), _dev(scales, "scales"), g,
                                _dev(y, "y"), workspace.data_ptr() if workspace is not None else None, ws_bytes,
                                _stream_handle(stream)))
+    return y
+
+
+def wq_gemm_w4a16_noalloc(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                          g: int = 128, y=None, stream=None) -> torch.Tensor:
+    """wq_gemm_w4a16 for callers that cannot allocate device memory: the C entry point takes no
+    workspace and uses the library's fixed 2 MiB scratch array (2 <= M <= 16, g = 128; see wq.h).
+    Pass `y` to avoid the output allocation here as well."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    _dense(x, "x")
+    M, K = x.shape
+    N = qweight.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dense(y, "y")
+    _check(lib().wq_gemm_w4a16_noalloc(_dev(x, "x"), M, N, K, _dev(qweight, "qweight"), _dev(scales, "scales"),
+                                       _dev(zeros, "zeros"), int(g), _dev(y, "y"), _stream_handle(stream)))
     return y
 
 

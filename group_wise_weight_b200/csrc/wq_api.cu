@@ -92,6 +92,22 @@ int *status_word()
 
 }  // namespace
 
+namespace wq {
+
+// Record `msg` as this thread's last error and return `status` (for entry points in other files).
+int record_error(int status, const char *msg)
+{
+    g_last_error = msg;
+    return status;
+}
+
+void clear_error() { g_last_error.clear(); }
+
+// Device address of the per-device status word on the current device (nullptr on failure).
+int *device_status_word() { return status_word(); }
+
+}  // namespace wq
+
 extern "C" {
 
 const char *wq_status_str(int status)

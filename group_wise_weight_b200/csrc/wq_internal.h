@@ -39,4 +39,9 @@ size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
 int launch_gemm_w4a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
                          const uint16_t *z, int g, uint16_t *y, void *workspace, int *status, cudaStream_t st);
 
+// Error reporting and the bounded-wait status word, for entry points outside wq_api.cu.
+int record_error(int status, const char *msg);
+void clear_error();
+int *device_status_word();
+
 }  // namespace wq

@@ -152,6 +152,30 @@ int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8
                   void *stream);
 
 /*
+ * W4A16 matmul for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this is an interface variant, not part of the method.
+ *
+ * Same operation, arguments and accuracy as wq_gemm_w4a16, but no workspace
+ * argument: the split-K partial sums and tile counters live in a fixed 2 MiB
+ * array inside the library (held on every GPU that loads the library until
+ * the process exits).  For callers that cannot call cudaMalloc -- it
+ * synchronises the device, and runtimes or plug-in hosts that own all device
+ * memory, or fixed-budget deployments, forbid allocation after start-up.
+ *
+ *   Accepted shapes: g == 128, 2 <= M <= 16, N >= 128, K >= 256, K % 128 == 0
+ *   (WQ_ERR_UNSUPPORTED otherwise), and M * N * 4 bytes plus one int per 128
+ *   rows of N must fit in the 2 MiB array (WQ_ERR_WORKSPACE otherwise).
+ *   The first call with a given device current looks up the array's device
+ *   address (cudaGetSymbolAddress); make it before any stream capture.
+ *   Each call clears the part of the array it uses on `stream` before its
+ *   kernel runs.  All calls share the array: calls whose executions overlap on
+ *   the GPU (other streams, other host threads) race on it.
+ *   Allocates nothing; calls no cudaMalloc or cudaFree.
+ */
+int wq_gemm_w4a16_noalloc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *qweight,
+                          const uint16_t *scales, const uint16_t *zeros, int g, uint16_t *y, void *stream);
+
+/*
  * Device status word.  Kernels with waits on barriers bound every wait; a
  * wait that runs out records a code on the device and the kernel returns
  * early instead of hanging.  This call synchronises `stream`, returns
