@@ -154,6 +154,7 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
     if (M <= 0 || N <= 0 || K <= 0) return 0;
     if (wbits == 4) {
         if (wq::gemm_tc_eligible(M, N, K, g)) return wq::gemm_tc_workspace_bytes(M, N, K, g);
+        if (wq::gemv_m1_eligible(M, N, K, g)) return wq::gemv_m1_workspace_bytes(M, N, K, g);
         return wq::gemv_tma_workspace_bytes(M, N, K, g);
     }
     return 0;
@@ -175,6 +176,13 @@ int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint
         if (!status) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: no device status word");
         if (wq::launch_gemm_w4a16_tc(x, M, N, K, qweight, scales, zeros, g, y, workspace, status, st) != 0)
             return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: tensor map encoding failed");
+        return check_launch("wq_gemm_w4a16");
+    }
+    if (wq::gemv_m1_eligible(M, N, K, g)) {
+        int *status = status_word();
+        if (!status) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: no device status word");
+        const int rc = wq::launch_gemv_w4a16_m1(x, N, K, qweight, scales, zeros, y, workspace, status, st);
+        if (rc == -1) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: tensor map encoding failed");
         return check_launch("wq_gemm_w4a16");
     }
     if (wq::gemv_tma_eligible(M, N, K, g)) {

@@ -19,6 +19,16 @@ void launch_gemv_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const
 void launch_gemv_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *q, const uint16_t *s,
                        int g, uint16_t *y, cudaStream_t st);
 
+// W4A16 for M = 1, group 128 (wq_gemv_m1.cu): persistent stream-K over
+// (32-row block, group) units, per-warp TMA pipelines, mma.sync.  Needs a
+// workspace of gemv_m1_workspace_bytes() (zero-filled before first use; the
+// kernel leaves its counters zeroed) and the device status word for its
+// bounded waits.  Returns 0, or -1 if a tensor map cannot be encoded.
+bool gemv_m1_eligible(int64_t M, int64_t N, int64_t K, int g);
+size_t gemv_m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
+int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
+                         const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st);
+
 // TMA-pipelined W4A16 for group 128 and M <= 16 (wq_gemv_tma.cu).  Needs a
 // workspace of gemv_tma_workspace_bytes() (zero-filled before first use; the
 // kernel leaves it zeroed).  Returns 0, or -1 if the tensor map could not be

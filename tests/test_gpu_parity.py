@@ -240,6 +240,31 @@ def test_gemm_w4a16_shapes(N, K, g, M):
     _w4_case(N, K, g, M, 7 * N + K + M)
 
 
+@pytest.mark.parametrize("N,K", [(1, 1024), (33, 1024), (31, 3072), (64, 32768), (4097, 2048), (8192, 8192),
+                                 (100, 65536), (4097, 1152)])
+def test_gemm_w4a16_m1_stream_k_edges(N, K):
+    """M = 1, group 128: a single row, ragged row blocks, the largest K of the TMA kernel, more warps than
+    units; and two shapes it does not take (K > 32768, K not a multiple of 1024)."""
+    _w4_case(N, K, 128, 1, 11 * N + K)
+
+
+def test_gemm_w4a16_m1_workspace_reuse():
+    """Calls that share one workspace find it ready (its counters re-zeroed by the previous call) and the
+    split-K combine runs in a fixed order: the same inputs give the same bytes every time."""
+    N, K = 3000, 4096
+    w = wq_inputs.llm_weight(N, K, 77)
+    q, s, z = wq.wq_quantize_int4(w.cuda(), 128)
+    ws = torch.zeros(wq.wq_gemm_workspace_bytes(1, N, K, 128, 4) + 16, dtype=torch.uint8, device="cuda")
+    outs = []
+    for seed in (1, 2, 1, 2, 1):
+        x = wq_inputs.activations(1, K, seed).cuda()
+        outs.append(wq.wq_gemm_w4a16(x, q, s, z, 128, workspace=ws).clone())
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[2]) and torch.equal(outs[0], outs[4])
+    assert torch.equal(outs[1], outs[3])
+    assert not torch.equal(outs[0], outs[1])
+
+
 def test_gemm_w4a16_degenerate_groups():
     w = wq_inputs.llm_weight(64, 512, 81, dtype=torch.float32)
     w[0] = 0.0
