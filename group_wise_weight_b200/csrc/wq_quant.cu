@@ -29,6 +29,25 @@ namespace {
 constexpr int kQuantThreads = 256;
 constexpr int kQuantUnroll = 4;  // row chunks in flight per warp
 
+// Position (row n, 256-weight chunk c) of a warp's task t = n * chunks + c, advanced by the grid's warp
+// count without a 64-bit division per task.
+struct TaskWalk {
+    int64_t n, c, dn, dc, chunks;
+    __device__ __forceinline__ TaskWalk(int64_t t, int64_t stride, int64_t chunks_) : chunks(chunks_)
+    {
+        n = t / chunks;
+        c = t - n * chunks;
+        dn = stride / chunks;
+        dc = stride - dn * chunks;
+    }
+    __device__ __forceinline__ void step()
+    {
+        n += dn;
+        c += dc;
+        if (c >= chunks) { c -= chunks; ++n; }
+    }
+};
+
 template <typename T>
 __device__ __forceinline__ void load8(const T *p, float v[8]);
 
@@ -79,17 +98,18 @@ quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
     const int64_t tasks = N * chunks;
     const int64_t G = K / g;
 
+    TaskWalk walk(warp0, n_warps, chunks);
     for (int64_t t0 = warp0; t0 < tasks; t0 += n_warps * kQuantUnroll) {
         float v[kQuantUnroll][8];
         int64_t n[kQuantUnroll], k0[kQuantUnroll];
         bool active[kQuantUnroll];
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
-            const int64_t t = t0 + u * n_warps;
-            n[u] = t / chunks;
-            k0[u] = (t - n[u] * chunks) * 256 + lane * 8;
-            active[u] = (t < tasks) && (k0[u] < K);
+            n[u] = walk.n;
+            k0[u] = walk.c * 256 + lane * 8;
+            active[u] = (walk.n < N) && (k0[u] < K);
             if (active[u]) load8<T>(w + n[u] * ldw + k0[u], v[u]);
+            walk.step();
         }
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
@@ -156,17 +176,18 @@ quant_int8_group_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t l
     const int64_t tasks = N * chunks;
     const int64_t G = K / g;
 
+    TaskWalk walk(warp0, n_warps, chunks);
     for (int64_t t0 = warp0; t0 < tasks; t0 += n_warps * kQuantUnroll) {
         float v[kQuantUnroll][8];
         int64_t n[kQuantUnroll], k0[kQuantUnroll];
         bool active[kQuantUnroll];
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
-            const int64_t t = t0 + u * n_warps;
-            n[u] = t / chunks;
-            k0[u] = (t - n[u] * chunks) * 256 + lane * 8;
-            active[u] = (t < tasks) && (k0[u] < K);
+            n[u] = walk.n;
+            k0[u] = walk.c * 256 + lane * 8;
+            active[u] = (walk.n < N) && (k0[u] < K);
             if (active[u]) load8<T>(w + n[u] * ldw + k0[u], v[u]);
+            walk.step();
         }
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
