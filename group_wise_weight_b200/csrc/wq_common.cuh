@@ -74,6 +74,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
     return (uint32_t)f32_to_bf16(a) | ((uint32_t)f32_to_bf16(b) << 16);
 }
 
+// (128 + q) - (128 + z) on a bf16 pair: exact for the integers of a code and a zero-point (any integer of
+// magnitude <= 256 is a bf16 value), so a matmul operand built this way holds q - z itself.
+__device__ __forceinline__ uint32_t sub_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 // ---------------------------------------------------------------------------
 // Mixed-precision FMA: d = a * b + c with bf16 a, b and binary32 c, d
 // (the product of two bf16 is exact in binary32; one rounding).

@@ -36,15 +36,18 @@
 //    of its part of the A operand of eight k16 steps; the k order inside a
 //    step is permuted accordingly and the activation pairs are staged in
 //    shared memory in the same permuted order.
-//  * Per group and row the binary32 accumulator takes
-//    s * (D - (128 + z) * X), D the tensor-core sum of x (128 + q) and X the
-//    group sum of x: (q - z) is never rounded and s is applied in binary32.
+//  * Subtracting the bf16 pair (128 + z, 128 + z) from each code pair gives
+//    the exact integers q - z, so the tensor core sums x (q - z) per group and
+//    the binary32 accumulator takes s * D: no term carries an offset that has
+//    to cancel later, rows whose weights are all zero give exactly zero, and
+//    the rounding error stays proportional to sum |x w_hat|.
 //  * A tile split between CTAs leaves one binary32 partial per segment in the
-//    workspace; the CTA that completes it (arrival counter) sums the partials
-//    in segment order, writes y and re-zeroes the counter, so results do not
+//    workspace; for each warp's 16 rows, the warp that arrives last (one
+//    arrival counter per tile and warp, no CTA barrier) sums the partials in
+//    segment order, writes y and re-zeroes the counter, so results do not
 //    depend on timing.
 //  * x is copied into shared memory with one bulk asynchronous copy, then
-//    permuted in place and its group sums formed.
+//    permuted in place.
 //  * Launched with programmatic dependent launch: in a stream of linears the
 //    next kernel's CTAs start as SMs free up, initialise their barriers and
 //    prefetch their first weight stages into L2 while this one finishes; they
@@ -76,10 +79,10 @@ constexpr uint32_t kSzBytes = kTile * 16;         // 256 rows x 8 groups x 2 B (
 constexpr uint32_t kBulkPiece = 16384;            // bytes per bulk copy of x
 constexpr int kPairsPerWindow = 4;                // 8 groups of s/z = 4 units
 
-// shared memory: [x pairs 2K][group sums K/128 x 4][pad to 1024][stages][s/z windows][barriers]
+// shared memory: [x pairs 2K][pad to 1024][stages][s/z windows][barriers]
 __host__ __device__ __forceinline__ size_t m1_ring_offset(int64_t K)
 {
-    return ((size_t)K * 2 + (size_t)(K / 128) * 4 + 1023) & ~(size_t)1023;
+    return ((size_t)K * 2 + 1023) & ~(size_t)1023;
 }
 __host__ __device__ __forceinline__ size_t m1_sz_offset(int64_t K) { return m1_ring_offset(K) + kStages * kStageBytes; }
 __host__ __device__ __forceinline__ size_t m1_bar_offset(int64_t K) { return m1_sz_offset(K) + 2 * 2 * kSzBytes; }
@@ -183,7 +186,6 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     // TMA destinations want 128-byte (we keep 1024-byte) alignment: align the base explicitly
     uint8_t *sm = m1_raw + ((1024u - (smem_u32(m1_raw) & 1023u)) & 1023u);
     uint4 *xp = reinterpret_cast<uint4 *>(sm);                    // K / 8 chunks of 8 activations
-    float *xg = reinterpret_cast<float *>(sm + (size_t)K * 2);    // K / 128 group sums
     uint8_t *ring = sm + m1_ring_offset(K);
     uint8_t *szr = sm + m1_sz_offset(K);                          // [2 windows][s, z][256 rows][8 groups]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + m1_bar_offset(K));
@@ -272,16 +274,11 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 
     // ================================ consumers ================================
     if (n > 0) {
-        // ---- x: wait for the bulk copy, permute each chunk in place, group sums ----
+        // ---- x: wait for the bulk copy, permute each chunk in place ----
         mbar_wait(xbar, 0, status, flags);
-        for (int c0 = 0; c0 < K / 8; c0 += kC * 32) {
-            const int c = c0 + tid;  // K / 8 is a multiple of 16: groups never straddle the bound
-            float part = 0.0f;
-            if (c < K / 8) {
+        for (int c = tid; c < K / 8; c += kC * 32) {
+            {
                 const uint4 v = xp[c];
-                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) part += __uint_as_float(u[i] << 16) + __uint_as_float(u[i] & 0xffff0000u);
                 uint4 pr;
                 pr.x = __byte_perm(v.x, v.z, 0x5410);  // (x0, x4)
                 pr.y = __byte_perm(v.x, v.z, 0x7632);  // (x1, x5)
@@ -289,9 +286,6 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 pr.w = __byte_perm(v.y, v.w, 0x7632);  // (x3, x7)
                 xp[c] = pr;
             }
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-            if (c < K / 8 && (c & 15) == 0) xg[c >> 4] = part;
         }
         named_bar_sync(1, kC * 32);
 
@@ -325,14 +319,16 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             const int kg = 2 * p;
             const uint32_t szsrc =
                 szr_u32 + (uint32_t)(win & 1) * 2u * kSzBytes + (uint32_t)r0 * 16u + (uint32_t)(kg & 7) * 2u;
-            float sv[2][2], zc[2][2];
+            float sv[2][2];
+            uint32_t zz[2][2];  // bf16 pairs (128 + z, 128 + z)
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
                     const uint32_t o = szsrc + (uint32_t)a * 8u * 16u + (uint32_t)h * 2u;
                     sv[h][a] = __uint_as_float(lds_u16(o) << 16);
-                    zc[h][a] = 128.0f + __uint_as_float(lds_u16(o + kSzBytes) << 16);
+                    const float zf = 128.0f + __uint_as_float(lds_u16(o + kSzBytes) << 16);
+                    zz[h][a] = pack_bf16x2(zf, zf);
                 }
             // the stage's weight bytes are in registers: hand the slot back to the producer
             __syncwarp();
@@ -342,22 +338,24 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 uint4 Pw[4];
 #pragma unroll
                 for (int w = 0; w < 4; ++w) Pw[w] = lds128(xp_u32 + (uint32_t)((kg + h) * 16 + tq * 4 + w) * 16u);
-                const float X = xg[kg + h];
                 float C0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, C1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
                     const uint32_t va = word_of(wv[h][0], w), vb = word_of(wv[h][1], w);
                     float *C = (w & 1) ? C1 : C0;
-                    mma_bf16(C, nib_pair(va, 0, nib_mask, bf16_magic), nib_pair(vb, 0, nib_mask, bf16_magic),
-                             nib_pair(va, 4, nib_mask, bf16_magic), nib_pair(vb, 4, nib_mask, bf16_magic), Pw[w].x,
-                             Pw[w].y);
-                    mma_bf16(C, nib_pair(va, 8, nib_mask, bf16_magic), nib_pair(vb, 8, nib_mask, bf16_magic),
-                             nib_pair(va, 12, nib_mask, bf16_magic), nib_pair(vb, 12, nib_mask, bf16_magic), Pw[w].z,
-                             Pw[w].w);
+                    const uint32_t za = zz[h][0], zb = zz[h][1];
+                    mma_bf16(C, sub_bf16x2(nib_pair(va, 0, nib_mask, bf16_magic), za),
+                             sub_bf16x2(nib_pair(vb, 0, nib_mask, bf16_magic), zb),
+                             sub_bf16x2(nib_pair(va, 4, nib_mask, bf16_magic), za),
+                             sub_bf16x2(nib_pair(vb, 4, nib_mask, bf16_magic), zb), Pw[w].x, Pw[w].y);
+                    mma_bf16(C, sub_bf16x2(nib_pair(va, 8, nib_mask, bf16_magic), za),
+                             sub_bf16x2(nib_pair(vb, 8, nib_mask, bf16_magic), zb),
+                             sub_bf16x2(nib_pair(va, 12, nib_mask, bf16_magic), za),
+                             sub_bf16x2(nib_pair(vb, 12, nib_mask, bf16_magic), zb), Pw[w].z, Pw[w].w);
                 }
                 // every column of D carries the same x: C[0] is row r0, C[2] row r0 + 8
-                acc[0] = fmaf(sv[h][0], fmaf(-zc[h][0], X, C0[0] + C1[0]), acc[0]);
-                acc[1] = fmaf(sv[h][1], fmaf(-zc[h][1], X, C0[2] + C1[2]), acc[1]);
+                acc[0] = fmaf(sv[h][0], C0[0] + C1[0], acc[0]);
+                acc[1] = fmaf(sv[h][1], C0[2] + C1[2], acc[1]);
             }
             // ---- end of a segment: the tile's last pair, or the end of this CTA's range ----
             const bool tile_done = (p + 1 == P);
@@ -369,39 +367,41 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                         if (row0 + 8 < N) y[row0 + 8] = f32_to_bf16(acc[1]);
                     }
                 } else {
-                    // partial: this CTA's slot; the CTA that completes the tile sums the slots in segment
-                    // order (a fixed order: the result does not depend on timing)
+                    // partial: this warp's 16 rows go to this CTA's slot; the warp that arrives last for those
+                    // rows (one counter per tile and warp) sums the slots in segment order -- even and odd
+                    // segments in two lanes, then added: a fixed order, so the result does not depend on timing
                     const int64_t c_first = cta_of((int64_t)t * P, units, B);
                     const int nseg = (int)(cta_of((int64_t)t * P + P - 1, units, B) - c_first) + 1;
-                    float *slots = ws + (size_t)t * max_segs * kTile;
+                    float *slots = ws + (size_t)t * max_segs * kTile + 16 * wid;
+                    int *wcnt = cnt + (size_t)t * kC + wid;
                     if (tq == 0) {
-                        slots[(bid - c_first) * kTile + r0] = acc[0];
-                        slots[(bid - c_first) * kTile + r0 + 8] = acc[1];
+                        slots[(bid - c_first) * kTile + gq] = acc[0];
+                        slots[(bid - c_first) * kTile + gq + 8] = acc[1];
                     }
-                    named_bar_sync(1, kC * 32);
-                    if (tid == 0) flags[1] = (atom_add_acq_rel(cnt + t, 1) + 1 == nseg) ? 1 : 0;
-                    named_bar_sync(1, kC * 32);
-                    if (flags[1]) {
-                        if (tid < kTile) {
-                            // thread tid sums row tid over the segments in order, four loads in flight
-                            const float *q = slots + tid;
-                            float v = 0.0f;
-                            int o = 0;
-                            for (; o + 4 <= nseg; o += 4) {
-                                const float a0 = __ldcg(q + (o + 0) * kTile), a1 = __ldcg(q + (o + 1) * kTile);
-                                const float a2 = __ldcg(q + (o + 2) * kTile), a3 = __ldcg(q + (o + 3) * kTile);
-                                v += a0;
-                                v += a1;
-                                v += a2;
-                                v += a3;
-                            }
-                            for (; o < nseg; ++o) v += __ldcg(q + o * kTile);
-                            const int row = t * kTile + tid;
-                            if (row < N) y[row] = f32_to_bf16(v);
+                    __syncwarp();
+                    int last = 0;
+                    if (lane == 0) last = (atom_add_acq_rel(wcnt, 1) + 1 == nseg) ? 1 : 0;
+                    last = __shfl_sync(0xffffffffu, last, 0);
+                    __syncwarp();
+                    if (last) {
+                        const int rr = lane & 15;
+                        const float *q = slots + rr;
+                        float v = 0.0f;
+                        int o = lane >> 4;
+                        for (; o + 6 < nseg; o += 8) {
+                            const float a0 = __ldcg(q + (o + 0) * kTile), a1 = __ldcg(q + (o + 2) * kTile);
+                            const float a2 = __ldcg(q + (o + 4) * kTile), a3 = __ldcg(q + (o + 6) * kTile);
+                            v += a0;
+                            v += a1;
+                            v += a2;
+                            v += a3;
                         }
-                        if (tid == 0) atomicExch(cnt + t, 0);
+                        for (; o < nseg; o += 2) v += __ldcg(q + o * kTile);
+                        v += __shfl_xor_sync(0xffffffffu, v, 16);
+                        const int row = t * kTile + 16 * wid + rr;
+                        if (lane < 16 && row < N) y[row] = f32_to_bf16(v);
+                        if (lane == 0) atomicExch(wcnt, 0);
                     }
-                    named_bar_sync(1, kC * 32);  // flags[1] is rewritten at the next partial segment
                 }
                 acc[0] = acc[1] = 0.0f;
             }
@@ -464,7 +464,7 @@ size_t gemv_m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
 {
     if (!gemv_m1_eligible(M, N, K, g)) return 0;
     const int64_t ntiles = (N + kTile - 1) / kTile;
-    return m1_slots_bytes(N, K, m1_grid(N, K)) + ((size_t)ntiles * 4 + 255) / 256 * 256;
+    return m1_slots_bytes(N, K, m1_grid(N, K)) + ((size_t)ntiles * kC * 4 + 255) / 256 * 256;
 }
 
 int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,

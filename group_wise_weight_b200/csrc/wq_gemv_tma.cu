@@ -17,13 +17,15 @@
 //    the consumers never wait on global-memory latency for weights.
 //  * Consumer warp w owns rows 16w..16w+15 of the tile.  Each lane reads the
 //    16 bytes of rows n and n+8 it needs (512 contiguous bytes per warp, no
-//    bank conflicts), turns every code pair into bf16 128 + q with one LOP3,
-//    and issues mma.sync m16n8k16 with the weights as the 16-row operand
-//    and the activations (pre-permuted to the same k order) as the 8-column
-//    operand; the k permutation is the one described in wq_gemv.cu.
-//  * Per chunk (= group) the binary32 accumulator takes
-//    s * (C - (128 + z) * X), X the group sum of the activations, so (q - z)
-//    is exact and s is applied in binary32.
+//    bank conflicts), turns every code pair into bf16 128 + q with one LOP3
+//    and subtracts the pair (128 + z, 128 + z), which leaves the exact
+//    integers q - z, and issues mma.sync m16n8k16 with the weights as the
+//    16-row operand and the activations (pre-permuted to the same k order) as
+//    the 8-column operand; the k permutation is the one described in
+//    wq_gemv.cu.
+//  * Per chunk (= group) the binary32 accumulator takes s * C: (q - z) is
+//    exact, s is applied in binary32, and no term carries an offset that
+//    would have to cancel later (rows of zeros give exactly zero).
 //  * A tile split between CTAs is combined in a binary32 workspace with
 //    atomics; the CTA whose contribution completes the tile's K range
 //    converts it to bf16, re-zeroes the workspace and resets the tile's
@@ -74,7 +76,7 @@ constexpr int kConsumers = 8;
 constexpr int kThreads = (kConsumers + 1) * 32;
 
 struct SmemLayout {
-    size_t bars, flags, xs, xp, total;
+    size_t bars, flags, xp, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -85,8 +87,7 @@ __host__ __device__ inline SmemLayout smem_layout(int64_t M, int64_t K, int MP, 
     const int64_t G = K >> 7;
     L.bars = (size_t)kStages * kStageBytes;
     L.flags = L.bars + 2 * kStages * sizeof(uint64_t);
-    L.xs = align_up(L.flags + 16, 16);
-    L.xp = align_up(L.xs + sizeof(float) * MP * G, 16);
+    L.xp = align_up(L.flags + 16, 16);
     // k-permuted activations of the M real rows, then one zero row (4 lanes x 4 words) for padding
     L.total = L.xp + (xsmem ? ((size_t)G * M * 16 + 16) * sizeof(uint4) : 0);
     return L;
@@ -132,13 +133,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr)
     return v;
 }
 
-__device__ __forceinline__ float lds_f32(uint32_t addr)
-{
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-    return v;
-}
-
 template <int NT, bool XSMEM, bool EVEN_G>
 __global__ void __launch_bounds__(kThreads)
 gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tmap, const uint16_t *__restrict__ x, int64_t M,
@@ -157,7 +151,6 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tmap, const uint16_t *
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.flags);
     volatile int *last_flag = abort_flag + 1;
     volatile int *zero_word = abort_flag + 2;  // written once (0) at start, never again
-    float *Xs = reinterpret_cast<float *>(smem + L.xs);
     uint4 *xp = reinterpret_cast<uint4 *>(smem + L.xp);
 
     const int G = (int)(K >> 7);
@@ -179,16 +172,6 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tmap, const uint16_t *
         *last_flag = 0;
         *zero_word = 0;
         fence_mbar_init();
-    }
-    // activation group sums X[m][g]; padded rows m >= M are zero
-    for (int t = tid; t < (MP - (int)M) * G; t += kThreads) Xs[(int)M * G + t] = 0.0f;
-    for (int t = wid; t < (int)M * G; t += kConsumers + 1) {
-        const int m = t / G, gi = t - m * G;
-        const uint2 p = *reinterpret_cast<const uint2 *>(x + (int64_t)m * K + gi * 128 + lane * 4);
-        float v = (__uint_as_float(p.x << 16) + __uint_as_float(p.x & 0xffff0000u)) +
-                  (__uint_as_float(p.y << 16) + __uint_as_float(p.y & 0xffff0000u));
-        v = warp_sum(v);
-        if (lane == 0) Xs[t] = v;
     }
     if (XSMEM) {
         // xp[((ch * M + m) * 4 + c) * 4 + i] = k-permuted pairs of x[m][ch*128 + 32c + 8i .. +8],
@@ -234,8 +217,6 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tmap, const uint16_t *
     const uint32_t opaque_zero = (uint32_t)*zero_word;  // always 0, but opaque to the compiler
     const int r4 = lane >> 2, c = lane & 3;
     const uint32_t stage0 = smem_u32(stage) + (uint32_t)((wid * 16 + r4) * kStageRowBytes + c * 16);
-    const uint32_t xs_a = smem_u32(Xs) + 4u * (uint32_t)(2 * c * G);      // X[2c][.]
-    const uint32_t xs_b = xs_a + 4u * (uint32_t)G;                        // X[2c+1][.]
     // k-permuted activations of this lane's rows m = nt*8 + r4 (the zero row when m >= M)
     uint32_t xp_row[NT], xp_step[NT];
 #pragma unroll
@@ -328,6 +309,7 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tmap, const uint16_t *
                 const float s_b = __uint_as_float(pc ? (szc[1] & 0xffff0000u) : (szc[1] << 16));
                 const float z_a = 128.0f + __uint_as_float(pc ? (szc[2] & 0xffff0000u) : (szc[2] << 16));
                 const float z_b = 128.0f + __uint_as_float(pc ? (szc[3] & 0xffff0000u) : (szc[3] << 16));
+                const uint32_t zz_a = pack_bf16x2(z_a, z_a), zz_b = pack_bf16x2(z_b, z_b);
                 uint32_t P[NT][4][4];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
@@ -358,8 +340,8 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tmap, const uint16_t *
                     uint32_t RA[4], RB[4];
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
-                        RA[t] = nib_pair_bf16(va, 4 * t);
-                        RB[t] = nib_pair_bf16(vb, 4 * t);
+                        RA[t] = sub_bf16x2(nib_pair_bf16(va, 4 * t), zz_a);  // exact q - z
+                        RB[t] = sub_bf16x2(nib_pair_bf16(vb, 4 * t), zz_b);
                     }
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
@@ -370,12 +352,10 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tmap, const uint16_t *
                 }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    const float x0 = lds_f32(xs_a + 4u * (uint32_t)(nt * 8 * G + chc));
-                    const float x1 = lds_f32(xs_b + 4u * (uint32_t)(nt * 8 * G + chc));
-                    acc[0][nt][0] = fmaf(s_a, fmaf(-z_a, x0, C[0][nt][0] + C[1][nt][0]), acc[0][nt][0]);
-                    acc[0][nt][1] = fmaf(s_a, fmaf(-z_a, x1, C[0][nt][1] + C[1][nt][1]), acc[0][nt][1]);
-                    acc[1][nt][0] = fmaf(s_b, fmaf(-z_b, x0, C[0][nt][2] + C[1][nt][2]), acc[1][nt][0]);
-                    acc[1][nt][1] = fmaf(s_b, fmaf(-z_b, x1, C[0][nt][3] + C[1][nt][3]), acc[1][nt][1]);
+                    acc[0][nt][0] = fmaf(s_a, C[0][nt][0] + C[1][nt][0], acc[0][nt][0]);
+                    acc[0][nt][1] = fmaf(s_a, C[0][nt][1] + C[1][nt][1], acc[0][nt][1]);
+                    acc[1][nt][0] = fmaf(s_b, C[0][nt][2] + C[1][nt][2], acc[1][nt][0]);
+                    acc[1][nt][1] = fmaf(s_b, C[0][nt][3] + C[1][nt][3], acc[1][nt][1]);
                 }
             }
             // advance the scale/zero window by one stage, fetching two stages ahead

@@ -265,6 +265,18 @@ def test_gemm_w4a16_m1_workspace_reuse():
     assert not torch.equal(outs[0], outs[1])
 
 
+@pytest.mark.parametrize("M", [1, 2, 5, 8, 16, 17, 40])
+def test_gemm_w4a16_zero_rows_exact(M):
+    """Rows (and groups) whose weights are all zero have w_hat = 0, so the bound is 0: y must be exactly 0,
+    even when the activations of a group span so many binades that their binary32 sums round."""
+    N, K = 640, 2048
+    w = wq_inputs.llm_weight(N, K, 91, dtype=torch.float32)
+    w[::5] = 0.0
+    w[3, 256:384] = 0.0  # one all-zero group inside a non-zero row
+    x = wq_inputs.wide_range_activations(M, K, 92 + M)
+    _w4_case(N, K, 128, M, 0, wgen=w, xgen=x)
+
+
 def test_gemm_w4a16_degenerate_groups():
     w = wq_inputs.llm_weight(64, 512, 81, dtype=torch.float32)
     w[0] = 0.0

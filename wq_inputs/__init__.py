@@ -94,6 +94,14 @@ def activations(M: int, K: int, seed: int, salient_frac: float = 0.01, salient_m
     return x.to(torch.bfloat16)
 
 
+def wide_range_activations(M: int, K: int, seed: int, spread: float = 4.0, device="cpu") -> torch.Tensor:
+    """bf16 [M][K]: N(0, 1) times exp(spread * N(0, 1)), so the values of one group span many binades
+    (their binary32 sums round, which makes exact cancellation a real test)."""
+    g = _gen(seed)
+    x = torch.randn(M, K, generator=g) * torch.exp(torch.randn(M, K, generator=g) * spread)
+    return x.to(torch.bfloat16).to(device)
+
+
 def plain_activations(M: int, K: int, seed: int, device="cpu") -> torch.Tensor:
     """bf16 [M][K] ~ N(0, 1)."""
     g = _gen(seed + 2_000_003, device)
