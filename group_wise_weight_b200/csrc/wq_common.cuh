@@ -132,6 +132,23 @@ __device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c)
     return f32x2{__uint_as_float((uint32_t)r), __uint_as_float((uint32_t)(r >> 32))};
 }
 
+// The same product-sum with the pairs joined and split inside the asm, so the compiler can keep each
+// pair in an aligned register pair (cheaper where the operands come from loads and stay in pairs, as in
+// the tensor-core kernel's promotion).
+__device__ __forceinline__ f32x2 fma2_pairs(f32x2 a, f32x2 b, f32x2 c)
+{
+    f32x2 r;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return r;
+}
+
 __device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b)
 {
     uint64_t r;

@@ -101,6 +101,14 @@ __device__ __forceinline__ uint32_t bf2_sub(uint32_t q128, uint32_t zc)
     return *reinterpret_cast<uint32_t *>(&a);
 }
 
+// t & mask | magic with both constants in registers (kernel arguments): one LOP3 instead of two.
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t t, uint32_t mask, uint32_t magic)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(t), "r"(mask), "r"(magic));
+    return d;
+}
+
 // Slot and phase of a ring of `n` buffers, advanced one use at a time.
 struct Ring {
     uint32_t slot = 0, phase = 0;
@@ -115,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, int64_t M,
                      int64_t N, int64_t K, const uint16_t *__restrict__ sc, const uint16_t *__restrict__ zp,
                      uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ counters, int max_segs,
-                     int *__restrict__ status)
+                     int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic)
 {
     using C = Cfg<BN>;
     constexpr int NG = kStageK / GROUP;     // groups per stage
@@ -294,7 +302,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < kChunk; i += 2) {
-                        const f32x2 r2 = fma2(s2, f32x2{__uint_as_float(v[i]), __uint_as_float(v[i + 1])},
+                        const f32x2 r2 = fma2_pairs(s2, f32x2{__uint_as_float(v[i]), __uint_as_float(v[i + 1])},
                                               f32x2{acc[c0 + i], acc[c0 + i + 1]});
                         acc[c0 + i] = r2.x;
                         acc[c0 + i + 1] = r2.y;
@@ -349,7 +357,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const uint32_t t = __byte_perm(v, v4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
-                            A[i * 16 + w * 4 + j] = bf2_sub((t & 0x000F000Fu) | 0x43004300u, z2);
+                            A[i * 16 + w * 4 + j] = bf2_sub(lop_and_or(t, nib_mask, bf16_magic), z2);
                         }
                     }
                 }
@@ -468,7 +476,8 @@ int run(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, co
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
     float *ws = reinterpret_cast<float *>(w8);
     int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, GROUP));
-    kern<<<(unsigned)grid, kThreads, smem, st>>>(wmap, xmap, M, N, K, s, z, y, ws, counters, max_segs, status);
+    kern<<<(unsigned)grid, kThreads, smem, st>>>(wmap, xmap, M, N, K, s, z, y, ws, counters, max_segs, status,
+                                                  0x000F000Fu, 0x43004300u);
     return 0;
 }
 

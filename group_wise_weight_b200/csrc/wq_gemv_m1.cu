@@ -147,6 +147,20 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t addr)
     return r;
 }
 
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
+{
+    uint32_t r;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
 {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
@@ -319,17 +333,20 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             const int kg = 2 * p;
             const uint32_t szsrc =
                 szr_u32 + (uint32_t)(win & 1) * 2u * kSzBytes + (uint32_t)r0 * 16u + (uint32_t)(kg & 7) * 2u;
+            // s and z of groups kg, kg + 1 are adjacent in the window box (kg is even): one 32-bit load per
+            // row and array; (128 + z) is formed by one bf16 addition (rounded like 128 + z in binary32
+            // then to bf16)
             float sv[2][2];
             uint32_t zz[2][2];  // bf16 pairs (128 + z, 128 + z)
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    const uint32_t o = szsrc + (uint32_t)a * 8u * 16u + (uint32_t)h * 2u;
-                    sv[h][a] = __uint_as_float(lds_u16(o) << 16);
-                    const float zf = 128.0f + __uint_as_float(lds_u16(o + kSzBytes) << 16);
-                    zz[h][a] = pack_bf16x2(zf, zf);
-                }
+            for (int a = 0; a < 2; ++a) {
+                const uint32_t o = szsrc + (uint32_t)a * 8u * 16u;
+                const uint32_t s2 = lds_u32(o), z2 = lds_u32(o + kSzBytes);
+                sv[0][a] = __uint_as_float(s2 << 16);
+                sv[1][a] = __uint_as_float(s2 & 0xffff0000u);
+                zz[0][a] = add_bf16x2(__byte_perm(z2, 0u, 0x1010), 0x43004300u);
+                zz[1][a] = add_bf16x2(__byte_perm(z2, 0u, 0x3232), 0x43004300u);
+            }
             // the stage's weight bytes are in registers: hand the slot back to the producer
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);

@@ -73,6 +73,27 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *p, flo
     }
 }
 
+// Correctly rounded quotients w / s for the codes, without a division per weight.  Markstein's final
+// correction step (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): with r = RN(1/s) and q0 = RN(w * r), the residual
+// e = w - q0 * s is exact (one fused multiply-add), and RN(q0 + e * r) = RN(w / s) provided the reciprocal
+// and the quotient stay in the normal range.  The scales here are bf16 values; for every bf16 significand
+// of s and every binary32 significand of w this identity was checked exhaustively (the check is part of
+// the test suite).  A group whose scale or largest quotient could leave the normal range uses the IEEE
+// division instead; quotients too small to be normal never change a code (t = RN(q + z) rounds to z, or
+// to 0 when z = 0).
+__device__ __forceinline__ bool quotients_by_reciprocal(float s, float maxabs)
+{
+    return s >= 0x1p-100f && s <= 0x1p100f && maxabs <= s * 0x1p100f;
+}
+
+__device__ __forceinline__ float quotient_rn(float w, float s, float r)
+{
+    const float q0 = __fmul_rn(w, r);
+    const float e = __fmaf_rn(-q0, s, w);
+    return __fmaf_rn(e, r, q0);
+}
+
 // s, z of one INT4 group from its min and max (the library contract).
 __device__ __forceinline__ void int4_params(float mn, float mx, float &s, float &z)
 {
@@ -127,10 +148,19 @@ quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
             if (!active[u]) continue;
             float s, z;
             int4_params(mn, mx, s, z);
+            float qd[8];  // RN(w / s)
+            if (quotients_by_reciprocal(s, fmaxf(fabsf(mn), fabsf(mx)))) {
+                const float r = __frcp_rn(s);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) qd[i] = quotient_rn(v[u][i], s, r);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) qd[i] = __fdiv_rn(v[u][i], s);
+            }
             uint32_t packed = 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                float q = rintf(__fadd_rn(__fdiv_rn(v[u][i], s), z));
+                float q = rintf(__fadd_rn(qd[i], z));
                 q = fminf(fmaxf(q, 0.0f), 15.0f);
                 packed |= (uint32_t)q << (4 * i);
             }
@@ -152,10 +182,19 @@ __device__ __forceinline__ float int8_scale(float amax)
 
 __device__ __forceinline__ uint2 int8_encode8(const float v[8], float s)
 {
+    float qd[8];  // RN(w / s); |w / s| <= 127.5, so only the scale's range decides the method
+    if (quotients_by_reciprocal(s, 0.0f)) {
+        const float r = __frcp_rn(s);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qd[i] = quotient_rn(v[i], s, r);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qd[i] = __fdiv_rn(v[i], s);
+    }
     uint32_t lo = 0, hi = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        float q = rintf(__fdiv_rn(v[i], s));
+        float q = rintf(qd[i]);
         q = fminf(fmaxf(q, -127.0f), 127.0f);
         const uint32_t b = (uint32_t)(int)q & 0xffu;
         if (i < 4) lo |= b << (8 * i); else hi |= b << (8 * (i - 4));
