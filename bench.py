@@ -281,20 +281,28 @@ def int8_rows(wq, device, copies=8, reps=5):
             {"us": gms * 1e3, "GB_s": gbytes / (gms * 1e-3) / 1e9, "shape": "K=N=8192 per-channel, M=1"})
 
 
-def per_linear_us(model, xs, ys, reps=3):
-    """Average device time of each linear shape at M = 1 (events around each call)."""
+def per_linear_us(model, xs, ys, reps=5):
+    """Average device time of each linear shape at M = 1: the 80 calls of one shape replayed as a CUDA
+    graph (as in the step), events around the replays."""
     out = {}
     for name, K, N in wq_inputs.FULL70B_LINEARS:
         idx = [i for i, l in enumerate(model.linears) if l[0] == name]
+
+        def calls():
+            for i in idx:
+                _, K_, N_, q, s, z = model.linears[i]
+                model.wq.wq_gemm_w4a16(xs[i], q, s, z, G, y=ys[i], workspace=model.ws)
+
+        g = graph_of(calls)
+        g.replay()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         e0.record()
         for _ in range(reps):
-            for i in idx:
-                _, K_, N_, q, s, z = model.linears[i]
-                model.wq.wq_gemm_w4a16(xs[i], q, s, z, G, y=ys[i], workspace=model.ws)
+            g.replay()
         e1.record()
         e1.synchronize()
+        del g
         us = e0.elapsed_time(e1) * 1e3 / (reps * len(idx))
         out[name] = {"us": round(us, 2), "GB_s": round(linear_bytes(1, N, K) / (us * 1e-6) / 1e9, 1)}
     return out

@@ -292,21 +292,30 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 #pragma unroll
             for (int gi = 0; gi < NG; ++gi) {
                 const f32x2 s2{sprev[gi], sprev[gi]};
+                // two tensor-memory loads in flight per wait
                 constexpr int kChunk = kCols < 16 ? kCols : 16;
+                constexpr int kBatch = kCols >= 2 * kChunk ? 2 : 1;
 #pragma unroll
-                for (int c0 = 0; c0 < kCols; c0 += kChunk) {
-                    uint32_t v[kChunk];
-                    const uint32_t col = dq_addr + pr.slot * (uint32_t)kDCols + (uint32_t)(gi * BN + c0);
-                    if (kChunk == 16) tmem_ld16(col, v);
-                    else tmem_ld8(col, v);
+                for (int c0 = 0; c0 < kCols; c0 += kChunk * kBatch) {
+                    uint32_t v[kBatch][kChunk];
+#pragma unroll
+                    for (int b = 0; b < kBatch; ++b) {
+                        const uint32_t col =
+                            dq_addr + pr.slot * (uint32_t)kDCols + (uint32_t)(gi * BN + c0 + b * kChunk);
+                        if (kChunk == 16) tmem_ld16(col, v[b]);
+                        else tmem_ld8(col, v[b]);
+                    }
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < kChunk; i += 2) {
-                        const f32x2 r2 = fma2_pairs(s2, f32x2{__uint_as_float(v[i]), __uint_as_float(v[i + 1])},
-                                              f32x2{acc[c0 + i], acc[c0 + i + 1]});
-                        acc[c0 + i] = r2.x;
-                        acc[c0 + i + 1] = r2.y;
-                    }
+                    for (int b = 0; b < kBatch; ++b)
+#pragma unroll
+                        for (int i = 0; i < kChunk; i += 2) {
+                            const int cc = c0 + b * kChunk + i;
+                            const f32x2 r2 = fma2_pairs(s2, f32x2{__uint_as_float(v[b][i]), __uint_as_float(v[b][i + 1])},
+                                                        f32x2{acc[cc], acc[cc + 1]});
+                            acc[cc] = r2.x;
+                            acc[cc + 1] = r2.y;
+                        }
                 }
             }
             tc_fence_before();
@@ -324,6 +333,16 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             const int64_t nrow = n < N ? n : N - 1;
             const uint16_t *sp = sc + nrow * G + (int64_t)ks0 * NG;  // scales of the stage's groups
             const uint16_t *zbase = zp + nrow * G;                    // zero-points of the row
+            // a warp's k range of a stage lies in one group when the group is at least that long
+            constexpr bool kOneZ = GROUP >= kKPerWarp;
+            constexpr int kZ = kOneZ ? 1 : kChunksPerWarp;
+            auto zidx = [&](int ks, int i) { return (ks * kStageK + (kq * kChunksPerWarp + i) * 32) / GROUP; };
+            // scales and zero-points are loaded one stage ahead of their use
+            uint16_t snext[NG], znext[kZ];
+#pragma unroll
+            for (int gi = 0; gi < NG; ++gi) snext[gi] = sp[gi];
+#pragma unroll
+            for (int i = 0; i < kZ; ++i) znext[i] = zbase[zidx(ks0, i)];
 #pragma unroll
             for (int c = 0; c < kCols; ++c) acc[c] = 0.0f;
 
@@ -340,16 +359,26 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                                  : "=r"(wv[i].x), "=r"(wv[i].y), "=r"(wv[i].z), "=r"(wv[i].w)
                                  : "r"(w_addr[i] + wr.slot * (uint32_t)kWeightStageBytes));
                 float scur[NG];
+                uint32_t z2s[kZ];
 #pragma unroll
-                for (int gi = 0; gi < NG; ++gi) scur[gi] = bf16_to_f32(sp[gi]);
+                for (int gi = 0; gi < NG; ++gi) scur[gi] = bf16_to_f32(snext[gi]);
+#pragma unroll
+                for (int i = 0; i < kZ; ++i) {
+                    const float zf = 128.0f + bf16_to_f32(znext[i]);
+                    z2s[i] = pack_bf16x2(zf, zf);
+                }
                 sp += NG;
+                if (ks + 1 < ks1) {
+#pragma unroll
+                    for (int gi = 0; gi < NG; ++gi) snext[gi] = sp[gi];
+#pragma unroll
+                    for (int i = 0; i < kZ; ++i) znext[i] = zbase[zidx(ks + 1, i)];
+                }
                 uint32_t A[kKPerWarp / 2];
 #pragma unroll
                 for (int i = 0; i < kChunksPerWarp; ++i) {
                     // zero-point of this 32-k chunk (a chunk never straddles a group: g >= 32)
-                    const int kc = ks * kStageK + (kq * kChunksPerWarp + i) * 32;
-                    const float zf = 128.0f + bf16_to_f32(zbase[kc / GROUP]);
-                    const uint32_t z2 = pack_bf16x2(zf, zf);
+                    const uint32_t z2 = z2s[kOneZ ? 0 : i];
 #pragma unroll
                     for (int w = 0; w < 4; ++w) {
                         const uint32_t v = word_of4(wv[i], w);
@@ -360,9 +389,9 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                             A[i * 16 + w * 4 + j] = bf2_sub(lop_and_or(t, nib_mask, bf16_magic), z2);
                         }
                     }
+                    // each 32-k chunk goes to tensor memory as soon as it is ready
+                    tmem_st16(a_addr + ar.slot * 64u + (uint32_t)(i * 16), A + i * 16);
                 }
-                if (kKPerWarp / 2 == 32) tmem_st32(a_addr + ar.slot * 64u, A);
-                else tmem_st16(a_addr + ar.slot * 64u, A);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
