@@ -49,6 +49,38 @@ METRIC = "W4A16 weight GB/s and % HBM peak at M=1; TFLOP/s and % tensor peak at 
 G = 128
 
 
+M1_PROFILE = os.path.join(ROOT, "profiles", "gemv_w4a16_m1_full70b_layer.txt")
+M1_SOURCES = [os.path.join(ROOT, "group_wise_weight_b200", "csrc", f)
+              for f in ("wq_gemv_m1.cu", "wq_common.cuh", "wq_sm100.cuh")]
+
+
+def kernel_source_hash(paths=None):
+    import hashlib
+    h = hashlib.sha256()
+    for p in (M1_SOURCES if paths is None else paths):
+        h.update(open(p, "rb").read())
+    return h.hexdigest()
+
+
+def m1_traffic_per_launch():
+    """DRAM bytes (read + write) per launch of the M = 1 kernel, averaged over the four linear shapes of
+    one layer, from the committed ncu summary -- or None when the kernel's sources have changed since
+    those counters were taken (the summary records the hash of the sources it profiled)."""
+    if not os.path.exists(M1_PROFILE):
+        return None
+    fields = {}
+    for line in open(M1_PROFILE):
+        if ":" in line and line.split(":", 1)[0].strip() in ("traffic_per_launch_bytes", "kernel_source_sha256"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    if fields.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return int(fields["traffic_per_launch_bytes"])
+    except (KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -480,9 +512,11 @@ def main():
             "a5_w4a16_m128": {"tflops": round(tflops128 / world, 1)},
             "a6_w8a16_m1": {k: (round(v, 2) if isinstance(v, float) else v) for k, v in g8_row.items()},
         },
-        "roofline": {"bound": "hbm", "kernel": "gemv_w4a16 (M=1)", "achieved": round(per_gpu_gbs, 1),
+        "roofline": {"bound": "hbm", "kernel": "gemv_w4a16_m1_kernel", "achieved": round(per_gpu_gbs, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(per_gpu_gbs / peaks["hbm_gbs"], 4),
-                     "peak_source": peaks["source"], "traffic": None,
+                     "peak_source": peaks["source"], "traffic": m1_traffic_per_launch(),
+                     "traffic_source": "profiles/gemv_w4a16_m1_full70b_layer.txt (ncu dram read + write per "
+                                       "launch, mean of one layer's four linears)",
                      "bytes_per_launch_avg": bytes1 // launches_per_step},
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": x_host.numel() * 2,
                 "d2h_bytes_per_step": y_host.numel() * 2, "ms_per_step": round(ms_e2e / args.steps, 4)},

@@ -5,10 +5,10 @@
 // roofline argument ("Quantization Methods Compared: INT8, GPTQ, AWQ, FP8,
 // FP4 and KV-Cache Quantization", section "Hardware, formats and the
 // roofline") puts it near or past the ridge point, so the tensor cores do
-// the work.  The 4-bit weights are dequantised inside the kernel
-// ("... real 4-bit kernels dequantise to fp16 inside the kernel"), with the
-// decode w_hat = s (q - z) of "Quantization for LLM inference: FP8, INT4
-// (GPTQ, AWQ) and GGUF", section "The minimum maths".
+// the work.  The 4-bit weights are dequantised inside the kernel, as that
+// section describes for practical 4-bit kernels, with the decode
+// w_hat = s (q - z) of "Quantization for LLM inference: FP8, INT4 (GPTQ, AWQ)
+// and GGUF", section "The minimum maths".
 //
 // Formulation: D[n][m] = sum_k w_hat[n][k] * x[m][k], a 128 x BN tile per
 // CTA at a time (MMA M = 128 weight rows, N = BN activation rows, K = 16 per
@@ -436,13 +436,20 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 }
                 named_bar_sync(1, kDequantWarps * 32);
                 if (*last_flag) {
+                    // sum the segments in segment order whichever CTA finishes last, so
+                    // repeated calls round identically
                     __threadfence();
+                    float tot[kCols];
+#pragma unroll
+                    for (int c = 0; c < kCols; ++c) tot[c] = 0.0f;
                     for (int64_t o = 0; o <= cta_last - cta_first; ++o) {
-                        if (o == my_seg) continue;
                         const float *other = ws + ((tile * max_segs + o) * BN) * kTileN;
 #pragma unroll
-                        for (int c = 0; c < kCols; ++c) acc[c] += __ldcg(other + (int64_t)(kq * kCols + c) * kTileN + r);
+                        for (int c = 0; c < kCols; ++c)
+                            tot[c] += (o == my_seg) ? acc[c] : __ldcg(other + (int64_t)(kq * kCols + c) * kTileN + r);
                     }
+#pragma unroll
+                    for (int c = 0; c < kCols; ++c) acc[c] = tot[c];
                     if (n < N) {
 #pragma unroll
                         for (int c = 0; c < kCols; ++c)

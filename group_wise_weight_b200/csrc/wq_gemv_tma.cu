@@ -20,9 +20,12 @@
 //    bank conflicts), turns every code pair into bf16 128 + q with one LOP3
 //    and subtracts the pair (128 + z, 128 + z), which leaves the exact
 //    integers q - z, and issues mma.sync m16n8k16 with the weights as the
-//    16-row operand and the activations (pre-permuted to the same k order) as
-//    the 8-column operand; the k permutation is the one described in
-//    wq_gemv.cu.
+//    16-row operand and the activations as the 8-column operand.  A 32-bit
+//    word of codes c_0 .. c_7 yields the bf16 pairs (c_i, c_{i+4}),
+//    i = 0 .. 3, one shift and one LOP3 each, so the k order inside an MMA
+//    step is permuted to put such a pair in each operand register; the
+//    activations are staged in shared memory as the matching pairs
+//    (x_i, x_{i+4}), and a dot product does not depend on the k order.
 //  * Per chunk (= group) the binary32 accumulator takes s * C: (q - z) is
 //    exact, s is applied in binary32, and no term carries an offset that
 //    would have to cancel later (rows of zeros give exactly zero).

@@ -14,8 +14,8 @@
  *       absmax INT8, s = max|w| / 127, q = round(w / s), w_hat = q * s;
  *       one scale per tensor, per output channel or per group of 128 (or 32)
  *       consecutive weights.  Section "Hardware, formats and the roofline":
- *       decode reads every weight once per step and real 4-bit kernels
- *       dequantise inside the matmul.
+ *       a decode step reads all the weights once, and 4-bit weights are
+ *       turned back into 16-bit values inside the matmul kernel.
  *
  * Conventions shared by every call
  *  - Weights are stored one row per output channel: W is [N][K] with K (the
@@ -121,18 +121,27 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
 
 /*
  * W4A16 weight-only matmul with in-kernel dequantisation
- * ([P2] decode w_hat = s * (q - z); [P3] "real 4-bit kernels dequantise ...
- * inside the kernel").
+ * ([P2] decode w_hat = s * (q - z); [P3] "Hardware, formats and the roofline":
+ * the 4-bit weights are expanded inside the matmul kernel).
  *
  *   x       [M][K] bf16 activations
  *   qweight, scales, zeros: as produced by wq_quantize_int4 with group g
  *   y       [M][N] bf16, y[m][n] = sum_k x[m][k] * s[n][k/g] * (q[n][k] - z[n][k/g])
  *
- * Arithmetic: binary32 accumulation, one final rounding to bf16.  M <= 16
- * runs a CUDA-core kernel that keeps (q - z) exact and applies s per group in
- * binary32.  Larger M runs a tcgen05 tensor-core kernel whose operand is
- * w_hat rounded once to bf16.  Either way |y - y_exact| stays within
- * 4e-3 * sum_k |x[m][k] * w_hat[n][k]| on the inputs this library is tested on.
+ * Arithmetic: every kernel forms the exact integers (q - z) in bf16 (a code
+ * pair 128 + q minus the pair 128 + z), multiplies them by x with binary32
+ * accumulation (tensor cores for the decode and batched kernels), applies s
+ * per group in binary32 and rounds y to bf16 once.  No term carries an
+ * offset that cancels later, so rows whose weights are all zero give exactly
+ * zero and |y - y_exact| stays within 4e-3 * sum_k |x[m][k] * w_hat[n][k]|
+ * on the inputs this library is tested on (including activations spanning
+ * ~e^+-20).  Split-K partial sums are combined in a fixed order, so repeated
+ * calls give identical bytes, except for 2 <= M <= 16, whose partials meet in
+ * binary32 atomics (the last bits of y may then vary between calls).
+ * Kernels: M = 1 with g = 128, 1024 <= K <= 32768, K % 1024 == 0: persistent
+ * TMA-fed kernel; 2 <= M <= 16 with g = 128: TMA-fed decode kernel; M > 16
+ * (N >= 128, K % 128 == 0): tcgen05 tensor-core kernel; other shapes: a
+ * CUDA-core kernel.
  * Requirements: M, N >= 1; K % 32 == 0; g in {32, 64, 128}, K % g == 0;
  * pointers 16-byte aligned; workspace of wq_gemm_workspace_bytes(M, N, K, g, 4)
  * bytes (may be NULL when that is 0).  x and y must not overlap.

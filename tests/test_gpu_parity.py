@@ -248,16 +248,17 @@ def test_gemm_w4a16_m1_stream_k_edges(N, K):
     _w4_case(N, K, 128, 1, 11 * N + K)
 
 
-def test_gemm_w4a16_m1_workspace_reuse():
+@pytest.mark.parametrize("M,N,K", [(1, 3000, 4096), (128, 256, 16384), (40, 384, 8192)])
+def test_gemm_w4a16_workspace_reuse_deterministic(M, N, K):
     """Calls that share one workspace find it ready (its counters re-zeroed by the previous call) and the
-    split-K combine runs in a fixed order: the same inputs give the same bytes every time."""
-    N, K = 3000, 4096
+    split-K combine runs in a fixed order: the same inputs give the same bytes every time.  M = 1 runs the
+    persistent decode kernel, M = 40 and 128 the tensor-core kernel with K split over many CTAs per tile."""
     w = wq_inputs.llm_weight(N, K, 77)
     q, s, z = wq.wq_quantize_int4(w.cuda(), 128)
-    ws = torch.zeros(wq.wq_gemm_workspace_bytes(1, N, K, 128, 4) + 16, dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(wq.wq_gemm_workspace_bytes(M, N, K, 128, 4) + 16, dtype=torch.uint8, device="cuda")
     outs = []
     for seed in (1, 2, 1, 2, 1):
-        x = wq_inputs.activations(1, K, seed).cuda()
+        x = wq_inputs.activations(M, K, seed).cuda()
         outs.append(wq.wq_gemm_w4a16(x, q, s, z, 128, workspace=ws).clone())
     torch.cuda.synchronize()
     assert torch.equal(outs[0], outs[2]) and torch.equal(outs[0], outs[4])
