@@ -42,10 +42,12 @@
 //    to cancel later, rows whose weights are all zero give exactly zero, and
 //    the rounding error stays proportional to sum |x w_hat|.
 //  * A tile split between CTAs leaves one binary32 partial per segment in the
-//    workspace; for each warp's 16 rows, the warp that arrives last (one
-//    arrival counter per tile and warp, no CTA barrier) sums the partials in
-//    segment order, writes y and re-zeroes the counter, so results do not
-//    depend on timing.
+//    workspace.  The consumers never wait on global memory for this: each
+//    warp drops its 16 row sums into a double-buffered shared-memory tile and
+//    moves on, and a separate combiner warp copies the tile to the
+//    segment's slot, bumps the tile's arrival counter and, if it is the last
+//    to arrive, sums the slots in segment order, writes y and re-zeroes the
+//    counter -- a fixed order, so results do not depend on timing.
 //  * x is copied into shared memory with one bulk asynchronous copy, then
 //    permuted in place.
 //  * Launched with programmatic dependent launch: in a stream of linears the
@@ -71,7 +73,9 @@ namespace wq {
 namespace {
 
 constexpr int kC = 16;                            // consumer warps
-constexpr int kT = (kC + 1) * 32;                 // threads: consumers, then the producer warp
+constexpr int kProducer = kC;                     // warp roles: consumers 0 .. kC-1, then these two
+constexpr int kCombiner = kC + 1;
+constexpr int kT = (kC + 2) * 32;                 // threads
 constexpr int kTile = 16 * kC;                    // rows per tile (256)
 constexpr int kStages = 3;                        // weight stages in flight
 constexpr uint32_t kStageBytes = kTile * 128;     // 256 rows x 2 groups x 64 B
@@ -79,14 +83,16 @@ constexpr uint32_t kSzBytes = kTile * 16;         // 256 rows x 8 groups x 2 B (
 constexpr uint32_t kBulkPiece = 16384;            // bytes per bulk copy of x
 constexpr int kPairsPerWindow = 4;                // 8 groups of s/z = 4 units
 
-// shared memory: [x pairs 2K][pad to 1024][stages][s/z windows][barriers]
+// shared memory: [x pairs 2K][pad to 1024][stages][s/z windows][2 partial tiles][barriers]
 __host__ __device__ __forceinline__ size_t m1_ring_offset(int64_t K)
 {
     return ((size_t)K * 2 + 1023) & ~(size_t)1023;
 }
 __host__ __device__ __forceinline__ size_t m1_sz_offset(int64_t K) { return m1_ring_offset(K) + kStages * kStageBytes; }
-__host__ __device__ __forceinline__ size_t m1_bar_offset(int64_t K) { return m1_sz_offset(K) + 2 * 2 * kSzBytes; }
-constexpr int kBars = 2 * kStages + 4 + 1 + 2;  // full/empty per stage, s/z full/empty x2, x, flags (2 x 8 B)
+__host__ __device__ __forceinline__ size_t m1_part_offset(int64_t K) { return m1_sz_offset(K) + 2 * 2 * kSzBytes; }
+__host__ __device__ __forceinline__ size_t m1_bar_offset(int64_t K) { return m1_part_offset(K) + 2 * kTile * 4; }
+// full/empty per stage, s/z full/empty x2, partial full/empty x2, x, flags (2 x 8 B)
+constexpr int kBars = 2 * kStages + 4 + 4 + 1 + 2;
 __host__ __device__ __forceinline__ size_t m1_smem_bytes(int64_t K) { return m1_bar_offset(K) + kBars * 8 + 1024; }
 
 // (v >> sh) & mask | magic with both constants in registers: one LOP3.
@@ -140,13 +146,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr)
     return r;
 }
 
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr)
-{
-    uint16_t r;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr));
-    return r;
-}
-
 __device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
 {
     uint32_t r;
@@ -189,7 +188,7 @@ __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity, int *
         if (global_ns() - t0 > kWaitLimitNs) { record_timeout(status); return; }
 }
 
-// 17 warps put five on one SM sub-partition, whose register file holds 16K registers: at most 96 each.
+// 18 warps put five on one SM sub-partition, whose register file holds 16K registers: at most 96 each.
 __global__ void __maxnreg__(96)
 gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                      const __grid_constant__ CUtensorMap zmap, const uint16_t *__restrict__ x, int N, int K,
@@ -202,10 +201,12 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     uint4 *xp = reinterpret_cast<uint4 *>(sm);                    // K / 8 chunks of 8 activations
     uint8_t *ring = sm + m1_ring_offset(K);
     uint8_t *szr = sm + m1_sz_offset(K);                          // [2 windows][s, z][256 rows][8 groups]
+    float *part = reinterpret_cast<float *>(sm + m1_part_offset(K));  // [2][256 rows] partial sums
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + m1_bar_offset(K));
     uint64_t *full = bars, *empty = bars + kStages;
     uint64_t *szfull = bars + 2 * kStages, *szempty = szfull + 2;
-    uint64_t *xbar = szempty + 2;
+    uint64_t *pfull = szempty + 2, *pempty = pfull + 2;
+    uint64_t *xbar = pempty + 2;
     volatile int *flags = reinterpret_cast<volatile int *>(xbar + 1);  // [0] abort, [1] last-arrival broadcast
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int G = K >> 7;
@@ -220,6 +221,8 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         for (int i = 0; i < 2; ++i) {
             mbar_init(&szfull[i], 1);
             mbar_init(&szempty[i], kC);
+            mbar_init(&pfull[i], kC);
+            mbar_init(&pempty[i], 1);
         }
         mbar_init(xbar, 1);
         flags[0] = 0;
@@ -240,7 +243,7 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     // Under programmatic dependent launch the previous kernel may still be running.  Nothing it writes may
     // be read before pdl_wait(), but an L2 prefetch is safe (L2 is where writes land): start pulling the
     // first stages from HBM now.
-    if (wid == kC && lane == 0) {
+    if (wid == kProducer && lane == 0) {
         int t = tile0, p = pair0;
         for (int i = 0; i < kStages && i < n; ++i) {
             tma_prefetch_l2_3d(&wmap, 0, t * kTile, 2 * p);
@@ -249,7 +252,7 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     }
     pdl_wait();
 
-    if (wid == kC) {
+    if (wid == kProducer) {
         // ================================ producer ================================
         if (lane == 0 && n > 0) {
             const uint32_t xbytes = (uint32_t)K * 2u;
@@ -272,6 +275,8 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     ++wins;
                 }
                 const int s = i % kStages;
+                // the first stage goes out alone with x and the first s/z window; the rest once x is in
+                if (i == 1 && !mbar_wait(xbar, 0, status, flags)) break;
                 if (i >= kStages && !mbar_wait(&empty[s], (uint32_t)(i / kStages - 1) & 1u, status, flags)) break;
                 mbar_arrive_expect_tx(&full[s], kStageBytes);
                 tma_load_3d(ring + (uint32_t)s * kStageBytes, &wmap, &full[s], 0, t * kTile, 2 * p);
@@ -281,6 +286,76 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             for (int j = max(0, i - kStages); j < i; ++j) wait_drain(&full[j % kStages], (uint32_t)(j / kStages) & 1u, status);
             for (int j = max(0, wins - 2); j < wins; ++j) wait_drain(&szfull[j & 1], (uint32_t)(j >> 1) & 1u, status);
             wait_drain(xbar, 0, status);
+        }
+        __syncthreads();
+        return;
+    }
+
+    if (wid == kCombiner) {
+        // ================================ combiner ================================
+        // The CTA's range splits a tile wherever it starts or ends inside one; walk those tiles in the
+        // consumers' order.  Lane l handles rows 8l .. 8l + 7 of the tile.
+        int pseg = 0;
+        for (int64_t tt = beg / P; tt * P < end; ++tt) {
+            if (tt * P >= beg && tt * P + P <= end) continue;  // whole tile: the consumers wrote y
+            const int b = pseg & 1;
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&pfull[b], (uint32_t)(pseg >> 1) & 1u, status, flags));
+            if (!ok) break;
+            const float4 v0 = *reinterpret_cast<const float4 *>(part + b * kTile + 8 * lane);
+            const float4 v1 = *reinterpret_cast<const float4 *>(part + b * kTile + 8 * lane + 4);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[b]);  // the shared tile is in registers: free it
+            ++pseg;
+            const int64_t c_first = cta_of(tt * P, units, B);
+            const int nseg = (int)(cta_of(tt * P + P - 1, units, B) - c_first) + 1;
+            float *slots = ws + (size_t)tt * max_segs * kTile;
+            float4 *mine = reinterpret_cast<float4 *>(slots + (bid - c_first) * kTile + 8 * lane);
+            mine[0] = v0;
+            mine[1] = v1;
+            // the release of the add below covers every lane's slot writes (ordered by the warp barrier)
+            __syncwarp();
+            int last = 0;
+            if (lane == 0) last = (atom_add_acq_rel(cnt + tt, 1) + 1 == nseg) ? 1 : 0;
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                // sum the segments' slots in segment order (independent of which CTA arrived last)
+                float v[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+                const float4 *q = reinterpret_cast<const float4 *>(slots + 8 * lane);
+                int o = 0;
+                for (; o + 4 <= nseg; o += 4) {
+                    float4 a[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        a[2 * j] = __ldcg(q + (size_t)(o + j) * (kTile / 4));
+                        a[2 * j + 1] = __ldcg(q + (size_t)(o + j) * (kTile / 4) + 1);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        v[0] += a[2 * j].x; v[1] += a[2 * j].y; v[2] += a[2 * j].z; v[3] += a[2 * j].w;
+                        v[4] += a[2 * j + 1].x; v[5] += a[2 * j + 1].y; v[6] += a[2 * j + 1].z; v[7] += a[2 * j + 1].w;
+                    }
+                }
+                for (; o < nseg; ++o) {
+                    const float4 a0 = __ldcg(q + (size_t)o * (kTile / 4)), a1 = __ldcg(q + (size_t)o * (kTile / 4) + 1);
+                    v[0] += a0.x; v[1] += a0.y; v[2] += a0.z; v[3] += a0.w;
+                    v[4] += a1.x; v[5] += a1.y; v[6] += a1.z; v[7] += a1.w;
+                }
+                const int64_t row = tt * kTile + 8 * lane;
+                if (row + 8 <= N) {
+                    uint4 pk;
+                    pk.x = (uint32_t)f32_to_bf16(v[0]) | ((uint32_t)f32_to_bf16(v[1]) << 16);
+                    pk.y = (uint32_t)f32_to_bf16(v[2]) | ((uint32_t)f32_to_bf16(v[3]) << 16);
+                    pk.z = (uint32_t)f32_to_bf16(v[4]) | ((uint32_t)f32_to_bf16(v[5]) << 16);
+                    pk.w = (uint32_t)f32_to_bf16(v[6]) | ((uint32_t)f32_to_bf16(v[7]) << 16);
+                    *reinterpret_cast<uint4 *>(y + row) = pk;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (row + j < N) y[row + j] = f32_to_bf16(v[j]);
+                }
+                __syncwarp();
+                if (lane == 0) atomicExch(cnt + tt, 0);
+            }
         }
         __syncthreads();
         return;
@@ -309,6 +384,7 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         float acc[2] = {0.0f, 0.0f};
         int t = tile0, p = pair0, seg_first = pair0;
         int win = -1;
+        int pseg = 0;  // partial segments handed to the combiner
         // A wait that runs out sets the abort flag and every later wait returns at once: the loop then runs
         // to its end on garbage, with the same control flow in every warp, so the barriers below still meet.
         for (int i = 0; i < n; ++i) {
@@ -384,41 +460,17 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                         if (row0 + 8 < N) y[row0 + 8] = f32_to_bf16(acc[1]);
                     }
                 } else {
-                    // partial: this warp's 16 rows go to this CTA's slot; the warp that arrives last for those
-                    // rows (one counter per tile and warp) sums the slots in segment order -- even and odd
-                    // segments in two lanes, then added: a fixed order, so the result does not depend on timing
-                    const int64_t c_first = cta_of((int64_t)t * P, units, B);
-                    const int nseg = (int)(cta_of((int64_t)t * P + P - 1, units, B) - c_first) + 1;
-                    float *slots = ws + (size_t)t * max_segs * kTile + 16 * wid;
-                    int *wcnt = cnt + (size_t)t * kC + wid;
+                    // partial: this warp's 16 row sums go to the shared tile of this segment; the combiner
+                    // warp takes it from there (tiles alternate between two buffers)
+                    const int b = pseg & 1;
+                    if (pseg >= 2) mbar_wait(&pempty[b], (uint32_t)((pseg >> 1) - 1) & 1u, status, flags);
                     if (tq == 0) {
-                        slots[(bid - c_first) * kTile + gq] = acc[0];
-                        slots[(bid - c_first) * kTile + gq + 8] = acc[1];
+                        part[b * kTile + r0] = acc[0];
+                        part[b * kTile + r0 + 8] = acc[1];
                     }
                     __syncwarp();
-                    int last = 0;
-                    if (lane == 0) last = (atom_add_acq_rel(wcnt, 1) + 1 == nseg) ? 1 : 0;
-                    last = __shfl_sync(0xffffffffu, last, 0);
-                    __syncwarp();
-                    if (last) {
-                        const int rr = lane & 15;
-                        const float *q = slots + rr;
-                        float v = 0.0f;
-                        int o = lane >> 4;
-                        for (; o + 6 < nseg; o += 8) {
-                            const float a0 = __ldcg(q + (o + 0) * kTile), a1 = __ldcg(q + (o + 2) * kTile);
-                            const float a2 = __ldcg(q + (o + 4) * kTile), a3 = __ldcg(q + (o + 6) * kTile);
-                            v += a0;
-                            v += a1;
-                            v += a2;
-                            v += a3;
-                        }
-                        for (; o < nseg; o += 2) v += __ldcg(q + o * kTile);
-                        v += __shfl_xor_sync(0xffffffffu, v, 16);
-                        const int row = t * kTile + 16 * wid + rr;
-                        if (lane < 16 && row < N) y[row] = f32_to_bf16(v);
-                        if (lane == 0) atomicExch(wcnt, 0);
-                    }
+                    if (lane == 0) mbar_arrive(&pfull[b]);
+                    ++pseg;
                 }
                 acc[0] = acc[1] = 0.0f;
             }
@@ -481,7 +533,7 @@ size_t gemv_m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
 {
     if (!gemv_m1_eligible(M, N, K, g)) return 0;
     const int64_t ntiles = (N + kTile - 1) / kTile;
-    return m1_slots_bytes(N, K, m1_grid(N, K)) + ((size_t)ntiles * kC * 4 + 255) / 256 * 256;
+    return m1_slots_bytes(N, K, m1_grid(N, K)) + ((size_t)ntiles * 4 + 255) / 256 * 256;
 }
 
 int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
