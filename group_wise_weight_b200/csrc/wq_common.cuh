@@ -83,6 +83,44 @@ __device__ __forceinline__ uint32_t sub_bf16x2(uint32_t a, uint32_t b)
     return d;
 }
 
+// Zero-points outside [0, 15].  z = round(-min / s) is not clamped, so a group that lies on one side of
+// zero, far from it compared with its width, has |z| up to thousands, and neither 128 + z nor q - z need
+// fit bf16's 8 significant bits.  The kernels then split z = z_hi + z_lo with z_lo in [0, 16) and z_hi a
+// multiple of 16: (128 + q) - (128 + z_lo) = q - z_lo is exact, and -z_hi times the group's activation sum
+// is added in binary32 (whose rounding is tiny next to s |q - z| sum |x|, since |q - z| >= |z_hi| - 15).
+// Returns z_lo; z is an integer.
+__device__ __forceinline__ float zp_split(float z, float &z_hi)
+{
+    z_hi = floorf(z * 0.0625f) * 16.0f;
+    return z - z_hi;
+}
+
+// bf16 pair (128 + v, 128 + v) for an integer v in [0, 16): exact.
+__device__ __forceinline__ uint32_t bf16_pair_128_plus(float v)
+{
+    return (__float_as_uint(128.0f + v) >> 16) * 0x10001u;
+}
+
+// Both halves of a bf16 pair (128 + z0, 128 + z1), formed by one bf16 addition, hold 128 .. 143,
+// i.e. z0 and z1 are integers in [0, 15] and the pair is exact.
+__device__ __forceinline__ bool zz_pair_in_range(uint32_t zz)
+{
+    return ((zz ^ 0x43004300u) & 0xFFF0FFF0u) == 0u;
+}
+
+// Sum of the 8 bf16 values of a uint4, in binary32, in a fixed order.
+__device__ __forceinline__ float sum_bf16x8(const uint4 &v)
+{
+    float t = __uint_as_float(v.x << 16) + __uint_as_float(v.x & 0xffff0000u);
+    t += __uint_as_float(v.y << 16);
+    t += __uint_as_float(v.y & 0xffff0000u);
+    t += __uint_as_float(v.z << 16);
+    t += __uint_as_float(v.z & 0xffff0000u);
+    t += __uint_as_float(v.w << 16);
+    t += __uint_as_float(v.w & 0xffff0000u);
+    return t;
+}
+
 // ---------------------------------------------------------------------------
 // Mixed-precision FMA: d = a * b + c with bf16 a, b and binary32 c, d
 // (the product of two bf16 is exact in binary32; one rounding).

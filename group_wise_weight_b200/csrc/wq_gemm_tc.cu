@@ -33,7 +33,10 @@
 // own accumulator region in tensor memory, and the dequant warps, one stage
 // behind the MMAs, add s * D_group into binary32 registers ("promotion"):
 // (q - z) is never rounded and s is applied in binary32, as in the decode
-// kernels.  Tensor memory: A 2 x 64 columns, D 2 stages x (128/g) groups x BN
+// kernels.  A zero-point outside [0, 15] is split (zp_split in wq_common.cuh):
+// the operand becomes q - z_lo, the dequant warp marks the stage, the MMA
+// warp sums that stage's activations per group into shared memory, and the
+// promotion adds -s z_hi times those sums.  Tensor memory: A 2 x 64 columns, D 2 stages x (128/g) groups x BN
 // columns (BN = 128 for g = 128, 64 for g = 64, 32 for g = 32).
 //
 // Scheduling: stream-K over (tile, stage) units so every SM gets the same
@@ -74,7 +77,9 @@ struct Cfg {
     static constexpr size_t kBarOff = kWOff + (size_t)kWStages * kWeightStageBytes;
     // x_full[XS], x_empty[XS], w_full[WS], w_empty[WS], a_full[A], a_empty[A], d_full[2], d_empty[2], done
     static constexpr size_t kFlagOff = kBarOff + (2 * kXStages + 2 * kWStages + 2 * kABufs + 4 + 1) * 8;
-    static constexpr size_t kBytes = kFlagOff + 64;
+    // flags: abort, last-arrival, tensor-memory address, far-zero-point marks; then activation sums
+    static constexpr size_t kXsumOff = kFlagOff + 64;
+    static constexpr size_t kBytes = kXsumOff + 2 * 128 * 4;  // [2 D buffers][groups][BN], groups x BN <= 128
 };
 
 struct Sched {
@@ -92,7 +97,7 @@ __device__ __forceinline__ uint32_t word_of4(const uint4 &v, int i)
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// (128 + q) - (128 + z) in bf16: exact for the integers involved (|q - z| <= 256).
+// (128 + q) - (128 + z) in bf16: exact for the integers involved (z in [0, 15], or z_lo of a split).
 __device__ __forceinline__ uint32_t bf2_sub(uint32_t q128, uint32_t zc)
 {
     __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&q128);
@@ -144,6 +149,12 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kFlagOff);
     volatile int *last_flag = abort_flag + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kFlagOff + 16);
+    // wide_mark[A buffer] = stage counter + 1 when a dequant warp split a zero-point of that stage;
+    // xs_wide[D buffer] = 1 when the MMA warp wrote the stage's activation sums to xsum
+    volatile int *wide_mark = reinterpret_cast<volatile int *>(smem + C::kFlagOff + 32);
+    volatile int *xs_wide = wide_mark + kABufs;
+    float *xsum = reinterpret_cast<float *>(smem + C::kXsumOff);
+    static_assert(NG * BN <= 128, "activation-sum buffer");
 
     const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
     Sched S;
@@ -171,9 +182,10 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&d_full[i], 1);
+            mbar_init(&d_full[i], 2);  // the MMAs' completion, and the MMA warp's activation sums
             mbar_init(&d_empty[i], kDequantWarps);
         }
+        for (uint32_t i = 0; i < kABufs; ++i) wide_mark[i] = 0;
         mbar_init(done, 1);
         *abort_flag = 0;
         *last_flag = 0;
@@ -224,22 +236,25 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         }
     } else if (wid == 1) {
         // ------------------------------ MMA issuer ------------------------------
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
-            constexpr int kStepsPerGroup = GROUP / 16;
-            Ring xr, ar, dr;  // activation ring, A buffers, D double buffers
-            uint32_t it = 0;
-            const uint32_t xbase = smem_u32(smem);
-            for (int64_t u = beg; u < end;) {
-                const int64_t tile = u / spt;
-                const int ks0 = (int)(u - tile * spt);
-                const int ks1 = (int)std::min<int64_t>(spt, ks0 + (end - u));
-                for (int ks = ks0; ks < ks1; ++ks, ++it) {
-                    mbar_wait_fast(&x_full[xr.slot], xr.phase, status, abort_flag);
-                    mbar_wait_fast(&a_full[ar.slot], ar.phase, status, abort_flag);
-                    if (it >= 2) mbar_wait_fast(&d_empty[dr.slot], dr.phase ^ 1u, status, abort_flag);
-                    tc_fence_after();
-                    const uint32_t xs = xbase + xr.slot * (uint32_t)C::kXStageBytes;
+        // Lane 0 issues the MMAs.  For a stage whose weights have a zero-point outside [0, 15] (marked by
+        // the dequant warps) the whole warp also sums the stage's activations per group, before the
+        // activation slot is released, for the dequant warps' correction -z_hi * sum x.
+        constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+        constexpr int kStepsPerGroup = GROUP / 16;
+        Ring xr, ar, dr;  // activation ring, A buffers, D double buffers
+        uint32_t it = 0;
+        const uint32_t xbase = smem_u32(smem);
+        for (int64_t u = beg; u < end;) {
+            const int64_t tile = u / spt;
+            const int ks0 = (int)(u - tile * spt);
+            const int ks1 = (int)std::min<int64_t>(spt, ks0 + (end - u));
+            for (int ks = ks0; ks < ks1; ++ks, ++it) {
+                mbar_wait_fast(&x_full[xr.slot], xr.phase, status, abort_flag);
+                mbar_wait_fast(&a_full[ar.slot], ar.phase, status, abort_flag);
+                if (it >= 2) mbar_wait_fast(&d_empty[dr.slot], dr.phase ^ 1u, status, abort_flag);
+                tc_fence_after();
+                const uint32_t xs = xbase + xr.slot * (uint32_t)C::kXStageBytes;
+                if (lane == 0) {
                     const uint32_t a_col = tmem + ar.slot * 64u;
                     const uint32_t d_col = d_tmem + dr.slot * (uint32_t)kDCols;
 #pragma unroll
@@ -248,15 +263,44 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                         tc_mma_ts(d_col + (uint32_t)((j / kStepsPerGroup) * BN), a_col + (uint32_t)j * 8u,
                                   smem_desc(baddr, 16, 1024, 2), idesc, (j % kStepsPerGroup) != 0 ? 1u : 0u);
                     }
+                }
+                const bool wide = wide_mark[ar.slot] == (int)(it + 1);
+                if (wide) {
+                    // rows m = lane, lane + 32, ...: two 128-byte-swizzled atoms of 64 k each
+                    for (int m = lane; m < BN; m += 32) {
+                        float xg[NG];
+#pragma unroll
+                        for (int gi = 0; gi < NG; ++gi) xg[gi] = 0.0f;
+#pragma unroll
+                        for (int a = 0; a < 2; ++a)
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                uint4 v;
+                                const uint32_t addr = xs + (uint32_t)a * C::kXAtomBytes + (uint32_t)m * 128u +
+                                                      (((uint32_t)c ^ ((uint32_t)m & 7u)) << 4);
+                                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+                                xg[(a * 64 + c * 8) / GROUP] += sum_bf16x8(v);
+                            }
+#pragma unroll
+                        for (int gi = 0; gi < NG; ++gi) xsum[(dr.slot * NG + gi) * BN + m] = xg[gi];
+                    }
+                }
+                if (lane == 0) xs_wide[dr.slot] = wide ? 1 : 0;
+                __syncwarp();
+                if (lane == 0) {
                     tc_commit(&x_empty[xr.slot]);
                     tc_commit(&a_empty[ar.slot]);
                     tc_commit(&d_full[dr.slot]);
-                    xr.next(XS);
-                    ar.next(kABufs);
-                    dr.next(2);
+                    mbar_arrive(&d_full[dr.slot]);
                 }
-                u += ks1 - ks0;
+                xr.next(XS);
+                ar.next(kABufs);
+                dr.next(2);
             }
+            u += ks1 - ks0;
+        }
+        if (lane == 0) {
             tc_commit(done);
             // every MMA must have completed before tensor memory is released
             const uint64_t t0 = global_ns();
@@ -284,11 +328,15 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         uint32_t it = 0;
         float acc[kCols];
         float sprev[NG];
+        const uint16_t *zrow = zp;  // zero-points of this thread's row in the current tile
 
-        // add s * D of the oldest unpromoted stage to acc, then hand its buffer back to the MMA warp
-        auto promote = [&]() {
+        // add s * D of the oldest unpromoted stage (stage ksp of the tile) to acc, then hand its buffer
+        // back to the MMA warp.  If the stage had a zero-point outside [0, 15], the dequant warps wrote
+        // q - z_lo (zp_split) and the MMA warp the activation sums: acc also takes -s * z_hi * sum x.
+        auto promote = [&](int ksp) {
             mbar_wait_fast(&d_full[pr.slot], pr.phase, status, abort_flag);
             tc_fence_after();
+            const bool wide = xs_wide[pr.slot] != 0;
 #pragma unroll
             for (int gi = 0; gi < NG; ++gi) {
                 const f32x2 s2{sprev[gi], sprev[gi]};
@@ -317,6 +365,16 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                             acc[cc + 1] = r2.y;
                         }
                 }
+                if (wide) {
+                    float zh;
+                    zp_split(bf16_to_f32(zrow[ksp * NG + gi]), zh);
+                    if (zh != 0.0f) {
+                        const float t = -sprev[gi] * zh;
+                        const float *xg = xsum + (pr.slot * NG + gi) * BN + kq * kCols;
+#pragma unroll
+                        for (int cc = 0; cc < kCols; ++cc) acc[cc] = fmaf(t, xg[cc], acc[cc]);
+                    }
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -333,6 +391,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             const int64_t nrow = n < N ? n : N - 1;
             const uint16_t *sp = sc + nrow * G + (int64_t)ks0 * NG;  // scales of the stage's groups
             const uint16_t *zbase = zp + nrow * G;                    // zero-points of the row
+            zrow = zbase;
             // a warp's k range of a stage lies in one group when the group is at least that long
             constexpr bool kOneZ = GROUP >= kKPerWarp;
             constexpr int kZ = kOneZ ? 1 : kChunksPerWarp;
@@ -360,12 +419,19 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                                  : "r"(w_addr[i] + wr.slot * (uint32_t)kWeightStageBytes));
                 float scur[NG];
                 uint32_t z2s[kZ];
+                bool wide = false;  // a zero-point outside [0, 15]: split by zp_split
 #pragma unroll
                 for (int gi = 0; gi < NG; ++gi) scur[gi] = bf16_to_f32(snext[gi]);
 #pragma unroll
                 for (int i = 0; i < kZ; ++i) {
-                    const float zf = 128.0f + bf16_to_f32(znext[i]);
-                    z2s[i] = pack_bf16x2(zf, zf);
+                    float zl = bf16_to_f32(znext[i]);
+                    if (!(zl >= 0.0f && zl <= 15.0f)) {
+                        float zh;
+                        zl = zp_split(zl, zh);
+                        wide = true;
+                    }
+                    const float zc = 128.0f + zl;  // 128 .. 143: exact in bf16
+                    z2s[i] = pack_bf16x2(zc, zc);
                 }
                 sp += NG;
                 if (ks + 1 < ks1) {
@@ -394,6 +460,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 }
                 tmem_wait_st();
                 tc_fence_before();
+                if (wide) wide_mark[ar.slot] = (int)it + 1;  // rare: tell the MMA warp to sum the activations
                 __syncwarp();
                 // tcgen05.st consumed the registers computed from the loaded codes, so no read of the
                 // weight slot can still be pending: hand both the slot and the A buffer over
@@ -404,11 +471,11 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 wr.next(kWStages);
                 ar.next(kABufs);
                 // promote the previous stage of this segment while this one is multiplied
-                if (ks > ks0) promote();
+                if (ks > ks0) promote(ks - 1);
 #pragma unroll
                 for (int gi = 0; gi < NG; ++gi) sprev[gi] = scur[gi];
             }
-            promote();  // the segment's last stage
+            promote(ks1 - 1);  // the segment's last stage
 
             // ---- segment output ----
             const int64_t mbase = mt * BN + kq * kCols;

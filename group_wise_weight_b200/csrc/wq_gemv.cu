@@ -25,7 +25,9 @@
 // in binary32.  No term carries an offset that would have to cancel later,
 // so rows of zeros give exactly zero and the rounding error stays
 // proportional to sum |x w_hat|; the only rounding beyond binary32
-// accumulation is the final bf16 store of y.
+// accumulation is the final bf16 store of y.  A zero-point outside [0, 15]
+// is split (zp_split in wq_common.cuh): the products use q - z_lo and the
+// slice adds -z_hi times its activation sum.
 //
 // INT8 arithmetic.  A slice is 16 codes.  Each code byte is flipped to
 // q + 128, placed under the exponent of 2^23 by a byte permute and shifted
@@ -108,15 +110,24 @@ gemv_w4a16_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t N, int64_t 
     for (; live && j < slices; j += step) {
         if (!PF) fetch(j);
         uint4 cw[R];
-        float s[R];
-        uint32_t zz[R];  // bf16 pairs (128 + z, 128 + z)
+        float s[R], zh[R];
+        uint32_t zz[R];  // bf16 pairs (128 + z, 128 + z), z split by zp_split when outside [0, 15]
+        bool wide = false;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             cw[r] = wq[r];
             s[r] = bf16_to_f32(sb[r]);
-            const float zc = 128.0f + bf16_to_f32(zb[r]);
-            zz[r] = pack_bf16x2(zc, zc);
+            float zl = bf16_to_f32(zb[r]);
+            zh[r] = 0.0f;
+            if (!(zl >= 0.0f && zl <= 15.0f)) {
+                zl = zp_split(zl, zh[r]);
+                wide = true;
+            }
+            zz[r] = bf16_pair_128_plus(zl);
         }
+        float xs[MT];  // activation sums of the slice, needed when a zero-point was split
+#pragma unroll
+        for (int m = 0; m < MT; ++m) xs[m] = 0.0f;
         if (PF && j + step < slices) fetch(j + step);
         const int64_t k0 = j << 5;
         float part[R][MT];
@@ -131,6 +142,7 @@ gemv_w4a16_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t N, int64_t 
             for (int m = 0; m < MT; ++m) {
                 const uint4 xv = ld_nc_v4(xr[m] + k0 + 8 * wd);
                 pair_activations(xv, xp[m]);
+                if (wide) xs[m] += sum_bf16x8(xv);
             }
 #pragma unroll
             for (int r = 0; r < R; ++r) {
@@ -143,6 +155,12 @@ gemv_w4a16_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t N, int64_t 
 #pragma unroll
                     for (int i = 0; i < 4; ++i) part[r][m] = fma_bf16x2(b[i], xp[m][i], part[r][m]);
             }
+        }
+        if (wide) {
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int m = 0; m < MT; ++m) part[r][m] = fmaf(-zh[r], xs[m], part[r][m]);
         }
 #pragma unroll
         for (int r = 0; r < R; ++r)

@@ -40,7 +40,9 @@
 //    the exact integers q - z, so the tensor core sums x (q - z) per group and
 //    the binary32 accumulator takes s * D: no term carries an offset that has
 //    to cancel later, rows whose weights are all zero give exactly zero, and
-//    the rounding error stays proportional to sum |x w_hat|.
+//    the rounding error stays proportional to sum |x w_hat|.  A zero-point
+//    outside [0, 15] is split (zp_split in wq_common.cuh): the operand is
+//    q - z_lo and the lane adds -s z_hi times the group's activation sum.
 //  * A tile split between CTAs leaves one binary32 partial per segment in the
 //    workspace.  The consumers never wait on global memory for this: each
 //    warp drops its 16 row sums into a double-buffered shared-memory tile and
@@ -255,10 +257,24 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     if (wid == kProducer) {
         // ================================ producer ================================
         if (lane == 0 && n > 0) {
+            // the part of x this CTA's units read (512 bytes per group pair): its pairs of the first tile,
+            // and those of the next tile if the range wraps; all of x once the range spans a whole tile
             const uint32_t xbytes = (uint32_t)K * 2u;
-            mbar_arrive_expect_tx(xbar, xbytes);
-            for (uint32_t o = 0; o < xbytes; o += kBulkPiece)
-                bulk_g2s(sm + o, reinterpret_cast<const uint8_t *>(x) + o, min(kBulkPiece, xbytes - o), xbar);
+            uint32_t r0 = 0, r1 = xbytes, w1 = 0;  // [r0, r1) and, when wrapping, [0, w1)
+            if (n < P) {
+                r0 = (uint32_t)pair0 * 512u;
+                if (pair0 + n <= P) {
+                    r1 = (uint32_t)(pair0 + n) * 512u;
+                } else {
+                    w1 = (uint32_t)(pair0 + n - P) * 512u;
+                    if (w1 >= r0) { r0 = 0; w1 = 0; }  // the two pieces meet: all of x
+                }
+            }
+            mbar_arrive_expect_tx(xbar, (r1 - r0) + w1);
+            for (uint32_t o = r0; o < r1; o += kBulkPiece)
+                bulk_g2s(sm + o, reinterpret_cast<const uint8_t *>(x) + o, min(kBulkPiece, r1 - o), xbar);
+            for (uint32_t o = 0; o < w1; o += kBulkPiece)
+                bulk_g2s(sm + o, reinterpret_cast<const uint8_t *>(x) + o, min(kBulkPiece, w1 - o), xbar);
             int t = tile0, p = pair0;
             int wins = 0;  // s/z windows issued
             int i = 0;
@@ -363,7 +379,8 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 
     // ================================ consumers ================================
     if (n > 0) {
-        // ---- x: wait for the bulk copy, permute each chunk in place ----
+        // ---- x: wait for the bulk copy, permute each chunk in place (chunks that were not copied hold
+        // stale bytes and are never read) ----
         mbar_wait(xbar, 0, status, flags);
         for (int c = tid; c < K / 8; c += kC * 32) {
             {
@@ -385,6 +402,11 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         int t = tile0, p = pair0, seg_first = pair0;
         int win = -1;
         int pseg = 0;  // partial segments handed to the combiner
+        int s = 0;     // stage slot of unit i, and the parity of its fill
+        uint32_t ph = 0, w_off = 0;
+        const uint32_t w_lane = ring_u32 + (uint32_t)r0 * 64u + (uint32_t)tq * 16u;
+        const uint32_t sz_lane = szr_u32 + (uint32_t)r0 * 16u;
+        const uint32_t x_lane = xp_u32 + (uint32_t)tq * 64u;
         // A wait that runs out sets the abort flag and every later wait returns at once: the loop then runs
         // to its end on garbage, with the same control flow in every warp, so the barriers below still meet.
         for (int i = 0; i < n; ++i) {
@@ -397,40 +419,57 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 ++win;
                 mbar_wait(&szfull[win & 1], (uint32_t)(win >> 1) & 1u, status, flags);
             }
-            const int s = i % kStages;
-            mbar_wait(&full[s], (uint32_t)(i / kStages) & 1u, status, flags);
+            mbar_wait(&full[s], ph, status, flags);
             // ---- loads from the stage: rows r0, r0 + 8 of both groups; their s, z ----
-            const uint32_t wsrc = ring_u32 + (uint32_t)s * kStageBytes + (uint32_t)r0 * 64u + (uint32_t)tq * 16u;
+            const uint32_t wsrc = w_lane + w_off;
             uint4 wv[2][2];  // [group h][row r0, row r0 + 8]
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int a = 0; a < 2; ++a) wv[h][a] = lds128(wsrc + (uint32_t)h * (kTile * 64u) + (uint32_t)a * 8u * 64u);
             const int kg = 2 * p;
-            const uint32_t szsrc =
-                szr_u32 + (uint32_t)(win & 1) * 2u * kSzBytes + (uint32_t)r0 * 16u + (uint32_t)(kg & 7) * 2u;
+            const uint32_t szsrc = sz_lane + (uint32_t)(win & 1) * 2u * kSzBytes + (uint32_t)(kg & 7) * 2u;
             // s and z of groups kg, kg + 1 are adjacent in the window box (kg is even): one 32-bit load per
-            // row and array; (128 + z) is formed by one bf16 addition (rounded like 128 + z in binary32
-            // then to bf16)
+            // row and array; (128 + z) is formed by one bf16 addition, exact when z is in [0, 15]
             float sv[2][2];
             uint32_t zz[2][2];  // bf16 pairs (128 + z, 128 + z)
+            uint32_t zraw[2], zin = 0u;  // zin & 0xFFF0FFF0: some z of this lane outside [0, 15]
 #pragma unroll
             for (int a = 0; a < 2; ++a) {
                 const uint32_t o = szsrc + (uint32_t)a * 8u * 16u;
-                const uint32_t s2 = lds_u32(o), z2 = lds_u32(o + kSzBytes);
+                zraw[a] = lds_u32(o + kSzBytes);
+                const uint32_t s2 = lds_u32(o), z2 = add_bf16x2(zraw[a], 0x43004300u);
                 sv[0][a] = __uint_as_float(s2 << 16);
                 sv[1][a] = __uint_as_float(s2 & 0xffff0000u);
-                zz[0][a] = add_bf16x2(__byte_perm(z2, 0u, 0x1010), 0x43004300u);
-                zz[1][a] = add_bf16x2(__byte_perm(z2, 0u, 0x3232), 0x43004300u);
+                zz[0][a] = __byte_perm(z2, 0u, 0x1010);
+                zz[1][a] = __byte_perm(z2, 0u, 0x3232);
+                zin |= z2 ^ 0x43004300u;
+            }
+            // a zero-point of this lane outside [0, 15] (rare): split it (zp_split) and add -s z_hi times the
+            // group's activation sum (all 128 values, in a fixed order) to the row sums right away
+            if ((zin & 0xFFF0FFF0u) != 0u) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float xs = 0.0f;
+                    for (int j = 0; j < 16; ++j) xs += sum_bf16x8(lds128(xp_u32 + (uint32_t)(kg + h) * 256u + (uint32_t)j * 16u));
+#pragma unroll
+                    for (int a = 0; a < 2; ++a) {
+                        const float zf = __uint_as_float(h ? (zraw[a] & 0xffff0000u) : (zraw[a] << 16));
+                        float zh;
+                        zz[h][a] = bf16_pair_128_plus(zp_split(zf, zh));
+                        acc[a] = fmaf(-sv[h][a] * zh, xs, acc[a]);
+                    }
+                }
             }
             // the stage's weight bytes are in registers: hand the slot back to the producer
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
+            if (++s == kStages) { s = 0; ph ^= 1u; w_off = 0; } else { w_off += kStageBytes; }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint4 Pw[4];
 #pragma unroll
-                for (int w = 0; w < 4; ++w) Pw[w] = lds128(xp_u32 + (uint32_t)((kg + h) * 16 + tq * 4 + w) * 16u);
+                for (int w = 0; w < 4; ++w) Pw[w] = lds128(x_lane + (uint32_t)(kg + h) * 256u + (uint32_t)w * 16u);
                 float C0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, C1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {

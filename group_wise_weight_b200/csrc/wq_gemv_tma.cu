@@ -28,7 +28,10 @@
 //    (x_i, x_{i+4}), and a dot product does not depend on the k order.
 //  * Per chunk (= group) the binary32 accumulator takes s * C: (q - z) is
 //    exact, s is applied in binary32, and no term carries an offset that
-//    would have to cancel later (rows of zeros give exactly zero).
+//    would have to cancel later (rows of zeros give exactly zero).  A warp
+//    that meets a zero-point outside [0, 15] splits it (zp_split in
+//    wq_common.cuh) and adds -z_hi times the group's activation sums, which
+//    the lanes form from the activation operand they already hold.
 //  * A tile split between CTAs is combined in a binary32 workspace with
 //    atomics; the CTA whose contribution completes the tile's K range
 //    converts it to bf16, re-zeroes the workspace and resets the tile's
@@ -310,9 +313,16 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tmap, const uint16_t *
                 // bf16 of chunk ch + pc: low half for pc = 0, high half for pc = 1
                 const float s_a = __uint_as_float(pc ? (szc[0] & 0xffff0000u) : (szc[0] << 16));
                 const float s_b = __uint_as_float(pc ? (szc[1] & 0xffff0000u) : (szc[1] << 16));
-                const float z_a = 128.0f + __uint_as_float(pc ? (szc[2] & 0xffff0000u) : (szc[2] << 16));
-                const float z_b = 128.0f + __uint_as_float(pc ? (szc[3] & 0xffff0000u) : (szc[3] << 16));
-                const uint32_t zz_a = pack_bf16x2(z_a, z_a), zz_b = pack_bf16x2(z_b, z_b);
+                float zl_a = __uint_as_float(pc ? (szc[2] & 0xffff0000u) : (szc[2] << 16));
+                float zl_b = __uint_as_float(pc ? (szc[3] & 0xffff0000u) : (szc[3] << 16));
+                // a zero-point outside [0, 15] anywhere in the warp: split it (zp_split) for this group
+                const bool wide = __any_sync(0xffffffffu, !(zl_a >= 0.0f && zl_a <= 15.0f && zl_b >= 0.0f && zl_b <= 15.0f));
+                float zh_a = 0.0f, zh_b = 0.0f;
+                if (wide) {
+                    zl_a = zp_split(zl_a, zh_a);
+                    zl_b = zp_split(zl_b, zh_b);
+                }
+                const uint32_t zz_a = bf16_pair_128_plus(zl_a), zz_b = bf16_pair_128_plus(zl_b);
                 uint32_t P[NT][4][4];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
@@ -355,10 +365,27 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tmap, const uint16_t *
                 }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    acc[0][nt][0] = fmaf(s_a, C[0][nt][0] + C[1][nt][0], acc[0][nt][0]);
-                    acc[0][nt][1] = fmaf(s_a, C[0][nt][1] + C[1][nt][1], acc[0][nt][1]);
-                    acc[1][nt][0] = fmaf(s_b, C[0][nt][2] + C[1][nt][2], acc[1][nt][0]);
-                    acc[1][nt][1] = fmaf(s_b, C[0][nt][3] + C[1][nt][3], acc[1][nt][1]);
+                    float d[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) d[e] = C[0][nt][e] + C[1][nt][e];
+                    if (wide) {
+                        // activation sums of this group: lane (r4, c) holds 32 values of row nt*8 + r4, the
+                        // four lanes of a quad the whole group; D's columns 2c, 2c + 1 need rows 2c, 2c + 1
+                        float xs = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) xs += sum_bf16x8(make_uint4(P[nt][i][0], P[nt][i][1], P[nt][i][2], P[nt][i][3]));
+                        xs += __shfl_xor_sync(0xffffffffu, xs, 1);
+                        xs += __shfl_xor_sync(0xffffffffu, xs, 2);
+                        const float x0 = __shfl_sync(0xffffffffu, xs, 8 * c), x1 = __shfl_sync(0xffffffffu, xs, 8 * c + 4);
+                        d[0] = fmaf(-zh_a, x0, d[0]);
+                        d[1] = fmaf(-zh_a, x1, d[1]);
+                        d[2] = fmaf(-zh_b, x0, d[2]);
+                        d[3] = fmaf(-zh_b, x1, d[3]);
+                    }
+                    acc[0][nt][0] = fmaf(s_a, d[0], acc[0][nt][0]);
+                    acc[0][nt][1] = fmaf(s_a, d[1], acc[0][nt][1]);
+                    acc[1][nt][0] = fmaf(s_b, d[2], acc[1][nt][0]);
+                    acc[1][nt][1] = fmaf(s_b, d[3], acc[1][nt][1]);
                 }
             }
             // advance the scale/zero window by one stage, fetching two stages ahead

@@ -131,7 +131,11 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * Arithmetic: every kernel forms the exact integers (q - z) in bf16 (a code
  * pair 128 + q minus the pair 128 + z), multiplies them by x with binary32
  * accumulation (tensor cores for the decode and batched kernels), applies s
- * per group in binary32 and rounds y to bf16 once.  No term carries an
+ * per group in binary32 and rounds y to bf16 once.  A zero-point outside
+ * [0, 15] (a group on one side of zero, far from it) is split as
+ * z = z_hi + z_lo with z_lo in [0, 16) and z_hi a multiple of 16: the
+ * operand is the exact q - z_lo and -z_hi times the group's activation sum
+ * is added in binary32.  No term carries an
  * offset that cancels later, so rows whose weights are all zero give exactly
  * zero and |y - y_exact| stays within 4e-3 * sum_k |x[m][k] * w_hat[n][k]|
  * on the inputs this library is tested on (including activations spanning

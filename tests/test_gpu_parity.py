@@ -278,6 +278,28 @@ def test_gemm_w4a16_zero_rows_exact(M):
     _w4_case(N, K, 128, M, 0, wgen=w, xgen=x)
 
 
+@pytest.mark.parametrize("M", [1, 2, 5, 8, 16, 17, 40, 128])
+def test_gemm_w4a16_far_zero_points(M):
+    """Groups on one side of zero, far from it compared with their width, get zero-points far outside
+    [0, 15] (z = round(-min / s) is not clamped), where neither 128 + z nor q - z need fit bf16's 8
+    significant bits.  With activations of one sign no rounding error cancels: every kernel must still
+    meet the bound (M = 1, 2..16 and > 16 each take their own kernel)."""
+    N, K = 640, 2048
+    w = wq_inputs.offset_group_weight(N, K, 93)
+    x = wq_inputs.positive_activations(M, K, 94 + M)
+    _w4_case(N, K, 128, M, 0, wgen=w, xgen=x)
+
+
+@pytest.mark.parametrize("g,M,K", [(32, 1, 1024), (64, 4, 1024), (128, 1, 1152), (32, 40, 1024), (64, 64, 1024)])
+def test_gemm_w4a16_far_zero_points_other_kernels(g, M, K):
+    """The same for the CUDA-core kernel (groups of 32 and 64, and K that the TMA kernels do not take) and
+    the tensor-core kernel with several groups per stage."""
+    N = 384
+    w = wq_inputs.offset_group_weight(N, K, 95 + g, group=g)
+    x = wq_inputs.positive_activations(M, K, 96 + M)
+    _w4_case(N, K, g, M, 0, wgen=w, xgen=x)
+
+
 def test_gemm_w4a16_degenerate_groups():
     w = wq_inputs.llm_weight(64, 512, 81, dtype=torch.float32)
     w[0] = 0.0

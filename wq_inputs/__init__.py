@@ -24,6 +24,8 @@ weights are used anywhere.
 """
 from __future__ import annotations
 
+import math
+
 import torch
 
 WEIGHT_STD = 0.02
@@ -121,6 +123,31 @@ def heavy_tail_weight(N: int, K: int, seed: int, dtype=torch.float32) -> torch.T
     z = torch.randn(N, K, generator=g)
     c = (torch.randn(N, K, 3, generator=g) ** 2).sum(-1) / 3.0
     return (z / c.sqrt() * WEIGHT_STD).to(dtype)
+
+
+def offset_group_weight(N: int, K: int, seed: int, group: int = 128, dtype=torch.float32) -> torch.Tensor:
+    """[N][K] ~ N(0, 0.02), except every third row, which repeats one block of `group` values along K: a
+    band of width b (10^-2 to 1) whose near edge lies d from zero, on either side, with d / b log-uniform
+    in [8, 300].  Every block of such a row lies on one side of zero, far from it compared with its width
+    (a pattern real weights rarely show but the format allows)."""
+    g = _gen(seed)
+    w = torch.randn(N, K, generator=g) * WEIGHT_STD
+    rows = torch.arange(0, N, 3)
+    n = len(rows)
+    t = torch.rand(n, group, generator=g)
+    t[:, 0], t[:, 1] = 0.0, 1.0  # the band's edges are taken
+    width = 10.0 ** (-2.0 * torch.rand(n, 1, generator=g))
+    dist = width * 10.0 ** (math.log10(8.0) + torch.rand(n, 1, generator=g) * math.log10(300.0 / 8.0))
+    sign = torch.where(torch.rand(n, 1, generator=g) < 0.5, -1.0, 1.0)
+    block = sign * (dist + width * t)
+    w[rows] = block.repeat(1, K // group)
+    return w.to(dtype)
+
+
+def positive_activations(M: int, K: int, seed: int, device="cpu") -> torch.Tensor:
+    """bf16 [M][K] = |N(0, 1)| + 0.05: activations of one sign, so no rounding error cancels in a sum."""
+    g = _gen(seed + 3_000_017)
+    return (torch.randn(M, K, generator=g).abs() + 0.05).to(torch.bfloat16).to(device)
 
 
 def one_signed_weight(N: int, K: int, seed: int, dtype=torch.float32) -> torch.Tensor:
