@@ -12,13 +12,24 @@
 // per-group parameters).  Layout of the work: a warp takes 256 consecutive
 // weights of one row, 8 per lane (one 16-byte load for bf16), so a group of
 // g weights spans g/8 adjacent lanes and its min/max (or absmax) is a
-// log2(g/8)-step xor-shuffle reduction.  Every lane then derives the same
-// (s, z) and encodes its 8 weights into one 32-bit word of nibbles (INT4) or
-// one 64-bit word of bytes (INT8); stores are 128 contiguous bytes per warp.
+// log2(g/8)-step xor-shuffle reduction (for bf16 weights, min and -max
+// travel as one bf16 pair).  Every lane then derives the same (s, z) and
+// encodes its 8 weights into one 32-bit word of nibbles (INT4) or one 64-bit
+// word of bytes (INT8); stores are 128 contiguous bytes per warp.
 //
 // Arithmetic matches the library contract bit for bit: binary32 with
 // explicit round-to-nearest-even intrinsics (no contraction is possible),
-// rintf (round half to even), bf16 rounding to nearest even.
+// round half to even, bf16 rounding to nearest even.  Three equivalences
+// save instructions without changing a bit:
+//  * every quotient (w / s, -min / s, range / 15, absmax / 127) is RN of the
+//    exact quotient, formed from a reciprocal and one correction
+//    (quotient_rn), with the IEEE division outside the proven range;
+//  * clipping to the code range before rounding gives the same integer as
+//    rounding first, and adding 1.5 * 2^23 does the rounding (rint_bits);
+//  * the eight rounded patterns, shifted into place and summed, minus their
+//    summed offsets, are the packed nibbles.
+#include <type_traits>
+
 #include "wq_common.cuh"
 #include "wq_internal.h"
 
@@ -94,15 +105,47 @@ __device__ __forceinline__ float quotient_rn(float w, float s, float r)
     return __fmaf_rn(e, r, q0);
 }
 
-// s, z of one INT4 group from its min and max (the library contract).
-__device__ __forceinline__ void int4_params(float mn, float mx, float &s, float &z)
+// RN(d / c) for a bf16-representable constant c (15 or 127) with rc = RN(1 / c): the same identity, with
+// the IEEE division where d could leave its proven range (d non-finite, above 2^100, or tiny but not 0).
+__device__ __forceinline__ float div_by_const_rn(float d, float c, float rc)
 {
-    s = round_bf16(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
+    const float ad = fabsf(d);
+    return (ad <= 0x1p100f && (ad >= 0x1p-90f || ad == 0.0f)) ? quotient_rn(d, c, rc) : __fdiv_rn(d, c);
+}
+constexpr float kRcp15 = 0x1.111112p-4f;   // RN(1 / 15)
+constexpr float kRcp127 = 0x1.020408p-7f;  // RN(1 / 127)
+
+// Round an integer-bound value t, already clipped to [-127, 127], to the nearest integer with ties to
+// even, and return the binary32 bit pattern of 1.5 * 2^23 + round(t): the integer sits in the low bits
+// (two's complement in the low byte for negative t).  Adding 1.5 * 2^23 leaves a unit in the last place
+// of 1, so the addition itself is the rounding.
+__device__ __forceinline__ uint32_t rint_bits(float t) { return __float_as_uint(__fadd_rn(t, 0x1.8p23f)); }
+constexpr uint32_t kRintBase = 0x4B400000u;  // bits of 1.5 * 2^23
+
+// s of one INT4 group from its min and max (the library contract): RN((max - min) / 15) rounded to bf16;
+// a zero range falls back to max(|min|, |max|), then to 1.
+__device__ __forceinline__ float int4_scale(float mn, float mx)
+{
+    float s = round_bf16(div_by_const_rn(__fsub_rn(mx, mn), 15.0f, kRcp15));
     if (s == 0.0f) {
         s = round_bf16(fmaxf(fabsf(mn), fabsf(mx)));
         if (s == 0.0f) s = 1.0f;
     }
-    z = round_bf16(__fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.0f));
+    return s;
+}
+
+// bf16x2 minimum (each half; a NaN half yields the other operand's half, as fminf does)
+__device__ __forceinline__ uint32_t bf16x2_min(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 template <typename T, int LPG>
@@ -119,9 +162,11 @@ quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
     const int64_t tasks = N * chunks;
     const int64_t G = K / g;
 
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     TaskWalk walk(warp0, n_warps, chunks);
     for (int64_t t0 = warp0; t0 < tasks; t0 += n_warps * kQuantUnroll) {
         float v[kQuantUnroll][8];
+        uint4 raw[kQuantUnroll];  // bf16 input: the 8 weights as loaded
         int64_t n[kQuantUnroll], k0[kQuantUnroll];
         bool active[kQuantUnroll];
 #pragma unroll
@@ -129,41 +174,68 @@ quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
             n[u] = walk.n;
             k0[u] = walk.c * 256 + lane * 8;
             active[u] = (walk.n < N) && (k0[u] < K);
-            if (active[u]) load8<T>(w + n[u] * ldw + k0[u], v[u]);
+            if (kBf16) {
+                raw[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (active[u]) raw[u] = ld_stream_v4(w + n[u] * ldw + k0[u]);
+            } else if (active[u]) {
+                load8<T>(w + n[u] * ldw + k0[u], v[u]);
+            }
             walk.step();
         }
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
             if (t0 + u * n_warps >= tasks) break;  // warp-uniform
-            float mn = INFINITY, mx = -INFINITY;
-            if (active[u]) {
+            float mn, mx;
+            if (kBf16) {
+                // bf16 weights are exact in bf16: reduce (min, -max) as one packed pair (a group's lanes are
+                // all active or all inactive; inactive ones contribute +inf to both minima)
+                const uint32_t lo = bf16x2_min(bf16x2_min(raw[u].x, raw[u].y), bf16x2_min(raw[u].z, raw[u].w));
+                const uint32_t hi = bf16x2_max(bf16x2_max(raw[u].x, raw[u].y), bf16x2_max(raw[u].z, raw[u].w)) ^ 0x80008000u;
+                uint32_t pk = active[u] ? bf16x2_min(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632)) : 0x7F807F80u;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) { mn = fminf(mn, v[u][i]); mx = fmaxf(mx, v[u][i]); }
-            }
+                for (int o = 1; o < LPG; o <<= 1) pk = bf16x2_min(pk, __shfl_xor_sync(0xffffffffu, pk, o));
+                mn = __uint_as_float(pk << 16);
+                mx = __uint_as_float((pk & 0xffff0000u) ^ 0x80000000u);
+                const uint32_t u4[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
 #pragma unroll
-            for (int o = 1; o < LPG; o <<= 1) {
-                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                for (int i = 0; i < 4; ++i) {
+                    v[u][2 * i] = __uint_as_float(u4[i] << 16);
+                    v[u][2 * i + 1] = __uint_as_float(u4[i] & 0xffff0000u);
+                }
+            } else {
+                mn = INFINITY;
+                mx = -INFINITY;
+                if (active[u]) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) { mn = fminf(mn, v[u][i]); mx = fmaxf(mx, v[u][i]); }
+                }
+#pragma unroll
+                for (int o = 1; o < LPG; o <<= 1) {
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                }
             }
             if (!active[u]) continue;
-            float s, z;
-            int4_params(mn, mx, s, z);
+            const float s = int4_scale(mn, mx);
             float qd[8];  // RN(w / s)
+            float z;      // round_bf16(rint(RN(-min / s)) + 0)
             if (quotients_by_reciprocal(s, fmaxf(fabsf(mn), fabsf(mx)))) {
                 const float r = __frcp_rn(s);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) qd[i] = quotient_rn(v[u][i], s, r);
+                z = round_bf16(__fadd_rn(rintf(quotient_rn(-mn, s, r)), 0.0f));
             } else {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) qd[i] = __fdiv_rn(v[u][i], s);
+                z = round_bf16(__fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.0f));
             }
-            uint32_t packed = 0;
+            // q = clip(rint(RN(w / s) + z), 0, 15): clipping before the rounding gives the same integer,
+            // and rint_bits leaves it in the low bits; the eight patterns shifted into place and summed,
+            // minus the summed offsets, are the eight nibbles
+            uint32_t packed = 0u - kRintBase * 0x11111111u;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float q = rintf(__fadd_rn(qd[i], z));
-                q = fminf(fmaxf(q, 0.0f), 15.0f);
-                packed |= (uint32_t)q << (4 * i);
-            }
+            for (int i = 0; i < 8; ++i)
+                packed += rint_bits(fminf(fmaxf(__fadd_rn(qd[i], z), 0.0f), 15.0f)) << (4 * i);
             *reinterpret_cast<uint32_t *>(qweight + n[u] * (K >> 1) + (k0[u] >> 1)) = packed;
             if ((lane & (LPG - 1)) == 0) {
                 const int64_t gi = n[u] * G + k0[u] / g;
@@ -176,7 +248,7 @@ quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
 
 __device__ __forceinline__ float int8_scale(float amax)
 {
-    float s = round_bf16(__fdiv_rn(amax, 127.0f));
+    float s = round_bf16(div_by_const_rn(amax, 127.0f, kRcp127));
     return s == 0.0f ? 1.0f : s;
 }
 
@@ -191,14 +263,12 @@ __device__ __forceinline__ uint2 int8_encode8(const float v[8], float s)
 #pragma unroll
         for (int i = 0; i < 8; ++i) qd[i] = __fdiv_rn(v[i], s);
     }
-    uint32_t lo = 0, hi = 0;
+    // q = clip(rint(RN(w / s)), -127, 127): clip, then rint_bits leaves the code in the low byte
+    uint32_t b[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        float q = rintf(qd[i]);
-        q = fminf(fmaxf(q, -127.0f), 127.0f);
-        const uint32_t b = (uint32_t)(int)q & 0xffu;
-        if (i < 4) lo |= b << (8 * i); else hi |= b << (8 * (i - 4));
-    }
+    for (int i = 0; i < 8; ++i) b[i] = rint_bits(fminf(fmaxf(qd[i], -127.0f), 127.0f));
+    const uint32_t lo = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+    const uint32_t hi = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
     return make_uint2(lo, hi);
 }
 

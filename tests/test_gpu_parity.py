@@ -161,6 +161,37 @@ def test_quantize_degenerate_and_one_signed_groups():
         assert np.array_equal(q8.cpu().numpy(), c8) and np.array_equal(bits(s8), s8b)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_extreme_magnitudes(dtype):
+    """Rows scaled towards the ends of the binary32 range, subnormal groups and a group mixing a huge and
+    tiny values: the quantisers' reciprocal quotients hand these to the IEEE division (scales or
+    quotients outside [2^-100, 2^100], ranges outside [2^-90, 2^100]); codes and parameters stay
+    bit-exact either way."""
+    w = wq_inputs.llm_weight(48, 512, 83, dtype=torch.float32)
+    for i, e in enumerate((-140, -130, -120, -110, -100, -92, -88, 88, 96, 100, 104, 110, 120, 124)):
+        w[i] *= 2.0 ** e
+    w[16, :128] = 1e-40                       # subnormal constant group
+    w[17, :64] = 2.0 ** -135                  # smallest subnormals
+    w[17, 64:128] = -(2.0 ** -140)
+    w[18, :128] = w[18, :128] * 1e-38         # a group of subnormals and tiny normals
+    w[19, :128] = 1e-3
+    w[19, 5] = 1e30                           # one huge value in a small group
+    w[20, 128:256] = -1e30
+    w[20, 130] = 3e30
+    w[21] = w[21].abs() * 2.0 ** 100 + 2.0 ** 110   # one-signed, huge offset
+    w = w.to(dtype)
+    for g in (32, 128):
+        check_q4(w, g)
+        q8, s8 = wq.wq_quantize_int8(w.cuda(), g)
+        torch.cuda.synchronize()
+        c8, _, s8b = oracle_q8(w, g)
+        assert np.array_equal(q8.cpu().numpy(), c8) and np.array_equal(bits(s8), s8b)
+    q8, s8 = wq.wq_quantize_int8(w.cuda(), None)  # per output channel
+    torch.cuda.synchronize()
+    c8, _, s8b = oracle_q8(w, 512)
+    assert np.array_equal(q8.cpu().numpy(), c8) and np.array_equal(bits(s8), s8b)
+
+
 def test_quantize_worked_example_on_gpu():
     # the page's 8-weight group, replicated into one 32-wide group of a row
     v = torch.tensor([0.31, -0.12, 0.78, -0.05, 1.42, -0.91, 0.23, 0.66], dtype=torch.float32)
