@@ -16,7 +16,9 @@ Sources, by page title and section:
     outlier example, granularity and bits per weight).
   * "Test-time quantization: quantising on the fly with no calibration
     dataset" -- "The error of quantising an outlier with the wrong scale"
-    (rounding error at most half a scale).
+    (rounding error at most half a scale; the symmetric scale M / 7 at 4 bits).
+  * The same comparison page -- "The methods compared" (the AWQ example:
+    symmetric int4 with codes -7 to 7).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (page values, closed forms, brute force, invariants, an independent binary64
@@ -58,6 +60,7 @@ def _bind(path: str):
     P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     lib.oracle_quantize_int4.argtypes = [P, I64, I64, I64, I64, I, P, P, P]
     lib.oracle_quantize_int8.argtypes = [P, I64, I64, I64, I64, I, P, P]
+    lib.oracle_quantize_int4_sym.argtypes = [P, I64, I64, I64, I64, I, P, P]
     lib.oracle_pack_int4.argtypes = [P, I64, I64, P]
     lib.oracle_unpack_int4.argtypes = [P, I64, I64, P]
     lib.oracle_dequant_int4.argtypes = [P, P, P, I64, I64, I64, P]
@@ -143,6 +146,21 @@ def quantize_int4(w, g: int, mode: int = STORED):
     _check(_load().oracle_quantize_int4(_ptr(w), N, K, K, g, mode, _ptr(codes), _ptr(s), _ptr(z)),
            "quantize_int4")
     return codes, s, z
+
+
+def quantize_int4_sym(w, g: int, mode: int = STORED):
+    """Symmetric INT4 per group of ``g`` weights: s = max|w| / 7, q = clip(round(w / s), -7, 7).
+
+    Returns (codes uint8 [N][K] holding q + 8 in 1..15, s float32 [N][K/g]); the codes decode as
+    s * (code - 8), i.e. as asymmetric INT4 with z = 8.
+    """
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.empty((N, K), dtype=np.uint8)
+    s = np.empty((N, K // g), dtype=np.float32)
+    _check(_load().oracle_quantize_int4_sym(_ptr(w), N, K, K, g, mode, _ptr(codes), _ptr(s)),
+           "quantize_int4_sym")
+    return codes, s
 
 
 def pack_int4(codes) -> np.ndarray:

@@ -177,6 +177,50 @@ int oracle_unpack_int4(const uint8_t *packed, int64_t N, int64_t K, uint8_t *cod
 }
 
 /* ---------------------------------------------------------------------- */
+/* Symmetric INT4, one s per group, levels -7..7.                           */
+/* [P1C] "The error of quantising an outlier with the wrong scale": a       */
+/*      b-bit symmetric range covering a largest magnitude M has            */
+/*      s = M / (2^(b-1) - 1), M/7 at 4 bits.  [P3] "The methods compared"  */
+/*      (the AWQ example): symmetric int4 with codes -7 to 7.               */
+/*      q = clip(round(w/s), -7, 7), w_hat = q*s; max|w| = 0 gives s = 1.   */
+/*      The code is stored as q + 8 (1..15) in the INT4 nibble layout, so   */
+/*      the asymmetric decode s*(code - z) with z = 8 reads it as q*s.      */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * codes  : [N][K] output codes q + 8, one per byte (unpacked)
+ * s_out  : [N][K/g] scale as used for encoding
+ */
+int oracle_quantize_int4_sym(const float *w, int64_t N, int64_t K, int64_t ldw, int64_t g, int mode,
+                             uint8_t *codes, float *s_out)
+{
+    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0 || ldw < K) return -1;
+    const int64_t G = K / g;
+    int64_t n;
+#pragma omp parallel for schedule(static)
+    for (n = 0; n < N; ++n) {
+        for (int64_t gi = 0; gi < G; ++gi) {
+            const float *wg = w + n * ldw + gi * g;
+            float amax = 0.0f;  /* largest magnitude of the group */
+            for (int64_t i = 0; i < g; ++i) {
+                const float a = fabsf(wg[i]);
+                if (a > amax) amax = a;
+            }
+            float s = store_param(amax / 7.0f, mode);
+            if (s == 0.0f) s = 1.0f;
+            s_out[n * G + gi] = s;
+            for (int64_t i = 0; i < g; ++i) {
+                float q = nearbyintf(wg[i] / s);
+                if (q < -7.0f) q = -7.0f;
+                if (q > 7.0f) q = 7.0f;
+                codes[n * K + gi * g + i] = (uint8_t)((int)q + 8);
+            }
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------- */
 /* Symmetric absmax INT8, one s per group (g = K: one per output channel).  */
 /* [P3] "What quantisation does": s = max|w| / 127, q = round(w/s),        */
 /*      w_hat = q*s.  q is clipped to [-127, 127] because the stored bf16   */

@@ -32,6 +32,11 @@ MUTANTS = {
     "pack_nibbles_swapped": ("(codes[n * K + 2 * j] & 0xf) | ((codes[n * K + 2 * j + 1] & 0xf) << 4)",
                              "(codes[n * K + 2 * j + 1] & 0xf) | ((codes[n * K + 2 * j] & 0xf) << 4)"),
     "bf16_truncates": ("if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u))) kept += 1u;", ";"),
+    "sym_levels_8": ("amax / 7.0f", "amax / 8.0f"),
+    "sym_offset_7": ("(uint8_t)((int)q + 8)", "(uint8_t)((int)q + 7)"),
+    "sym_truncate": ("float q = nearbyintf(wg[i] / s);", "float q = truncf(wg[i] / s);"),
+    "sym_ties_away": ("float q = nearbyintf(wg[i] / s);", "float q = roundf(wg[i] / s);"),
+    "sym_signed_max": ("const float a = fabsf(wg[i]);", "const float a = wg[i];"),
 }
 
 PINS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

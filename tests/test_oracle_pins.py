@@ -348,3 +348,146 @@ def test_gemm_w4a16_reference_tiny():
         sl = slice(gi * 128, (gi + 1) * 128)
         ref += s[:, gi].astype(np.float64) * ((codes[:, sl].astype(np.float64) - z[:, gi:gi + 1]) @ xs[sl])
     assert np.all(np.abs(y[0] - ref) <= 1e-12 * a[0])
+
+
+# --------------------------------------------------------------------------
+# Symmetric INT4 (levels -7..7): "Test-time quantization ...", "The error of
+# quantising an outlier with the wrong scale"; the comparison page, "The
+# methods compared" (the AWQ example)
+# --------------------------------------------------------------------------
+
+def _sym_fixture():
+    sc, _ = read("int4_symmetric_examples.txt")
+    return sc
+
+
+def _sym_group(typical, outlier=None, g=32):
+    """A group whose typical magnitude is `typical` (values of both signs, the largest exactly `typical`),
+    plus one channel of magnitude |outlier| placed on the negative side."""
+    base = np.array([1.0, -1.0, 0.75, -0.5, 0.25, -0.875, 0.625, -0.125], dtype=np.float32) * typical
+    w = np.resize(base, g).astype(np.float32)
+    if outlier is not None:
+        w[3] = -outlier
+    return w[None, :]
+
+
+@pytest.mark.parametrize("mode", [oracle.EXACT, oracle.STORED])
+def test_sym_int4_shared_scale_with_outlier(mode):
+    """One 30x channel sets the scale: s = 30 / 7 (printed 4.29), half a step 2.14, so a value of
+    magnitude 1 may be off by up to 214 %; every error stays within half a step."""
+    sc = _sym_fixture()
+    w = _sym_group(scalar(sc, "typical_magnitude"), scalar(sc, "outlier_magnitude"))
+    codes, s = oracle.quantize_int4_sym(w, w.shape[1], mode)
+    s0 = float(s[0, 0])
+    if mode == oracle.EXACT:
+        assert round(s0, 2) == scalar(sc, "s_shared_printed")
+        assert round(s0 / 2, 2) == scalar(sc, "half_step_shared_printed")
+        assert round(100 * (s0 / 2) / scalar(sc, "typical_magnitude")) == scalar(sc, "rel_error_shared_percent_printed")
+    else:
+        assert abs(s0 - 30.0 / 7) <= U_BF16 * 30.0 / 7
+    q = codes[0].astype(np.int64) - 8
+    assert q.min() >= -7 and q.max() <= 7 and q[3] == -7
+    w_hat = q * np.float64(s0)
+    assert np.all(np.abs(w_hat - w[0]) <= 0.5 * s0 * (1 + 1e-6))
+    # the typical values all collapse onto the levels 0 and +-1 of the inflated scale
+    assert set(np.unique(np.delete(q, 3))) <= {-1, 0, 1}
+
+
+@pytest.mark.parametrize("mode", [oracle.EXACT, oracle.STORED])
+def test_sym_int4_segregated_scale(mode):
+    """Without the outlier (M = 1): s = 1/7 (printed 0.143), half a step 0.071, about 7 % of a value of
+    magnitude 1."""
+    sc = _sym_fixture()
+    w = _sym_group(scalar(sc, "typical_magnitude"))
+    codes, s = oracle.quantize_int4_sym(w, w.shape[1], mode)
+    s0 = float(s[0, 0])
+    if mode == oracle.EXACT:
+        assert round(s0, 3) == scalar(sc, "s_segregated_printed")
+        assert round(s0 / 2, 3) == scalar(sc, "half_step_segregated_printed")
+        assert round(100 * s0 / 2) == scalar(sc, "rel_error_segregated_percent_printed")
+    q = codes[0].astype(np.int64) - 8
+    assert np.all(np.abs(q * np.float64(s0) - w[0]) <= 0.5 * s0 * (1 + 1e-6))
+    assert q[0] == 7 and q[1] == -7  # +-1, the largest magnitude, sit on the end levels
+
+
+def _awq():
+    sc = _sym_fixture()
+    w = np.array([[float(v) for v in sc["awq_weights"][0]]], dtype=np.float32)
+    x = np.array([float(v) for v in sc["awq_activations"][0]])
+    return sc, w, x
+
+
+def test_sym_int4_awq_example_codes():
+    """Codes of the AWQ example (the page's table is lost; recomputed from s = max|w| / 7): within
+    the printed range -7..7, the largest weight on the top level."""
+    sc, w, x = _awq()
+    codes, s = oracle.quantize_int4_sym(w, w.shape[1], oracle.EXACT)
+    q = codes[0].astype(np.int64) - 8
+    assert q.tolist() == [2, -4, 3, 7]
+    assert q.min() >= scalar(sc, "awq_code_min") and q.max() <= scalar(sc, "awq_code_max")
+    assert abs(float(s[0, 0]) - 0.90 / 7) < 1e-7
+
+
+def test_sym_int4_awq_scaling_helps_only_the_salient_channel():
+    """Scaling the salient channel (activation 10x the others) up by 2 before quantising and its
+    activation down by 2 (the factor the page used is lost; 2 keeps the group maximum): the other
+    channels' codes and rounding errors do not change, the salient channel's error in the output falls,
+    and so does the output error."""
+    sc, w, x = _awq()
+    g = w.shape[1]
+    codes, s = oracle.quantize_int4_sym(w, g, oracle.EXACT)
+    w_hat = (codes[0].astype(np.float64) - 8) * float(s[0, 0])
+    f = np.array([2.0, 1.0, 1.0, 1.0])
+    ws = (w * f).astype(np.float32)
+    codes2, s2 = oracle.quantize_int4_sym(ws, g, oracle.EXACT)
+    assert float(s2[0, 0]) == float(s[0, 0])  # the group maximum, 0.90, is unchanged
+    w_hat2 = (codes2[0].astype(np.float64) - 8) * float(s2[0, 0]) / f  # effective weights seen by x
+    assert codes2[0, 1:].tolist() == codes[0, 1:].tolist()
+    assert np.allclose(w_hat2[1:] - w[0, 1:], w_hat[1:] - w[0, 1:])
+    assert abs(w_hat2[0] - w[0, 0]) < abs(w_hat[0] - w[0, 0])
+    y = float(x @ w[0].astype(np.float64))
+    assert abs(float(x @ w_hat2) - y) < abs(float(x @ w_hat) - y)
+
+
+@pytest.mark.parametrize("g", [8, 32, 128])
+def test_sym_int4_error_at_most_half_scale(g):
+    w = _groups(61, 2000 // g * 8, g)
+    codes, s = oracle.quantize_int4_sym(w, g, oracle.EXACT)
+    q = codes.astype(np.float64) - 8
+    err = np.abs(q * np.repeat(s.astype(np.float64), g, axis=1) - w.astype(np.float64))
+    assert np.all(err <= 0.5 * np.repeat(s.astype(np.float64), g, axis=1) * (1 + 1e-5))
+    # the largest magnitude of every group sits on +-7
+    idx = np.abs(w).argmax(axis=1)
+    assert np.all(np.abs(q[np.arange(w.shape[0]), idx]) == 7)
+
+
+@pytest.mark.parametrize("mode", [oracle.EXACT, oracle.STORED])
+def test_sym_int4_codes_are_nearest_levels(mode):
+    w = _groups(71, 300, 8)
+    codes, s = oracle.quantize_int4_sym(w, 8, mode)
+    amax = np.abs(w).max(1).astype(np.float64)
+    rel = 1e-6 if mode == oracle.EXACT else U_BF16 * 1.0001
+    assert np.all(np.abs(s[:, 0] - amax / 7) <= rel * amax / 7)
+    levels = np.arange(-7, 8, dtype=np.float64)
+    for i in range(w.shape[0]):
+        t = w[i].astype(np.float64) / float(s[i, 0])
+        d = np.abs(t[:, None] - levels[None, :])
+        chosen = d[np.arange(8), codes[i].astype(np.int64) - 1]
+        assert np.all(chosen <= d.min(axis=1) + 1e-5)
+
+
+def test_sym_int4_special_groups_and_asymmetric_decode():
+    """An all-zero group gets s = 1 and code 8 (q = 0); a constant group sits on +-7; ties go to even;
+    and the stored codes decode through the asymmetric INT4 formula with z = 8."""
+    w = np.zeros((4, 8), dtype=np.float32)
+    w[1, :] = -0.25
+    w[2, :] = np.array([7.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5])  # s = 1 exactly, halves tie
+    w[3, :] = np.array([0.3, -0.1, 0.7, 0.05, -0.6, 0.2, 0.45, -0.35])
+    for mode in (oracle.EXACT, oracle.STORED):
+        codes, s = oracle.quantize_int4_sym(w, 8, mode)
+        q = codes.astype(np.int64) - 8
+        assert s[0, 0] == 1.0 and q[0].tolist() == [0] * 8
+        assert q[1].tolist() == [-7] * 8
+        assert s[2, 0] == 1.0 and q[2].tolist() == [7, 0, 2, 2, 0, -2, -2, 4]
+        z = np.full(s.shape, 8.0, dtype=np.float32)
+        assert np.array_equal(oracle.dequant_int4(codes, s, z, 8), q * np.repeat(s.astype(np.float64), 8, axis=1))
