@@ -313,6 +313,31 @@ def int8_rows(wq, device, copies=8, reps=5):
             {"us": gms * 1e3, "GB_s": gbytes / (gms * 1e-3) / 1e9, "shape": "K=N=8192 per-channel, M=1"})
 
 
+def sym_int4_row(wq, device, copies=8, reps=5):
+    """Symmetric INT4 quantisation (levels -7..7, g = 128) at K = N = 8192, rotating over copies (> 3x L2)."""
+    K = N = 8192
+    ws = [wq_inputs.llm_weight(N, K, wq_inputs.SEEDS["gran"] + 100 + c, device=device) for c in range(copies)]
+    qs = [torch.empty((N, K // 2), dtype=torch.uint8, device=device) for _ in range(copies)]
+    ss = [torch.empty((N, K // G), dtype=torch.bfloat16, device=device) for _ in range(copies)]
+    zs = [torch.empty((N, K // G), dtype=torch.bfloat16, device=device) for _ in range(copies)]
+    for c in range(copies):
+        wq.wq_quantize_int4_sym(ws[c], G, qs[c], ss[c], zs[c])
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for r in range(reps):
+        for c in range(copies):
+            wq.wq_quantize_int4_sym(ws[c], G, qs[c], ss[c], zs[c])
+    e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * copies)
+    del ws
+    torch.cuda.empty_cache()
+    nbytes = N * K * 2 + N * K // 2 + 4 * N * (K // G)
+    return {"us": round(ms * 1e3, 2), "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "shape": "K=N=8192 bf16->symmetric int4 g128 (zero-points 8)"}
+
+
 def per_linear_us(model, xs, ys, reps=5):
     """Average device time of each linear shape at M = 1: the 80 calls of one shape replayed as a CUDA
     graph (as in the step), events around the replays."""
@@ -480,6 +505,7 @@ def main():
     torch.cuda.empty_cache()
 
     q8_row, g8_row = int8_rows(wq, device)
+    sym_row = sym_int4_row(wq, device)
 
     quant_gbs = model.quant_bytes / (model.quant_ms * 1e-3) / 1e9
 
@@ -511,6 +537,7 @@ def main():
             "a4_w4a16_m1_per_linear": lin,
             "a5_w4a16_m128": {"tflops": round(tflops128 / world, 1)},
             "a6_w8a16_m1": {k: (round(v, 2) if isinstance(v, float) else v) for k, v in g8_row.items()},
+            "f1_quantize_int4_sym": sym_row,
         },
         "roofline": {"bound": "hbm", "kernel": "gemv_w4a16_m1_kernel", "achieved": round(per_gpu_gbs, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(per_gpu_gbs / peaks["hbm_gbs"], 4),

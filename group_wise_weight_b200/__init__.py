@@ -60,6 +60,8 @@ def lib():
         L.wq_version.restype = I
         L.wq_quantize_int4.argtypes = [P, I, I64, I64, I64, I, P, P, P, P]
         L.wq_quantize_int4.restype = I
+        L.wq_quantize_int4_sym.argtypes = [P, I, I64, I64, I64, I, P, P, P, P]
+        L.wq_quantize_int4_sym.restype = I
         L.wq_quantize_int8.argtypes = [P, I, I64, I64, I64, I, P, P, P]
         L.wq_quantize_int8.restype = I
         L.wq_gemm_workspace_bytes.argtypes = [I64, I64, I64, I, I]
@@ -136,6 +138,29 @@ def wq_quantize_int4(w: torch.Tensor, g: int = 128, qweight=None, scales=None, z
         _dense(t, n)
     _check(lib().wq_quantize_int4(_dev(w, "w"), wtype, N, K, w.stride(0), int(g), _dev(qweight, "qweight"),
                                   _dev(scales, "scales"), _dev(zeros, "zeros"), _stream_handle(stream)))
+    return qweight, scales, zeros
+
+
+def wq_quantize_int4_sym(w: torch.Tensor, g: int = 128, qweight=None, scales=None, zeros=None, stream=None):
+    """Symmetric INT4 (levels -7..7) per group of g weights along K, in the INT4 format of
+    wq_quantize_int4 with every zero-point 8 (codes q + 8), ready for wq_gemm_w4a16.
+
+    Returns (qweight uint8 [N][K/2], scales bf16 [N][K/g], zeros bf16 [N][K/g] all 8).
+    """
+    if w.dim() != 2 or w.stride(1) != 1:
+        raise ValueError("w must be a 2-D tensor with unit stride along K")
+    wtype = {torch.float32: WQ_F32, torch.bfloat16: WQ_BF16}.get(w.dtype)
+    if wtype is None:
+        raise TypeError("w must be float32 or bfloat16")
+    N, K = w.shape
+    dev = w.device
+    qweight = torch.empty((N, K // 2), dtype=torch.uint8, device=dev) if qweight is None else qweight
+    scales = torch.empty((N, K // g), dtype=torch.bfloat16, device=dev) if scales is None else scales
+    zeros = torch.empty((N, K // g), dtype=torch.bfloat16, device=dev) if zeros is None else zeros
+    for t, n in ((qweight, "qweight"), (scales, "scales"), (zeros, "zeros")):
+        _dense(t, n)
+    _check(lib().wq_quantize_int4_sym(_dev(w, "w"), wtype, N, K, w.stride(0), int(g), _dev(qweight, "qweight"),
+                                      _dev(scales, "scales"), _dev(zeros, "zeros"), _stream_handle(stream)))
     return qweight, scales, zeros
 
 

@@ -139,6 +139,16 @@ int wq_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw
     return check_launch("wq_quantize_int4");
 }
 
+int wq_quantize_int4_sym(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *qweight,
+                         uint16_t *scales, uint16_t *zeros, void *stream)
+{
+    g_last_error.clear();
+    int rc = check_quantize("wq_quantize_int4_sym", w, wtype, N, K, ldw, g, qweight, scales, zeros, false);
+    if (rc != WQ_OK) return rc;
+    wq::launch_quantize_int4_sym(w, wtype, N, K, ldw, g, qweight, scales, zeros, static_cast<cudaStream_t>(stream));
+    return check_launch("wq_quantize_int4_sym");
+}
+
 int wq_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, int8_t *qweight,
                      uint16_t *scales, void *stream)
 {

@@ -6,7 +6,8 @@
 // s = (max - min) / 15, z = round(-min / s), q = clip(round(w / s + z), 0, 15).
 // Symmetric INT8 follows "Quantization Methods Compared: INT8, GPTQ, AWQ, FP8,
 // FP4 and KV-Cache Quantization", section "What quantisation does":
-// s = max|w| / 127, q = round(w / s).
+// s = max|w| / 127, q = round(w / s).  Symmetric INT4 (levels -7..7,
+// s = max|w| / 7) is described at quant_int4_sym_kernel.
 //
 // Both are HBM streams (read 2 or 4 B per weight, write 0.5 or 1 B plus the
 // per-group parameters).  Layout of the work: a warp takes 256 consecutive
@@ -113,6 +114,7 @@ __device__ __forceinline__ float div_by_const_rn(float d, float c, float rc)
     return (ad <= 0x1p100f && (ad >= 0x1p-90f || ad == 0.0f)) ? quotient_rn(d, c, rc) : __fdiv_rn(d, c);
 }
 constexpr float kRcp15 = 0x1.111112p-4f;   // RN(1 / 15)
+constexpr float kRcp7 = 0x1.24924ap-3f;    // RN(1 / 7)
 constexpr float kRcp127 = 0x1.020408p-7f;  // RN(1 / 127)
 
 // Round an integer-bound value t, already clipped to [-127, 127], to the nearest integer with ties to
@@ -364,6 +366,83 @@ quant_int8_row_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw
     }
 }
 
+// Symmetric INT4 ("Test-time quantization: quantising on the fly with no calibration dataset", section
+// "The error of quantising an outlier with the wrong scale": s = M / (2^(b-1) - 1) = max|w| / 7 at 4
+// bits; the comparison page's AWQ example: codes -7 to 7).  q = clip(rint(RN(w / s)), -7, 7), stored as
+// the nibble q + 8 with a zero-point of 8, so the asymmetric decode s (code - z) reads it as s q.
+__device__ __forceinline__ float int4_sym_scale(float amax)
+{
+    float s = round_bf16(div_by_const_rn(amax, 7.0f, kRcp7));
+    return s == 0.0f ? 1.0f : s;
+}
+
+__device__ __forceinline__ uint32_t int4_sym_encode8(const float v[8], float s, float amax)
+{
+    float qd[8];  // RN(w / s)
+    if (quotients_by_reciprocal(s, amax)) {
+        const float r = __frcp_rn(s);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qd[i] = quotient_rn(v[i], s, r);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qd[i] = __fdiv_rn(v[i], s);
+    }
+    // rint_bits leaves q (two's complement) in the low bits: the shifted patterns summed, minus their
+    // offsets, plus 8 in every nibble, are the eight nibbles q + 8 (each in 1..15, so nothing carries)
+    uint32_t packed = 0x88888888u - kRintBase * 0x11111111u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) packed += rint_bits(fminf(fmaxf(qd[i], -7.0f), 7.0f)) << (4 * i);
+    return packed;
+}
+
+template <typename T, int LPG>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_int4_sym_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw, uint8_t *__restrict__ qweight,
+                      uint16_t *__restrict__ scales, uint16_t *__restrict__ zeros)
+{
+    constexpr int g = LPG * 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t chunks = (K + 255) >> 8;
+    const int64_t tasks = N * chunks;
+    const int64_t G = K / g;
+
+    TaskWalk walk(warp0, n_warps, chunks);
+    for (int64_t t0 = warp0; t0 < tasks; t0 += n_warps * kQuantUnroll) {
+        float v[kQuantUnroll][8];
+        int64_t n[kQuantUnroll], k0[kQuantUnroll];
+        bool active[kQuantUnroll];
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            n[u] = walk.n;
+            k0[u] = walk.c * 256 + lane * 8;
+            active[u] = (walk.n < N) && (k0[u] < K);
+            if (active[u]) load8<T>(w + n[u] * ldw + k0[u], v[u]);
+            walk.step();
+        }
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            if (t0 + u * n_warps >= tasks) break;  // warp-uniform
+            float amax = 0.0f;
+            if (active[u]) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[u][i]));
+            }
+#pragma unroll
+            for (int o = 1; o < LPG; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            if (!active[u]) continue;
+            const float s = int4_sym_scale(amax);
+            *reinterpret_cast<uint32_t *>(qweight + n[u] * (K >> 1) + (k0[u] >> 1)) = int4_sym_encode8(v[u], s, amax);
+            if ((lane & (LPG - 1)) == 0) {
+                const int64_t gi = n[u] * G + k0[u] / g;
+                scales[gi] = f32_to_bf16(s);
+                zeros[gi] = 0x4100u;  // 8.0 in bf16
+            }
+        }
+    }
+}
+
 template <typename KernelT>
 int persistent_grid(KernelT kernel, int64_t tasks_in_warps)
 {
@@ -407,6 +486,27 @@ void dispatch_int4(const void *w, int64_t N, int64_t K, int64_t ldw, int g, uint
     }
 }
 
+template <typename T, int LPG>
+void launch_int4_sym(const void *w, int64_t N, int64_t K, int64_t ldw, uint8_t *q, uint16_t *s, uint16_t *z,
+                     cudaStream_t st)
+{
+    auto k = quant_int4_sym_kernel<T, LPG>;
+    const int64_t tasks = N * ((K + 255) / 256);
+    const int grid = persistent_grid(k, tasks);
+    k<<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(w), N, K, ldw, q, s, z);
+}
+
+template <typename T>
+void dispatch_int4_sym(const void *w, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *q, uint16_t *s,
+                       uint16_t *z, cudaStream_t st)
+{
+    switch (g) {
+    case 32: launch_int4_sym<T, 4>(w, N, K, ldw, q, s, z, st); break;
+    case 64: launch_int4_sym<T, 8>(w, N, K, ldw, q, s, z, st); break;
+    default: launch_int4_sym<T, 16>(w, N, K, ldw, q, s, z, st); break;
+    }
+}
+
 template <typename T>
 void dispatch_int8(const void *w, int64_t N, int64_t K, int64_t ldw, int g, int8_t *q, uint16_t *s,
                    cudaStream_t st)
@@ -429,6 +529,13 @@ void launch_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_
 {
     if (wtype == WQ_F32) dispatch_int4<float>(w, N, K, ldw, g, q, s, z, st);
     else dispatch_int4<__nv_bfloat16>(w, N, K, ldw, g, q, s, z, st);
+}
+
+void launch_quantize_int4_sym(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *q,
+                              uint16_t *s, uint16_t *z, cudaStream_t st)
+{
+    if (wtype == WQ_F32) dispatch_int4_sym<float>(w, N, K, ldw, g, q, s, z, st);
+    else dispatch_int4_sym<__nv_bfloat16>(w, N, K, ldw, g, q, s, z, st);
 }
 
 void launch_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, int8_t *q,

@@ -15,7 +15,12 @@
  *       one scale per tensor, per output channel or per group of 128 (or 32)
  *       consecutive weights.  Section "Hardware, formats and the roofline":
  *       a decode step reads all the weights once, and 4-bit weights are
- *       turned back into 16-bit values inside the matmul kernel.
+ *       turned back into 16-bit values inside the matmul kernel.  Section
+ *       "The methods compared": the AWQ example, symmetric int4 with codes
+ *       -7 to 7.
+ *  [P1C] "Test-time quantization: quantising on the fly with no calibration
+ *       dataset", section "The error of quantising an outlier with the wrong
+ *       scale": a b-bit symmetric scale s = M / (2^(b-1) - 1), M / 7 at 4 bits.
  *
  * Conventions shared by every call
  *  - Weights are stored one row per output channel: W is [N][K] with K (the
@@ -90,6 +95,23 @@ int wq_version(void);
  */
 int wq_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g,
                      uint8_t *qweight, uint16_t *scales, uint16_t *zeros, void *stream);
+
+/*
+ * Symmetric INT4 quantisation, one scale per group of g consecutive weights,
+ * levels -7..7  ([P1C] "The error of quantising an outlier with the wrong
+ * scale"; [P3] "The methods compared").  The output is the asymmetric INT4
+ * format above with every zero-point 8, so wq_gemm_w4a16 consumes it as is.
+ *
+ *   w, qweight, scales, zeros: as wq_quantize_int4
+ *
+ * Per group, in binary32:
+ *   s  = bf16(max|w| / 7); if s == 0: s = 1
+ *   q  = clip(round(w / s), -7, 7)            with the stored s
+ *   stored code q + 8 (1..15), zero-point 8: s * (code - 8) = s * q
+ * Requirements: as wq_quantize_int4.
+ */
+int wq_quantize_int4_sym(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g,
+                         uint8_t *qweight, uint16_t *scales, uint16_t *zeros, void *stream);
 
 /*
  * Symmetric absmax INT8 quantisation  ([P3] "What quantisation does").

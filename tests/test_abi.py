@@ -72,6 +72,19 @@ def test_quantize_int4_rejects(L, kw, code):
     assert wq.wq_last_error() != ""
 
 
+def _q4s(L, w=A, wt=wq.WQ_BF16, N=4, K=256, ldw=256, g=128, q=A, s=A, z=A):
+    return L.wq_quantize_int4_sym(w, wt, N, K, ldw, g, q, s, z, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(z=None), wq.WQ_ERR_ARG), (dict(N=0), wq.WQ_ERR_ARG), (dict(g=256), wq.WQ_ERR_UNSUPPORTED),
+    (dict(wt=3), wq.WQ_ERR_UNSUPPORTED), (dict(K=96, ldw=96), wq.WQ_ERR_SHAPE), (dict(z=MIS), wq.WQ_ERR_ALIGN),
+])
+def test_quantize_int4_sym_rejects(L, kw, code):
+    assert _q4s(L, **kw) == code
+    assert wq.wq_last_error() != ""
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(s=None), wq.WQ_ERR_ARG), (dict(g=100), wq.WQ_ERR_UNSUPPORTED),
     (dict(K=160, ldw=160, g=128), wq.WQ_ERR_SHAPE), (dict(q=MIS), wq.WQ_ERR_ALIGN),

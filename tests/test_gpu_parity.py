@@ -192,6 +192,59 @@ def test_quantize_extreme_magnitudes(dtype):
     assert np.array_equal(q8.cpu().numpy(), c8) and np.array_equal(bits(s8), s8b)
 
 
+def check_q4_sym(w: torch.Tensor, g: int):
+    q, s, z = wq.wq_quantize_int4_sym(w.cuda(), g)
+    torch.cuda.synchronize()
+    codes, so = oracle.quantize_int4_sym(w_f32(w), g)
+    assert np.array_equal(q.cpu().numpy(), oracle.pack_int4(codes)), "packed symmetric codes differ"
+    assert np.array_equal(bits(s), oracle.bf16_bits(so)), "symmetric scales differ"
+    assert np.all(bits(z) == oracle.bf16_bits(np.float32(8.0))), "zero-points are not all 8"
+    return q, s, z, (codes, so)
+
+
+def _sym_weights(N, K, seed, dtype=torch.float32):
+    w = wq_inputs.llm_weight(N, K, seed, dtype=torch.float32)
+    w[0] = 0.0                                            # all-zero row: s = 1, codes 8
+    w[1, :128] = -0.25                                    # constant group: -7
+    w[2, :8] = torch.tensor([7.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 3.5])  # s = 1 with g = 8 .. ties
+    w[3, 5] = -30.0                                       # one 30x outlier channel
+    w[4] = w[4].abs() + 0.5                               # one-signed row
+    return w.to(dtype)
+
+
+@pytest.mark.parametrize("g", [32, 64, 128])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_int4_sym(g, dtype):
+    check_q4_sym(_sym_weights(300, 1024, 120 + g, dtype), g)
+
+
+def test_quantize_int4_sym_padded_and_extreme():
+    base = wq_inputs.llm_weight(40, 520, 131, dtype=torch.float32)
+    for i, e in enumerate((-140, -120, -100, -90, 90, 100, 110, 124)):
+        base[i] *= 2.0 ** e
+    base[9, :64] = 1e-40
+    base[10, 3] = 1e30
+    # a column slice of a wider matrix (ldw = 520 > K = 512)
+    q, s, z = wq.wq_quantize_int4_sym(base.cuda()[:, :512], 64)
+    torch.cuda.synchronize()
+    codes, so = oracle.quantize_int4_sym(base[:, :512].contiguous().numpy(), 64)
+    assert np.array_equal(q.cpu().numpy(), oracle.pack_int4(codes)) and np.array_equal(bits(s), oracle.bf16_bits(so))
+
+
+@pytest.mark.parametrize("M", [1, 2, 8, 40, 128])
+def test_gemm_w4a16_on_symmetric_codes(M):
+    """Symmetric codes go through the W4A16 matmul unchanged (zero-point 8): within the bound of the
+    oracle's s * q decode."""
+    N, K, g = 640, 2048, 128
+    w = _sym_weights(N, K, 140)
+    x = wq_inputs.activations(M, K, 141 + M)
+    q, s, z, (codes, so) = check_q4_sym(w, g)
+    y = wq.wq_gemm_w4a16(x.cuda(), q, s, z, g)
+    torch.cuda.synchronize()
+    y_ref, a_ref = oracle.gemm_w4a16(x.double().numpy(), codes, so, np.full(so.shape, 8.0, np.float32), g)
+    check_y(y.cpu(), y_ref, a_ref)
+
+
 def test_quantize_worked_example_on_gpu():
     # the page's 8-weight group, replicated into one 32-wide group of a row
     v = torch.tensor([0.31, -0.12, 0.78, -0.05, 1.42, -0.91, 0.23, 0.66], dtype=torch.float32)
