@@ -29,7 +29,10 @@
 //    rounding first, and adding 1.5 * 2^23 does the rounding (rint_bits);
 //  * the eight rounded patterns, shifted into place and summed, minus their
 //    summed offsets, are the packed nibbles.
+#include <map>
+#include <mutex>
 #include <type_traits>
+#include <utility>
 
 #include "wq_common.cuh"
 #include "wq_internal.h"
@@ -443,16 +446,29 @@ quant_int4_sym_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw
     }
 }
 
+// Grid of a persistent quantiser: enough CTAs for the work, at most the resident capacity of the device
+// (SMs x resident CTAs of this kernel), which is looked up once per kernel and device.
 template <typename KernelT>
 int persistent_grid(KernelT kernel, int64_t tasks_in_warps)
 {
-    int dev = 0, sms = 148, per_sm = 1;
+    static std::mutex mu;
+    static std::map<std::pair<int, const void *>, int64_t> cap_of;  // (device, kernel) -> capacity
+    int dev = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQuantThreads, 0);
-    if (per_sm < 1) per_sm = 1;
+    const std::pair<int, const void *> key(dev, reinterpret_cast<const void *>(kernel));
+    int64_t cap;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cap_of.find(key);
+        if (it == cap_of.end()) {
+            int sms = 148, per_sm = 1;
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kQuantThreads, 0);
+            it = cap_of.emplace(key, (int64_t)sms * (per_sm < 1 ? 1 : per_sm)).first;
+        }
+        cap = it->second;
+    }
     const int64_t want = (tasks_in_warps + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
-    const int64_t cap = (int64_t)sms * per_sm;
     return (int)(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
