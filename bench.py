@@ -113,11 +113,17 @@ def barrier(world):
         dist.barrier()
 
 
+def _scalar_device():
+    """Where the scalars that cross ranks live: the GPU under NCCL, the host under gloo."""
+    import torch.distributed as dist
+    return torch.device("cuda") if dist.get_backend() == "nccl" else torch.device("cpu")
+
+
 def reduce_max(v: float, world: int) -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_scalar_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -126,9 +132,14 @@ def reduce_sum(v: float, world: int) -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_scalar_device())
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def job_throughput(bytes_this_rank: float, ms_this_rank: float, world: int) -> float:
+    """Whole-job GB/s of independent replicas: the bytes all ranks moved over the slowest rank's time."""
+    return reduce_sum(bytes_this_rank, world) / (reduce_max(ms_this_rank, world) * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------------------
@@ -464,11 +475,11 @@ def main():
     run1 = (lambda: g1.replay()) if g1 is not None else step1
 
     with Clocks(local) as clk:
-        ms1 = time_steps(run1, args.steps, args.warmup, world)
+        ms1_rank = time_steps(run1, args.steps, args.warmup, world)
     clocks = clk.summary()
-    ms1 = reduce_max(ms1, world)
+    ms1 = reduce_max(ms1_rank, world)
     t_step = ms1 / args.steps
-    value = reduce_sum(bytes1 * args.steps, world) / (ms1 * 1e-3) / 1e9
+    value = job_throughput(bytes1 * args.steps, ms1_rank, world)
 
     # the same step through the C ABI with host buffers: pinned H2D of every activation, D2H of every output
     x_host = torch.cat([x.reshape(-1) for x in xs1]).cpu().pin_memory()
@@ -487,8 +498,9 @@ def main():
         model.step(xs_view, ys_view)
         y_host.copy_(y_dev, non_blocking=True)
 
-    ms_e2e = reduce_max(time_steps(e2e_step, args.steps, args.warmup, world), world)
-    e2e_value = reduce_sum(bytes1 * args.steps, world) / (ms_e2e * 1e-3) / 1e9
+    ms_e2e_rank = time_steps(e2e_step, args.steps, args.warmup, world)
+    ms_e2e = reduce_max(ms_e2e_rank, world)
+    e2e_value = job_throughput(bytes1 * args.steps, ms_e2e_rank, world)
 
     lin = per_linear_us(model, xs1, ys1)
 
