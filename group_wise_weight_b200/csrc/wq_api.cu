@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <string>
 
 #include "wq_common.cuh"
@@ -79,15 +80,19 @@ namespace {
 // Device address of the status word on the current device (looked up once per device).
 int *status_word()
 {
-    static int *addr[128] = {};
+    // the device address of the status word, looked up once per device (host threads may race to fill
+    // an entry; they store the same address)
+    static std::atomic<int *> addr[128] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
-    if (!addr[dev]) {
+    int *a = addr[dev].load(std::memory_order_acquire);
+    if (!a) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_wq_device_status) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<int *>(p);
+        a = static_cast<int *>(p);
+        addr[dev].store(a, std::memory_order_release);
     }
-    return addr[dev];
+    return a;
 }
 
 }  // namespace

@@ -22,10 +22,12 @@ void launch_gemv_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const
                        int g, uint16_t *y, cudaStream_t st);
 
 // W4A16 for M = 1, group 128 (wq_gemv_m1.cu): persistent stream-K over
-// (32-row block, group) units, per-warp TMA pipelines, mma.sync.  Needs a
+// (256-row tile, group pair) units, one TMA producer warp per CTA feeding
+// 16 mma.sync consumer warps, a combiner warp for split tiles.  Needs a
 // workspace of gemv_m1_workspace_bytes() (zero-filled before first use; the
 // kernel leaves its counters zeroed) and the device status word for its
-// bounded waits.  Returns 0, or -1 if a tensor map cannot be encoded.
+// bounded waits.  Returns 0, -1 if a tensor map cannot be encoded, -2 if the
+// launch fails.
 bool gemv_m1_eligible(int64_t M, int64_t N, int64_t K, int g);
 size_t gemv_m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
 int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
