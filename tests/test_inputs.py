@@ -28,3 +28,15 @@ def test_offset_group_weight_reaches_zero_points_bf16_cannot_shift():
 def test_positive_activations_have_one_sign():
     x = wq_inputs.positive_activations(4, 1024, 7).float().numpy()
     assert (x > 0).all()
+
+
+def test_activations_channel_seed_fixes_the_salient_channels():
+    """With channel_seed, two draws share their salient channels (inputs of one layer); without it the
+    channels follow the seed."""
+    import numpy as np
+    a = wq_inputs.activations(64, 1024, 1, channel_seed=9).float().abs().mean(0).numpy()
+    b = wq_inputs.activations(64, 1024, 2, channel_seed=9).float().abs().mean(0).numpy()
+    top_a, top_b = set(np.argsort(a)[-10:]), set(np.argsort(b)[-10:])
+    assert top_a == top_b
+    c = wq_inputs.activations(64, 1024, 2).float().abs().mean(0).numpy()
+    assert set(np.argsort(c)[-10:]) != top_a

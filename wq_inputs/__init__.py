@@ -85,13 +85,16 @@ def block_outlier_weight(N: int, K: int, seed: int, block: int = 1024, mult: flo
 
 
 def activations(M: int, K: int, seed: int, salient_frac: float = 0.01, salient_mult: float = 20.0,
-                device="cpu") -> torch.Tensor:
-    """bf16 [M][K] ~ N(0, 1); a random ``salient_frac`` of the K channels multiplied by salient_mult."""
+                device="cpu", channel_seed: int | None = None) -> torch.Tensor:
+    """bf16 [M][K] ~ N(0, 1); a random ``salient_frac`` of the K channels multiplied by salient_mult.
+    With ``channel_seed`` the salient channels are fixed by it (the same channels for every ``seed``, as
+    the inputs of one layer would be); without it they follow ``seed``."""
     g = _gen(seed + 1_000_003, device)
     x = torch.randn(M, K, generator=g, device=device)
     n_sal = int(round(salient_frac * K))
     if n_sal > 0:
-        ch = torch.randperm(K, generator=g, device=device)[:n_sal]
+        gc = g if channel_seed is None else _gen(channel_seed + 7_000_001, device)
+        ch = torch.randperm(K, generator=gc, device=device)[:n_sal]
         x[:, ch] *= salient_mult
     return x.to(torch.bfloat16)
 
