@@ -37,7 +37,7 @@ def _rank(rank, world, port, out):
 
 def test_two_gloo_ranks_agree_on_the_job_throughput():
     world, port = 2, _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_rank, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
         got = dict(out)
