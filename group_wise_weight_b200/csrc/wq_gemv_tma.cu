@@ -99,7 +99,7 @@ struct SmemLayout {
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-__host__ __device__ inline SmemLayout smem_layout(int64_t M, int64_t K, int MP, bool xsmem)
+__host__ __device__ inline SmemLayout smem_layout(int64_t M, int64_t K, bool xsmem)
 {
     SmemLayout L;
     const int64_t G = K >> 7;
@@ -158,11 +158,10 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tmap, const uint16_t *
                       uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ counters,
                       int *__restrict__ status)
 {
-    constexpr int MP = 8 * NT;
     extern __shared__ uint8_t smem_raw[];
     // 1 KB-align the ring (TMA destinations want 128 B at least)
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    const SmemLayout L = smem_layout(M, K, MP, XSMEM);
+    const SmemLayout L = smem_layout(M, K, XSMEM);
     uint8_t *stage = smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *empty = full + kStages;
@@ -474,7 +473,7 @@ int run(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, co
                         kStageRowBytes, kTileRows, CU_TENSOR_MAP_SWIZZLE_NONE))
         return -1;
     auto kern = gemv_w4a16_tma_kernel<NT, XSMEM, EVEN_G>;
-    const size_t smem = smem_layout(M, K, 8 * NT, XSMEM).total + 1024;
+    const size_t smem = smem_layout(M, K, XSMEM).total + 1024;
     // launch shape per (device, shared-memory size), computed once
     static std::mutex mu;
     static std::map<std::pair<int, size_t>, int> capacity;
