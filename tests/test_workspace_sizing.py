@@ -1,0 +1,62 @@
+"""The workspace size the library asks for covers every slot its split-K kernels index (CPU only).
+
+The persistent decode kernel (M = 1) and the tensor-core kernel (M > 16) split tiles between CTAs with
+equal contiguous ranges of units (stream-K); each segment of a split tile writes a binary32 partial into
+slot (CTA - first CTA of the tile), and each tile has an arrival counter.  This test models those ranges
+for many shapes, finds the largest number of segments any tile really has, and checks that
+wq_gemm_workspace_bytes (queried without a GPU; the library then assumes a B200's 148 SMs) leaves room for
+all of them.
+"""
+import math
+
+import pytest
+
+import group_wise_weight_b200 as wq
+
+SMS = 148
+
+
+def _m1_needed(N, K):
+    P = K // 256                      # group pairs per 256-row tile
+    ntiles = math.ceil(N / 256)
+    units = ntiles * P
+    B = min(units, SMS)
+    cta_of = lambda u: ((u + 1) * B - 1) // units  # noqa: E731
+    for b in (0, B // 2, B - 1):      # the formula agrees with the ranges [units b / B, units (b+1) / B)
+        lo, hi = units * b // B, units * (b + 1) // B
+        assert all(cta_of(u) == b for u in range(lo, hi))
+    max_seg = max(cta_of(t * P + P - 1) - cta_of(t * P) + 1 for t in range(ntiles))
+    return ntiles * max_seg * 256 * 4 + ntiles * 4
+
+
+def _tc_needed(M, N, K, g):
+    BN = min(32 if M <= 32 else (64 if M <= 64 else 128), g)
+    tiles = math.ceil(N / 128) * math.ceil(M / BN)
+    spt = K // 128
+    total = tiles * spt
+    grid = max(1, min(total, SMS))
+    per, extra = total // grid, total % grid
+    big = extra * (per + 1)
+    cta_of = lambda u: u // (per + 1) if u < big else extra + (u - big) // per  # noqa: E731
+    max_seg = max(cta_of(t * spt + spt - 1) - cta_of(t * spt) + 1 for t in range(tiles))
+    return tiles * max_seg * BN * 128 * 4 + tiles * 4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    wq.lib()
+
+
+@pytest.mark.parametrize("N,K", [(1, 1024), (33, 1024), (31, 3072), (64, 32768), (4097, 2048), (3000, 4096),
+                                 (8192, 8192), (10240, 8192), (57344, 8192), (8192, 28672), (14336, 4096),
+                                 (256 * 148, 1024), (256 * 149 + 1, 2048), (300000, 1024)])
+def test_m1_workspace_covers_every_segment(N, K):
+    assert wq.wq_gemm_workspace_bytes(1, N, K, 128, 4) >= _m1_needed(N, K)
+
+
+@pytest.mark.parametrize("M,N,K,g", [(17, 128, 128, 32), (32, 256, 256, 64), (40, 384, 8192, 128),
+                                     (64, 384, 1024, 32), (128, 130, 384, 128), (128, 256, 16384, 128),
+                                     (128, 10240, 8192, 128), (128, 57344, 8192, 128), (128, 8192, 28672, 128),
+                                     (200, 512, 640, 128), (256, 128, 128, 32), (129, 4097, 4096, 64)])
+def test_tc_workspace_covers_every_segment(M, N, K, g):
+    assert wq.wq_gemm_workspace_bytes(M, N, K, g, 4) >= _tc_needed(M, N, K, g)
