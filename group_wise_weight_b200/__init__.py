@@ -60,6 +60,8 @@ def lib():
         L.wq_version.restype = I
         L.wq_quantize_int4.argtypes = [P, I, I64, I64, I64, I, P, P, P, P]
         L.wq_quantize_int4.restype = I
+        L.wq_quantize_int4_scaled.argtypes = [P, I, I64, I64, I64, I, P, P, P, P, P]
+        L.wq_quantize_int4_scaled.restype = I
         L.wq_quantize_int4_sym.argtypes = [P, I, I64, I64, I64, I, P, P, P, P]
         L.wq_quantize_int4_sym.restype = I
         L.wq_quantize_int8.argtypes = [P, I, I64, I64, I64, I, P, P, P]
@@ -138,6 +140,31 @@ def wq_quantize_int4(w: torch.Tensor, g: int = 128, qweight=None, scales=None, z
         _dense(t, n)
     _check(lib().wq_quantize_int4(_dev(w, "w"), wtype, N, K, w.stride(0), int(g), _dev(qweight, "qweight"),
                                   _dev(scales, "scales"), _dev(zeros, "zeros"), _stream_handle(stream)))
+    return qweight, scales, zeros
+
+
+def wq_quantize_int4_scaled(w: torch.Tensor, col_scale: torch.Tensor, g: int = 128, qweight=None, scales=None,
+                            zeros=None, stream=None):
+    """wq_quantize_int4 of w[n][k] * col_scale[k] (binary32 products): the weight side of an activation-aware
+    per-input-channel scaling.  col_scale: float32 [K] on CUDA.  Returns (qweight, scales, zeros)."""
+    if w.dim() != 2 or w.stride(1) != 1:
+        raise ValueError("w must be a 2-D tensor with unit stride along K")
+    wtype = {torch.float32: WQ_F32, torch.bfloat16: WQ_BF16}.get(w.dtype)
+    if wtype is None:
+        raise TypeError("w must be float32 or bfloat16")
+    N, K = w.shape
+    if col_scale.dtype != torch.float32 or col_scale.numel() != K:
+        raise TypeError("col_scale must be a float32 tensor of K values")
+    _dense(col_scale, "col_scale")
+    dev = w.device
+    qweight = torch.empty((N, K // 2), dtype=torch.uint8, device=dev) if qweight is None else qweight
+    scales = torch.empty((N, K // g), dtype=torch.bfloat16, device=dev) if scales is None else scales
+    zeros = torch.empty((N, K // g), dtype=torch.bfloat16, device=dev) if zeros is None else zeros
+    for t, n in ((qweight, "qweight"), (scales, "scales"), (zeros, "zeros")):
+        _dense(t, n)
+    _check(lib().wq_quantize_int4_scaled(_dev(w, "w"), wtype, N, K, w.stride(0), int(g), _dev(col_scale, "col_scale"),
+                                         _dev(qweight, "qweight"), _dev(scales, "scales"), _dev(zeros, "zeros"),
+                                         _stream_handle(stream)))
     return qweight, scales, zeros
 
 

@@ -144,6 +144,20 @@ int wq_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw
     return check_launch("wq_quantize_int4");
 }
 
+int wq_quantize_int4_scaled(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g,
+                            const float *col_scale, uint8_t *qweight, uint16_t *scales, uint16_t *zeros,
+                            void *stream)
+{
+    g_last_error.clear();
+    int rc = check_quantize("wq_quantize_int4_scaled", w, wtype, N, K, ldw, g, qweight, scales, zeros, false);
+    if (rc != WQ_OK) return rc;
+    if (!col_scale) return fail(WQ_ERR_ARG, "wq_quantize_int4_scaled: null col_scale");
+    if (!aligned16(col_scale)) return fail(WQ_ERR_ALIGN, "wq_quantize_int4_scaled: col_scale must be 16-byte aligned");
+    wq::launch_quantize_int4_scaled(w, wtype, N, K, ldw, g, col_scale, qweight, scales, zeros,
+                                    static_cast<cudaStream_t>(stream));
+    return check_launch("wq_quantize_int4_scaled");
+}
+
 int wq_quantize_int4_sym(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *qweight,
                          uint16_t *scales, uint16_t *zeros, void *stream)
 {

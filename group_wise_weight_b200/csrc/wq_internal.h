@@ -9,6 +9,8 @@ namespace wq {
 // Quantisers (wq_quant.cu).  Arguments are validated by the caller.
 void launch_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *q,
                           uint16_t *s, uint16_t *z, cudaStream_t st);
+void launch_quantize_int4_scaled(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g,
+                                 const float *col_scale, uint8_t *q, uint16_t *s, uint16_t *z, cudaStream_t st);
 void launch_quantize_int4_sym(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *q,
                               uint16_t *s, uint16_t *z, cudaStream_t st);
 void launch_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, int8_t *q,

@@ -153,11 +153,14 @@ __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b)
     return d;
 }
 
-template <typename T, int LPG>
+// SCALED: quantise w[n][k] * col_scale[k] (each product rounded to binary32), the weights an
+// activation-aware per-input-channel scaling hands the quantiser ("Quantization Methods Compared",
+// section "The methods compared": AWQ scales the salient channels up before quantising).
+template <typename T, int LPG, bool SCALED>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
                   uint8_t *__restrict__ qweight, uint16_t *__restrict__ scales,
-                  uint16_t *__restrict__ zeros)
+                  uint16_t *__restrict__ zeros, const float *__restrict__ col_scale)
 {
     constexpr int g = LPG * 8;
     const int lane = threadIdx.x & 31;
@@ -167,7 +170,8 @@ quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
     const int64_t tasks = N * chunks;
     const int64_t G = K / g;
 
-    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    // packed bf16 min/max only for unscaled bf16 weights (scaled products are binary32 values)
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value && !SCALED;
     TaskWalk walk(warp0, n_warps, chunks);
     for (int64_t t0 = warp0; t0 < tasks; t0 += n_warps * kQuantUnroll) {
         float v[kQuantUnroll][8];
@@ -184,6 +188,12 @@ quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
                 if (active[u]) raw[u] = ld_stream_v4(w + n[u] * ldw + k0[u]);
             } else if (active[u]) {
                 load8<T>(w + n[u] * ldw + k0[u], v[u]);
+                if (SCALED) {
+                    float c[8];
+                    load8<float>(col_scale + k0[u], c);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[u][i] = __fmul_rn(v[u][i], c[i]);
+                }
             }
             walk.step();
         }
@@ -472,14 +482,14 @@ int persistent_grid(KernelT kernel, int64_t tasks_in_warps)
     return (int)(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
-template <typename T, int LPG>
+template <typename T, int LPG, bool SCALED>
 void launch_int4(const void *w, int64_t N, int64_t K, int64_t ldw, uint8_t *q, uint16_t *s, uint16_t *z,
-                 cudaStream_t st)
+                 const float *cs, cudaStream_t st)
 {
-    auto k = quant_int4_kernel<T, LPG>;
+    auto k = quant_int4_kernel<T, LPG, SCALED>;
     const int64_t tasks = N * ((K + 255) / 256);
     const int grid = persistent_grid(k, tasks);
-    k<<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(w), N, K, ldw, q, s, z);
+    k<<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(w), N, K, ldw, q, s, z, cs);
 }
 
 template <typename T, int LPG>
@@ -491,14 +501,14 @@ void launch_int8(const void *w, int64_t N, int64_t K, int64_t ldw, int8_t *q, ui
     k<<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(w), N, K, ldw, q, s);
 }
 
-template <typename T>
+template <typename T, bool SCALED>
 void dispatch_int4(const void *w, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *q, uint16_t *s,
-                   uint16_t *z, cudaStream_t st)
+                   uint16_t *z, const float *cs, cudaStream_t st)
 {
     switch (g) {
-    case 32: launch_int4<T, 4>(w, N, K, ldw, q, s, z, st); break;
-    case 64: launch_int4<T, 8>(w, N, K, ldw, q, s, z, st); break;
-    default: launch_int4<T, 16>(w, N, K, ldw, q, s, z, st); break;
+    case 32: launch_int4<T, 4, SCALED>(w, N, K, ldw, q, s, z, cs, st); break;
+    case 64: launch_int4<T, 8, SCALED>(w, N, K, ldw, q, s, z, cs, st); break;
+    default: launch_int4<T, 16, SCALED>(w, N, K, ldw, q, s, z, cs, st); break;
     }
 }
 
@@ -543,8 +553,15 @@ void dispatch_int8(const void *w, int64_t N, int64_t K, int64_t ldw, int g, int8
 void launch_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *q,
                           uint16_t *s, uint16_t *z, cudaStream_t st)
 {
-    if (wtype == WQ_F32) dispatch_int4<float>(w, N, K, ldw, g, q, s, z, st);
-    else dispatch_int4<__nv_bfloat16>(w, N, K, ldw, g, q, s, z, st);
+    if (wtype == WQ_F32) dispatch_int4<float, false>(w, N, K, ldw, g, q, s, z, nullptr, st);
+    else dispatch_int4<__nv_bfloat16, false>(w, N, K, ldw, g, q, s, z, nullptr, st);
+}
+
+void launch_quantize_int4_scaled(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g,
+                                 const float *col_scale, uint8_t *q, uint16_t *s, uint16_t *z, cudaStream_t st)
+{
+    if (wtype == WQ_F32) dispatch_int4<float, true>(w, N, K, ldw, g, q, s, z, col_scale, st);
+    else dispatch_int4<__nv_bfloat16, true>(w, N, K, ldw, g, q, s, z, col_scale, st);
 }
 
 void launch_quantize_int4_sym(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *q,

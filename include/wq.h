@@ -97,6 +97,22 @@ int wq_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw
                      uint8_t *qweight, uint16_t *scales, uint16_t *zeros, void *stream);
 
 /*
+ * Asymmetric INT4 quantisation of column-scaled weights: exactly
+ * wq_quantize_int4 applied to w[n][k] * col_scale[k], each product rounded
+ * to binary32 -- the weights an activation-aware per-input-channel scaling
+ * hands the quantiser ([P3] "The methods compared": AWQ scales the salient
+ * channels up before quantising; the activations are divided by the same
+ * scales, so the product is unchanged up to the quantisation).
+ *
+ *   col_scale  [K] binary32, device, 16-byte aligned; other arguments as
+ *              wq_quantize_int4
+ * Requirements: as wq_quantize_int4; col_scale non-NULL.
+ */
+int wq_quantize_int4_scaled(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g,
+                            const float *col_scale, uint8_t *qweight, uint16_t *scales, uint16_t *zeros,
+                            void *stream);
+
+/*
  * Symmetric INT4 quantisation, one scale per group of g consecutive weights,
  * levels -7..7  ([P1C] "The error of quantising an outlier with the wrong
  * scale"; [P3] "The methods compared").  The output is the asymmetric INT4

@@ -72,6 +72,19 @@ def test_quantize_int4_rejects(L, kw, code):
     assert wq.wq_last_error() != ""
 
 
+def _q4c(L, w=A, wt=wq.WQ_BF16, N=4, K=256, ldw=256, g=128, c=A, q=A, s=A, z=A):
+    return L.wq_quantize_int4_scaled(w, wt, N, K, ldw, g, c, q, s, z, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(c=None), wq.WQ_ERR_ARG), (dict(c=MIS), wq.WQ_ERR_ALIGN), (dict(w=None), wq.WQ_ERR_ARG),
+    (dict(g=16), wq.WQ_ERR_UNSUPPORTED), (dict(K=96, ldw=96), wq.WQ_ERR_SHAPE),
+])
+def test_quantize_int4_scaled_rejects(L, kw, code):
+    assert _q4c(L, **kw) == code
+    assert wq.wq_last_error() != ""
+
+
 def _q4s(L, w=A, wt=wq.WQ_BF16, N=4, K=256, ldw=256, g=128, q=A, s=A, z=A):
     return L.wq_quantize_int4_sym(w, wt, N, K, ldw, g, q, s, z, None)
 

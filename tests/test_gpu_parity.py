@@ -192,6 +192,23 @@ def test_quantize_extreme_magnitudes(dtype):
     assert np.array_equal(q8.cpu().numpy(), c8) and np.array_equal(bits(s8), s8b)
 
 
+@pytest.mark.parametrize("g", [32, 128])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_int4_column_scaled(g, dtype):
+    """The weight side of activation-aware scaling: the codes of w[n][k] * s_k are those the oracle gets
+    for the same binary32 products, bit for bit; scales from activations with salient channels."""
+    from oracle import awq
+    N, K = 200, 1024
+    w = wq_inputs.llm_weight(N, K, 150 + g, dtype=torch.float32).to(dtype)
+    x_cal = wq_inputs.activations(32, K, 151, channel_seed=150 + g).double().numpy()
+    sc = awq.channel_scales(awq.channel_magnitude(x_cal), 0.5)
+    q, s, z = wq.wq_quantize_int4_scaled(w.cuda(), torch.from_numpy(sc).cuda(), g)
+    torch.cuda.synchronize()
+    codes, so, zo = oracle.quantize_int4(awq.scaled_weights(w_f32(w), sc), g)
+    assert np.array_equal(q.cpu().numpy(), oracle.pack_int4(codes))
+    assert np.array_equal(bits(s), oracle.bf16_bits(so)) and np.array_equal(bits(z), oracle.bf16_bits(zo))
+
+
 def check_q4_sym(w: torch.Tensor, g: int):
     q, s, z = wq.wq_quantize_int4_sym(w.cuda(), g)
     torch.cuda.synchronize()
