@@ -30,6 +30,21 @@ int fail(int status, const char *fmt, ...)
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// a * b * c bytes, saturating (the ranges compared below never wrap)
+uint64_t span(int64_t a, int64_t b, int64_t c)
+{
+    const unsigned __int128 v = (unsigned __int128)(uint64_t)a * (uint64_t)b * (uint64_t)c;
+    return v > (unsigned __int128)UINT64_MAX ? UINT64_MAX : (uint64_t)v;
+}
+
+// [a, a + an) and [b, b + bn) share a byte
+bool overlap(const void *a, uint64_t an, const void *b, uint64_t bn)
+{
+    if (!a || !b || an == 0 || bn == 0) return false;
+    const unsigned __int128 a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + bn && b0 < a0 + an;
+}
+
 int check_launch(const char *what)
 {
     const cudaError_t e = cudaGetLastError();
@@ -52,6 +67,12 @@ int check_quantize(const char *what, const void *w, int wtype, int64_t N, int64_
     if (N > 0x7fffffffLL) return fail(WQ_ERR_SHAPE, "%s: N too large", what);
     if (ldw % 8 != 0 || !aligned16(w) || !aligned16(q) || !aligned16(s) || (z && !aligned16(z)))
         return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned and ldw a multiple of 8", what);
+    // the outputs must not overlap the weights or one another
+    const uint64_t wb = span(N - 1, ldw, wtype == WQ_F32 ? 4 : 2) + span(1, K, wtype == WQ_F32 ? 4 : 2);
+    const uint64_t qb = span(N, K, 1) / (int8 ? 1 : 2), pb = span(N, K / g, 2);
+    if (overlap(q, qb, w, wb) || overlap(s, pb, w, wb) || overlap(z, pb, w, wb) || overlap(q, qb, s, pb) ||
+        overlap(q, qb, z, pb) || overlap(s, pb, z, pb))
+        return fail(WQ_ERR_ARG, "%s: output buffers overlap the weights or each other", what);
     return WQ_OK;
 }
 
@@ -67,6 +88,8 @@ int check_gemm(const char *what, const void *x, int64_t M, int64_t N, int64_t K,
     if (N > 0x7fffffffLL * 8 || M > 0x7fffffffLL) return fail(WQ_ERR_SHAPE, "%s: M or N too large", what);
     if (!aligned16(x) || !aligned16(q) || !aligned16(s) || (z && !aligned16(z)) || !aligned16(y))
         return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned", what);
+    if (wq::output_overlaps_inputs(x, M, N, K, q, s, z, g, y, int8))
+        return fail(WQ_ERR_ARG, "%s: y overlaps x, the codes, the scales or the zero-points", what);
     return WQ_OK;
 }
 
@@ -98,6 +121,14 @@ int *status_word()
 }  // namespace
 
 namespace wq {
+
+bool output_overlaps_inputs(const void *x, int64_t M, int64_t N, int64_t K, const void *q, const void *s,
+                            const void *z, int g, const void *y, bool int8)
+{
+    const uint64_t yb = span(M, N, 2), xb = span(M, K, 2);
+    const uint64_t qb = span(N, K, 1) / (int8 ? 1 : 2), pb = span(N, K / g, 2);
+    return overlap(y, yb, x, xb) || overlap(y, yb, q, qb) || overlap(y, yb, s, pb) || overlap(y, yb, z, pb);
+}
 
 // Record `msg` as this thread's last error and return `status` (for entry points in other files).
 int record_error(int status, const char *msg)

@@ -6,6 +6,10 @@
 
 namespace wq {
 
+// y [M][N] bf16 overlaps x [M][K] bf16, the codes, the scales or the zero-points (wq_api.cu).
+bool output_overlaps_inputs(const void *x, int64_t M, int64_t N, int64_t K, const void *q, const void *s,
+                            const void *z, int g, const void *y, bool int8);
+
 // Quantisers (wq_quant.cu).  Arguments are validated by the caller.
 void launch_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g, uint8_t *q,
                           uint16_t *s, uint16_t *z, cudaStream_t st);

@@ -69,6 +69,8 @@ extern "C" int wq_gemm_w4a16_noalloc(const uint16_t *x, int64_t M, int64_t N, in
     if (K % 128 != 0) return wq::record_error(WQ_ERR_SHAPE, "wq_gemm_w4a16_noalloc: K % 128 != 0");
     if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y))
         return wq::record_error(WQ_ERR_ALIGN, "wq_gemm_w4a16_noalloc: pointers must be 16-byte aligned");
+    if (wq::output_overlaps_inputs(x, M, N, K, qweight, scales, zeros, g, y, false))
+        return wq::record_error(WQ_ERR_ARG, "wq_gemm_w4a16_noalloc: y overlaps x, the codes, the scales or the zero-points");
     const size_t need = wq::gemv_tma_workspace_bytes(M, N, K, g);
     if (need > kScratchBytes) {
         char msg[256];

@@ -91,7 +91,8 @@ int wq_version(void);
  *   z  = bf16(round(-mn / s) + 0)             (+0 turns -0 into +0)
  *   q  = clip(round(w / s + z), 0, 15)        with the stored s and z
  * Requirements: N >= 1; K >= 32, K % 32 == 0; g in {32, 64, 128}, K % g == 0;
- * ldw >= K, ldw % 8 == 0; all pointers 16-byte aligned.
+ * ldw >= K, ldw % 8 == 0; all pointers 16-byte aligned; the outputs must not
+ * overlap w or one another (WQ_ERR_ARG otherwise).
  */
 int wq_quantize_int4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int g,
                      uint8_t *qweight, uint16_t *scales, uint16_t *zeros, void *stream);
@@ -186,7 +187,8 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * CUDA-core kernel.
  * Requirements: M, N >= 1; K % 32 == 0; g in {32, 64, 128}, K % g == 0;
  * pointers 16-byte aligned; workspace of wq_gemm_workspace_bytes(M, N, K, g, 4)
- * bytes (may be NULL when that is 0).  x and y must not overlap.
+ * bytes (may be NULL when that is 0).  y must not overlap x, qweight,
+ * scales or zeros (WQ_ERR_ARG otherwise).
  */
 int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *qweight,
                   const uint16_t *scales, const uint16_t *zeros, int g, uint16_t *y,

@@ -72,7 +72,7 @@ def test_quantize_int4_rejects(L, kw, code):
     assert wq.wq_last_error() != ""
 
 
-def _q4c(L, w=A, wt=wq.WQ_BF16, N=4, K=256, ldw=256, g=128, c=A, q=A, s=A, z=A):
+def _q4c(L, w=A, wt=wq.WQ_BF16, N=4, K=256, ldw=256, g=128, c=A, q=A + (1 << 16), s=A + (2 << 16), z=A + (3 << 16)):
     return L.wq_quantize_int4_scaled(w, wt, N, K, ldw, g, c, q, s, z, None)
 
 
@@ -139,3 +139,32 @@ def test_python_binding_refuses_cpu_tensors(L):
     with pytest.raises(TypeError):
         wq.wq_gemm_w4a16(torch.zeros(1, 256, dtype=torch.bfloat16), torch.zeros(4, 128, dtype=torch.uint8),
                          torch.zeros(4, 2, dtype=torch.bfloat16), torch.zeros(4, 2, dtype=torch.bfloat16), 128)
+
+
+# Distinct fake buffers, 16 MB apart (never dereferenced: validation must decide first).
+def _bufs(n):
+    return [(1 << 30) + i * (1 << 24) for i in range(n)]
+
+
+def test_gemm_rejects_output_overlapping_an_input(L):
+    x, q, s, z, y = _bufs(5)
+    M, N, K = 1, 1024, 1024
+    # distinct buffers get past the argument checks (here to the missing workspace of the M = 1 kernel)
+    assert _g4(L, x=x, M=M, N=N, K=K, q=q, s=s, z=z, y=y) == wq.WQ_ERR_WORKSPACE
+    for kw in (dict(y=x + 16), dict(y=q + 512), dict(y=s), dict(y=z - 16 * 16)):
+        args = dict(x=x, M=M, N=N, K=K, q=q, s=s, z=z, y=y)
+        args.update(kw)
+        assert _g4(L, **args) == wq.WQ_ERR_ARG, kw
+        assert "overlaps" in wq.wq_last_error()
+    assert _g8(L, x=x, M=M, N=N, K=K, q=q, s=s, y=q + N * K - 16) == wq.WQ_ERR_ARG
+
+
+def test_quantize_rejects_outputs_overlapping(L):
+    w, q, s, z = _bufs(4)
+    N, K = 64, 1024
+    for kw in (dict(q=w + 16), dict(s=w + (N - 1) * K * 2), dict(z=s), dict(z=q + 16)):
+        args = dict(w=w, N=N, K=K, ldw=K, q=q, s=s, z=z)
+        args.update(kw)
+        assert _q4(L, **args) == wq.WQ_ERR_ARG, kw
+        assert "overlap" in wq.wq_last_error()
+    assert _q8(L, w=w, N=N, K=K, ldw=K, q=w + N * K * 2 - 16, s=s) == wq.WQ_ERR_ARG
