@@ -26,3 +26,29 @@ def model_gigabytes(n_params: float, b: int, g: int, scale_bits: int = 16, zero_
 def example_bytes(n_weights: int, b: int, scale_bits: int, zero_bits: int) -> float:
     """Bytes for one group of n_weights codes plus one scale and one zero-point."""
     return (n_weights * b + scale_bits + zero_bits) / 8
+
+
+# ---------------------------------------------------------------------------
+# KV cache (the NEXT row on KV-cache quantisation)
+#   * "Quantization for LLM inference: FP8, INT4 (GPTQ, AWQ) and GGUF" -- "KV cache quantization": a bf16
+#     cache holds 2 bytes per dimension x heads x head_dim x 2 (K and V); fp8 holds 1 byte; int4 with
+#     blocks of 128 holds half a byte plus the scale overhead and divides the cache by about 3.5.
+#   * "Quantization Methods Compared ..." -- "Hardware, formats and the roofline": the worked decode step
+#     of the 70B model at batch 128 and 8,000-token contexts reads 140 GB of fp16 weights against 335.5 GB
+#     of KV cache, so 4-bit weights (about 36 GB) buy only about 1.28x.
+# ---------------------------------------------------------------------------
+
+def kv_cache_bytes(layers: int, kv_heads: int, head_dim: int, tokens: int, batch: int,
+                   bytes_per_element: float) -> float:
+    """K and V of every layer, head and dimension for tokens x batch positions."""
+    return 2 * layers * kv_heads * head_dim * tokens * batch * bytes_per_element
+
+
+def block_bytes_per_element(bits: int, block: int, param_bits: int) -> float:
+    """Bytes per cached element when every block of `block` values carries param_bits of parameters."""
+    return bits / 8 + param_bits / 8 / block
+
+
+def decode_step_speedup(weight_bytes_before: float, weight_bytes_after: float, other_bytes: float) -> float:
+    """Memory-bound decode: the step time scales with the bytes read, weights plus everything else."""
+    return (weight_bytes_before + other_bytes) / (weight_bytes_after + other_bytes)

@@ -491,3 +491,33 @@ def test_sym_int4_special_groups_and_asymmetric_decode():
         assert s[2, 0] == 1.0 and q[2].tolist() == [7, 0, 2, 2, 0, -2, -2, 4]
         z = np.full(s.shape, 8.0, dtype=np.float32)
         assert np.array_equal(oracle.dequant_int4(codes, s, z, 8), q * np.repeat(s.astype(np.float64), 8, axis=1))
+
+
+# --------------------------------------------------------------------------
+# KV-cache accounting (groundwork for the KV-cache row)
+# --------------------------------------------------------------------------
+
+def test_kv_cache_worked_decode_step():
+    from oracle.accounting import kv_cache_bytes, decode_step_speedup
+    sc, _ = read("kv_cache_accounting.txt")
+    g = lambda k: scalar(sc, k)  # noqa: E731
+    kv = kv_cache_bytes(int(g("layers")), int(g("kv_heads")), int(g("head_dim")), int(g("tokens")),
+                        int(g("batch")), 2)
+    assert round(kv / 1e9, 1) == g("kv_gb_printed")
+    gain = decode_step_speedup(g("weights_fp16_gb_printed") * 1e9, g("weights_int4_gb_printed") * 1e9, kv)
+    assert round(gain, 2) == g("int4_gain_printed")
+    # the KV bytes dwarf the weights at this batch and context
+    assert kv > 2 * g("weights_fp16_gb_printed") * 1e9
+
+
+def test_kv_cache_formats():
+    from oracle.accounting import kv_cache_bytes, block_bytes_per_element
+    sc, _ = read("kv_cache_accounting.txt")
+    bf16 = kv_cache_bytes(80, 8, 128, 1000, 1, 2)
+    assert bf16 / kv_cache_bytes(80, 8, 128, 1000, 1, 1) == scalar(sc, "fp8_kv_factor_printed")
+    block = int(scalar(sc, "int4_kv_block"))
+    # "about 3.5": 16- or 32-bit scales (with or without a zero-point) per block of 128 give 3.56 to 3.88
+    factors = [2 / block_bytes_per_element(4, block, p) for p in (16, 32, 64)]
+    assert all(3.5 <= f <= 3.9 for f in factors)
+    assert min(abs(f - scalar(sc, "int4_kv_factor_printed")) for f in factors) < 0.1
+    assert block_bytes_per_element(4, block, 0) == 0.5
