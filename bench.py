@@ -204,6 +204,15 @@ class Clocks:
 # the model
 # ---------------------------------------------------------------------------
 
+def workload_config(layers: int) -> dict:
+    """The workload both arms report (the 70B-shaped decode step at M = 1)."""
+    shapes = [(K, N) for _ in range(layers) for _, K, N in wq_inputs.FULL70B_LINEARS]
+    return {"workload": f"full70b decode step: {layers} layers x (qkv 8192->10240, o 8192->8192, "
+                        "gate+up 8192->57344, down 28672->8192), W4A16 g128 bf16 s/z, M=1",
+            "layers": layers, "linears_per_step": len(shapes), "weights": sum(K * N for K, N in shapes),
+            "bytes_per_step": sum(linear_bytes(1, N, K) for K, N in shapes)}
+
+
 def linear_bytes(M, N, K, g=G):
     """Algorithmic bytes of one W4A16 call: packed codes, bf16 s and z, bf16 x and y."""
     return N * K // 2 + 2 * 2 * N * (K // g) + 2 * M * K + 2 * M * N
@@ -431,7 +440,7 @@ def run_reference(args, world, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": "full70b decode step, W4A16 g128, M=1 (bounded CPU sample per step)"},
+            "config": dict(workload_config(args.layers), sample="bounded CPU sample of the step per timed step"),
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": desc + " per step"},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -39,3 +39,21 @@ def test_clock_summary_flags_throttle_reasons():
     assert s["samples"] == 2  # the idle sample (power <= 200 W) is not under load
     assert s["reasons"] == ["sw_power_cap"]
     assert s["sm_max_mhz"] == 1965.0
+
+
+def test_workload_config_counts_the_model():
+    c = bench.workload_config(80)
+    assert c["linears_per_step"] == 320 and c["layers"] == 80
+    assert c["weights"] == 80 * (8192 * 10240 + 8192 * 8192 + 8192 * 57344 + 28672 * 8192)
+    assert c["bytes_per_step"] == 80 * sum(bench.linear_bytes(1, N, K) for K, N in
+                                           ((8192, 10240), (8192, 8192), (8192, 57344), (28672, 8192)))
+
+
+def test_both_arms_describe_the_same_workload():
+    """The reference arm's config is workload_config; the GPU arm spells the same keys out in its line."""
+    import inspect
+    src = inspect.getsource(bench.main)
+    c = bench.workload_config(80)
+    for key in c:
+        assert f'"{key}"' in src, key
+    assert "W4A16 g128 bf16 s/z, M=1" in c["workload"] and "W4A16 g128 bf16 s/z, M=1" in src
