@@ -150,7 +150,7 @@ const char *wq_status_str(int status)
 {
     switch (status) {
     case WQ_OK: return "WQ_OK";
-    case WQ_ERR_ARG: return "WQ_ERR_ARG: null pointer or non-positive size";
+    case WQ_ERR_ARG: return "WQ_ERR_ARG: null pointer, non-positive size or overlapping buffers";
     case WQ_ERR_SHAPE: return "WQ_ERR_SHAPE: K, g or ldw do not fit the layout";
     case WQ_ERR_ALIGN: return "WQ_ERR_ALIGN: pointer or leading dimension misaligned";
     case WQ_ERR_UNSUPPORTED: return "WQ_ERR_UNSUPPORTED: group size or dtype not supported";

@@ -54,7 +54,7 @@ extern "C" {
 #endif
 
 #define WQ_OK 0
-#define WQ_ERR_ARG (-1)            /* null pointer, or a size <= 0                      */
+#define WQ_ERR_ARG (-1)            /* null pointer, a size <= 0, or an output overlapping an input */
 #define WQ_ERR_SHAPE (-2)          /* K not a multiple of 32, g does not divide K, ldw < K */
 #define WQ_ERR_ALIGN (-3)          /* a pointer not 16-byte aligned, or ldw % 8 != 0      */
 #define WQ_ERR_UNSUPPORTED (-4)    /* group size or dtype outside the supported set       */
