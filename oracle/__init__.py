@@ -61,6 +61,14 @@ def _bind(path: str):
     lib.oracle_quantize_int4.argtypes = [P, I64, I64, I64, I64, I, P, P, P]
     lib.oracle_quantize_int8.argtypes = [P, I64, I64, I64, I64, I, P, P]
     lib.oracle_quantize_int4_sym.argtypes = [P, I64, I64, I64, I64, I, P, P]
+    lib.oracle_fp8_decode.argtypes = [ctypes.c_uint8, I]
+    lib.oracle_fp8_decode.restype = ctypes.c_double
+    lib.oracle_fp8_encode.argtypes = [ctypes.c_float, I]
+    lib.oracle_fp8_encode.restype = ctypes.c_uint8
+    lib.oracle_fp8_max.argtypes = [I]
+    lib.oracle_fp8_max.restype = ctypes.c_double
+    lib.oracle_quantize_fp8_rows.argtypes = [P, I64, I64, I64, I, P, P]
+    lib.oracle_dequant_fp8_rows.argtypes = [P, P, I64, I64, I, P]
     lib.oracle_pack_int4.argtypes = [P, I64, I64, P]
     lib.oracle_unpack_int4.argtypes = [P, I64, I64, P]
     lib.oracle_dequant_int4.argtypes = [P, P, P, I64, I64, I64, P]
@@ -161,6 +169,42 @@ def quantize_int4_sym(w, g: int, mode: int = STORED):
     _check(_load().oracle_quantize_int4_sym(_ptr(w), N, K, K, g, mode, _ptr(codes), _ptr(s)),
            "quantize_int4_sym")
     return codes, s
+
+
+E4M3 = 0  # FP8 formats
+E5M2 = 1
+
+
+def fp8_decode(code: int, fmt: int) -> float:
+    return float(_load().oracle_fp8_decode(int(code) & 0xff, fmt))
+
+
+def fp8_encode(v: float, fmt: int) -> int:
+    return int(_load().oracle_fp8_encode(float(v), fmt))
+
+
+def fp8_max(fmt: int) -> float:
+    return float(_load().oracle_fp8_max(fmt))
+
+
+def quantize_fp8_rows(w, fmt: int = E4M3):
+    """FP8 per output channel: s = max|w| / max_fmt per row, codes = nearest FP8 of w / s.
+    Returns (codes uint8 [N][K], s float32 [N])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.empty((N, K), dtype=np.uint8)
+    s = np.empty(N, dtype=np.float32)
+    _check(_load().oracle_quantize_fp8_rows(_ptr(w), N, K, K, fmt, _ptr(codes), _ptr(s)), "quantize_fp8_rows")
+    return codes, s
+
+
+def dequant_fp8_rows(codes, s, fmt: int = E4M3) -> np.ndarray:
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    N, K = c.shape
+    out = np.empty((N, K), dtype=np.float64)
+    _check(_load().oracle_dequant_fp8_rows(_ptr(c), _ptr(s), N, K, fmt, _ptr(out)), "dequant_fp8_rows")
+    return out
 
 
 def pack_int4(codes) -> np.ndarray:

@@ -308,3 +308,90 @@ int oracle_matmul(const double *x, const double *w_hat, int64_t M, int64_t N, in
     }
     return 0;
 }
+
+/* ---------------------------------------------------------------------- */
+/* FP8 (groundwork for the FP8 W8A8 row).                                   */
+/* "Quantization for LLM inference: FP8, INT4 (GPTQ, AWQ) and GGUF",        */
+/* section "FP8: the Hopper/Blackwell datacenter format": E4M3 has 4        */
+/* exponent and 3 mantissa bits, range +-448; E5M2 has 5 and 2, range       */
+/* +-57,344.  Reading: binary formats with exponent bias 2^(e-1) - 1 and    */
+/* subnormals.  E4M3 keeps finite values in its all-ones exponent (448 is   */
+/* 1.75 * 2^8) and only the all-ones pattern is NaN; E5M2 keeps the         */
+/* all-ones exponent for infinities and NaN (57,344 = 1.75 * 2^15).         */
+/* Encoding rounds to the nearest value, ties to the even code, and         */
+/* saturates finite values beyond the range to +-max.                       */
+/* fmt 0 = E4M3, fmt 1 = E5M2.                                              */
+/* ---------------------------------------------------------------------- */
+
+/* The value of an FP8 code; NaN for NaN codes, +-inf for E5M2 infinities. */
+double oracle_fp8_decode(uint8_t code, int fmt)
+{
+    const int ebits = fmt == 0 ? 4 : 5, mbits = fmt == 0 ? 3 : 2;
+    const int bias = (1 << (ebits - 1)) - 1;
+    const int sign = code >> 7;
+    const int e = (code >> mbits) & ((1 << ebits) - 1);
+    const int m = code & ((1 << mbits) - 1);
+    double v;
+    if (fmt == 0 && e == 15 && m == 7) return NAN;
+    if (fmt == 1 && e == 31) v = m == 0 ? INFINITY : NAN;
+    else if (e == 0) v = ldexp((double)m, 1 - bias - mbits);
+    else v = ldexp(1.0 + (double)m / (double)(1 << mbits), e - bias);
+    return sign ? -v : v;
+}
+
+/* Largest finite value of the format. */
+double oracle_fp8_max(int fmt) { return fmt == 0 ? 448.0 : 57344.0; }
+
+/* Nearest finite FP8 code to v (ties to the even code), saturating beyond +-max; NaN for non-finite v.
+ * Plain exhaustive search over the codes of v's sign. */
+uint8_t oracle_fp8_encode(float v, int fmt)
+{
+    const uint8_t nan_code = fmt == 0 ? 0x7f : 0x7f;
+    if (!isfinite(v)) return nan_code;
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a > oracle_fp8_max(fmt)) a = oracle_fp8_max(fmt);
+    int best = -1;
+    double best_d = 0.0;
+    for (int c = 0; c < 128; ++c) {
+        const double cv = oracle_fp8_decode((uint8_t)c, fmt);
+        if (!isfinite(cv)) continue;
+        const double d = fabs(cv - a);
+        if (best < 0 || d < best_d || (d == best_d && (c & 1) == 0)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* FP8 quantisation, one binary32 scale per row (per output channel):
+ * s = max|w| / max_fmt (1 when the row is all zero), code = encode(w / s). */
+int oracle_quantize_fp8_rows(const float *w, int64_t N, int64_t K, int64_t ldw, int fmt, uint8_t *codes,
+                             float *s_out)
+{
+    if (N <= 0 || K <= 0 || ldw < K || (fmt != 0 && fmt != 1)) return -1;
+    int64_t n;
+#pragma omp parallel for schedule(static)
+    for (n = 0; n < N; ++n) {
+        const float *row = w + n * ldw;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k)
+            if (fabsf(row[k]) > amax) amax = fabsf(row[k]);
+        float s = amax / (float)oracle_fp8_max(fmt);
+        if (s == 0.0f) s = 1.0f;
+        s_out[n] = s;
+        for (int64_t k = 0; k < K; ++k) codes[n * K + k] = oracle_fp8_encode(row[k] / s, fmt);
+    }
+    return 0;
+}
+
+/* w_hat[n][k] = s[n] * value(code) in binary64. */
+int oracle_dequant_fp8_rows(const uint8_t *codes, const float *s, int64_t N, int64_t K, int fmt, double *out)
+{
+    if (N <= 0 || K <= 0) return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            out[n * K + k] = (double)s[n] * oracle_fp8_decode(codes[n * K + k], fmt);
+    return 0;
+}

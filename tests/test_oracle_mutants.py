@@ -37,6 +37,10 @@ MUTANTS = {
     "sym_truncate": ("float q = nearbyintf(wg[i] / s);", "float q = truncf(wg[i] / s);"),
     "sym_ties_away": ("float q = nearbyintf(wg[i] / s);", "float q = roundf(wg[i] / s);"),
     "sym_signed_max": ("const float a = fabsf(wg[i]);", "const float a = wg[i];"),
+    "fp8_bias_off_by_one": ("const int bias = (1 << (ebits - 1)) - 1;", "const int bias = (1 << (ebits - 1));"),
+    "fp8_ties_to_odd": ("(d == best_d && (c & 1) == 0)", "(d == best_d && (c & 1) == 1)"),
+    "fp8_subnormal_exponent": ("ldexp((double)m, 1 - bias - mbits)", "ldexp((double)m, -bias - mbits)"),
+    "fp8_rows_int8_scale": ("amax / (float)oracle_fp8_max(fmt)", "amax / 127.0f"),
 }
 
 PINS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

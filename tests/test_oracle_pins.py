@@ -521,3 +521,82 @@ def test_kv_cache_formats():
     assert all(3.5 <= f <= 3.9 for f in factors)
     assert min(abs(f - scalar(sc, "int4_kv_factor_printed")) for f in factors) < 0.1
     assert block_bytes_per_element(4, block, 0) == 0.5
+
+
+# --------------------------------------------------------------------------
+# FP8 codec and per-channel FP8 quantisation (groundwork for the FP8 W8A8 row):
+# "Quantization for LLM inference ...", "FP8: the Hopper/Blackwell datacenter format"
+# --------------------------------------------------------------------------
+
+def _fp8_values(fmt):
+    vals = {c: oracle.fp8_decode(c, fmt) for c in range(128)}
+    return {c: v for c, v in vals.items() if np.isfinite(v)}
+
+
+@pytest.mark.parametrize("fmt,key", [(oracle.E4M3, "e4m3"), (oracle.E5M2, "e5m2")])
+def test_fp8_ranges_and_structure(fmt, key):
+    sc, _ = read("fp8_formats.txt")
+    vals = _fp8_values(fmt)
+    assert max(vals.values()) == scalar(sc, f"{key}_range_printed") == oracle.fp8_max(fmt)
+    ebits, mbits = int(scalar(sc, f"{key}_exponent_bits")), int(scalar(sc, f"{key}_mantissa_bits"))
+    bias = 2 ** (ebits - 1) - 1
+    assert min(v for v in vals.values() if v > 0) == 2.0 ** (1 - bias - mbits)   # smallest subnormal
+    assert oracle.fp8_decode(1 << mbits, fmt) == 2.0 ** (1 - bias)                # smallest normal
+    # positive codes are ordered like their values, and negative codes mirror them
+    pos = [vals[c] for c in sorted(vals)]
+    assert all(a < b for a, b in zip(pos, pos[1:]))
+    for c in vals:
+        assert oracle.fp8_decode(c | 0x80, fmt) == -vals[c]
+
+
+@pytest.mark.parametrize("fmt", [oracle.E4M3, oracle.E5M2])
+def test_fp8_encode_nearest_ties_even_saturating(fmt):
+    vals = _fp8_values(fmt)
+    codes = sorted(vals)
+    for c in codes:  # exact values round-trip, with either sign
+        assert oracle.fp8_encode(vals[c], fmt) == c
+        if vals[c] != 0:
+            assert oracle.fp8_encode(-vals[c], fmt) == (c | 0x80)
+    for a, b in zip(codes, codes[1:]):  # midpoints go to the even code, neighbours to the nearer value
+        lo, hi = vals[a], vals[b]
+        mid = np.float32((lo + hi) / 2)
+        if float(mid) == (lo + hi) / 2:
+            assert oracle.fp8_encode(mid, fmt) == (a if a % 2 == 0 else b)
+        assert oracle.fp8_encode(np.nextafter(np.float32((lo + hi) / 2), np.float32(0)), fmt) in (a, b)
+        assert oracle.fp8_encode(np.float32(lo + (hi - lo) * 0.25), fmt) == a
+        assert oracle.fp8_encode(np.float32(lo + (hi - lo) * 0.75), fmt) == b
+    top = max(codes)
+    assert oracle.fp8_encode(1e30, fmt) == top and oracle.fp8_encode(-1e30, fmt) == (top | 0x80)
+
+
+@pytest.mark.parametrize("fmt,dtype", [(oracle.E4M3, torch.float8_e4m3fn), (oracle.E5M2, torch.float8_e5m2)])
+def test_fp8_encode_matches_torch(fmt, dtype):
+    """torch's conversion to its FP8 types rounds to nearest even as well (it does not saturate, so only
+    values within range are compared)."""
+    g = torch.Generator().manual_seed(7)
+    v = torch.randn(20000, generator=g) * torch.exp(torch.randn(20000, generator=g) * 3)
+    v = v[v.abs() < oracle.fp8_max(fmt)]
+    want = v.to(dtype).view(torch.uint8).numpy()
+    got = np.array([oracle.fp8_encode(float(x), fmt) for x in v.numpy()], dtype=np.uint8)
+    assert np.array_equal(got, want)
+
+
+def test_fp8_rows_quantisation():
+    w = wq_inputs.llm_weight(64, 256, 501, dtype=torch.float32).numpy()
+    w[3] = 0.0
+    for fmt in (oracle.E4M3, oracle.E5M2):
+        codes, s = oracle.quantize_fp8_rows(w, fmt)
+        assert s[3] == 1.0 and np.all(oracle.dequant_fp8_rows(codes, s, fmt)[3] == 0.0)
+        amax = np.abs(w).max(1)
+        live = amax > 0
+        assert np.allclose(s[live], (amax / oracle.fp8_max(fmt))[live], rtol=1e-7)
+        w_hat = oracle.dequant_fp8_rows(codes, s, fmt)
+        # the largest magnitude of every row lands on +-max; elsewhere the relative error is at most half
+        # an ulp of the mantissa (2^-4 for E4M3, 2^-3 for E5M2) where the value is normal in the format
+        idx = np.abs(w).argmax(1)
+        assert np.allclose(np.abs(w_hat[np.arange(64), idx])[live], amax[live], rtol=1e-6)
+        mbits = 3 if fmt == oracle.E4M3 else 2
+        min_normal = oracle.fp8_decode(1 << mbits, fmt)
+        normal = np.abs(w) / s[:, None] >= min_normal
+        rel = np.abs(w_hat - w)[normal] / np.abs(w)[normal]
+        assert rel.max() <= 2.0 ** -(mbits + 1) * (1 + 1e-6)
