@@ -207,6 +207,23 @@ def dequant_fp8_rows(codes, s, fmt: int = E4M3) -> np.ndarray:
     return out
 
 
+def quantize_fp8_tensor(x, fmt: int = E4M3):
+    """FP8 with one scale for the whole tensor (the pages' dynamic per-tensor scaling of activations):
+    s = max|x| / max_fmt.  Returns (codes uint8, s float32 scalar)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    codes, s = quantize_fp8_rows(x.reshape(1, -1), fmt)
+    return codes.reshape(x.shape), s[0]
+
+
+def gemm_w8a8_fp8(x, w, fmt: int = E4M3):
+    """Reference for an FP8 W8A8 matmul: activations quantised per tensor, weights per output channel, the
+    products of the decoded values summed in binary64.  Returns (y, a) as matmul does."""
+    xc, sx = quantize_fp8_tensor(x, fmt)
+    wc, sw = quantize_fp8_rows(w, fmt)
+    x_hat = dequant_fp8_rows(xc.reshape(1, -1), np.array([sx], dtype=np.float32), fmt).reshape(np.shape(x))
+    return matmul(x_hat, dequant_fp8_rows(wc, sw, fmt))
+
+
 def pack_int4(codes) -> np.ndarray:
     """[N][K] codes -> [N][K/2] bytes, code 2j in the low nibble of byte j."""
     c = np.ascontiguousarray(codes, dtype=np.uint8)

@@ -600,3 +600,17 @@ def test_fp8_rows_quantisation():
         normal = np.abs(w) / s[:, None] >= min_normal
         rel = np.abs(w_hat - w)[normal] / np.abs(w)[normal]
         assert rel.max() <= 2.0 ** -(mbits + 1) * (1 + 1e-6)
+
+
+def test_fp8_w8a8_reference():
+    """The W8A8 reference: the exact product of the decoded operands; close to the unquantised product
+    within the formats' half-ulp (E4M3: 2^-4 relative per operand, so about 2^-3 on sum|x w|)."""
+    x = wq_inputs.plain_activations(4, 256, 503).float().numpy()
+    w = wq_inputs.llm_weight(32, 256, 504, dtype=torch.float32).numpy()
+    y, a = oracle.gemm_w8a8_fp8(x, w)
+    xc, sx = oracle.quantize_fp8_tensor(x)
+    assert xc.shape == x.shape and sx == np.float32(np.abs(x).max() / 448.0)
+    exact = x.astype(np.float64) @ w.astype(np.float64).T
+    bound = np.abs(x).astype(np.float64) @ np.abs(w).astype(np.float64).T
+    assert np.all(np.abs(y - exact) <= 2.0 ** -3 * bound + 1e-12)
+    assert np.all(a <= bound * (1 + 2.0 ** -3))
