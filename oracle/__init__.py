@@ -69,6 +69,12 @@ def _bind(path: str):
     lib.oracle_fp8_max.restype = ctypes.c_double
     lib.oracle_quantize_fp8_rows.argtypes = [P, I64, I64, I64, I, P, P]
     lib.oracle_dequant_fp8_rows.argtypes = [P, P, I64, I64, I, P]
+    lib.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e2m1_decode.restype = ctypes.c_double
+    lib.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+    lib.oracle_e2m1_encode.restype = ctypes.c_uint8
+    lib.oracle_quantize_nvfp4.argtypes = [P, I64, I64, I64, P, P, P]
+    lib.oracle_dequant_nvfp4.argtypes = [P, P, ctypes.c_float, I64, I64, P]
     lib.oracle_pack_int4.argtypes = [P, I64, I64, P]
     lib.oracle_unpack_int4.argtypes = [P, I64, I64, P]
     lib.oracle_dequant_int4.argtypes = [P, P, P, I64, I64, I64, P]
@@ -222,6 +228,35 @@ def gemm_w8a8_fp8(x, w, fmt: int = E4M3):
     wc, sw = quantize_fp8_rows(w, fmt)
     x_hat = dequant_fp8_rows(xc.reshape(1, -1), np.array([sx], dtype=np.float32), fmt).reshape(np.shape(x))
     return matmul(x_hat, dequant_fp8_rows(wc, sw, fmt))
+
+
+def e2m1_decode(code: int) -> float:
+    return float(_load().oracle_e2m1_decode(int(code) & 0xf))
+
+
+def e2m1_encode(v: float) -> int:
+    return int(_load().oracle_e2m1_encode(float(v)))
+
+
+def quantize_nvfp4(w):
+    """NVFP4: E2M1 values, one E4M3 scale per 16 values of a row, one binary32 tensor scale.
+    Returns (codes uint8 [N][K], block_codes uint8 [N][K/16], tensor_scale float)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.empty((N, K), dtype=np.uint8)
+    blocks = np.empty((N, K // 16), dtype=np.uint8)
+    st = np.empty(1, dtype=np.float32)
+    _check(_load().oracle_quantize_nvfp4(_ptr(w), N, K, K, _ptr(codes), _ptr(blocks), _ptr(st)), "quantize_nvfp4")
+    return codes, blocks, float(st[0])
+
+
+def dequant_nvfp4(codes, block_codes, tensor_scale: float) -> np.ndarray:
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    b = np.ascontiguousarray(block_codes, dtype=np.uint8)
+    N, K = c.shape
+    out = np.empty((N, K), dtype=np.float64)
+    _check(_load().oracle_dequant_nvfp4(_ptr(c), _ptr(b), tensor_scale, N, K, _ptr(out)), "dequant_nvfp4")
+    return out
 
 
 def pack_int4(codes) -> np.ndarray:

@@ -395,3 +395,87 @@ int oracle_dequant_fp8_rows(const uint8_t *codes, const float *s, int64_t N, int
             out[n * K + k] = (double)s[n] * oracle_fp8_decode(codes[n * K + k], fmt);
     return 0;
 }
+
+/* ---------------------------------------------------------------------- */
+/* NVFP4 (groundwork for the NVFP4 row).                                    */
+/* "Quantization Methods Compared: INT8, GPTQ, AWQ, FP8, FP4 and KV-Cache   */
+/* Quantization", section "Hardware, formats and the roofline": NVFP4 holds */
+/* 4-bit values with one 8-bit (E4M3) scale per 16 values plus an fp32      */
+/* tensor scale, 4.5 bits per weight; "Quantization for LLM inference ...", */
+/* section "Microscaling: NVFP4 and MXFP4": small blocks (16 or 32 values)  */
+/* with an FP8 scale.  Readings (the pages do not define the 4-bit values   */
+/* or how the scales are chosen): the 4-bit values are E2M1 (sign, 2        */
+/* exponent bits with bias 1, 1 mantissa bit: 0, 0.5, 1, 1.5, 2, 3, 4, 6);  */
+/* the tensor scale is max|w| / (6 * 448), so block scales fit E4M3; a      */
+/* block's scale is the E4M3 code of (block max|w| / 6) / tensor scale;     */
+/* values are the nearest E2M1 of w / (block scale * tensor scale), ties to */
+/* the even code, saturating at +-6.                                        */
+/* ---------------------------------------------------------------------- */
+
+double oracle_e2m1_decode(uint8_t code)
+{
+    const int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    const double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sign ? -v : v;
+}
+
+/* Nearest E2M1 code to v (ties to the even code), saturating at +-6; exhaustive over the 8 magnitudes. */
+uint8_t oracle_e2m1_encode(float v)
+{
+    const uint8_t sign = signbit(v) ? 8 : 0;
+    double a = fabs((double)v);
+    if (!(a <= 6.0)) a = 6.0;  /* also maps NaN to the largest magnitude */
+    int best = 0;
+    double best_d = fabs(oracle_e2m1_decode(0) - a);
+    for (int c = 1; c < 8; ++c) {
+        const double d = fabs(oracle_e2m1_decode((uint8_t)c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/*
+ * codes       : [N][K] E2M1 codes, one per byte
+ * block_codes : [N][K/16] E4M3 codes of the block scales
+ * tensor_scale: the binary32 tensor scale
+ */
+int oracle_quantize_nvfp4(const float *w, int64_t N, int64_t K, int64_t ldw, uint8_t *codes,
+                          uint8_t *block_codes, float *tensor_scale)
+{
+    if (N <= 0 || K <= 0 || K % 16 != 0 || ldw < K) return -1;
+    float amax = 0.0f;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            if (fabsf(w[n * ldw + k]) > amax) amax = fabsf(w[n * ldw + k]);
+    float st = amax / (6.0f * 448.0f);
+    if (st == 0.0f) st = 1.0f;
+    *tensor_scale = st;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t b = 0; b < K / 16; ++b) {
+            const float *wb = w + n * ldw + b * 16;
+            float bmax = 0.0f;
+            for (int i = 0; i < 16; ++i)
+                if (fabsf(wb[i]) > bmax) bmax = fabsf(wb[i]);
+            const uint8_t sc = oracle_fp8_encode((bmax / 6.0f) / st, 0);
+            block_codes[n * (K / 16) + b] = sc;
+            const float S = (float)oracle_fp8_decode(sc, 0) * st;
+            for (int i = 0; i < 16; ++i)
+                codes[n * K + b * 16 + i] = S == 0.0f ? 0 : oracle_e2m1_encode(wb[i] / S);
+        }
+    return 0;
+}
+
+/* w_hat = e2m1(code) * e4m3(block code) * tensor scale, binary64. */
+int oracle_dequant_nvfp4(const uint8_t *codes, const uint8_t *block_codes, float tensor_scale, int64_t N,
+                         int64_t K, double *out)
+{
+    if (N <= 0 || K <= 0 || K % 16 != 0) return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            out[n * K + k] = oracle_e2m1_decode(codes[n * K + k]) *
+                             oracle_fp8_decode(block_codes[n * (K / 16) + k / 16], 0) * (double)tensor_scale;
+    return 0;
+}

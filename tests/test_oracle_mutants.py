@@ -41,6 +41,10 @@ MUTANTS = {
     "fp8_ties_to_odd": ("(d == best_d && (c & 1) == 0)", "(d == best_d && (c & 1) == 1)"),
     "fp8_subnormal_exponent": ("ldexp((double)m, 1 - bias - mbits)", "ldexp((double)m, -bias - mbits)"),
     "fp8_rows_int8_scale": ("amax / (float)oracle_fp8_max(fmt)", "amax / 127.0f"),
+    "e2m1_bias_2": ("ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e - 2)"),
+    "e2m1_ties_to_odd": ("if (d < best_d || (d == best_d && (c & 1) == 0)) {", "if (d < best_d || (d == best_d && (c & 1) == 1)) {"),
+    "nvfp4_tensor_scale_int8": ("float st = amax / (6.0f * 448.0f);", "float st = amax / (6.0f * 127.0f);"),
+    "nvfp4_block_scale_over_7": ("oracle_fp8_encode((bmax / 6.0f) / st, 0)", "oracle_fp8_encode((bmax / 7.0f) / st, 0)"),
 }
 
 PINS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

@@ -614,3 +614,47 @@ def test_fp8_w8a8_reference():
     bound = np.abs(x).astype(np.float64) @ np.abs(w).astype(np.float64).T
     assert np.all(np.abs(y - exact) <= 2.0 ** -3 * bound + 1e-12)
     assert np.all(a <= bound * (1 + 2.0 ** -3))
+
+
+# --------------------------------------------------------------------------
+# NVFP4 (groundwork for the NVFP4 row): the comparison page, "Hardware, formats and the roofline", and
+# "Quantization for LLM inference ...", "Microscaling: NVFP4 and MXFP4"
+# --------------------------------------------------------------------------
+
+def test_e2m1_values_and_rounding():
+    mags = [oracle.e2m1_decode(c) for c in range(8)]
+    # sign, 2 exponent bits with bias 1, 1 mantissa bit; exponent 0 is subnormal (0 and 0.5)
+    assert mags == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert [oracle.e2m1_decode(c | 8) for c in range(8)] == [-m for m in mags]
+    for c, v in enumerate(mags):
+        assert oracle.e2m1_encode(v) == c
+    for a in range(7):  # midpoints to the even code, quarter points to the nearer value
+        lo, hi = mags[a], mags[a + 1]
+        assert oracle.e2m1_encode((lo + hi) / 2) == (a if a % 2 == 0 else a + 1)
+        assert oracle.e2m1_encode(lo + (hi - lo) / 4) == a and oracle.e2m1_encode(lo + 3 * (hi - lo) / 4) == a + 1
+    assert oracle.e2m1_encode(100.0) == 7 and oracle.e2m1_encode(-100.0) == 15
+
+
+def test_nvfp4_blocks_and_scales():
+    from oracle.accounting import bits_per_weight
+    w = wq_inputs.llm_weight(24, 256, 601, dtype=torch.float32).numpy()
+    w[2] = 0.0
+    w[5, 16:32] *= 40.0   # one loud block
+    codes, blocks, st = oracle.quantize_nvfp4(w)
+    assert codes.shape == w.shape and blocks.shape == (24, 256 // 16)
+    assert st == np.float32(np.abs(w).max() / (6.0 * 448.0))          # block scales fit E4M3
+    w_hat = oracle.dequant_nvfp4(codes, blocks, st)
+    assert np.all(w_hat[2] == 0.0)
+    S = np.array([[oracle.fp8_decode(b, oracle.E4M3) for b in row] for row in blocks]) * st
+    wb = np.abs(w).reshape(24, 16, 16).max(-1)
+    live = wb > 0
+    # each block scale is its max / 6 up to E4M3 rounding (half an ulp: 2^-4 relative)
+    assert np.all(np.abs(S[live] - wb[live] / 6) <= 2.0 ** -4 * wb[live] / 6 * (1 + 1e-6))
+    # every block's largest magnitude lands on the top value 6; every error is within one block scale
+    vals = np.abs(np.vectorize(oracle.e2m1_decode)(codes)).reshape(24, 16, 16)
+    idx = np.abs(w).reshape(24, 16, 16).argmax(-1)
+    top = np.take_along_axis(vals, idx[..., None], -1)[..., 0]
+    assert np.all(top[live] == 6.0)
+    assert np.all(np.abs(w_hat - w) <= np.repeat(S, 16, axis=1) * (1 + 1e-6))
+    # 4-bit values plus an 8-bit scale per 16: the printed 4.5 bits per weight
+    assert bits_per_weight(4, 16, 8, 0) == 4.5
