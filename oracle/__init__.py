@@ -259,6 +259,15 @@ def dequant_nvfp4(codes, block_codes, tensor_scale: float) -> np.ndarray:
     return out
 
 
+def gemm_nvfp4(x, w):
+    """Reference for an NVFP4 W4A4 matmul: activations and weights each quantised to NVFP4 (blocks of 16
+    along K, each operand with its own tensor scale), the products of the decoded values summed in
+    binary64.  Returns (y, a) as matmul does."""
+    xc, xb, xs = quantize_nvfp4(x)
+    wc, wb, ws = quantize_nvfp4(w)
+    return matmul(dequant_nvfp4(xc, xb, xs), dequant_nvfp4(wc, wb, ws))
+
+
 def pack_int4(codes) -> np.ndarray:
     """[N][K] codes -> [N][K/2] bytes, code 2j in the low nibble of byte j."""
     c = np.ascontiguousarray(codes, dtype=np.uint8)

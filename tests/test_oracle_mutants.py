@@ -45,6 +45,9 @@ MUTANTS = {
     "e2m1_ties_to_odd": ("if (d < best_d || (d == best_d && (c & 1) == 0)) {", "if (d < best_d || (d == best_d && (c & 1) == 1)) {"),
     "nvfp4_tensor_scale_int8": ("float st = amax / (6.0f * 448.0f);", "float st = amax / (6.0f * 127.0f);"),
     "nvfp4_block_scale_over_7": ("oracle_fp8_encode((bmax / 6.0f) / st, 0)", "oracle_fp8_encode((bmax / 7.0f) / st, 0)"),
+    "nvfp4_dequant_block_index": ("block_codes[n * (K / 16) + k / 16]", "block_codes[n * (K / 16) + k % (K / 16)]"),
+    "nvfp4_dequant_scale_as_e5m2": ("oracle_fp8_decode(block_codes[n * (K / 16) + k / 16], 0)",
+                                    "oracle_fp8_decode(block_codes[n * (K / 16) + k / 16], 1)"),
 }
 
 PINS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

@@ -658,3 +658,28 @@ def test_nvfp4_blocks_and_scales():
     assert np.all(np.abs(w_hat - w) <= np.repeat(S, 16, axis=1) * (1 + 1e-6))
     # 4-bit values plus an 8-bit scale per 16: the printed 4.5 bits per weight
     assert bits_per_weight(4, 16, 8, 0) == 4.5
+
+
+def test_nvfp4_w4a4_reference():
+    """The NVFP4 matmul reference: the binary64 product of operands decoded from their codes with a table
+    of the eight E2M1 magnitudes (the microscaling formats' 4-bit element, Rouhani et al., cited by the
+    page's "Microscaling: NVFP4 and MXFP4") and torch's E4M3 decode; within one block scale per operand
+    of the unquantised product."""
+    x = wq_inputs.plain_activations(4, 256, 605).float().numpy()
+    w = wq_inputs.llm_weight(32, 256, 606, dtype=torch.float32).numpy()
+    y, a = oracle.gemm_nvfp4(x, w)
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+    def decode(v):
+        c, b, st = oracle.quantize_nvfp4(v)
+        vals = np.where(c & 8, -1.0, 1.0) * mags[c & 7]
+        S = torch.from_numpy(b).view(torch.float8_e4m3fn).double().numpy() * st
+        return vals * np.repeat(S, 16, axis=1), np.repeat(S, 16, axis=1)
+
+    xd, sx = decode(x)
+    wd, sw = decode(w)
+    np.testing.assert_allclose(y, xd @ wd.T, rtol=1e-13, atol=1e-13)
+    exact = x.astype(np.float64) @ w.astype(np.float64).T
+    bound = np.abs(x) @ sw.T + sx @ np.abs(w).T + sx @ sw.T
+    assert np.all(np.abs(y - exact) <= bound * (1 + 1e-9))
+    assert np.all(np.abs(y) <= a * (1 + 1e-12))
