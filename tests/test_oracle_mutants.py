@@ -45,6 +45,19 @@ MUTANTS = {
     "e2m1_ties_to_odd": ("if (d < best_d || (d == best_d && (c & 1) == 0)) {", "if (d < best_d || (d == best_d && (c & 1) == 1)) {"),
     "nvfp4_tensor_scale_int8": ("float st = amax / (6.0f * 448.0f);", "float st = amax / (6.0f * 127.0f);"),
     "nvfp4_block_scale_over_7": ("oracle_fp8_encode((bmax / 6.0f) / st, 0)", "oracle_fp8_encode((bmax / 7.0f) / st, 0)"),
+    "unpack_high_nibble_unmasked": ("codes[n * K + 2 * j + 1] = packed[n * (K / 2) + j] >> 4;",
+                                    "codes[n * K + 2 * j + 1] = packed[n * (K / 2) + j] >> 3;"),
+    "int8_dequant_group_index": ("(double)s[n * G + k / g] * (double)codes[n * K + k]",
+                                 "(double)s[n * G + k % G] * (double)codes[n * K + k]"),
+    "int8_zero_scale_kept": ("float s = store_param(amax / 127.0f, mode);\n            if (s == 0.0f) s = 1.0f;",
+                             "float s = store_param(amax / 127.0f, mode);"),
+    "fp8_rows_zero_scale_kept": ("float s = amax / (float)oracle_fp8_max(fmt);\n        if (s == 0.0f) s = 1.0f;",
+                                 "float s = amax / (float)oracle_fp8_max(fmt);"),
+    "fp8_no_saturation": ("if (a > oracle_fp8_max(fmt)) a = oracle_fp8_max(fmt);", ";"),
+    "e2m1_no_saturation": ("if (!(a <= 6.0)) a = 6.0;", ";"),
+    "nvfp4_global_amax_per_row": ("if (fabsf(w[n * ldw + k]) > amax) amax = fabsf(w[n * ldw + k]);",
+                                  "if (n == 0 && fabsf(w[n * ldw + k]) > amax) amax = fabsf(w[n * ldw + k]);"),
+    "matmul_bound_without_a": ("if (a) a[m * N + n] = aacc;", "if (a) a[m * N + n] = fabs(acc);"),
     "nvfp4_dequant_block_index": ("block_codes[n * (K / 16) + k / 16]", "block_codes[n * (K / 16) + k % (K / 16)]"),
     "nvfp4_dequant_scale_as_e5m2": ("oracle_fp8_decode(block_codes[n * (K / 16) + k / 16], 0)",
                                     "oracle_fp8_decode(block_codes[n * (K / 16) + k / 16], 1)"),
