@@ -2,7 +2,6 @@
 include/wq.h declares, and rejects bad arguments on the host before any
 launch.  CPU only: no call here reaches a kernel launch (every call fails
 validation, or is a pure host query)."""
-import ctypes
 import subprocess
 
 import pytest
