@@ -212,6 +212,25 @@ def test_quantised_values_move_the_output_by_at_most_their_error():
     assert np.abs(v_hat - v).max() <= 0.56 * s.max()
 
 
+def test_fp8_cache_read_error_and_zero_cache():
+    """E4M3 with a per-tensor scale: with exact keys, each output moves by at most the largest value error,
+    itself at most 2^-4 relative (half a step of a 3-bit mantissa) above the subnormal range; an all-zero
+    cache takes the scale 1 and reads back zeros."""
+    B, T, H, D = 2, 24, 1, 128
+    k, v = _cache(19, B, T, H, D), _cache(20, B, T, H, D)
+    q = _cache(21, 1, B, 2, D)[0]
+    codes, s = kv.quantize_kv_fp8(v)
+    v_hat = kv.dequant_kv_fp8(codes, s)
+    o, _ = kv.decode_attention(q, k, v, [24, 9])
+    oq, _ = kv.decode_attention(q, k, v_hat, [24, 9])
+    verr = np.abs(v_hat - v)
+    assert 0 < np.abs(oq - o).max() <= verr.max() * (1 + 1e-12)
+    normal = np.abs(v) >= 2.0 ** -6 * float(s)
+    assert (verr[normal] <= 2.0 ** -4 * np.abs(v[normal]) * (1 + 1e-6)).all()
+    zc, zs = kv.quantize_kv_fp8(np.zeros((1, 4, 1, D), dtype=np.float32))
+    assert zs == 1.0 and not zc.any() and not kv.dequant_kv_fp8(zc, zs).any()
+
+
 PINS = [test_int4_block_holds_the_page_example, test_int4_blocks_run_along_head_dim,
         test_int4_cache_storage_matches_the_page,
         lambda: [test_fp8_cache_scale_and_codes(f, d) for f, d in
@@ -220,7 +239,7 @@ PINS = [test_int4_block_holds_the_page_example, test_int4_blocks_run_along_head_
         lambda: [test_scores_scaled_by_sqrt_head_dim(d) for d in (16, 64, 128)],
         test_query_heads_share_consecutive_kv_heads, test_tokens_beyond_length_are_ignored,
         test_large_scores_select_the_best_token, test_output_is_a_convex_combination_and_order_free,
-        test_quantised_values_move_the_output_by_at_most_their_error]
+        test_quantised_values_move_the_output_by_at_most_their_error, test_fp8_cache_read_error_and_zero_cache]
 
 MUTANTS = {
     "no_sqrt_scale": ("score = k[b, :n, kv, :] @ q[b, h] / math.sqrt(D)", "score = k[b, :n, kv, :] @ q[b, h]"),
