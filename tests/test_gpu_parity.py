@@ -144,22 +144,6 @@ def test_quantize_padded_rows_and_odd_sizes():
         assert np.array_equal(q8.cpu().numpy(), c8) and np.array_equal(bits(s8), s8b)
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_quantize_ragged_last_chunk(dtype):
-    """K not a multiple of 256: a warp's last 256-weight chunk of a row runs past K, and the lanes beyond K
-    must sit out of the group reductions (for bf16 input the asymmetric quantiser carries min and -max as
-    one packed pair).  Every quantiser, both input types; K = 128 with g = 128 is one group per row, the
-    layout of a KV cache quantised in blocks of 128."""
-    for N, K, g in ((7, 96, 32), (5, 128, 128), (9, 128, 64), (3, 288, 32), (4, 640, 128)):
-        w = wq_inputs.llm_weight(N, K, 90 + K + g, dtype=torch.float32).to(dtype)
-        check_q4(w, g)
-        check_q4_sym(w, g)
-        q8, s8 = wq.wq_quantize_int8(w.cuda(), g)
-        torch.cuda.synchronize()
-        c8, _, s8b = oracle_q8(w, g)
-        assert np.array_equal(q8.cpu().numpy(), c8) and np.array_equal(bits(s8), s8b)
-
-
 def test_quantize_degenerate_and_one_signed_groups():
     w = wq_inputs.llm_weight(64, 512, 81, dtype=torch.float32)
     w[0] = 0.0                    # all-zero row
@@ -536,3 +520,19 @@ def test_awq_search_on_the_gpu_tracks_the_oracle_search():
     _, _, o_errors = oawq.search(x.double().numpy(), w.numpy(), deq)
     assert np.allclose(errors, o_errors, rtol=0.05)
     assert alpha > 0 and o_errors[gawq.GRID.index(alpha)] <= 1.05 * min(o_errors)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_ragged_last_chunk(dtype):
+    """K not a multiple of 256: a warp's last 256-weight chunk of a row runs past K, and the lanes beyond K
+    must sit out of the group reductions (for bf16 input the asymmetric quantiser carries min and -max as
+    one packed pair).  Every quantiser, both input types; K = 128 with g = 128 is one group per row, the
+    layout of a KV cache quantised in blocks of 128."""
+    for N, K, g in ((7, 96, 32), (5, 128, 128), (9, 128, 64), (3, 288, 32), (4, 640, 128)):
+        w = wq_inputs.llm_weight(N, K, 90 + K + g, dtype=torch.float32).to(dtype)
+        check_q4(w, g)
+        check_q4_sym(w, g)
+        q8, s8 = wq.wq_quantize_int8(w.cuda(), g)
+        torch.cuda.synchronize()
+        c8, _, s8b = oracle_q8(w, g)
+        assert np.array_equal(q8.cpu().numpy(), c8) and np.array_equal(bits(s8), s8b)
