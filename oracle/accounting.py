@@ -52,3 +52,33 @@ def block_bytes_per_element(bits: int, block: int, param_bits: int) -> float:
 def decode_step_speedup(weight_bytes_before: float, weight_bytes_after: float, other_bytes: float) -> float:
     """Memory-bound decode: the step time scales with the bytes read, weights plus everything else."""
     return (weight_bytes_before + other_bytes) / (weight_bytes_after + other_bytes)
+
+
+# ---------------------------------------------------------------------------
+# Roofline of the decode step (the measurement's basis)
+#   * "Quantization Methods Compared ..." -- "Hardware, formats and the roofline": a decode step reads every
+#     weight once and does 2 x parameters x batch flops; with 1,000 TFLOP/s and 3.3 TB/s the ridge point is
+#     1,000 / 3.3 = 303 flop per byte; fp16 weights (2 bytes) give an intensity of batch flop per byte, so
+#     decode stays memory-bound until batch about 300; 4-bit weights (0.5 bytes) give 4 x batch and cross the
+#     ridge near batch 76.  The worked step (70B, batch 128, 8 GPUs: 26.4 TB/s and 8,000 TFLOP/s together)
+#     computes for about 2.2 ms, far below its memory time.
+# ---------------------------------------------------------------------------
+
+def ridge_point(flops_per_s: float, bytes_per_s: float) -> float:
+    """Arithmetic intensity (flop per byte) above which a kernel is compute-bound."""
+    return flops_per_s / bytes_per_s
+
+
+def decode_intensity(batch: int, bytes_per_weight: float) -> float:
+    """Flop per byte of a decode step: 2 x batch flops per weight over the weight's bytes."""
+    return 2.0 * batch / bytes_per_weight
+
+
+def crossover_batch(ridge: float, bytes_per_weight: float) -> float:
+    """The batch at which decode_intensity reaches the ridge point."""
+    return ridge * bytes_per_weight / 2.0
+
+
+def decode_compute_seconds(n_params: float, batch: int, flops_per_s: float) -> float:
+    """Compute time of one decode step: 2 x parameters x batch flops."""
+    return 2.0 * n_params * batch / flops_per_s

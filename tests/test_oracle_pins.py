@@ -683,3 +683,22 @@ def test_nvfp4_w4a4_reference():
     bound = np.abs(x) @ sw.T + sx @ np.abs(w).T + sx @ sw.T
     assert np.all(np.abs(y - exact) <= bound * (1 + 1e-9))
     assert np.all(np.abs(y) <= a * (1 + 1e-12))
+
+
+def test_roofline_closed_forms():
+    """[P3] "Hardware, formats and the roofline": ridge 1,000 / 3.3 = 303 flop/B; fp16 intensity = batch
+    (memory-bound to about 300); 4-bit intensity 4 x batch (crossing near 76); the worked 70B step at batch
+    128 on 8 GPUs computes for about 2.2 ms."""
+    from oracle.accounting import crossover_batch, decode_compute_seconds, decode_intensity, ridge_point
+    sc, _ = read("roofline_closed_forms.txt")
+    ridge = ridge_point(scalar(sc, "tflops_assumed") * 1e12, scalar(sc, "tbs_assumed") * 1e12)
+    assert round(ridge) == scalar(sc, "ridge_printed")
+    assert decode_intensity(128, 2.0) == 128 and decode_intensity(128, 0.5) == 4 * 128
+    assert abs(crossover_batch(ridge, 2.0) - scalar(sc, "fp16_crossover_printed")) < 5   # "about 300"
+    assert round(crossover_batch(ridge, 0.5)) == scalar(sc, "int4_crossover_printed")
+    n = scalar(sc, "gpus")
+    assert round(n * scalar(sc, "tbs_assumed"), 1) == scalar(sc, "aggregate_tbs_printed")
+    assert n * scalar(sc, "tflops_assumed") == scalar(sc, "aggregate_tflops_printed")
+    t = decode_compute_seconds(scalar(sc, "params"), int(scalar(sc, "batch")),
+                               scalar(sc, "aggregate_tflops_printed") * 1e12)
+    assert round(t * 1e3, 1) == scalar(sc, "compute_ms_printed")
