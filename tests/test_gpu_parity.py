@@ -329,7 +329,8 @@ def test_gemm_w4a16_batch_sizes(M):
 
 
 @pytest.mark.parametrize("M,N,K,g", [(32, 128, 128, 128), (17, 256, 256, 64), (64, 384, 1024, 32),
-                                     (128, 130, 384, 128), (200, 512, 640, 128), (256, 128, 128, 32)])
+                                     (128, 130, 384, 128), (200, 512, 640, 128), (256, 128, 128, 32),
+                                     (255, 384, 512, 64)])
 def test_gemm_w4a16_tensor_core_tiles(M, N, K, g):
     """Shapes around the tcgen05 kernel's tile edges: one tile, ragged N, several M tiles, split K."""
     _w4_case(N, K, g, M, 17 * M + N)
