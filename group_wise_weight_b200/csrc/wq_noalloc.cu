@@ -20,7 +20,10 @@
 // All calls share the one array: the part a call uses is cleared on the
 // call's stream before the kernel runs, and calls whose executions overlap on
 // the GPU (different streams, or the same array from several host threads at
-// once) race on it.
+// once) race on it.  The cached address belongs to the CUDA context current
+// at the first call: the library must not be used across a cudaDeviceReset
+// (nor is the device status word's address, cached the same way in
+// wq_api.cu, looked up again after one).
 #include <cstdio>
 #include <mutex>
 
@@ -62,11 +65,10 @@ extern "C" int wq_gemm_w4a16_noalloc(const uint16_t *x, int64_t M, int64_t N, in
         return wq::record_error(WQ_ERR_ARG, "wq_gemm_w4a16_noalloc: null pointer");
     if (M <= 0 || N <= 0 || K <= 0)
         return wq::record_error(WQ_ERR_ARG, "wq_gemm_w4a16_noalloc: M, N and K must be positive");
-    if (!wq::gemv_tma_eligible(M, N, K, g))
+    if (!wq::gemv_tma_eligible(M, N, K, g) || K % 128 != 0)
         return wq::record_error(WQ_ERR_UNSUPPORTED,
                                 "wq_gemm_w4a16_noalloc: needs g = 128, 2 <= M <= 16, N >= 128, K >= 256 and "
                                 "K % 128 == 0 (other shapes: wq_gemm_w4a16)");
-    if (K % 128 != 0) return wq::record_error(WQ_ERR_SHAPE, "wq_gemm_w4a16_noalloc: K % 128 != 0");
     if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y))
         return wq::record_error(WQ_ERR_ALIGN, "wq_gemm_w4a16_noalloc: pointers must be 16-byte aligned");
     if (wq::output_overlaps_inputs(x, M, N, K, qweight, scales, zeros, g, y, false))

@@ -152,9 +152,12 @@ int wq_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw
  * Bytes of device workspace wq_gemm_w4a16 (wbits = 4) or wq_gemm_w8a16
  * (wbits = 8) needs for this shape; 0 when the chosen kernel needs none.
  * The workspace holds binary32 partial sums of a K-split and per-tile
- * arrival counters; the library leaves the counters zeroed on return, so
- * a workspace must be zero-filled once before its first use and may then be
- * reused by later calls on the same stream.
+ * arrival counters; a call that completes normally leaves the counters
+ * zeroed, so a workspace must be zero-filled once before its first use and
+ * may then be reused by later calls on the same stream.  A call whose kernel
+ * gave up on a bounded wait (wq_device_status returns WQ_ERR_DEVICE_TIMEOUT)
+ * can leave counters of the tiles it did not finish non-zero: zero-fill the
+ * workspace again before reusing it after such a status.
  */
 size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits);
 
@@ -234,7 +237,13 @@ int wq_gemm_w4a16_noalloc(const uint16_t *x, int64_t M, int64_t N, int64_t K, co
  * early instead of hanging.  This call synchronises `stream`, returns
  * WQ_ERR_DEVICE_TIMEOUT if any kernel of this library recorded a timeout on
  * the current device since the last call (and clears it), WQ_ERR_CUDA if the
- * stream reports an error, else WQ_OK.
+ * stream reports an error, else WQ_OK.  After WQ_ERR_DEVICE_TIMEOUT the
+ * outputs of the calls since the last check are unspecified and every
+ * workspace they used must be zero-filled again before its next use.
+ *
+ * The device addresses of the status word and of the no-allocation scratch
+ * array are looked up once per device and cached: do not keep using the
+ * library after cudaDeviceReset in the same process.
  */
 int wq_device_status(void *stream);
 

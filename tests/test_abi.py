@@ -167,3 +167,42 @@ def test_quantize_rejects_outputs_overlapping(L):
         assert _q4(L, **args) == wq.WQ_ERR_ARG, kw
         assert "overlap" in wq.wq_last_error()
     assert _q8(L, w=w, N=N, K=K, ldw=K, q=w + N * K * 2 - 16, s=s) == wq.WQ_ERR_ARG
+
+
+def _g4n(L, x=A, M=4, N=256, K=512, q=None, s=None, z=None, g=128, y=None):
+    # distinct fake buffers so that only the argument under test can fail
+    xb, qb, sb, zb, yb = _bufs(5)
+    x = xb if x == A else x
+    q = qb if q is None else q
+    s = sb if s is None else s
+    z = zb if z is None else z
+    y = yb if y is None else y
+    return L.wq_gemm_w4a16_noalloc(x, M, N, K, q, s, z, g, y, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=None), wq.WQ_ERR_ARG), (dict(q=0), wq.WQ_ERR_ARG), (dict(z=0), wq.WQ_ERR_ARG),
+    (dict(y=0), wq.WQ_ERR_ARG), (dict(M=0), wq.WQ_ERR_ARG), (dict(N=-5), wq.WQ_ERR_ARG),
+    (dict(K=0), wq.WQ_ERR_ARG),
+    (dict(M=1), wq.WQ_ERR_UNSUPPORTED), (dict(M=17), wq.WQ_ERR_UNSUPPORTED), (dict(g=64), wq.WQ_ERR_UNSUPPORTED),
+    (dict(N=100), wq.WQ_ERR_UNSUPPORTED), (dict(K=128), wq.WQ_ERR_UNSUPPORTED),
+    (dict(K=320), wq.WQ_ERR_UNSUPPORTED), (dict(K=4096 + 64), wq.WQ_ERR_UNSUPPORTED),
+    (dict(x=MIS), wq.WQ_ERR_ALIGN), (dict(q=(1 << 30) + (1 << 24) + 8), wq.WQ_ERR_ALIGN),
+    (dict(y=(1 << 30) + 4 * (1 << 24) + 2), wq.WQ_ERR_ALIGN),
+])
+def test_gemm_w4a16_noalloc_rejects(L, kw, code):
+    assert _g4n(L, **kw) == code
+    assert wq.wq_last_error() != ""
+
+
+def test_gemm_w4a16_noalloc_rejects_overlap_and_oversize(L):
+    x, q, s, z, y = _bufs(5)
+    for yy in (x + 16, q + 512, s, z):
+        assert _g4n(L, y=yy) == wq.WQ_ERR_ARG
+        assert "overlaps" in wq.wq_last_error()
+    # the scratch need is M * N * 4 bytes (rounded up to 256) plus one int per 128 rows (rounded up to 256):
+    # at M = 16 the largest N that fits 2 MiB is 32752 (exactly 2 MiB); one more row does not fit.  The
+    # accepted shape goes on to look up the array's address, which needs a device, so only the refusal
+    # is checked here (the GPU test runs the exact-limit shape).
+    assert _g4n(L, M=16, N=32753, K=256) == wq.WQ_ERR_WORKSPACE
+    assert "scratch" in wq.wq_last_error()

@@ -6,8 +6,11 @@ workspace wq_gemm_w4a16 asks for; this entry point takes none and uses the
 library's fixed scratch array.  Its results must match the regular entry
 point's within the tolerance every matmul test here uses
 (|y - y_ref| <= 4e-3 * sum_k |x * w_hat|), on two calls in a row (the second
-call finds the array as the first left it).  This file is collected last, so
-that a run stopping at the first failure has already run every other test.
+call finds the array as the first left it), and each call must also meet that
+bound against the oracle's binary64 product on its own, so that the two
+kernels' errors cannot add up unnoticed.  One shape needs exactly the array's
+2 MiB.  This file is collected last, so that a run stopping at the first
+failure has already run every other test.
 """
 import numpy as np
 import pytest
@@ -35,13 +38,16 @@ def _quantised(N, K, seed):
     return q, s, z, codes, so, zo
 
 
-@pytest.mark.parametrize("M,N,K", [(2, 1000, 512), (8, 14336, 4096), (16, 4096, 8192), (5, 300, 256)])
+# (16, 32752, 256): M * N * 4 bytes plus one int per 128 rows, each rounded up to 256 bytes, is exactly
+# the array's 2 MiB -- the largest N accepted at M = 16 (N = 32753 is refused, tests/test_abi.py).
+@pytest.mark.parametrize("M,N,K", [(2, 1000, 512), (8, 14336, 4096), (16, 4096, 8192), (5, 300, 256),
+                                   (16, 32752, 256)])
 def test_noalloc_matches_regular_entry_point_twice(M, N, K):
     q, s, z, codes, so, zo = _quantised(N, K, 900 + M)
     x = wq_inputs.activations(M, K, 901 + M).cuda()
     y_ref = wq.wq_gemm_w4a16(x, q, s, z, 128)
     torch.cuda.synchronize()
-    _, a_ref = oracle.gemm_w4a16(x.double().cpu().numpy(), codes, so, zo, 128)
+    y_exact, a_ref = oracle.gemm_w4a16(x.double().cpu().numpy(), codes, so, zo, 128)
     bound = TOL * a_ref
     yr = y_ref.double().cpu().numpy()
     for call in range(2):
@@ -51,6 +57,7 @@ def test_noalloc_matches_regular_entry_point_twice(M, N, K):
         yn = y.double().cpu().numpy()
         assert np.all(np.isfinite(yn)), f"call {call}: output not fully written"
         assert np.all(np.abs(yn - yr) <= bound), f"call {call}: differs from wq_gemm_w4a16"
+        assert np.all(np.abs(yn - y_exact) <= bound), f"call {call}: outside the bound against the oracle"
     assert wq.wq_device_status() == wq.WQ_OK
 
 
