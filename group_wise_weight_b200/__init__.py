@@ -32,6 +32,8 @@ WQ_ERR_WORKSPACE = -6
 WQ_ERR_DEVICE_TIMEOUT = -7
 WQ_F32 = 0
 WQ_BF16 = 1
+WQ_FP8_E4M3 = 0
+WQ_FP8_E5M2 = 1
 
 _lib = None
 
@@ -76,6 +78,22 @@ def lib():
         L.wq_gemm_w4a16_noalloc.restype = I
         L.wq_device_status.argtypes = [P]
         L.wq_device_status.restype = I
+        L.wq_quantize_fp8.argtypes = [P, I, I64, I64, I64, I, P, P, P]
+        L.wq_quantize_fp8.restype = I
+        L.wq_quantize_fp8_tensor.argtypes = [P, I, I64, I64, I, P, P, P]
+        L.wq_quantize_fp8_tensor.restype = I
+        L.wq_gemm_w8a8_fp8_workspace_bytes.argtypes = [I64, I64, I64]
+        L.wq_gemm_w8a8_fp8_workspace_bytes.restype = SZ
+        L.wq_gemm_w8a8_fp8.argtypes = [P, P, I64, I64, I64, P, P, P, P, SZ, P]
+        L.wq_gemm_w8a8_fp8.restype = I
+        L.wq_nvfp4_scale_bytes.argtypes = [I64, I64]
+        L.wq_nvfp4_scale_bytes.restype = SZ
+        L.wq_quantize_nvfp4.argtypes = [P, I, I64, I64, I64, P, P, P, P]
+        L.wq_quantize_nvfp4.restype = I
+        L.wq_gemm_nvfp4_workspace_bytes.argtypes = [I64, I64, I64]
+        L.wq_gemm_nvfp4_workspace_bytes.restype = SZ
+        L.wq_gemm_nvfp4.argtypes = [P, P, P, I64, I64, I64, P, P, P, P, P, SZ, P]
+        L.wq_gemm_nvfp4.restype = I
         _lib = L
     return _lib
 
@@ -283,3 +301,120 @@ def wq_gemm_w4a16_noalloc(x: torch.Tensor, qweight: torch.Tensor, scales: torch.
 def wq_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word as a WQ_* code."""
     return int(lib().wq_device_status(_stream_handle(stream)))
+
+
+def _wtype(t: torch.Tensor) -> int:
+    wtype = {torch.float32: WQ_F32, torch.bfloat16: WQ_BF16}.get(t.dtype)
+    if wtype is None:
+        raise TypeError("input must be float32 or bfloat16")
+    return wtype
+
+
+def wq_quantize_fp8(w: torch.Tensor, fmt: int = WQ_FP8_E4M3, qweight=None, scales=None, stream=None):
+    """FP8 per output channel.  w: [N][K] (row stride >= K) fp32 or bf16 on CUDA.
+
+    Returns (qweight uint8 [N][K] FP8 codes, scales float32 [N])."""
+    if w.dim() != 2 or w.stride(1) != 1:
+        raise ValueError("w must be a 2-D tensor with unit stride along K")
+    wtype = _wtype(w)
+    N, K = w.shape
+    qweight = torch.empty((N, K), dtype=torch.uint8, device=w.device) if qweight is None else qweight
+    scales = torch.empty((N,), dtype=torch.float32, device=w.device) if scales is None else scales
+    _dense(qweight, "qweight")
+    _dense(scales, "scales")
+    _check(lib().wq_quantize_fp8(_dev(w, "w"), wtype, N, K, w.stride(0), int(fmt), _dev(qweight, "qweight"),
+                                 _dev(scales, "scales"), _stream_handle(stream)))
+    return qweight, scales
+
+
+def wq_quantize_fp8_tensor(x: torch.Tensor, fmt: int = WQ_FP8_E4M3, q=None, scale=None, stream=None):
+    """FP8 with one scale for the whole tensor.  x: dense [M][K] fp32 or bf16 on CUDA.
+
+    Returns (q uint8 [M][K] FP8 codes, scale float32 [1] on the device)."""
+    if x.dim() != 2:
+        raise ValueError("x must be a 2-D tensor")
+    _dense(x, "x")
+    xtype = _wtype(x)
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if q is None else q
+    scale = torch.empty((1,), dtype=torch.float32, device=x.device) if scale is None else scale
+    _dense(q, "q")
+    _check(lib().wq_quantize_fp8_tensor(_dev(x, "x"), xtype, M, K, int(fmt), _dev(q, "q"), _dev(scale, "scale"),
+                                        _stream_handle(stream)))
+    return q, scale
+
+
+def wq_gemm_w8a8_fp8_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().wq_gemm_w8a8_fp8_workspace_bytes(int(M), int(N), int(K)))
+
+
+def wq_gemm_w8a8_fp8(xq: torch.Tensor, xscale: torch.Tensor, wq: torch.Tensor, wscales: torch.Tensor, y=None,
+                     workspace=None, stream=None) -> torch.Tensor:
+    """y[M][N] = (xq . wq^T) * xscale * wscales[n] with E4M3 codes multiplied on the tensor cores.  bf16 out."""
+    if xq.dtype != torch.uint8 or wq.dtype != torch.uint8 or xq.dim() != 2 or wq.dim() != 2:
+        raise TypeError("xq and wq must be 2-D uint8 tensors of FP8 codes")
+    for t, n in ((xq, "xq"), (wq, "wq"), (wscales, "wscales")):
+        _dense(t, n)
+    M, K = xq.shape
+    N = wq.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device) if y is None else y
+    _dense(y, "y")
+    need = wq_gemm_w8a8_fp8_workspace_bytes(M, N, K)
+    workspace, ws_bytes = _workspace(workspace, need, xq.device)
+    _check(lib().wq_gemm_w8a8_fp8(_dev(xq, "xq"), _dev(xscale, "xscale"), M, N, K, _dev(wq, "wq"),
+                                  _dev(wscales, "wscales"), _dev(y, "y"),
+                                  workspace.data_ptr() if workspace is not None else None, ws_bytes,
+                                  _stream_handle(stream)))
+    return y
+
+
+def wq_nvfp4_scale_bytes(N: int, K: int) -> int:
+    return int(lib().wq_nvfp4_scale_bytes(int(N), int(K)))
+
+
+def wq_quantize_nvfp4(w: torch.Tensor, codes=None, block_scales=None, tensor_scale=None, stream=None):
+    """NVFP4: E2M1 values, an E4M3 scale per 16 values of a row, one binary32 tensor scale.
+    w: [N][K] (row stride >= K) fp32 or bf16 on CUDA.
+
+    Returns (codes uint8 [N][K/2], block_scales uint8 [wq_nvfp4_scale_bytes(N, K)] in the tensor-core
+    layout, tensor_scale float32 [1] on the device)."""
+    if w.dim() != 2 or w.stride(1) != 1:
+        raise ValueError("w must be a 2-D tensor with unit stride along K")
+    wtype = _wtype(w)
+    N, K = w.shape
+    dev = w.device
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev) if codes is None else codes
+    nsb = wq_nvfp4_scale_bytes(N, K)
+    block_scales = torch.empty((max(nsb, 1),), dtype=torch.uint8, device=dev) if block_scales is None else block_scales
+    tensor_scale = torch.empty((1,), dtype=torch.float32, device=dev) if tensor_scale is None else tensor_scale
+    _dense(codes, "codes")
+    _check(lib().wq_quantize_nvfp4(_dev(w, "w"), wtype, N, K, w.stride(0), _dev(codes, "codes"),
+                                   _dev(block_scales, "block_scales"), _dev(tensor_scale, "tensor_scale"),
+                                   _stream_handle(stream)))
+    return codes, block_scales, tensor_scale
+
+
+def wq_gemm_nvfp4_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().wq_gemm_nvfp4_workspace_bytes(int(M), int(N), int(K)))
+
+
+def wq_gemm_nvfp4(x_codes: torch.Tensor, x_scales: torch.Tensor, x_tscale: torch.Tensor, w_codes: torch.Tensor,
+                  w_scales: torch.Tensor, w_tscale: torch.Tensor, y=None, workspace=None, stream=None) -> torch.Tensor:
+    """NVFP4 W4A4 matmul with the block scales applied inside the tensor-core MMA.  Operands as returned by
+    wq_quantize_nvfp4 (x_codes [M][K/2], w_codes [N][K/2]).  bf16 out [M][N]."""
+    if x_codes.dtype != torch.uint8 or w_codes.dtype != torch.uint8 or x_codes.dim() != 2 or w_codes.dim() != 2:
+        raise TypeError("codes must be 2-D uint8 tensors")
+    for t, n in ((x_codes, "x_codes"), (w_codes, "w_codes")):
+        _dense(t, n)
+    M, K = x_codes.shape[0], x_codes.shape[1] * 2
+    N = w_codes.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x_codes.device) if y is None else y
+    _dense(y, "y")
+    need = wq_gemm_nvfp4_workspace_bytes(M, N, K)
+    workspace, ws_bytes = _workspace(workspace, need, x_codes.device)
+    _check(lib().wq_gemm_nvfp4(_dev(x_codes, "x_codes"), _dev(x_scales, "x_scales"), _dev(x_tscale, "x_tscale"),
+                               M, N, K, _dev(w_codes, "w_codes"), _dev(w_scales, "w_scales"),
+                               _dev(w_tscale, "w_tscale"), _dev(y, "y"),
+                               workspace.data_ptr() if workspace is not None else None, ws_bytes,
+                               _stream_handle(stream)))
+    return y

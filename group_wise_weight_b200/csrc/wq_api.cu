@@ -269,6 +269,147 @@ int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8
     return check_launch("wq_gemm_w8a16");
 }
 
+int wq_quantize_fp8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int fmt, uint8_t *qweight,
+                    float *scales, void *stream)
+{
+    g_last_error.clear();
+    const char *what = "wq_quantize_fp8";
+    if (!w || !qweight || !scales) return fail(WQ_ERR_ARG, "%s: null pointer", what);
+    if (N <= 0 || K <= 0 || ldw <= 0) return fail(WQ_ERR_ARG, "%s: N, K and ldw must be positive", what);
+    if (wtype != WQ_F32 && wtype != WQ_BF16) return fail(WQ_ERR_UNSUPPORTED, "%s: wtype %d", what, wtype);
+    if (fmt != WQ_FP8_E4M3 && fmt != WQ_FP8_E5M2) return fail(WQ_ERR_UNSUPPORTED, "%s: fmt %d", what, fmt);
+    if (K % 32 != 0 || ldw < K)
+        return fail(WQ_ERR_SHAPE, "%s: need K %% 32 == 0 and ldw >= K (K=%lld ldw=%lld)", what, (long long)K,
+                    (long long)ldw);
+    if (ldw % 8 != 0 || !aligned16(w) || !aligned16(qweight) || !aligned16(scales))
+        return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned and ldw a multiple of 8", what);
+    const uint64_t wb = span(N - 1, ldw, wtype == WQ_F32 ? 4 : 2) + span(1, K, wtype == WQ_F32 ? 4 : 2);
+    const uint64_t qb = span(N, K, 1), sb = span(N, 1, 4);
+    if (overlap(qweight, qb, w, wb) || overlap(scales, sb, w, wb) || overlap(qweight, qb, scales, sb))
+        return fail(WQ_ERR_ARG, "%s: output buffers overlap the weights or each other", what);
+    wq::launch_quantize_fp8_rows(w, wtype, N, K, ldw, fmt, qweight, scales, static_cast<cudaStream_t>(stream));
+    return check_launch(what);
+}
+
+int wq_quantize_fp8_tensor(const void *x, int xtype, int64_t M, int64_t K, int fmt, uint8_t *q, float *scale,
+                           void *stream)
+{
+    g_last_error.clear();
+    const char *what = "wq_quantize_fp8_tensor";
+    if (!x || !q || !scale) return fail(WQ_ERR_ARG, "%s: null pointer", what);
+    if (M <= 0 || K <= 0) return fail(WQ_ERR_ARG, "%s: M and K must be positive", what);
+    if (xtype != WQ_F32 && xtype != WQ_BF16) return fail(WQ_ERR_UNSUPPORTED, "%s: xtype %d", what, xtype);
+    if (fmt != WQ_FP8_E4M3 && fmt != WQ_FP8_E5M2) return fail(WQ_ERR_UNSUPPORTED, "%s: fmt %d", what, fmt);
+    if (K % 32 != 0) return fail(WQ_ERR_SHAPE, "%s: need K %% 32 == 0 (K=%lld)", what, (long long)K);
+    if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+        return fail(WQ_ERR_ALIGN, "%s: x and q must be 16-byte aligned, scale 4-byte aligned", what);
+    const uint64_t xb = span(M, K, xtype == WQ_F32 ? 4 : 2), qb = span(M, K, 1);
+    if (overlap(q, qb, x, xb) || overlap(scale, 4, x, xb) || overlap(scale, 4, q, qb))
+        return fail(WQ_ERR_ARG, "%s: q or scale overlaps x, or each other", what);
+    if (wq::launch_quantize_fp8_tensor(x, xtype, M * K, fmt, q, scale, static_cast<cudaStream_t>(stream)) != 0)
+        return fail(WQ_ERR_CUDA, "%s: clearing the scale failed: %s", what, cudaGetErrorString(cudaGetLastError()));
+    return check_launch(what);
+}
+
+size_t wq_gemm_w8a8_fp8_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    return wq::gemm_fp8_workspace_bytes(M, N, K);
+}
+
+int wq_gemm_w8a8_fp8(const uint8_t *xq, const float *xscale, int64_t M, int64_t N, int64_t K, const uint8_t *wq_,
+                     const float *wscales, uint16_t *y, void *workspace, size_t ws_bytes, void *stream)
+{
+    g_last_error.clear();
+    const char *what = "wq_gemm_w8a8_fp8";
+    if (!xq || !xscale || !wq_ || !wscales || !y) return fail(WQ_ERR_ARG, "%s: null pointer", what);
+    if (M <= 0 || N <= 0 || K <= 0) return fail(WQ_ERR_ARG, "%s: M, N and K must be positive", what);
+    if (K % 128 != 0) return fail(WQ_ERR_SHAPE, "%s: need K %% 128 == 0 (K=%lld)", what, (long long)K);
+    if (M > 0x7fffffffLL || N > 0x7fffffffLL) return fail(WQ_ERR_SHAPE, "%s: M or N too large", what);
+    if (!aligned16(xq) || !aligned16(wq_) || !aligned16(wscales) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(xscale) & 3u) != 0)
+        return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned (xscale 4-byte)", what);
+    const uint64_t yb = span(M, N, 2);
+    if (overlap(y, yb, xq, span(M, K, 1)) || overlap(y, yb, wq_, span(N, K, 1)) || overlap(y, yb, wscales, span(N, 1, 4)) ||
+        overlap(y, yb, xscale, 4))
+        return fail(WQ_ERR_ARG, "%s: y overlaps an input", what);
+    const size_t need = wq::gemm_fp8_workspace_bytes(M, N, K);
+    if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+        return fail(WQ_ERR_WORKSPACE, "%s: need %zu workspace bytes", what, need);
+    int *status = status_word();
+    if (!status) return fail(WQ_ERR_CUDA, "%s: no device status word", what);
+    if (wq::launch_gemm_w8a8_fp8(xq, xscale, M, N, K, wq_, wscales, y, workspace, status,
+                                 static_cast<cudaStream_t>(stream)) != 0)
+        return fail(WQ_ERR_CUDA, "%s: tensor map encoding failed", what);
+    return check_launch(what);
+}
+
+size_t wq_nvfp4_scale_bytes(int64_t N, int64_t K)
+{
+    if (N <= 0 || K <= 0 || K % 64 != 0) return 0;
+    return wq::nvfp4_scale_bytes(N, K);
+}
+
+int wq_quantize_nvfp4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, uint8_t *codes,
+                      uint8_t *block_scales, float *tensor_scale, void *stream)
+{
+    g_last_error.clear();
+    const char *what = "wq_quantize_nvfp4";
+    if (!w || !codes || !block_scales || !tensor_scale) return fail(WQ_ERR_ARG, "%s: null pointer", what);
+    if (N <= 0 || K <= 0 || ldw <= 0) return fail(WQ_ERR_ARG, "%s: N, K and ldw must be positive", what);
+    if (wtype != WQ_F32 && wtype != WQ_BF16) return fail(WQ_ERR_UNSUPPORTED, "%s: wtype %d", what, wtype);
+    if (K % 64 != 0 || ldw < K)
+        return fail(WQ_ERR_SHAPE, "%s: need K %% 64 == 0 and ldw >= K (K=%lld ldw=%lld)", what, (long long)K,
+                    (long long)ldw);
+    if (N > 0x7fffffffLL) return fail(WQ_ERR_SHAPE, "%s: N too large", what);
+    if (ldw % 8 != 0 || !aligned16(w) || !aligned16(codes) || !aligned16(block_scales) ||
+        (reinterpret_cast<uintptr_t>(tensor_scale) & 3u) != 0)
+        return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned (tensor_scale 4-byte), ldw %% 8 == 0", what);
+    const uint64_t wb = span(N - 1, ldw, wtype == WQ_F32 ? 4 : 2) + span(1, K, wtype == WQ_F32 ? 4 : 2);
+    const uint64_t cb = span(N, K, 1) / 2, sb = wq::nvfp4_scale_bytes(N, K);
+    if (overlap(codes, cb, w, wb) || overlap(block_scales, sb, w, wb) || overlap(tensor_scale, 4, w, wb) ||
+        overlap(codes, cb, block_scales, sb) || overlap(codes, cb, tensor_scale, 4) ||
+        overlap(block_scales, sb, tensor_scale, 4))
+        return fail(WQ_ERR_ARG, "%s: output buffers overlap the input or each other", what);
+    if (wq::launch_quantize_nvfp4(w, wtype, N, K, ldw, codes, block_scales, tensor_scale,
+                                  static_cast<cudaStream_t>(stream)) != 0)
+        return fail(WQ_ERR_CUDA, "%s: clearing the outputs failed: %s", what, cudaGetErrorString(cudaGetLastError()));
+    return check_launch(what);
+}
+
+size_t wq_gemm_nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    return wq::gemm_nvfp4_workspace_bytes(M, N, K);
+}
+
+int wq_gemm_nvfp4(const uint8_t *xc, const uint8_t *xsf, const float *xts, int64_t M, int64_t N, int64_t K,
+                  const uint8_t *wc, const uint8_t *wsf, const float *wts, uint16_t *y, void *workspace,
+                  size_t ws_bytes, void *stream)
+{
+    g_last_error.clear();
+    const char *what = "wq_gemm_nvfp4";
+    if (!xc || !xsf || !xts || !wc || !wsf || !wts || !y) return fail(WQ_ERR_ARG, "%s: null pointer", what);
+    if (M <= 0 || N <= 0 || K <= 0) return fail(WQ_ERR_ARG, "%s: M, N and K must be positive", what);
+    if (K % 256 != 0) return fail(WQ_ERR_SHAPE, "%s: need K %% 256 == 0 (K=%lld)", what, (long long)K);
+    if (M > 0x7fffffffLL || N > 0x7fffffffLL) return fail(WQ_ERR_SHAPE, "%s: M or N too large", what);
+    if (!aligned16(xc) || !aligned16(xsf) || !aligned16(wc) || !aligned16(wsf) || !aligned16(y) ||
+        (reinterpret_cast<uintptr_t>(xts) & 3u) != 0 || (reinterpret_cast<uintptr_t>(wts) & 3u) != 0)
+        return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned (tensor scales 4-byte)", what);
+    const uint64_t yb = span(M, N, 2);
+    if (overlap(y, yb, xc, span(M, K, 1) / 2) || overlap(y, yb, wc, span(N, K, 1) / 2) ||
+        overlap(y, yb, xsf, wq::nvfp4_scale_bytes(M, K)) || overlap(y, yb, wsf, wq::nvfp4_scale_bytes(N, K)) ||
+        overlap(y, yb, xts, 4) || overlap(y, yb, wts, 4))
+        return fail(WQ_ERR_ARG, "%s: y overlaps an input", what);
+    const size_t need = wq::gemm_nvfp4_workspace_bytes(M, N, K);
+    if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+        return fail(WQ_ERR_WORKSPACE, "%s: need %zu workspace bytes", what, need);
+    int *status = status_word();
+    if (!status) return fail(WQ_ERR_CUDA, "%s: no device status word", what);
+    if (wq::launch_gemm_nvfp4(xc, xsf, xts, M, N, K, wc, wsf, wts, y, workspace, status,
+                              static_cast<cudaStream_t>(stream)) != 0)
+        return fail(WQ_ERR_CUDA, "%s: tensor map encoding failed", what);
+    return check_launch(what);
+}
+
 int wq_device_status(void *stream)
 {
     g_last_error.clear();

@@ -59,6 +59,32 @@ size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
 int launch_gemm_w4a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
                          const uint16_t *z, int g, uint16_t *y, void *workspace, int *status, cudaStream_t st);
 
+// FP8 quantisers (wq_quant_fp8.cu): per output channel, and per tensor (the latter returns -1 if the
+// scale cannot be cleared before its grid-wide maximum).
+void launch_quantize_fp8_rows(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int fmt, uint8_t *q,
+                              float *s, cudaStream_t st);
+int launch_quantize_fp8_tensor(const void *x, int xtype, int64_t count, int fmt, uint8_t *q, float *scale,
+                               cudaStream_t st);
+
+// FP8 W8A8 tcgen05 matmul (wq_gemm_lowp.cu): K % 128 == 0.  Workspace of gemm_fp8_workspace_bytes():
+// per-segment binary32 partials and per-tile counters (zero-filled before first use; the kernel leaves the
+// counters zeroed).  Returns 0, or -1 if a tensor map cannot be encoded.
+size_t gemm_fp8_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int launch_gemm_w8a8_fp8(const uint8_t *xq, const float *xscale, int64_t M, int64_t N, int64_t K, const uint8_t *wq,
+                         const float *wscale, uint16_t *y, void *workspace, int *status, cudaStream_t st);
+
+// NVFP4 quantiser (wq_quant_nvfp4.cu): codes [N][K/2], block scales in the tensor-core atom layout
+// (nvfp4_scale_bytes(N, K) bytes, rows padded to 128), binary32 tensor scale.  Returns -1 if a clear fails.
+size_t nvfp4_scale_bytes(int64_t N, int64_t K);
+int launch_quantize_nvfp4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, uint8_t *codes, uint8_t *sf,
+                          float *tscale, cudaStream_t st);
+
+// NVFP4 W4A4 tcgen05 matmul (wq_gemm_lowp.cu): K % 256 == 0.  Workspace as the FP8 matmul's.
+size_t gemm_nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int launch_gemm_nvfp4(const uint8_t *xc, const uint8_t *xsf, const float *xts, int64_t M, int64_t N, int64_t K,
+                      const uint8_t *wc, const uint8_t *wsf, const float *wts, uint16_t *y, void *workspace,
+                      int *status, cudaStream_t st);
+
 // Error reporting and the bounded-wait status word, for entry points outside wq_api.cu.
 int record_error(int status, const char *msg);
 void clear_error();

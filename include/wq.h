@@ -66,6 +66,10 @@ extern "C" {
 #define WQ_F32 0
 #define WQ_BF16 1
 
+/* FP8 formats: E4M3 (range +-448) and E5M2 (range +-57,344). */
+#define WQ_FP8_E4M3 0
+#define WQ_FP8_E5M2 1
+
 /* Text for a status code (static storage; never NULL). */
 const char *wq_status_str(int status);
 
@@ -206,6 +210,119 @@ int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint
 int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *qweight,
                   const uint16_t *scales, int g, uint16_t *y, void *workspace, size_t ws_bytes,
                   void *stream);
+
+/*
+ * FP8 quantisation with one binary32 scale per output channel (row)
+ * ("Quantization for LLM inference: FP8, INT4 (GPTQ, AWQ) and GGUF", section
+ * "FP8: the Hopper/Blackwell datacenter format": E4M3 = 4 exponent and 3
+ * mantissa bits, range +-448; E5M2 = 5 and 2, range +-57,344).
+ *
+ *   w       [N][ldw] of WQ_F32 or WQ_BF16
+ *   fmt     WQ_FP8_E4M3 or WQ_FP8_E5M2
+ *   qweight [N][K] FP8 codes (sign, exponent with bias 2^(e-1) - 1, mantissa;
+ *           subnormals kept; E4M3 has no infinities)
+ *   scales  [N] binary32
+ *
+ * Per row, in binary32:
+ *   s    = max|w| / max_fmt; if s == 0: s = 1
+ *   code = nearest FP8 value to w / s, ties to the even code, finite values
+ *          beyond the range saturated to +-max_fmt
+ * Requirements: as wq_quantize_int4 (without g); fmt one of the two formats
+ * (WQ_ERR_UNSUPPORTED otherwise).
+ */
+int wq_quantize_fp8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, int fmt, uint8_t *qweight,
+                    float *scales, void *stream);
+
+/*
+ * FP8 quantisation of a whole tensor with one scale: the dynamic per-tensor
+ * scaling of the activations of an FP8 W8A8 matmul (same page and section).
+ *
+ *   x      [M][K] dense, WQ_F32 or WQ_BF16 (xtype)
+ *   q      [M][K] FP8 codes
+ *   scale  one binary32 value on the device: s = max|x| / max_fmt (1 if 0)
+ * Arithmetic as wq_quantize_fp8 with the tensor as one row.  Launches a
+ * clear of *scale and three kernels (maximum, encode, scale); *scale holds
+ * the maximum in between, so read it only after the call's work completes.
+ * Requirements: M, K >= 1, K % 32 == 0; x, q 16-byte aligned, scale 4-byte
+ * aligned; q and scale must not overlap x or each other.
+ */
+int wq_quantize_fp8_tensor(const void *x, int xtype, int64_t M, int64_t K, int fmt, uint8_t *q, float *scale,
+                           void *stream);
+
+/* Bytes of device workspace wq_gemm_w8a8_fp8 needs for this shape (same contract as
+ * wq_gemm_workspace_bytes: zero-filled once, reusable after calls that complete normally). */
+size_t wq_gemm_w8a8_fp8_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * FP8 W8A8 matmul on the tensor cores (same page and section: FP8 weights and
+ * activations, multiplied by the tensor cores directly).
+ *
+ *   xq, xscale   [M][K] E4M3 codes and their per-tensor scale (one binary32
+ *                value on the device), as from wq_quantize_fp8_tensor
+ *   wq, wscales  [N][K] E4M3 codes and [N] binary32 scales, as from
+ *                wq_quantize_fp8
+ *   y            [M][N] bf16,
+ *                y[m][n] = bf16((sum_k e4m3(xq[m][k]) * e4m3(wq[n][k])) * xscale * wscales[n])
+ * The products are exact and accumulate in binary32 (tcgen05 kind::f8f6f4);
+ * split-K partials are combined in a fixed order, so repeated calls give
+ * identical bytes.  |y - y_exact| <= 4e-3 * sum_k |x_hat * w_hat| on the
+ * inputs this library is tested on.
+ * Requirements: M, N >= 1; K >= 128, K % 128 == 0; xq, wq, wscales, y 16-byte
+ * aligned, xscale 4-byte aligned; workspace of
+ * wq_gemm_w8a8_fp8_workspace_bytes bytes; y must not overlap an input.
+ */
+int wq_gemm_w8a8_fp8(const uint8_t *xq, const float *xscale, int64_t M, int64_t N, int64_t K, const uint8_t *wq,
+                     const float *wscales, uint16_t *y, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * NVFP4 quantisation ("Quantization Methods Compared: INT8, GPTQ, AWQ, FP8,
+ * FP4 and KV-Cache Quantization", section "Hardware, formats and the
+ * roofline": 4-bit values, one E4M3 scale per 16 values, one fp32 tensor
+ * scale, 4.5 bits per value; "Quantization for LLM inference ...", section
+ * "Microscaling: NVFP4 and MXFP4").  The 4-bit values are E2M1 (0, 0.5, 1,
+ * 1.5, 2, 3, 4, 6 and their negatives).  In binary32, every division IEEE:
+ *   st   = max|w over the whole tensor| / (6 * 448)      (1 if that is 0)
+ *   sb   = E4M3 code of ((max|w over the block of 16| / 6) / st)
+ *   code = nearest E2M1 value to w / (e4m3(sb) * st), ties to the even code,
+ *          saturated at +-6 (0 when e4m3(sb) * st == 0)
+ *
+ *   w             [N][ldw] of WQ_F32 or WQ_BF16 (weights, or activations
+ *                 [M][K] for the activation operand)
+ *   codes         [N][K/2] bytes, value 2j of a row in bits 0-3 of byte j
+ *   block_scales  wq_nvfp4_scale_bytes(N, K) bytes: E4M3 codes in the layout
+ *                 the tensor cores read (512-byte atoms of 128 rows x 64
+ *                 values of K; the scale of row r, block b sits at byte
+ *                 16 (r % 32) + 4 ((r % 128) / 32) + (b % 4) of atom
+ *                 (r / 128) * (K / 64) + b / 4); rows past N hold 0
+ *   tensor_scale  one binary32 value on the device (holds the maximum while
+ *                 the call's kernels run; read it after they complete)
+ * Requirements: N >= 1; K >= 64, K % 64 == 0; ldw >= K, ldw % 8 == 0; w,
+ * codes and block_scales 16-byte aligned, tensor_scale 4-byte aligned; no
+ * output overlaps w or another output.
+ */
+size_t wq_nvfp4_scale_bytes(int64_t N, int64_t K);
+int wq_quantize_nvfp4(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw, uint8_t *codes,
+                      uint8_t *block_scales, float *tensor_scale, void *stream);
+
+/* Bytes of device workspace wq_gemm_nvfp4 needs for this shape (contract as wq_gemm_workspace_bytes). */
+size_t wq_gemm_nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * NVFP4 W4A4 matmul on the tensor cores with the block scales applied inside
+ * the MMA (tcgen05.mma kind::mxf4nvf4, one E4M3 scale per 16 values):
+ *   y[m][n] = bf16( (sum_b bx[m][b] bw[n][b] sum_{k in block b} e2m1(x[m][k]) e2m1(w[n][k]))
+ *                   * x_tensor_scale * w_tensor_scale )
+ * with both operands as produced by wq_quantize_nvfp4.  Products and their
+ * block scalings are exact, sums binary32; split-K partials combine in a
+ * fixed order.  |y - y_exact| <= 4e-3 * sum_k |x_hat * w_hat| on the inputs
+ * this library is tested on.
+ * Requirements: M, N >= 1; K >= 256, K % 256 == 0; every pointer 16-byte
+ * aligned except the two tensor scales (4-byte); workspace of
+ * wq_gemm_nvfp4_workspace_bytes bytes; y must not overlap an input.
+ */
+int wq_gemm_nvfp4(const uint8_t *x_codes, const uint8_t *x_block_scales, const float *x_tensor_scale, int64_t M,
+                  int64_t N, int64_t K, const uint8_t *w_codes, const uint8_t *w_block_scales,
+                  const float *w_tensor_scale, uint16_t *y, void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * W4A16 matmul for callers that cannot allocate device memory.  The pages

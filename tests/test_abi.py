@@ -206,3 +206,39 @@ def test_gemm_w4a16_noalloc_rejects_overlap_and_oversize(L):
     # is checked here (the GPU test runs the exact-limit shape).
     assert _g4n(L, M=16, N=32753, K=256) == wq.WQ_ERR_WORKSPACE
     assert "scratch" in wq.wq_last_error()
+
+
+# ---- FP8 and NVFP4 entry points: host-side refusals (no launch) ----
+
+def test_fp8_and_nvfp4_entry_points_reject(L):
+    w, q, s, x, y = _bufs(5)
+    # wq_quantize_fp8(w, wtype, N, K, ldw, fmt, q, s)
+    assert L.wq_quantize_fp8(None, 1, 4, 256, 256, 0, q, s, None) == wq.WQ_ERR_ARG
+    assert L.wq_quantize_fp8(w, 1, 4, 256, 256, 2, q, s, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_quantize_fp8(w, 3, 4, 256, 256, 0, q, s, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_quantize_fp8(w, 1, 4, 96 + 8, 104, 0, q, s, None) == wq.WQ_ERR_SHAPE
+    assert L.wq_quantize_fp8(w, 1, 4, 256, 128, 0, q, s, None) == wq.WQ_ERR_SHAPE
+    assert L.wq_quantize_fp8(w + 2, 1, 4, 256, 256, 0, q, s, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_quantize_fp8(w, 1, 4, 256, 256, 0, w + 256, s, None) == wq.WQ_ERR_ARG
+    # wq_quantize_fp8_tensor(x, xtype, M, K, fmt, q, scale)
+    assert L.wq_quantize_fp8_tensor(x, 1, 0, 256, 0, q, s, None) == wq.WQ_ERR_ARG
+    assert L.wq_quantize_fp8_tensor(x, 1, 2, 48, 0, q, s, None) == wq.WQ_ERR_SHAPE
+    assert L.wq_quantize_fp8_tensor(x, 1, 2, 256, 0, q, s + 2, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_quantize_fp8_tensor(x, 1, 2, 256, 0, q, x + 64, None) == wq.WQ_ERR_ARG
+    # wq_gemm_w8a8_fp8(xq, xs, M, N, K, wq, ws, y, ws, wsb)
+    assert L.wq_gemm_w8a8_fp8(x, s, 4, 128, 192, w, s, y, None, 0, None) == wq.WQ_ERR_SHAPE
+    assert L.wq_gemm_w8a8_fp8(x, None, 4, 128, 256, w, s, y, None, 0, None) == wq.WQ_ERR_ARG
+    assert L.wq_gemm_w8a8_fp8(x, s, 4, 128, 256, w, s, x + 32, None, 0, None) == wq.WQ_ERR_ARG
+    assert L.wq_gemm_w8a8_fp8(x, s + 1, 4, 128, 256, w, s, y, None, 0, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_gemm_w8a8_fp8(x, s, 4, 128, 256, w, s, y, None, 0, None) == wq.WQ_ERR_WORKSPACE
+    # wq_quantize_nvfp4(w, wtype, N, K, ldw, codes, sf, ts)
+    assert wq.wq_nvfp4_scale_bytes(130, 256) == 256 * 16 and wq.wq_nvfp4_scale_bytes(1, 96) == 0
+    assert L.wq_quantize_nvfp4(w, 1, 4, 96, 96, q, s, y, None) == wq.WQ_ERR_SHAPE
+    assert L.wq_quantize_nvfp4(w, 1, 4, 128, 128, q, s, None, None) == wq.WQ_ERR_ARG
+    assert L.wq_quantize_nvfp4(w, 1, 4, 128, 128, q, s + 8, y, None) == wq.WQ_ERR_ALIGN
+    assert L.wq_quantize_nvfp4(w, 1, 4, 128, 128, q, q + 64, y, None) == wq.WQ_ERR_ARG
+    # wq_gemm_nvfp4(xc, xsf, xts, M, N, K, wc, wsf, wts, y, ws, wsb)
+    assert L.wq_gemm_nvfp4(x, x + 4096, s, 4, 128, 128, w, w + 65536, s, y, None, 0, None) == wq.WQ_ERR_SHAPE
+    assert L.wq_gemm_nvfp4(x, x + 4096, s, 4, 128, 256, w, w + 65536, s, y, None, 0, None) == wq.WQ_ERR_WORKSPACE
+    assert L.wq_gemm_nvfp4(x, x + 4096, s, 4, 128, 256, w, w + 65536, s, w + 65536, None, 0, None) == wq.WQ_ERR_ARG
+    assert L.wq_gemm_nvfp4(x, x + 4100, s, 4, 128, 256, w, w + 65536, s, y, None, 0, None) == wq.WQ_ERR_ALIGN
