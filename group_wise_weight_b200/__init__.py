@@ -94,6 +94,12 @@ def lib():
         L.wq_gemm_nvfp4_workspace_bytes.restype = SZ
         L.wq_gemm_nvfp4.argtypes = [P, P, P, I64, I64, I64, P, P, P, P, P, SZ, P]
         L.wq_gemm_nvfp4.restype = I
+        L.wq_decode_attention_workspace_bytes.argtypes = [I64, I64, I64]
+        L.wq_decode_attention_workspace_bytes.restype = SZ
+        L.wq_decode_attention_int4.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, P, P, SZ, P]
+        L.wq_decode_attention_int4.restype = I
+        L.wq_decode_attention_fp8.argtypes = [P, P, P, P, P, P, I64, I64, I64, I64, I64, P, P, SZ, P]
+        L.wq_decode_attention_fp8.restype = I
         _lib = L
     return _lib
 
@@ -418,3 +424,57 @@ def wq_gemm_nvfp4(x_codes: torch.Tensor, x_scales: torch.Tensor, x_tscale: torch
                                workspace.data_ptr() if workspace is not None else None, ws_bytes,
                                _stream_handle(stream)))
     return y
+
+
+def wq_decode_attention_workspace_bytes(B: int, T: int, H: int) -> int:
+    return int(lib().wq_decode_attention_workspace_bytes(int(B), int(T), int(H)))
+
+
+def _attention_out(q: torch.Tensor, lengths: torch.Tensor, o, workspace, B: int, T: int, H: int):
+    if q.dtype != torch.bfloat16 or q.dim() != 3:
+        raise TypeError("q must be a bfloat16 [B][Hq][D] tensor")
+    if lengths.dtype != torch.int32 or lengths.numel() != B:
+        raise TypeError("lengths must be an int32 tensor of B values")
+    _dense(q, "q")
+    _dense(lengths, "lengths")
+    o = torch.empty(q.shape, dtype=torch.float32, device=q.device) if o is None else o
+    _dense(o, "o")
+    need = wq_decode_attention_workspace_bytes(B, T, H)
+    workspace = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    return o, workspace
+
+
+def wq_decode_attention_int4(q: torch.Tensor, k_codes: torch.Tensor, k_scales: torch.Tensor, k_zeros: torch.Tensor,
+                             v_codes: torch.Tensor, v_scales: torch.Tensor, v_zeros: torch.Tensor,
+                             lengths: torch.Tensor, o=None, workspace=None, stream=None) -> torch.Tensor:
+    """Decode attention over an int4 KV cache.  q [B][Hq][128] bf16; codes [B][T][H][64] uint8; scales and
+    zero-points [B][T][H] (any shape with B*T*H values) bf16; lengths int32 [B].  Returns o float32
+    [B][Hq][128]."""
+    B, T, H = k_codes.shape[0], k_codes.shape[1], k_codes.shape[2]
+    o, workspace = _attention_out(q, lengths, o, workspace, B, T, H)
+    for t, n in ((k_codes, "k_codes"), (v_codes, "v_codes"), (k_scales, "k_scales"), (k_zeros, "k_zeros"),
+                 (v_scales, "v_scales"), (v_zeros, "v_zeros")):
+        _dense(t, n)
+    _check(lib().wq_decode_attention_int4(_dev(q, "q"), _dev(k_codes, "k_codes"), _dev(k_scales, "k_scales"),
+                                          _dev(k_zeros, "k_zeros"), _dev(v_codes, "v_codes"),
+                                          _dev(v_scales, "v_scales"), _dev(v_zeros, "v_zeros"),
+                                          _dev(lengths, "lengths"), B, T, H, q.shape[1], q.shape[2], _dev(o, "o"),
+                                          workspace.data_ptr(), workspace.numel(), _stream_handle(stream)))
+    return o
+
+
+def wq_decode_attention_fp8(q: torch.Tensor, k_codes: torch.Tensor, k_scale: torch.Tensor, v_codes: torch.Tensor,
+                            v_scale: torch.Tensor, lengths: torch.Tensor, o=None, workspace=None,
+                            stream=None) -> torch.Tensor:
+    """Decode attention over an fp8 (E4M3, one scale per tensor) KV cache.  q [B][Hq][128] bf16; codes
+    [B][T][H][128] uint8; k_scale, v_scale float32 [1] on the device; lengths int32 [B].  Returns o float32
+    [B][Hq][128]."""
+    B, T, H = k_codes.shape[0], k_codes.shape[1], k_codes.shape[2]
+    o, workspace = _attention_out(q, lengths, o, workspace, B, T, H)
+    for t, n in ((k_codes, "k_codes"), (v_codes, "v_codes")):
+        _dense(t, n)
+    _check(lib().wq_decode_attention_fp8(_dev(q, "q"), _dev(k_codes, "k_codes"), _dev(k_scale, "k_scale"),
+                                         _dev(v_codes, "v_codes"), _dev(v_scale, "v_scale"), _dev(lengths, "lengths"),
+                                         B, T, H, q.shape[1], q.shape[2], _dev(o, "o"), workspace.data_ptr(),
+                                         workspace.numel(), _stream_handle(stream)))
+    return o

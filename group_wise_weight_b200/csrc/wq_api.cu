@@ -410,6 +410,72 @@ int wq_gemm_nvfp4(const uint8_t *xc, const uint8_t *xsf, const float *xts, int64
     return check_launch(what);
 }
 
+size_t wq_decode_attention_workspace_bytes(int64_t B, int64_t T, int64_t H)
+{
+    if (B <= 0 || T <= 0 || H <= 0) return 0;
+    return wq::kv_attn_workspace_bytes(B, T, H);
+}
+
+namespace {
+
+int check_attention(const char *what, bool fp8, const void *q, const void *kc, const void *ks, const void *kz,
+                    const void *vc, const void *vs, const void *vz, const void *lengths, int64_t B, int64_t T,
+                    int64_t H, int64_t Hq, int64_t D, const void *o, const void *ws, size_t ws_bytes)
+{
+    if (!q || !kc || !ks || !vc || !vs || !lengths || !o || (!fp8 && (!kz || !vz)))
+        return fail(WQ_ERR_ARG, "%s: null pointer", what);
+    if (B <= 0 || T <= 0 || H <= 0 || Hq <= 0 || D <= 0)
+        return fail(WQ_ERR_ARG, "%s: B, T, H, Hq and D must be positive", what);
+    if (D != 128 || Hq % H != 0 || Hq / H > 8)
+        return fail(WQ_ERR_UNSUPPORTED, "%s: needs D == 128 and Hq a multiple of H with Hq / H <= 8 (D=%lld H=%lld Hq=%lld)",
+                    what, (long long)D, (long long)H, (long long)Hq);
+    if (B > 65535 || T > 0x7fffffffLL / 2 || H > 65535 || B * T * H > 0x7fffffffffffLL)
+        return fail(WQ_ERR_SHAPE, "%s: B, T or H too large", what);
+    const bool al = aligned16(q) && aligned16(kc) && aligned16(vc) && aligned16(lengths) && aligned16(o) &&
+                    (fp8 ? ((reinterpret_cast<uintptr_t>(ks) & 3u) == 0 && (reinterpret_cast<uintptr_t>(vs) & 3u) == 0)
+                         : (aligned16(ks) && aligned16(kz) && aligned16(vs) && aligned16(vz)));
+    if (!al) return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned (fp8 scales 4-byte)", what);
+    const uint64_t ob = span(B, Hq, D * 4), cb = span(B * T, H, fp8 ? D : D / 2), pb = fp8 ? 4 : span(B * T, H, 2);
+    if (overlap(o, ob, q, span(B, Hq, D * 2)) || overlap(o, ob, kc, cb) || overlap(o, ob, vc, cb) ||
+        overlap(o, ob, ks, pb) || overlap(o, ob, vs, pb) || overlap(o, ob, kz, fp8 ? 0 : pb) ||
+        overlap(o, ob, vz, fp8 ? 0 : pb) || overlap(o, ob, lengths, span(B, 4, 1)))
+        return fail(WQ_ERR_ARG, "%s: o overlaps an input", what);
+    const size_t need = wq::kv_attn_workspace_bytes(B, T, H);
+    if (!ws || ws_bytes < need || !aligned16(ws)) return fail(WQ_ERR_WORKSPACE, "%s: need %zu workspace bytes", what, need);
+    if (overlap(ws, need, o, ob)) return fail(WQ_ERR_ARG, "%s: the workspace overlaps o", what);
+    return WQ_OK;
+}
+
+}  // namespace
+
+int wq_decode_attention_int4(const uint16_t *q, const uint8_t *kc, const uint16_t *ks, const uint16_t *kz,
+                             const uint8_t *vc, const uint16_t *vs, const uint16_t *vz, const int32_t *lengths,
+                             int64_t B, int64_t T, int64_t H, int64_t Hq, int64_t D, float *o, void *workspace,
+                             size_t ws_bytes, void *stream)
+{
+    g_last_error.clear();
+    const char *what = "wq_decode_attention_int4";
+    const int rc = check_attention(what, false, q, kc, ks, kz, vc, vs, vz, lengths, B, T, H, Hq, D, o, workspace, ws_bytes);
+    if (rc != WQ_OK) return rc;
+    wq::launch_kv_attn(false, q, kc, ks, kz, nullptr, vc, vs, vz, nullptr, lengths, B, T, H, Hq, o, workspace,
+                       static_cast<cudaStream_t>(stream));
+    return check_launch(what);
+}
+
+int wq_decode_attention_fp8(const uint16_t *q, const uint8_t *kc, const float *ks, const uint8_t *vc, const float *vs,
+                            const int32_t *lengths, int64_t B, int64_t T, int64_t H, int64_t Hq, int64_t D, float *o,
+                            void *workspace, size_t ws_bytes, void *stream)
+{
+    g_last_error.clear();
+    const char *what = "wq_decode_attention_fp8";
+    const int rc = check_attention(what, true, q, kc, ks, nullptr, vc, vs, nullptr, lengths, B, T, H, Hq, D, o,
+                                   workspace, ws_bytes);
+    if (rc != WQ_OK) return rc;
+    wq::launch_kv_attn(true, q, kc, nullptr, nullptr, ks, vc, nullptr, nullptr, vs, lengths, B, T, H, Hq, o,
+                       workspace, static_cast<cudaStream_t>(stream));
+    return check_launch(what);
+}
+
 int wq_device_status(void *stream)
 {
     g_last_error.clear();

@@ -85,6 +85,14 @@ int launch_gemm_nvfp4(const uint8_t *xc, const uint8_t *xsf, const float *xts, i
                       const uint8_t *wc, const uint8_t *wsf, const float *wts, uint16_t *y, void *workspace,
                       int *status, cudaStream_t st);
 
+// Decode attention over an int4 or fp8 KV cache (wq_kv_attn.cu): D = 128, Hq / H <= 8.  Workspace of
+// kv_attn_workspace_bytes() binary32 chunk partials (no zero-fill needed).
+size_t kv_attn_workspace_bytes(int64_t B, int64_t T, int64_t H);
+int launch_kv_attn(bool fp8, const uint16_t *q, const uint8_t *kc, const uint16_t *ks, const uint16_t *kz,
+                   const float *k8s, const uint8_t *vc, const uint16_t *vs, const uint16_t *vz, const float *v8s,
+                   const int *lengths, int64_t B, int64_t T, int64_t H, int64_t Hq, float *o, void *workspace,
+                   cudaStream_t st);
+
 // Error reporting and the bounded-wait status word, for entry points outside wq_api.cu.
 int record_error(int status, const char *msg);
 void clear_error();

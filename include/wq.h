@@ -325,6 +325,47 @@ int wq_gemm_nvfp4(const uint8_t *x_codes, const uint8_t *x_block_scales, const f
                   const float *w_tensor_scale, uint16_t *y, void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Decode attention over a quantised KV cache: one new query token per
+ * sequence against its first lengths[b] cached tokens ("Quantization Methods
+ * Compared: INT8, GPTQ, AWQ, FP8, FP4 and KV-Cache Quantization", section
+ * "Hardware, formats and the roofline": every decode step reads the whole
+ * cache of every sequence; "Quantization for LLM inference: FP8, INT4 (GPTQ,
+ * AWQ) and GGUF", section "KV cache quantization": fp8 caches, and int4
+ * caches in blocks of 128 values).  Scaled dot-product attention:
+ *   score_t = (q_j . k_hat_t) / sqrt(D), p = softmax over t < lengths[b],
+ *   o_j = sum_t p_t v_hat_t,   query head j reading KV head j / (Hq / H);
+ *   lengths[b] == 0 gives o_j = 0 (lengths are clamped to [0, T]).
+ *
+ *   q        [B][Hq][D] bf16
+ *   int4 cache (K and V alike, each vector one block of 128 in the format of
+ *            wq_quantize_int4 with g = 128 applied to the cache viewed as
+ *            [B*T*H][D] rows): codes [B][T][H][D/2] bytes, scales and
+ *            zero-points [B][T][H] bf16; v_hat = s (q - z)
+ *   fp8 cache: E4M3 codes [B][T][H][D] and one binary32 scale per tensor on
+ *            the device, as from wq_quantize_fp8_tensor; v_hat = s e4m3(code)
+ *   lengths  [B] int32 on the device
+ *   o        [B][Hq][D] binary32
+ * Arithmetic: int4 keys and values enter the tensor cores as the exact
+ * integers q - z (bf16), fp8 ones as exact f16 values; scores and sums are
+ * binary32; p times the token's V scale (int4) or p (fp8) is rounded to
+ * bf16 / f16 as the MMA operand.  |o - o_exact| <= 4e-3 * sum_t p_t |v_hat_t|
+ * on the inputs this library is tested on.
+ * Requirements: D == 128 and Hq % H == 0 with Hq / H <= 8
+ * (WQ_ERR_UNSUPPORTED otherwise); B, T, H >= 1; every pointer 16-byte
+ * aligned (the fp8 scales 4-byte); workspace of
+ * wq_decode_attention_workspace_bytes(B, T, H) bytes (no zero-fill needed);
+ * o must not overlap an input.
+ */
+size_t wq_decode_attention_workspace_bytes(int64_t B, int64_t T, int64_t H);
+int wq_decode_attention_int4(const uint16_t *q, const uint8_t *k_codes, const uint16_t *k_scales,
+                             const uint16_t *k_zeros, const uint8_t *v_codes, const uint16_t *v_scales,
+                             const uint16_t *v_zeros, const int32_t *lengths, int64_t B, int64_t T, int64_t H,
+                             int64_t Hq, int64_t D, float *o, void *workspace, size_t ws_bytes, void *stream);
+int wq_decode_attention_fp8(const uint16_t *q, const uint8_t *k_codes, const float *k_scale, const uint8_t *v_codes,
+                            const float *v_scale, const int32_t *lengths, int64_t B, int64_t T, int64_t H, int64_t Hq,
+                            int64_t D, float *o, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * W4A16 matmul for callers that cannot allocate device memory.  The pages
  * have no counterpart: this is an interface variant, not part of the method.
  *

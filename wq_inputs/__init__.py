@@ -157,3 +157,27 @@ def one_signed_weight(N: int, K: int, seed: int, dtype=torch.float32) -> torch.T
     """[N][K] strictly positive draws in every row (|N(0, 0.02)| + 0.01)."""
     g = _gen(seed)
     return (torch.randn(N, K, generator=g).abs() * WEIGHT_STD + 0.01).to(dtype)
+
+
+# KV cache of one layer for the decode-attention read: [B][T][H][D] (sequences, token slots, KV heads,
+# head_dim) bf16, and the decode step's queries [B][Hq][D].  The pages' geometry for the 70B model at batch
+# 128 is H = 8 KV heads, Hq = 64 query heads, D = 128, 8,000-token contexts.
+KV_70B = {"H": 8, "Hq": 64, "D": 128, "B": 128, "T": 8000}
+
+
+def kv_cache(B: int, T: int, H: int, D: int, seed: int, offset: float = 0.0, device="cpu") -> torch.Tensor:
+    """bf16 [B][T][H][D] ~ N(0, 1) (+ offset: with a large offset every vector lies on one side of zero)."""
+    g = _gen(seed + 4_000_037, device)
+    return (torch.randn(B, T, H, D, generator=g, device=device) + offset).to(torch.bfloat16)
+
+
+def queries(B: int, Hq: int, D: int, seed: int, device="cpu") -> torch.Tensor:
+    """bf16 [B][Hq][D] ~ N(0, 1)."""
+    g = _gen(seed + 5_000_011, device)
+    return torch.randn(B, Hq, D, generator=g, device=device).to(torch.bfloat16)
+
+
+def sequence_lengths(B: int, T: int, seed: int) -> torch.Tensor:
+    """int32 [B] uniform in [1, T] (a mix of short and long contexts)."""
+    g = _gen(seed + 6_000_001)
+    return torch.randint(1, T + 1, (B,), generator=g, dtype=torch.int64).to(torch.int32)
