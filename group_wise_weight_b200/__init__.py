@@ -94,6 +94,14 @@ def lib():
         L.wq_gemm_nvfp4_workspace_bytes.restype = SZ
         L.wq_gemm_nvfp4.argtypes = [P, P, P, I64, I64, I64, P, P, P, P, P, SZ, P]
         L.wq_gemm_nvfp4.restype = I
+        L.wq_gemm_w4a16_colscaled_workspace_bytes.argtypes = [I64, I64, I64, I]
+        L.wq_gemm_w4a16_colscaled_workspace_bytes.restype = SZ
+        L.wq_gemm_w4a16_colscaled.argtypes = [P, P, I64, I64, I64, P, P, P, I, P, P, SZ, P]
+        L.wq_gemm_w4a16_colscaled.restype = I
+        L.wq_awq_channel_magnitudes.argtypes = [P, I64, I64, P, P]
+        L.wq_awq_channel_magnitudes.restype = I
+        L.wq_awq_channel_scales.argtypes = [P, I64, ctypes.c_double, P, P]
+        L.wq_awq_channel_scales.restype = I
         L.wq_decode_attention_workspace_bytes.argtypes = [I64, I64, I64]
         L.wq_decode_attention_workspace_bytes.restype = SZ
         L.wq_decode_attention_int4.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, P, P, SZ, P]
@@ -478,3 +486,49 @@ def wq_decode_attention_fp8(q: torch.Tensor, k_codes: torch.Tensor, k_scale: tor
                                          B, T, H, q.shape[1], q.shape[2], _dev(o, "o"), workspace.data_ptr(),
                                          workspace.numel(), _stream_handle(stream)))
     return o
+
+
+def wq_gemm_w4a16_colscaled(x: torch.Tensor, col_scale: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+                            zeros: torch.Tensor, g: int = 128, y=None, workspace=None, stream=None) -> torch.Tensor:
+    """y = bf16(x / col_scale) @ w_hat^T for weights quantised by wq_quantize_int4_scaled with the same col_scale
+    (float32 [K] on CUDA).  bf16 in, bf16 out."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    _dense(x, "x")
+    M, K = x.shape
+    if col_scale.dtype != torch.float32 or col_scale.numel() != K:
+        raise TypeError("col_scale must be a float32 tensor of K values")
+    _dense(col_scale, "col_scale")
+    N = qweight.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dense(y, "y")
+    need = int(lib().wq_gemm_w4a16_colscaled_workspace_bytes(M, N, K, int(g)))
+    workspace, ws_bytes = _workspace(workspace, need, x.device)
+    _check(lib().wq_gemm_w4a16_colscaled(_dev(x, "x"), _dev(col_scale, "col_scale"), M, N, K,
+                                         _dev(qweight, "qweight"), _dev(scales, "scales"), _dev(zeros, "zeros"),
+                                         int(g), _dev(y, "y"), workspace.data_ptr() if workspace is not None else None,
+                                         ws_bytes, _stream_handle(stream)))
+    return y
+
+
+def wq_awq_channel_magnitudes(x: torch.Tensor, magnitudes=None, stream=None) -> torch.Tensor:
+    """Mean |x| per input channel over the rows of x (bf16 [M][K] on CUDA), float64 [K]."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise TypeError("x must be a 2-D bfloat16 tensor")
+    _dense(x, "x")
+    M, K = x.shape
+    magnitudes = torch.empty(K, dtype=torch.float64, device=x.device) if magnitudes is None else magnitudes
+    _check(lib().wq_awq_channel_magnitudes(_dev(x, "x"), M, K, _dev(magnitudes, "magnitudes"),
+                                           _stream_handle(stream)))
+    return magnitudes
+
+
+def wq_awq_channel_scales(magnitudes: torch.Tensor, alpha: float, col_scale=None, stream=None) -> torch.Tensor:
+    """s_c = m_c ** alpha normalised to max * min = 1 (float64 magnitudes [K] on CUDA), float32 [K]."""
+    if magnitudes.dtype != torch.float64 or magnitudes.dim() != 1:
+        raise TypeError("magnitudes must be a 1-D float64 tensor")
+    K = magnitudes.numel()
+    col_scale = torch.empty(K, dtype=torch.float32, device=magnitudes.device) if col_scale is None else col_scale
+    _check(lib().wq_awq_channel_scales(_dev(magnitudes, "magnitudes"), K, float(alpha), _dev(col_scale, "col_scale"),
+                                       _stream_handle(stream)))
+    return col_scale

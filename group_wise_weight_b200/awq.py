@@ -9,46 +9,39 @@ the quantisation; AWQ takes the activation statistics offline, over a calibratio
 
 The scale of channel c is s_c = m_c ** alpha with m_c the mean |x[m][c]| over the calibration rows,
 normalised so that max(s) * min(s) = 1; alpha runs over a grid and the value whose quantised product is
-closest, in squared error over the calibration rows, to the exact product wins.  For each alpha the
-weights are quantised by wq_quantize_int4_scaled (w[n][c] * s_c in binary32 on the GPU) and the
-calibration rows, divided by s and rounded to bf16, go through wq_gemm_w4a16.  The statistics, the exact
-reference product and the squared errors are host-side bookkeeping of this offline search (binary64); the
-decode-time path is unchanged: the layer that produces x is expected to absorb 1 / s, as the pages say
-AWQ's scales are absorbed into neighbouring layers.
+closest, in squared error over the calibration rows, to the exact product wins.  Every step on the data runs
+in libwq's kernels: the channel magnitudes (wq_awq_channel_magnitudes, once) and, for each alpha, the scales
+(wq_awq_channel_scales), the weights w[n][c] * s_c quantised (wq_quantize_int4_scaled) and the calibration
+rows divided by s inside the matmul (wq_gemm_w4a16_colscaled).  The exact reference product and the squared
+errors are the offline search's bookkeeping (binary64 on the host, one reference product per search).  At
+decode time the same col_scale goes to wq_gemm_w4a16_colscaled, or the layer that produces x absorbs 1 / s,
+as the pages say AWQ's scales are absorbed into neighbouring layers.
 """
 from __future__ import annotations
 
 import numpy as np
 import torch
 
-from . import wq_gemm_w4a16, wq_quantize_int4_scaled
+from . import (wq_awq_channel_magnitudes, wq_awq_channel_scales, wq_gemm_w4a16_colscaled,
+               wq_quantize_int4_scaled)
 
 GRID = tuple(i / 20 for i in range(21))
 
 
-def channel_scales(magnitude: np.ndarray, alpha: float) -> np.ndarray:
-    """s_c = m_c ** alpha, normalised to max * min = 1; a silent channel (m_c = 0) takes the smallest
-    positive magnitude.  float32, the precision the weights are scaled in."""
-    m = np.asarray(magnitude, dtype=np.float64)
-    pos = m[m > 0]
-    s = np.where(m > 0, m, pos.min() if pos.size else 1.0) ** alpha
-    return (s / np.sqrt(s.max() * s.min())).astype(np.float32)
-
-
 def search(w: torch.Tensor, x_cal: torch.Tensor, g: int = 128, grid=GRID):
-    """w: [N][K] float32 or bfloat16 on CUDA; x_cal: [M][K] calibration activations (any device).
+    """w: [N][K] float32 or bfloat16 on CUDA; x_cal: [M][K] bf16 calibration activations (any device).
     Returns (alpha, s float32 [K] numpy, errors list aligned with grid)."""
     if not w.is_cuda:
-        raise TypeError("w must be a CUDA tensor (the quantiser and the matmul run on the GPU)")
-    x64 = x_cal.detach().double().cpu().numpy()
-    mag = np.mean(np.abs(x64), axis=0)
-    exact = x64 @ w.detach().double().cpu().numpy().T
-    errors = []
+        raise TypeError("w must be a CUDA tensor (the statistics, quantiser and matmul run on the GPU)")
+    x = x_cal.detach().to(torch.bfloat16).contiguous().to(w.device)
+    mag = wq_awq_channel_magnitudes(x)
+    exact = x.double().cpu().numpy() @ w.detach().double().cpu().numpy().T
+    errors, scales = [], []
     for a in grid:
-        s = channel_scales(mag, a)
-        q, sc, z = wq_quantize_int4_scaled(w, torch.from_numpy(s).to(w.device), g)
-        xs = torch.from_numpy((x64 / s.astype(np.float64)).astype(np.float32)).to(torch.bfloat16).to(w.device)
-        y = wq_gemm_w4a16(xs, q, sc, z, g)
+        s = wq_awq_channel_scales(mag, a)
+        q, sc, z = wq_quantize_int4_scaled(w, s, g)
+        y = wq_gemm_w4a16_colscaled(x, s, q, sc, z, g)
         errors.append(float(np.sum((y.double().cpu().numpy() - exact) ** 2)))
+        scales.append(s)
     best = int(np.argmin(errors))
-    return grid[best], channel_scales(mag, grid[best]), errors
+    return grid[best], scales[best].cpu().numpy(), errors

@@ -144,6 +144,48 @@ int *device_status_word() { return status_word(); }
 
 }  // namespace wq
 
+namespace {
+
+// The W4A16 dispatch after the argument checks.  col_scale, when given, is applied by the M = 1 kernel while
+// it stages x; callers pass it only when gemv_m1_eligible holds.
+int run_w4a16(const char *what, const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *qweight,
+              const uint16_t *scales, const uint16_t *zeros, int g, uint16_t *y, void *workspace, cudaStream_t st,
+              const float *col_scale)
+{
+    if (wq::gemm_tc_eligible(M, N, K, g)) {
+        int *status = status_word();
+        if (!status) return fail(WQ_ERR_CUDA, "%s: no device status word", what);
+        if (wq::launch_gemm_w4a16_tc(x, M, N, K, qweight, scales, zeros, g, y, workspace, status, st) != 0)
+            return fail(WQ_ERR_CUDA, "%s: tensor map encoding failed", what);
+        return check_launch(what);
+    }
+    if (wq::gemv_m1_eligible(M, N, K, g)) {
+        int *status = status_word();
+        if (!status) return fail(WQ_ERR_CUDA, "%s: no device status word", what);
+        const int rc = wq::launch_gemv_w4a16_m1(x, N, K, qweight, scales, zeros, y, workspace, status, st, col_scale);
+        if (rc == -1) return fail(WQ_ERR_CUDA, "%s: tensor map encoding failed", what);
+        return check_launch(what);
+    }
+    if (wq::gemv_tma_eligible(M, N, K, g)) {
+        int *status = status_word();
+        if (!status) return fail(WQ_ERR_CUDA, "%s: no device status word", what);
+        if (wq::launch_gemv_w4a16_tma(x, M, N, K, qweight, scales, zeros, y, workspace, status, st) != 0)
+            return fail(WQ_ERR_CUDA, "%s: tensor map encoding failed", what);
+        return check_launch(what);
+    }
+    wq::launch_gemv_w4a16(x, M, N, K, qweight, scales, zeros, g, y, st);
+    return check_launch(what);
+}
+
+// Bytes of the bf16(x / s) staging area of wq_gemm_w4a16_colscaled (none when the M = 1 kernel applies the
+// scales itself), rounded up to 256.
+size_t colscaled_x_bytes(int64_t M, int64_t N, int64_t K, int g)
+{
+    return wq::gemv_m1_eligible(M, N, K, g) ? 0 : (span(M, K, 2) + 255) / 256 * 256;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *wq_status_str(int status)
@@ -230,30 +272,8 @@ int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint
     const size_t need = wq_gemm_workspace_bytes(M, N, K, g, 4);
     if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
         return fail(WQ_ERR_WORKSPACE, "wq_gemm_w4a16: need %zu workspace bytes", need);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (wq::gemm_tc_eligible(M, N, K, g)) {
-        int *status = status_word();
-        if (!status) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: no device status word");
-        if (wq::launch_gemm_w4a16_tc(x, M, N, K, qweight, scales, zeros, g, y, workspace, status, st) != 0)
-            return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: tensor map encoding failed");
-        return check_launch("wq_gemm_w4a16");
-    }
-    if (wq::gemv_m1_eligible(M, N, K, g)) {
-        int *status = status_word();
-        if (!status) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: no device status word");
-        const int rc = wq::launch_gemv_w4a16_m1(x, N, K, qweight, scales, zeros, y, workspace, status, st);
-        if (rc == -1) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: tensor map encoding failed");
-        return check_launch("wq_gemm_w4a16");
-    }
-    if (wq::gemv_tma_eligible(M, N, K, g)) {
-        int *status = status_word();
-        if (!status) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: no device status word");
-        if (wq::launch_gemv_w4a16_tma(x, M, N, K, qweight, scales, zeros, y, workspace, status, st) != 0)
-            return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: tensor map encoding failed");
-        return check_launch("wq_gemm_w4a16");
-    }
-    wq::launch_gemv_w4a16(x, M, N, K, qweight, scales, zeros, g, y, st);
-    return check_launch("wq_gemm_w4a16");
+    return run_w4a16("wq_gemm_w4a16", x, M, N, K, qweight, scales, zeros, g, y, workspace,
+                     static_cast<cudaStream_t>(stream), nullptr);
 }
 
 int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *qweight,
@@ -473,6 +493,67 @@ int wq_decode_attention_fp8(const uint16_t *q, const uint8_t *kc, const float *k
     if (rc != WQ_OK) return rc;
     wq::launch_kv_attn(true, q, kc, nullptr, nullptr, ks, vc, nullptr, nullptr, vs, lengths, B, T, H, Hq, o,
                        workspace, static_cast<cudaStream_t>(stream));
+    return check_launch(what);
+}
+
+size_t wq_gemm_w4a16_colscaled_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
+{
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    return colscaled_x_bytes(M, N, K, g) + wq_gemm_workspace_bytes(M, N, K, g, 4);
+}
+
+int wq_gemm_w4a16_colscaled(const uint16_t *x, const float *col_scale, int64_t M, int64_t N, int64_t K,
+                            const uint8_t *qweight, const uint16_t *scales, const uint16_t *zeros, int g, uint16_t *y,
+                            void *workspace, size_t ws_bytes, void *stream)
+{
+    g_last_error.clear();
+    const char *what = "wq_gemm_w4a16_colscaled";
+    int rc = check_gemm(what, x, M, N, K, qweight, scales, zeros, g, y, false);
+    if (rc != WQ_OK) return rc;
+    if (!col_scale) return fail(WQ_ERR_ARG, "%s: null col_scale", what);
+    if (!aligned16(col_scale)) return fail(WQ_ERR_ALIGN, "%s: col_scale must be 16-byte aligned", what);
+    if (overlap(y, span(M, N, 2), col_scale, span(K, 4, 1)))
+        return fail(WQ_ERR_ARG, "%s: y overlaps col_scale", what);
+    const size_t xb = colscaled_x_bytes(M, N, K, g), need = xb + wq_gemm_workspace_bytes(M, N, K, g, 4);
+    if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
+        return fail(WQ_ERR_WORKSPACE, "%s: need %zu workspace bytes", what, need);
+    if (need > 0 && (overlap(workspace, need, x, span(M, K, 2)) || overlap(workspace, need, y, span(M, N, 2))))
+        return fail(WQ_ERR_ARG, "%s: the workspace overlaps x or y", what);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (xb == 0)  // the M = 1 kernel divides x by the scales while it stages x
+        return run_w4a16(what, x, M, N, K, qweight, scales, zeros, g, y, workspace, st, col_scale);
+    uint16_t *xs = static_cast<uint16_t *>(workspace);
+    wq::launch_colscale_x(x, M, K, col_scale, xs, st);
+    rc = check_launch(what);
+    if (rc != WQ_OK) return rc;
+    return run_w4a16(what, xs, M, N, K, qweight, scales, zeros, g, y, static_cast<uint8_t *>(workspace) + xb, st,
+                     nullptr);
+}
+
+int wq_awq_channel_magnitudes(const uint16_t *x, int64_t M, int64_t K, double *magnitudes, void *stream)
+{
+    g_last_error.clear();
+    const char *what = "wq_awq_channel_magnitudes";
+    if (!x || !magnitudes) return fail(WQ_ERR_ARG, "%s: null pointer", what);
+    if (M <= 0 || K <= 0) return fail(WQ_ERR_ARG, "%s: M and K must be positive", what);
+    if (!aligned16(x) || !aligned16(magnitudes)) return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned", what);
+    if (overlap(magnitudes, span(K, 8, 1), x, span(M, K, 2))) return fail(WQ_ERR_ARG, "%s: output overlaps x", what);
+    wq::launch_channel_magnitudes(x, M, K, magnitudes, nullptr, static_cast<cudaStream_t>(stream));
+    return check_launch(what);
+}
+
+int wq_awq_channel_scales(const double *magnitudes, int64_t K, double alpha, float *col_scale, void *stream)
+{
+    g_last_error.clear();
+    const char *what = "wq_awq_channel_scales";
+    if (!magnitudes || !col_scale) return fail(WQ_ERR_ARG, "%s: null pointer", what);
+    if (K <= 0) return fail(WQ_ERR_ARG, "%s: K must be positive", what);
+    if (!(alpha >= 0.0 && alpha <= 1.0)) return fail(WQ_ERR_ARG, "%s: alpha must lie in [0, 1]", what);
+    if (!aligned16(magnitudes) || !aligned16(col_scale))
+        return fail(WQ_ERR_ALIGN, "%s: pointers must be 16-byte aligned", what);
+    if (overlap(col_scale, span(K, 4, 1), magnitudes, span(K, 8, 1)))
+        return fail(WQ_ERR_ARG, "%s: output overlaps the magnitudes", what);
+    wq::launch_channel_scales(magnitudes, K, alpha, col_scale, static_cast<cudaStream_t>(stream));
     return check_launch(what);
 }
 

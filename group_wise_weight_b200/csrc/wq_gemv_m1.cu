@@ -182,6 +182,20 @@ __host__ __device__ __forceinline__ int64_t cta_of(int64_t u, int64_t units, int
     return ((u + 1) * B - 1) / units;
 }
 
+// Eight activations divided by their input channels' scales: bf16(x / s) with an IEEE binary32 quotient
+// (the activation side of per-input-channel scaling, wq_gemm_w4a16_colscaled).
+__device__ __forceinline__ uint4 colscale8(uint4 v, const float *s)
+{
+    const float4 s0 = __ldg(reinterpret_cast<const float4 *>(s)), s1 = __ldg(reinterpret_cast<const float4 *>(s) + 1);
+    const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        w[i] = pack_bf16x2(__fdiv_rn(__uint_as_float(w[i] << 16), sc[2 * i]),
+                           __fdiv_rn(__uint_as_float(w[i] & 0xffff0000u), sc[2 * i + 1]));
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // Bounded wait used on the drain path (ignores the abort flag).
 __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity, int *status)
 {
@@ -195,7 +209,8 @@ __global__ void __maxnreg__(96)
 gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                      const __grid_constant__ CUtensorMap zmap, const uint16_t *__restrict__ x, int N, int K,
                      uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ cnt, int max_segs,
-                     int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic)
+                     int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic,
+                     const float *__restrict__ col_scale)
 {
     extern __shared__ __align__(1024) uint8_t m1_raw[];
     // TMA destinations want 128-byte (we keep 1024-byte) alignment: align the base explicitly
@@ -384,7 +399,8 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         mbar_wait(xbar, 0, status, flags);
         for (int c = tid; c < K / 8; c += kC * 32) {
             {
-                const uint4 v = xp[c];
+                uint4 v = xp[c];
+                if (col_scale) v = colscale8(v, col_scale + 8 * c);
                 uint4 pr;
                 pr.x = __byte_perm(v.x, v.z, 0x5410);  // (x0, x4)
                 pr.y = __byte_perm(v.x, v.z, 0x7632);  // (x1, x5)
@@ -576,7 +592,8 @@ size_t gemv_m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
 }
 
 int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
-                         const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st)
+                         const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st,
+                         const float *col_scale)
 {
     // packed codes seen as (64-byte group slice, row, group): strides K/2 bytes (row) and 64 bytes (group)
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
@@ -621,7 +638,7 @@ int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, gemv_w4a16_m1_kernel, wmap, smap, zmap, x, (int)N, (int)K, y, ws, cnt, max_segs,
-                           status, 0x000F000Fu, 0x43004300u) != cudaSuccess)
+                           status, 0x000F000Fu, 0x43004300u, col_scale) != cudaSuccess)
         return -2;
     return 0;
 }

@@ -36,8 +36,10 @@ void launch_gemv_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const
 // launch fails.
 bool gemv_m1_eligible(int64_t M, int64_t N, int64_t K, int g);
 size_t gemv_m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
+// col_scale (optional, binary32 [K]): the kernel stages bf16(x / col_scale) instead of x.
 int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
-                         const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st);
+                         const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st,
+                         const float *col_scale = nullptr);
 
 // TMA-pipelined W4A16 for group 128 and M <= 16 (wq_gemv_tma.cu).  Needs a
 // workspace of gemv_tma_workspace_bytes() (zero-filled before first use; the
@@ -92,6 +94,15 @@ int launch_kv_attn(bool fp8, const uint16_t *q, const uint8_t *kc, const uint16_
                    const float *k8s, const uint8_t *vc, const uint16_t *vs, const uint16_t *vz, const float *v8s,
                    const int *lengths, int64_t B, int64_t T, int64_t H, int64_t Hq, float *o, void *workspace,
                    cudaStream_t st);
+
+// x_out[m][k] = bf16(x[m][k] / col_scale[k]) (IEEE binary32 quotient), M rows of K (wq_colscale.cu).
+void launch_colscale_x(const uint16_t *x, int64_t M, int64_t K, const float *col_scale, uint16_t *x_out,
+                       cudaStream_t st);
+// mag64[k] = mean over the M rows of |x[m][k]| (binary64, rows in order; mag, if not null, its binary32
+// rounding), and s[k] = m'[k]^alpha / sqrt(max_k m'^alpha * min_k m'^alpha) in binary64 rounded to binary32,
+// m' = m or the smallest positive m where m == 0 (wq_colscale.cu).
+void launch_channel_magnitudes(const uint16_t *x, int64_t M, int64_t K, double *mag64, float *mag, cudaStream_t st);
+void launch_channel_scales(const double *mag64, int64_t K, double alpha, float *s, cudaStream_t st);
 
 // Error reporting and the bounded-wait status word, for entry points outside wq_api.cu.
 int record_error(int status, const char *msg);

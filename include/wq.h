@@ -212,6 +212,47 @@ int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8
                   void *stream);
 
 /*
+ * W4A16 matmul of column-scaled activations: the activation side of
+ * per-input-channel (AWQ-style) scaling ([P3] "The methods compared": AWQ
+ * scales the salient channels up before quantising and the activations
+ * compensate; [P1C] "The idea": the activations are divided by the same
+ * scales, so the product is unchanged up to the quantisation).
+ *
+ *   y[m][n] = sum_k bf16(x[m][k] / col_scale[k]) * w_hat[n][k]
+ *
+ * with the weights quantised by wq_quantize_int4_scaled with the same
+ * col_scale (binary32 [K], device, 16-byte aligned) and x / col_scale an IEEE
+ * binary32 quotient rounded to bf16.  The M = 1 decode kernel divides while
+ * it stages x (no extra pass); other shapes write the scaled activations to
+ * the front of the workspace first.  Arguments, accuracy and the rest of the
+ * contract as wq_gemm_w4a16, with a workspace of
+ * wq_gemm_w4a16_colscaled_workspace_bytes(M, N, K, g) bytes that must not
+ * overlap x or y.
+ */
+size_t wq_gemm_w4a16_colscaled_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
+int wq_gemm_w4a16_colscaled(const uint16_t *x, const float *col_scale, int64_t M, int64_t N, int64_t K,
+                            const uint8_t *qweight, const uint16_t *scales, const uint16_t *zeros, int g, uint16_t *y,
+                            void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Channel statistics of the offline AWQ-style scale search ([P3] "The methods
+ * compared": AWQ finds the salient channels from activation magnitudes and
+ * searches the scale per channel; the pages give no formula, the reading
+ * here is s_c = m_c^alpha normalised to max(s) * min(s) = 1).
+ *
+ * wq_awq_channel_magnitudes: magnitudes[k] = mean over the M rows of
+ *   |x[m][k]|, binary64, rows summed in order (x [M][K] bf16; magnitudes [K]
+ *   binary64, device).
+ * wq_awq_channel_scales: col_scale[k] = m'^alpha / sqrt(max m'^alpha *
+ *   min m'^alpha) in binary64, rounded once to binary32, with m' = m or, where
+ *   m == 0, the smallest positive magnitude (1 if none); alpha in [0, 1].
+ * Requirements: sizes >= 1, pointers 16-byte aligned, outputs not overlapping
+ * the inputs.
+ */
+int wq_awq_channel_magnitudes(const uint16_t *x, int64_t M, int64_t K, double *magnitudes, void *stream);
+int wq_awq_channel_scales(const double *magnitudes, int64_t K, double alpha, float *col_scale, void *stream);
+
+/*
  * FP8 quantisation with one binary32 scale per output channel (row)
  * ("Quantization for LLM inference: FP8, INT4 (GPTQ, AWQ) and GGUF", section
  * "FP8: the Hopper/Blackwell datacenter format": E4M3 = 4 exponent and 3

@@ -1,6 +1,6 @@
-"""The AWQ search's orchestration on the CPU: the library calls are replaced by the oracle's quantiser and
-matmul (CPU tensors), so the loop, the scales and the bookkeeping run without a GPU.  The GPU run of the
-same search is a parity test in test_gpu_parity.py."""
+"""The AWQ search's orchestration on the CPU: the library calls are replaced by the oracle's statistics,
+quantiser and matmul (CPU tensors), so the loop, the scales and the bookkeeping run without a GPU.  The GPU
+run of the same search is a parity test in test_gpu_parity.py."""
 import numpy as np
 import torch
 
@@ -9,20 +9,36 @@ import wq_inputs
 from oracle import awq as oawq
 
 
+def _fake_magnitudes(x):
+    return torch.from_numpy(oawq.channel_magnitude(x.double().numpy()))
+
+
+def _fake_scales(mag, alpha):
+    return torch.from_numpy(oawq.channel_scales(mag.numpy(), alpha))
+
+
 def _fake_quantize_scaled(w, col_scale, g):
     codes, s, z = oracle.quantize_int4(oawq.scaled_weights(w.float().numpy(), col_scale.numpy()), g)
     return torch.from_numpy(codes), torch.from_numpy(s), torch.from_numpy(z)
 
 
-def _fake_gemm(x, codes, s, z, g):
-    y, _ = oracle.gemm_w4a16(x.double().numpy(), codes.numpy(), s.numpy(), z.numpy(), g)
+def scaled_x(x, s):
+    """bf16(x / s) with a binary32 quotient, as the library's kernels stage it."""
+    q = (x.float().numpy() / s.astype(np.float32)[None, :]).astype(np.float32)
+    return oracle.bf16_value(oracle.bf16_bits(q)).astype(np.float64)
+
+
+def _fake_gemm_colscaled(x, col_scale, codes, s, z, g):
+    y, _ = oracle.gemm_w4a16(scaled_x(x, col_scale.numpy()), codes.numpy(), s.numpy(), z.numpy(), g)
     return torch.from_numpy(y).to(torch.bfloat16)
 
 
 def test_search_orchestration_matches_the_oracle_search(monkeypatch):
     import group_wise_weight_b200.awq as gawq
+    monkeypatch.setattr(gawq, "wq_awq_channel_magnitudes", _fake_magnitudes)
+    monkeypatch.setattr(gawq, "wq_awq_channel_scales", _fake_scales)
     monkeypatch.setattr(gawq, "wq_quantize_int4_scaled", _fake_quantize_scaled)
-    monkeypatch.setattr(gawq, "wq_gemm_w4a16", _fake_gemm)
+    monkeypatch.setattr(gawq, "wq_gemm_w4a16_colscaled", _fake_gemm_colscaled)
 
     class _CudaLike(torch.Tensor):  # the search insists on CUDA weights; the fakes take CPU tensors
         @property

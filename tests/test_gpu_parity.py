@@ -504,25 +504,6 @@ def test_gemm_output_offsets_and_canaries():
     check_y(y.cpu(), y_ref, a_ref)
 
 
-def test_awq_search_on_the_gpu_tracks_the_oracle_search():
-    """The offline AWQ-style search through the library's kernels (column-scaled quantiser, W4A16 matmul)
-    against the oracle's search on the same calibration rows: the per-alpha errors agree up to the bf16
-    rounding of x / s and of y, and the chosen alpha is (within 5 %) the oracle's best."""
-    from group_wise_weight_b200 import awq as gawq
-    from oracle import awq as oawq
-    w = wq_inputs.llm_weight(256, 1024, 411, dtype=torch.float32)
-    x = wq_inputs.activations(48, 1024, 412, channel_seed=411)
-    alpha, s, errors = gawq.search(w.cuda(), x, 128)
-    torch.cuda.synchronize()
-
-    def deq(w32):
-        codes, so, zo = oracle.quantize_int4(w32, 128)
-        return oracle.dequant_int4(codes, so, zo, 128)
-    _, _, o_errors = oawq.search(x.double().numpy(), w.numpy(), deq)
-    assert np.allclose(errors, o_errors, rtol=0.05)
-    assert alpha > 0 and o_errors[gawq.GRID.index(alpha)] <= 1.05 * min(o_errors)
-
-
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_quantize_ragged_last_chunk(dtype):
     """K not a multiple of 256: a warp's last 256-weight chunk of a row runs past K, and the lanes beyond K

@@ -181,3 +181,10 @@ def sequence_lengths(B: int, T: int, seed: int) -> torch.Tensor:
     """int32 [B] uniform in [1, T] (a mix of short and long contexts)."""
     g = _gen(seed + 6_000_001)
     return torch.randint(1, T + 1, (B,), generator=g, dtype=torch.int64).to(torch.int32)
+
+
+def channel_scales(K: int, seed: int, spread: float = 0.5) -> torch.Tensor:
+    """float32 [K] positive per-input-channel scales exp(spread * N(0, 1)) (stand-ins for the scales an
+    activation-aware search produces)."""
+    g = _gen(seed + 7_000_019)
+    return torch.exp(torch.randn(K, generator=g) * spread).float()
