@@ -358,6 +358,195 @@ def sym_int4_row(wq, device, copies=8, reps=5):
             "shape": "K=N=8192 bf16->symmetric int4 g128 (zero-points 8)"}
 
 
+def _time_rotating(calls, reps):
+    """Average device time of one call: the calls (over rotating buffers, together larger than L2) captured
+    in one CUDA graph, replayed reps times between events."""
+    g = graph_of(lambda: [c() for c in calls])
+    g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    e1.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (reps * len(calls))  # us
+
+
+def _w4_copies(wq, N, K, g, copies, seed, device):
+    out = []
+    for c in range(copies):
+        w = wq_inputs.llm_weight(N, K, seed + c, device=device)
+        out.append(wq.wq_quantize_int4(w, g))
+        del w
+    torch.cuda.empty_cache()
+    return out
+
+
+def config_rows(wq, device, peaks, reps=10):
+    """The named configurations other than the 70B step, each with its weights rotated past L2:
+    decode up-projection at M = 1; the batch sweep M in {1, 8, 32, 128} on K = 8192, N = 28672 with the
+    bf16 unquantised matmul (cuBLAS through torch) on the same shapes as the reference point; the
+    granularity variants at K = N = 8192 (INT4 g32 at M = 1, 16; W8A16 per channel at M = 16)."""
+    rows = {}
+    hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    # config 2: K = 4096, N = 14336, M = 1, 13 copies of 31.2 MB (> 3 x L2)
+    K, N = 4096, 14336
+    cps = _w4_copies(wq, N, K, G, 13, 20_000, device)
+    x = wq_inputs.activations(1, K, 2, device=device)
+    y = torch.empty((1, N), dtype=torch.bfloat16, device=device)
+    ws = torch.zeros(max(16, wq.wq_gemm_workspace_bytes(1, N, K, G, 4)), dtype=torch.uint8, device=device)
+    us = _time_rotating([lambda c=c: wq.wq_gemm_w4a16(x, *c, G, y=y, workspace=ws) for c in cps], reps)
+    b = linear_bytes(1, N, K)
+    rows["cfg2_decode_up_m1"] = {"us": round(us, 2), "GB_s": round(b / us / 1e3, 1),
+                                 "frac_hbm": round(b / us / 1e3 / hbm, 3), "ideal_us": round(b / hbm / 1e3, 2),
+                                 "shape": "K=4096 N=14336 M=1 W4A16 g128, 13 weight copies rotated"}
+    # f1: the same shape through the column-scaled entry point (x / s fused into the M = 1 kernel's staging)
+    sc = wq_inputs.channel_scales(K, 2).to(device)
+    us_cs = _time_rotating([lambda c=c: wq.wq_gemm_w4a16_colscaled(x, sc, *c, G, y=y, workspace=ws) for c in cps], reps)
+    rows["f1_colscaled_m1"] = {"us": round(us_cs, 2), "GB_s": round(b / us_cs / 1e3, 1),
+                               "vs_plain": round(us_cs / us, 3),
+                               "shape": "as cfg2, y = bf16(x / s) w_hat, s per input channel"}
+    del cps
+    torch.cuda.empty_cache()
+    # config 3: K = 8192, N = 28672, 4 copies of 124.8 MB; bf16 reference: 1 copy of 470 MB
+    K, N = 8192, 28672
+    cps = _w4_copies(wq, N, K, G, 4, 30_000, device)
+    wb = wq_inputs.llm_weight(N, K, 30_100, device=device)
+    sweep = {}
+    for M in (1, 8, 32, 128):
+        x = wq_inputs.activations(M, K, 3, device=device)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        ws = torch.zeros(max(16, wq.wq_gemm_workspace_bytes(M, N, K, G, 4)), dtype=torch.uint8, device=device)
+        us = _time_rotating([lambda c=c: wq.wq_gemm_w4a16(x, *c, G, y=y, workspace=ws) for c in cps], reps)
+        yb = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        us_bf16 = _time_rotating([lambda: torch.matmul(x, wb.t(), out=yb)], reps)
+        b4, bb = linear_bytes(M, N, K), N * K * 2 + 2 * M * K + 2 * M * N
+        fl = 2.0 * M * N * K
+        sweep[f"M{M}"] = {"w4_us": round(us, 2), "w4_GB_s": round(b4 / us / 1e3, 1), "w4_TF_s": round(fl / us / 1e6, 1),
+                          "w4_frac": round(max(b4 / us / 1e3 / hbm, fl / us / 1e6 / tc), 3),
+                          "bf16_us": round(us_bf16, 2), "bf16_TF_s": round(fl / us_bf16 / 1e6, 1),
+                          "w4_speedup_vs_bf16": round(us_bf16 / us, 2)}
+    rows["cfg3_batch_sweep"] = dict(sweep, shape="K=8192 N=28672 W4A16 g128 (4 copies rotated) vs bf16 "
+                                                 "torch.matmul (cuBLAS, 470 MB weight)")
+    del cps, wb
+    torch.cuda.empty_cache()
+    # config 4: INT4 g32 at M = 1, 16 (10 copies of 41.9 MB); W8A16 per channel at M = 16 (8 copies of 67 MB)
+    K = N = 8192
+    cps = []
+    for c in range(10):
+        w = wq_inputs.block_outlier_weight(N, K, 40_000 + c, device=device)
+        cps.append(wq.wq_quantize_int4(w, 32))
+        del w
+    g32 = {}
+    for M in (1, 16):
+        x = wq_inputs.activations(M, K, 4, device=device)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        ws = torch.zeros(max(16, wq.wq_gemm_workspace_bytes(M, N, K, 32, 4)), dtype=torch.uint8, device=device)
+        us = _time_rotating([lambda c=c: wq.wq_gemm_w4a16(x, *c, 32, y=y, workspace=ws) for c in cps], reps)
+        b = linear_bytes(M, N, K, 32)
+        g32[f"M{M}"] = {"us": round(us, 2), "GB_s": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / hbm, 3)}
+    rows["cfg4_int4_g32"] = dict(g32, shape="K=N=8192 INT4 g32 (5.0 bits stored), 10 copies rotated")
+    del cps
+    torch.cuda.empty_cache()
+    cps8 = []
+    for c in range(8):
+        w = wq_inputs.block_outlier_weight(N, K, 41_000 + c, device=device)
+        cps8.append(wq.wq_quantize_int8(w, None))
+        del w
+    w8 = {}
+    for M in (1, 16):
+        x = wq_inputs.activations(M, K, 4, device=device)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        us = _time_rotating([lambda c=c: wq.wq_gemm_w8a16(x, *c, None, y=y) for c in cps8], reps)
+        b = N * K + 2 * N + 2 * M * K + 2 * M * N
+        w8[f"M{M}"] = {"us": round(us, 2), "GB_s": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / hbm, 3)}
+    rows["cfg4_w8a16_per_channel"] = dict(w8, shape="K=N=8192 INT8 per channel, 8 copies rotated")
+    del cps8
+    torch.cuda.empty_cache()
+    return rows
+
+
+def next_rows(wq, device, peaks, reps=5):
+    """The NEXT rows on the 70B linear shapes at M = 128 (FP8 W8A8, NVFP4 W4A4: weights of one layer's four
+    linears, each shape's copies rotated past L2) and the KV-cache read at the pages' geometry (batch 128,
+    8,000-token contexts, 8 KV heads, 64 query heads, head_dim 128, one layer)."""
+    rows = {}
+    hbm = peaks["hbm_gbs"]
+    M = 128
+    fp8, nv = {}, {}
+    tot_fp8 = tot_nv = 0.0
+    for name, K, N in wq_inputs.FULL70B_LINEARS:
+        copies = max(2, -(-400_000_000 // (N * K)))  # > 3 x L2 of FP8 weights
+        x = wq_inputs.activations(M, K, 5, device=device)
+        qx, sx = wq.wq_quantize_fp8_tensor(x)
+        nx = wq.wq_quantize_nvfp4(x)
+        c8, c4 = [], []
+        for c in range(copies):
+            w = wq_inputs.llm_weight(N, K, 50_000 + c, device=device)
+            c8.append(wq.wq_quantize_fp8(w))
+            c4.append(wq.wq_quantize_nvfp4(w))
+            del w
+        torch.cuda.empty_cache()
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        ws8 = torch.zeros(max(16, wq.wq_gemm_w8a8_fp8_workspace_bytes(M, N, K)), dtype=torch.uint8, device=device)
+        ws4 = torch.zeros(max(16, wq.wq_gemm_nvfp4_workspace_bytes(M, N, K)), dtype=torch.uint8, device=device)
+        us8 = _time_rotating([lambda c=c: wq.wq_gemm_w8a8_fp8(qx, sx, *c, y=y, workspace=ws8) for c in c8], reps)
+        us4 = _time_rotating([lambda c=c: wq.wq_gemm_nvfp4(*nx, *c, y=y, workspace=ws4) for c in c4], reps)
+        fl = 2.0 * M * N * K
+        b8 = N * K + 4 * N + M * K + 2 * M * N
+        b4 = N * K // 2 + N * K // 16 + M * K // 2 + M * K // 16 + 2 * M * N
+        fp8[name] = {"us": round(us8, 2), "TF_s": round(fl / us8 / 1e6, 1), "GB_s": round(b8 / us8 / 1e3, 1),
+                     "frac_hbm": round(b8 / us8 / 1e3 / hbm, 3)}
+        nv[name] = {"us": round(us4, 2), "TF_s": round(fl / us4 / 1e6, 1), "GB_s": round(b4 / us4 / 1e3, 1),
+                    "frac_hbm": round(b4 / us4 / 1e3 / hbm, 3)}
+        tot_fp8 += us8
+        tot_nv += us4
+        del c8, c4
+        torch.cuda.empty_cache()
+    rows["f4_w8a8_fp8_m128"] = dict(fp8, step_ms_80_layers=round(80 * tot_fp8 / 1e3, 3),
+                                    shape="E4M3 weights per channel, activations per tensor, M=128")
+    rows["f2_nvfp4_m128"] = dict(nv, step_ms_80_layers=round(80 * tot_nv / 1e3, 3),
+                                 shape="E2M1 + E4M3 block scales (16) + fp32 tensor scale, both operands, M=128")
+    # KV-cache read: one layer at batch 128, 8,000 tokens, int4 (blocks of 128) and fp8
+    g = wq_inputs.KV_70B
+    B, T, H, Hq, D = g["B"], g["T"], g["H"], g["Hq"], g["D"]
+    q = wq_inputs.queries(B, Hq, D, 6, device=device)
+    lens = torch.full((B,), T, dtype=torch.int32, device=device)
+    ws = torch.empty(wq.wq_decode_attention_workspace_bytes(B, T, H), dtype=torch.uint8, device=device)
+    o = torch.empty((B, Hq, D), dtype=torch.float32, device=device)
+    kv4 = []
+    for j in range(2):
+        c = wq_inputs.kv_cache(B, T, H, D, 60 + j, device=device)
+        qq, s, z = wq.wq_quantize_int4(c.reshape(B * T * H, D), 128)
+        kv4.append((qq.reshape(B, T, H, D // 2), s, z))
+        del c
+    torch.cuda.empty_cache()
+    us = _time_rotating([lambda: wq.wq_decode_attention_int4(q, *kv4[0], *kv4[1], lens, o=o, workspace=ws)], reps)
+    b = 2 * B * T * H * (D // 2 + 4) + B * Hq * D * (2 + 4)
+    rows["f3_kv_int4_read"] = {"us": round(us, 1), "GB_s": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / hbm, 3),
+                               "step_ms_80_layers": round(80 * us / 1e3, 2),
+                               "shape": "decode attention, B=128 T=8000 H=8 Hq=64 D=128, int4 K and V (g=128)"}
+    del kv4
+    torch.cuda.empty_cache()
+    kv8 = []
+    for j in range(2):
+        c = wq_inputs.kv_cache(B, T, H, D, 62 + j, device=device)
+        qq, s = wq.wq_quantize_fp8_tensor(c.reshape(B * T * H, D))
+        kv8.append((qq.reshape(B, T, H, D), s))
+        del c
+    torch.cuda.empty_cache()
+    us = _time_rotating([lambda: wq.wq_decode_attention_fp8(q, *kv8[0], *kv8[1], lens, o=o, workspace=ws)], reps)
+    b = 2 * B * T * H * D + B * Hq * D * (2 + 4)
+    rows["f3_kv_fp8_read"] = {"us": round(us, 1), "GB_s": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / hbm, 3),
+                              "step_ms_80_layers": round(80 * us / 1e3, 2),
+                              "shape": "decode attention, B=128 T=8000 H=8 Hq=64 D=128, fp8 E4M3 K and V"}
+    del kv8
+    torch.cuda.empty_cache()
+    return rows
+
+
 def per_linear_us(model, xs, ys, reps=5):
     """Average device time of each linear shape at M = 1: the 80 calls of one shape replayed as a CUDA
     graph (as in the step), events around the replays."""
@@ -459,6 +648,7 @@ def main():
     ap.add_argument("--m128-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-configuration and NEXT rows")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -527,6 +717,10 @@ def main():
 
     q8_row, g8_row = int8_rows(wq, device)
     sym_row = sym_int4_row(wq, device)
+    extra = {}
+    if not args.no_rows:
+        extra.update(config_rows(wq, device, peaks))
+        extra.update(next_rows(wq, device, peaks))
 
     quant_gbs = model.quant_bytes / (model.quant_ms * 1e-3) / 1e9
 
@@ -548,8 +742,10 @@ def main():
                    "parallelism": f"replicas x{world}"},
         "pct_hbm_peak": round(100 * per_gpu_gbs / peaks["hbm_gbs"], 1),
         "m128": {"tflops": round(tflops128, 1), "ms_per_step": round(ms128 / m128_steps, 3),
-                 "pct_bf16_peak": round(100 * tflops128 / world / peaks["bf16_tflops_sustained"], 1),
-                 "peak_tflops": peaks["bf16_tflops_sustained"], "peak_kind": "sustained (kernel inside a long step)",
+                 "pct_bf16_peak": round(100 * tflops128 / world / peaks["bf16_tflops"], 1),
+                 "peak_tflops": peaks["bf16_tflops"],
+                 "peak_kind": "burst (the timed region is %d steps of ~%d ms)" % (m128_steps, round(ms128 / m128_steps)),
+                 "pct_bf16_sustained_peak": round(100 * tflops128 / world / peaks["bf16_tflops_sustained"], 1),
                  "steps": m128_steps},
         "rows": {
             "a1_quantize_int4": {"GB_s": round(quant_gbs, 1), "ms_total": round(model.quant_ms, 2),
@@ -559,6 +755,7 @@ def main():
             "a5_w4a16_m128": {"tflops": round(tflops128 / world, 1)},
             "a6_w8a16_m1": {k: (round(v, 2) if isinstance(v, float) else v) for k, v in g8_row.items()},
             "f1_quantize_int4_sym": sym_row,
+            **extra,
         },
         "roofline": {"bound": "hbm", "kernel": "gemv_w4a16_m1_kernel", "achieved": round(per_gpu_gbs, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(per_gpu_gbs / peaks["hbm_gbs"], 4),

@@ -102,6 +102,8 @@ def lib():
         L.wq_awq_channel_magnitudes.restype = I
         L.wq_awq_channel_scales.argtypes = [P, I64, ctypes.c_double, P, P]
         L.wq_awq_channel_scales.restype = I
+        L.wq_test_skip_weight_copy.argtypes = [I64]
+        L.wq_test_skip_weight_copy.restype = None
         L.wq_decode_attention_workspace_bytes.argtypes = [I64, I64, I64]
         L.wq_decode_attention_workspace_bytes.restype = SZ
         L.wq_decode_attention_int4.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I64, I64, P, P, SZ, P]

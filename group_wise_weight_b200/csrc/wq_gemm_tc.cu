@@ -44,6 +44,7 @@
 // per segment in the workspace; the CTA whose stages complete the tile sums
 // the partials of the others and writes y.  Every barrier wait is bounded.
 #include <algorithm>
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, int64_t M,
                      int64_t N, int64_t K, const uint16_t *__restrict__ sc, const uint16_t *__restrict__ zp,
                      uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ counters, int max_segs,
-                     int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic)
+                     int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic, int64_t skip_unit)
 {
     using C = Cfg<BN>;
     constexpr int NG = kStageK / GROUP;     // groups per stage
@@ -214,9 +215,13 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 if (issued >= nst && !mbar_wait_fast(&emptyb[rg.slot], rg.phase ^ 1u, status, abort_flag)) break;
                 const int nt = (int)(tile % S.n_tiles), mt = (int)(tile / S.n_tiles);
                 if (weights) {
-                    mbar_arrive_expect_tx(&fullb[rg.slot], kWeightStageBytes);
-                    tma_load_2d(smem + C::kWOff + rg.slot * kWeightStageBytes, &wmap, &fullb[rg.slot],
-                                ks * (kStageK / 2), nt * kTileN);
+                    // skip_unit (tests of the failure path only, -1 otherwise): this stage's weights are never
+                    // requested, so the waits on them run out; no copy is left in flight
+                    if (u != skip_unit) {
+                        mbar_arrive_expect_tx(&fullb[rg.slot], kWeightStageBytes);
+                        tma_load_2d(smem + C::kWOff + rg.slot * kWeightStageBytes, &wmap, &fullb[rg.slot],
+                                    ks * (kStageK / 2), nt * kTileN);
+                    }
                 } else {
                     uint8_t *st = smem + rg.slot * C::kXStageBytes;
                     mbar_arrive_expect_tx(&fullb[rg.slot], C::kXStageBytes);
@@ -227,8 +232,10 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 rg.next(nst);
                 if (++ks == spt) { ks = 0; ++tile; }
             }
-            // drain: every issued copy must land before the CTA may exit (bounded, ignoring abort)
+            // drain: every issued copy must land before the CTA may exit (bounded, ignoring abort); a skipped
+            // stage was never requested and is not waited for
             for (uint32_t j = issued > nst ? issued - nst : 0; j < issued; ++j) {
+                if (weights && beg + (int64_t)j == skip_unit) continue;
                 const uint64_t t0 = global_ns();
                 while (!mbar_try_wait(&fullb[j % nst], (j / nst) & 1u))
                     if (global_ns() - t0 > kWaitLimitNs) { record_timeout(status); break; }
@@ -536,6 +543,12 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     if (wid == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
+// Failure-path tests: the (tile, stage) unit whose weight copy the next launch leaves out (-1: none).  Set
+// by wq_test_skip_weight_copy, consumed by one launch.
+std::atomic<int64_t> g_skip_unit{-1};
+
+int64_t test_take_skip_unit() { return g_skip_unit.exchange(-1); }
+
 template <int BN, int GROUP>
 int run(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s, const uint16_t *z,
         uint16_t *y, void *workspace, int *status, cudaStream_t st)
@@ -580,7 +593,7 @@ int run(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, co
     float *ws = reinterpret_cast<float *>(w8);
     int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, GROUP));
     kern<<<(unsigned)grid, kThreads, smem, st>>>(wmap, xmap, M, N, K, s, z, y, ws, counters, max_segs, status,
-                                                  0x000F000Fu, 0x43004300u);
+                                                  0x000F000Fu, 0x43004300u, test_take_skip_unit());
     return 0;
 }
 
@@ -641,3 +654,7 @@ int launch_gemm_w4a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, con
 }
 
 }  // namespace wq
+
+// Test hook of the failure path (declared in wq.h): the next tensor-core W4A16 launch leaves out the weight
+// copy of (tile, stage) unit `unit`, so the waits on it run out.
+extern "C" void wq_test_skip_weight_copy(int64_t unit) { wq::g_skip_unit.store(unit); }

@@ -446,6 +446,16 @@ int wq_gemm_w4a16_noalloc(const uint16_t *x, int64_t M, int64_t N, int64_t K, co
  */
 int wq_device_status(void *stream);
 
+/*
+ * Test hook of the failure path, for the library's own tests: the next
+ * tensor-core W4A16 launch (wq_gemm_w4a16 with M > 16) never requests the
+ * weight copy of its stream-K unit `unit` (tile * (K / 128) + stage), so
+ * the waits on that copy run out after the bounded-wait limit (about 1 s):
+ * the call returns, wq_device_status reports WQ_ERR_DEVICE_TIMEOUT and the
+ * library stays usable.  No copy is left in flight.  Pass -1 to disarm.
+ */
+void wq_test_skip_weight_copy(int64_t unit);
+
 #ifdef __cplusplus
 }
 #endif
