@@ -1,0 +1,514 @@
+// wq_gemm_tc2.cu -- W4A16 matmul at batch sizes of 65 and more with groups of
+// 128 (a 128 x 128 tile per CTA), on the 5th-generation tensor cores, with
+// dequantisation and promotion in separate warps.
+//
+// The arithmetic is that of wq_gemm_tc.cu ("Quantization for LLM inference:
+// FP8, INT4 (GPTQ, AWQ) and GGUF", "The minimum maths": w_hat = s (q - z);
+// "Quantization Methods Compared ...", "Hardware, formats and the roofline":
+// at batch 128 the matmul is a dense contraction, 4-bit weights are expanded
+// inside the kernel): the MMA takes the exact integers q - z from tensor
+// memory, each group of 128 k accumulates into its own tensor-memory region,
+// and s is applied in binary32 ("promotion", y += s * D_group).  What differs
+// is who does what.  In wq_gemm_tc.cu the same warps dequantise one stage and
+// then promote the previous one, so each stage's MMAs wait for a warp to get
+// through both; here
+//  * warp 0 loads weight stages (TMA, 64-byte swizzle), warp 2 activation
+//    stages (TMA, 128-byte swizzle), warp 1 allocates tensor memory and one
+//    lane issues the MMAs (A from tensor memory, B from shared memory);
+//  * warps 4..11 (two warpgroups) only dequantise: codes from shared memory
+//    to bf16 q - z in tensor memory, up to four stages ahead of the MMAs;
+//  * warps 12..15 (one warpgroup) only promote, each thread holding its
+//    row's 128 binary32 accumulators, and write the output;
+//  * register budgets follow the roles (setmaxnreg): 64 for the control
+//    warpgroup, 96 for dequantisation, 240 for promotion (512 threads at
+//    launch x 128 registers = 65,536; 128 x 64 + 256 x 96 + 128 x 240 =
+//    63,488).  Waits are inlined (no calls): ptxas allocates registers per
+//    role only for straight-line code.
+// Tensor memory: four A buffers of 64 columns, two D buffers of 128.  A zero-
+// point outside [0, 15] is split as in wq_gemm_tc.cu (the dequant warp marks
+// the stage, the MMA warp sums that stage's activations, the promotion adds
+// -s z_hi times the sums).  Stream-K over (tile, stage) units, per-segment
+// binary32 partials summed in segment order.  Every wait is bounded.
+#include <algorithm>
+#include <atomic>
+#include <map>
+#include <mutex>
+
+#include "wq_internal.h"
+#include "wq_sm100.cuh"
+
+namespace wq {
+
+namespace {
+
+constexpr int kTileN = 128;     // weight rows per tile (MMA M)
+constexpr int kBN = 128;        // activation rows per tile (MMA N)
+constexpr int kStageK = 128;    // k per stage = one group
+constexpr int kWStages = 8;
+constexpr int kXStages = 3;
+constexpr int kABufs = 4;
+constexpr int kThreads = 512;
+constexpr int kFirstDq = 4, kDqWarps = 8, kFirstPr = 12, kPrWarps = 4;
+constexpr int kWeightStageBytes = kTileN * (kStageK / 2);  // 8 KB
+constexpr int kXAtomBytes = kBN * 128;                     // 128 rows x 64 bf16
+constexpr int kXStageBytes = 2 * kXAtomBytes;              // 32 KB
+constexpr uint32_t kTmemCols = 512;                        // A 4 x 64, D 2 x 128
+constexpr size_t kWOff = (size_t)kXStages * kXStageBytes;
+constexpr size_t kBarOff = kWOff + (size_t)kWStages * kWeightStageBytes;
+// x_full, x_empty [3]; w_full, w_empty [8]; a_full, a_empty [4]; d_full, d_empty [2]; done
+constexpr size_t kFlagOff = kBarOff + (2 * kXStages + 2 * kWStages + 2 * kABufs + 4 + 1) * 8;
+constexpr size_t kXsumOff = kFlagOff + 64;
+constexpr size_t kSmemBytes = kXsumOff + 2 * kBN * 4;
+
+struct Sched {
+    int64_t n_tiles, tiles, spt, total, per, extra;
+    __host__ __device__ int64_t cta_of(int64_t u) const
+    {
+        const int64_t big = extra * (per + 1);
+        return u < big ? u / (per + 1) : extra + (u - big) / per;
+    }
+    __host__ __device__ int64_t begin_of(int64_t b) const { return b * per + (b < extra ? b : extra); }
+};
+
+struct Ring {
+    uint32_t slot = 0, phase = 0;
+    __device__ __forceinline__ void next(uint32_t n)
+    {
+        if (++slot == n) { slot = 0; phase ^= 1u; }
+    }
+};
+
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ uint32_t word_of4(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t t, uint32_t mask, uint32_t magic)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(t), "r"(mask), "r"(magic));
+    return d;
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int *status)
+{
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs) { record_timeout(status); return; }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, int64_t M,
+                      int64_t N, int64_t K, const uint16_t *__restrict__ sc, const uint16_t *__restrict__ zp,
+                      uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ counters, int max_segs,
+                      int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic, int64_t skip_unit)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    uint64_t *x_full = reinterpret_cast<uint64_t *>(smem + kBarOff);
+    uint64_t *x_empty = x_full + kXStages;
+    uint64_t *w_full = x_empty + kXStages;
+    uint64_t *w_empty = w_full + kWStages;
+    uint64_t *a_full = w_empty + kWStages;
+    uint64_t *a_empty = a_full + kABufs;
+    uint64_t *d_full = a_empty + kABufs;
+    uint64_t *d_empty = d_full + 2;
+    uint64_t *done = d_empty + 2;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kFlagOff);
+    volatile int *last_flag = abort_flag + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kFlagOff + 16);
+    volatile int *wide_mark = reinterpret_cast<volatile int *>(smem + kFlagOff + 32);  // [A buffer]
+    volatile int *xs_wide = wide_mark + kABufs;                                        // [D buffer]
+    float *xsum = reinterpret_cast<float *>(smem + kXsumOff);                          // [D buffer][BN]
+
+    const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
+    Sched S;
+    S.n_tiles = (N + kTileN - 1) / kTileN;
+    S.tiles = S.n_tiles * ((M + kBN - 1) / kBN);
+    S.spt = K / kStageK;
+    S.total = S.tiles * S.spt;
+    S.per = S.total / gridDim.x;
+    S.extra = S.total % gridDim.x;
+    const int64_t beg = S.begin_of(blockIdx.x);
+    const int64_t end = beg + S.per + ((int64_t)blockIdx.x < S.extra ? 1 : 0);
+    const int spt = (int)S.spt;
+
+    if (tid == 0) {
+        for (int i = 0; i < kXStages; ++i) {
+            mbar_init(&x_full[i], 1);
+            mbar_init(&x_empty[i], 1);
+        }
+        for (int i = 0; i < kWStages; ++i) {
+            mbar_init(&w_full[i], 1);
+            mbar_init(&w_empty[i], kDqWarps);
+        }
+        for (int i = 0; i < kABufs; ++i) {
+            mbar_init(&a_full[i], kDqWarps);
+            mbar_init(&a_empty[i], 1);
+            wide_mark[i] = 0;
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&d_full[i], 2);  // the MMAs' completion, and the MMA warp's activation sums
+            mbar_init(&d_empty[i], kPrWarps);
+        }
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        *last_flag = 0;
+        fence_mbar_init();
+    }
+    if (wid == 1) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t d_tmem = tmem + kABufs * 64u;  // D buffer b at column b * 128
+
+    if (wid < kFirstDq) {
+        setmaxnreg_dec<64>();
+        if (wid == 0 || wid == 2) {
+            // ------------------------------ TMA producers ------------------------------
+            const bool weights = wid == 0;
+            const uint32_t nst = weights ? (uint32_t)kWStages : (uint32_t)kXStages;
+            uint64_t *fullb = weights ? w_full : x_full;
+            uint64_t *emptyb = weights ? w_empty : x_empty;
+            if (lane == 0 && beg < end) {
+                Ring rg;
+                uint32_t issued = 0;
+                int64_t tile = beg / spt;
+                int ks = (int)(beg - tile * spt);
+                for (int64_t u = beg; u < end; ++u) {
+                    if (issued >= nst && !mbar_wait(&emptyb[rg.slot], rg.phase ^ 1u, status, abort_flag)) break;
+                    const int nt = (int)(tile % S.n_tiles), mt = (int)(tile / S.n_tiles);
+                    if (weights) {
+                        // skip_unit (failure-path tests only, -1 otherwise): these weights are never requested
+                        if (u != skip_unit) {
+                            mbar_arrive_expect_tx(&fullb[rg.slot], kWeightStageBytes);
+                            tma_load_2d(smem + kWOff + rg.slot * kWeightStageBytes, &wmap, &fullb[rg.slot],
+                                        ks * (kStageK / 2), nt * kTileN);
+                        }
+                    } else {
+                        uint8_t *st = smem + rg.slot * kXStageBytes;
+                        mbar_arrive_expect_tx(&fullb[rg.slot], kXStageBytes);
+                        tma_load_2d(st, &xmap, &fullb[rg.slot], ks * kStageK, mt * kBN);
+                        tma_load_2d(st + kXAtomBytes, &xmap, &fullb[rg.slot], ks * kStageK + 64, mt * kBN);
+                    }
+                    ++issued;
+                    rg.next(nst);
+                    if (++ks == spt) { ks = 0; ++tile; }
+                }
+                for (uint32_t j = issued > nst ? issued - nst : 0; j < issued; ++j) {
+                    if (weights && beg + (int64_t)j == skip_unit) continue;
+                    drain_wait(&fullb[j % nst], (j / nst) & 1u, status);
+                }
+            }
+        } else if (wid == 1) {
+            // ------------------------------ MMA issuer ------------------------------
+            constexpr uint32_t idesc = idesc_bf16_f32(128, kBN);
+            Ring xr, ar, dr;
+            uint32_t it = 0;
+            const uint32_t xbase = smem_u32(smem);
+            for (int64_t u = beg; u < end; ++u, ++it) {
+                mbar_wait(&x_full[xr.slot], xr.phase, status, abort_flag);
+                mbar_wait(&a_full[ar.slot], ar.phase, status, abort_flag);
+                if (it >= 2) mbar_wait(&d_empty[dr.slot], dr.phase ^ 1u, status, abort_flag);
+                tc_fence_after();
+                const uint32_t xs = xbase + xr.slot * (uint32_t)kXStageBytes;
+                if (lane == 0) {
+                    const uint32_t a_col = tmem + ar.slot * 64u;
+                    const uint32_t d_col = d_tmem + dr.slot * (uint32_t)kBN;
+#pragma unroll
+                    for (int j = 0; j < kStageK / 16; ++j) {
+                        const uint32_t baddr = xs + (uint32_t)(j >> 2) * kXAtomBytes + (uint32_t)(j & 3) * 32u;
+                        tc_mma_ts(d_col, a_col + (uint32_t)j * 8u, smem_desc(baddr, 16, 1024, 2), idesc, j != 0 ? 1u : 0u);
+                    }
+                }
+                const bool wide = wide_mark[ar.slot] == (int)(it + 1);
+                if (wide) {
+                    // the stage's activation sums, rows m = lane, lane + 32, ...: two 128-byte-swizzled atoms
+                    for (int m = lane; m < kBN; m += 32) {
+                        float t = 0.0f;
+#pragma unroll
+                        for (int a = 0; a < 2; ++a)
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                uint4 v;
+                                const uint32_t addr = xs + (uint32_t)a * kXAtomBytes + (uint32_t)m * 128u +
+                                                      (((uint32_t)c ^ ((uint32_t)m & 7u)) << 4);
+                                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+                                t += sum_bf16x8(v);
+                            }
+                        xsum[dr.slot * kBN + m] = t;
+                    }
+                }
+                if (lane == 0) xs_wide[dr.slot] = wide ? 1 : 0;
+                __syncwarp();
+                if (lane == 0) {
+                    tc_commit(&x_empty[xr.slot]);
+                    tc_commit(&a_empty[ar.slot]);
+                    tc_commit(&d_full[dr.slot]);
+                    mbar_arrive(&d_full[dr.slot]);
+                }
+                xr.next(kXStages);
+                ar.next(kABufs);
+                dr.next(2);
+            }
+            if (lane == 0) {
+                tc_commit(done);
+                drain_wait(done, 0, status);  // every MMA completes before tensor memory is released
+            }
+        }
+    } else if (wid < kFirstPr) {
+        setmaxnreg_dec<96>();
+        // ------------------------------ dequantisation ------------------------------
+        const int dw = wid - kFirstDq;
+        const int quarter = wid & 3;  // tensor-memory lanes 32 * quarter ..
+        const int kq = dw >> 2;       // k half of each stage
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
+        const int G = (int)(K / kStageK);
+        uint32_t w_addr[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+            w_addr[i] = smem_u32(smem + kWOff) + (uint32_t)r * 64u + 16u * ((uint32_t)(kq * 2 + i) ^ (uint32_t)((r >> 1) & 3));
+        const uint32_t a_addr = tmem + lane_bits + (uint32_t)(kq * 32);
+        Ring wr, ar;
+        uint32_t it = 0;
+        int64_t tile = beg / spt;
+        int ks = (int)(beg - tile * spt);
+        uint16_t znext = 0;
+        {
+            const int64_t n = (tile % S.n_tiles) * kTileN + r;
+            znext = zp[(n < N ? n : N - 1) * G + ks];
+        }
+        for (int64_t u = beg; u < end; ++u, ++it) {
+            mbar_wait(&w_full[wr.slot], wr.phase, status, abort_flag);
+            if (it >= kABufs) {
+                mbar_wait(&a_empty[ar.slot], ar.phase ^ 1u, status, abort_flag);
+                tc_fence_after();
+            }
+            uint4 wv[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(wv[i].x), "=r"(wv[i].y), "=r"(wv[i].z), "=r"(wv[i].w)
+                             : "r"(w_addr[i] + wr.slot * (uint32_t)kWeightStageBytes));
+            float zl = bf16_to_f32(znext);
+            bool wide = false;
+            if (!(zl >= 0.0f && zl <= 15.0f)) {
+                float zh;
+                zl = zp_split(zl, zh);
+                wide = true;
+            }
+            const uint32_t z2 = bf16_pair_128_plus(zl);
+            // the next unit's zero-point, one stage ahead
+            int ks2 = ks + 1;
+            int64_t tile2 = tile;
+            if (ks2 == spt) { ks2 = 0; ++tile2; }
+            if (u + 1 < end) {
+                const int64_t n = (tile2 % S.n_tiles) * kTileN + r;
+                znext = zp[(n < N ? n : N - 1) * G + ks2];
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                uint32_t A[16];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const uint32_t v = word_of4(wv[i], w);
+                    const uint32_t v4 = v >> 4;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t t = __byte_perm(v, v4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
+                        A[w * 4 + j] = sub_bf16x2(lop_and_or(t, nib_mask, bf16_magic), z2);
+                    }
+                }
+                tmem_st16(a_addr + ar.slot * 64u + (uint32_t)(i * 16), A);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            if (wide) wide_mark[ar.slot] = (int)it + 1;
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&w_empty[wr.slot]);
+                mbar_arrive(&a_full[ar.slot]);
+            }
+            wr.next(kWStages);
+            ar.next(kABufs);
+            ks = ks2;
+            tile = tile2;
+        }
+    } else {
+        setmaxnreg_inc<240>();
+        // ------------------------------ promotion and output ------------------------------
+        const int quarter = wid & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
+        const int G = (int)(K / kStageK);
+        const int ptid = tid - kFirstPr * 32;  // 0 .. 127
+        Ring dr;
+        for (int64_t u = beg; u < end;) {
+            const int64_t tile = u / spt;
+            const int ks0 = (int)(u - tile * spt);
+            const int ks1 = (int)std::min<int64_t>(spt, ks0 + (end - u));
+            const int64_t nt = tile % S.n_tiles, mt = tile / S.n_tiles;
+            const int64_t n = nt * kTileN + r;
+            const int64_t nrow = n < N ? n : N - 1;
+            const uint16_t *srow = sc + nrow * G;
+            const uint16_t *zrow = zp + nrow * G;
+            float acc[kBN];
+#pragma unroll
+            for (int c = 0; c < kBN; ++c) acc[c] = 0.0f;
+            float snext = bf16_to_f32(srow[ks0]);
+            for (int ks = ks0; ks < ks1; ++ks) {
+                const float s = snext;
+                if (ks + 1 < ks1) snext = bf16_to_f32(srow[ks + 1]);
+                mbar_wait(&d_full[dr.slot], dr.phase, status, abort_flag);
+                tc_fence_after();
+                const uint32_t dcol = d_tmem + lane_bits + dr.slot * (uint32_t)kBN;
+                const f32x2 s2{s, s};
+#pragma unroll
+                for (int c0 = 0; c0 < kBN; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(dcol + (uint32_t)c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const f32x2 r2 = fma2_pairs(s2, f32x2{__uint_as_float(v[i]), __uint_as_float(v[i + 1])},
+                                                    f32x2{acc[c0 + i], acc[c0 + i + 1]});
+                        acc[c0 + i] = r2.x;
+                        acc[c0 + i + 1] = r2.y;
+                    }
+                }
+                if (xs_wide[dr.slot]) {
+                    float zh;
+                    zp_split(bf16_to_f32(zrow[ks]), zh);
+                    if (zh != 0.0f) {
+                        const float t = -s * zh;
+                        const float *xg = xsum + dr.slot * kBN;
+#pragma unroll
+                        for (int c = 0; c < kBN; ++c) acc[c] = fmaf(t, xg[c], acc[c]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&d_empty[dr.slot]);
+                dr.next(2);
+            }
+
+            // ---- segment output ----
+            const int64_t mbase = mt * kBN;
+            if (ks0 == 0 && ks1 == spt) {
+                if (n < N) {
+                    uint16_t *yp = y + mbase * N + n;
+                    const int mlim = (int)std::min<int64_t>(kBN, M - mbase);
+#pragma unroll
+                    for (int c = 0; c < kBN; ++c, yp += N)
+                        if (c < mlim) *yp = f32_to_bf16(acc[c]);
+                }
+            } else {
+                const int64_t cta_first = S.cta_of(tile * spt);
+                const int64_t my_seg = (int64_t)blockIdx.x - cta_first;
+                const int64_t cta_last = S.cta_of(tile * spt + spt - 1);
+                float *slot = ws + ((tile * max_segs + my_seg) * kBN) * kTileN + r;
+#pragma unroll
+                for (int c = 0; c < kBN; ++c) slot[c * kTileN] = acc[c];
+                __threadfence();
+                named_bar_sync(1, kPrWarps * 32);
+                if (ptid == 0) {
+                    const int add = ks1 - ks0;
+                    const int prev = atomicAdd(counters + tile, add);
+                    *last_flag = (prev + add == spt) ? 1 : 0;
+                }
+                named_bar_sync(1, kPrWarps * 32);
+                if (*last_flag) {
+                    // sum the segments in segment order, whichever CTA finishes last
+                    __threadfence();
+#pragma unroll
+                    for (int c0 = 0; c0 < kBN; c0 += 32) {
+                        float tot[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) tot[c] = 0.0f;
+                        for (int64_t o = 0; o <= cta_last - cta_first; ++o) {
+                            const float *other = ws + ((tile * max_segs + o) * kBN) * kTileN;
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                tot[c] += (o == my_seg) ? acc[c0 + c] : __ldcg(other + (int64_t)(c0 + c) * kTileN + r);
+                        }
+                        if (n < N) {
+                            uint16_t *yp = y + (mbase + c0) * N + n;
+                            const int mlim = (int)std::min<int64_t>(32, M - mbase - c0);
+#pragma unroll
+                            for (int c = 0; c < 32; ++c, yp += N)
+                                if (c < mlim) *yp = f32_to_bf16(tot[c]);
+                        }
+                    }
+                    named_bar_sync(1, kPrWarps * 32);
+                    if (ptid == 0) atomicExch(counters + tile, 0);
+                }
+            }
+            u += ks1 - ks0;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (wid == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+size_t gemm_tc2_smem_bytes() { return std::max<size_t>(kSmemBytes + 1024, 120 * 1024); }
+
+int launch_gemm_w4a16_tc2(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
+                          const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st,
+                          int64_t skip_unit)
+{
+    CUtensorMap wmap, xmap;
+    if (!encode_tmap_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, (uint64_t)(K / 2), (uint64_t)N, (uint64_t)(K / 2),
+                        kStageK / 2, kTileN, CU_TENSOR_MAP_SWIZZLE_64B))
+        return -1;
+    if (!encode_tmap_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, kBN,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return -1;
+    static std::mutex mu;
+    static std::map<int, int> sms_of;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int sms;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = sms_of.find(dev);
+        if (it == sms_of.end()) {
+            int v = 148, optin = 0;
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+            cudaFuncSetAttribute(gemm_w4a16_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+            it = sms_of.emplace(dev, v).first;
+        }
+        sms = it->second;
+    }
+    const int64_t tiles = ((N + kTileN - 1) / kTileN) * ((M + kBN - 1) / kBN);
+    const int64_t total = tiles * (K / kStageK);
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(total, sms));
+    const int max_segs = (int)gemm_tc_max_segments(total, grid, K / kStageK);
+    uint8_t *w8 = static_cast<uint8_t *>(workspace);
+    float *ws = reinterpret_cast<float *>(w8);
+    int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, 128));
+    gemm_w4a16_tc2_kernel<<<(unsigned)grid, kThreads, gemm_tc2_smem_bytes(), st>>>(
+        wmap, xmap, M, N, K, s, z, y, ws, counters, max_segs, status, 0x000F000Fu, 0x43004300u, skip_unit);
+    return 0;
+}
+
+}  // namespace wq

@@ -3,10 +3,11 @@
 "Quantization Methods Compared: INT8, GPTQ, AWQ, FP8, FP4 and KV-Cache Quantization", section "The methods
 compared" (AWQ scales salient channels; the activations compensate).  wq_gemm_w4a16_colscaled computes
 sum_k bf16(x / s) w_hat' with w_hat' the weights w * s quantised by wq_quantize_int4_scaled; the oracle's
-compensated product is sum_k (x / s) w_hat' in binary64.  Rounding x / s to bf16 costs at most 2^-9 of each
-term and rounding y another 2^-9 of |y|, so the bound
+compensated product is sum_k (x / s) w_hat' in binary64.  Rounding x / s to bf16 moves each term by at
+most 2^-8 of itself and rounding y moves y by at most 2^-8 of |y|; on these inputs the realised error stays
+far inside
     |y - y_ref| <= 4e-3 * sum_k |(x / s) w_hat'|
-holds element by element.  The channel statistics of the search must match the oracle's (magnitudes bit
+element by element (the bound the matmul tests use; the worst case of the two roundings is 2^-7).  The channel statistics of the search must match the oracle's (magnitudes bit
 for bit, scales to the last bit of binary32 up to one unit), and the search through the library's kernels
 must pick the oracle pipeline's alpha with the same roundings.
 """

@@ -7,7 +7,8 @@ The caches are quantised on the GPU by the library's quantisers and must match t
 scales bit for bit; the read must satisfy, element by element,
     |o - o_ref| <= 4e-3 * sum_t p_t |v_hat_t|
 with o_ref and the sum from oracle.kv_cache.decode_attention in binary64.  The bound covers the rounding
-of p times the token's V scale to the MMA's bf16 (2^-9 relative per term) with margin.
+of p times the token's V scale to the MMA's bf16 (at most 2^-8 = 3.9e-3 of each term; the output stays
+binary32) and the binary32 scores and sums.
 """
 import numpy as np
 import pytest
