@@ -258,13 +258,28 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     const int tile0 = (int)(beg / P), pair0 = (int)(beg - (int64_t)tile0 * P);
 
     // Under programmatic dependent launch the previous kernel may still be running.  Nothing it writes may
-    // be read before pdl_wait(), but an L2 prefetch is safe (L2 is where writes land): start pulling the
-    // first stages from HBM now.
+    // be read before pdl_wait().  The packed weights, scales and zero-points are inputs that the preceding
+    // call does not write (a call of this kernel writes only y and its workspace; the library's other
+    // kernels do not launch dependents early), so the producer issues the first stages and the first s/z
+    // window into shared memory now, and only the activations wait.
+    int pt = tile0, pp = pair0;  // producer position: tile, group pair
+    int wins = 0;                // s/z windows issued
+    int pi = 0;                  // stages issued
+    auto issue_window = [&](int slot) {
+        mbar_arrive_expect_tx(&szfull[slot], 2 * kSzBytes);
+        uint8_t *d = szr + (uint32_t)slot * 2u * kSzBytes;
+        const int g8 = (2 * pp) & ~7;
+        tma_load_2d(d, &smap, &szfull[slot], g8, pt * kTile);
+        tma_load_2d(d + kSzBytes, &zmap, &szfull[slot], g8, pt * kTile);
+        ++wins;
+    };
     if (wid == kProducer && lane == 0) {
-        int t = tile0, p = pair0;
-        for (int i = 0; i < kStages && i < n; ++i) {
-            tma_prefetch_l2_3d(&wmap, 0, t * kTile, 2 * p);
-            if (++p == P) { p = 0; ++t; }
+        // at most two windows start within the first kStages pairs, so no window slot needs a wait here
+        for (; pi < kStages && pi < n; ++pi) {
+            if (pi == 0 || (pp & (kPairsPerWindow - 1)) == 0) issue_window(wins & 1);
+            mbar_arrive_expect_tx(&full[pi], kStageBytes);
+            tma_load_3d(ring + (uint32_t)pi * kStageBytes, &wmap, &full[pi], 0, pt * kTile, 2 * pp);
+            if (++pp == P) { pp = 0; ++pt; }
         }
     }
     pdl_wait();
@@ -290,28 +305,19 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 bulk_g2s(sm + o, reinterpret_cast<const uint8_t *>(x) + o, min(kBulkPiece, r1 - o), xbar);
             for (uint32_t o = 0; o < w1; o += kBulkPiece)
                 bulk_g2s(sm + o, reinterpret_cast<const uint8_t *>(x) + o, min(kBulkPiece, w1 - o), xbar);
-            int t = tile0, p = pair0;
-            int wins = 0;  // s/z windows issued
-            int i = 0;
+            int i = pi;
             for (; i < n; ++i) {
-                // s/z window: at the range start and at every 4th pair of a tile
-                if (i == 0 || (p & (kPairsPerWindow - 1)) == 0) {
+                // s/z window: at every 4th pair of a tile
+                if ((pp & (kPairsPerWindow - 1)) == 0) {
                     const int slot = wins & 1;
                     if (wins >= 2 && !mbar_wait(&szempty[slot], (uint32_t)((wins >> 1) - 1) & 1u, status, flags)) break;
-                    mbar_arrive_expect_tx(&szfull[slot], 2 * kSzBytes);
-                    uint8_t *d = szr + (uint32_t)slot * 2u * kSzBytes;
-                    const int g8 = (2 * p) & ~7;
-                    tma_load_2d(d, &smap, &szfull[slot], g8, t * kTile);
-                    tma_load_2d(d + kSzBytes, &zmap, &szfull[slot], g8, t * kTile);
-                    ++wins;
+                    issue_window(slot);
                 }
                 const int s = i % kStages;
-                // the first stage goes out alone with x and the first s/z window; the rest once x is in
-                if (i == 1 && !mbar_wait(xbar, 0, status, flags)) break;
-                if (i >= kStages && !mbar_wait(&empty[s], (uint32_t)(i / kStages - 1) & 1u, status, flags)) break;
+                if (!mbar_wait(&empty[s], (uint32_t)(i / kStages - 1) & 1u, status, flags)) break;
                 mbar_arrive_expect_tx(&full[s], kStageBytes);
-                tma_load_3d(ring + (uint32_t)s * kStageBytes, &wmap, &full[s], 0, t * kTile, 2 * p);
-                if (++p == P) { p = 0; ++t; }
+                tma_load_3d(ring + (uint32_t)s * kStageBytes, &wmap, &full[s], 0, pt * kTile, 2 * pp);
+                if (++pp == P) { pp = 0; ++pt; }
             }
             // drain: the copies issued last must land before the CTA can end (bounded, ignores abort)
             for (int j = max(0, i - kStages); j < i; ++j) wait_drain(&full[j % kStages], (uint32_t)(j / kStages) & 1u, status);

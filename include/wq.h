@@ -196,6 +196,11 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * pointers 16-byte aligned; workspace of wq_gemm_workspace_bytes(M, N, K, g, 4)
  * bytes (may be NULL when that is 0).  y must not overlap x, qweight,
  * scales or zeros (WQ_ERR_ARG otherwise).
+ * The M = 1 kernel is launched with programmatic dependent launch: it starts
+ * while the previous M = 1 call on the stream finishes, reads x and writes
+ * only after that call has completed, but requests its qweight, scales and
+ * zeros at once -- so they must not be the y or the workspace of the call
+ * just before it on the same stream.
  */
 int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *qweight,
                   const uint16_t *scales, const uint16_t *zeros, int g, uint16_t *y,
