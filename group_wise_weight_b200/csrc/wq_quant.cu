@@ -156,73 +156,104 @@ __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b)
 // SCALED: quantise w[n][k] * col_scale[k] (each product rounded to binary32), the weights an
 // activation-aware per-input-channel scaling hands the quantiser ("Quantization Methods Compared",
 // section "The methods compared": AWQ scales the salient channels up before quantising).
-template <typename T, int LPG, bool SCALED>
+//
+// A lane takes kWordsPerLane x 8 = 32 consecutive weights of a row (two 32-byte loads for bf16), so a group
+// of G weights spans G / 32 lanes (1, 2 or 4) and a warp task is 1,024 weights.  The group's parameters
+// (min, max, s, 1/s, z) are formed once per 32 weights instead of once per 8, which is where the
+// instructions of an issue-bound quantiser went.
+constexpr int kWordsPerLane = 4;                        // 8-weight words per lane
+constexpr int kLaneWeights = 8 * kWordsPerLane;         // 32
+constexpr int kWarpWeights = 32 * kLaneWeights;         // 1,024 weights per warp task
+constexpr int kInt4Unroll = 2;                          // tasks in flight per warp
+
+// Weight i of 32 held either as widened binary32 values (v) or as the loaded bf16 words (raw).
+template <bool BF16>
+__device__ __forceinline__ float lane_weight(const float *v, const uint4 *raw, int i)
+{
+    if (BF16) {
+        const uint4 &r = raw[i >> 3];
+        const int w = (i >> 1) & 3;
+        const uint32_t word = w == 0 ? r.x : w == 1 ? r.y : w == 2 ? r.z : r.w;
+        return __uint_as_float((i & 1) ? (word & 0xffff0000u) : (word << 16));
+    }
+    return v[i];
+}
+
+template <typename T, int G, bool SCALED>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
                   uint8_t *__restrict__ qweight, uint16_t *__restrict__ scales,
                   uint16_t *__restrict__ zeros, const float *__restrict__ col_scale)
 {
-    constexpr int g = LPG * 8;
+    constexpr int LPG = G / kLaneWeights;  // lanes per group
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int64_t chunks = (K + 255) >> 8;
+    const int64_t chunks = (K + kWarpWeights - 1) / kWarpWeights;
     const int64_t tasks = N * chunks;
-    const int64_t G = K / g;
+    const int64_t Gn = K / G;
 
     // packed bf16 min/max only for unscaled bf16 weights (scaled products are binary32 values)
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value && !SCALED;
     TaskWalk walk(warp0, n_warps, chunks);
-    for (int64_t t0 = warp0; t0 < tasks; t0 += n_warps * kQuantUnroll) {
-        float v[kQuantUnroll][8];
-        uint4 raw[kQuantUnroll];  // bf16 input: the 8 weights as loaded
-        int64_t n[kQuantUnroll], k0[kQuantUnroll];
-        bool active[kQuantUnroll];
+    for (int64_t t0 = warp0; t0 < tasks; t0 += n_warps * kInt4Unroll) {
+        float v[kInt4Unroll][kBf16 ? 1 : kLaneWeights];  // binary32 input or scaled products
+        uint4 raw[kInt4Unroll][kWordsPerLane];             // bf16 input: the weights as loaded
+        int64_t n[kInt4Unroll], k0[kInt4Unroll];
+        bool active[kInt4Unroll];
 #pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
+        for (int u = 0; u < kInt4Unroll; ++u) {
             n[u] = walk.n;
-            k0[u] = walk.c * 256 + lane * 8;
+            k0[u] = walk.c * kWarpWeights + lane * kLaneWeights;
             active[u] = (walk.n < N) && (k0[u] < K);
             if (kBf16) {
-                raw[u] = make_uint4(0u, 0u, 0u, 0u);
-                if (active[u]) raw[u] = ld_stream_v4(w + n[u] * ldw + k0[u]);
-            } else if (active[u]) {
-                load8<T>(w + n[u] * ldw + k0[u], v[u]);
-                if (SCALED) {
-                    float c[8];
-                    load8<float>(col_scale + k0[u], c);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) v[u][i] = __fmul_rn(v[u][i], c[i]);
+                for (int j = 0; j < kWordsPerLane; ++j) raw[u][j] = make_uint4(0u, 0u, 0u, 0u);
+                if (active[u]) {
+#pragma unroll
+                    for (int j = 0; j < kWordsPerLane; ++j) raw[u][j] = ld_stream_v4(w + n[u] * ldw + k0[u] + 8 * j);
+                }
+            } else if (active[u]) {
+#pragma unroll
+                for (int j = 0; j < kWordsPerLane; ++j) {
+                    load8<T>(w + n[u] * ldw + k0[u] + 8 * j, v[u] + 8 * j);
+                    if (SCALED) {
+                        float c[8];
+                        load8<float>(col_scale + k0[u] + 8 * j, c);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) v[u][8 * j + i] = __fmul_rn(v[u][8 * j + i], c[i]);
+                    }
                 }
             }
             walk.step();
         }
 #pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
+        for (int u = 0; u < kInt4Unroll; ++u) {
             if (t0 + u * n_warps >= tasks) break;  // warp-uniform
             float mn, mx;
             if (kBf16) {
                 // bf16 weights are exact in bf16: reduce (min, -max) as one packed pair (a group's lanes are
                 // all active or all inactive; inactive ones contribute +inf to both minima)
-                const uint32_t lo = bf16x2_min(bf16x2_min(raw[u].x, raw[u].y), bf16x2_min(raw[u].z, raw[u].w));
-                const uint32_t hi = bf16x2_max(bf16x2_max(raw[u].x, raw[u].y), bf16x2_max(raw[u].z, raw[u].w)) ^ 0x80008000u;
+                uint32_t lo = bf16x2_min(raw[u][0].x, raw[u][0].y), hi = bf16x2_max(raw[u][0].x, raw[u][0].y);
+                lo = bf16x2_min(lo, bf16x2_min(raw[u][0].z, raw[u][0].w));
+                hi = bf16x2_max(hi, bf16x2_max(raw[u][0].z, raw[u][0].w));
+#pragma unroll
+                for (int j = 1; j < kWordsPerLane; ++j) {
+                    lo = bf16x2_min(lo, bf16x2_min(bf16x2_min(raw[u][j].x, raw[u][j].y), bf16x2_min(raw[u][j].z, raw[u][j].w)));
+                    hi = bf16x2_max(hi, bf16x2_max(bf16x2_max(raw[u][j].x, raw[u][j].y), bf16x2_max(raw[u][j].z, raw[u][j].w)));
+                }
+                hi ^= 0x80008000u;
                 uint32_t pk = active[u] ? bf16x2_min(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632)) : 0x7F807F80u;
 #pragma unroll
                 for (int o = 1; o < LPG; o <<= 1) pk = bf16x2_min(pk, __shfl_xor_sync(0xffffffffu, pk, o));
                 mn = __uint_as_float(pk << 16);
                 mx = __uint_as_float((pk & 0xffff0000u) ^ 0x80000000u);
-                const uint32_t u4[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    v[u][2 * i] = __uint_as_float(u4[i] << 16);
-                    v[u][2 * i + 1] = __uint_as_float(u4[i] & 0xffff0000u);
-                }
             } else {
                 mn = INFINITY;
                 mx = -INFINITY;
                 if (active[u]) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) { mn = fminf(mn, v[u][i]); mx = fmaxf(mx, v[u][i]); }
+                    for (int i = 0; i < kLaneWeights; ++i) { mn = fminf(mn, v[u][i]); mx = fmaxf(mx, v[u][i]); }
                 }
 #pragma unroll
                 for (int o = 1; o < LPG; o <<= 1) {
@@ -232,28 +263,40 @@ quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
             }
             if (!active[u]) continue;
             const float s = int4_scale(mn, mx);
-            float qd[8];  // RN(w / s)
-            float z;      // round_bf16(rint(RN(-min / s)) + 0)
+            float z;  // round_bf16(rint(RN(-min / s)) + 0)
+            uint32_t packed[kWordsPerLane];
+            // q = clip(rint(RN(w / s) + z), 0, 15): clipping before the rounding gives the same integer, and
+            // rint_bits leaves it in the low bits; the eight patterns shifted into place and summed, minus
+            // the summed offsets, are the eight nibbles of a word
             if (quotients_by_reciprocal(s, fmaxf(fabsf(mn), fabsf(mx)))) {
                 const float r = __frcp_rn(s);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) qd[i] = quotient_rn(v[u][i], s, r);
                 z = round_bf16(__fadd_rn(rintf(quotient_rn(-mn, s, r)), 0.0f));
+#pragma unroll
+                for (int j = 0; j < kWordsPerLane; ++j) {
+                    uint32_t pw = 0u - kRintBase * 0x11111111u;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        pw += rint_bits(fminf(fmaxf(__fadd_rn(quotient_rn(lane_weight<kBf16>(v[u], raw[u], 8 * j + i), s, r),
+                                                              z), 0.0f), 15.0f))
+                              << (4 * i);
+                    packed[j] = pw;
+                }
             } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) qd[i] = __fdiv_rn(v[u][i], s);
                 z = round_bf16(__fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.0f));
-            }
-            // q = clip(rint(RN(w / s) + z), 0, 15): clipping before the rounding gives the same integer,
-            // and rint_bits leaves it in the low bits; the eight patterns shifted into place and summed,
-            // minus the summed offsets, are the eight nibbles
-            uint32_t packed = 0u - kRintBase * 0x11111111u;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                packed += rint_bits(fminf(fmaxf(__fadd_rn(qd[i], z), 0.0f), 15.0f)) << (4 * i);
-            *reinterpret_cast<uint32_t *>(qweight + n[u] * (K >> 1) + (k0[u] >> 1)) = packed;
+                for (int j = 0; j < kWordsPerLane; ++j) {
+                    uint32_t pw = 0u - kRintBase * 0x11111111u;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        pw += rint_bits(fminf(fmaxf(__fadd_rn(__fdiv_rn(lane_weight<kBf16>(v[u], raw[u], 8 * j + i), s), z),
+                                                    0.0f), 15.0f)) << (4 * i);
+                    packed[j] = pw;
+                }
+            }
+            *reinterpret_cast<uint4 *>(qweight + n[u] * (K >> 1) + (k0[u] >> 1)) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
             if ((lane & (LPG - 1)) == 0) {
-                const int64_t gi = n[u] * G + k0[u] / g;
+                const int64_t gi = n[u] * Gn + k0[u] / G;
                 scales[gi] = f32_to_bf16(s);
                 zeros[gi] = f32_to_bf16(z);
             }
@@ -482,12 +525,12 @@ int persistent_grid(KernelT kernel, int64_t tasks_in_warps)
     return (int)(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
-template <typename T, int LPG, bool SCALED>
+template <typename T, int G, bool SCALED>
 void launch_int4(const void *w, int64_t N, int64_t K, int64_t ldw, uint8_t *q, uint16_t *s, uint16_t *z,
                  const float *cs, cudaStream_t st)
 {
-    auto k = quant_int4_kernel<T, LPG, SCALED>;
-    const int64_t tasks = N * ((K + 255) / 256);
+    auto k = quant_int4_kernel<T, G, SCALED>;
+    const int64_t tasks = N * ((K + kWarpWeights - 1) / kWarpWeights);
     const int grid = persistent_grid(k, tasks);
     k<<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(w), N, K, ldw, q, s, z, cs);
 }
@@ -506,9 +549,9 @@ void dispatch_int4(const void *w, int64_t N, int64_t K, int64_t ldw, int g, uint
                    uint16_t *z, const float *cs, cudaStream_t st)
 {
     switch (g) {
-    case 32: launch_int4<T, 4, SCALED>(w, N, K, ldw, q, s, z, cs, st); break;
-    case 64: launch_int4<T, 8, SCALED>(w, N, K, ldw, q, s, z, cs, st); break;
-    default: launch_int4<T, 16, SCALED>(w, N, K, ldw, q, s, z, cs, st); break;
+    case 32: launch_int4<T, 32, SCALED>(w, N, K, ldw, q, s, z, cs, st); break;
+    case 64: launch_int4<T, 64, SCALED>(w, N, K, ldw, q, s, z, cs, st); break;
+    default: launch_int4<T, 128, SCALED>(w, N, K, ldw, q, s, z, cs, st); break;
     }
 }
 
