@@ -24,6 +24,10 @@
 //    launch x 128 registers = 65,536; 128 x 64 + 256 x 96 + 128 x 240 =
 //    63,488).  Waits are inlined (no calls): ptxas allocates registers per
 //    role only for straight-line code.
+// Scales and zero-points reach shared memory by TMA in windows of 8 groups x
+// 128 rows (rings of 4), issued by the weight producer with the weight
+// stages, so no warp waits on a global load of a parameter (needs
+// K % 1024 == 0 for the windows' row stride; other K take wq_gemm_tc.cu).
 // Tensor memory: four A buffers of 64 columns, two D buffers of 128.  A zero-
 // point outside [0, 15] is split as in wq_gemm_tc.cu (the dequant warp marks
 // the stage, the MMA warp sums that stage's activations, the promotion adds
@@ -53,12 +57,20 @@ constexpr int kWeightStageBytes = kTileN * (kStageK / 2);  // 8 KB
 constexpr int kXAtomBytes = kBN * 128;                     // 128 rows x 64 bf16
 constexpr int kXStageBytes = 2 * kXAtomBytes;              // 32 KB
 constexpr uint32_t kTmemCols = 512;                        // A 4 x 64, D 2 x 128
+constexpr int kWinGroups = 8;                              // groups (stages) per s / z window
+constexpr int kWinSlots = 4;                               // windows in flight per ring
+constexpr int kWinBytes = kTileN * kWinGroups * 2;         // 128 rows x 8 bf16 = 2 KB
 constexpr size_t kWOff = (size_t)kXStages * kXStageBytes;
-constexpr size_t kBarOff = kWOff + (size_t)kWStages * kWeightStageBytes;
-// x_full, x_empty [3]; w_full, w_empty [8]; a_full, a_empty [4]; d_full, d_empty [2]; done
-constexpr size_t kFlagOff = kBarOff + (2 * kXStages + 2 * kWStages + 2 * kABufs + 4 + 1) * 8;
-constexpr size_t kXsumOff = kFlagOff + 64;
-constexpr size_t kSmemBytes = kXsumOff + 2 * kBN * 4;
+constexpr size_t kZwOff = kWOff + (size_t)kWStages * kWeightStageBytes;  // zero-point windows
+constexpr size_t kSwOff = kZwOff + (size_t)kWinSlots * kWinBytes;        // scale windows
+constexpr size_t kBarOff = kSwOff + (size_t)kWinSlots * kWinBytes;
+// x_full, x_empty [3]; w_full, w_empty [8]; a_full, a_empty [4]; d_full, d_empty [2]; done;
+// zw_full, zw_empty, sw_full, sw_empty [4]
+constexpr size_t kFlagOff = kBarOff + (2 * kXStages + 2 * kWStages + 2 * kABufs + 4 + 1 + 4 * kWinSlots) * 8;
+constexpr size_t kXsumOff = kFlagOff + 64;                    // [D buffer][BN] activation sums
+constexpr size_t kZhiAOff = kXsumOff + 2 * kBN * 4;           // [A buffer][row] z_hi of the stage
+constexpr size_t kZhiDOff = kZhiAOff + kABufs * kTileN * 4;   // [D buffer][row] the same, for the promotion
+constexpr size_t kSmemBytes = kZhiDOff + 2 * kTileN * 4;
 
 struct Sched {
     int64_t n_tiles, tiles, spt, total, per, extra;
@@ -109,9 +121,9 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int *
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, int64_t M,
-                      int64_t N, int64_t K, const uint16_t *__restrict__ sc, const uint16_t *__restrict__ zp,
-                      uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ counters, int max_segs,
+gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
+                      const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap zmap, int64_t M,
+                      int64_t N, int64_t K, uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ counters, int max_segs,
                       int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic, int64_t skip_unit)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -125,12 +137,18 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
     uint64_t *d_full = a_empty + kABufs;
     uint64_t *d_empty = d_full + 2;
     uint64_t *done = d_empty + 2;
+    uint64_t *zw_full = done + 1;
+    uint64_t *zw_empty = zw_full + kWinSlots;
+    uint64_t *sw_full = zw_empty + kWinSlots;
+    uint64_t *sw_empty = sw_full + kWinSlots;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kFlagOff);
     volatile int *last_flag = abort_flag + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kFlagOff + 16);
     volatile int *wide_mark = reinterpret_cast<volatile int *>(smem + kFlagOff + 32);  // [A buffer]
     volatile int *xs_wide = wide_mark + kABufs;                                        // [D buffer]
     float *xsum = reinterpret_cast<float *>(smem + kXsumOff);                          // [D buffer][BN]
+    float *zhi_a = reinterpret_cast<float *>(smem + kZhiAOff);                         // [A buffer][row]
+    float *zhi_d = reinterpret_cast<float *>(smem + kZhiDOff);                         // [D buffer][row]
 
     const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
     Sched S;
@@ -163,6 +181,12 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
             mbar_init(&d_empty[i], kPrWarps);
         }
         mbar_init(done, 1);
+        for (int i = 0; i < kWinSlots; ++i) {
+            mbar_init(&zw_full[i], 1);
+            mbar_init(&zw_empty[i], kDqWarps);
+            mbar_init(&sw_full[i], 1);
+            mbar_init(&sw_empty[i], kPrWarps);
+        }
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
@@ -187,9 +211,23 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 uint32_t issued = 0;
                 int64_t tile = beg / spt;
                 int ks = (int)(beg - tile * spt);
+                uint32_t wins = 0;  // s / z windows issued (weight producer)
                 for (int64_t u = beg; u < end; ++u) {
                     if (issued >= nst && !mbar_wait(&emptyb[rg.slot], rg.phase ^ 1u, status, abort_flag)) break;
                     const int nt = (int)(tile % S.n_tiles), mt = (int)(tile / S.n_tiles);
+                    if (weights && (u == beg || (ks % kWinGroups) == 0)) {
+                        // the s and z of groups (ks & ~7) .. + 7 of the tile's 128 rows, one window each
+                        const uint32_t ws_ = wins % kWinSlots, wph = (wins / kWinSlots) & 1u;
+                        if (wins >= (uint32_t)kWinSlots &&
+                            (!mbar_wait(&zw_empty[ws_], wph ^ 1u, status, abort_flag) ||
+                             !mbar_wait(&sw_empty[ws_], wph ^ 1u, status, abort_flag)))
+                            break;
+                        mbar_arrive_expect_tx(&zw_full[ws_], kWinBytes);
+                        tma_load_2d(smem + kZwOff + ws_ * kWinBytes, &zmap, &zw_full[ws_], ks & ~(kWinGroups - 1), nt * kTileN);
+                        mbar_arrive_expect_tx(&sw_full[ws_], kWinBytes);
+                        tma_load_2d(smem + kSwOff + ws_ * kWinBytes, &smap, &sw_full[ws_], ks & ~(kWinGroups - 1), nt * kTileN);
+                        ++wins;
+                    }
                     if (weights) {
                         // skip_unit (failure-path tests only, -1 otherwise): these weights are never requested
                         if (u != skip_unit) {
@@ -210,6 +248,10 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 for (uint32_t j = issued > nst ? issued - nst : 0; j < issued; ++j) {
                     if (weights && beg + (int64_t)j == skip_unit) continue;
                     drain_wait(&fullb[j % nst], (j / nst) & 1u, status);
+                }
+                for (uint32_t j = wins > (uint32_t)kWinSlots ? wins - kWinSlots : 0; j < wins; ++j) {
+                    drain_wait(&zw_full[j % kWinSlots], (j / kWinSlots) & 1u, status);
+                    drain_wait(&sw_full[j % kWinSlots], (j / kWinSlots) & 1u, status);
                 }
             }
         } else if (wid == 1) {
@@ -251,6 +293,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                             }
                         xsum[dr.slot * kBN + m] = t;
                     }
+                    for (int row = lane; row < kTileN; row += 32) zhi_d[dr.slot * kTileN + row] = zhi_a[ar.slot * kTileN + row];
                 }
                 if (lane == 0) xs_wide[dr.slot] = wide ? 1 : 0;
                 __syncwarp();
@@ -277,7 +320,6 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
         const int kq = dw >> 2;       // k half of each stage
         const int r = quarter * 32 + lane;
         const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
-        const int G = (int)(K / kStageK);
         uint32_t w_addr[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i)
@@ -287,12 +329,21 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
         uint32_t it = 0;
         int64_t tile = beg / spt;
         int ks = (int)(beg - tile * spt);
-        uint16_t znext = 0;
-        {
-            const int64_t n = (tile % S.n_tiles) * kTileN + r;
-            znext = zp[(n < N ? n : N - 1) * G + ks];
-        }
+        int win = -1;  // s / z window in use (the producer's sequence: a new one at the start and every 8th group)
+        const uint32_t zw_row = smem_u32(smem + kZwOff) + (uint32_t)r * (kWinGroups * 2);
         for (int64_t u = beg; u < end; ++u, ++it) {
+            if (u == beg || (ks % kWinGroups) == 0) {
+                if (win >= 0) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&zw_empty[win % kWinSlots]);
+                }
+                ++win;
+                mbar_wait(&zw_full[win % kWinSlots], (uint32_t)(win / kWinSlots) & 1u, status, abort_flag);
+            }
+            uint16_t zraw;
+            asm volatile("ld.shared.u16 %0, [%1];"
+                         : "=h"(zraw)
+                         : "r"(zw_row + (uint32_t)(win % kWinSlots) * kWinBytes + (uint32_t)(ks % kWinGroups) * 2u));
             mbar_wait(&w_full[wr.slot], wr.phase, status, abort_flag);
             if (it >= kABufs) {
                 mbar_wait(&a_empty[ar.slot], ar.phase ^ 1u, status, abort_flag);
@@ -304,22 +355,16 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                              : "=r"(wv[i].x), "=r"(wv[i].y), "=r"(wv[i].z), "=r"(wv[i].w)
                              : "r"(w_addr[i] + wr.slot * (uint32_t)kWeightStageBytes));
-            float zl = bf16_to_f32(znext);
+            float zl = bf16_to_f32(zraw), zh = 0.0f;
             bool wide = false;
             if (!(zl >= 0.0f && zl <= 15.0f)) {
-                float zh;
                 zl = zp_split(zl, zh);
                 wide = true;
             }
             const uint32_t z2 = bf16_pair_128_plus(zl);
-            // the next unit's zero-point, one stage ahead
             int ks2 = ks + 1;
             int64_t tile2 = tile;
             if (ks2 == spt) { ks2 = 0; ++tile2; }
-            if (u + 1 < end) {
-                const int64_t n = (tile2 % S.n_tiles) * kTileN + r;
-                znext = zp[(n < N ? n : N - 1) * G + ks2];
-            }
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 uint32_t A[16];
@@ -337,6 +382,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
             }
             tmem_wait_st();
             tc_fence_before();
+            if (kq == 0) zhi_a[ar.slot * kTileN + r] = zh;  // read by the MMA warp only for a marked stage
             if (wide) wide_mark[ar.slot] = (int)it + 1;
             __syncwarp();
             if (lane == 0) {
@@ -354,36 +400,44 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
         const int quarter = wid & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
-        const int G = (int)(K / kStageK);
         const int ptid = tid - kFirstPr * 32;  // 0 .. 127
         Ring dr;
+        int win = -1;  // s window in use (same sequence as the producer's)
+        const uint32_t sw_row = smem_u32(smem + kSwOff) + (uint32_t)r * (kWinGroups * 2);
         for (int64_t u = beg; u < end;) {
             const int64_t tile = u / spt;
             const int ks0 = (int)(u - tile * spt);
             const int ks1 = (int)std::min<int64_t>(spt, ks0 + (end - u));
             const int64_t nt = tile % S.n_tiles, mt = tile / S.n_tiles;
             const int64_t n = nt * kTileN + r;
-            const int64_t nrow = n < N ? n : N - 1;
-            const uint16_t *srow = sc + nrow * G;
-            const uint16_t *zrow = zp + nrow * G;
             float acc[kBN];
 #pragma unroll
             for (int c = 0; c < kBN; ++c) acc[c] = 0.0f;
-            float snext = bf16_to_f32(srow[ks0]);
             for (int ks = ks0; ks < ks1; ++ks) {
-                const float s = snext;
-                if (ks + 1 < ks1) snext = bf16_to_f32(srow[ks + 1]);
+                if ((u == beg && ks == ks0) || (ks % kWinGroups) == 0) {
+                    if (win >= 0) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sw_empty[win % kWinSlots]);
+                    }
+                    ++win;
+                    mbar_wait(&sw_full[win % kWinSlots], (uint32_t)(win / kWinSlots) & 1u, status, abort_flag);
+                }
+                const uint32_t wslot = (uint32_t)(win % kWinSlots) * kWinBytes + (uint32_t)(ks % kWinGroups) * 2u;
+                uint16_t sraw;
+                asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sraw) : "r"(sw_row + wslot));
+                const float s = bf16_to_f32(sraw);
                 mbar_wait(&d_full[dr.slot], dr.phase, status, abort_flag);
                 tc_fence_after();
                 const uint32_t dcol = d_tmem + lane_bits + dr.slot * (uint32_t)kBN;
                 const f32x2 s2{s, s};
 #pragma unroll
-                for (int c0 = 0; c0 < kBN; c0 += 32) {
-                    uint32_t v[32];
+                for (int c0 = 0; c0 < kBN; c0 += 64) {
+                    uint32_t v[64];
                     tmem_ld32(dcol + (uint32_t)c0, v);
+                    tmem_ld32(dcol + (uint32_t)c0 + 32u, v + 32);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
+                    for (int i = 0; i < 64; i += 2) {
                         const f32x2 r2 = fma2_pairs(s2, f32x2{__uint_as_float(v[i]), __uint_as_float(v[i + 1])},
                                                     f32x2{acc[c0 + i], acc[c0 + i + 1]});
                         acc[c0 + i] = r2.x;
@@ -391,8 +445,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                     }
                 }
                 if (xs_wide[dr.slot]) {
-                    float zh;
-                    zp_split(bf16_to_f32(zrow[ks]), zh);
+                    const float zh = zhi_d[dr.slot * kTileN + r];
                     if (zh != 0.0f) {
                         const float t = -s * zh;
                         const float *xg = xsum + dr.slot * kBN;
@@ -482,6 +535,15 @@ int launch_gemm_w4a16_tc2(const uint16_t *x, int64_t M, int64_t N, int64_t K, co
     if (!encode_tmap_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, kBN,
                         CU_TENSOR_MAP_SWIZZLE_128B))
         return -1;
+    // scales and zero-points [N][G] bf16 in windows of 8 groups x 128 rows (the row stride G * 2 bytes is a
+    // multiple of 16 because K % 1024 == 0)
+    CUtensorMap smap, zmap;
+    const uint64_t G = (uint64_t)K / kStageK;
+    if (!encode_tmap_2d(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, s, G, (uint64_t)N, G * 2, kWinGroups, kTileN,
+                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_tmap_2d(&zmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, z, G, (uint64_t)N, G * 2, kWinGroups, kTileN,
+                        CU_TENSOR_MAP_SWIZZLE_NONE))
+        return -1;
     static std::mutex mu;
     static std::map<int, int> sms_of;
     int dev = 0;
@@ -507,7 +569,7 @@ int launch_gemm_w4a16_tc2(const uint16_t *x, int64_t M, int64_t N, int64_t K, co
     float *ws = reinterpret_cast<float *>(w8);
     int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, 128));
     gemm_w4a16_tc2_kernel<<<(unsigned)grid, kThreads, gemm_tc2_smem_bytes(), st>>>(
-        wmap, xmap, M, N, K, s, z, y, ws, counters, max_segs, status, 0x000F000Fu, 0x43004300u, skip_unit);
+        wmap, xmap, smap, zmap, M, N, K, y, ws, counters, max_segs, status, 0x000F000Fu, 0x43004300u, skip_unit);
     return 0;
 }
 

@@ -336,6 +336,25 @@ def test_gemm_w4a16_tensor_core_tiles(M, N, K, g):
     _w4_case(N, K, g, M, 17 * M + N)
 
 
+@pytest.mark.parametrize("M,N,K", [(65, 1000, 1024), (127, 300, 2048), (128, 128, 1024), (129, 640, 3072),
+                                   (200, 1000, 8192), (256, 257, 1024), (384, 384, 2048)])
+def test_gemm_w4a16_tensor_core_split_roles(M, N, K):
+    """The 128 x 128-tile form (g = 128, K a multiple of 1024) with dequantisation and promotion in separate
+    warps and the scales and zero-points in shared-memory windows: one and several M tiles, ragged N and M,
+    K ranges whose windows start mid-way through a CTA's share."""
+    _w4_case(N, K, 128, M, 31 * M + N + K)
+
+
+@pytest.mark.parametrize("M", [65, 128, 200])
+def test_gemm_w4a16_split_roles_zero_rows_and_far_zero_points(M):
+    N, K = 640, 2048
+    w = wq_inputs.llm_weight(N, K, 96, dtype=torch.float32)
+    w[::7] = 0.0
+    _w4_case(N, K, 128, M, 0, wgen=w, xgen=wq_inputs.wide_range_activations(M, K, 97 + M))
+    _w4_case(N, K, 128, M, 0, wgen=wq_inputs.offset_group_weight(N, K, 98),
+             xgen=wq_inputs.positive_activations(M, K, 99 + M))
+
+
 @pytest.mark.parametrize("N,K,g", [(1, 32, 32), (7, 64, 32), (129, 128, 64), (300, 1024, 128), (33, 4096, 32)])
 @pytest.mark.parametrize("M", [1, 4, 16, 40])
 def test_gemm_w4a16_shapes(N, K, g, M):
