@@ -629,7 +629,10 @@ size_t gemm_tc_partials_bytes(int64_t M, int64_t N, int64_t K, int g)
 
 bool gemm_tc_eligible(int64_t M, int64_t N, int64_t K, int g)
 {
-    return M > 16 && N >= kTileN && K >= kStageK && K % kStageK == 0 && (g == 32 || g == 64 || g == 128) &&
+    // M > 16; also 2 <= M <= 16 for groups of 32 and 64, which the TMA decode kernel does not take (the
+    // tensor cores still beat the CUDA-core kernel there: it spends one FMA per code and row of x)
+    const bool m_ok = M > 16 || (M >= 2 && (g == 32 || g == 64));
+    return m_ok && N >= kTileN && K >= kStageK && K % kStageK == 0 && (g == 32 || g == 64 || g == 128) &&
            K / 2 <= 0xffffffffLL && M <= 0x7fffffffLL;
 }
 

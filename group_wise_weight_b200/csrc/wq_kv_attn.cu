@@ -246,49 +246,65 @@ kv_attn_chunk_kernel(const KvArgs a)
 
     // ---------------- phase 1: scores of this warp's tokens ----------------
     const int wt0 = t0 + wid * kTokPerWarp;
+    // the next 16-token tile's loads are issued before the current tile is dequantised and multiplied
+    struct KRaw {
+        uint4 c0, c1, d0, d1;  // code bytes of tokens base + g (c) and base + g + 8 (d); int4 uses c0, d0
+        uint16_t sa, za, sb, zb;
+    };
+    auto load_k = [&](int base) {
+        KRaw t;
+        t.c0 = t.c1 = t.d0 = t.d1 = make_uint4(0, 0, 0, 0);
+        t.sa = t.sb = 0;
+        t.za = t.zb = 0;
+        const int ta = base + g, tb = base + g + 8;
+        if (ta < tend) {
+            const size_t v = vec0 + (size_t)ta * row_stride;
+            if (FP8) {
+                const uint4 *p = reinterpret_cast<const uint4 *>(a.kc + v * kRowBytes + 32 * tq);
+                t.c0 = ld_nc_v4(p);
+                t.c1 = ld_nc_v4(p + 1);
+            } else {
+                t.c0 = ld_nc_v4(a.kc + v * kRowBytes + 16 * tq);
+                t.sa = ld_nc_u16(a.ks + v);
+                t.za = ld_nc_u16(a.kz + v);
+            }
+        }
+        if (tb < tend) {
+            const size_t v = vec0 + (size_t)tb * row_stride;
+            if (FP8) {
+                const uint4 *p = reinterpret_cast<const uint4 *>(a.kc + v * kRowBytes + 32 * tq);
+                t.d0 = ld_nc_v4(p);
+                t.d1 = ld_nc_v4(p + 1);
+            } else {
+                t.d0 = ld_nc_v4(a.kc + v * kRowBytes + 16 * tq);
+                t.sb = ld_nc_u16(a.ks + v);
+                t.zb = ld_nc_u16(a.kz + v);
+            }
+        }
+        return t;
+    };
+    KRaw nxt = load_k(wt0);
 #pragma unroll 1
     for (int base = wt0; base < wt0 + kTokPerWarp && base < tend; base += 16) {
         const int ta = base + g, tb = base + g + 8;
         const bool la = ta < tend, lb = tb < tend;
+        const KRaw cur = nxt;
+        if (base + 16 < wt0 + kTokPerWarp && base + 16 < tend) nxt = load_k(base + 16);
         uint32_t A0[8][2], A1[8][2];
         float sa = 0.0f, sb = 0.0f, zha = 0.0f, zhb = 0.0f;
         if (FP8) {
-            uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0, d0 = c0, d1 = c0;
-            if (la) {
-                const uint4 *p = reinterpret_cast<const uint4 *>(a.kc + (vec0 + (size_t)ta * row_stride) * kRowBytes + 32 * tq);
-                c0 = ld_nc_v4(p);
-                c1 = ld_nc_v4(p + 1);
-            }
-            if (lb) {
-                const uint4 *p = reinterpret_cast<const uint4 *>(a.kc + (vec0 + (size_t)tb * row_stride) * kRowBytes + 32 * tq);
-                d0 = ld_nc_v4(p);
-                d1 = ld_nc_v4(p + 1);
-            }
-            fp8_row(c0, c1, A0);
-            fp8_row(d0, d1, A1);
+            fp8_row(cur.c0, cur.c1, A0);
+            fp8_row(cur.d0, cur.d1, A1);
             sa = k8;
             sb = k8;
         } else {
-            uint4 c = make_uint4(0, 0, 0, 0), d = c;
-            uint32_t za = 0x43004300u, zb = 0x43004300u;  // 128 + 0
-            if (la) {
-                const size_t v = vec0 + (size_t)ta * row_stride;
-                c = ld_nc_v4(a.kc + v * kRowBytes + 16 * tq);
-                sa = bf16_to_f32(ld_nc_u16(a.ks + v));
-                float z = bf16_to_f32(ld_nc_u16(a.kz + v));
-                if (!(z >= 0.0f && z <= 15.0f)) z = zp_split(z, zha);
-                za = bf16_pair_128_plus(z);
-            }
-            if (lb) {
-                const size_t v = vec0 + (size_t)tb * row_stride;
-                d = ld_nc_v4(a.kc + v * kRowBytes + 16 * tq);
-                sb = bf16_to_f32(ld_nc_u16(a.ks + v));
-                float z = bf16_to_f32(ld_nc_u16(a.kz + v));
-                if (!(z >= 0.0f && z <= 15.0f)) z = zp_split(z, zhb);
-                zb = bf16_pair_128_plus(z);
-            }
-            int4_row(c, za, A0);
-            int4_row(d, zb, A1);
+            sa = bf16_to_f32(cur.sa);
+            sb = bf16_to_f32(cur.sb);
+            float za = bf16_to_f32(cur.za), zb = bf16_to_f32(cur.zb);
+            if (!(za >= 0.0f && za <= 15.0f)) za = zp_split(za, zha);
+            if (!(zb >= 0.0f && zb <= 15.0f)) zb = zp_split(zb, zhb);
+            int4_row(cur.c0, bf16_pair_128_plus(za), A0);
+            int4_row(cur.d0, bf16_pair_128_plus(zb), A1);
         }
         float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
@@ -336,8 +352,40 @@ kv_attn_chunk_kernel(const KvArgs a)
     float lsum = 0.0f;   // sum of p over this thread's tokens, head g
     float zcorr = 0.0f;  // sum of p' z_hi over this thread's tokens, head g (zero-points outside [0, 15])
     const float mg = g < a.r ? hmax[g] : 0.0f;
+    // V codes (and, int4, the V scales and zero-points) of the 4 tokens 4 tq + u of a 16-token step: the
+    // next step's are loaded before the current one is used
+    struct VRaw {
+        uint4 c[4];  // fp8: 16 bytes (d = 16 g ..) per token; int4: 8 bytes in .x, .y
+        uint16_t s[4], z[4];
+    };
+    auto load_v = [&](int base) {
+        VRaw t;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int tt = base + 4 * tq + u;
+            t.c[u] = make_uint4(0, 0, 0, 0);
+            t.s[u] = 0;
+            t.z[u] = 0;
+            if (tt < tend) {
+                const size_t v = vec0 + (size_t)tt * row_stride;
+                if (FP8) {
+                    t.c[u] = ld_nc_v4(a.vc + v * kRowBytes + 16 * g);
+                } else {
+                    const uint2 w2 = *reinterpret_cast<const uint2 *>(a.vc + v * kRowBytes + 8 * g);
+                    t.c[u].x = w2.x;
+                    t.c[u].y = w2.y;
+                    t.s[u] = ld_nc_u16(a.vs + v);
+                    t.z[u] = ld_nc_u16(a.vz + v);
+                }
+            }
+        }
+        return t;
+    };
+    VRaw vnext = load_v(wt0);
 #pragma unroll 1
     for (int base = wt0; base < wt0 + kTokPerWarp && base < tend; base += 16) {
+        const VRaw vcur = vnext;
+        if (base + 16 < wt0 + kTokPerWarp && base + 16 < tend) vnext = load_v(base + 16);
         float pv[4];  // p' of tokens 4 tq + u, head g: p * s_t (int4) or p (fp8; its scale is applied at the end)
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -347,45 +395,27 @@ kv_attn_chunk_kernel(const KvArgs a)
             pv[u] = p;
         }
         if constexpr (FP8) {
-            // 16 code bytes (d = 16 g .. 16 g + 15) of each of the 4 tokens
-            uint4 c[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int t = base + 4 * tq + u;
-                c[u] = t < tend ? ld_nc_v4(a.vc + (vec0 + (size_t)t * row_stride) * kRowBytes + 16 * g)
-                                : make_uint4(0, 0, 0, 0);
-            }
             const uint32_t b0 = f16x2_of(pv[0], pv[1]), b1 = f16x2_of(pv[2], pv[3]);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 // m tile i: row g takes d = 16 g + 2 i, row g + 8 takes d = 16 g + 2 i + 1 (bytes 2 i, 2 i + 1)
                 const int wi = i >> 1;
                 const uint32_t s_lo = (i & 1) ? 0x0062u : 0x0040u, s_hi = (i & 1) ? 0x0073u : 0x0051u;
-                const uint32_t x0 = word_of4(c[0], wi), x1 = word_of4(c[1], wi);
-                const uint32_t x2 = word_of4(c[2], wi), x3 = word_of4(c[3], wi);
+                const uint32_t x0 = word_of4(vcur.c[0], wi), x1 = word_of4(vcur.c[1], wi);
+                const uint32_t x2 = word_of4(vcur.c[2], wi), x3 = word_of4(vcur.c[3], wi);
                 mma_f16(o[i], e4m3x2_f16x2(__byte_perm(x0, x1, s_lo)), e4m3x2_f16x2(__byte_perm(x0, x1, s_hi)),
                         e4m3x2_f16x2(__byte_perm(x2, x3, s_lo)), e4m3x2_f16x2(__byte_perm(x2, x3, s_hi)), b0, b1);
             }
         } else {
-            // 8 code bytes (d = 16 g .. 16 g + 15) of each of the 4 tokens, their V scales and zero-points
-            uint2 c[4];
             float zh[4];
             uint32_t zlo[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int t = base + 4 * tq + u;
-                c[u] = make_uint2(0, 0);
                 zh[u] = 0.0f;
-                float s = 0.0f, z = 0.0f;
-                if (t < tend) {
-                    const size_t v = vec0 + (size_t)t * row_stride;
-                    c[u] = *reinterpret_cast<const uint2 *>(a.vc + v * kRowBytes + 8 * g);
-                    s = bf16_to_f32(ld_nc_u16(a.vs + v));
-                    z = bf16_to_f32(ld_nc_u16(a.vz + v));
-                    if (!(z >= 0.0f && z <= 15.0f)) z = zp_split(z, zh[u]);
-                }
+                float z = bf16_to_f32(vcur.z[u]);
+                if (!(z >= 0.0f && z <= 15.0f)) z = zp_split(z, zh[u]);
                 zlo[u] = __float_as_uint(128.0f + z) >> 16;  // bf16 of 128 + z_lo (exact)
-                pv[u] *= s;
+                pv[u] *= bf16_to_f32(vcur.s[u]);
             }
             const uint32_t zz0 = zlo[0] | (zlo[1] << 16), zz1 = zlo[2] | (zlo[3] << 16);
             const uint32_t b0 = pack_bf16x2(pv[0], pv[1]), b1 = pack_bf16x2(pv[2], pv[3]);
@@ -399,8 +429,8 @@ kv_attn_chunk_kernel(const KvArgs a)
                 // byte bi of the first token to bits 0-7, of the second to bits 16-23 (bytes 1 and 3 take a copy
                 // of byte 0 of the first word, which the nibble masks below discard)
                 const uint32_t sel = (uint32_t)(bi | ((4 + bi) << 8));
-                const uint32_t x0 = wi ? c[0].y : c[0].x, x1 = wi ? c[1].y : c[1].x;
-                const uint32_t x2 = wi ? c[2].y : c[2].x, x3 = wi ? c[3].y : c[3].x;
+                const uint32_t x0 = wi ? vcur.c[0].y : vcur.c[0].x, x1 = wi ? vcur.c[1].y : vcur.c[1].x;
+                const uint32_t x2 = wi ? vcur.c[2].y : vcur.c[2].x, x3 = wi ? vcur.c[3].y : vcur.c[3].x;
                 const uint32_t pa = __byte_perm(x0, x1, sel);
                 const uint32_t pb = __byte_perm(x2, x3, sel);
                 mma_bf16(o[i], sub_bf16x2(lop_nib(pa), zz0), sub_bf16x2(lop_nib(pa >> 4), zz0),

@@ -189,9 +189,9 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * calls give identical bytes, except for 2 <= M <= 16, whose partials meet in
  * binary32 atomics (the last bits of y may then vary between calls).
  * Kernels: M = 1 with g = 128, 1024 <= K <= 32768, K % 1024 == 0: persistent
- * TMA-fed kernel; 2 <= M <= 16 with g = 128: TMA-fed decode kernel; M > 16
- * (N >= 128, K % 128 == 0): tcgen05 tensor-core kernel; other shapes: a
- * CUDA-core kernel.
+ * TMA-fed kernel; 2 <= M <= 16 with g = 128: TMA-fed decode kernel; M > 16,
+ * or 2 <= M <= 16 with g = 32 or 64 (N >= 128, K % 128 == 0): tcgen05
+ * tensor-core kernels; other shapes: a CUDA-core kernel.
  * Requirements: M, N >= 1; K % 32 == 0; g in {32, 64, 128}, K % g == 0;
  * pointers 16-byte aligned; workspace of wq_gemm_workspace_bytes(M, N, K, g, 4)
  * bytes (may be NULL when that is 0).  y must not overlap x, qweight,
