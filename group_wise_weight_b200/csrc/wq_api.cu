@@ -259,6 +259,7 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
         if (wq::gemv_m1_eligible(M, N, K, g)) return wq::gemv_m1_workspace_bytes(M, N, K, g);
         return wq::gemv_tma_workspace_bytes(M, N, K, g);
     }
+    if (wbits == 8) return wq::gemm_tc_w8_workspace_bytes(M, N, K, g);
     return 0;
 }
 
@@ -285,6 +286,14 @@ int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8
     const size_t need = wq_gemm_workspace_bytes(M, N, K, g, 8);
     if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
         return fail(WQ_ERR_WORKSPACE, "wq_gemm_w8a16: need %zu workspace bytes", need);
+    if (wq::gemm_tc_w8_eligible(M, N, K, g)) {
+        int *status = status_word();
+        if (!status) return fail(WQ_ERR_CUDA, "wq_gemm_w8a16: no device status word");
+        if (wq::launch_gemm_w8a16_tc(x, M, N, K, qweight, scales, g, y, workspace, status,
+                                     static_cast<cudaStream_t>(stream)) != 0)
+            return fail(WQ_ERR_CUDA, "wq_gemm_w8a16: tensor map encoding failed");
+        return check_launch("wq_gemm_w8a16");
+    }
     wq::launch_gemv_w8a16(x, M, N, K, qweight, scales, g, y, static_cast<cudaStream_t>(stream));
     return check_launch("wq_gemm_w8a16");
 }

@@ -65,19 +65,23 @@ constexpr int kKPerWarp = 128 / kWPQ;       // k of a stage each dequant warp ha
 constexpr int kChunksPerWarp = kKPerWarp / 32;  // 16-byte code chunks per thread and stage
 constexpr int kFirstDequantWarp = 3;  // warps 0, 1, 2: weight producer, MMA issuer, activation producer
 constexpr int kThreads = (kFirstDequantWarp + kDequantWarps) * 32;
-constexpr int kWeightStageBytes = kTileN * (kStageK / 2);  // 8 KB
 constexpr uint32_t kTmemCols = 512;  // A: kABufs x 64 columns, D: 2 x 128/g x BN = 256 columns
 constexpr uint32_t kABufs = 4;       // dequantised weight tiles in tensor memory
 
-template <int BN>
+// W8: int8 weights (W8A16), one byte per code, 128-byte rows per stage with the 128-byte swizzle;
+// otherwise packed INT4, 64-byte rows with the 64-byte swizzle.
+template <int BN, bool W8 = false>
 struct Cfg {
+    static constexpr int kWRowBytes = W8 ? 128 : 64;             // bytes of a weight row per stage
+    static constexpr int kWStageBytes = kTileN * kWRowBytes;     // 16 KB or 8 KB
+    static constexpr int kWSt = W8 ? 6 : kWStages;               // weight stages in flight
     static constexpr int kXAtomBytes = BN * 128;             // BN rows x 64 bf16
     static constexpr int kXStageBytes = 2 * kXAtomBytes;     // 128 k of activations
     static constexpr int kXStages = BN == 128 ? 3 : (BN == 64 ? 4 : 6);
     static constexpr size_t kWOff = (size_t)kXStages * kXStageBytes;
-    static constexpr size_t kBarOff = kWOff + (size_t)kWStages * kWeightStageBytes;
+    static constexpr size_t kBarOff = kWOff + (size_t)kWSt * kWStageBytes;
     // x_full[XS], x_empty[XS], w_full[WS], w_empty[WS], a_full[A], a_empty[A], d_full[2], d_empty[2], done
-    static constexpr size_t kFlagOff = kBarOff + (2 * kXStages + 2 * kWStages + 2 * kABufs + 4 + 1) * 8;
+    static constexpr size_t kFlagOff = kBarOff + (2 * kXStages + 2 * kWSt + 2 * kABufs + 4 + 1) * 8;
     // flags: abort, last-arrival, tensor-memory address, far-zero-point marks; then activation sums
     static constexpr size_t kXsumOff = kFlagOff + 64;
     static constexpr size_t kBytes = kXsumOff + 2 * 128 * 4;  // [2 D buffers][groups][BN], groups x BN <= 128
@@ -124,14 +128,34 @@ struct Ring {
     }
 };
 
-template <int BN, int GROUP>
+// Eight int8 codes (two words) as four exact bf16 pairs (k, k + 1): each byte, flipped to q + 128, is placed
+// under the exponent of 2^23 by one byte permute (2^23 + q + 128, exact in binary32), one subtraction gives q,
+// and the pair is packed to bf16 (exact: |q| <= 128 has at most 8 significant bits).
+__device__ __forceinline__ void int8x8_bf16(uint32_t w0, uint32_t w1, uint32_t out[4])
+{
+    const uint32_t u[2] = {w0 ^ 0x80808080u, w1 ^ 0x80808080u};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float f[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            f[j] = __fsub_rn(__uint_as_float(__byte_perm(u[h], 0x4B000000u, 0x7540u | (uint32_t)j)), 8388736.0f);
+        out[2 * h] = pack_bf16x2(f[0], f[1]);
+        out[2 * h + 1] = pack_bf16x2(f[2], f[3]);
+    }
+}
+
+template <int BN, int GROUP, bool W8>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, int64_t M,
                      int64_t N, int64_t K, const uint16_t *__restrict__ sc, const uint16_t *__restrict__ zp,
                      uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ counters, int max_segs,
-                     int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic, int64_t skip_unit)
+                     int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic, int64_t skip_unit,
+                     int s_per_row)
 {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, W8>;
+    constexpr int kWStagesK = C::kWSt;
+    constexpr int kWeightStageBytes = C::kWStageBytes;
     constexpr int NG = kStageK / GROUP;     // groups per stage
     constexpr int kDCols = NG * BN;         // accumulator columns per stage
     constexpr uint32_t XS = (uint32_t)C::kXStages;
@@ -141,8 +165,8 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     uint64_t *x_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *x_empty = x_full + XS;
     uint64_t *w_full = x_empty + XS;
-    uint64_t *w_empty = w_full + kWStages;
-    uint64_t *a_full = w_empty + kWStages;
+    uint64_t *w_empty = w_full + kWStagesK;
+    uint64_t *a_full = w_empty + kWStagesK;
     uint64_t *a_empty = a_full + kABufs;
     uint64_t *d_full = a_empty + kABufs;
     uint64_t *d_empty = d_full + 2;
@@ -174,7 +198,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             mbar_init(&x_full[i], 1);
             mbar_init(&x_empty[i], 1);
         }
-        for (int i = 0; i < kWStages; ++i) {
+        for (int i = 0; i < kWStagesK; ++i) {
             mbar_init(&w_full[i], 1);
             mbar_init(&w_empty[i], kDequantWarps);
         }
@@ -203,7 +227,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         // ------------------------------ TMA producers ------------------------------
         // warp 0: weight boxes into the weight ring; warp 2: activation boxes into the activation ring
         const bool weights = wid == 0;
-        const uint32_t nst = weights ? (uint32_t)kWStages : XS;
+        const uint32_t nst = weights ? (uint32_t)kWStagesK : XS;
         uint64_t *fullb = weights ? w_full : x_full;
         uint64_t *emptyb = weights ? w_empty : x_empty;
         if (lane == 0 && beg < end) {
@@ -220,7 +244,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     if (u != skip_unit) {
                         mbar_arrive_expect_tx(&fullb[rg.slot], kWeightStageBytes);
                         tma_load_2d(smem + C::kWOff + rg.slot * kWeightStageBytes, &wmap, &fullb[rg.slot],
-                                    ks * (kStageK / 2), nt * kTileN);
+                                    ks * C::kWRowBytes, nt * kTileN);
                     }
                 } else {
                     uint8_t *st = smem + rg.slot * C::kXStageBytes;
@@ -323,12 +347,15 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
         constexpr int kCols = BN / kWPQ;         // accumulator columns this warp promotes
         const int G = (int)(K / GROUP);
-        // this thread's code chunks in a weight slot: row r, chunks kq*kChunksPerWarp + i, 64-byte swizzle
-        uint32_t w_addr[kChunksPerWarp];
+        // this thread's 16-byte code chunks in a weight slot: row r; INT4: chunks kq*2 + i of a 64-byte row
+        // (64-byte swizzle); int8: chunks kq*4 + i of a 128-byte row (128-byte swizzle)
+        constexpr int kCh = W8 ? 4 : kChunksPerWarp;
+        uint32_t w_addr[kCh];
 #pragma unroll
-        for (int i = 0; i < kChunksPerWarp; ++i)
-            w_addr[i] = smem_u32(smem + C::kWOff) + (uint32_t)r * 64u +
-                        16u * ((uint32_t)(kq * kChunksPerWarp + i) ^ (uint32_t)((r >> 1) & 3));
+        for (int i = 0; i < kCh; ++i)
+            w_addr[i] = W8 ? smem_u32(smem + C::kWOff) + (uint32_t)r * 128u + 16u * ((uint32_t)(kq * 4 + i) ^ (uint32_t)(r & 7))
+                           : smem_u32(smem + C::kWOff) + (uint32_t)r * 64u +
+                                 16u * ((uint32_t)(kq * kChunksPerWarp + i) ^ (uint32_t)((r >> 1) & 3));
         const uint32_t a_addr = tmem + lane_bits + (uint32_t)(kq * kKPerWarp / 2);
         const uint32_t dq_addr = d_tmem + lane_bits + (uint32_t)(kq * kCols);
         Ring wr, ar, pr;  // weight ring, A buffers, D buffers being promoted
@@ -396,8 +423,10 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             const int64_t nt = tile % S.n_tiles, mt = tile / S.n_tiles;
             const int64_t n = nt * kTileN + r;
             const int64_t nrow = n < N ? n : N - 1;
-            const uint16_t *sp = sc + nrow * G + (int64_t)ks0 * NG;  // scales of the stage's groups
-            const uint16_t *zbase = zp + nrow * G;                    // zero-points of the row
+            // scales of the stage's groups (one scale per row when s_per_row: int8 per channel)
+            const uint16_t *sp = s_per_row ? sc + nrow : sc + nrow * G + (int64_t)ks0 * NG;
+            const int sp_step = s_per_row ? 0 : NG;
+            const uint16_t *zbase = W8 ? nullptr : zp + nrow * G;    // zero-points of the row
             zrow = zbase;
             // a warp's k range of a stage lies in one group when the group is at least that long
             constexpr bool kOneZ = GROUP >= kKPerWarp;
@@ -406,9 +435,9 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             // scales and zero-points are loaded one stage ahead of their use
             uint16_t snext[NG], znext[kZ];
 #pragma unroll
-            for (int gi = 0; gi < NG; ++gi) snext[gi] = sp[gi];
+            for (int gi = 0; gi < NG; ++gi) snext[gi] = sp[s_per_row ? 0 : gi];
 #pragma unroll
-            for (int i = 0; i < kZ; ++i) znext[i] = zbase[zidx(ks0, i)];
+            for (int i = 0; i < kZ; ++i) znext[i] = W8 ? (uint16_t)0 : zbase[zidx(ks0, i)];
 #pragma unroll
             for (int c = 0; c < kCols; ++c) acc[c] = 0.0f;
 
@@ -418,9 +447,9 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     mbar_wait_fast(&a_empty[ar.slot], ar.phase ^ 1u, status, abort_flag);
                     tc_fence_after();  // the tcgen05.st below must not move ahead of this wait
                 }
-                uint4 wv[kChunksPerWarp];
+                uint4 wv[kCh];
 #pragma unroll
-                for (int i = 0; i < kChunksPerWarp; ++i)
+                for (int i = 0; i < kCh; ++i)
                     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                                  : "=r"(wv[i].x), "=r"(wv[i].y), "=r"(wv[i].z), "=r"(wv[i].w)
                                  : "r"(w_addr[i] + wr.slot * (uint32_t)kWeightStageBytes));
@@ -432,7 +461,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 #pragma unroll
                 for (int i = 0; i < kZ; ++i) {
                     float zl = bf16_to_f32(znext[i]);
-                    if (!(zl >= 0.0f && zl <= 15.0f)) {
+                    if (!W8 && !(zl >= 0.0f && zl <= 15.0f)) {
                         float zh;
                         zl = zp_split(zl, zh);
                         wide = true;
@@ -440,14 +469,26 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     const float zc = 128.0f + zl;  // 128 .. 143: exact in bf16
                     z2s[i] = pack_bf16x2(zc, zc);
                 }
-                sp += NG;
+                sp += sp_step;
                 if (ks + 1 < ks1) {
 #pragma unroll
-                    for (int gi = 0; gi < NG; ++gi) snext[gi] = sp[gi];
+                    for (int gi = 0; gi < NG; ++gi) snext[gi] = sp[s_per_row ? 0 : gi];
+                    if (!W8) {
 #pragma unroll
-                    for (int i = 0; i < kZ; ++i) znext[i] = zbase[zidx(ks + 1, i)];
+                        for (int i = 0; i < kZ; ++i) znext[i] = zbase[zidx(ks + 1, i)];
+                    }
                 }
                 uint32_t A[kKPerWarp / 2];
+                if (W8) {
+                    // int8 codes are the operand itself: q exactly in bf16, natural k order
+#pragma unroll
+                    for (int i = 0; i < kCh; ++i) {
+                        int8x8_bf16(wv[i].x, wv[i].y, A + i * 8);
+                        int8x8_bf16(wv[i].z, wv[i].w, A + i * 8 + 4);
+                    }
+                    tmem_st16(a_addr + ar.slot * 64u, A);
+                    tmem_st16(a_addr + ar.slot * 64u + 16u, A + 16);
+                } else
 #pragma unroll
                 for (int i = 0; i < kChunksPerWarp; ++i) {
                     // zero-point of this 32-k chunk (a chunk never straddles a group: g >= 32)
@@ -475,7 +516,7 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     mbar_arrive(&w_empty[wr.slot]);
                     mbar_arrive(&a_full[ar.slot]);
                 }
-                wr.next(kWStages);
+                wr.next(kWStagesK);
                 ar.next(kABufs);
                 // promote the previous stage of this segment while this one is multiplied
                 if (ks > ks0) promote(ks - 1);
@@ -549,22 +590,24 @@ std::atomic<int64_t> g_skip_unit{-1};
 
 int64_t test_take_skip_unit() { return g_skip_unit.exchange(-1); }
 
-template <int BN, int GROUP>
+template <int BN, int GROUP, bool W8>
 int run(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s, const uint16_t *z,
-        uint16_t *y, void *workspace, int *status, cudaStream_t st)
+        int s_per_row, uint16_t *y, void *workspace, int *status, cudaStream_t st)
 {
+    using C = Cfg<BN, W8>;
     CUtensorMap wmap, xmap;
-    if (!encode_tmap_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, (uint64_t)(K / 2), (uint64_t)N, (uint64_t)(K / 2),
-                        kStageK / 2, kTileN, CU_TENSOR_MAP_SWIZZLE_64B))
+    const uint64_t rowb = W8 ? (uint64_t)K : (uint64_t)(K / 2);
+    if (!encode_tmap_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, rowb, (uint64_t)N, rowb, C::kWRowBytes, kTileN,
+                        W8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
         return -1;
     if (!encode_tmap_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, BN,
                         CU_TENSOR_MAP_SWIZZLE_128B))
         return -1;
-    auto kern = gemm_w4a16_tc_kernel<BN, GROUP>;
+    auto kern = gemm_w4a16_tc_kernel<BN, GROUP, W8>;
     // at least 120 KB so that one CTA owns each SM (and its tensor memory)
-    const size_t smem = std::max<size_t>(Cfg<BN>::kBytes + 1024, 120 * 1024);
+    const size_t smem = std::max<size_t>(C::kBytes + 1024, 120 * 1024);
     static std::mutex mu;
-    static std::map<int, int> sms_of;
+    static std::map<int, int> sms_of;  // per device, for this instantiation: SM count once its attribute is set
     int dev = 0;
     cudaGetDevice(&dev);
     int sms;
@@ -575,12 +618,7 @@ int run(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, co
             int v = 148, optin = 0;
             cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
             cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<32, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<32, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<64, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<32, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<64, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-            cudaFuncSetAttribute(gemm_w4a16_tc_kernel<128, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
             it = sms_of.emplace(dev, v).first;
         }
         sms = it->second;
@@ -593,7 +631,8 @@ int run(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, co
     float *ws = reinterpret_cast<float *>(w8);
     int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, GROUP));
     kern<<<(unsigned)grid, kThreads, smem, st>>>(wmap, xmap, M, N, K, s, z, y, ws, counters, max_segs, status,
-                                                  0x000F000Fu, 0x43004300u, test_take_skip_unit());
+                                                  0x000F000Fu, 0x43004300u, W8 ? -1 : test_take_skip_unit(),
+                                                  s_per_row);
     return 0;
 }
 
@@ -651,12 +690,45 @@ int launch_gemm_w4a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, con
     // the 128 x 128-tile, g = 128 case runs the form with dequantisation and promotion in separate warps
     if (bn == 128 && g == 128 && K % 1024 == 0)
         return launch_gemm_w4a16_tc2(x, M, N, K, q, s, z, y, workspace, status, st, test_take_skip_unit());
-    if (g == 32) return run<32, 32>(x, M, N, K, q, s, z, y, workspace, status, st);
-    if (g == 64) return bn == 32 ? run<32, 64>(x, M, N, K, q, s, z, y, workspace, status, st)
-                                 : run<64, 64>(x, M, N, K, q, s, z, y, workspace, status, st);
-    if (bn == 32) return run<32, 128>(x, M, N, K, q, s, z, y, workspace, status, st);
-    if (bn == 64) return run<64, 128>(x, M, N, K, q, s, z, y, workspace, status, st);
-    return run<128, 128>(x, M, N, K, q, s, z, y, workspace, status, st);
+    if (g == 32) return run<32, 32, false>(x, M, N, K, q, s, z, 0, y, workspace, status, st);
+    if (g == 64) return bn == 32 ? run<32, 64, false>(x, M, N, K, q, s, z, 0, y, workspace, status, st)
+                                 : run<64, 64, false>(x, M, N, K, q, s, z, 0, y, workspace, status, st);
+    if (bn == 32) return run<32, 128, false>(x, M, N, K, q, s, z, 0, y, workspace, status, st);
+    if (bn == 64) return run<64, 128, false>(x, M, N, K, q, s, z, 0, y, workspace, status, st);
+    return run<128, 128, false>(x, M, N, K, q, s, z, 0, y, workspace, status, st);
+}
+
+bool gemm_tc_w8_eligible(int64_t M, int64_t N, int64_t K, int g)
+{
+    return M >= 2 && N >= kTileN && K >= kStageK && K % kStageK == 0 &&
+           (g == 32 || g == 64 || g == 128 || (int64_t)g == K) && K <= 0x7fffffffLL && M <= 0x7fffffffLL;
+}
+
+// The promotion group of an int8 call: its group size, or 128 (one stage) for one scale per row.
+static int w8_group(int64_t K, int g) { return (int64_t)g == K ? 128 : g; }
+
+size_t gemm_tc_w8_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
+{
+    if (!gemm_tc_w8_eligible(M, N, K, g)) return 0;
+    const int ge = w8_group(K, g);
+    const int BN = gemm_tc_bn(M, ge);
+    const int64_t tiles = ((N + kTileN - 1) / kTileN) * ((M + BN - 1) / BN);
+    return gemm_tc_partials_bytes(M, N, K, ge) + (sizeof(int) * (size_t)tiles + 255) / 256 * 256;
+}
+
+int launch_gemm_w8a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *q8, const uint16_t *s,
+                         int g, uint16_t *y, void *workspace, int *status, cudaStream_t st)
+{
+    const uint8_t *q = reinterpret_cast<const uint8_t *>(q8);
+    const int ge = w8_group(K, g);
+    const int per_row = (int64_t)g == K ? 1 : 0;
+    const int bn = gemm_tc_bn(M, ge);
+    if (ge == 32) return run<32, 32, true>(x, M, N, K, q, s, nullptr, per_row, y, workspace, status, st);
+    if (ge == 64) return bn == 32 ? run<32, 64, true>(x, M, N, K, q, s, nullptr, per_row, y, workspace, status, st)
+                                  : run<64, 64, true>(x, M, N, K, q, s, nullptr, per_row, y, workspace, status, st);
+    if (bn == 32) return run<32, 128, true>(x, M, N, K, q, s, nullptr, per_row, y, workspace, status, st);
+    if (bn == 64) return run<64, 128, true>(x, M, N, K, q, s, nullptr, per_row, y, workspace, status, st);
+    return run<128, 128, true>(x, M, N, K, q, s, nullptr, per_row, y, workspace, status, st);
 }
 
 }  // namespace wq

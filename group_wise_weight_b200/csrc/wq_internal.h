@@ -60,6 +60,12 @@ bool gemm_tc_eligible(int64_t M, int64_t N, int64_t K, int g);
 size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
 int launch_gemm_w4a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
                          const uint16_t *z, int g, uint16_t *y, void *workspace, int *status, cudaStream_t st);
+// W8A16 on the same tensor-core kernel (int8 codes converted exactly to bf16 in the dequant warps):
+// M >= 2, N >= 128, K % 128 == 0, g in {32, 64, 128, K}.  Workspace as the W4A16 form's.
+bool gemm_tc_w8_eligible(int64_t M, int64_t N, int64_t K, int g);
+size_t gemm_tc_w8_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
+int launch_gemm_w8a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *q, const uint16_t *s,
+                         int g, uint16_t *y, void *workspace, int *status, cudaStream_t st);
 // The 128 x 128-tile, g = 128 form with dequantisation and promotion in separate warps (wq_gemm_tc2.cu): the
 // same workspace layout as gemm_tc_workspace_bytes(M, N, K, 128) with BN = 128.  skip_unit: failure-path
 // tests only (-1 otherwise).

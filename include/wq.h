@@ -209,8 +209,12 @@ int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint
 /*
  * W8A16 weight-only matmul: y[m][n] = sum_k x[m][k] * s[n][k/g] * q[n][k]
  * ([P3] dequantised value q * s).  qweight [N][K] int8, scales [N][K/g]
- * bf16, g in {32, 64, 128, K}.  Other arguments and guarantees as
- * wq_gemm_w4a16.
+ * bf16, g in {32, 64, 128, K}.  Kernels: M >= 2 with N >= 128 and
+ * K % 128 == 0: the tcgen05 tensor-core kernel (q converted exactly to bf16,
+ * binary32 accumulation per group of g, or per 128 k for g = K, scaled and
+ * summed in binary32); otherwise a CUDA-core kernel.  Workspace of
+ * wq_gemm_workspace_bytes(M, N, K, g, 8) bytes.  Other arguments and
+ * guarantees as wq_gemm_w4a16 (y is deterministic for every M here).
  */
 int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *qweight,
                   const uint16_t *scales, int g, uint16_t *y, void *workspace, size_t ws_bytes,

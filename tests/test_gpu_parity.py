@@ -472,11 +472,39 @@ def _w8_case(w, x, g, rows=None):
 
 
 @pytest.mark.parametrize("M", [1, 2, 5, 16, 17, 64, 128])
-@pytest.mark.parametrize("g", [None, 32, 128])
+@pytest.mark.parametrize("g", [None, 32, 64, 128])
 def test_gemm_w8a16(M, g):
     w = wq_inputs.block_outlier_weight(600, 1024, 200 + M)
     x = wq_inputs.activations(M, 1024, 300 + M)
     _w8_case(w, x, g)
+
+
+@pytest.mark.parametrize("M,N,K,g", [
+    (4, 100, 1024, 32),     # N < 128: CUDA-core kernel
+    (4, 256, 1056, 32),     # K % 128 != 0: CUDA-core kernel
+    (130, 300, 384, None),  # two 128-row activation tiles, the second of 2 rows; ragged N
+    (40, 128, 128, 128),    # one stage, one weight tile
+    (3, 1000, 2048, 64),    # many K-splits of a few tiles
+])
+def test_gemm_w8a16_kernel_boundaries(M, N, K, g):
+    w = wq_inputs.block_outlier_weight(N, K, 17 * M + N)
+    x = wq_inputs.activations(M, K, 19 * M + K)
+    _w8_case(w, x, g)
+
+
+def test_gemm_w8a16_repeatable_and_zero_rows():
+    """The tensor-core W8A16 path combines K-splits in a fixed order (identical bytes on repeat); rows of
+    zero weights give exactly zero."""
+    w = wq_inputs.block_outlier_weight(512, 4096, 23)
+    w[7] = 0.0
+    w[300] = 0.0
+    x = wq_inputs.activations(16, 4096, 29).cuda()
+    q, s = wq.wq_quantize_int8(w.cuda(), 128)
+    y1 = wq.wq_gemm_w8a16(x, q, s, 128)
+    y2 = wq.wq_gemm_w8a16(x, q, s, 128)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert not y1[:, 7].any() and not y1[:, 300].any()
 
 
 def test_gemm_w8a16_gran_per_channel():
