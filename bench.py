@@ -638,6 +638,74 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------------------
 
+CASES = ("fp8", "nvfp4", "quant_int4", "kv_int4", "kv_fp8", "w8a16", "w4a16_m128", "w4a16_m1")
+
+
+def run_case(name, wq, dev):
+    """One small case of one kernel, run twice (a warm-up launch, then the one a profiler captures): the
+    gate+up shape (K = 8192, N = 57,344) for the matmuls and the quantiser, 32 sequences of 8,000 tokens for
+    the KV-cache read.  Prints one JSON line with the second launch's time."""
+    M, N, K = 128, 57344, 8192
+    calls = []
+    if name in ("fp8", "nvfp4"):
+        w = wq_inputs.llm_weight(N, K, 1, device=dev)
+        x = wq_inputs.activations(M, K, 2, device=dev)
+        if name == "fp8":
+            qw, sw = wq.wq_quantize_fp8(w)
+            qx, sx = wq.wq_quantize_fp8_tensor(x)
+            calls.append(lambda: wq.wq_gemm_w8a8_fp8(qx, sx, qw, sw))
+        else:
+            nw, nx = wq.wq_quantize_nvfp4(w), wq.wq_quantize_nvfp4(x)
+            calls.append(lambda: wq.wq_gemm_nvfp4(*nx, *nw))
+        del w
+    elif name == "quant_int4":
+        w = wq_inputs.llm_weight(N, K, 3, device=dev)
+        calls.append(lambda: wq.wq_quantize_int4(w, 128))
+    elif name in ("kv_int4", "kv_fp8"):
+        B, T, H, Hq, D = 32, 8000, 8, 64, 128
+        q = wq_inputs.queries(B, Hq, D, 6, device=dev)
+        lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+        kv = []
+        for j in range(2):
+            c = wq_inputs.kv_cache(B, T, H, D, 60 + j, device=dev)
+            if name == "kv_int4":
+                qq, s, z = wq.wq_quantize_int4(c.reshape(B * T * H, D), 128)
+                kv.append((qq.reshape(B, T, H, D // 2), s, z))
+            else:
+                qq, s = wq.wq_quantize_fp8_tensor(c.reshape(B * T * H, D))
+                kv.append((qq.reshape(B, T, H, D), s))
+            del c
+        fn = wq.wq_decode_attention_int4 if name == "kv_int4" else wq.wq_decode_attention_fp8
+        calls.append(lambda: fn(q, *kv[0], *kv[1], lens))
+    elif name == "w8a16":
+        w = wq_inputs.llm_weight(8192, 8192, 7, device=dev)
+        q8, s8 = wq.wq_quantize_int8(w, None)
+        del w
+        x = wq_inputs.plain_activations(M, 8192, 8, device=dev)
+        calls.append(lambda: wq.wq_gemm_w8a16(x, q8, s8, None))
+    elif name in ("w4a16_m128", "w4a16_m1"):
+        w = wq_inputs.llm_weight(N, K, 9, outlier_frac=0.0, device=dev)
+        q4, s4, z4 = wq.wq_quantize_int4(w, 128)
+        del w
+        x = wq_inputs.plain_activations(M if name == "w4a16_m128" else 1, K, 10, device=dev)
+        ws = torch.zeros(max(1, wq.wq_gemm_workspace_bytes(x.shape[0], N, K, 128, 4)), dtype=torch.uint8, device=dev)
+        calls.append(lambda: wq.wq_gemm_w4a16(x, q4, s4, z4, 128, workspace=ws))
+    else:
+        raise SystemExit(f"unknown case {name}; one of {', '.join(CASES)}")
+    for c in calls:
+        c()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for c in calls:
+        c()
+    e1.record()
+    e1.synchronize()
+    if wq.wq_device_status() != wq.WQ_OK:
+        raise SystemExit(f"case {name}: device status {wq.wq_device_status()}")
+    print(json.dumps({"case": name, "us": round(e0.elapsed_time(e1) * 1e3, 2)}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -649,6 +717,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-configuration and NEXT rows")
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="run one small case of one kernel twice (for a profiler capture) and exit")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -661,6 +731,9 @@ def main():
     wq.lib()  # fails loudly if the CUDA library is missing
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    if args.case:
+        run_case(args.case, wq, device)
+        return
     peaks = load_peaks()
 
     model = Model(args.layers, wq, device)
