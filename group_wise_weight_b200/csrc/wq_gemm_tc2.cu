@@ -9,30 +9,43 @@
 // inside the kernel): the MMA takes the exact integers q - z from tensor
 // memory, each group of 128 k accumulates into its own tensor-memory region,
 // and s is applied in binary32 ("promotion", y += s * D_group).  What differs
-// is who does what.  In wq_gemm_tc.cu the same warps dequantise one stage and
-// then promote the previous one, so each stage's MMAs wait for a warp to get
-// through both; here
-//  * warp 0 loads weight stages (TMA, 64-byte swizzle), warp 2 activation
-//    stages (TMA, 128-byte swizzle), warp 1 allocates tensor memory and one
-//    lane issues the MMAs (A from tensor memory, B from shared memory);
+// is who does what:
+//  * warp 0 loads weight stages (TMA, 64-byte swizzle) and the scale and
+//    zero-point windows, warp 2 activation stages (TMA, 128-byte swizzle),
+//    warp 1 allocates tensor memory and its lane 0 alone runs the MMA loop
+//    (A from tensor memory, B from shared memory);
 //  * warps 4..11 (two warpgroups) only dequantise: codes from shared memory
-//    to bf16 q - z in tensor memory, up to four stages ahead of the MMAs;
-//  * warps 12..15 (one warpgroup) only promote, each thread holding its
-//    row's 128 binary32 accumulators, and write the output;
-//  * register budgets follow the roles (setmaxnreg): 64 for the control
-//    warpgroup, 96 for dequantisation, 240 for promotion (512 threads at
-//    launch x 128 registers = 65,536; 128 x 64 + 256 x 96 + 128 x 240 =
-//    63,488).  Waits are inlined (no calls): ptxas allocates registers per
-//    role only for straight-line code.
+//    to bf16 q - z in tensor memory, up to four stages ahead of the MMAs, and
+//    announce them two stages at a time (one tensor-memory store wait per
+//    pair);
+//  * warps 12..19 (two warpgroups) only promote, each thread holding 64 of its
+//    row's binary32 accumulators (warpgroup c has columns 64c .. 64c + 63),
+//    and write the output.
+// Per stage the MMA lane waits twice (activations landed; the stage's A
+// written and its D buffer promoted, one barrier that the dequantisation and
+// promotion warps both arrive on) and commits once: a single "MMA done"
+// barrier tells the activation producer, the dequantisation warps and the
+// promotion warps alike that the stage's buffers may be reused or read.
+// (Measured on this kernel's previous form: a 128 x 128 x 16 MMA with A in
+// tensor memory occupies the tensor core ~94 cycles, so 8 per stage ~750, and
+// three waits, three commits and a warp-wide loop in the MMA warp had
+// stretched each stage to ~1,700.)
+// Register budgets follow the roles (setmaxnreg): 640 threads at launch x 96
+// registers = 61,440 = 128 x 56 + 256 x 80 + 256 x 128 + 2,048 spare.  Waits
+// are inlined (no calls): ptxas allocates registers per role only for
+// straight-line code.
 // Scales and zero-points reach shared memory by TMA in windows of 8 groups x
-// 128 rows (rings of 4), issued by the weight producer with the weight
-// stages, so no warp waits on a global load of a parameter (needs
-// K % 1024 == 0 for the windows' row stride; other K take wq_gemm_tc.cu).
-// Tensor memory: four A buffers of 64 columns, two D buffers of 128.  A zero-
-// point outside [0, 15] is split as in wq_gemm_tc.cu (the dequant warp marks
-// the stage, the MMA warp sums that stage's activations, the promotion adds
-// -s z_hi times the sums).  Stream-K over (tile, stage) units, per-segment
-// binary32 partials summed in segment order.  Every wait is bounded.
+// 128 rows, issued by the weight producer (needs K % 1024 == 0 for the
+// windows' row stride; other K take wq_gemm_tc.cu).  Tensor memory: four A
+// buffers of 64 columns, two D buffers of 128.  A zero-point outside [0, 15]
+// is split as in wq_gemm_tc.cu: the dequantisation warps record z_hi per row
+// and mark the stage; each promotion warp then sums that stage's activations
+// for its 64 columns from global memory (in k order) and adds -s z_hi times
+// the sums.  The dequantisation and promotion warps do not leave their loops
+// when a wait fails (the abort flag makes every later wait return at once), so
+// their warp-level and named barriers stay matched.
+// Stream-K over (tile, stage) units, per-segment binary32 partials summed in
+// segment order.  Every wait is bounded.
 #include <algorithm>
 #include <atomic>
 #include <map>
@@ -48,29 +61,37 @@ namespace {
 constexpr int kTileN = 128;     // weight rows per tile (MMA M)
 constexpr int kBN = 128;        // activation rows per tile (MMA N)
 constexpr int kStageK = 128;    // k per stage = one group
-constexpr int kWStages = 8;
-constexpr int kXStages = 3;
+constexpr int kWStages = 6;
+constexpr int kXStages = 4;
 constexpr int kABufs = 4;
-constexpr int kThreads = 512;
-constexpr int kFirstDq = 4, kDqWarps = 8, kFirstPr = 12, kPrWarps = 4;
+constexpr int kRing = 4;        // stage-ready / MMA-done barriers, indexed by stage % kRing
+constexpr int kWideRing = 8;    // far-zero-point records, indexed by stage % kWideRing
+constexpr int kThreads = 640;
+constexpr int kFirstDq = 4, kDqWarps = 8, kFirstPr = 12, kPrWarps = 8;
+constexpr int kRegCtl = 56, kRegDq = 80, kRegPr = 128;
 constexpr int kWeightStageBytes = kTileN * (kStageK / 2);  // 8 KB
 constexpr int kXAtomBytes = kBN * 128;                     // 128 rows x 64 bf16
 constexpr int kXStageBytes = 2 * kXAtomBytes;              // 32 KB
 constexpr uint32_t kTmemCols = 512;                        // A 4 x 64, D 2 x 128
 constexpr int kWinGroups = 8;                              // groups (stages) per s / z window
-constexpr int kWinSlots = 4;                               // windows in flight per ring
+constexpr int kWinSlots = 2;                               // windows in flight per ring
 constexpr int kWinBytes = kTileN * kWinGroups * 2;         // 128 rows x 8 bf16 = 2 KB
 constexpr size_t kWOff = (size_t)kXStages * kXStageBytes;
 constexpr size_t kZwOff = kWOff + (size_t)kWStages * kWeightStageBytes;  // zero-point windows
 constexpr size_t kSwOff = kZwOff + (size_t)kWinSlots * kWinBytes;        // scale windows
 constexpr size_t kBarOff = kSwOff + (size_t)kWinSlots * kWinBytes;
-// x_full, x_empty [3]; w_full, w_empty [8]; a_full, a_empty [4]; d_full, d_empty [2]; done;
-// zw_full, zw_empty, sw_full, sw_empty [4]
-constexpr size_t kFlagOff = kBarOff + (2 * kXStages + 2 * kWStages + 2 * kABufs + 4 + 1 + 4 * kWinSlots) * 8;
-constexpr size_t kXsumOff = kFlagOff + 64;                    // [D buffer][BN] activation sums
-constexpr size_t kZhiAOff = kXsumOff + 2 * kBN * 4;           // [A buffer][row] z_hi of the stage
-constexpr size_t kZhiDOff = kZhiAOff + kABufs * kTileN * 4;   // [D buffer][row] the same, for the promotion
-constexpr size_t kSmemBytes = kZhiDOff + 2 * kTileN * 4;
+// x_full[XS]; w_full, w_empty [WS]; ready, done [R]; zw_full, zw_empty, sw_full, sw_empty [2]; drain
+constexpr int kBars = kXStages + 2 * kWStages + 2 * kRing + 4 * kWinSlots + 1;
+constexpr size_t kFlagOff = kBarOff + (size_t)kBars * 8;
+// flags: abort, last-arrival, tensor-memory address; far-zero-point marks [kWideRing] at +32
+constexpr size_t kZhiOff = kFlagOff + 64;  // [kWideRing][row] z_hi
+constexpr size_t kSmemBytes = kZhiOff + kWideRing * kTileN * 4;
+
+static_assert(kRing >= kXStages && kRing >= kABufs && kRing >= 3, "stage rings must cover the buffers");
+static_assert(kWideRing >= kABufs + 2, "far-zero-point records must outlive the promotion of their stage");
+static_assert(kWOff % 1024 == 0 && kZwOff % 128 == 0 && kSwOff % 128 == 0, "TMA destinations");
+static_assert(4 * kRegCtl + kDqWarps * kRegDq + kPrWarps * kRegPr <= (65536 / kThreads) / 8 * 8 * (kThreads / 32),
+              "register budgets exceed the launch's registers");
 
 struct Sched {
     int64_t n_tiles, tiles, spt, total, per, extra;
@@ -113,6 +134,12 @@ __device__ __forceinline__ uint32_t lop_and_or(uint32_t t, uint32_t mask, uint32
     return d;
 }
 
+// `count` arrivals at once (the promotion warps' share of the first two stages, whose D buffers start free).
+__device__ __forceinline__ void mbar_arrive_n(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int *status)
 {
     const uint64_t t0 = global_ns();
@@ -122,33 +149,28 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int *
 
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
-                      const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap zmap, int64_t M,
-                      int64_t N, int64_t K, uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ counters, int max_segs,
-                      int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic, int64_t skip_unit)
+                      const __grid_constant__ CUtensorMap smap, const __grid_constant__ CUtensorMap zmap,
+                      const uint16_t *__restrict__ x, int64_t M, int64_t N, int64_t K, uint16_t *__restrict__ y,
+                      float *__restrict__ ws, int *__restrict__ counters, int max_segs, int *__restrict__ status,
+                      uint32_t nib_mask, uint32_t bf16_magic, int64_t skip_unit)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     uint64_t *x_full = reinterpret_cast<uint64_t *>(smem + kBarOff);
-    uint64_t *x_empty = x_full + kXStages;
-    uint64_t *w_full = x_empty + kXStages;
+    uint64_t *w_full = x_full + kXStages;
     uint64_t *w_empty = w_full + kWStages;
-    uint64_t *a_full = w_empty + kWStages;
-    uint64_t *a_empty = a_full + kABufs;
-    uint64_t *d_full = a_empty + kABufs;
-    uint64_t *d_empty = d_full + 2;
-    uint64_t *done = d_empty + 2;
-    uint64_t *zw_full = done + 1;
+    uint64_t *ready = w_empty + kWStages;  // stage A written (8 dequant warps) and its D buffer free (8 promotion)
+    uint64_t *done = ready + kRing;        // the stage's MMAs completed (one commit)
+    uint64_t *zw_full = done + kRing;
     uint64_t *zw_empty = zw_full + kWinSlots;
     uint64_t *sw_full = zw_empty + kWinSlots;
     uint64_t *sw_empty = sw_full + kWinSlots;
+    uint64_t *drain = sw_empty + kWinSlots;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kFlagOff);
     volatile int *last_flag = abort_flag + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kFlagOff + 16);
-    volatile int *wide_mark = reinterpret_cast<volatile int *>(smem + kFlagOff + 32);  // [A buffer]
-    volatile int *xs_wide = wide_mark + kABufs;                                        // [D buffer]
-    float *xsum = reinterpret_cast<float *>(smem + kXsumOff);                          // [D buffer][BN]
-    float *zhi_a = reinterpret_cast<float *>(smem + kZhiAOff);                         // [A buffer][row]
-    float *zhi_d = reinterpret_cast<float *>(smem + kZhiDOff);                         // [D buffer][row]
+    volatile int *wide_mark = reinterpret_cast<volatile int *>(smem + kFlagOff + 32);  // [kWideRing]
+    float *zhi = reinterpret_cast<float *>(smem + kZhiOff);                             // [kWideRing][row]
 
     const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
     Sched S;
@@ -163,33 +185,29 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
     const int spt = (int)S.spt;
 
     if (tid == 0) {
-        for (int i = 0; i < kXStages; ++i) {
-            mbar_init(&x_full[i], 1);
-            mbar_init(&x_empty[i], 1);
-        }
+        for (int i = 0; i < kXStages; ++i) mbar_init(&x_full[i], 1);
         for (int i = 0; i < kWStages; ++i) {
             mbar_init(&w_full[i], 1);
             mbar_init(&w_empty[i], kDqWarps);
         }
-        for (int i = 0; i < kABufs; ++i) {
-            mbar_init(&a_full[i], kDqWarps);
-            mbar_init(&a_empty[i], 1);
-            wide_mark[i] = 0;
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(&ready[i], kDqWarps + kPrWarps);
+            mbar_init(&done[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&d_full[i], 2);  // the MMAs' completion, and the MMA warp's activation sums
-            mbar_init(&d_empty[i], kPrWarps);
-        }
-        mbar_init(done, 1);
         for (int i = 0; i < kWinSlots; ++i) {
             mbar_init(&zw_full[i], 1);
             mbar_init(&zw_empty[i], kDqWarps);
             mbar_init(&sw_full[i], 1);
             mbar_init(&sw_empty[i], kPrWarps);
         }
+        mbar_init(drain, 1);
+        for (int i = 0; i < kWideRing; ++i) wide_mark[i] = 0;
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
+        // stages 0 and 1 find their D buffers free
+        mbar_arrive_n(&ready[0], kPrWarps);
+        mbar_arrive_n(&ready[1], kPrWarps);
     }
     if (wid == 1) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
@@ -199,121 +217,94 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
     const uint32_t d_tmem = tmem + kABufs * 64u;  // D buffer b at column b * 128
 
     if (wid < kFirstDq) {
-        setmaxnreg_dec<64>();
-        if (wid == 0 || wid == 2) {
-            // ------------------------------ TMA producers ------------------------------
-            const bool weights = wid == 0;
-            const uint32_t nst = weights ? (uint32_t)kWStages : (uint32_t)kXStages;
-            uint64_t *fullb = weights ? w_full : x_full;
-            uint64_t *emptyb = weights ? w_empty : x_empty;
-            if (lane == 0 && beg < end) {
-                Ring rg;
-                uint32_t issued = 0;
-                int64_t tile = beg / spt;
-                int ks = (int)(beg - tile * spt);
-                uint32_t wins = 0;  // s / z windows issued (weight producer)
-                for (int64_t u = beg; u < end; ++u) {
-                    if (issued >= nst && !mbar_wait(&emptyb[rg.slot], rg.phase ^ 1u, status, abort_flag)) break;
-                    const int nt = (int)(tile % S.n_tiles), mt = (int)(tile / S.n_tiles);
-                    if (weights && (u == beg || (ks % kWinGroups) == 0)) {
-                        // the s and z of groups (ks & ~7) .. + 7 of the tile's 128 rows, one window each
-                        const uint32_t ws_ = wins % kWinSlots, wph = (wins / kWinSlots) & 1u;
-                        if (wins >= (uint32_t)kWinSlots &&
-                            (!mbar_wait(&zw_empty[ws_], wph ^ 1u, status, abort_flag) ||
-                             !mbar_wait(&sw_empty[ws_], wph ^ 1u, status, abort_flag)))
-                            break;
-                        mbar_arrive_expect_tx(&zw_full[ws_], kWinBytes);
-                        tma_load_2d(smem + kZwOff + ws_ * kWinBytes, &zmap, &zw_full[ws_], ks & ~(kWinGroups - 1), nt * kTileN);
-                        mbar_arrive_expect_tx(&sw_full[ws_], kWinBytes);
-                        tma_load_2d(smem + kSwOff + ws_ * kWinBytes, &smap, &sw_full[ws_], ks & ~(kWinGroups - 1), nt * kTileN);
-                        ++wins;
-                    }
-                    if (weights) {
-                        // skip_unit (failure-path tests only, -1 otherwise): these weights are never requested
-                        if (u != skip_unit) {
-                            mbar_arrive_expect_tx(&fullb[rg.slot], kWeightStageBytes);
-                            tma_load_2d(smem + kWOff + rg.slot * kWeightStageBytes, &wmap, &fullb[rg.slot],
-                                        ks * (kStageK / 2), nt * kTileN);
-                        }
-                    } else {
-                        uint8_t *st = smem + rg.slot * kXStageBytes;
-                        mbar_arrive_expect_tx(&fullb[rg.slot], kXStageBytes);
-                        tma_load_2d(st, &xmap, &fullb[rg.slot], ks * kStageK, mt * kBN);
-                        tma_load_2d(st + kXAtomBytes, &xmap, &fullb[rg.slot], ks * kStageK + 64, mt * kBN);
-                    }
-                    ++issued;
-                    rg.next(nst);
-                    if (++ks == spt) { ks = 0; ++tile; }
+        setmaxnreg_dec<kRegCtl>();
+        if (wid == 0 && lane == 0 && beg < end) {
+            // ------------------------------ weight and s / z producer ------------------------------
+            Ring rg;
+            uint32_t issued = 0, wins = 0;
+            int64_t tile = beg / spt;
+            int ks = (int)(beg - tile * spt);
+            for (int64_t u = beg; u < end; ++u) {
+                if (issued >= (uint32_t)kWStages && !mbar_wait(&w_empty[rg.slot], rg.phase ^ 1u, status, abort_flag))
+                    break;
+                const int nt = (int)(tile % S.n_tiles);
+                if (u == beg || (ks % kWinGroups) == 0) {
+                    // the s and z of groups (ks & ~7) .. + 7 of the tile's 128 rows, one window each
+                    const uint32_t ws_ = wins % kWinSlots, wph = (wins / kWinSlots) & 1u;
+                    if (wins >= (uint32_t)kWinSlots &&
+                        (!mbar_wait(&zw_empty[ws_], wph ^ 1u, status, abort_flag) ||
+                         !mbar_wait(&sw_empty[ws_], wph ^ 1u, status, abort_flag)))
+                        break;
+                    mbar_arrive_expect_tx(&zw_full[ws_], kWinBytes);
+                    tma_load_2d(smem + kZwOff + ws_ * kWinBytes, &zmap, &zw_full[ws_], ks & ~(kWinGroups - 1), nt * kTileN);
+                    mbar_arrive_expect_tx(&sw_full[ws_], kWinBytes);
+                    tma_load_2d(smem + kSwOff + ws_ * kWinBytes, &smap, &sw_full[ws_], ks & ~(kWinGroups - 1), nt * kTileN);
+                    ++wins;
                 }
-                for (uint32_t j = issued > nst ? issued - nst : 0; j < issued; ++j) {
-                    if (weights && beg + (int64_t)j == skip_unit) continue;
-                    drain_wait(&fullb[j % nst], (j / nst) & 1u, status);
+                // skip_unit (failure-path tests only, -1 otherwise): these weights are never requested
+                if (u != skip_unit) {
+                    mbar_arrive_expect_tx(&w_full[rg.slot], kWeightStageBytes);
+                    tma_load_2d(smem + kWOff + rg.slot * kWeightStageBytes, &wmap, &w_full[rg.slot],
+                                ks * (kStageK / 2), nt * kTileN);
                 }
-                for (uint32_t j = wins > (uint32_t)kWinSlots ? wins - kWinSlots : 0; j < wins; ++j) {
-                    drain_wait(&zw_full[j % kWinSlots], (j / kWinSlots) & 1u, status);
-                    drain_wait(&sw_full[j % kWinSlots], (j / kWinSlots) & 1u, status);
-                }
+                ++issued;
+                rg.next(kWStages);
+                if (++ks == spt) { ks = 0; ++tile; }
             }
-        } else if (wid == 1) {
-            // ------------------------------ MMA issuer ------------------------------
-            constexpr uint32_t idesc = idesc_bf16_f32(128, kBN);
-            Ring xr, ar, dr;
+            for (uint32_t j = issued > (uint32_t)kWStages ? issued - kWStages : 0; j < issued; ++j) {
+                if (beg + (int64_t)j == skip_unit) continue;
+                drain_wait(&w_full[j % kWStages], (j / kWStages) & 1u, status);
+            }
+            for (uint32_t j = wins > (uint32_t)kWinSlots ? wins - kWinSlots : 0; j < wins; ++j) {
+                drain_wait(&zw_full[j % kWinSlots], (j / kWinSlots) & 1u, status);
+                drain_wait(&sw_full[j % kWinSlots], (j / kWinSlots) & 1u, status);
+            }
+        } else if (wid == 2 && lane == 0 && beg < end) {
+            // ------------------------------ activation producer ------------------------------
             uint32_t it = 0;
-            const uint32_t xbase = smem_u32(smem);
+            int64_t tile = beg / spt;
+            int ks = (int)(beg - tile * spt);
             for (int64_t u = beg; u < end; ++u, ++it) {
-                mbar_wait(&x_full[xr.slot], xr.phase, status, abort_flag);
-                mbar_wait(&a_full[ar.slot], ar.phase, status, abort_flag);
-                if (it >= 2) mbar_wait(&d_empty[dr.slot], dr.phase ^ 1u, status, abort_flag);
+                // the slot's previous stage (it - kXStages) has been multiplied
+                if (it >= (uint32_t)kXStages) {
+                    const uint32_t p = it - kXStages;
+                    if (!mbar_wait(&done[p % kRing], (p / kRing) & 1u, status, abort_flag)) break;
+                }
+                const int mt = (int)(tile / S.n_tiles);
+                uint8_t *st = smem + (it % kXStages) * kXStageBytes;
+                uint64_t *bar = &x_full[it % kXStages];
+                mbar_arrive_expect_tx(bar, kXStageBytes);
+                tma_load_2d(st, &xmap, bar, ks * kStageK, mt * kBN);
+                tma_load_2d(st + kXAtomBytes, &xmap, bar, ks * kStageK + 64, mt * kBN);
+                if (++ks == spt) { ks = 0; ++tile; }
+            }
+            for (uint32_t j = it > (uint32_t)kXStages ? it - kXStages : 0; j < it; ++j)
+                drain_wait(&x_full[j % kXStages], (j / kXStages) & 1u, status);
+        } else if (wid == 1 && lane == 0) {
+            // ------------------------------ MMA issuer (one lane) ------------------------------
+            constexpr uint32_t idesc = idesc_bf16_f32(128, kBN);
+            const uint32_t xbase = smem_u32(smem);
+            const uint32_t n_units = (uint32_t)(end - beg);
+            for (uint32_t it = 0; it < n_units; ++it) {
+                if (!mbar_wait(&x_full[it % kXStages], (it / kXStages) & 1u, status, abort_flag) ||
+                    !mbar_wait(&ready[it % kRing], (it / kRing) & 1u, status, abort_flag))
+                    break;
                 tc_fence_after();
-                const uint32_t xs = xbase + xr.slot * (uint32_t)kXStageBytes;
-                if (lane == 0) {
-                    const uint32_t a_col = tmem + ar.slot * 64u;
-                    const uint32_t d_col = d_tmem + dr.slot * (uint32_t)kBN;
+                const uint32_t xs = xbase + (it % kXStages) * (uint32_t)kXStageBytes;
+                const uint32_t a_col = tmem + (it % kABufs) * 64u;
+                const uint32_t d_col = d_tmem + (it & 1u) * (uint32_t)kBN;
 #pragma unroll
-                    for (int j = 0; j < kStageK / 16; ++j) {
-                        const uint32_t baddr = xs + (uint32_t)(j >> 2) * kXAtomBytes + (uint32_t)(j & 3) * 32u;
-                        tc_mma_ts(d_col, a_col + (uint32_t)j * 8u, smem_desc(baddr, 16, 1024, 2), idesc, j != 0 ? 1u : 0u);
-                    }
+                for (int j = 0; j < kStageK / 16; ++j) {
+                    const uint32_t baddr = xs + (uint32_t)(j >> 2) * kXAtomBytes + (uint32_t)(j & 3) * 32u;
+                    tc_mma_ts(d_col, a_col + (uint32_t)j * 8u, smem_desc(baddr, 16, 1024, 2), idesc, j != 0 ? 1u : 0u);
                 }
-                const bool wide = wide_mark[ar.slot] == (int)(it + 1);
-                if (wide) {
-                    // the stage's activation sums, rows m = lane, lane + 32, ...: two 128-byte-swizzled atoms
-                    for (int m = lane; m < kBN; m += 32) {
-                        float t = 0.0f;
-#pragma unroll
-                        for (int a = 0; a < 2; ++a)
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                uint4 v;
-                                const uint32_t addr = xs + (uint32_t)a * kXAtomBytes + (uint32_t)m * 128u +
-                                                      (((uint32_t)c ^ ((uint32_t)m & 7u)) << 4);
-                                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-                                t += sum_bf16x8(v);
-                            }
-                        xsum[dr.slot * kBN + m] = t;
-                    }
-                    for (int row = lane; row < kTileN; row += 32) zhi_d[dr.slot * kTileN + row] = zhi_a[ar.slot * kTileN + row];
-                }
-                if (lane == 0) xs_wide[dr.slot] = wide ? 1 : 0;
-                __syncwarp();
-                if (lane == 0) {
-                    tc_commit(&x_empty[xr.slot]);
-                    tc_commit(&a_empty[ar.slot]);
-                    tc_commit(&d_full[dr.slot]);
-                    mbar_arrive(&d_full[dr.slot]);
-                }
-                xr.next(kXStages);
-                ar.next(kABufs);
-                dr.next(2);
+                tc_commit(&done[it % kRing]);
             }
-            if (lane == 0) {
-                tc_commit(done);
-                drain_wait(done, 0, status);  // every MMA completes before tensor memory is released
-            }
+            tc_commit(drain);
+            drain_wait(drain, 0, status);  // every MMA completes before tensor memory is released
         }
     } else if (wid < kFirstPr) {
-        setmaxnreg_dec<96>();
+        setmaxnreg_dec<kRegDq>();
         // ------------------------------ dequantisation ------------------------------
         const int dw = wid - kFirstDq;
         const int quarter = wid & 3;  // tensor-memory lanes 32 * quarter ..
@@ -325,10 +316,10 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
         for (int i = 0; i < 2; ++i)
             w_addr[i] = smem_u32(smem + kWOff) + (uint32_t)r * 64u + 16u * ((uint32_t)(kq * 2 + i) ^ (uint32_t)((r >> 1) & 3));
         const uint32_t a_addr = tmem + lane_bits + (uint32_t)(kq * 32);
-        Ring wr, ar;
+        Ring wr;
         uint32_t it = 0;
-        int64_t tile = beg / spt;
-        int ks = (int)(beg - tile * spt);
+        bool pending = false;  // the previous stage's A is stored but not yet announced
+        int ks = (int)(beg % spt);
         int win = -1;  // s / z window in use (the producer's sequence: a new one at the start and every 8th group)
         const uint32_t zw_row = smem_u32(smem + kZwOff) + (uint32_t)r * (kWinGroups * 2);
         for (int64_t u = beg; u < end; ++u, ++it) {
@@ -345,8 +336,10 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                          : "=h"(zraw)
                          : "r"(zw_row + (uint32_t)(win % kWinSlots) * kWinBytes + (uint32_t)(ks % kWinGroups) * 2u));
             mbar_wait(&w_full[wr.slot], wr.phase, status, abort_flag);
-            if (it >= kABufs) {
-                mbar_wait(&a_empty[ar.slot], ar.phase ^ 1u, status, abort_flag);
+            if (it >= (uint32_t)kABufs) {
+                // the A buffer's previous stage (it - kABufs) has been multiplied
+                const uint32_t p = it - kABufs;
+                mbar_wait(&done[p % kRing], (p / kRing) & 1u, status, abort_flag);
                 tc_fence_after();
             }
             uint4 wv[2];
@@ -362,9 +355,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 wide = true;
             }
             const uint32_t z2 = bf16_pair_128_plus(zl);
-            int ks2 = ks + 1;
-            int64_t tile2 = tile;
-            if (ks2 == spt) { ks2 = 0; ++tile2; }
+            const uint32_t a_slot = a_addr + (it % kABufs) * 64u;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 uint32_t A[16];
@@ -378,42 +369,55 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                         A[w * 4 + j] = sub_bf16x2(lop_and_or(t, nib_mask, bf16_magic), z2);
                     }
                 }
-                tmem_st16(a_addr + ar.slot * 64u + (uint32_t)(i * 16), A);
+                tmem_st16(a_slot + (uint32_t)(i * 16), A);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            if (kq == 0) zhi_a[ar.slot * kTileN + r] = zh;  // read by the MMA warp only for a marked stage
-            if (wide) wide_mark[ar.slot] = (int)it + 1;
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&w_empty[wr.slot]);
-                mbar_arrive(&a_full[ar.slot]);
+            if (kq == 0) zhi[(it % kWideRing) * kTileN + r] = zh;  // read by the promotion of a marked stage
+            if (wide) wide_mark[it % kWideRing] = (int)it + 1;
+            if (pending || u + 1 == end) {
+                // announce this stage (and the previous one): stores complete, weights consumed
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (pending) {
+                        mbar_arrive(&ready[(it - 1) % kRing]);
+                        mbar_arrive(&w_empty[(wr.slot + kWStages - 1) % kWStages]);
+                    }
+                    mbar_arrive(&ready[it % kRing]);
+                    mbar_arrive(&w_empty[wr.slot]);
+                }
+                pending = false;
+            } else {
+                pending = true;
             }
             wr.next(kWStages);
-            ar.next(kABufs);
-            ks = ks2;
-            tile = tile2;
+            if (++ks == spt) ks = 0;
         }
+        tmem_wait_st();
     } else {
-        setmaxnreg_inc<240>();
+        setmaxnreg_inc<kRegPr>();
         // ------------------------------ promotion and output ------------------------------
+        const int pw = wid - kFirstPr;
         const int quarter = wid & 3;
+        const int ch = pw >> 2;  // columns 64 ch .. 64 ch + 63
         const int r = quarter * 32 + lane;
         const uint32_t lane_bits = (uint32_t)(quarter * 32) << 16;
-        const int ptid = tid - kFirstPr * 32;  // 0 .. 127
-        Ring dr;
+        const int ptid = tid - kFirstPr * 32;  // 0 .. 255
+        uint32_t it = 0;
         int win = -1;  // s window in use (same sequence as the producer's)
         const uint32_t sw_row = smem_u32(smem + kSwOff) + (uint32_t)r * (kWinGroups * 2);
+        // A failed wait does not end the loop: the abort flag makes every later wait return at once, and all
+        // promotion warps keep taking the same named barriers.
         for (int64_t u = beg; u < end;) {
             const int64_t tile = u / spt;
             const int ks0 = (int)(u - tile * spt);
             const int ks1 = (int)std::min<int64_t>(spt, ks0 + (end - u));
             const int64_t nt = tile % S.n_tiles, mt = tile / S.n_tiles;
             const int64_t n = nt * kTileN + r;
-            float acc[kBN];
+            float acc[64];
 #pragma unroll
-            for (int c = 0; c < kBN; ++c) acc[c] = 0.0f;
-            for (int ks = ks0; ks < ks1; ++ks) {
+            for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
+            for (int ks = ks0; ks < ks1; ++ks, ++it) {
                 if ((u == beg && ks == ks0) || (ks % kWinGroups) == 0) {
                     if (win >= 0) {
                         __syncwarp();
@@ -426,56 +430,73 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 uint16_t sraw;
                 asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sraw) : "r"(sw_row + wslot));
                 const float s = bf16_to_f32(sraw);
-                mbar_wait(&d_full[dr.slot], dr.phase, status, abort_flag);
+                mbar_wait(&done[it % kRing], (it / kRing) & 1u, status, abort_flag);
                 tc_fence_after();
-                const uint32_t dcol = d_tmem + lane_bits + dr.slot * (uint32_t)kBN;
+                const uint32_t dcol = d_tmem + lane_bits + (it & 1u) * (uint32_t)kBN + (uint32_t)(ch * 64);
                 const f32x2 s2{s, s};
 #pragma unroll
-                for (int c0 = 0; c0 < kBN; c0 += 64) {
-                    uint32_t v[64];
+                for (int c0 = 0; c0 < 64; c0 += 32) {
+                    uint32_t v[32];
                     tmem_ld32(dcol + (uint32_t)c0, v);
-                    tmem_ld32(dcol + (uint32_t)c0 + 32u, v + 32);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 64; i += 2) {
+                    for (int i = 0; i < 32; i += 2) {
                         const f32x2 r2 = fma2_pairs(s2, f32x2{__uint_as_float(v[i]), __uint_as_float(v[i + 1])},
                                                     f32x2{acc[c0 + i], acc[c0 + i + 1]});
                         acc[c0 + i] = r2.x;
                         acc[c0 + i + 1] = r2.y;
                     }
                 }
-                if (xs_wide[dr.slot]) {
-                    const float zh = zhi_d[dr.slot * kTileN + r];
-                    if (zh != 0.0f) {
-                        const float t = -s * zh;
-                        const float *xg = xsum + dr.slot * kBN;
-#pragma unroll
-                        for (int c = 0; c < kBN; ++c) acc[c] = fmaf(t, xg[c], acc[c]);
-                    }
-                }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&d_empty[dr.slot]);
-                dr.next(2);
+                // the D buffer is free for stage it + 2
+                if (lane == 0) mbar_arrive(&ready[(it + 2) % kRing]);
+                // the stage's far-zero-point record: written by the dequantisation warps before they announced
+                // the stage (its ready phase, complete since the stage was multiplied, orders those writes); one
+                // lane reads the mark, so the branch is the same for the whole warp
+                mbar_wait(&ready[it % kRing], (it / kRing) & 1u, status, abort_flag);
+                const int mark = __shfl_sync(0xffffffffu, lane == 0 ? wide_mark[it % kWideRing] : 0, 0);
+                if (mark == (int)it + 1) {
+                    // -s z_hi times the stage's activation sums: lane l sums tokens 64 ch + l and 64 ch + 32 + l
+                    // over the stage's 128 k (16-byte chunks in k order), read from global memory
+                    float tsum[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int64_t row = mt * kBN + ch * 64 + h * 32 + lane;
+                        float t = 0.0f;
+                        if (row < M) {
+                            const uint4 *p = reinterpret_cast<const uint4 *>(x + row * K + (int64_t)ks * kStageK);
+                            for (int c = 0; c < kStageK / 8; ++c) t += sum_bf16x8(__ldg(p + c));
+                        }
+                        tsum[h] = t;
+                    }
+                    const float zh = zhi[(it % kWideRing) * kTileN + r];
+                    const float t = -s * zh;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        const float xs = __shfl_sync(0xffffffffu, tsum[c >> 5], c & 31);
+                        if (zh != 0.0f) acc[c] = fmaf(t, xs, acc[c]);
+                    }
+                }
             }
 
-            // ---- segment output ----
-            const int64_t mbase = mt * kBN;
+            // ---- segment output (this warpgroup's 64 columns) ----
+            const int64_t mbase = mt * kBN + ch * 64;
             if (ks0 == 0 && ks1 == spt) {
                 if (n < N) {
                     uint16_t *yp = y + mbase * N + n;
-                    const int mlim = (int)std::min<int64_t>(kBN, M - mbase);
+                    const int mlim = (int)std::max<int64_t>(0, std::min<int64_t>(64, M - mbase));
 #pragma unroll
-                    for (int c = 0; c < kBN; ++c, yp += N)
+                    for (int c = 0; c < 64; ++c, yp += N)
                         if (c < mlim) *yp = f32_to_bf16(acc[c]);
                 }
             } else {
                 const int64_t cta_first = S.cta_of(tile * spt);
                 const int64_t my_seg = (int64_t)blockIdx.x - cta_first;
                 const int64_t cta_last = S.cta_of(tile * spt + spt - 1);
-                float *slot = ws + ((tile * max_segs + my_seg) * kBN) * kTileN + r;
+                float *slot = ws + ((tile * max_segs + my_seg) * kBN + ch * 64) * kTileN + r;
 #pragma unroll
-                for (int c = 0; c < kBN; ++c) slot[c * kTileN] = acc[c];
+                for (int c = 0; c < 64; ++c) slot[c * kTileN] = acc[c];
                 __threadfence();
                 named_bar_sync(1, kPrWarps * 32);
                 if (ptid == 0) {
@@ -488,19 +509,19 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                     // sum the segments in segment order, whichever CTA finishes last
                     __threadfence();
 #pragma unroll
-                    for (int c0 = 0; c0 < kBN; c0 += 32) {
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
                         float tot[32];
 #pragma unroll
                         for (int c = 0; c < 32; ++c) tot[c] = 0.0f;
                         for (int64_t o = 0; o <= cta_last - cta_first; ++o) {
-                            const float *other = ws + ((tile * max_segs + o) * kBN) * kTileN;
+                            const float *other = ws + ((tile * max_segs + o) * kBN + ch * 64) * kTileN;
 #pragma unroll
                             for (int c = 0; c < 32; ++c)
                                 tot[c] += (o == my_seg) ? acc[c0 + c] : __ldcg(other + (int64_t)(c0 + c) * kTileN + r);
                         }
                         if (n < N) {
                             uint16_t *yp = y + (mbase + c0) * N + n;
-                            const int mlim = (int)std::min<int64_t>(32, M - mbase - c0);
+                            const int mlim = (int)std::max<int64_t>(0, std::min<int64_t>(32, M - mbase - c0));
 #pragma unroll
                             for (int c = 0; c < 32; ++c, yp += N)
                                 if (c < mlim) *yp = f32_to_bf16(tot[c]);
@@ -569,7 +590,7 @@ int launch_gemm_w4a16_tc2(const uint16_t *x, int64_t M, int64_t N, int64_t K, co
     float *ws = reinterpret_cast<float *>(w8);
     int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, 128));
     gemm_w4a16_tc2_kernel<<<(unsigned)grid, kThreads, gemm_tc2_smem_bytes(), st>>>(
-        wmap, xmap, smap, zmap, M, N, K, y, ws, counters, max_segs, status, 0x000F000Fu, 0x43004300u, skip_unit);
+        wmap, xmap, smap, zmap, x, M, N, K, y, ws, counters, max_segs, status, 0x000F000Fu, 0x43004300u, skip_unit);
     return 0;
 }
 
