@@ -31,7 +31,7 @@
 // three waits, three commits and a warp-wide loop in the MMA warp had
 // stretched each stage to ~1,700.)
 // Register budgets follow the roles (setmaxnreg): 640 threads at launch x 96
-// registers = 61,440 = 128 x 56 + 256 x 80 + 256 x 128 + 2,048 spare.  Waits
+// registers = 61,440 = 128 x 48 + 256 x 72 + 256 x 144.  Waits
 // are inlined (no calls): ptxas allocates registers per role only for
 // straight-line code.
 // Scales and zero-points reach shared memory by TMA in windows of 8 groups x
@@ -68,7 +68,7 @@ constexpr int kRing = 4;        // stage-ready / MMA-done barriers, indexed by s
 constexpr int kWideRing = 8;    // far-zero-point records, indexed by stage % kWideRing
 constexpr int kThreads = 640;
 constexpr int kFirstDq = 4, kDqWarps = 8, kFirstPr = 12, kPrWarps = 8;
-constexpr int kRegCtl = 56, kRegDq = 80, kRegPr = 128;
+constexpr int kRegCtl = 48, kRegDq = 72, kRegPr = 144;
 constexpr int kWeightStageBytes = kTileN * (kStageK / 2);  // 8 KB
 constexpr int kXAtomBytes = kBN * 128;                     // 128 rows x 64 bf16
 constexpr int kXStageBytes = 2 * kXAtomBytes;              // 32 KB
@@ -160,7 +160,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
     uint64_t *w_full = x_full + kXStages;
     uint64_t *w_empty = w_full + kWStages;
     uint64_t *ready = w_empty + kWStages;  // stage A written (8 dequant warps) and its D buffer free (8 promotion)
-    uint64_t *done = ready + kRing;        // the stage's MMAs completed (one commit)
+    uint64_t *done = ready + kRing;        // the stage's MMAs completed (commit) and the MMA lane's release
     uint64_t *zw_full = done + kRing;
     uint64_t *zw_empty = zw_full + kWinSlots;
     uint64_t *sw_full = zw_empty + kWinSlots;
@@ -192,7 +192,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
         }
         for (int i = 0; i < kRing; ++i) {
             mbar_init(&ready[i], kDqWarps + kPrWarps);
-            mbar_init(&done[i], 1);
+            mbar_init(&done[i], 2);  // the MMAs' completion and the MMA lane's arrive
         }
         for (int i = 0; i < kWinSlots; ++i) {
             mbar_init(&zw_full[i], 1);
@@ -299,6 +299,9 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                     tc_mma_ts(d_col, a_col + (uint32_t)j * 8u, smem_desc(baddr, 16, 1024, 2), idesc, j != 0 ? 1u : 0u);
                 }
                 tc_commit(&done[it % kRing]);
+                // the second arrival on the stage's MMA-done barrier: a release by the thread that acquired
+                // the stage's ready phase, so the promotion warps also see what the dequantisation warps wrote
+                mbar_arrive(&done[it % kRing]);
             }
             tc_commit(drain);
             drain_wait(drain, 0, status);  // every MMA completes before tensor memory is released
@@ -406,6 +409,24 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
         uint32_t it = 0;
         int win = -1;  // s window in use (same sequence as the producer's)
         const uint32_t sw_row = smem_u32(smem + kSwOff) + (uint32_t)r * (kWinGroups * 2);
+        // The scale of unit (it, ks), read one stage ahead: a new window at the first unit and every 8th group,
+        // the previous one released (all of its scales have been read by then).
+        auto load_s = [&](bool first, int ks) -> float {
+            if (first || (ks % kWinGroups) == 0) {
+                if (win >= 0) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sw_empty[win % kWinSlots]);
+                }
+                ++win;
+                mbar_wait(&sw_full[win % kWinSlots], (uint32_t)(win / kWinSlots) & 1u, status, abort_flag);
+            }
+            uint16_t sraw;
+            asm volatile("ld.shared.u16 %0, [%1];"
+                         : "=h"(sraw)
+                         : "r"(sw_row + (uint32_t)(win % kWinSlots) * kWinBytes + (uint32_t)(ks % kWinGroups) * 2u));
+            return bf16_to_f32(sraw);
+        };
+        float s_next = beg < end ? load_s(true, (int)(beg % spt)) : 0.0f;
         // A failed wait does not end the loop: the abort flag makes every later wait return at once, and all
         // promotion warps keep taking the same named barriers.
         for (int64_t u = beg; u < end;) {
@@ -418,45 +439,31 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
 #pragma unroll
             for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
             for (int ks = ks0; ks < ks1; ++ks, ++it) {
-                if ((u == beg && ks == ks0) || (ks % kWinGroups) == 0) {
-                    if (win >= 0) {
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sw_empty[win % kWinSlots]);
-                    }
-                    ++win;
-                    mbar_wait(&sw_full[win % kWinSlots], (uint32_t)(win / kWinSlots) & 1u, status, abort_flag);
-                }
-                const uint32_t wslot = (uint32_t)(win % kWinSlots) * kWinBytes + (uint32_t)(ks % kWinGroups) * 2u;
-                uint16_t sraw;
-                asm volatile("ld.shared.u16 %0, [%1];" : "=h"(sraw) : "r"(sw_row + wslot));
-                const float s = bf16_to_f32(sraw);
+                const float s = s_next;
+                // the stage's MMAs are complete (and, through the MMA lane's arrive, the dequantisation warps'
+                // far-zero-point record of the stage is visible)
                 mbar_wait(&done[it % kRing], (it / kRing) & 1u, status, abort_flag);
                 tc_fence_after();
                 const uint32_t dcol = d_tmem + lane_bits + (it & 1u) * (uint32_t)kBN + (uint32_t)(ch * 64);
-                const f32x2 s2{s, s};
-#pragma unroll
-                for (int c0 = 0; c0 < 64; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(dcol + (uint32_t)c0, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const f32x2 r2 = fma2_pairs(s2, f32x2{__uint_as_float(v[i]), __uint_as_float(v[i + 1])},
-                                                    f32x2{acc[c0 + i], acc[c0 + i + 1]});
-                        acc[c0 + i] = r2.x;
-                        acc[c0 + i + 1] = r2.y;
-                    }
-                }
+                uint32_t v[64];
+                tmem_ld32(dcol, v);
+                tmem_ld32(dcol + 32u, v + 32);
+                tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                // the D buffer is free for stage it + 2
+                // the D buffer is free for stage it + 2 as soon as it is in registers
                 if (lane == 0) mbar_arrive(&ready[(it + 2) % kRing]);
-                // the stage's far-zero-point record: written by the dequantisation warps before they announced
-                // the stage (its ready phase, complete since the stage was multiplied, orders those writes); one
-                // lane reads the mark, so the branch is the same for the whole warp
-                mbar_wait(&ready[it % kRing], (it / kRing) & 1u, status, abort_flag);
-                const int mark = __shfl_sync(0xffffffffu, lane == 0 ? wide_mark[it % kWideRing] : 0, 0);
-                if (mark == (int)it + 1) {
+                const int mark = wide_mark[it % kWideRing];  // the same word for every lane
+                if ((int64_t)beg + it + 1 < end) s_next = load_s(false, ks + 1 == spt ? 0 : ks + 1);
+                const f32x2 s2{s, s};
+#pragma unroll
+                for (int i = 0; i < 64; i += 2) {
+                    const f32x2 r2 = fma2_pairs(s2, f32x2{__uint_as_float(v[i]), __uint_as_float(v[i + 1])},
+                                                f32x2{acc[i], acc[i + 1]});
+                    acc[i] = r2.x;
+                    acc[i + 1] = r2.y;
+                }
+                if (__shfl_sync(0xffffffffu, mark, 0) == (int)it + 1) {
                     // -s z_hi times the stage's activation sums: lane l sums tokens 64 ch + l and 64 ch + 32 + l
                     // over the stage's 128 k (16-byte chunks in k order), read from global memory
                     float tsum[2];
