@@ -12,8 +12,8 @@
 // is who does what:
 //  * warp 0 loads weight stages (TMA, 64-byte swizzle) and the scale and
 //    zero-point windows, warp 2 activation stages (TMA, 128-byte swizzle),
-//    warp 1 allocates tensor memory and its lane 0 alone runs the MMA loop
-//    (A from tensor memory, B from shared memory);
+//    warp 1 allocates tensor memory, and lane 0 of warps 1 and 3 issue the
+//    MMAs of alternate stages (A from tensor memory, B from shared memory);
 //  * warps 4..11 (two warpgroups) only dequantise: codes from shared memory
 //    to bf16 q - z in tensor memory, up to four stages ahead of the MMAs, and
 //    announce them two stages at a time (one tensor-memory store wait per
@@ -21,15 +21,15 @@
 //  * warps 12..19 (two warpgroups) only promote, each thread holding 64 of its
 //    row's binary32 accumulators (warpgroup c has columns 64c .. 64c + 63),
 //    and write the output.
-// Per stage the MMA lane waits twice (activations landed; the stage's A
+// Per stage an MMA lane waits twice (activations landed; the stage's A
 // written and its D buffer promoted, one barrier that the dequantisation and
 // promotion warps both arrive on) and commits once: a single "MMA done"
 // barrier tells the activation producer, the dequantisation warps and the
 // promotion warps alike that the stage's buffers may be reused or read.
-// (Measured on this kernel's previous form: a 128 x 128 x 16 MMA with A in
-// tensor memory occupies the tensor core ~94 cycles, so 8 per stage ~750, and
-// three waits, three commits and a warp-wide loop in the MMA warp had
-// stretched each stage to ~1,700.)
+// (Measured: a 128 x 128 x 16 MMA with A in tensor memory occupies the tensor
+// core ~94 cycles, so 8 per stage ~750; issuing them blocks the lane for about
+// that long, and the lane's commit, arrive and next waits then took ~400
+// cycles in which the tensor core had nothing queued -- hence two lanes.)
 // Register budgets follow the roles (setmaxnreg): 640 threads at launch x 96
 // registers = 61,440 = 128 x 48 + 256 x 72 + 256 x 144.  Waits
 // are inlined (no calls): ptxas allocates registers per role only for
@@ -200,7 +200,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
             mbar_init(&sw_full[i], 1);
             mbar_init(&sw_empty[i], kPrWarps);
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, 2);  // one commit per MMA lane
         for (int i = 0; i < kWideRing; ++i) wide_mark[i] = 0;
         *abort_flag = 0;
         *last_flag = 0;
@@ -280,12 +280,17 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
             }
             for (uint32_t j = it > (uint32_t)kXStages ? it - kXStages : 0; j < it; ++j)
                 drain_wait(&x_full[j % kXStages], (j / kXStages) & 1u, status);
-        } else if (wid == 1 && lane == 0) {
-            // ------------------------------ MMA issuer (one lane) ------------------------------
+        } else if ((wid == 1 || wid == 3) && lane == 0) {
+            // ------------------------------ MMA issuers ------------------------------
+            // Two lanes take alternate stages (warp 1 the even ones, warp 3 the odd ones): issuing a stage's
+            // MMAs blocks a lane until the tensor core has nearly run them, so a single lane left the tensor
+            // core idle while it committed and waited for the next stage.  Stages have their own A, D and
+            // activation buffers, so the order in which the two lanes' MMAs run does not matter, and each
+            // lane's commits track its own MMAs.
             constexpr uint32_t idesc = idesc_bf16_f32(128, kBN);
             const uint32_t xbase = smem_u32(smem);
             const uint32_t n_units = (uint32_t)(end - beg);
-            for (uint32_t it = 0; it < n_units; ++it) {
+            for (uint32_t it = wid == 1 ? 0u : 1u; it < n_units; it += 2) {
                 if (!mbar_wait(&x_full[it % kXStages], (it / kXStages) & 1u, status, abort_flag) ||
                     !mbar_wait(&ready[it % kRing], (it / kRing) & 1u, status, abort_flag))
                     break;
@@ -304,7 +309,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 mbar_arrive(&done[it % kRing]);
             }
             tc_commit(drain);
-            drain_wait(drain, 0, status);  // every MMA completes before tensor memory is released
+            drain_wait(drain, 0, status);  // every MMA (both lanes') completes before tensor memory is released
         }
     } else if (wid < kFirstPr) {
         setmaxnreg_dec<kRegDq>();
