@@ -39,9 +39,10 @@
 // windows' row stride; other K take wq_gemm_tc.cu).  Tensor memory: four A
 // buffers of 64 columns, two D buffers of 128.  A zero-point outside [0, 15]
 // is split as in wq_gemm_tc.cu: the dequantisation warps record z_hi per row
-// and mark the stage; each promotion warp then sums that stage's activations
-// for its 64 columns from global memory (in k order) and adds -s z_hi times
-// the sums.  The dequantisation and promotion warps do not leave their loops
+// and mark the stage; when a promotion warp finishes a window's stages it sums
+// each marked stage's activations for its 64 columns from global memory (in k
+// order) and adds -s z_hi times the sums.  A window's 8 scales reach the
+// promotion warps' registers in one load, so no stage waits on a scale.  The dequantisation and promotion warps do not leave their loops
 // when a wait fails (the abort flag makes every later wait return at once), so
 // their warp-level and named barriers stay matched.
 // Stream-K over (tile, stage) units, per-segment binary32 partials summed in
@@ -65,7 +66,7 @@ constexpr int kWStages = 6;
 constexpr int kXStages = 4;
 constexpr int kABufs = 4;
 constexpr int kRing = 4;        // stage-ready / MMA-done barriers, indexed by stage % kRing
-constexpr int kWideRing = 8;    // far-zero-point records, indexed by stage % kWideRing
+constexpr int kWideRing = 16;   // far-zero-point records, indexed by stage % kWideRing
 constexpr int kThreads = 640;
 constexpr int kFirstDq = 4, kDqWarps = 8, kFirstPr = 12, kPrWarps = 8;
 constexpr int kRegCtl = 48, kRegDq = 72, kRegPr = 144;
@@ -83,12 +84,15 @@ constexpr size_t kBarOff = kSwOff + (size_t)kWinSlots * kWinBytes;
 // x_full[XS]; w_full, w_empty [WS]; ready, done [R]; zw_full, zw_empty, sw_full, sw_empty [2]; drain
 constexpr int kBars = kXStages + 2 * kWStages + 2 * kRing + 4 * kWinSlots + 1;
 constexpr size_t kFlagOff = kBarOff + (size_t)kBars * 8;
-// flags: abort, last-arrival, tensor-memory address; far-zero-point marks [kWideRing] at +32
-constexpr size_t kZhiOff = kFlagOff + 64;  // [kWideRing][row] z_hi
+// flags: abort, last-arrival, tensor-memory address
+constexpr size_t kMarkOff = kFlagOff + 64;                    // [kWideRing] far-zero-point marks
+constexpr size_t kZhiOff = kMarkOff + kWideRing * 4;          // [kWideRing][row] z_hi
 constexpr size_t kSmemBytes = kZhiOff + kWideRing * kTileN * 4;
 
 static_assert(kRing >= kXStages && kRing >= kABufs && kRing >= 3, "stage rings must cover the buffers");
-static_assert(kWideRing >= kABufs + 2, "far-zero-point records must outlive the promotion of their stage");
+// a record is read when the promotion finishes its stage's window (at most 7 stages later); the dequantisation
+// warps reach stage j + kWideRing only after the promotion has freed the D buffer of stage j + kWideRing - 6
+static_assert(kWideRing >= kWinGroups + kABufs + 2, "far-zero-point records must outlive their window's promotion");
 static_assert(kWOff % 1024 == 0 && kZwOff % 128 == 0 && kSwOff % 128 == 0, "TMA destinations");
 static_assert(4 * kRegCtl + kDqWarps * kRegDq + kPrWarps * kRegPr <= (65536 / kThreads) / 8 * 8 * (kThreads / 32),
               "register budgets exceed the launch's registers");
@@ -169,7 +173,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kFlagOff);
     volatile int *last_flag = abort_flag + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kFlagOff + 16);
-    volatile int *wide_mark = reinterpret_cast<volatile int *>(smem + kFlagOff + 32);  // [kWideRing]
+    volatile int *wide_mark = reinterpret_cast<volatile int *>(smem + kMarkOff);       // [kWideRing]
     float *zhi = reinterpret_cast<float *>(smem + kZhiOff);                             // [kWideRing][row]
 
     const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
@@ -414,24 +418,30 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
         uint32_t it = 0;
         int win = -1;  // s window in use (same sequence as the producer's)
         const uint32_t sw_row = smem_u32(smem + kSwOff) + (uint32_t)r * (kWinGroups * 2);
-        // The scale of unit (it, ks), read one stage ahead: a new window at the first unit and every 8th group,
-        // the previous one released (all of its scales have been read by then).
-        auto load_s = [&](bool first, int ks) -> float {
-            if (first || (ks % kWinGroups) == 0) {
-                if (win >= 0) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sw_empty[win % kWinSlots]);
-                }
-                ++win;
-                mbar_wait(&sw_full[win % kWinSlots], (uint32_t)(win / kWinSlots) & 1u, status, abort_flag);
+        // This row's 8 scales of the window in use (bf16; group g of the window at bits 16 (g % 4) of
+        // sw[g / 4]), read with one 16-byte load when the window opens: a new window at the first unit and at
+        // every 8th group, the previous one released (all of its scales are in registers by then).
+        uint64_t sw[2] = {0, 0};
+        auto open_window = [&]() {
+            if (win >= 0) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sw_empty[win % kWinSlots]);
             }
-            uint16_t sraw;
-            asm volatile("ld.shared.u16 %0, [%1];"
-                         : "=h"(sraw)
-                         : "r"(sw_row + (uint32_t)(win % kWinSlots) * kWinBytes + (uint32_t)(ks % kWinGroups) * 2u));
-            return bf16_to_f32(sraw);
+            ++win;
+            mbar_wait(&sw_full[win % kWinSlots], (uint32_t)(win / kWinSlots) & 1u, status, abort_flag);
+            uint4 w4;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w4.x), "=r"(w4.y), "=r"(w4.z), "=r"(w4.w)
+                         : "r"(sw_row + (uint32_t)(win % kWinSlots) * kWinBytes));
+            sw[0] = ((uint64_t)w4.y << 32) | w4.x;
+            sw[1] = ((uint64_t)w4.w << 32) | w4.z;
         };
-        float s_next = beg < end ? load_s(true, (int)(beg % spt)) : 0.0f;
+        auto scale_of = [&](int ks) -> float {
+            const int g = ks & (kWinGroups - 1);
+            const uint64_t w = g < 4 ? sw[0] : sw[1];
+            return __uint_as_float((uint32_t)((w >> (16 * (g & 3))) & 0xFFFFu) << 16);
+        };
+        if (beg < end) open_window();
         // A failed wait does not end the loop: the abort flag makes every later wait return at once, and all
         // promotion warps keep taking the same named barriers.
         for (int64_t u = beg; u < end;) {
@@ -443,8 +453,8 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
             float acc[64];
 #pragma unroll
             for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
+            int ks_w0 = ks0;  // first group of the window's stages not yet checked for far zero-points
             for (int ks = ks0; ks < ks1; ++ks, ++it) {
-                const float s = s_next;
                 // the stage's MMAs are complete (and, through the MMA lane's arrive, the dequantisation warps'
                 // far-zero-point record of the stage is visible)
                 mbar_wait(&done[it % kRing], (it / kRing) & 1u, status, abort_flag);
@@ -458,8 +468,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 __syncwarp();
                 // the D buffer is free for stage it + 2 as soon as it is in registers
                 if (lane == 0) mbar_arrive(&ready[(it + 2) % kRing]);
-                const int mark = wide_mark[it % kWideRing];  // the same word for every lane
-                if ((int64_t)beg + it + 1 < end) s_next = load_s(false, ks + 1 == spt ? 0 : ks + 1);
+                const float s = scale_of(ks);
                 const f32x2 s2{s, s};
 #pragma unroll
                 for (int i = 0; i < 64; i += 2) {
@@ -468,27 +477,36 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                     acc[i] = r2.x;
                     acc[i + 1] = r2.y;
                 }
-                if (__shfl_sync(0xffffffffu, mark, 0) == (int)it + 1) {
-                    // -s z_hi times the stage's activation sums: lane l sums tokens 64 ch + l and 64 ch + 32 + l
-                    // over the stage's 128 k (16-byte chunks in k order), read from global memory
-                    float tsum[2];
+                if ((ks & (kWinGroups - 1)) == kWinGroups - 1 || ks + 1 == ks1) {
+                    // the window's last stage here: its marked stages get -s z_hi times their activation sums
+                    // (lane l sums tokens 64 ch + l and 64 ch + 32 + l over the stage's 128 k, 16-byte chunks in
+                    // k order, from global memory); lane 0 reads each mark, so branches are warp-uniform
+                    for (int kw = ks_w0; kw <= ks; ++kw) {
+                        const uint32_t jt = it - (uint32_t)(ks - kw);
+                        const int mark = __shfl_sync(0xffffffffu, lane == 0 ? wide_mark[jt % kWideRing] : 0, 0);
+                        if (mark != (int)jt + 1) continue;
+                        float tsum[2];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int64_t row = mt * kBN + ch * 64 + h * 32 + lane;
-                        float t = 0.0f;
-                        if (row < M) {
-                            const uint4 *p = reinterpret_cast<const uint4 *>(x + row * K + (int64_t)ks * kStageK);
-                            for (int c = 0; c < kStageK / 8; ++c) t += sum_bf16x8(__ldg(p + c));
+                        for (int h = 0; h < 2; ++h) {
+                            const int64_t row = mt * kBN + ch * 64 + h * 32 + lane;
+                            float t = 0.0f;
+                            if (row < M) {
+                                const uint4 *p = reinterpret_cast<const uint4 *>(x + row * K + (int64_t)kw * kStageK);
+                                for (int c = 0; c < kStageK / 8; ++c) t += sum_bf16x8(__ldg(p + c));
+                            }
+                            tsum[h] = t;
                         }
-                        tsum[h] = t;
-                    }
-                    const float zh = zhi[(it % kWideRing) * kTileN + r];
-                    const float t = -s * zh;
+                        const float zh = zhi[(jt % kWideRing) * kTileN + r];
+                        const float t = -scale_of(kw) * zh;
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        const float xs = __shfl_sync(0xffffffffu, tsum[c >> 5], c & 31);
-                        if (zh != 0.0f) acc[c] = fmaf(t, xs, acc[c]);
+                        for (int c = 0; c < 64; ++c) {
+                            const float xs = __shfl_sync(0xffffffffu, tsum[c >> 5], c & 31);
+                            if (zh != 0.0f) acc[c] = fmaf(t, xs, acc[c]);
+                        }
                     }
+                    ks_w0 = ks + 1;
+                    // the next unit opens a new window (a multiple of 8 groups, or a new tile at group 0)
+                    if ((int64_t)beg + it + 1 < end) open_window();
                 }
             }
 
