@@ -289,8 +289,8 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
             // Two lanes take alternate stages (warp 1 the even ones, warp 3 the odd ones): issuing a stage's
             // MMAs blocks a lane until the tensor core has nearly run them, so a single lane left the tensor
             // core idle while it committed and waited for the next stage.  Stages have their own A, D and
-            // activation buffers, so the order in which the two lanes' MMAs run does not matter, and each
-            // lane's commits track its own MMAs.
+            // activation buffers, so the order in which the two lanes' MMAs run does not matter (making the
+            // lanes take turns was measured slower), and each lane's commits track its own MMAs.
             constexpr uint32_t idesc = idesc_bf16_f32(128, kBN);
             const uint32_t xbase = smem_u32(smem);
             const uint32_t n_units = (uint32_t)(end - beg);
@@ -481,10 +481,14 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                     // the window's last stage here: its marked stages get -s z_hi times their activation sums
                     // (lane l sums tokens 64 ch + l and 64 ch + 32 + l over the stage's 128 k, 16-byte chunks in
                     // k order, from global memory); lane 0 reads each mark, so branches are warp-uniform
-                    for (int kw = ks_w0; kw <= ks; ++kw) {
+                    // lane l looks at the window's l-th checked stage; one ballot gives the marked ones
+                    const int nchk = ks - ks_w0 + 1;  // 1 .. 8
+                    const uint32_t jl = it - (uint32_t)(ks - ks_w0) + (uint32_t)lane;
+                    const uint32_t marked =
+                        __ballot_sync(0xffffffffu, lane < nchk && wide_mark[jl % kWideRing] == (int)jl + 1);
+                    for (uint32_t mbits = marked; mbits != 0u; mbits &= mbits - 1u) {
+                        const int kw = ks_w0 + __ffs((int)mbits) - 1;
                         const uint32_t jt = it - (uint32_t)(ks - kw);
-                        const int mark = __shfl_sync(0xffffffffu, lane == 0 ? wide_mark[jt % kWideRing] : 0, 0);
-                        if (mark != (int)jt + 1) continue;
                         float tsum[2];
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
@@ -521,12 +525,18 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                         if (c < mlim) *yp = f32_to_bf16(acc[c]);
                 }
             } else {
+                // Partial sums of a split tile: segment slot [column / 4][row][4] floats, so each thread writes
+                // and reads its 64 columns as 16 float4 and a warp's access is 512 contiguous bytes.
                 const int64_t cta_first = S.cta_of(tile * spt);
                 const int64_t my_seg = (int64_t)blockIdx.x - cta_first;
-                const int64_t cta_last = S.cta_of(tile * spt + spt - 1);
-                float *slot = ws + ((tile * max_segs + my_seg) * kBN + ch * 64) * kTileN + r;
+                const int64_t nseg = S.cta_of(tile * spt + spt - 1) - cta_first + 1;
+                auto seg_ptr = [&](int64_t o, int q) -> float4 * {  // this thread's float4 q (columns 4q..4q+3)
+                    return reinterpret_cast<float4 *>(ws) +
+                           ((tile * max_segs + o) * (kBN / 4) + ch * 16 + q) * kTileN + r;
+                };
 #pragma unroll
-                for (int c = 0; c < 64; ++c) slot[c * kTileN] = acc[c];
+                for (int q = 0; q < 16; ++q)
+                    *seg_ptr(my_seg, q) = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
                 __threadfence();
                 named_bar_sync(1, kPrWarps * 32);
                 if (ptid == 0) {
@@ -536,24 +546,44 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 }
                 named_bar_sync(1, kPrWarps * 32);
                 if (*last_flag) {
-                    // sum the segments in segment order, whichever CTA finishes last
+                    // sum the segments in segment order, whichever CTA finishes last; 16 columns at a time, the
+                    // next segment's values requested before the current ones are added
                     __threadfence();
 #pragma unroll
-                    for (int c0 = 0; c0 < 64; c0 += 32) {
-                        float tot[32];
+                    for (int c0 = 0; c0 < 64; c0 += 16) {
+                        float tot[16];
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) tot[c] = 0.0f;
-                        for (int64_t o = 0; o <= cta_last - cta_first; ++o) {
-                            const float *other = ws + ((tile * max_segs + o) * kBN + ch * 64) * kTileN;
+                        for (int c = 0; c < 16; ++c) tot[c] = 0.0f;
+                        float4 nxt[4];
+                        auto fetch = [&](int64_t o) {
 #pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                tot[c] += (o == my_seg) ? acc[c0 + c] : __ldcg(other + (int64_t)(c0 + c) * kTileN + r);
+                            for (int q = 0; q < 4; ++q)
+                                nxt[q] = o == my_seg ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcg(seg_ptr(o, c0 / 4 + q));
+                        };
+                        fetch(0);
+                        for (int64_t o = 0; o < nseg; ++o) {
+                            float4 cur[4];
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
+                            if (o + 1 < nseg) fetch(o + 1);
+                            if (o == my_seg) {
+#pragma unroll
+                                for (int c = 0; c < 16; ++c) tot[c] += acc[c0 + c];
+                            } else {
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    tot[4 * q] += cur[q].x;
+                                    tot[4 * q + 1] += cur[q].y;
+                                    tot[4 * q + 2] += cur[q].z;
+                                    tot[4 * q + 3] += cur[q].w;
+                                }
+                            }
                         }
                         if (n < N) {
                             uint16_t *yp = y + (mbase + c0) * N + n;
-                            const int mlim = (int)std::max<int64_t>(0, std::min<int64_t>(32, M - mbase - c0));
+                            const int mlim = (int)std::max<int64_t>(0, std::min<int64_t>(16, M - mbase - c0));
 #pragma unroll
-                            for (int c = 0; c < 32; ++c, yp += N)
+                            for (int c = 0; c < 16; ++c, yp += N)
                                 if (c < mlim) *yp = f32_to_bf16(tot[c]);
                         }
                     }
