@@ -15,9 +15,8 @@
 //    warp 1 allocates tensor memory, and lane 0 of warps 1 and 3 issue the
 //    MMAs of alternate stages (A from tensor memory, B from shared memory);
 //  * warps 4..11 (two warpgroups) only dequantise: codes from shared memory
-//    to bf16 q - z in tensor memory, up to four stages ahead of the MMAs, and
-//    announce them two stages at a time (one tensor-memory store wait per
-//    pair);
+//    to bf16 q - z in registers, stored into one of two tensor-memory A
+//    buffers as soon as the MMA two stages back has freed it;
 //  * warps 12..19 (two warpgroups) only promote, each thread holding 64 of its
 //    row's binary32 accumulators (warpgroup c has columns 64c .. 64c + 63),
 //    and write the output.
@@ -36,8 +35,11 @@
 // straight-line code.
 // Scales and zero-points reach shared memory by TMA in windows of 8 groups x
 // 128 rows, issued by the weight producer (needs K % 1024 == 0 for the
-// windows' row stride; other K take wq_gemm_tc.cu).  Tensor memory: four A
-// buffers of 64 columns, two D buffers of 128.  A zero-point outside [0, 15]
+// windows' row stride; other K take wq_gemm_tc.cu).  Tensor memory: two A
+// buffers of 64 columns and three D buffers of 128, so the MMAs of a stage
+// wait for the promotion of the stage three back (with two, the chain of MMA
+// completion, promotion and the next issue set the stage time; three were
+// measured 5.7% faster on the 8-layer step, a fourth does not fit).  A zero-point outside [0, 15]
 // is split as in wq_gemm_tc.cu: the dequantisation warps record z_hi per row
 // and mark the stage; when a promotion warp finishes a window's stages it sums
 // each marked stage's activations for its 64 columns from global memory (in k
@@ -64,7 +66,8 @@ constexpr int kBN = 128;        // activation rows per tile (MMA N)
 constexpr int kStageK = 128;    // k per stage = one group
 constexpr int kWStages = 6;
 constexpr int kXStages = 4;
-constexpr int kABufs = 4;
+constexpr int kABufs = 2;        // dequantised A stages in tensor memory (64 columns each)
+constexpr int kDBufs = 3;        // accumulator stages in tensor memory (128 columns each)
 constexpr int kRing = 4;        // stage-ready / MMA-done barriers, indexed by stage % kRing
 constexpr int kWideRing = 16;   // far-zero-point records, indexed by stage % kWideRing
 constexpr int kThreads = 640;
@@ -73,7 +76,7 @@ constexpr int kRegCtl = 48, kRegDq = 72, kRegPr = 144;
 constexpr int kWeightStageBytes = kTileN * (kStageK / 2);  // 8 KB
 constexpr int kXAtomBytes = kBN * 128;                     // 128 rows x 64 bf16
 constexpr int kXStageBytes = 2 * kXAtomBytes;              // 32 KB
-constexpr uint32_t kTmemCols = 512;                        // A 4 x 64, D 2 x 128
+constexpr uint32_t kTmemCols = 512;                        // A 2 x 64, D 3 x 128
 constexpr int kWinGroups = 8;                              // groups (stages) per s / z window
 constexpr int kWinSlots = 2;                               // windows in flight per ring
 constexpr int kWinBytes = kTileN * kWinGroups * 2;         // 128 rows x 8 bf16 = 2 KB
@@ -89,10 +92,11 @@ constexpr size_t kMarkOff = kFlagOff + 64;                    // [kWideRing] far
 constexpr size_t kZhiOff = kMarkOff + kWideRing * 4;          // [kWideRing][row] z_hi
 constexpr size_t kSmemBytes = kZhiOff + kWideRing * kTileN * 4;
 
-static_assert(kRing >= kXStages && kRing >= kABufs && kRing >= 3, "stage rings must cover the buffers");
+static_assert(kRing >= kXStages && kRing >= kABufs && kRing > kDBufs, "stage rings must cover the buffers");
+static_assert(kABufs * 64 + kDBufs * kBN <= (int)kTmemCols, "tensor memory");
 // a record is read when the promotion finishes its stage's window (at most 7 stages later); the dequantisation
 // warps reach stage j + kWideRing only after the promotion has freed the D buffer of stage j + kWideRing - 6
-static_assert(kWideRing >= kWinGroups + kABufs + 2, "far-zero-point records must outlive their window's promotion");
+static_assert(kWideRing >= kWinGroups + kABufs + kDBufs, "far-zero-point records must outlive their window's promotion");
 static_assert(kWOff % 1024 == 0 && kZwOff % 128 == 0 && kSwOff % 128 == 0, "TMA destinations");
 static_assert(4 * kRegCtl + kDqWarps * kRegDq + kPrWarps * kRegPr <= (65536 / kThreads) / 8 * 8 * (kThreads / 32),
               "register budgets exceed the launch's registers");
@@ -209,16 +213,15 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
-        // stages 0 and 1 find their D buffers free
-        mbar_arrive_n(&ready[0], kPrWarps);
-        mbar_arrive_n(&ready[1], kPrWarps);
+        // the first kDBufs stages find their D buffers free
+        for (int i = 0; i < kDBufs; ++i) mbar_arrive_n(&ready[i], kPrWarps);
     }
     if (wid == 1) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t d_tmem = tmem + kABufs * 64u;  // D buffer b at column b * 128
+    const uint32_t d_tmem = tmem + kABufs * 64u;  // D buffer b at column kABufs * 64 + b * 128
 
     if (wid < kFirstDq) {
         setmaxnreg_dec<kRegCtl>();
@@ -301,7 +304,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 tc_fence_after();
                 const uint32_t xs = xbase + (it % kXStages) * (uint32_t)kXStageBytes;
                 const uint32_t a_col = tmem + (it % kABufs) * 64u;
-                const uint32_t d_col = d_tmem + (it & 1u) * (uint32_t)kBN;
+                const uint32_t d_col = d_tmem + (it % (uint32_t)kDBufs) * (uint32_t)kBN;
 #pragma unroll
                 for (int j = 0; j < kStageK / 16; ++j) {
                     const uint32_t baddr = xs + (uint32_t)(j >> 2) * kXAtomBytes + (uint32_t)(j & 3) * 32u;
@@ -330,7 +333,6 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
         const uint32_t a_addr = tmem + lane_bits + (uint32_t)(kq * 32);
         Ring wr;
         uint32_t it = 0;
-        bool pending = false;  // the previous stage's A is stored but not yet announced
         int ks = (int)(beg % spt);
         int win = -1;  // s / z window in use (the producer's sequence: a new one at the start and every 8th group)
         const uint32_t zw_row = smem_u32(smem + kZwOff) + (uint32_t)r * (kWinGroups * 2);
@@ -348,12 +350,6 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                          : "=h"(zraw)
                          : "r"(zw_row + (uint32_t)(win % kWinSlots) * kWinBytes + (uint32_t)(ks % kWinGroups) * 2u));
             mbar_wait(&w_full[wr.slot], wr.phase, status, abort_flag);
-            if (it >= (uint32_t)kABufs) {
-                // the A buffer's previous stage (it - kABufs) has been multiplied
-                const uint32_t p = it - kABufs;
-                mbar_wait(&done[p % kRing], (p / kRing) & 1u, status, abort_flag);
-                tc_fence_after();
-            }
             uint4 wv[2];
 #pragma unroll
             for (int i = 0; i < 2; ++i)
@@ -367,10 +363,11 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 wide = true;
             }
             const uint32_t z2 = bf16_pair_128_plus(zl);
-            const uint32_t a_slot = a_addr + (it % kABufs) * 64u;
+            // the stage's q - z are formed in registers before the A buffer is waited for, so the stores
+            // follow the MMA that frees it at once
+            uint32_t A[32];
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
-                uint32_t A[16];
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
                     const uint32_t v = word_of4(wv[i], w);
@@ -378,29 +375,28 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint32_t t = __byte_perm(v, v4, (uint32_t)(j | (j << 4) | ((4 + j) << 8) | ((4 + j) << 12)));
-                        A[w * 4 + j] = sub_bf16x2(lop_and_or(t, nib_mask, bf16_magic), z2);
+                        A[i * 16 + w * 4 + j] = sub_bf16x2(lop_and_or(t, nib_mask, bf16_magic), z2);
                     }
                 }
-                tmem_st16(a_slot + (uint32_t)(i * 16), A);
             }
+            if (it >= (uint32_t)kABufs) {
+                // the A buffer's previous stage (it - kABufs) has been multiplied
+                const uint32_t p = it - kABufs;
+                mbar_wait(&done[p % kRing], (p / kRing) & 1u, status, abort_flag);
+                tc_fence_after();
+            }
+            const uint32_t a_slot = a_addr + (it % kABufs) * 64u;
+            tmem_st16(a_slot, A);
+            tmem_st16(a_slot + 16u, A + 16);
             if (kq == 0) zhi[(it % kWideRing) * kTileN + r] = zh;  // read by the promotion of a marked stage
             if (wide) wide_mark[it % kWideRing] = (int)it + 1;
-            if (pending || u + 1 == end) {
-                // announce this stage (and the previous one): stores complete, weights consumed
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    if (pending) {
-                        mbar_arrive(&ready[(it - 1) % kRing]);
-                        mbar_arrive(&w_empty[(wr.slot + kWStages - 1) % kWStages]);
-                    }
-                    mbar_arrive(&ready[it % kRing]);
-                    mbar_arrive(&w_empty[wr.slot]);
-                }
-                pending = false;
-            } else {
-                pending = true;
+            // announce the stage: stores complete, weights consumed
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&ready[it % kRing]);
+                mbar_arrive(&w_empty[wr.slot]);
             }
             wr.next(kWStages);
             if (++ks == spt) ks = 0;
@@ -459,15 +455,15 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                 // far-zero-point record of the stage is visible)
                 mbar_wait(&done[it % kRing], (it / kRing) & 1u, status, abort_flag);
                 tc_fence_after();
-                const uint32_t dcol = d_tmem + lane_bits + (it & 1u) * (uint32_t)kBN + (uint32_t)(ch * 64);
+                const uint32_t dcol = d_tmem + lane_bits + (it % (uint32_t)kDBufs) * (uint32_t)kBN + (uint32_t)(ch * 64);
                 uint32_t v[64];
                 tmem_ld32(dcol, v);
                 tmem_ld32(dcol + 32u, v + 32);
                 tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
-                // the D buffer is free for stage it + 2 as soon as it is in registers
-                if (lane == 0) mbar_arrive(&ready[(it + 2) % kRing]);
+                // the D buffer is free for stage it + kDBufs as soon as it is in registers
+                if (lane == 0) mbar_arrive(&ready[(it + kDBufs) % kRing]);
                 const float s = scale_of(ks);
                 const f32x2 s2{s, s};
 #pragma unroll
