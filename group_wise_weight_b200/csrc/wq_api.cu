@@ -155,7 +155,7 @@ int run_w4a16(const char *what, const uint16_t *x, int64_t M, int64_t N, int64_t
     if (wq::gemm_tc_eligible(M, N, K, g)) {
         int *status = status_word();
         if (!status) return fail(WQ_ERR_CUDA, "%s: no device status word", what);
-        if (wq::launch_gemm_w4a16_tc(x, M, N, K, qweight, scales, zeros, g, y, workspace, status, st) != 0)
+        if (wq::launch_gemm_w4a16_tc(x, M, N, K, qweight, scales, zeros, g, y, workspace, status, st) == -1)
             return fail(WQ_ERR_CUDA, "%s: tensor map encoding failed", what);
         return check_launch(what);
     }

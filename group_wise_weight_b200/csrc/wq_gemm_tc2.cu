@@ -148,6 +148,11 @@ __device__ __forceinline__ void mbar_arrive_n(uint64_t *bar, uint32_t count)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
 
+// Programmatic dependent launch: let the next kernel in the stream start launching, and wait until the
+// preceding one has completed and its memory is visible.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity, int *status)
 {
     const uint64_t t0 = global_ns();
@@ -192,6 +197,10 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
     const int64_t end = beg + S.per + ((int64_t)blockIdx.x < S.extra ? 1 : 0);
     const int spt = (int)S.spt;
 
+    // The next call's CTAs may start as this grid's CTAs leave their SMs: they set up, load weights, scales
+    // and zero-points and dequantise, and wait for this grid to finish before they read x or write anything
+    // to global memory (y, the workspace).
+    pdl_launch_dependents();
     if (tid == 0) {
         for (int i = 0; i < kXStages; ++i) mbar_init(&x_full[i], 1);
         for (int i = 0; i < kWStages; ++i) {
@@ -268,6 +277,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
             }
         } else if (wid == 2 && lane == 0 && beg < end) {
             // ------------------------------ activation producer ------------------------------
+            pdl_wait();  // x may be the preceding call's y
             uint32_t it = 0;
             int64_t tile = beg / spt;
             int ks = (int)(beg - tile * spt);
@@ -438,6 +448,7 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
             return __uint_as_float((uint32_t)((w >> (16 * (g & 3))) & 0xFFFFu) << 16);
         };
         if (beg < end) open_window();
+        pdl_wait();  // y and the workspace may still be in use by the preceding call until it completes
         // A failed wait does not end the loop: the abort flag makes every later wait return at once, and all
         // promotion warps keep taking the same named barriers.
         for (int64_t u = beg; u < end;) {
@@ -645,8 +656,21 @@ int launch_gemm_w4a16_tc2(const uint16_t *x, int64_t M, int64_t N, int64_t K, co
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
     float *ws = reinterpret_cast<float *>(w8);
     int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, 128));
-    gemm_w4a16_tc2_kernel<<<(unsigned)grid, kThreads, gemm_tc2_smem_bytes(), st>>>(
-        wmap, xmap, smap, zmap, x, M, N, K, y, ws, counters, max_segs, status, 0x000F000Fu, 0x43004300u, skip_unit);
+    // programmatic dependent launch: this grid may start while the previous kernel in the stream finishes;
+    // it reads nothing that kernel may write, and writes nothing, before griddepcontrol.wait
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = gemm_tc2_smem_bytes();
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_w4a16_tc2_kernel, wmap, xmap, smap, zmap, x, M, N, K, y, ws, counters,
+                           max_segs, status, 0x000F000Fu, 0x43004300u, skip_unit) != cudaSuccess)
+        return -2;
     return 0;
 }
 

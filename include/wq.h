@@ -196,11 +196,13 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * pointers 16-byte aligned; workspace of wq_gemm_workspace_bytes(M, N, K, g, 4)
  * bytes (may be NULL when that is 0).  y must not overlap x, qweight,
  * scales or zeros (WQ_ERR_ARG otherwise).
- * The M = 1 kernel is launched with programmatic dependent launch: it starts
- * while the previous M = 1 call on the stream finishes, reads x and writes
- * only after that call has completed, but requests its qweight, scales and
- * zeros at once -- so they must not be the y or the workspace of the call
- * just before it on the same stream.
+ * The M = 1 kernel and the M > 64, g = 128 tensor-core kernel are launched
+ * with programmatic dependent launch: they start while the previous kernel
+ * on the stream finishes, read x and write only after that kernel has
+ * completed, but request their qweight, scales and zeros at once -- so
+ * those must not have been written by the kernel just before on the same
+ * stream (the y or workspace of the previous call, or the quantiser that
+ * produced them: put another operation or an event between).
  */
 int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *qweight,
                   const uint16_t *scales, const uint16_t *zeros, int g, uint16_t *y,
