@@ -127,6 +127,35 @@ constexpr float kRcp127 = 0x1.020408p-7f;  // RN(1 / 127)
 __device__ __forceinline__ uint32_t rint_bits(float t) { return __float_as_uint(__fadd_rn(t, 0x1.8p23f)); }
 constexpr uint32_t kRintBase = 0x4B400000u;  // bits of 1.5 * 2^23
 
+// Packed binary32 pairs (sm_100 f32x2 arithmetic; round to nearest, no fused contraction across the pair):
+// the low 32 bits hold the first value.
+__device__ __forceinline__ uint64_t f32x2_bits(float lo, float hi)
+{
+    return ((uint64_t)__float_as_uint(hi) << 32) | (uint64_t)__float_as_uint(lo);
+}
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
 // s of one INT4 group from its min and max (the library contract): RN((max - min) / 15) rounded to bf16;
 // a zero range falls back to max(|min|, |max|), then to 1.
 __device__ __forceinline__ float int4_scale(float mn, float mx)
@@ -268,9 +297,35 @@ quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
             // q = clip(rint(RN(w / s) + z), 0, 15): clipping before the rounding gives the same integer, and
             // rint_bits leaves it in the low bits; the eight patterns shifted into place and summed, minus
             // the summed offsets, are the eight nibbles of a word
-            if (quotients_by_reciprocal(s, fmaxf(fabsf(mn), fabsf(mx)))) {
+            const float maxabs = fmaxf(fabsf(mn), fabsf(mx));
+            if (quotients_by_reciprocal(s, maxabs)) {
                 const float r = __frcp_rn(s);
                 z = round_bf16(__fadd_rn(rintf(quotient_rn(-mn, s, r)), 0.0f));
+                if (kBf16 && maxabs <= s * 8192.0f && fabsf(z) <= 8192.0f) {
+                    // two weights per instruction: the same correctly rounded quotients (packed binary32
+                    // multiply and fused multiply-adds), + z, and the rounding by 1.5 * 2^23; |t| < 2^14 here,
+                    // so each rounded t is the low half-word of its bit pattern, and the pair is clipped to
+                    // [0, 15] as two 16-bit integers
+                    const uint64_t r2 = f32x2_bits(r, r), ns2 = f32x2_bits(-s, -s), z2 = f32x2_bits(z, z);
+                    const uint64_t m2 = f32x2_bits(0x1.8p23f, 0x1.8p23f);
+#pragma unroll
+                    for (int j = 0; j < kWordsPerLane; ++j) {
+                        uint32_t b[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const uint32_t wd = word_of(raw[u][j], h);
+                            const uint64_t w2 = ((uint64_t)(wd & 0xffff0000u) << 32) | (uint64_t)(wd << 16);
+                            const uint64_t q0 = f32x2_mul(w2, r2);
+                            const uint64_t q = f32x2_fma(f32x2_fma(q0, ns2, w2), r2, q0);
+                            const uint64_t t = f32x2_add(f32x2_add(q, z2), m2);
+                            uint32_t p2 = __byte_perm((uint32_t)t, (uint32_t)(t >> 32), 0x5410);
+                            p2 = __vmins2(__vmaxs2(p2, 0u), 0x000F000Fu);
+                            b[h] = p2 | (p2 >> 12);  // byte 0: q of the pair's first weight | second << 4
+                        }
+                        packed[j] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040),
+                                                0x5410);
+                    }
+                } else {
 #pragma unroll
                 for (int j = 0; j < kWordsPerLane; ++j) {
                     uint32_t pw = 0u - kRintBase * 0x11111111u;
@@ -280,6 +335,7 @@ quant_int4_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
                                                               z), 0.0f), 15.0f))
                               << (4 * i);
                     packed[j] = pw;
+                }
                 }
             } else {
                 z = round_bf16(__fadd_rn(rintf(__fdiv_rn(-mn, s)), 0.0f));
