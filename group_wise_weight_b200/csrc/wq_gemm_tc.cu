@@ -629,7 +629,7 @@ int run(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, co
     const int max_segs = (int)gemm_tc_max_segments(total, grid, K / kStageK);
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
     float *ws = reinterpret_cast<float *>(w8);
-    int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, GROUP));
+    int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, BN));
     kern<<<(unsigned)grid, kThreads, smem, st>>>(wmap, xmap, M, N, K, s, z, y, ws, counters, max_segs, status,
                                                   0x000F000Fu, 0x43004300u, W8 ? -1 : test_take_skip_unit(),
                                                   s_per_row);
@@ -651,9 +651,16 @@ int64_t gemm_tc_max_segments(int64_t total, int64_t grid, int64_t spt)
     return (spt + per - 1) / per + 1;
 }
 
-size_t gemm_tc_partials_bytes(int64_t M, int64_t N, int64_t K, int g)
+// Tile width (activation rows) of the W4A16 tensor-core call: 128 when the split-role kernel runs it
+// (g = 128, K a multiple of 1024: for every M > 16, since a stage costs the tensor core the same for any
+// N <= 128), else gemm_tc_bn.
+int gemm_tc_w4_bn(int64_t M, int64_t K, int g)
 {
-    const int BN = gemm_tc_bn(M, g);
+    return (g == 128 && K % 1024 == 0) ? 128 : gemm_tc_bn(M, g);
+}
+
+size_t gemm_tc_partials_bytes(int64_t M, int64_t N, int64_t K, int BN)
+{
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -678,17 +685,18 @@ bool gemm_tc_eligible(int64_t M, int64_t N, int64_t K, int g)
 size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
 {
     if (!gemm_tc_eligible(M, N, K, g)) return 0;
-    const int BN = gemm_tc_bn(M, g);
+    const int BN = gemm_tc_w4_bn(M, K, g);
     const int64_t tiles = ((N + kTileN - 1) / kTileN) * ((M + BN - 1) / BN);
-    return gemm_tc_partials_bytes(M, N, K, g) + (sizeof(int) * (size_t)tiles + 255) / 256 * 256;
+    return gemm_tc_partials_bytes(M, N, K, BN) + (sizeof(int) * (size_t)tiles + 255) / 256 * 256;
 }
 
 int launch_gemm_w4a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
                          const uint16_t *z, int g, uint16_t *y, void *workspace, int *status, cudaStream_t st)
 {
     const int bn = gemm_tc_bn(M, g);
-    // the 128 x 128-tile, g = 128 case runs the form with dequantisation and promotion in separate warps
-    if (bn == 128 && g == 128 && K % 1024 == 0)
+    // g = 128 with K a multiple of 1024 runs the form with dequantisation and promotion in separate warps
+    // (128 x 128 tiles for every M here; measured faster than the narrower tiles below at M = 32 too)
+    if (gemm_tc_w4_bn(M, K, g) == 128 && g == 128 && K % 1024 == 0)
         return launch_gemm_w4a16_tc2(x, M, N, K, q, s, z, y, workspace, status, st, test_take_skip_unit());
     if (g == 32) return run<32, 32, false>(x, M, N, K, q, s, z, 0, y, workspace, status, st);
     if (g == 64) return bn == 32 ? run<32, 64, false>(x, M, N, K, q, s, z, 0, y, workspace, status, st)
@@ -713,7 +721,7 @@ size_t gemm_tc_w8_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
     const int ge = w8_group(K, g);
     const int BN = gemm_tc_bn(M, ge);
     const int64_t tiles = ((N + kTileN - 1) / kTileN) * ((M + BN - 1) / BN);
-    return gemm_tc_partials_bytes(M, N, K, ge) + (sizeof(int) * (size_t)tiles + 255) / 256 * 256;
+    return gemm_tc_partials_bytes(M, N, K, BN) + (sizeof(int) * (size_t)tiles + 255) / 256 * 256;
 }
 
 int launch_gemm_w8a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *q8, const uint16_t *s,

@@ -1,5 +1,5 @@
-// wq_gemm_tc2.cu -- W4A16 matmul at batch sizes of 65 and more with groups of
-// 128 (a 128 x 128 tile per CTA), on the 5th-generation tensor cores, with
+// wq_gemm_tc2.cu -- W4A16 matmul at batch sizes above 16 with groups of 128
+// (a 128 x 128 tile per CTA), on the 5th-generation tensor cores, with
 // dequantisation and promotion in separate warps.
 //
 // The arithmetic is that of wq_gemm_tc.cu ("Quantization for LLM inference:
@@ -655,7 +655,7 @@ int launch_gemm_w4a16_tc2(const uint16_t *x, int64_t M, int64_t N, int64_t K, co
     const int max_segs = (int)gemm_tc_max_segments(total, grid, K / kStageK);
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
     float *ws = reinterpret_cast<float *>(w8);
-    int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, 128));
+    int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, kBN));
     // programmatic dependent launch: this grid may start while the previous kernel in the stream finishes;
     // it reads nothing that kernel may write, and writes nothing, before griddepcontrol.wait
     cudaLaunchConfig_t cfg = {};

@@ -55,7 +55,8 @@ int launch_gemv_w4a16_tma(const uint16_t *x, int64_t M, int64_t N, int64_t K, co
 // counters (zero-filled before first use; the kernel leaves the counters zeroed).
 int gemm_tc_bn(int64_t M, int g);
 int64_t gemm_tc_max_segments(int64_t total, int64_t grid, int64_t spt);
-size_t gemm_tc_partials_bytes(int64_t M, int64_t N, int64_t K, int g);
+int gemm_tc_w4_bn(int64_t M, int64_t K, int g);
+size_t gemm_tc_partials_bytes(int64_t M, int64_t N, int64_t K, int BN);
 bool gemm_tc_eligible(int64_t M, int64_t N, int64_t K, int g);
 size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
 int launch_gemm_w4a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,

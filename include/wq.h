@@ -196,7 +196,8 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * pointers 16-byte aligned; workspace of wq_gemm_workspace_bytes(M, N, K, g, 4)
  * bytes (may be NULL when that is 0).  y must not overlap x, qweight,
  * scales or zeros (WQ_ERR_ARG otherwise).
- * The M = 1 kernel and the M > 64, g = 128 tensor-core kernel are launched
+ * The M = 1 kernel and the tensor-core kernel for M > 16, g = 128 and
+ * K % 1024 == 0 are launched
  * with programmatic dependent launch: they start while the previous kernel
  * on the stream finishes, read x and write only after that kernel has
  * completed, but request their qweight, scales and zeros at once -- so

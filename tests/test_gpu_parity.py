@@ -336,12 +336,14 @@ def test_gemm_w4a16_tensor_core_tiles(M, N, K, g):
     _w4_case(N, K, g, M, 17 * M + N)
 
 
-@pytest.mark.parametrize("M,N,K", [(65, 1000, 1024), (127, 300, 2048), (128, 128, 1024), (129, 640, 3072),
+@pytest.mark.parametrize("M,N,K", [(17, 384, 2048), (32, 1000, 1024), (40, 128, 3072), (64, 700, 1024),
+                                   (65, 1000, 1024), (127, 300, 2048), (128, 128, 1024), (129, 640, 3072),
                                    (200, 1000, 8192), (256, 257, 1024), (384, 384, 2048)])
 def test_gemm_w4a16_tensor_core_split_roles(M, N, K):
-    """The 128 x 128-tile form (g = 128, K a multiple of 1024) with dequantisation and promotion in separate
-    warps and the scales and zero-points in shared-memory windows: one and several M tiles, ragged N and M,
-    K ranges whose windows start mid-way through a CTA's share."""
+    """The 128 x 128-tile form (g = 128, K a multiple of 1024, every M > 16) with dequantisation and
+    promotion in separate warps and the scales and zero-points in shared-memory windows: one and several M
+    tiles, M well below the tile, ragged N and M, K ranges whose windows start mid-way through a CTA's
+    share."""
     _w4_case(N, K, 128, M, 31 * M + N + K)
 
 

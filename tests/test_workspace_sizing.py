@@ -30,7 +30,8 @@ def _m1_needed(N, K):
 
 
 def _tc_needed(M, N, K, g):
-    BN = min(32 if M <= 32 else (64 if M <= 64 else 128), g)
+    # g = 128 with K a multiple of 1024 runs the split-role kernel: 128-row activation tiles for every M
+    BN = 128 if (g == 128 and K % 1024 == 0) else min(32 if M <= 32 else (64 if M <= 64 else 128), g)
     tiles = math.ceil(N / 128) * math.ceil(M / BN)
     spt = K // 128
     total = tiles * spt
@@ -57,6 +58,8 @@ def test_m1_workspace_covers_every_segment(N, K):
 @pytest.mark.parametrize("M,N,K,g", [(17, 128, 128, 32), (32, 256, 256, 64), (40, 384, 8192, 128),
                                      (64, 384, 1024, 32), (128, 130, 384, 128), (128, 256, 16384, 128),
                                      (128, 10240, 8192, 128), (128, 57344, 8192, 128), (128, 8192, 28672, 128),
-                                     (200, 512, 640, 128), (256, 128, 128, 32), (129, 4097, 4096, 64)])
+                                     (200, 512, 640, 128), (256, 128, 128, 32), (129, 4097, 4096, 64),
+                                     (17, 8192, 8192, 128), (32, 28672, 8192, 128), (64, 57344, 8192, 128),
+                                     (24, 1000, 3072, 128)])
 def test_tc_workspace_covers_every_segment(M, N, K, g):
     assert wq.wq_gemm_workspace_bytes(M, N, K, g, 4) >= _tc_needed(M, N, K, g)
