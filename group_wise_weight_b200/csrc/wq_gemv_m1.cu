@@ -8,13 +8,33 @@
 // weight as possible on the dequantisation w_hat = s (q - z) ("Quantization
 // for LLM inference: FP8, INT4 (GPTQ, AWQ) and GGUF", "The minimum maths").
 //
-// Why mma.sync at M = 1.  On CUDA cores every code costs one mixed
-// bf16 x bf16 -> binary32 FMA, and that pipe saturates near 4.5 TB/s of
-// packed weights on B200, below the HBM roofline.  One m16n8k16 tensor
-// instruction instead takes the 256 codes of a 16-row x 16-k block (the
-// activation vector fills all 8 columns of the other operand, so every lane
-// ends up holding its rows' sums), leaving the LOP3 code extraction as the
-// only per-code work.
+// Integer products.  Per group g of 128 inputs,
+//     sum_k w_hat_k x_k = s (sum_k q_k x_k - z sum_k x_k),
+// and both sums are computed exactly in integers:
+//  * x is written, once per CTA, as D = 4 planes of signed radix-128 digits
+//    per group: x_k = 2^(E_g - 5) sum_c d_ck 128^-c, |d_ck| <= 64, where 2^E_g
+//    <= max |x| of the group < 2^(E_g + 1).  bf16 has 8 significant bits, so
+//    every x_k of magnitude at least 2^(E_g - 19) is represented exactly;
+//    smaller ones are rounded to the nearest multiple of 2^(E_g - 26), far
+//    below the binary32 rounding of the sums they enter.
+//  * The codes enter the tensor core as they are: a 32-bit word of 8 nibbles
+//    becomes two words of 4 unsigned bytes (one LOP3 for the even codes, a
+//    shift and a LOP3 for the odd ones; 3 instructions per 8 codes, against
+//    11 for an exact bf16 q - z), and mma.sync m16n8k32 u8 x s8 -> s32 takes
+//    512 codes of 16 rows per instruction against the digit planes in its B
+//    columns.  The column sums D_c = sum_k q_k d_ck are exact integers.
+//  * The accumulator starts at the bits of 1.5 * 2^23, so the result read as
+//    binary32 minus 1.5 * 2^23 is D_c itself (|D_c| < 2^17) with no
+//    conversion instruction.  The lane then forms D_c - z S_c (S_c = sum_k
+//    d_ck, exact for any zero-point up to 2^11 in magnitude, one rounding
+//    beyond) and adds s 2^(E_g - 5) (D_c - z S_c) to the binary32 sum of
+//    its column; the columns meet, weighted by 128^-c, once per segment.
+//  The legacy mma.sync integer path issues at the rate of the bf16 one on
+//  B200, so the tensor core has room to spare; the point is the ALU: the
+//  exact-bf16 form of this kernel was bound by its LOP3/shift rate near 75% of
+//  HBM bandwidth in steady state.  Rows whose weights are all zero (q = z)
+//  still give exactly zero, and zero-points far outside [0, 15] need no
+//  special path.
 //
 // Memory pipeline.  TMA throughput on B200 depends on the size of each copy:
 // copies of 2 KB stream at about 4 TB/s, copies of 8 KB and more at over
@@ -22,27 +42,22 @@
 // rows x 2 groups, fetched through a 3-D view of the packed codes (64-byte
 // group slices, rows, groups; the group stride is 64 bytes) that lands in
 // shared memory as [group][row][64 B], so the consumers' 16-byte reads are
-// free of bank conflicts.  Three stages are in flight; the scales and
-// zero-points follow in [256 rows x 8 groups] boxes, double buffered.
+// free of bank conflicts.  Three stages are in flight (two when the digit
+// planes of a long K need the room); the scales and zero-points follow in
+// [256 rows x 8 groups] boxes, double buffered.
 //
 // Work layout.
 //  * A unit is (tile of 256 rows, pair of groups).  The grid is persistent
 //    (one CTA per SM) and every CTA takes an equal contiguous range of units,
 //    tile by tile along K (stream-K), so no SM idles behind a short last wave.
+//    A CTA's range touches at most min(n, K / 256) distinct group pairs of x,
+//    and only their digit planes are made and kept.
 //  * Consumer warp w (16 of them) owns rows 16w .. 16w+15 of the tile.  Lane
 //    (g, t) (g = lane / 4, t = lane % 4) reads 16 bytes -- codes 32t .. 32t+31
-//    of the group -- of rows g and g + 8.  Each 32-bit word gives, with one
-//    shift and one LOP3 per pair, the bf16 pairs (128 + q_i, 128 + q_{i+4})
-//    of its part of the A operand of eight k16 steps; the k order inside a
-//    step is permuted accordingly and the activation pairs are staged in
-//    shared memory in the same permuted order.
-//  * Subtracting the bf16 pair (128 + z, 128 + z) from each code pair gives
-//    the exact integers q - z, so the tensor core sums x (q - z) per group and
-//    the binary32 accumulator takes s * D: no term carries an offset that has
-//    to cancel later, rows whose weights are all zero give exactly zero, and
-//    the rounding error stays proportional to sum |x w_hat|.  A zero-point
-//    outside [0, 15] is split (zp_split in wq_common.cuh): the operand is
-//    q - z_lo and the lane adds -s z_hi times the group's activation sum.
+//    of the group -- of rows g and g + 8; word w of them is the A operand of
+//    the group's w-th k32 step (even codes in the first k half, odd codes in
+//    the second), and the digit planes are laid out in the same k order, one
+//    16-byte load per lane and two steps.
 //  * A tile split between CTAs leaves one binary32 partial per segment in the
 //    workspace.  The consumers never wait on global memory for this: each
 //    warp drops its 16 row sums into a double-buffered shared-memory tile and
@@ -50,12 +65,11 @@
 //    segment's slot, bumps the tile's arrival counter and, if it is the last
 //    to arrive, sums the slots in segment order, writes y and re-zeroes the
 //    counter -- a fixed order, so results do not depend on timing.
-//  * x is copied into shared memory with one bulk asynchronous copy, then
-//    permuted in place.
 //  * Launched with programmatic dependent launch: in a stream of linears the
-//    next kernel's CTAs start as SMs free up, initialise their barriers and
-//    prefetch their first weight stages into L2 while this one finishes; they
-//    read x and write anything only after griddepcontrol.wait.
+//    next kernel's CTAs start as SMs free up, initialise their barriers, load
+//    their first weight stages into shared memory and the next ones into L2
+//    while this one finishes; they read x and write anything only after
+//    griddepcontrol.wait.
 //  * Every mbarrier wait is bounded; on a timeout the kernel records it in the
 //    status word, the producer stops issuing, and every later wait returns at
 //    once: the consumers finish their loop (on garbage) with unchanged control
@@ -79,47 +93,40 @@ constexpr int kProducer = kC;                     // warp roles: consumers 0 .. 
 constexpr int kCombiner = kC + 1;
 constexpr int kT = (kC + 2) * 32;                 // threads
 constexpr int kTile = 16 * kC;                    // rows per tile (256)
-constexpr int kStages = 3;                        // weight stages in flight
+constexpr int kMaxStages = 3;                     // weight stages in flight (2 for the longest K)
 constexpr uint32_t kStageBytes = kTile * 128;     // 256 rows x 2 groups x 64 B
 constexpr uint32_t kSzBytes = kTile * 16;         // 256 rows x 8 groups x 2 B (one of s or z)
-constexpr uint32_t kBulkPiece = 16384;            // bytes per bulk copy of x
 constexpr int kPairsPerWindow = 4;                // 8 groups of s/z = 4 units
+constexpr int kDigits = 4;                        // radix-128 digit planes of x
+constexpr uint32_t kDigitPairBytes = 2 * 2 * 4 * kDigits * 16;  // [group][half][t][digit][16 B]
+constexpr int kL2Ahead = 8;                       // units requested into L2 before the grid-dependency wait
+constexpr float kMagic = 12582912.0f;             // 1.5 * 2^23
+constexpr uint32_t kMagicBits = 0x4B400000u;
 
-// shared memory: [x pairs 2K][pad to 1024][stages][s/z windows][2 partial tiles][barriers]
-__host__ __device__ __forceinline__ size_t m1_ring_offset(int64_t K)
-{
-    return ((size_t)K * 2 + 1023) & ~(size_t)1023;
-}
-__host__ __device__ __forceinline__ size_t m1_sz_offset(int64_t K) { return m1_ring_offset(K) + kStages * kStageBytes; }
-__host__ __device__ __forceinline__ size_t m1_part_offset(int64_t K) { return m1_sz_offset(K) + 2 * 2 * kSzBytes; }
-__host__ __device__ __forceinline__ size_t m1_bar_offset(int64_t K) { return m1_part_offset(K) + 2 * kTile * 4; }
-// full/empty per stage, s/z full/empty x2, partial full/empty x2, x, flags (2 x 8 B)
-constexpr int kBars = 2 * kStages + 4 + 4 + 1 + 2;
-__host__ __device__ __forceinline__ size_t m1_smem_bytes(int64_t K) { return m1_bar_offset(K) + kBars * 8 + 1024; }
+// shared memory: [stages][s/z windows][2 partial tiles][digit planes][S sums][group factors][barriers]
+struct M1Layout {
+    size_t sz, part, dig, gsum, gfac, bar, total;
+    __host__ __device__ M1Layout(int stages, int npairs)
+    {
+        sz = (size_t)stages * kStageBytes;
+        part = sz + 2 * 2 * kSzBytes;
+        dig = part + 2 * kTile * 4;
+        gsum = dig + (size_t)npairs * kDigitPairBytes;
+        gfac = gsum + (size_t)npairs * 2 * kDigits * 4;
+        bar = (gfac + (size_t)npairs * 2 * 4 + 7) & ~(size_t)7;
+        total = bar + (2 * kMaxStages + 4 + 4 + 2) * 8 + 1024;
+    }
+};
 
-// (v >> sh) & mask | magic with both constants in registers: one LOP3.
-__device__ __forceinline__ uint32_t nib_pair(uint32_t v, int sh, uint32_t mask, uint32_t magic)
+// D += A B for one m16n8k32 step (A unsigned bytes, B signed bytes, exact 32-bit integer accumulation), with the
+// accumulator's input given separately.
+__device__ __forceinline__ void mma_u8s8(uint32_t d[4], const uint32_t c[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1)
 {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(v >> sh), "r"(mask), "r"(magic));
-    return d;
-}
-
-// D += A B for one m16n8k16 step (bf16 in, binary32 accumulate); no side effects.
-__device__ __forceinline__ void mma_bf16(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                         uint32_t b1)
-{
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(c[0]), "r"(c[1]), "r"(c[2]), "r"(c[3]));
 }
 
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y, int z)
@@ -155,11 +162,18 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
     return r;
 }
 
-__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b)
+__device__ __forceinline__ float2 lds_f2(uint32_t addr)
 {
-    uint32_t d;
-    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
+    float2 r;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(r.x), "=f"(r.y) : "r"(addr));
+    return r;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr)
+{
+    float r;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(r) : "r"(addr));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
@@ -177,9 +191,9 @@ __device__ __forceinline__ int atom_add_acq_rel(int *p, int v)
 }
 
 // The CTA whose equal share [units * b / B, units * (b + 1) / B) holds unit u.
-__host__ __device__ __forceinline__ int64_t cta_of(int64_t u, int64_t units, int64_t B)
+__host__ __device__ __forceinline__ int cta_of(int64_t u, int64_t units, int64_t B)
 {
-    return ((u + 1) * B - 1) / units;
+    return (int)(((u + 1) * B - 1) / units);
 }
 
 // Eight activations divided by their input channels' scales: bf16(x / s) with an IEEE binary32 quotient
@@ -204,34 +218,91 @@ __device__ __forceinline__ void wait_drain(uint64_t *bar, uint32_t parity, int *
         if (global_ns() - t0 > kWaitLimitNs) { record_timeout(status); return; }
 }
 
+// 2^e as binary32 for e in [-126, 127].
+__device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// The digit planes, column sums and scale factor of one group of x (one warp).  Lane L takes word L / 2 of
+// the group (inputs 8 (L / 2) .. + 7) and of it the inputs of parity L % 2: 2 i + L % 2, i = 0 .. 3, the byte
+// order of the A operand's even (L % 2 = 0) and odd code words.
+__device__ __forceinline__ void make_digits(const uint16_t *__restrict__ xg, const float *__restrict__ csg,
+                                            uint32_t dig_pair, uint32_t gsum_g, uint32_t gfac_g, int h, int lane)
+{
+    const int wq_ = lane >> 1, par = lane & 1;
+    uint4 v = *reinterpret_cast<const uint4 *>(xg + 8 * wq_);
+    if (csg) v = colscale8(v, csg + 8 * wq_);
+    float e[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t wd = word_of(v, i);
+        e[i] = __uint_as_float(par ? (wd & 0xffff0000u) : (wd << 16));
+    }
+    float m = fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    // 2^E <= m < 2^(E + 1); a group of zeros gets E = 0 (all digits 0)
+    int E = m > 0.0f ? (int)((__float_as_uint(m) >> 23) & 0xff) - 127 : 0;
+    if (m > 0.0f && E == -127) E = -127 + (31 - __clz((int)(__float_as_uint(m) & 0x7fffff))) - 22;  // subnormal
+    // X = x 2^(5 - E) in (-64, 64), applied in two exact power-of-two steps
+    const int a1 = (5 - E) / 2, a2 = (5 - E) - a1;
+    const float sc1 = exp2i(a1), sc2 = exp2i(a2);
+    uint32_t t[4][kDigits];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float X = (e[i] * sc1) * sc2;
+#pragma unroll
+        for (int c = 0; c < kDigits; ++c) {
+            const float tt = X + kMagic;            // the nearest integer sits in the low bits
+            t[i][c] = __float_as_uint(tt);
+            X = (X - (tt - kMagic)) * 128.0f;      // exact
+        }
+    }
+    const int t_ = wq_ >> 2, w = wq_ & 3, half = w >> 1;
+    const uint32_t dst = dig_pair + (uint32_t)(((h * 2 + half) * 4 + t_) * (kDigits * 16) + (w & 1) * 8 + par * 4);
+#pragma unroll
+    for (int c = 0; c < kDigits; ++c) {
+        const uint32_t lo = __byte_perm(t[0][c], t[1][c], 0x0040), hi = __byte_perm(t[2][c], t[3][c], 0x0040);
+        const uint32_t packed = __byte_perm(lo, hi, 0x5410);
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst + (uint32_t)c * 16u), "r"(packed) : "memory");
+        // the digit values (wrapping 32-bit arithmetic: the four magic offsets cancel)
+        const int sum = (int)(t[0][c] + t[1][c] + t[2][c] + t[3][c] - 4u * kMagicBits);
+        const int tot = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(gsum_g + (uint32_t)c * 4u), "f"((float)tot) : "memory");
+    }
+    // weight of digit 0: 2^(E - 5) (binary32 loses precision only below 2^-126)
+    if (lane == 0) {
+        const int ef = E - 5;
+        const float f = ef >= -126 ? exp2i(ef) : exp2i(ef + 64) * 5.421010862427522e-20f;  // 2^-64
+        asm volatile("st.shared.f32 [%0], %1;" ::"r"(gfac_g), "f"(f) : "memory");
+    }
+}
+
 // 18 warps put five on one SM sub-partition, whose register file holds 16K registers: at most 96 each.
+template <int STAGES>
 __global__ void __maxnreg__(96)
 gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                      const __grid_constant__ CUtensorMap zmap, const uint16_t *__restrict__ x, int N, int K,
                      uint16_t *__restrict__ y, float *__restrict__ ws, int *__restrict__ cnt, int max_segs,
-                     int *__restrict__ status, uint32_t nib_mask, uint32_t bf16_magic,
-                     const float *__restrict__ col_scale)
+                     int *__restrict__ status, int npairs, const float *__restrict__ col_scale)
 {
     extern __shared__ __align__(1024) uint8_t m1_raw[];
     // TMA destinations want 128-byte (we keep 1024-byte) alignment: align the base explicitly
     uint8_t *sm = m1_raw + ((1024u - (smem_u32(m1_raw) & 1023u)) & 1023u);
-    uint4 *xp = reinterpret_cast<uint4 *>(sm);                    // K / 8 chunks of 8 activations
-    uint8_t *ring = sm + m1_ring_offset(K);
-    uint8_t *szr = sm + m1_sz_offset(K);                          // [2 windows][s, z][256 rows][8 groups]
-    float *part = reinterpret_cast<float *>(sm + m1_part_offset(K));  // [2][256 rows] partial sums
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + m1_bar_offset(K));
-    uint64_t *full = bars, *empty = bars + kStages;
-    uint64_t *szfull = bars + 2 * kStages, *szempty = szfull + 2;
+    const M1Layout L(STAGES, npairs);
+    uint8_t *ring = sm;
+    uint8_t *szr = sm + L.sz;                                     // [2 windows][s, z][256 rows][8 groups]
+    float *part = reinterpret_cast<float *>(sm + L.part);         // [2][256 rows] partial sums
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L.bar);
+    uint64_t *full = bars, *empty = bars + kMaxStages;
+    uint64_t *szfull = bars + 2 * kMaxStages, *szempty = szfull + 2;
     uint64_t *pfull = szempty + 2, *pempty = pfull + 2;
-    uint64_t *xbar = pempty + 2;
-    volatile int *flags = reinterpret_cast<volatile int *>(xbar + 1);  // [0] abort, [1] last-arrival broadcast
+    volatile int *flags = reinterpret_cast<volatile int *>(pempty + 2);  // [0] abort, [1] unused
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int G = K >> 7;
     const int P = G >> 1;  // group pairs (units) per tile
 
     pdl_launch_dependents();
     if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) {
+        for (int i = 0; i < STAGES; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], kC);
         }
@@ -241,7 +312,6 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             mbar_init(&pfull[i], kC);
             mbar_init(&pempty[i], 1);
         }
-        mbar_init(xbar, 1);
         flags[0] = 0;
         flags[1] = 0;
         fence_mbar_init();
@@ -261,7 +331,7 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     // be read before pdl_wait().  The packed weights, scales and zero-points are inputs that the preceding
     // call does not write (a call of this kernel writes only y and its workspace; the library's other
     // kernels do not launch dependents early), so the producer issues the first stages and the first s/z
-    // window into shared memory now, and only the activations wait.
+    // window into shared memory, and the next units into L2, now; only the activations wait.
     int pt = tile0, pp = pair0;  // producer position: tile, group pair
     int wins = 0;                // s/z windows issued
     int pi = 0;                  // stages issued
@@ -274,12 +344,17 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         ++wins;
     };
     if (wid == kProducer && lane == 0) {
-        // at most two windows start within the first kStages pairs, so no window slot needs a wait here
-        for (; pi < kStages && pi < n; ++pi) {
+        // at most two windows start within the first STAGES pairs, so no window slot needs a wait here
+        for (; pi < STAGES && pi < n; ++pi) {
             if (pi == 0 || (pp & (kPairsPerWindow - 1)) == 0) issue_window(wins & 1);
             mbar_arrive_expect_tx(&full[pi], kStageBytes);
             tma_load_3d(ring + (uint32_t)pi * kStageBytes, &wmap, &full[pi], 0, pt * kTile, 2 * pp);
             if (++pp == P) { pp = 0; ++pt; }
+        }
+        int qt = pt, qp = pp;
+        for (int j = pi; j < n && j < pi + kL2Ahead; ++j) {
+            tma_prefetch_l2_3d(&wmap, 0, qt * kTile, 2 * qp);
+            if (++qp == P) { qp = 0; ++qt; }
         }
     }
     pdl_wait();
@@ -287,24 +362,6 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     if (wid == kProducer) {
         // ================================ producer ================================
         if (lane == 0 && n > 0) {
-            // the part of x this CTA's units read (512 bytes per group pair): its pairs of the first tile,
-            // and those of the next tile if the range wraps; all of x once the range spans a whole tile
-            const uint32_t xbytes = (uint32_t)K * 2u;
-            uint32_t r0 = 0, r1 = xbytes, w1 = 0;  // [r0, r1) and, when wrapping, [0, w1)
-            if (n < P) {
-                r0 = (uint32_t)pair0 * 512u;
-                if (pair0 + n <= P) {
-                    r1 = (uint32_t)(pair0 + n) * 512u;
-                } else {
-                    w1 = (uint32_t)(pair0 + n - P) * 512u;
-                    if (w1 >= r0) { r0 = 0; w1 = 0; }  // the two pieces meet: all of x
-                }
-            }
-            mbar_arrive_expect_tx(xbar, (r1 - r0) + w1);
-            for (uint32_t o = r0; o < r1; o += kBulkPiece)
-                bulk_g2s(sm + o, reinterpret_cast<const uint8_t *>(x) + o, min(kBulkPiece, r1 - o), xbar);
-            for (uint32_t o = 0; o < w1; o += kBulkPiece)
-                bulk_g2s(sm + o, reinterpret_cast<const uint8_t *>(x) + o, min(kBulkPiece, w1 - o), xbar);
             int i = pi;
             for (; i < n; ++i) {
                 // s/z window: at every 4th pair of a tile
@@ -313,16 +370,15 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     if (wins >= 2 && !mbar_wait(&szempty[slot], (uint32_t)((wins >> 1) - 1) & 1u, status, flags)) break;
                     issue_window(slot);
                 }
-                const int s = i % kStages;
-                if (!mbar_wait(&empty[s], (uint32_t)(i / kStages - 1) & 1u, status, flags)) break;
+                const int s = i % STAGES;
+                if (!mbar_wait(&empty[s], (uint32_t)(i / STAGES - 1) & 1u, status, flags)) break;
                 mbar_arrive_expect_tx(&full[s], kStageBytes);
                 tma_load_3d(ring + (uint32_t)s * kStageBytes, &wmap, &full[s], 0, pt * kTile, 2 * pp);
                 if (++pp == P) { pp = 0; ++pt; }
             }
             // drain: the copies issued last must land before the CTA can end (bounded, ignores abort)
-            for (int j = max(0, i - kStages); j < i; ++j) wait_drain(&full[j % kStages], (uint32_t)(j / kStages) & 1u, status);
+            for (int j = max(0, i - STAGES); j < i; ++j) wait_drain(&full[j % STAGES], (uint32_t)(j / STAGES) & 1u, status);
             for (int j = max(0, wins - 2); j < wins; ++j) wait_drain(&szfull[j & 1], (uint32_t)(j >> 1) & 1u, status);
-            wait_drain(xbar, 0, status);
         }
         __syncthreads();
         return;
@@ -343,8 +399,8 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             __syncwarp();
             if (lane == 0) mbar_arrive(&pempty[b]);  // the shared tile is in registers: free it
             ++pseg;
-            const int64_t c_first = cta_of(tt * P, units, B);
-            const int nseg = (int)(cta_of(tt * P + P - 1, units, B) - c_first) + 1;
+            const int c_first = cta_of(tt * P, units, B);
+            const int nseg = cta_of(tt * P + P - 1, units, B) - c_first + 1;
             float *slots = ws + (size_t)tt * max_segs * kTile;
             float4 *mine = reinterpret_cast<float4 *>(slots + (bid - c_first) * kTile + 8 * lane);
             mine[0] = v0;
@@ -400,35 +456,38 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 
     // ================================ consumers ================================
     if (n > 0) {
-        // ---- x: wait for the bulk copy, permute each chunk in place (chunks that were not copied hold
-        // stale bytes and are never read) ----
-        mbar_wait(xbar, 0, status, flags);
-        for (int c = tid; c < K / 8; c += kC * 32) {
-            {
-                uint4 v = xp[c];
-                if (col_scale) v = colscale8(v, col_scale + 8 * c);
-                uint4 pr;
-                pr.x = __byte_perm(v.x, v.z, 0x5410);  // (x0, x4)
-                pr.y = __byte_perm(v.x, v.z, 0x7632);  // (x1, x5)
-                pr.z = __byte_perm(v.y, v.w, 0x5410);  // (x2, x6)
-                pr.w = __byte_perm(v.y, v.w, 0x7632);  // (x3, x7)
-                xp[c] = pr;
-            }
+        const uint32_t dig_u32 = smem_u32(sm + L.dig), gsum_u32 = smem_u32(sm + L.gsum), gfac_u32 = smem_u32(sm + L.gfac);
+        // ---- digit planes of the group pairs this CTA touches: pair (pair0 + j) mod P in slot j ----
+        const int nslots = min(n, P);
+        for (int j = wid; j < 2 * nslots; j += kC) {
+            const int js = j >> 1, h = j & 1;
+            int pj = pair0 + js;
+            if (pj >= P) pj -= P;
+            const int kg = 2 * pj + h;
+            make_digits(x + (size_t)kg * 128, col_scale ? col_scale + (size_t)kg * 128 : nullptr,
+                        dig_u32 + (uint32_t)js * kDigitPairBytes, gsum_u32 + (uint32_t)(js * 2 + h) * (kDigits * 4),
+                        gfac_u32 + (uint32_t)(js * 2 + h) * 4u, h, lane);
         }
         named_bar_sync(1, kC * 32);
 
         const int gq = lane >> 2, tq = lane & 3;
-        const uint32_t ring_u32 = smem_u32(ring), szr_u32 = smem_u32(szr), xp_u32 = smem_u32(xp);
+        const uint32_t ring_u32 = smem_u32(ring), szr_u32 = smem_u32(szr);
         const int r0 = 16 * wid + gq;  // this lane's rows in the tile: r0 and r0 + 8
-        float acc[2] = {0.0f, 0.0f};
+        // this lane's B columns are digits gq (all k) and its accumulator columns 2 tq, 2 tq + 1
+        const bool bcol = gq < kDigits, ccol = 2 * tq < kDigits;
+        const float cw0 = ccol ? exp2i(-14 * tq) : 0.0f, cw1 = ccol ? exp2i(-14 * tq - 7) : 0.0f;  // 128^-c
+        float acc[2][2] = {{0.0f, 0.0f}, {0.0f, 0.0f}};  // [row r0, r0 + 8][column 2 tq, 2 tq + 1]
+        const uint32_t cmag[4] = {kMagicBits, kMagicBits, kMagicBits, kMagicBits};
         int t = tile0, p = pair0, seg_first = pair0;
         int win = -1;
         int pseg = 0;  // partial segments handed to the combiner
         int s = 0;     // stage slot of unit i, and the parity of its fill
+        int di = 0;    // digit slot of pair p
         uint32_t ph = 0, w_off = 0;
         const uint32_t w_lane = ring_u32 + (uint32_t)r0 * 64u + (uint32_t)tq * 16u;
         const uint32_t sz_lane = szr_u32 + (uint32_t)r0 * 16u;
-        const uint32_t x_lane = xp_u32 + (uint32_t)tq * 64u;
+        const uint32_t b_lane = dig_u32 + (uint32_t)(tq * (kDigits * 16) + gq * 16);
+        const uint32_t s_lane = gsum_u32 + (uint32_t)(2 * tq) * 4u;
         // A wait that runs out sets the abort flag and every later wait returns at once: the loop then runs
         // to its end on garbage, with the same control flow in every warp, so the barriers below still meet.
         for (int i = 0; i < n; ++i) {
@@ -451,74 +510,69 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 for (int a = 0; a < 2; ++a) wv[h][a] = lds128(wsrc + (uint32_t)h * (kTile * 64u) + (uint32_t)a * 8u * 64u);
             const int kg = 2 * p;
             const uint32_t szsrc = sz_lane + (uint32_t)(win & 1) * 2u * kSzBytes + (uint32_t)(kg & 7) * 2u;
-            // s and z of groups kg, kg + 1 are adjacent in the window box (kg is even): one 32-bit load per
-            // row and array; (128 + z) is formed by one bf16 addition, exact when z is in [0, 15]
-            float sv[2][2];
-            uint32_t zz[2][2];  // bf16 pairs (128 + z, 128 + z)
-            uint32_t zraw[2], zin = 0u;  // zin & 0xFFF0FFF0: some z of this lane outside [0, 15]
+            // s and z of groups kg, kg + 1 are adjacent in the window box (kg is even): one 32-bit load per row
+            // and array
+            float sv[2][2], zv[2][2];
 #pragma unroll
             for (int a = 0; a < 2; ++a) {
                 const uint32_t o = szsrc + (uint32_t)a * 8u * 16u;
-                zraw[a] = lds_u32(o + kSzBytes);
-                const uint32_t s2 = lds_u32(o), z2 = add_bf16x2(zraw[a], 0x43004300u);
+                const uint32_t s2 = lds_u32(o), z2 = lds_u32(o + kSzBytes);
                 sv[0][a] = __uint_as_float(s2 << 16);
                 sv[1][a] = __uint_as_float(s2 & 0xffff0000u);
-                zz[0][a] = __byte_perm(z2, 0u, 0x1010);
-                zz[1][a] = __byte_perm(z2, 0u, 0x3232);
-                zin |= z2 ^ 0x43004300u;
-            }
-            // a zero-point of this lane outside [0, 15] (rare): split it (zp_split) and add -s z_hi times the
-            // group's activation sum (all 128 values, in a fixed order) to the row sums right away
-            if ((zin & 0xFFF0FFF0u) != 0u) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    float xs = 0.0f;
-                    for (int j = 0; j < 16; ++j) xs += sum_bf16x8(lds128(xp_u32 + (uint32_t)(kg + h) * 256u + (uint32_t)j * 16u));
-#pragma unroll
-                    for (int a = 0; a < 2; ++a) {
-                        const float zf = __uint_as_float(h ? (zraw[a] & 0xffff0000u) : (zraw[a] << 16));
-                        float zh;
-                        zz[h][a] = bf16_pair_128_plus(zp_split(zf, zh));
-                        acc[a] = fmaf(-sv[h][a] * zh, xs, acc[a]);
-                    }
-                }
+                zv[0][a] = __uint_as_float(z2 << 16);
+                zv[1][a] = __uint_as_float(z2 & 0xffff0000u);
             }
             // the stage's weight bytes are in registers: hand the slot back to the producer
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
-            if (++s == kStages) { s = 0; ph ^= 1u; w_off = 0; } else { w_off += kStageBytes; }
+            if (++s == STAGES) { s = 0; ph ^= 1u; w_off = 0; } else { w_off += kStageBytes; }
+            const uint32_t bsrc = b_lane + (uint32_t)di * kDigitPairBytes;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                uint4 Pw[4];
+                // digit column gq of this lane's 8 inputs of each k32 step: steps 0, 1 then 2, 3
+                uint4 Bv[2];
 #pragma unroll
-                for (int w = 0; w < 4; ++w) Pw[w] = lds128(x_lane + (uint32_t)(kg + h) * 256u + (uint32_t)w * 16u);
-                float C0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, C1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                for (int hf = 0; hf < 2; ++hf)
+                    Bv[hf] = bcol ? lds128(bsrc + (uint32_t)((h * 2 + hf) * 4) * (kDigits * 16)) : make_uint4(0u, 0u, 0u, 0u);
+                uint32_t C[4];
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
                     const uint32_t va = word_of(wv[h][0], w), vb = word_of(wv[h][1], w);
-                    float *C = (w & 1) ? C1 : C0;
-                    const uint32_t za = zz[h][0], zb = zz[h][1];
-                    mma_bf16(C, sub_bf16x2(nib_pair(va, 0, nib_mask, bf16_magic), za),
-                             sub_bf16x2(nib_pair(vb, 0, nib_mask, bf16_magic), zb),
-                             sub_bf16x2(nib_pair(va, 4, nib_mask, bf16_magic), za),
-                             sub_bf16x2(nib_pair(vb, 4, nib_mask, bf16_magic), zb), Pw[w].x, Pw[w].y);
-                    mma_bf16(C, sub_bf16x2(nib_pair(va, 8, nib_mask, bf16_magic), za),
-                             sub_bf16x2(nib_pair(vb, 8, nib_mask, bf16_magic), zb),
-                             sub_bf16x2(nib_pair(va, 12, nib_mask, bf16_magic), za),
-                             sub_bf16x2(nib_pair(vb, 12, nib_mask, bf16_magic), zb), Pw[w].z, Pw[w].w);
+                    const uint32_t b0 = word_of(Bv[w >> 1], (w & 1) * 2), b1 = word_of(Bv[w >> 1], (w & 1) * 2 + 1);
+                    mma_u8s8(C, w == 0 ? cmag : C, va & 0x0F0F0F0Fu, vb & 0x0F0F0F0Fu, (va >> 4) & 0x0F0F0F0Fu,
+                             (vb >> 4) & 0x0F0F0F0Fu, b0, b1);
                 }
-                // every column of D carries the same x: C[0] is row r0, C[2] row r0 + 8
-                acc[0] = fmaf(sv[h][0], C0[0] + C1[0], acc[0]);
-                acc[1] = fmaf(sv[h][1], C0[2] + C1[2], acc[1]);
+                // C: (row r0, column 2 tq), (r0, 2 tq + 1), (r0 + 8, 2 tq), (r0 + 8, 2 tq + 1), each 1.5 2^23 + D_c
+                const float2 S = ccol ? lds_f2(s_lane + (uint32_t)(di * 2 + h) * (kDigits * 4)) : make_float2(0.0f, 0.0f);
+                const float F = lds_f32(gfac_u32 + (uint32_t)(di * 2 + h) * 4u);
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    const float sF = sv[h][a] * F;
+                    const float d0 = fmaf(-zv[h][a], S.x, __uint_as_float(C[2 * a]) - kMagic);
+                    const float d1 = fmaf(-zv[h][a], S.y, __uint_as_float(C[2 * a + 1]) - kMagic);
+                    acc[a][0] = fmaf(sF, d0, acc[a][0]);
+                    acc[a][1] = fmaf(sF, d1, acc[a][1]);
+                }
             }
+            if (++di == P) di = 0;
             // ---- end of a segment: the tile's last pair, or the end of this CTA's range ----
             const bool tile_done = (p + 1 == P);
             if (tile_done || i + 1 == n) {
+                // the row sums: columns weighted by 128^-c, then summed over the four tq lanes
+                float rs[2];
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    float v = fmaf(acc[a][1], cw1, acc[a][0] * cw0);
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    rs[a] = v;
+                    acc[a][0] = acc[a][1] = 0.0f;
+                }
                 const int row0 = t * kTile + r0;
                 if (seg_first == 0 && tile_done) {
                     if (tq == 0) {
-                        if (row0 < N) y[row0] = f32_to_bf16(acc[0]);
-                        if (row0 + 8 < N) y[row0 + 8] = f32_to_bf16(acc[1]);
+                        if (row0 < N) y[row0] = f32_to_bf16(rs[0]);
+                        if (row0 + 8 < N) y[row0 + 8] = f32_to_bf16(rs[1]);
                     }
                 } else {
                     // partial: this warp's 16 row sums go to the shared tile of this segment; the combiner
@@ -526,14 +580,13 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     const int b = pseg & 1;
                     if (pseg >= 2) mbar_wait(&pempty[b], (uint32_t)((pseg >> 1) - 1) & 1u, status, flags);
                     if (tq == 0) {
-                        part[b * kTile + r0] = acc[0];
-                        part[b * kTile + r0 + 8] = acc[1];
+                        part[b * kTile + r0] = rs[0];
+                        part[b * kTile + r0 + 8] = rs[1];
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pfull[b]);
                     ++pseg;
                 }
-                acc[0] = acc[1] = 0.0f;
             }
             if (++p == P) { p = 0; ++t; seg_first = 0; }
         }
@@ -541,29 +594,43 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     __syncthreads();
 }
 
-// Grid of the persistent kernel for this shape on the current device: one CTA per SM, fewer when there
-// is less work.  Cached per device.
-int m1_grid(int64_t N, int64_t K)
+// Shape-dependent launch parameters, cached per (device, N, K): grid (one CTA per SM, fewer when there is
+// less work), the digit slots a CTA needs, and the stage count that fits shared memory.
+struct M1Config {
+    int grid, npairs, stages;
+    size_t smem;
+};
+
+M1Config m1_config(int64_t N, int64_t K)
 {
     static std::mutex mu;
-    static std::map<int, int> sms_of;
+    static std::map<int, std::pair<int, int>> dev_of;  // SMs, opt-in shared memory per block
     int dev = 0;
     cudaGetDevice(&dev);
-    int sms;
+    int sms, optin;
     {
         std::lock_guard<std::mutex> lock(mu);
-        auto it = sms_of.find(dev);
-        if (it == sms_of.end()) {
-            int v = 148, optin = 0;
+        auto it = dev_of.find(dev);
+        if (it == dev_of.end()) {
+            int v = 148, o = 0;
             cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-            cudaFuncSetAttribute(gemv_w4a16_m1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-            it = sms_of.emplace(dev, v).first;
+            cudaDeviceGetAttribute(&o, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+            cudaFuncSetAttribute(gemv_w4a16_m1_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, o);
+            cudaFuncSetAttribute(gemv_w4a16_m1_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, o);
+            it = dev_of.emplace(dev, std::make_pair(v, o)).first;
         }
-        sms = it->second;
+        sms = it->second.first;
+        optin = it->second.second;
     }
-    const int64_t units = ((N + kTile - 1) / kTile) * (K / 256);
-    return (int)std::max<int64_t>(1, std::min<int64_t>(units, sms));
+    const int64_t P = K / 256;
+    const int64_t units = ((N + kTile - 1) / kTile) * P;
+    M1Config c;
+    c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(units, sms));
+    const int64_t per = (units + c.grid - 1) / c.grid;  // most units any CTA takes
+    c.npairs = (int)std::min<int64_t>(per, P);
+    c.stages = M1Layout(3, c.npairs).total <= (size_t)optin ? 3 : 2;
+    c.smem = M1Layout(c.stages, c.npairs).total;
+    return c;
 }
 
 // Most segments (CTAs) any tile is split into, for this grid.
@@ -586,7 +653,7 @@ size_t m1_slots_bytes(int64_t N, int64_t K, int grid)
 bool gemv_m1_eligible(int64_t M, int64_t N, int64_t K, int g)
 {
     // K % 1024: the s/z row stride (K / 128 bf16) must be a multiple of 16 bytes for their tensor maps;
-    // K <= 32768: x and the stages fit in shared memory
+    // K <= 32768: the digit planes of a CTA's group pairs and two stages fit in shared memory
     return M == 1 && g == 128 && K >= 1024 && K % 1024 == 0 && K <= 32768 && N >= 1 && N <= 0x7fffffffLL;
 }
 
@@ -594,7 +661,7 @@ size_t gemv_m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
 {
     if (!gemv_m1_eligible(M, N, K, g)) return 0;
     const int64_t ntiles = (N + kTile - 1) / kTile;
-    return m1_slots_bytes(N, K, m1_grid(N, K)) + ((size_t)ntiles * 4 + 255) / 256 * 256;
+    return m1_slots_bytes(N, K, m1_config(N, K).grid) + ((size_t)ntiles * 4 + 255) / 256 * 256;
 }
 
 int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
@@ -626,7 +693,8 @@ int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t 
         !encode_tmap_2d(&zmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, z, G, (uint64_t)N, G * 2, 8, kTile,
                         CU_TENSOR_MAP_SWIZZLE_NONE))
         return -1;
-    const int grid = m1_grid(N, K);
+    const M1Config c = m1_config(N, K);
+    const int grid = c.grid;
     const int max_segs = m1_max_segments(N, K, grid);
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
     float *ws = reinterpret_cast<float *>(w8);
@@ -636,16 +704,19 @@ int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kT);
-    cfg.dynamicSmemBytes = m1_smem_bytes(K);
+    cfg.dynamicSmemBytes = c.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gemv_w4a16_m1_kernel, wmap, smap, zmap, x, (int)N, (int)K, y, ws, cnt, max_segs,
-                           status, 0x000F000Fu, 0x43004300u, col_scale) != cudaSuccess)
-        return -2;
+    const cudaError_t e =
+        c.stages == 3 ? cudaLaunchKernelEx(&cfg, gemv_w4a16_m1_kernel<3>, wmap, smap, zmap, x, (int)N, (int)K, y, ws, cnt,
+                                           max_segs, status, c.npairs, col_scale)
+                      : cudaLaunchKernelEx(&cfg, gemv_w4a16_m1_kernel<2>, wmap, smap, zmap, x, (int)N, (int)K, y, ws, cnt,
+                                           max_segs, status, c.npairs, col_scale);
+    if (e != cudaSuccess) return -2;
     return 0;
 }
 
