@@ -806,7 +806,7 @@ def main():
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(t_step, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16 x int4 -> f32 accumulate", "data": "synthetic",
+        "vs_baseline": None, "dtype": "u8 x s8 -> s32 per group (int4 codes x exact radix-128 digits of bf16 x), f32 across groups", "data": "synthetic",
         "config": {"workload": f"full70b decode step: {args.layers} layers x (qkv 8192->10240, o 8192->8192, "
                                "gate+up 8192->57344, down 28672->8192), W4A16 g128 bf16 s/z, M=1",
                    "layers": args.layers, "linears_per_step": launches_per_step, "weights": weights_total,
