@@ -364,10 +364,11 @@ def test_gemm_w4a16_shapes(N, K, g, M):
 
 
 @pytest.mark.parametrize("N,K", [(1, 1024), (33, 1024), (31, 3072), (64, 32768), (4097, 2048), (8192, 8192),
-                                 (100, 65536), (4097, 1152)])
+                                 (100, 65536), (4097, 1152), (65536, 1024), (40000, 2048)])
 def test_gemm_w4a16_m1_stream_k_edges(N, K):
     """M = 1, group 128: a single row, ragged row blocks, the largest K of the TMA kernel, more warps than
-    units; and two shapes it does not take (K > 32768, K not a multiple of 1024)."""
+    units, CTAs whose range holds whole tiles between two split ones (the last two); and two shapes it does
+    not take (K > 32768, K not a multiple of 1024)."""
     _w4_case(N, K, 128, 1, 11 * N + K)
 
 
