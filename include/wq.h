@@ -174,10 +174,16 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  *   qweight, scales, zeros: as produced by wq_quantize_int4 with group g
  *   y       [M][N] bf16, y[m][n] = sum_k x[m][k] * s[n][k/g] * (q[n][k] - z[n][k/g])
  *
- * Arithmetic: every kernel forms the exact integers (q - z) in bf16 (a code
- * pair 128 + q minus the pair 128 + z), multiplies them by x with binary32
- * accumulation (tensor cores for the decode and batched kernels), applies s
- * per group in binary32 and rounds y to bf16 once.  A zero-point outside
+ * Arithmetic: the M = 1 kernel writes x, per group of 128, as 4 planes of
+ * radix-128 integer digits (x_k = 2^(E-5) * sum_c d_ck * 128^-c, |d| <= 64,
+ * 2^E <= max |x| of the group: exact for every |x_k| >= 2^(E-19), others
+ * rounded to a multiple of 2^(E-26)), takes the exact integer sums
+ * sum_k q_k d_ck on the tensor core and applies s * (D_c - z * sum_k d_ck)
+ * per group in binary32.  Every other kernel forms the exact integers (q - z)
+ * in bf16 (a code pair 128 + q minus the pair 128 + z), multiplies them by x
+ * with binary32 accumulation (tensor cores for the decode and batched
+ * kernels), applies s per group in binary32.  y is rounded to bf16 once.
+ * In those kernels a zero-point outside
  * [0, 15] (a group on one side of zero, far from it) is split as
  * z = z_hi + z_lo with z_lo in [0, 16) and z_hi a multiple of 16: the
  * operand is the exact q - z_lo and -z_hi times the group's activation sum
@@ -186,18 +192,22 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * zero and |y - y_exact| stays within 4e-3 * sum_k |x[m][k] * w_hat[n][k]|
  * on the inputs this library is tested on (including activations spanning
  * ~e^+-20).  Split-K partial sums are combined in a fixed order, so repeated
- * calls give identical bytes, except for 2 <= M <= 16, whose partials meet in
+ * calls give identical bytes, except on the older 2 <= M <= 16 kernel (the
+ * shapes below that the persistent one does not take), whose partials meet in
  * binary32 atomics (the last bits of y may then vary between calls).
  * Kernels: M = 1 with g = 128, 1024 <= K <= 32768, K % 1024 == 0: persistent
- * TMA-fed kernel; 2 <= M <= 16 with g = 128: TMA-fed decode kernel; M > 16,
+ * TMA-fed kernel on integer products (exact digits of x, see below);
+ * 2 <= M <= 16 with g = 128 and the same K: the persistent TMA-fed kernel
+ * with the M rows as the MMA's columns, when the activations of a CTA's share
+ * fit shared memory, else a TMA-fed decode kernel (N >= 128, K >= 256); M > 16,
  * or 2 <= M <= 16 with g = 32 or 64 (N >= 128, K % 128 == 0): tcgen05
  * tensor-core kernels; other shapes: a CUDA-core kernel.
  * Requirements: M, N >= 1; K % 32 == 0; g in {32, 64, 128}, K % g == 0;
  * pointers 16-byte aligned; workspace of wq_gemm_workspace_bytes(M, N, K, g, 4)
  * bytes (may be NULL when that is 0).  y must not overlap x, qweight,
  * scales or zeros (WQ_ERR_ARG otherwise).
- * The M = 1 kernel and the tensor-core kernel for M > 16, g = 128 and
- * K % 1024 == 0 are launched
+ * The persistent M = 1 and 2 <= M <= 16 kernels and the tensor-core kernel
+ * for M > 16, g = 128 and K % 1024 == 0 are launched
  * with programmatic dependent launch: they start while the previous kernel
  * on the stream finishes, read x and write only after that kernel has
  * completed, but request their qweight, scales and zeros at once -- so

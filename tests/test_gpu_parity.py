@@ -372,11 +372,13 @@ def test_gemm_w4a16_m1_stream_k_edges(N, K):
     _w4_case(N, K, 128, 1, 11 * N + K)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 3000, 4096), (128, 256, 16384), (40, 384, 8192)])
+@pytest.mark.parametrize("M,N,K", [(1, 3000, 4096), (8, 3000, 4096), (16, 1000, 8192), (128, 256, 16384),
+                                   (40, 384, 8192)])
 def test_gemm_w4a16_workspace_reuse_deterministic(M, N, K):
     """Calls that share one workspace find it ready (its counters re-zeroed by the previous call) and the
     split-K combine runs in a fixed order: the same inputs give the same bytes every time.  M = 1 runs the
-    persistent decode kernel, M = 40 and 128 the tensor-core kernel with K split over many CTAs per tile."""
+    persistent decode kernel, M = 8 and 16 its small-batch form, M = 40 and 128 the tensor-core kernel with
+    K split over many CTAs per tile."""
     w = wq_inputs.llm_weight(N, K, 77)
     q, s, z = wq.wq_quantize_int4(w.cuda(), 128)
     ws = torch.zeros(wq.wq_gemm_workspace_bytes(M, N, K, 128, 4) + 16, dtype=torch.uint8, device="cuda")
@@ -388,6 +390,25 @@ def test_gemm_w4a16_workspace_reuse_deterministic(M, N, K):
     assert torch.equal(outs[0], outs[2]) and torch.equal(outs[0], outs[4])
     assert torch.equal(outs[1], outs[3])
     assert not torch.equal(outs[0], outs[1])
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 1, 1024), (3, 300, 1024), (8, 4097, 2048), (16, 4097, 2048),
+                                   (9, 40000, 2048), (12, 256, 32768), (5, 8192, 8192), (7, 33, 3072)])
+def test_gemm_w4a16_small_batch_persistent(M, N, K):
+    """2 <= M <= 16, group 128, K % 1024 = 0: the persistent small-batch kernel with the M rows as the
+    MMA's columns (8 or 16), a single row, ragged row blocks, tiles split over several CTAs, CTAs holding
+    whole tiles, the longest K, a 2-row-short column tile."""
+    _w4_case(N, K, 128, M, 13 * N + K + M)
+
+
+@pytest.mark.parametrize("M", [8, 16])
+def test_gemm_w4a16_small_batch_large_shape(M):
+    """The gate+up shape at M = 8 (the persistent kernel with two weight stages, its activations filling
+    shared memory) and M = 16 (too many activations for it: the older TMA kernel); rows sampled."""
+    N, K = 57344, 8192
+    w = wq_inputs.llm_weight(N, K, 333)
+    rows = np.r_[0:64, 20000:20064, N - 64:N]
+    _sampled_w4(N, K, 128, (M,), 334, w, rows)  # asserts the bound on every sampled output
 
 
 @pytest.mark.parametrize("M", [1, 2, 5, 8, 16, 17, 40])

@@ -29,6 +29,25 @@ def _m1_needed(N, K):
     return ntiles * max_seg * 256 * 4 + ntiles * 4
 
 
+def _mt_needed(M, N, K):
+    """2 <= M <= 16, g = 128: the persistent kernel's [segment][m][256] slots when the CTA's activation pairs
+    fit shared memory (as the library decides it for a B200), else the older kernel's M x N binary32 buffer."""
+    P = K // 256
+    ntiles = math.ceil(N / 256)
+    units = ntiles * P
+    B = min(units, SMS)
+    npairs = min(-(-units // B), P)
+
+    def total(stages):
+        return stages * 32768 + 16384 + 2 * M * 256 * 4 + npairs * 2 * M * 256 + 16 * 8 + 1024
+
+    if total(3) > 232448 and total(2) > 232448:
+        return M * N * 4
+    cta_of = lambda u: ((u + 1) * B - 1) // units  # noqa: E731
+    max_seg = max(cta_of(t * P + P - 1) - cta_of(t * P) + 1 for t in range(ntiles))
+    return ntiles * max_seg * M * 256 * 4 + ntiles * 4
+
+
 def _tc_needed(M, N, K, g):
     # g = 128 with K a multiple of 1024 runs the split-role kernel: 128-row activation tiles for every M
     BN = 128 if (g == 128 and K % 1024 == 0) else min(32 if M <= 32 else (64 if M <= 64 else 128), g)
@@ -63,3 +82,10 @@ def test_m1_workspace_covers_every_segment(N, K):
                                      (24, 1000, 3072, 128)])
 def test_tc_workspace_covers_every_segment(M, N, K, g):
     assert wq.wq_gemm_workspace_bytes(M, N, K, g, 4) >= _tc_needed(M, N, K, g)
+
+
+@pytest.mark.parametrize("M,N,K", [(2, 1, 1024), (3, 4097, 2048), (8, 28672, 8192), (8, 57344, 8192),
+                                   (8, 8192, 28672), (16, 10240, 8192), (16, 57344, 8192), (5, 300000, 1024),
+                                   (9, 33, 32768), (16, 256 * 149 + 1, 2048)])
+def test_mt_workspace_covers_every_segment(M, N, K):
+    assert wq.wq_gemm_workspace_bytes(M, N, K, 128, 4) >= _mt_needed(M, N, K)
