@@ -27,7 +27,7 @@
 // and KV head for K and V together), and at 4,096 flop per 136 bytes it needs
 // tensor cores to keep up with HBM.  The query heads that share a KV head
 // (r = Hq / H <= 8) share every cache read.
-//  * Kernel 1: one CTA (4 warps) per (KV head, chunk of 512 tokens,
+//  * Kernel 1: one CTA (4 warps) per (KV head, chunk of 1,024 tokens,
 //    sequence).  Phase 1: each warp takes 16-token tiles, dequantises K into
 //    the A operand of mma.sync m16n8k16 (tokens x d) and multiplies by the r
 //    queries (d x heads, padded to 8).  int4 codes become the exact integers
@@ -58,10 +58,10 @@ namespace wq {
 namespace {
 
 constexpr int kD = 128;          // head_dim
-constexpr int kChunk = 512;      // tokens per CTA
+constexpr int kChunk = 1024;     // tokens per CTA: 256 per warp (128 measured 25% slower, 512 slower again)
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kTokPerWarp = kChunk / kWarps;  // 128
+constexpr int kTokPerWarp = kChunk / kWarps;  // 256
 constexpr int kR = 8;            // query heads per KV head, padded
 
 __device__ __forceinline__ void mma_bf16(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
