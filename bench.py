@@ -638,7 +638,7 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------------------
 
-CASES = ("fp8", "nvfp4", "quant_int4", "kv_int4", "kv_fp8", "w8a16", "w4a16_m128", "w4a16_m1")
+CASES = ("fp8", "nvfp4", "quant_int4", "kv_int4", "kv_fp8", "w8a16", "w4a16_m128", "w4a16_m1", "w4a16_m8")
 
 
 def run_case(name, wq, dev):
@@ -683,11 +683,11 @@ def run_case(name, wq, dev):
         del w
         x = wq_inputs.plain_activations(M, 8192, 8, device=dev)
         calls.append(lambda: wq.wq_gemm_w8a16(x, q8, s8, None))
-    elif name in ("w4a16_m128", "w4a16_m1"):
+    elif name in ("w4a16_m128", "w4a16_m1", "w4a16_m8"):
         w = wq_inputs.llm_weight(N, K, 9, outlier_frac=0.0, device=dev)
         q4, s4, z4 = wq.wq_quantize_int4(w, 128)
         del w
-        x = wq_inputs.plain_activations(M if name == "w4a16_m128" else 1, K, 10, device=dev)
+        x = wq_inputs.plain_activations({"w4a16_m128": M, "w4a16_m1": 1, "w4a16_m8": 8}[name], K, 10, device=dev)
         ws = torch.zeros(max(1, wq.wq_gemm_workspace_bytes(x.shape[0], N, K, 128, 4)), dtype=torch.uint8, device=dev)
         calls.append(lambda: wq.wq_gemm_w4a16(x, q4, s4, z4, 128, workspace=ws))
     else:
