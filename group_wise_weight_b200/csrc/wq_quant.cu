@@ -478,6 +478,69 @@ quant_int8_row_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw
     }
 }
 
+// The same for rows that fit in registers: each thread keeps its CH chunks of 8 weights (chunk i at
+// k = 8 (256 i + thread)) as loaded, so the row crosses HBM once and the absmax and the encode read registers.
+template <typename T, int CH>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_int8_row_reg_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw,
+                          int8_t *__restrict__ qweight, uint16_t *__restrict__ scales)
+{
+    constexpr int W = sizeof(T) == 2 ? 1 : 2;  // 16-byte words per chunk of 8 weights
+    __shared__ float warp_max[kQuantThreads / 32];
+    const int64_t n = blockIdx.x;
+    const T *row = w + n * ldw;
+    uint4 r[CH][W];
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+        const int64_t k = ((int64_t)i * kQuantThreads + threadIdx.x) * 8;
+#pragma unroll
+        for (int j = 0; j < W; ++j)
+            r[i][j] = k < K ? ld_stream_v4(row + k + 4 * j) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    auto unpack = [&](int i, float v[8]) {
+        if (sizeof(T) == 2) {
+            const uint32_t u[4] = {r[i][0].x, r[i][0].y, r[i][0].z, r[i][0].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                v[2 * e] = __uint_as_float(u[e] << 16);
+                v[2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+            }
+        } else {
+            const uint4 a = r[i][0], b = r[i][W - 1];
+            v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y);
+            v[2] = __uint_as_float(a.z); v[3] = __uint_as_float(a.w);
+            v[4] = __uint_as_float(b.x); v[5] = __uint_as_float(b.y);
+            v[6] = __uint_as_float(b.z); v[7] = __uint_as_float(b.w);
+        }
+    };
+    float amax = 0.0f;  // chunks past K hold zeros
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+        float v[8];
+        unpack(i, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = warp_max[0];
+#pragma unroll
+    for (int i = 1; i < kQuantThreads / 32; ++i) amax = fmaxf(amax, warp_max[i]);
+    const float s = int8_scale(amax);
+    if (threadIdx.x == 0) scales[n] = f32_to_bf16(s);
+#pragma unroll
+    for (int i = 0; i < CH; ++i) {
+        const int64_t k = ((int64_t)i * kQuantThreads + threadIdx.x) * 8;
+        if (k < K) {
+            float v[8];
+            unpack(i, v);
+            *reinterpret_cast<uint2 *>(qweight + n * K + k) = int8_encode8(v, s);
+        }
+    }
+}
+
 // Symmetric INT4 ("Test-time quantization: quantising on the fly with no calibration dataset", section
 // "The error of quantising an outlier with the wrong scale": s = M / (2^(b-1) - 1) = max|w| / 7 at 4
 // bits; the comparison page's AWQ example: codes -7 to 7).  q = clip(rint(RN(w / s)), -7, 7), stored as
@@ -637,7 +700,13 @@ void dispatch_int8(const void *w, int64_t N, int64_t K, int64_t ldw, int g, int8
                    cudaStream_t st)
 {
     if (g == K) {
-        quant_int8_row_kernel<T><<<(unsigned)N, kQuantThreads, 0, st>>>(static_cast<const T *>(w), N, K, ldw, q, s);
+        // one read of the row when it fits in registers (up to 8 chunks of 8 per thread: K <= 16384; 16 chunks
+        // were slower than two passes at K = 28672, B200)
+        const int64_t per = (K / 8 + kQuantThreads - 1) / kQuantThreads;
+        const T *wt = static_cast<const T *>(w);
+        if (per <= 4) quant_int8_row_reg_kernel<T, 4><<<(unsigned)N, kQuantThreads, 0, st>>>(wt, N, K, ldw, q, s);
+        else if (per <= 8) quant_int8_row_reg_kernel<T, 8><<<(unsigned)N, kQuantThreads, 0, st>>>(wt, N, K, ldw, q, s);
+        else quant_int8_row_kernel<T><<<(unsigned)N, kQuantThreads, 0, st>>>(wt, N, K, ldw, q, s);
         return;
     }
     switch (g) {

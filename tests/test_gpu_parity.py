@@ -129,6 +129,20 @@ def test_quantize_int8_gran_per_channel_fp32():
     assert np.array_equal(bits(s), sb)
 
 
+@pytest.mark.parametrize("N,K,ldw,dtype", [(64, 28672, 28672, torch.bfloat16), (32, 16384, 16384, torch.float32),
+                                            (16, 65536, 65536, torch.bfloat16), (5, 8224, 8232, torch.bfloat16),
+                                            (3, 96, 104, torch.float32)])
+def test_quantize_int8_per_channel_row_lengths(N, K, ldw, dtype):
+    """Per output channel: rows held in registers (4 or 8 chunks of 8 per thread), rows too long for that
+    (two passes), a ragged last chunk row and a padded leading dimension."""
+    base = wq_inputs.block_outlier_weight(N, ldw, 41 + N, dtype=dtype)
+    q, s = wq.wq_quantize_int8(base.cuda()[:, :K])  # a column slice: leading dimension ldw
+    torch.cuda.synchronize()
+    codes, so, sb = oracle_q8(base[:, :K].contiguous(), K)
+    assert np.array_equal(q.cpu().numpy(), codes)
+    assert np.array_equal(bits(s), sb)
+
+
 def test_quantize_padded_rows_and_odd_sizes():
     # ldw > K (a column slice of a wider matrix), N = 1 and N not a multiple of anything
     for N, K, ldw in ((1, 32, 32), (7, 96, 104), (129, 4096 + 128, 4352), (3, 288, 296)):
