@@ -317,13 +317,14 @@ def int8_rows(wq, device, copies=8, reps=5):
     qms = e0.elapsed_time(e1) / (reps * copies)
     del ws
     torch.cuda.empty_cache()
+    wsp = torch.zeros(max(16, wq.wq_gemm_workspace_bytes(1, N, K, K, 8)), dtype=torch.uint8, device=device)
     for c in range(copies):
-        wq.wq_gemm_w8a16(x, qs[c], ss[c], None, y=y)
+        wq.wq_gemm_w8a16(x, qs[c], ss[c], None, y=y, workspace=wsp)
     torch.cuda.synchronize()
     e0.record()
     for r in range(reps * 4):
         for c in range(copies):
-            wq.wq_gemm_w8a16(x, qs[c], ss[c], None, y=y)
+            wq.wq_gemm_w8a16(x, qs[c], ss[c], None, y=y, workspace=wsp)
     e1.record()
     e1.synchronize()
     gms = e0.elapsed_time(e1) / (reps * 4 * copies)
@@ -459,7 +460,8 @@ def config_rows(wq, device, peaks, reps=10):
     for M in (1, 16):
         x = wq_inputs.activations(M, K, 4, device=device)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-        us = _time_rotating([lambda c=c: wq.wq_gemm_w8a16(x, *c, None, y=y) for c in cps8], reps)
+        wsp = torch.zeros(max(16, wq.wq_gemm_workspace_bytes(M, N, K, K, 8)), dtype=torch.uint8, device=device)
+        us = _time_rotating([lambda c=c: wq.wq_gemm_w8a16(x, *c, None, y=y, workspace=wsp) for c in cps8], reps)
         b = N * K + 2 * N + 2 * M * K + 2 * M * N
         w8[f"M{M}"] = {"us": round(us, 2), "GB_s": round(b / us / 1e3, 1), "frac_hbm": round(b / us / 1e3 / hbm, 3)}
     rows["cfg4_w8a16_per_channel"] = dict(w8, shape="K=N=8192 INT8 per channel, 8 copies rotated")
@@ -638,7 +640,8 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------------------
 
-CASES = ("fp8", "nvfp4", "quant_int4", "kv_int4", "kv_fp8", "w8a16", "w4a16_m128", "w4a16_m1", "w4a16_m8")
+CASES = ("fp8", "nvfp4", "quant_int4", "kv_int4", "kv_fp8", "w8a16", "w8a16_m1", "w4a16_m128", "w4a16_m1",
+         "w4a16_m8")
 
 
 def run_case(name, wq, dev):
@@ -677,12 +680,14 @@ def run_case(name, wq, dev):
             del c
         fn = wq.wq_decode_attention_int4 if name == "kv_int4" else wq.wq_decode_attention_fp8
         calls.append(lambda: fn(q, *kv[0], *kv[1], lens))
-    elif name == "w8a16":
+    elif name in ("w8a16", "w8a16_m1"):
         w = wq_inputs.llm_weight(8192, 8192, 7, device=dev)
         q8, s8 = wq.wq_quantize_int8(w, None)
         del w
-        x = wq_inputs.plain_activations(M, 8192, 8, device=dev)
-        calls.append(lambda: wq.wq_gemm_w8a16(x, q8, s8, None))
+        x = wq_inputs.plain_activations(M if name == "w8a16" else 1, 8192, 8, device=dev)
+        ws8 = torch.zeros(max(16, wq.wq_gemm_workspace_bytes(x.shape[0], 8192, 8192, 8192, 8)), dtype=torch.uint8,
+                          device=dev)
+        calls.append(lambda: wq.wq_gemm_w8a16(x, q8, s8, None, workspace=ws8))
     elif name in ("w4a16_m128", "w4a16_m1", "w4a16_m8"):
         w = wq_inputs.llm_weight(N, K, 9, outlier_frac=0.0, device=dev)
         q4, s4, z4 = wq.wq_quantize_int4(w, 128)

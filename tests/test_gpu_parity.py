@@ -545,6 +545,33 @@ def test_gemm_w8a16_repeatable_and_zero_rows():
     assert not y1[:, 7].any() and not y1[:, 300].any()
 
 
+@pytest.mark.parametrize("N,K", [(1, 128), (33, 256), (4097, 1152), (300, 28672), (65536, 1024), (100, 65536),
+                                 (1000, 8192)])
+def test_gemm_w8a16_m1_per_channel_shapes(N, K):
+    """M = 1, per output channel: the persistent integer kernel (one row, ragged row blocks, K not a multiple
+    of 1024, CTAs holding whole tiles, the longest K)."""
+    w = wq_inputs.block_outlier_weight(N, K, 31 * N + K)
+    x = wq_inputs.activations(1, K, 37 * N + K)
+    _w8_case(w, x, None)
+
+
+def test_gemm_w8a16_m1_exact_zero_rows_and_repeatable():
+    """M = 1, per output channel: rows of zero weights give exactly zero even for activations spanning many
+    binades, and the split-K combine runs in a fixed order (identical bytes on repeat)."""
+    N, K = 640, 2048
+    w = wq_inputs.block_outlier_weight(N, K, 43)
+    w[::5] = 0.0
+    x = wq_inputs.wide_range_activations(1, K, 47)
+    _w8_case(w, x, None)
+    q, s = wq.wq_quantize_int8(w.cuda(), None)
+    xd = x.cuda()
+    y1 = wq.wq_gemm_w8a16(xd, q, s, None)
+    y2 = wq.wq_gemm_w8a16(xd, q, s, None)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert not y1[:, ::5].any()
+
+
 def test_gemm_w8a16_gran_per_channel():
     w = wq_inputs.block_outlier_weight(8192, 8192, wq_inputs.SEEDS["gran"])
     rows = sample_rows(8192, 192, 5)

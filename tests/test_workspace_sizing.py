@@ -89,3 +89,22 @@ def test_tc_workspace_covers_every_segment(M, N, K, g):
                                    (9, 33, 32768), (16, 256 * 149 + 1, 2048)])
 def test_mt_workspace_covers_every_segment(M, N, K):
     assert wq.wq_gemm_workspace_bytes(M, N, K, 128, 4) >= _mt_needed(M, N, K)
+
+
+def _w8m1_needed(N, K):
+    G = K // 128                      # groups of 128 inputs (units) per 256-row tile
+    ntiles = math.ceil(N / 256)
+    units = ntiles * G
+    B = min(units, SMS)
+    nslots = min(-(-units // B), G)
+    if 3 * 32768 + 2048 + nslots * 516 + 96 + 1024 > 232448:
+        return 0                      # not taken: another kernel, another workspace
+    cta_of = lambda u: ((u + 1) * B - 1) // units  # noqa: E731
+    max_seg = max(cta_of(t * G + G - 1) - cta_of(t * G) + 1 for t in range(ntiles))
+    return ntiles * max_seg * 256 * 4 + ntiles * 4
+
+
+@pytest.mark.parametrize("N,K", [(1, 128), (33, 256), (4097, 1152), (300, 28672), (65536, 1024), (100, 65536),
+                                 (8192, 8192), (57344, 8192)])
+def test_w8m1_workspace_covers_every_segment(N, K):
+    assert wq.wq_gemm_workspace_bytes(1, N, K, K, 8) >= _w8m1_needed(N, K)
