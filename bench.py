@@ -226,19 +226,24 @@ class Model:
         quant_bytes = 0
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         for layer in range(layers):
+            # a layer's four bf16 weights (1.7 GB) are generated first, then quantised back to back, the way a
+            # model is quantised: events around the layer's four calls
+            ws, outs = [], []
             for j, (name, K, N) in enumerate(wq_inputs.FULL70B_LINEARS):
-                w = wq_inputs.llm_weight(N, K, wq_inputs.full70b_seed(layer, j), outlier_frac=0.0, device=device)
-                q = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
-                s = torch.empty((N, K // G), dtype=torch.bfloat16, device=device)
-                z = torch.empty((N, K // G), dtype=torch.bfloat16, device=device)
-                ev0.record()
+                ws.append(wq_inputs.llm_weight(N, K, wq_inputs.full70b_seed(layer, j), outlier_frac=0.0, device=device))
+                outs.append((name, K, N, torch.empty((N, K // 2), dtype=torch.uint8, device=device),
+                             torch.empty((N, K // G), dtype=torch.bfloat16, device=device),
+                             torch.empty((N, K // G), dtype=torch.bfloat16, device=device)))
+            ev0.record()
+            for w, (name, K, N, q, s, z) in zip(ws, outs):
                 wq.wq_quantize_int4(w, G, q, s, z)
-                ev1.record()
-                ev1.synchronize()
-                quant_ms += ev0.elapsed_time(ev1)
+            ev1.record()
+            ev1.synchronize()
+            quant_ms += ev0.elapsed_time(ev1)
+            for name, K, N, q, s, z in outs:
                 quant_bytes += N * K * 2 + N * K // 2 + 4 * N * (K // G)
-                del w
                 self.linears.append((name, K, N, q, s, z))
+            del ws
         torch.cuda.empty_cache()
         self.quant_ms, self.quant_bytes = quant_ms, quant_bytes
         self.weights = sum(K * N for _, K, N, *_ in self.linears)
@@ -827,7 +832,7 @@ def main():
                  "steps": m128_steps},
         "rows": {
             "a1_quantize_int4": {"GB_s": round(quant_gbs, 1), "ms_total": round(model.quant_ms, 2),
-                                 "shape": "all 320 linears, bf16 -> int4 g128"},
+                                 "shape": "all 320 linears, bf16 -> int4 g128, each layer's four calls back to back"},
             "a2_quantize_int8": {k: (round(v, 2) if isinstance(v, float) else v) for k, v in q8_row.items()},
             "a4_w4a16_m1_per_linear": lin,
             "a5_w4a16_m128": {"tflops": round(tflops128 / world, 1)},
