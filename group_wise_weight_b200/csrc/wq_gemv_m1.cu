@@ -230,6 +230,10 @@ __device__ __forceinline__ void make_digits(const uint16_t *__restrict__ xg, con
     float m = fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3])));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    // an infinite or NaN activation makes the group's factor NaN, so y is not finite, as x * w_hat would be
+    const bool nonfinite = __any_sync(0xffffffffu, !(fabsf(e[0]) < INFINITY && fabsf(e[1]) < INFINITY &&
+                                                     fabsf(e[2]) < INFINITY && fabsf(e[3]) < INFINITY));
+    if (nonfinite) m = 0.0f;
     // 2^E <= m < 2^(E + 1); a group of zeros gets E = 0 (all digits 0)
     int E = m > 0.0f ? (int)((__float_as_uint(m) >> 23) & 0xff) - 127 : 0;
     if (m > 0.0f && E == -127) E = -127 + (31 - __clz((int)(__float_as_uint(m) & 0x7fffff))) - 22;  // subnormal
@@ -262,7 +266,8 @@ __device__ __forceinline__ void make_digits(const uint16_t *__restrict__ xg, con
     // weight of digit 0: 2^(E - 5) (binary32 loses precision only below 2^-126)
     if (lane == 0) {
         const int ef = E - 5;
-        const float f = ef >= -126 ? exp2i(ef) : exp2i(ef + 64) * 5.421010862427522e-20f;  // 2^-64
+        float f = ef >= -126 ? exp2i(ef) : exp2i(ef + 64) * 5.421010862427522e-20f;  // 2^-64
+        if (nonfinite) f = __int_as_float(0x7fc00000);                                 // NaN
         asm volatile("st.shared.f32 [%0], %1;" ::"r"(gfac_g), "f"(f) : "memory");
     }
 }

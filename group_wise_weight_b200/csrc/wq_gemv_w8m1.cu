@@ -130,6 +130,10 @@ __device__ __forceinline__ void make_digits8(uint4 v, uint32_t dig_g, uint32_t g
     float m = fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3])));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    // an infinite or NaN activation makes the group's factor NaN, so y is not finite, as x * w_hat would be
+    const bool nonfinite = __any_sync(0xffffffffu, !(fabsf(e[0]) < INFINITY && fabsf(e[1]) < INFINITY &&
+                                                     fabsf(e[2]) < INFINITY && fabsf(e[3]) < INFINITY));
+    if (nonfinite) m = 0.0f;
     int E = m > 0.0f ? (int)((__float_as_uint(m) >> 23) & 0xff) - 127 : 0;
     if (m > 0.0f && E == -127) E = -127 + (31 - __clz((int)(__float_as_uint(m) & 0x7fffff))) - 22;  // subnormal
     const int a1 = (5 - E) / 2, a2 = (5 - E) - a1;
@@ -154,7 +158,8 @@ __device__ __forceinline__ void make_digits8(uint4 v, uint32_t dig_g, uint32_t g
     }
     if (lane == 0) {
         const int ef = E - 5;
-        const float f = ef >= -126 ? exp2i(ef) : exp2i(ef + 64) * 5.421010862427522e-20f;  // 2^-64
+        float f = ef >= -126 ? exp2i(ef) : exp2i(ef + 64) * 5.421010862427522e-20f;  // 2^-64
+        if (nonfinite) f = __int_as_float(0x7fc00000);                                 // NaN
         asm volatile("st.shared.f32 [%0], %1;" ::"r"(gfac_g), "f"(f) : "memory");
     }
 }

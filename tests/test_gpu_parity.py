@@ -425,6 +425,23 @@ def test_gemm_w4a16_small_batch_large_shape(M):
     _sampled_w4(N, K, 128, (M,), 334, w, rows)  # asserts the bound on every sampled output
 
 
+@pytest.mark.parametrize("M", [1, 4, 128])
+def test_gemm_nonfinite_activation_propagates(M):
+    """An infinite activation makes every output non-finite (x_k * w_hat_nk is +-inf, or NaN where
+    w_hat_nk = 0), on every kernel; the M = 1 kernels carry it through their digit planes as a NaN factor."""
+    N, K = 512, 2048
+    w = wq_inputs.llm_weight(N, K, 51)
+    x = wq_inputs.activations(M, K, 52)
+    x[:, 300] = float("inf")
+    q, s, z = wq.wq_quantize_int4(w.cuda(), 128)
+    y = wq.wq_gemm_w4a16(x.cuda(), q, s, z, 128)
+    q8, s8 = wq.wq_quantize_int8(w.cuda(), None)
+    y8 = wq.wq_gemm_w8a16(x.cuda(), q8, s8, None)
+    torch.cuda.synchronize()
+    assert not torch.isfinite(y.float()).any()
+    assert not torch.isfinite(y8.float()).any()
+
+
 @pytest.mark.parametrize("M", [1, 2, 5, 8, 16, 17, 40])
 def test_gemm_w4a16_zero_rows_exact(M):
     """Rows (and groups) whose weights are all zero have w_hat = 0, so the bound is 0: y must be exactly 0,
