@@ -268,7 +268,7 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
         return wq::gemv_tma_workspace_bytes(M, N, K, g);
     }
     if (wbits == 8) {
-        if (wq::gemv_w8m1_eligible(M, N, K, g)) return wq::gemv_w8m1_workspace_bytes(M, N, K, g);
+        if (wq::gemv_w8int_eligible(M, N, K, g)) return wq::gemv_w8int_workspace_bytes(M, N, K, g);
         return wq::gemm_tc_w8_workspace_bytes(M, N, K, g);
     }
     return 0;
@@ -297,11 +297,11 @@ int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8
     const size_t need = wq_gemm_workspace_bytes(M, N, K, g, 8);
     if (need > 0 && (!workspace || ws_bytes < need || !aligned16(workspace)))
         return fail(WQ_ERR_WORKSPACE, "wq_gemm_w8a16: need %zu workspace bytes", need);
-    if (wq::gemv_w8m1_eligible(M, N, K, g)) {
+    if (wq::gemv_w8int_eligible(M, N, K, g)) {
         int *status = status_word();
         if (!status) return fail(WQ_ERR_CUDA, "wq_gemm_w8a16: no device status word");
-        const int rc = wq::launch_gemv_w8a16_m1(x, N, K, qweight, scales, y, workspace, status,
-                                                static_cast<cudaStream_t>(stream));
+        const int rc = wq::launch_gemv_w8a16_int(x, M, N, K, qweight, scales, y, workspace, status,
+                                                 static_cast<cudaStream_t>(stream));
         if (rc == -1) return fail(WQ_ERR_CUDA, "wq_gemm_w8a16: tensor map encoding failed");
         return check_launch("wq_gemm_w8a16");
     }

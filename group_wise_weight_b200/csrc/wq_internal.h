@@ -51,15 +51,16 @@ size_t gemv_mt_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
 int launch_gemv_w4a16_mt(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
                          const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st);
 
-// W8A16 per output channel at M = 1 (wq_gemv_w8m1.cu): persistent TMA-fed stream of the int8 codes, integer
-// mma.sync s8 x s8 against exact digit planes of x.  Eligible for g == K, K % 128 == 0, 128 <= K <= 65536
-// when a CTA's digit planes fit shared memory.  Workspace of gemv_w8m1_workspace_bytes() (zero-filled before
-// first use; the kernel leaves its counters zeroed); the device status word for its bounded waits.  Returns
-// 0, -1 if the tensor map cannot be encoded, -2 if the launch fails.
-bool gemv_w8m1_eligible(int64_t M, int64_t N, int64_t K, int g);
-size_t gemv_w8m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
-int launch_gemv_w8a16_m1(const uint16_t *x, int64_t N, int64_t K, const int8_t *q, const uint16_t *s, uint16_t *y,
-                         void *workspace, int *status, cudaStream_t st);
+// W8A16 per output channel at 1 <= M <= 8 (wq_gemv_w8int.cu): persistent TMA-fed stream of the int8 codes,
+// integer mma.sync s8 x s8 against exact digit planes of x.  Eligible for g == K, K % 128 == 0,
+// 128 <= K <= 65536 when a CTA's digit planes and two stages fit shared memory.  Workspace of
+// gemv_w8int_workspace_bytes() (zero-filled before first use; the kernel leaves its counters zeroed); the
+// device status word for its bounded waits.  Returns 0, -1 if the tensor map cannot be encoded, -2 if the
+// launch fails.
+bool gemv_w8int_eligible(int64_t M, int64_t N, int64_t K, int g);
+size_t gemv_w8int_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
+int launch_gemv_w8a16_int(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *q, const uint16_t *s,
+                          uint16_t *y, void *workspace, int *status, cudaStream_t st);
 
 // TMA-pipelined W4A16 for group 128 and M <= 16 (wq_gemv_tma.cu).  Needs a
 // workspace of gemv_tma_workspace_bytes() (zero-filled before first use; the

@@ -222,13 +222,14 @@ int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint
 /*
  * W8A16 weight-only matmul: y[m][n] = sum_k x[m][k] * s[n][k/g] * q[n][k]
  * ([P3] dequantised value q * s).  qweight [N][K] int8, scales [N][K/g]
- * bf16, g in {32, 64, 128, K}.  Kernels: M = 1 with g = K (per output
- * channel), K % 128 == 0 and 128 <= K <= 65536: a persistent TMA-fed kernel
+ * bf16, g in {32, 64, 128, K}.  Kernels: 1 <= M <= 8 with g = K (per output
+ * channel), K % 128 == 0 and 128 <= K <= 65536, when the digit planes of a
+ * CTA's share of K fit shared memory: a persistent TMA-fed kernel
  * on exact integer products (q as signed bytes against the radix-128 digit
  * planes of x described under wq_gemm_w4a16, s applied per row in binary32),
  * launched with programmatic dependent launch (qweight must not have been
- * written by the kernel just before on the same stream); M >= 2 with N >= 128
- * and K % 128 == 0: the tcgen05 tensor-core kernel (q converted exactly to
+ * written by the kernel just before on the same stream); other M >= 2 with
+ * N >= 128 and K % 128 == 0: the tcgen05 tensor-core kernel (q converted exactly to
  * bf16, binary32 accumulation per group of g, or per 128 k for g = K, scaled
  * and summed in binary32); otherwise a CUDA-core kernel.  Workspace of
  * wq_gemm_workspace_bytes(M, N, K, g, 8) bytes.  Other arguments and

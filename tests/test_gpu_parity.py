@@ -572,6 +572,17 @@ def test_gemm_w8a16_m1_per_channel_shapes(N, K):
     _w8_case(w, x, None)
 
 
+@pytest.mark.parametrize("M,N,K", [(2, 1, 128), (3, 300, 1152), (4, 4097, 2048), (8, 1000, 8192), (9, 257, 4096),
+                                   (16, 8192, 8192), (16, 40000, 1024)])
+def test_gemm_w8a16_small_batch_per_channel(M, N, K):
+    """2 <= M <= 16, per output channel: the persistent integer kernel with M rows x 4 digits in the MMA's
+    B columns (1, 2 or 4 column tiles, M <= 8), or, at M > 8 and where its digit planes do not fit, the
+    tensor-core kernel."""
+    w = wq_inputs.block_outlier_weight(N, K, 53 * N + K + M)
+    x = wq_inputs.activations(M, K, 59 * N + K + M)
+    _w8_case(w, x, None, rows=None if N * K <= 8192 * 1024 else sample_rows(N, 256, M))
+
+
 def test_gemm_w8a16_m1_exact_zero_rows_and_repeatable():
     """M = 1, per output channel: rows of zero weights give exactly zero even for activations spanning many
     binades, and the split-K combine runs in a fixed order (identical bytes on repeat)."""

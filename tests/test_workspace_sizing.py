@@ -91,20 +91,31 @@ def test_mt_workspace_covers_every_segment(M, N, K):
     assert wq.wq_gemm_workspace_bytes(M, N, K, 128, 4) >= _mt_needed(M, N, K)
 
 
-def _w8m1_needed(N, K):
+def _w8int_needed(M, N, K):
+    """W8A16 per channel, 1 <= M <= 8: the persistent integer kernel's [segment][m][256] slots when a CTA's
+    digit planes fit shared memory with two or three stages (as the library decides for a B200); 0 when
+    another kernel takes the shape."""
     G = K // 128                      # groups of 128 inputs (units) per 256-row tile
     ntiles = math.ceil(N / 256)
     units = ntiles * G
     B = min(units, SMS)
     nslots = min(-(-units // B), G)
-    if 3 * 32768 + 2048 + nslots * 516 + 96 + 1024 > 232448:
-        return 0                      # not taken: another kernel, another workspace
+    if M > 8:
+        return 0
+    NT = 1 if M <= 2 else 2 if M <= 4 else 4
+
+    def total(stages):
+        return stages * 32768 + 2 * M * 1024 + nslots * 1024 * NT + nslots * 64 + 14 * 8 + 1024
+
+    if total(3) > 232448 and total(2) > 232448:
+        return 0
     cta_of = lambda u: ((u + 1) * B - 1) // units  # noqa: E731
     max_seg = max(cta_of(t * G + G - 1) - cta_of(t * G) + 1 for t in range(ntiles))
-    return ntiles * max_seg * 256 * 4 + ntiles * 4
+    return ntiles * max_seg * M * 256 * 4 + ntiles * 4
 
 
-@pytest.mark.parametrize("N,K", [(1, 128), (33, 256), (4097, 1152), (300, 28672), (65536, 1024), (100, 65536),
-                                 (8192, 8192), (57344, 8192)])
-def test_w8m1_workspace_covers_every_segment(N, K):
-    assert wq.wq_gemm_workspace_bytes(1, N, K, K, 8) >= _w8m1_needed(N, K)
+@pytest.mark.parametrize("M,N,K", [(1, 1, 128), (1, 33, 256), (1, 4097, 1152), (1, 300, 28672), (1, 65536, 1024),
+                                   (1, 100, 65536), (1, 8192, 8192), (1, 57344, 8192), (2, 4097, 2048),
+                                   (5, 8192, 8192), (8, 10240, 8192), (16, 8192, 8192), (16, 57344, 8192)])
+def test_w8int_workspace_covers_every_segment(M, N, K):
+    assert wq.wq_gemm_workspace_bytes(M, N, K, K, 8) >= _w8int_needed(M, N, K)
