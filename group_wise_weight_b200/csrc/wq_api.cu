@@ -166,6 +166,13 @@ int run_w4a16(const char *what, const uint16_t *x, int64_t M, int64_t N, int64_t
         if (rc == -1) return fail(WQ_ERR_CUDA, "%s: tensor map encoding failed", what);
         return check_launch(what);
     }
+    if (wq::gemv_i4mt_eligible(M, N, K, g)) {
+        int *status = status_word();
+        if (!status) return fail(WQ_ERR_CUDA, "%s: no device status word", what);
+        const int rc = wq::launch_gemv_w4a16_i4mt(x, M, N, K, qweight, scales, zeros, y, workspace, status, st);
+        if (rc == -1) return fail(WQ_ERR_CUDA, "%s: tensor map encoding failed", what);
+        return check_launch(what);
+    }
     if (wq::gemv_mt_eligible(M, N, K, g)) {
         int *status = status_word();
         if (!status) return fail(WQ_ERR_CUDA, "%s: no device status word", what);
@@ -264,6 +271,7 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
     if (wbits == 4) {
         if (wq::gemm_tc_eligible(M, N, K, g)) return wq::gemm_tc_workspace_bytes(M, N, K, g);
         if (wq::gemv_m1_eligible(M, N, K, g)) return wq::gemv_m1_workspace_bytes(M, N, K, g);
+        if (wq::gemv_i4mt_eligible(M, N, K, g)) return wq::gemv_i4mt_workspace_bytes(M, N, K, g);
         if (wq::gemv_mt_eligible(M, N, K, g)) return wq::gemv_mt_workspace_bytes(M, N, K, g);
         return wq::gemv_tma_workspace_bytes(M, N, K, g);
     }

@@ -123,7 +123,8 @@ __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t
 // The digit planes and the scale factor of one group of x (one warp).  Lane L holds word L / 2 of the group
 // (inputs 8 (L / 2) .. + 7) and takes of it the four inputs 4 (L % 2) .. + 3, the byte order of the A
 // operand's words: codes k .. k + 3 of the first word of a step, k + 4 .. k + 7 of the second.
-// cols: the columns of the group's tile layout (8 per tile); column 4 row + c holds digit c of that row.
+// cols: the columns of the group's tile layout (8 per tile); column 4 row + c holds digit c of that row, stored
+// at (4 row + c) ^ 2 t so that the 8 lanes of a shared-memory phase (two columns, four quads) read 8 bank groups.
 __device__ __forceinline__ void make_digits8(uint4 v, uint32_t dig_g, int cols, int row, uint32_t gfac_g, int lane)
 {
     const int wq_ = lane >> 1, par = lane & 1;
@@ -156,11 +157,13 @@ __device__ __forceinline__ void make_digits8(uint4 v, uint32_t dig_g, int cols, 
         }
     }
     const int t_ = wq_ >> 2, w = wq_ & 3, half = w >> 1;
-    const uint32_t dst = dig_g + (uint32_t)(((half * 4 + t_) * cols + 4 * row) * 16 + (w & 1) * 8 + par * 4);
+    const uint32_t dst0 = dig_g + (uint32_t)(((half * 4 + t_) * cols) * 16 + (w & 1) * 8 + par * 4);
 #pragma unroll
     for (int c = 0; c < kDigits; ++c) {
         const uint32_t lo = __byte_perm(t[0][c], t[1][c], 0x0040), hi = __byte_perm(t[2][c], t[3][c], 0x0040);
-        asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst + (uint32_t)c * 16u), "r"(__byte_perm(lo, hi, 0x5410)) : "memory");
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst0 + (uint32_t)(((4 * row + c) ^ (2 * t_)) * 16)),
+                     "r"(__byte_perm(lo, hi, 0x5410))
+                     : "memory");
     }
     if (lane == 0) {
         const int ef = E - 5;
@@ -383,7 +386,8 @@ gemv_w8a16_int_kernel(const __grid_constant__ CUtensorMap wmap, const uint16_t *
                 uint4 Bv[2];
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf)
-                    Bv[hf] = bok ? lds128(slot + (uint32_t)(((hf * 4 + tq) * kCols + col) * 16)) : make_uint4(0u, 0u, 0u, 0u);
+                    Bv[hf] = bok ? lds128(slot + (uint32_t)(((hf * 4 + tq) * kCols + (col ^ (2 * tq))) * 16))
+                                 : make_uint4(0u, 0u, 0u, 0u);
                 uint32_t C[4];
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {

@@ -41,6 +41,17 @@ int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t 
                          const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st,
                          const float *col_scale = nullptr);
 
+// W4A16 for group 128 and M = 2 on integer products (wq_gemv_i4mt.cu): the M = 1 kernel with 2 rows x 4 digits
+// in the MMA's B columns.  Eligible for 1024 <= K <= 32768, K % 1024 == 0 when a CTA's digit planes and
+// two stages fit shared memory.  Workspace of gemv_i4mt_workspace_bytes() (zero-filled before first use; the
+// kernel leaves its counters zeroed); the device status word.  Returns 0, -1 if a tensor map cannot be
+// encoded, -2 if the launch fails.
+bool gemv_i4mt_eligible(int64_t M, int64_t N, int64_t K, int g);
+size_t gemv_i4mt_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
+int launch_gemv_w4a16_i4mt(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
+                           const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st,
+                           const float *col_scale = nullptr);
+
 // W4A16 for group 128 and 2 <= M <= 16 (wq_gemv_mt.cu): the M = 1 kernel's weight stream with the M
 // activation rows as the bf16 columns of mma.sync and exact bf16 q - z operands.  Eligible when, in addition,
 // 1024 <= K <= 32768, K % 1024 == 0 and the CTA's activation pairs fit shared memory.  Workspace of
