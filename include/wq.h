@@ -198,8 +198,9 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * Kernels: M = 1 with g = 128, 1024 <= K <= 32768, K % 1024 == 0: persistent
  * TMA-fed kernel on integer products (exact digits of x, see below);
  * 2 <= M <= 16 with g = 128 and the same K: the persistent TMA-fed kernel
- * with the M rows as the MMA's columns, when the activations of a CTA's share
- * fit shared memory, else a TMA-fed decode kernel (N >= 128, K >= 256); M > 16,
+ * with the M rows as the MMA's columns (at M = 2 on the integer products of
+ * the M = 1 kernel), when the activations of a CTA's share fit shared
+ * memory, else a TMA-fed decode kernel (N >= 128, K >= 256); M > 16,
  * or 2 <= M <= 16 with g = 32 or 64 (N >= 128, K % 128 == 0): tcgen05
  * tensor-core kernels; other shapes: a CUDA-core kernel.
  * Requirements: M, N >= 1; K % 32 == 0; g in {32, 64, 128}, K % g == 0;

@@ -386,8 +386,8 @@ def test_gemm_w4a16_m1_stream_k_edges(N, K):
     _w4_case(N, K, 128, 1, 11 * N + K)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 3000, 4096), (8, 3000, 4096), (16, 1000, 8192), (128, 256, 16384),
-                                   (40, 384, 8192)])
+@pytest.mark.parametrize("M,N,K", [(1, 3000, 4096), (2, 3000, 4096), (8, 3000, 4096), (16, 1000, 8192),
+                                   (128, 256, 16384), (40, 384, 8192)])
 def test_gemm_w4a16_workspace_reuse_deterministic(M, N, K):
     """Calls that share one workspace find it ready (its counters re-zeroed by the previous call) and the
     split-K combine runs in a fixed order: the same inputs give the same bytes every time.  M = 1 runs the
@@ -425,7 +425,7 @@ def test_gemm_w4a16_small_batch_large_shape(M):
     _sampled_w4(N, K, 128, (M,), 334, w, rows)  # asserts the bound on every sampled output
 
 
-@pytest.mark.parametrize("M", [1, 4, 128])
+@pytest.mark.parametrize("M", [1, 2, 4, 128])
 def test_gemm_nonfinite_activation_propagates(M):
     """An infinite activation makes every output non-finite (x_k * w_hat_nk is +-inf, or NaN where
     w_hat_nk = 0), on every kernel; the M = 1 kernels carry it through their digit planes as a NaN factor."""
