@@ -162,7 +162,7 @@ int run_w4a16(const char *what, const uint16_t *x, int64_t M, int64_t N, int64_t
     if (wq::gemv_m1_eligible(M, N, K, g)) {
         int *status = status_word();
         if (!status) return fail(WQ_ERR_CUDA, "%s: no device status word", what);
-        const int rc = wq::launch_gemv_w4a16_m1(x, N, K, qweight, scales, zeros, y, workspace, status, st, col_scale);
+        const int rc = wq::launch_gemv_w4a16_m1(x, N, K, qweight, scales, zeros, g, y, workspace, status, st, col_scale);
         if (rc == -1) return fail(WQ_ERR_CUDA, "%s: tensor map encoding failed", what);
         return check_launch(what);
     }

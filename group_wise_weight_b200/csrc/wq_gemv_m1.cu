@@ -95,7 +95,6 @@ constexpr int kTile = 16 * kC;                    // rows per tile (256)
 constexpr int kMaxStages = 3;                     // weight stages in flight (2 for the longest K)
 constexpr uint32_t kStageBytes = kTile * 128;     // 256 rows x 2 groups x 64 B
 constexpr uint32_t kSzBytes = kTile * 16;         // 256 rows x 8 groups x 2 B (one of s or z)
-constexpr int kPairsPerWindow = 4;                // 8 groups of s/z = 4 units
 constexpr int kDigits = 4;                        // radix-128 digit planes of x
 constexpr uint32_t kDigitPairBytes = 2 * 2 * 4 * kDigits * 16;  // [group][half][t][digit][16 B]
 constexpr float kMagic = 12582912.0f;             // 1.5 * 2^23
@@ -104,13 +103,13 @@ constexpr uint32_t kMagicBits = 0x4B400000u;
 // shared memory: [stages][s/z windows][2 partial tiles][digit planes][S sums][group factors][barriers]
 struct M1Layout {
     size_t sz, part, dig, gsum, gfac, bar, total;
-    __host__ __device__ M1Layout(int stages, int npairs)
+    __host__ __device__ M1Layout(int stages, int npairs, int sub)
     {
         sz = (size_t)stages * kStageBytes;
         part = sz + 2 * 2 * kSzBytes;
         dig = part + 2 * kTile * 4;
         gsum = dig + (size_t)npairs * kDigitPairBytes;
-        gfac = gsum + (size_t)npairs * 2 * kDigits * 4;
+        gfac = gsum + (size_t)npairs * 2 * sub * kDigits * 4;
         bar = (gfac + (size_t)npairs * 2 * 4 + 7) & ~(size_t)7;
         total = bar + (2 * kMaxStages + 4 + 4 + 2) * 8 + 1024;
     }
@@ -150,6 +149,13 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t addr)
 {
     uint32_t r;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
+    return r;
+}
+
+__device__ __forceinline__ uint16_t lds_u16(uint32_t addr)
+{
+    uint16_t r;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr));
     return r;
 }
 
@@ -215,6 +221,9 @@ __device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t
 // The digit planes, column sums and scale factor of one group of x (one warp).  Lane L takes word L / 2 of
 // the group (inputs 8 (L / 2) .. + 7) and of it the inputs of parity L % 2: 2 i + L % 2, i = 0 .. 3, the byte
 // order of the A operand's even (L % 2 = 0) and odd code words.
+// SUB quantisation groups share the 128 inputs (groups of 128 / SUB): their column sums are kept apart, each
+// over the lanes that hold its inputs (32 / SUB consecutive lanes).
+template <int SUB>
 __device__ __forceinline__ void make_digits(const uint16_t *__restrict__ xg, const float *__restrict__ csg,
                                             uint32_t dig_pair, uint32_t gsum_g, uint32_t gfac_g, int h, int lane)
 {
@@ -260,8 +269,18 @@ __device__ __forceinline__ void make_digits(const uint16_t *__restrict__ xg, con
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst + (uint32_t)c * 16u), "r"(packed) : "memory");
         // the digit values (wrapping 32-bit arithmetic: the four magic offsets cancel)
         const int sum = (int)(t[0][c] + t[1][c] + t[2][c] + t[3][c] - 4u * kMagicBits);
-        const int tot = __reduce_add_sync(0xffffffffu, sum);
-        if (lane == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(gsum_g + (uint32_t)c * 4u), "f"((float)tot) : "memory");
+        if constexpr (SUB == 1) {
+            const int tot = __reduce_add_sync(0xffffffffu, sum);
+            if (lane == 0) asm volatile("st.shared.f32 [%0], %1;" ::"r"(gsum_g + (uint32_t)c * 4u), "f"((float)tot) : "memory");
+        } else {
+            int tot = sum;  // over the 32 / SUB lanes of this lane's group
+#pragma unroll
+            for (int o = 1; o < 32 / SUB; o <<= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+            if ((lane & (32 / SUB - 1)) == 0)
+                asm volatile("st.shared.f32 [%0], %1;" ::"r"(gsum_g + (uint32_t)((lane / (32 / SUB)) * kDigits + c) * 4u),
+                             "f"((float)tot)
+                             : "memory");
+        }
     }
     // weight of digit 0: 2^(E - 5) (binary32 loses precision only below 2^-126)
     if (lane == 0) {
@@ -273,7 +292,7 @@ __device__ __forceinline__ void make_digits(const uint16_t *__restrict__ xg, con
 }
 
 // 18 warps put five on one SM sub-partition, whose register file holds 16K registers: at most 96 each.
-template <int STAGES>
+template <int GROUP, int STAGES>
 __global__ void __maxnreg__(96)
 gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                      const __grid_constant__ CUtensorMap zmap, const uint16_t *__restrict__ x, int N, int K,
@@ -283,7 +302,9 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     extern __shared__ __align__(1024) uint8_t m1_raw[];
     // TMA destinations want 128-byte (we keep 1024-byte) alignment: align the base explicitly
     uint8_t *sm = m1_raw + ((1024u - (smem_u32(m1_raw) & 1023u)) & 1023u);
-    const M1Layout L(STAGES, npairs);
+    constexpr int SUB = 128 / GROUP;  // quantisation groups per 128 inputs
+    constexpr int UPW = GROUP / 32;   // units per s/z window of 8 groups
+    const M1Layout L(STAGES, npairs, SUB);
     uint8_t *ring = sm;
     uint8_t *szr = sm + L.sz;                                     // [2 windows][s, z][256 rows][8 groups]
     float *part = reinterpret_cast<float *>(sm + L.part);         // [2][256 rows] partial sums
@@ -335,15 +356,17 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     auto issue_window = [&](int slot) {
         mbar_arrive_expect_tx(&szfull[slot], 2 * kSzBytes);
         uint8_t *d = szr + (uint32_t)slot * 2u * kSzBytes;
-        const int g8 = (2 * pp) & ~7;
+        const int g8 = (2 * SUB * pp) & ~7;  // the window's first group
         tma_load_2d(d, &smap, &szfull[slot], g8, pt * kTile);
         tma_load_2d(d + kSzBytes, &zmap, &szfull[slot], g8, pt * kTile);
         ++wins;
     };
     if (wid == kProducer && lane == 0) {
-        // at most two windows start within the first STAGES pairs, so no window slot needs a wait here
+        // the prologue issues at most two windows (the ring's slots) and leaves a third to the main loop
         for (; pi < STAGES && pi < n; ++pi) {
-            if (pi == 0 || (pp & (kPairsPerWindow - 1)) == 0) issue_window(wins & 1);
+            const bool nw = pi == 0 || (pp & (UPW - 1)) == 0;
+            if (nw && wins >= 2) break;
+            if (nw) issue_window(wins & 1);
             mbar_arrive_expect_tx(&full[pi], kStageBytes);
             tma_load_3d(ring + (uint32_t)pi * kStageBytes, &wmap, &full[pi], 0, pt * kTile, 2 * pp);
             if (++pp == P) { pp = 0; ++pt; }
@@ -356,8 +379,8 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         if (lane == 0 && n > 0) {
             int i = pi;
             for (; i < n; ++i) {
-                // s/z window: at every 4th pair of a tile
-                if ((pp & (kPairsPerWindow - 1)) == 0) {
+                // s/z window: at the first unit and at every UPW-th pair of a tile
+                if (i == 0 || (pp & (UPW - 1)) == 0) {
                     const int slot = wins & 1;
                     if (wins >= 2 && !mbar_wait(&szempty[slot], (uint32_t)((wins >> 1) - 1) & 1u, status, flags)) break;
                     issue_window(slot);
@@ -456,9 +479,10 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             int pj = pair0 + js;
             if (pj >= P) pj -= P;
             const int kg = 2 * pj + h;
-            make_digits(x + (size_t)kg * 128, col_scale ? col_scale + (size_t)kg * 128 : nullptr,
-                        dig_u32 + (uint32_t)js * kDigitPairBytes, gsum_u32 + (uint32_t)(js * 2 + h) * (kDigits * 4),
-                        gfac_u32 + (uint32_t)(js * 2 + h) * 4u, h, lane);
+            make_digits<SUB>(x + (size_t)kg * 128, col_scale ? col_scale + (size_t)kg * 128 : nullptr,
+                             dig_u32 + (uint32_t)js * kDigitPairBytes,
+                             gsum_u32 + (uint32_t)(js * 2 + h) * (SUB * kDigits * 4), gfac_u32 + (uint32_t)(js * 2 + h) * 4u,
+                             h, lane);
         }
         named_bar_sync(1, kC * 32);
 
@@ -480,11 +504,18 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         const uint32_t sz_lane = szr_u32 + (uint32_t)r0 * 16u;
         const uint32_t b_lane = dig_u32 + (uint32_t)(tq * (kDigits * 16) + gq * 16);
         const uint32_t s_lane = gsum_u32 + (uint32_t)(2 * tq) * 4u;
+        // groups of 32 or 64: lane tq's codes of a 128-input block are group lsub of it; its B column gq is
+        // non-zero only for that group's inputs (group gq / 2 or gq / 4 of the block), so the MMA's column sums
+        // stay per group, and its accumulator columns 2 tq, 2 tq + 1 are digits of its own group
+        const int lsub = SUB == 4 ? tq : SUB == 2 ? (tq >> 1) : 0;
+        const bool bown = SUB == 4 ? (gq >> 1) == tq : SUB == 2 ? (gq >> 2) == (tq >> 1) : false;
+        const uint32_t b_lane_g = dig_u32 + (uint32_t)(tq * (kDigits * 16) + (SUB == 4 ? (gq & 1) : (gq & 3)) * 16);
+        float accg[2] = {0.0f, 0.0f};  // groups of 32 or 64: [row r0, r0 + 8], digit weights applied
         // A wait that runs out sets the abort flag and every later wait returns at once: the loop then runs
         // to its end on garbage, with the same control flow in every warp, so the barriers below still meet.
         for (int i = 0; i < n; ++i) {
             // ---- s/z window ----
-            if (i == 0 || (p & (kPairsPerWindow - 1)) == 0) {
+            if (i == 0 || (p & (UPW - 1)) == 0) {
                 if (win >= 0) {  // the previous window is consumed
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&szempty[win & 1]);
@@ -500,25 +531,39 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int a = 0; a < 2; ++a) wv[h][a] = lds128(wsrc + (uint32_t)h * (kTile * 64u) + (uint32_t)a * 8u * 64u);
-            const int kg = 2 * p;
-            const uint32_t szsrc = sz_lane + (uint32_t)(win & 1) * 2u * kSzBytes + (uint32_t)(kg & 7) * 2u;
-            // s and z of groups kg, kg + 1 are adjacent in the window box (kg is even): one 32-bit load per row
-            // and array
-            float sv[2][2], zv[2][2];
+            float sv[2][2], zv[2][2];  // [block h][row r0, r0 + 8]: the (lane's) group's s and z
+            if constexpr (SUB == 1) {
+                const int kg = 2 * p;
+                const uint32_t szsrc = sz_lane + (uint32_t)(win & 1) * 2u * kSzBytes + (uint32_t)(kg & 7) * 2u;
+                // s and z of groups kg, kg + 1 are adjacent in the window box (kg is even): one 32-bit load per
+                // row and array
 #pragma unroll
-            for (int a = 0; a < 2; ++a) {
-                const uint32_t o = szsrc + (uint32_t)a * 8u * 16u;
-                const uint32_t s2 = lds_u32(o), z2 = lds_u32(o + kSzBytes);
-                sv[0][a] = __uint_as_float(s2 << 16);
-                sv[1][a] = __uint_as_float(s2 & 0xffff0000u);
-                zv[0][a] = __uint_as_float(z2 << 16);
-                zv[1][a] = __uint_as_float(z2 & 0xffff0000u);
+                for (int a = 0; a < 2; ++a) {
+                    const uint32_t o = szsrc + (uint32_t)a * 8u * 16u;
+                    const uint32_t s2 = lds_u32(o), z2 = lds_u32(o + kSzBytes);
+                    sv[0][a] = __uint_as_float(s2 << 16);
+                    sv[1][a] = __uint_as_float(s2 & 0xffff0000u);
+                    zv[0][a] = __uint_as_float(z2 << 16);
+                    zv[1][a] = __uint_as_float(z2 & 0xffff0000u);
+                }
+            } else {
+                const int g0 = 2 * SUB * p;  // the unit's first group
+                const uint32_t szw = sz_lane + (uint32_t)(win & 1) * 2u * kSzBytes;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int a = 0; a < 2; ++a) {
+                        const uint32_t o = szw + (uint32_t)a * 8u * 16u + (uint32_t)((g0 + h * SUB + lsub) & 7) * 2u;
+                        sv[h][a] = __uint_as_float((uint32_t)lds_u16(o) << 16);
+                        zv[h][a] = __uint_as_float((uint32_t)lds_u16(o + kSzBytes) << 16);
+                    }
             }
             // the stage's weight bytes are in registers: hand the slot back to the producer
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
             if (++s == STAGES) { s = 0; ph ^= 1u; w_off = 0; } else { w_off += kStageBytes; }
             const uint32_t bsrc = b_lane + (uint32_t)di * kDigitPairBytes;
+            if constexpr (SUB == 1) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 // digit column gq of this lane's 8 inputs of each k32 step: steps 0, 1 then 2, 3
@@ -546,6 +591,40 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     acc[a][1] = fmaf(sF, d1, acc[a][1]);
                 }
             }
+            } else {
+            const uint32_t bsrc_g = b_lane_g + (uint32_t)di * kDigitPairBytes;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float F = lds_f32(gfac_u32 + (uint32_t)(di * 2 + h) * 4u);
+                // groups of 32: two passes, digits 0, 1 then 2, 3 of each group; groups of 64: one pass, digits
+                // 2 (tq % 2), + 1 of the lane's group in its accumulator columns
+#pragma unroll
+                for (int pass = 0; pass < (SUB == 4 ? 2 : 1); ++pass) {
+                    uint4 Bv[2];
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf)
+                        Bv[hf] = bown ? lds128(bsrc_g + (uint32_t)((h * 2 + hf) * 4) * (kDigits * 16) + (uint32_t)pass * 32u)
+                                      : make_uint4(0u, 0u, 0u, 0u);
+                    uint32_t C[4];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const uint32_t va = word_of(wv[h][0], w), vb = word_of(wv[h][1], w);
+                        const uint32_t b0 = word_of(Bv[w >> 1], (w & 1) * 2), b1 = word_of(Bv[w >> 1], (w & 1) * 2 + 1);
+                        mma_u8s8(C, w == 0 ? cmag : C, va & 0x0F0F0F0Fu, vb & 0x0F0F0F0Fu, (va >> 4) & 0x0F0F0F0Fu,
+                                 (vb >> 4) & 0x0F0F0F0Fu, b0, b1);
+                    }
+                    const int d0i = SUB == 4 ? 2 * pass : 2 * (tq & 1);  // the digits in columns 2 tq, 2 tq + 1
+                    const float2 S = lds_f2(gsum_u32 + (uint32_t)(((di * 2 + h) * SUB + lsub) * kDigits + d0i) * 4u);
+                    const float w0 = exp2i(-7 * d0i), w1 = exp2i(-7 * d0i - 7);
+#pragma unroll
+                    for (int a = 0; a < 2; ++a) {
+                        const float d0 = fmaf(-zv[h][a], S.x, __uint_as_float(C[2 * a]) - kMagic);
+                        const float d1 = fmaf(-zv[h][a], S.y, __uint_as_float(C[2 * a + 1]) - kMagic);
+                        accg[a] = fmaf(sv[h][a] * F, fmaf(d1, w1, d0 * w0), accg[a]);
+                    }
+                }
+            }
+            }
             if (++di == P) di = 0;
             // ---- end of a segment: the tile's last pair, or the end of this CTA's range ----
             const bool tile_done = (p + 1 == P);
@@ -554,7 +633,8 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 float rs[2];
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
-                    float v = fmaf(acc[a][1], cw1, acc[a][0] * cw0);
+                    float v = SUB == 1 ? fmaf(acc[a][1], cw1, acc[a][0] * cw0) : accg[a];
+                    accg[a] = 0.0f;
                     v += __shfl_xor_sync(0xffffffffu, v, 1);
                     v += __shfl_xor_sync(0xffffffffu, v, 2);
                     rs[a] = v;
@@ -593,7 +673,7 @@ struct M1Config {
     size_t smem;
 };
 
-M1Config m1_config(int64_t N, int64_t K)
+M1Config m1_config(int64_t N, int64_t K, int g)
 {
     static std::mutex mu;
     static std::map<int, std::pair<int, int>> dev_of;  // SMs, opt-in shared memory per block
@@ -607,8 +687,9 @@ M1Config m1_config(int64_t N, int64_t K)
             int v = 148, o = 0;
             cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
             cudaDeviceGetAttribute(&o, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-            cudaFuncSetAttribute(gemv_w4a16_m1_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, o);
-            cudaFuncSetAttribute(gemv_w4a16_m1_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, o);
+#define WQ_M1_ATTR(G_, S_) cudaFuncSetAttribute(gemv_w4a16_m1_kernel<G_, S_>, cudaFuncAttributeMaxDynamicSharedMemorySize, o)
+            WQ_M1_ATTR(128, 3); WQ_M1_ATTR(128, 2); WQ_M1_ATTR(64, 3); WQ_M1_ATTR(64, 2); WQ_M1_ATTR(32, 3); WQ_M1_ATTR(32, 2);
+#undef WQ_M1_ATTR
             it = dev_of.emplace(dev, std::make_pair(v, o)).first;
         }
         sms = it->second.first;
@@ -620,8 +701,9 @@ M1Config m1_config(int64_t N, int64_t K)
     c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(units, sms));
     const int64_t per = (units + c.grid - 1) / c.grid;  // most units any CTA takes
     c.npairs = (int)std::min<int64_t>(per, P);
-    c.stages = M1Layout(3, c.npairs).total <= (size_t)optin ? 3 : 2;
-    c.smem = M1Layout(c.stages, c.npairs).total;
+    const int sub = 128 / g;
+    c.stages = M1Layout(3, c.npairs, sub).total <= (size_t)optin ? 3 : 2;
+    c.smem = M1Layout(c.stages, c.npairs, sub).total;
     return c;
 }
 
@@ -644,20 +726,24 @@ size_t m1_slots_bytes(int64_t N, int64_t K, int grid)
 
 bool gemv_m1_eligible(int64_t M, int64_t N, int64_t K, int g)
 {
-    // K % 1024: the s/z row stride (K / 128 bf16) must be a multiple of 16 bytes for their tensor maps;
-    // K <= 32768: the digit planes of a CTA's group pairs and two stages fit in shared memory
-    return M == 1 && g == 128 && K >= 1024 && K % 1024 == 0 && K <= 32768 && N >= 1 && N <= 0x7fffffffLL;
+    // groups of 32, 64 or 128; K % 1024: the s/z row stride (K / g bf16) must be a multiple of 16 bytes for
+    // their tensor maps; two stages and the digit planes and sums of every group pair of a tile must fit in the
+    // 227 KB of shared memory a block can have (K <= 32768 for groups of 64 and 128, K <= 31744 for 32)
+    if (M != 1 || !(g == 128 || g == 64 || g == 32) || K < 1024 || K % 1024 != 0 || K > 32768 || N < 1 ||
+        N > 0x7fffffffLL)
+        return false;
+    return M1Layout(2, (int)(K / 256), 128 / g).total <= (size_t)232448;
 }
 
 size_t gemv_m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
 {
     if (!gemv_m1_eligible(M, N, K, g)) return 0;
     const int64_t ntiles = (N + kTile - 1) / kTile;
-    return m1_slots_bytes(N, K, m1_config(N, K).grid) + ((size_t)ntiles * 4 + 255) / 256 * 256;
+    return m1_slots_bytes(N, K, m1_config(N, K, g).grid) + ((size_t)ntiles * 4 + 255) / 256 * 256;
 }
 
 int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
-                         const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st,
+                         const uint16_t *z, int g, uint16_t *y, void *workspace, int *status, cudaStream_t st,
                          const float *col_scale)
 {
     // packed codes seen as (64-byte group slice, row, group): strides K/2 bytes (row) and 64 bytes (group)
@@ -680,12 +766,13 @@ int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t 
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return -1;
-    if (!encode_tmap_2d(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, s, G, (uint64_t)N, G * 2, 8, kTile,
+    const uint64_t Gs = (uint64_t)K / (uint64_t)g;  // s and z: one per group of g
+    if (!encode_tmap_2d(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, s, Gs, (uint64_t)N, Gs * 2, 8, kTile,
                         CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_tmap_2d(&zmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, z, G, (uint64_t)N, G * 2, 8, kTile,
+        !encode_tmap_2d(&zmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, z, Gs, (uint64_t)N, Gs * 2, 8, kTile,
                         CU_TENSOR_MAP_SWIZZLE_NONE))
         return -1;
-    const M1Config c = m1_config(N, K);
+    const M1Config c = m1_config(N, K, g);
     const int grid = c.grid;
     const int max_segs = m1_max_segments(N, K, grid);
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
@@ -704,11 +791,16 @@ int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     // three stages in flight measured the same as four on the 70B-shaped linears
-    const cudaError_t e =
-        c.stages == 3 ? cudaLaunchKernelEx(&cfg, gemv_w4a16_m1_kernel<3>, wmap, smap, zmap, x, (int)N, (int)K, y, ws, cnt,
-                                           max_segs, status, c.npairs, col_scale)
-                      : cudaLaunchKernelEx(&cfg, gemv_w4a16_m1_kernel<2>, wmap, smap, zmap, x, (int)N, (int)K, y, ws, cnt,
-                                           max_segs, status, c.npairs, col_scale);
+    cudaError_t e = cudaErrorInvalidValue;
+#define WQ_M1_LAUNCH(G_)                                                                                           \
+    e = c.stages == 3 ? cudaLaunchKernelEx(&cfg, gemv_w4a16_m1_kernel<G_, 3>, wmap, smap, zmap, x, (int)N, (int)K, y, \
+                                           ws, cnt, max_segs, status, c.npairs, col_scale)                            \
+                      : cudaLaunchKernelEx(&cfg, gemv_w4a16_m1_kernel<G_, 2>, wmap, smap, zmap, x, (int)N, (int)K, y, \
+                                           ws, cnt, max_segs, status, c.npairs, col_scale)
+    if (g == 128) WQ_M1_LAUNCH(128);
+    else if (g == 64) WQ_M1_LAUNCH(64);
+    else WQ_M1_LAUNCH(32);
+#undef WQ_M1_LAUNCH
     if (e != cudaSuccess) return -2;
     return 0;
 }

@@ -38,7 +38,7 @@ bool gemv_m1_eligible(int64_t M, int64_t N, int64_t K, int g);
 size_t gemv_m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
 // col_scale (optional, binary32 [K]): the kernel stages bf16(x / col_scale) instead of x.
 int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
-                         const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st,
+                         const uint16_t *z, int g, uint16_t *y, void *workspace, int *status, cudaStream_t st,
                          const float *col_scale = nullptr);
 
 // W4A16 for group 128 and M = 2 on integer products (wq_gemv_i4mt.cu): the M = 1 kernel with 2 rows x 4 digits

@@ -174,12 +174,12 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  *   qweight, scales, zeros: as produced by wq_quantize_int4 with group g
  *   y       [M][N] bf16, y[m][n] = sum_k x[m][k] * s[n][k/g] * (q[n][k] - z[n][k/g])
  *
- * Arithmetic: the M = 1 kernel writes x, per group of 128, as 4 planes of
- * radix-128 integer digits (x_k = 2^(E-5) * sum_c d_ck * 128^-c, |d| <= 64,
- * 2^E <= max |x| of the group: exact for every |x_k| >= 2^(E-19), others
+ * Arithmetic: the M = 1 kernel writes x, per block of 128 inputs, as 4 planes
+ * of radix-128 integer digits (x_k = 2^(E-5) * sum_c d_ck * 128^-c, |d| <= 64,
+ * 2^E <= max |x| of the block: exact for every |x_k| >= 2^(E-19), others
  * rounded to a multiple of 2^(E-26)), takes the exact integer sums
- * sum_k q_k d_ck on the tensor core and applies s * (D_c - z * sum_k d_ck)
- * per group in binary32.  Every other kernel forms the exact integers (q - z)
+ * sum_k q_k d_ck of each group on the tensor core and applies
+ * s * (D_c - z * sum_k d_ck) per group in binary32.  Every other kernel forms the exact integers (q - z)
  * in bf16 (a code pair 128 + q minus the pair 128 + z), multiplies them by x
  * with binary32 accumulation (tensor cores for the decode and batched
  * kernels), applies s per group in binary32.  y is rounded to bf16 once.
@@ -195,8 +195,9 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * calls give identical bytes, except on the older 2 <= M <= 16 kernel (the
  * shapes below that the persistent one does not take), whose partials meet in
  * binary32 atomics (the last bits of y may then vary between calls).
- * Kernels: M = 1 with g = 128, 1024 <= K <= 32768, K % 1024 == 0: persistent
- * TMA-fed kernel on integer products (exact digits of x, see below);
+ * Kernels: M = 1 with 1024 <= K <= 32768, K % 1024 == 0 (K <= 31744 for
+ * g = 32): persistent TMA-fed kernel on integer products (exact digits of x,
+ * above; groups of 32 and 64 keep their digit sums in separate MMA columns);
  * 2 <= M <= 16 with g = 128 and the same K: the persistent TMA-fed kernel
  * with the M rows as the MMA's columns (at M = 2 on the integer products of
  * the M = 1 kernel), when the activations of a CTA's share fit shared

@@ -39,7 +39,8 @@ def _no_device_timeouts():
 
 
 @pytest.mark.parametrize("M,N,K,g", [(1, 14336, 4096, 128), (8, 2048, 4096, 128), (128, 1024, 8192, 128),
-                                     (1, 300, 512, 64), (40, 256, 1024, 32)])
+                                     (1, 300, 512, 64), (40, 256, 1024, 32), (1, 3000, 2048, 32),
+                                     (1, 2048, 4096, 64)])
 def test_gemm_w4a16_colscaled(M, N, K, g):
     w = wq_inputs.llm_weight(N, K, 300 + M, dtype=torch.bfloat16)
     x = wq_inputs.activations(M, K, 301 + M)
@@ -58,18 +59,19 @@ def test_gemm_w4a16_colscaled(M, N, K, g):
     assert not bad.any(), f"{bad.sum()} outputs outside the bound; max ratio {np.max(err / a_ref):.3e}"
 
 
-def test_colscaled_m1_matches_prescaled_activations():
+@pytest.mark.parametrize("g", [128, 32])
+def test_colscaled_m1_matches_prescaled_activations(g):
     """At M = 1 the decode kernel divides x while staging it; the result must equal, bit for bit, the plain
     matmul of bf16(x / s) computed by the pre-pass used at other shapes."""
     N, K = 8192, 8192
     w = wq_inputs.llm_weight(N, K, 310, dtype=torch.bfloat16).cuda()
     s = wq_inputs.channel_scales(K, 311).cuda()
-    q, sc, z = wq.wq_quantize_int4_scaled(w, s, 128)
+    q, sc, z = wq.wq_quantize_int4_scaled(w, s, g)
     x = wq_inputs.activations(2, K, 312).cuda()
-    y1 = wq.wq_gemm_w4a16_colscaled(x[:1], s, q, sc, z, 128)   # fused (M = 1 kernel)
-    y2 = wq.wq_gemm_w4a16_colscaled(x, s, q, sc, z, 128)       # pre-pass, then the M = 2 kernel
+    y1 = wq.wq_gemm_w4a16_colscaled(x[:1], s, q, sc, z, g)     # fused (M = 1 kernel)
+    y2 = wq.wq_gemm_w4a16_colscaled(x, s, q, sc, z, g)         # pre-pass, then an M = 2 kernel
     xs = (x[:1].float() / s[None, :]).to(torch.bfloat16)        # torch's IEEE binary32 quotient, RNE to bf16
-    y3 = wq.wq_gemm_w4a16(xs, q, sc, z, 128)                    # plain M = 1 kernel on pre-scaled x
+    y3 = wq.wq_gemm_w4a16(xs, q, sc, z, g)                      # plain M = 1 kernel on pre-scaled x
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y3.view(torch.int16))
     assert np.allclose(y1.float().cpu().numpy(), y2[:1].float().cpu().numpy(), rtol=1e-2, atol=1e-3)

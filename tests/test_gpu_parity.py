@@ -386,6 +386,37 @@ def test_gemm_w4a16_m1_stream_k_edges(N, K):
     _w4_case(N, K, 128, 1, 11 * N + K)
 
 
+@pytest.mark.parametrize("g", [32, 64])
+@pytest.mark.parametrize("N,K", [(1, 1024), (33, 1024), (31, 3072), (4097, 2048), (3000, 4096), (65536, 1024),
+                                 (40000, 2048), (64, 31744), (64, 32768)])
+def test_gemm_w4a16_m1_small_groups(N, K, g):
+    """M = 1 with groups of 32 and 64 on the decode kernel: each 128-input block holds 4 or 2 groups, whose
+    digit sums the MMA keeps in separate columns; ragged row blocks, tiles split over CTAs, CTAs with whole
+    tiles between split ones, the longest K each group size takes (groups of 32 at K = 32768 do not fit
+    shared memory and go to the CUDA-core kernel)."""
+    _w4_case(N, K, g, 1, 19 * N + K + g)
+
+
+@pytest.mark.parametrize("g", [32, 64])
+def test_gemm_w4a16_m1_small_groups_exact_zeros_far_zero_points_nonfinite(g):
+    """Groups of 32 and 64 at M = 1: all-zero rows and a single all-zero group give exactly 0 under
+    activations spanning many binades; zero-points far outside [0, 15] with one-signed activations meet the
+    bound; an infinite activation makes every output non-finite."""
+    N, K = 640, 2048
+    w = wq_inputs.llm_weight(N, K, 191, dtype=torch.float32)
+    w[::5] = 0.0
+    w[3, 256:256 + g] = 0.0
+    _w4_case(N, K, g, 1, 0, wgen=w, xgen=wq_inputs.wide_range_activations(1, K, 192 + g))
+    _w4_case(N, K, g, 1, 0, wgen=wq_inputs.offset_group_weight(N, K, 193, group=g),
+             xgen=wq_inputs.positive_activations(1, K, 194 + g))
+    x = wq_inputs.activations(1, K, 195)
+    x[:, 300] = float("inf")
+    q, s, z = wq.wq_quantize_int4(w.cuda(), g)
+    y = wq.wq_gemm_w4a16(x.cuda(), q, s, z, g)
+    torch.cuda.synchronize()
+    assert not torch.isfinite(y.float()).any()
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 3000, 4096), (2, 3000, 4096), (8, 3000, 4096), (16, 1000, 8192),
                                    (128, 256, 16384), (40, 384, 8192)])
 def test_gemm_w4a16_workspace_reuse_deterministic(M, N, K):
@@ -468,8 +499,9 @@ def test_gemm_w4a16_far_zero_points(M):
 
 @pytest.mark.parametrize("g,M,K", [(32, 1, 1024), (64, 4, 1024), (128, 1, 1152), (32, 40, 1024), (64, 64, 1024)])
 def test_gemm_w4a16_far_zero_points_other_kernels(g, M, K):
-    """The same for the CUDA-core kernel (groups of 32 and 64, and K that the TMA kernels do not take) and
-    the tensor-core kernel with several groups per stage."""
+    """The same for the decode kernel with groups of 32, the small-batch CUDA-core kernel (groups of 64), the
+    M = 1 CUDA-core kernel (K that the TMA kernels do not take) and the tensor-core kernel with several groups
+    per stage."""
     N = 384
     w = wq_inputs.offset_group_weight(N, K, 95 + g, group=g)
     x = wq_inputs.positive_activations(M, K, 96 + M)
