@@ -676,8 +676,16 @@ size_t gemm_tc_partials_bytes(int64_t M, int64_t N, int64_t K, int BN)
 bool gemm_tc_eligible(int64_t M, int64_t N, int64_t K, int g)
 {
     // M > 16; also 2 <= M <= 16 for groups of 32 and 64, which the TMA decode kernel does not take (the
-    // tensor cores still beat the CUDA-core kernel there: it spends one FMA per code and row of x)
-    const bool m_ok = M > 16 || (M >= 2 && (g == 32 || g == 64));
+    // tensor cores still beat the CUDA-core kernel there: it spends one FMA per code and row of x); and
+    // 9 <= M <= 16 with g = 128 and K % 1024 == 0 (the 128 x 128-tile kernel), except up to 12 rows where the
+    // persistent small-batch kernel runs with three weight stages.  Measured on B200 (K = 8192, N = 28672):
+    // the 128 x 128-tile kernel takes 70 us at any M from 8 to 16; the small-batch kernels 43.8 us at M = 8
+    // but 99-101 us at M = 12 and 16 (two column tiles of 8, and two stages or the older TMA kernel where the
+    // activations take the room); on K = N = 8192 (three stages) the persistent one is ahead at M = 12 (29.1
+    // against 31.4 us) and behind at M = 16 (33.9 against 31.3 us).
+    const bool tc_small_batch =
+        g == 128 && K % 1024 == 0 && M >= 9 && M <= 16 && !(M <= 12 && gemv_mt_stages(M, N, K, g) == 3);
+    const bool m_ok = M > 16 || (M >= 2 && (g == 32 || g == 64)) || tc_small_batch;
     return m_ok && N >= kTileN && K >= kStageK && K % kStageK == 0 && (g == 32 || g == 64 || g == 128) &&
            K / 2 <= 0xffffffffLL && M <= 0x7fffffffLL;
 }

@@ -608,6 +608,11 @@ bool gemv_mt_eligible(int64_t M, int64_t N, int64_t K, int g)
     return mt_config(M, N, K).stages != 0;
 }
 
+int gemv_mt_stages(int64_t M, int64_t N, int64_t K, int g)
+{
+    return gemv_mt_eligible(M, N, K, g) ? mt_config(M, N, K).stages : 0;
+}
+
 size_t gemv_mt_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
 {
     if (!gemv_mt_eligible(M, N, K, g)) return 0;

@@ -58,6 +58,7 @@ int launch_gemv_w4a16_i4mt(const uint16_t *x, int64_t M, int64_t N, int64_t K, c
 // gemv_mt_workspace_bytes() (zero-filled before first use; the kernel leaves its counters zeroed); the device
 // status word for its bounded waits.  Returns 0, -1 if a tensor map cannot be encoded, -2 if the launch fails.
 bool gemv_mt_eligible(int64_t M, int64_t N, int64_t K, int g);
+int gemv_mt_stages(int64_t M, int64_t N, int64_t K, int g);  // weight stages in flight; 0 when not eligible
 size_t gemv_mt_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
 int launch_gemv_w4a16_mt(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
                          const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st);

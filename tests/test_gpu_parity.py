@@ -422,8 +422,8 @@ def test_gemm_w4a16_m1_small_groups_exact_zeros_far_zero_points_nonfinite(g):
 def test_gemm_w4a16_workspace_reuse_deterministic(M, N, K):
     """Calls that share one workspace find it ready (its counters re-zeroed by the previous call) and the
     split-K combine runs in a fixed order: the same inputs give the same bytes every time.  M = 1 runs the
-    persistent decode kernel, M = 8 and 16 its small-batch form, M = 40 and 128 the tensor-core kernel with
-    K split over many CTAs per tile."""
+    persistent decode kernel, M = 2 and 8 its small-batch forms, M = 16, 40 and 128 the tensor-core kernel
+    with K split over many CTAs per tile."""
     w = wq_inputs.llm_weight(N, K, 77)
     q, s, z = wq.wq_quantize_int4(w.cuda(), 128)
     ws = torch.zeros(wq.wq_gemm_workspace_bytes(M, N, K, 128, 4) + 16, dtype=torch.uint8, device="cuda")
@@ -446,10 +446,19 @@ def test_gemm_w4a16_small_batch_persistent(M, N, K):
     _w4_case(N, K, 128, M, 13 * N + K + M)
 
 
+@pytest.mark.parametrize("M,N,K", [(13, 1000, 8192), (16, 4097, 2048), (9, 2000, 28672), (12, 3000, 4096),
+                                   (16, 128, 1024), (14, 300, 32768)])
+def test_gemm_w4a16_small_batch_on_tensor_cores(M, N, K):
+    """9 to 16 rows, g = 128, K % 1024 = 0: the 128 x 128-tile tensor-core kernel takes the shapes where the
+    persistent small-batch kernel would run with fewer than three stages or more than 12 rows; its tile holds
+    the M rows and zeros (the activation copies fill rows past M)."""
+    _w4_case(N, K, 128, M, 23 * M + N + K)
+
+
 @pytest.mark.parametrize("M", [8, 16])
 def test_gemm_w4a16_small_batch_large_shape(M):
     """The gate+up shape at M = 8 (the persistent kernel with two weight stages, its activations filling
-    shared memory) and M = 16 (too many activations for it: the older TMA kernel); rows sampled."""
+    shared memory) and M = 16 (too many activations for it: the tensor-core kernel); rows sampled."""
     N, K = 57344, 8192
     w = wq_inputs.llm_weight(N, K, 333)
     rows = np.r_[0:64, 20000:20064, N - 64:N]
@@ -537,7 +546,7 @@ def test_gemm_w4a16_decode_up_m1():
 
 def test_gemm_w4a16_sweep_sampled():
     w = wq_inputs.llm_weight(28672, 8192, wq_inputs.SEEDS["sweep"])
-    _sampled_w4(28672, 8192, 128, [1, 8, 32, 128], 3, w, sample_rows(28672, 192, 3))
+    _sampled_w4(28672, 8192, 128, [1, 8, 16, 32, 128], 3, w, sample_rows(28672, 192, 3))
 
 
 def test_gemm_w4a16_gran_g32():

@@ -29,6 +29,25 @@ def _m1_needed(N, K):
     return ntiles * max_seg * 256 * 4 + ntiles * 4
 
 
+def _mt_stages(M, N, K):
+    """Weight stages of the persistent small-batch kernel (2 <= M <= 16, g = 128) as the library decides it
+    for a B200: 3 or 2 when the CTA's activation pairs fit shared memory beside them, else 0."""
+    P = K // 256
+    units = math.ceil(N / 256) * P
+    npairs = min(-(-units // min(units, SMS)), P)
+
+    def total(stages):
+        return stages * 32768 + 16384 + 2 * M * 256 * 4 + npairs * 2 * M * 256 + 16 * 8 + 1024
+
+    return 3 if total(3) <= 232448 else 2 if total(2) <= 232448 else 0
+
+
+def _tc_takes_small_batch(M, N, K):
+    """9 <= M <= 16, g = 128, K % 1024 == 0, N >= 128: the 128 x 128-tile tensor-core kernel, unless M <= 12 and
+    the persistent small-batch kernel runs with three stages."""
+    return 9 <= M <= 16 and N >= 128 and K % 1024 == 0 and not (M <= 12 and _mt_stages(M, N, K) == 3)
+
+
 def _mt_needed(M, N, K):
     """2 <= M <= 16, g = 128: the persistent kernel's [segment][m][256] slots when the CTA's activation pairs
     fit shared memory (as the library decides it for a B200), else the older kernel's M x N binary32 buffer."""
@@ -36,12 +55,7 @@ def _mt_needed(M, N, K):
     ntiles = math.ceil(N / 256)
     units = ntiles * P
     B = min(units, SMS)
-    npairs = min(-(-units // B), P)
-
-    def total(stages):
-        return stages * 32768 + 16384 + 2 * M * 256 * 4 + npairs * 2 * M * 256 + 16 * 8 + 1024
-
-    if total(3) > 232448 and total(2) > 232448:
+    if _mt_stages(M, N, K) == 0:
         return M * N * 4
     cta_of = lambda u: ((u + 1) * B - 1) // units  # noqa: E731
     max_seg = max(cta_of(t * P + P - 1) - cta_of(t * P) + 1 for t in range(ntiles))
@@ -89,9 +103,13 @@ def test_tc_workspace_covers_every_segment(M, N, K, g):
 
 @pytest.mark.parametrize("M,N,K", [(2, 1, 1024), (3, 4097, 2048), (8, 28672, 8192), (8, 57344, 8192),
                                    (8, 8192, 28672), (16, 10240, 8192), (16, 57344, 8192), (5, 300000, 1024),
-                                   (9, 33, 32768), (16, 256 * 149 + 1, 2048)])
+                                   (9, 33, 32768), (16, 256 * 149 + 1, 2048), (12, 10240, 8192), (12, 8192, 28672),
+                                   (9, 57344, 8192), (13, 8192, 8192), (16, 100, 8192)])
 def test_mt_workspace_covers_every_segment(M, N, K):
-    assert wq.wq_gemm_workspace_bytes(M, N, K, 128, 4) >= _mt_needed(M, N, K)
+    """2 <= M <= 16, g = 128: the small-batch kernels' slots, or the tensor-core kernel's where it takes the
+    shape (9 to 16 rows)."""
+    need = _tc_needed(M, N, K, 128) if _tc_takes_small_batch(M, N, K) else _mt_needed(M, N, K)
+    assert wq.wq_gemm_workspace_bytes(M, N, K, 128, 4) >= need
 
 
 def _w8int_needed(M, N, K):
