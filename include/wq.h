@@ -202,8 +202,10 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * with the M rows as the MMA's columns (at M = 2 on the integer products of
  * the M = 1 kernel), when the activations of a CTA's share fit shared
  * memory, else a TMA-fed decode kernel (N >= 128, K >= 256); M > 16,
- * or 2 <= M <= 16 with g = 32 or 64 (N >= 128, K % 128 == 0): tcgen05
- * tensor-core kernels; other shapes: a CUDA-core kernel.
+ * 2 <= M <= 16 with g = 32 or 64, or 9 <= M <= 16 with g = 128 and
+ * K % 1024 == 0 unless M <= 12 and the persistent kernel keeps three weight
+ * stages (N >= 128, K % 128 == 0): tcgen05 tensor-core kernels; other shapes:
+ * a CUDA-core kernel.
  * Requirements: M, N >= 1; K % 32 == 0; g in {32, 64, 128}, K % g == 0;
  * pointers 16-byte aligned; workspace of wq_gemm_workspace_bytes(M, N, K, g, 4)
  * bytes (may be NULL when that is 0).  y must not overlap x, qweight,
