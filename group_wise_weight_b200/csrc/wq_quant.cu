@@ -551,66 +551,128 @@ __device__ __forceinline__ float int4_sym_scale(float amax)
     return s == 0.0f ? 1.0f : s;
 }
 
-__device__ __forceinline__ uint32_t int4_sym_encode8(const float v[8], float s, float amax)
-{
-    float qd[8];  // RN(w / s)
-    if (quotients_by_reciprocal(s, amax)) {
-        const float r = __frcp_rn(s);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) qd[i] = quotient_rn(v[i], s, r);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) qd[i] = __fdiv_rn(v[i], s);
-    }
-    // rint_bits leaves q (two's complement) in the low bits: the shifted patterns summed, minus their
-    // offsets, plus 8 in every nibble, are the eight nibbles q + 8 (each in 1..15, so nothing carries)
-    uint32_t packed = 0x88888888u - kRintBase * 0x11111111u;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) packed += rint_bits(fminf(fmaxf(qd[i], -7.0f), 7.0f)) << (4 * i);
-    return packed;
-}
-
-template <typename T, int LPG>
+// The layout of quant_int4_kernel: a lane takes 32 consecutive weights of a row, a group of G spans G / 32
+// lanes, the scale is formed once per 32 weights; for bf16 weights the absolute maximum is reduced as a
+// packed bf16 pair and, on the reciprocal path, two quotients are formed per instruction.
+template <typename T, int G>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_int4_sym_kernel(const T *__restrict__ w, int64_t N, int64_t K, int64_t ldw, uint8_t *__restrict__ qweight,
                       uint16_t *__restrict__ scales, uint16_t *__restrict__ zeros)
 {
-    constexpr int g = LPG * 8;
+    constexpr int LPG = G / kLaneWeights;  // lanes per group
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int64_t chunks = (K + 255) >> 8;
+    const int64_t chunks = (K + kWarpWeights - 1) / kWarpWeights;
     const int64_t tasks = N * chunks;
-    const int64_t G = K / g;
+    const int64_t Gn = K / G;
 
     TaskWalk walk(warp0, n_warps, chunks);
-    for (int64_t t0 = warp0; t0 < tasks; t0 += n_warps * kQuantUnroll) {
-        float v[kQuantUnroll][8];
-        int64_t n[kQuantUnroll], k0[kQuantUnroll];
-        bool active[kQuantUnroll];
+    for (int64_t t0 = warp0; t0 < tasks; t0 += n_warps * kInt4Unroll) {
+        float v[kInt4Unroll][kBf16 ? 1 : kLaneWeights];  // binary32 input
+        uint4 raw[kInt4Unroll][kWordsPerLane];             // bf16 input: the weights as loaded
+        int64_t n[kInt4Unroll], k0[kInt4Unroll];
+        bool active[kInt4Unroll];
 #pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
+        for (int u = 0; u < kInt4Unroll; ++u) {
             n[u] = walk.n;
-            k0[u] = walk.c * 256 + lane * 8;
+            k0[u] = walk.c * kWarpWeights + lane * kLaneWeights;
             active[u] = (walk.n < N) && (k0[u] < K);
-            if (active[u]) load8<T>(w + n[u] * ldw + k0[u], v[u]);
+            if (kBf16) {
+#pragma unroll
+                for (int j = 0; j < kWordsPerLane; ++j) raw[u][j] = make_uint4(0u, 0u, 0u, 0u);
+                if (active[u]) {
+#pragma unroll
+                    for (int j = 0; j < kWordsPerLane; ++j) raw[u][j] = ld_stream_v4(w + n[u] * ldw + k0[u] + 8 * j);
+                }
+            } else if (active[u]) {
+#pragma unroll
+                for (int j = 0; j < kWordsPerLane; ++j) load8<T>(w + n[u] * ldw + k0[u] + 8 * j, v[u] + 8 * j);
+            }
             walk.step();
         }
 #pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
+        for (int u = 0; u < kInt4Unroll; ++u) {
             if (t0 + u * n_warps >= tasks) break;  // warp-uniform
-            float amax = 0.0f;
-            if (active[u]) {
+            float amax;
+            if (kBf16) {
+                // |w| of both halves (sign bits cleared), the packed maximum over the lane's 32 weights and then
+                // over the group's lanes (inactive lanes hold zeros)
+                uint32_t m2 = 0u;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[u][i]));
+                for (int j = 0; j < kWordsPerLane; ++j)
+                    m2 = bf16x2_max(m2, bf16x2_max(bf16x2_max(raw[u][j].x & 0x7FFF7FFFu, raw[u][j].y & 0x7FFF7FFFu),
+                                                   bf16x2_max(raw[u][j].z & 0x7FFF7FFFu, raw[u][j].w & 0x7FFF7FFFu)));
+#pragma unroll
+                for (int o = 1; o < LPG; o <<= 1) m2 = bf16x2_max(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+                amax = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xffff0000u));
+            } else {
+                amax = 0.0f;
+                if (active[u]) {
+#pragma unroll
+                    for (int i = 0; i < kLaneWeights; ++i) amax = fmaxf(amax, fabsf(v[u][i]));
+                }
+#pragma unroll
+                for (int o = 1; o < LPG; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             }
-#pragma unroll
-            for (int o = 1; o < LPG; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             if (!active[u]) continue;
             const float s = int4_sym_scale(amax);
-            *reinterpret_cast<uint32_t *>(qweight + n[u] * (K >> 1) + (k0[u] >> 1)) = int4_sym_encode8(v[u], s, amax);
+            uint32_t packed[kWordsPerLane];
+            if (quotients_by_reciprocal(s, amax)) {
+                const float r = __frcp_rn(s);
+                if (kBf16) {
+                    // two weights per instruction: the correctly rounded quotients (packed binary32 multiply and
+                    // fused multiply-adds), then + 8 + 1.5 * 2^23 in one addition, which rounds (rint(q + 8) =
+                    // rint(q) + 8: 8 is even); |w / s| < 8 here, so each rounded q + 8 is the low half-word of
+                    // its bit pattern, clipped to [1, 15] (q to [-7, 7]) as two 16-bit integers
+                    const uint64_t r2 = f32x2_bits(r, r), ns2 = f32x2_bits(-s, -s);
+                    const uint64_t m2 = f32x2_bits(0x1.8p23f + 8.0f, 0x1.8p23f + 8.0f);
+#pragma unroll
+                    for (int j = 0; j < kWordsPerLane; ++j) {
+                        uint32_t b[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const uint32_t wd = word_of(raw[u][j], h);
+                            const uint64_t w2 = ((uint64_t)(wd & 0xffff0000u) << 32) | (uint64_t)(wd << 16);
+                            const uint64_t q0 = f32x2_mul(w2, r2);
+                            const uint64_t q = f32x2_fma(f32x2_fma(q0, ns2, w2), r2, q0);
+                            const uint64_t t = f32x2_add(q, m2);
+                            uint32_t p2 = __byte_perm((uint32_t)t, (uint32_t)(t >> 32), 0x5410);
+                            p2 = __vmins2(__vmaxs2(p2, 0x00010001u), 0x000F000Fu);
+                            b[h] = p2 | (p2 >> 12);  // byte 0: q + 8 of the pair's first weight | second << 4
+                        }
+                        packed[j] = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040),
+                                                0x5410);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < kWordsPerLane; ++j) {
+                        // rint_bits leaves q (two's complement) in the low bits: the shifted patterns summed, minus
+                        // their offsets, plus 8 in every nibble, are the eight nibbles q + 8 (1..15, no carries)
+                        uint32_t pw = 0x88888888u - kRintBase * 0x11111111u;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            pw += rint_bits(fminf(fmaxf(quotient_rn(v[u][8 * j + i], s, r), -7.0f), 7.0f)) << (4 * i);
+                        packed[j] = pw;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < kWordsPerLane; ++j) {
+                    uint32_t pw = 0x88888888u - kRintBase * 0x11111111u;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        pw += rint_bits(fminf(fmaxf(__fdiv_rn(lane_weight<kBf16>(v[u], raw[u], 8 * j + i), s), -7.0f),
+                                              7.0f))
+                              << (4 * i);
+                    packed[j] = pw;
+                }
+            }
+            *reinterpret_cast<uint4 *>(qweight + n[u] * (K >> 1) + (k0[u] >> 1)) =
+                make_uint4(packed[0], packed[1], packed[2], packed[3]);
             if ((lane & (LPG - 1)) == 0) {
-                const int64_t gi = n[u] * G + k0[u] / g;
+                const int64_t gi = n[u] * Gn + k0[u] / G;
                 scales[gi] = f32_to_bf16(s);
                 zeros[gi] = 0x4100u;  // 8.0 in bf16
             }
@@ -674,12 +736,12 @@ void dispatch_int4(const void *w, int64_t N, int64_t K, int64_t ldw, int g, uint
     }
 }
 
-template <typename T, int LPG>
+template <typename T, int G>
 void launch_int4_sym(const void *w, int64_t N, int64_t K, int64_t ldw, uint8_t *q, uint16_t *s, uint16_t *z,
                      cudaStream_t st)
 {
-    auto k = quant_int4_sym_kernel<T, LPG>;
-    const int64_t tasks = N * ((K + 255) / 256);
+    auto k = quant_int4_sym_kernel<T, G>;
+    const int64_t tasks = N * ((K + kWarpWeights - 1) / kWarpWeights);
     const int grid = persistent_grid(k, tasks);
     k<<<grid, kQuantThreads, 0, st>>>(static_cast<const T *>(w), N, K, ldw, q, s, z);
 }
@@ -689,9 +751,9 @@ void dispatch_int4_sym(const void *w, int64_t N, int64_t K, int64_t ldw, int g, 
                        uint16_t *z, cudaStream_t st)
 {
     switch (g) {
-    case 32: launch_int4_sym<T, 4>(w, N, K, ldw, q, s, z, st); break;
-    case 64: launch_int4_sym<T, 8>(w, N, K, ldw, q, s, z, st); break;
-    default: launch_int4_sym<T, 16>(w, N, K, ldw, q, s, z, st); break;
+    case 32: launch_int4_sym<T, 32>(w, N, K, ldw, q, s, z, st); break;
+    case 64: launch_int4_sym<T, 64>(w, N, K, ldw, q, s, z, st); break;
+    default: launch_int4_sym<T, 128>(w, N, K, ldw, q, s, z, st); break;
     }
 }
 
