@@ -354,12 +354,16 @@ gemm_lowp_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant
                         float tot[32];
 #pragma unroll
                         for (int c = 0; c < 32; ++c) tot[c] = 0.0f;
+                        // each value read is cleared behind the read: the workspace is left zero, as it was found
+                        // (a later call of another shape may place its arrival counters where these slots are)
                         for (int64_t o = 0; o < nseg; ++o) {
-                            const float *other = p.part + ((tile * p.max_segs + o) * BN) * kTileN;
+                            float *other = p.part + ((tile * p.max_segs + o) * BN) * kTileN;
 #pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                tot[c] += (o == my_seg) ? __uint_as_float(v[c])
-                                                        : __ldcg(other + (int64_t)(c0 + c) * kTileN + r);
+                            for (int c = 0; c < 32; ++c) {
+                                float *pv = other + (int64_t)(c0 + c) * kTileN + r;
+                                tot[c] += (o == my_seg) ? __uint_as_float(v[c]) : __ldcg(pv);
+                                __stcg(pv, 0.0f);
+                            }
                         }
                         if (n < N) {
 #pragma unroll

@@ -557,11 +557,16 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     float tot[kCols];
 #pragma unroll
                     for (int c = 0; c < kCols; ++c) tot[c] = 0.0f;
+                    // each value read is cleared behind the read: the workspace is left zero, as it was found (a
+                    // later call of another shape may place its arrival counters where these slots are)
                     for (int64_t o = 0; o <= cta_last - cta_first; ++o) {
-                        const float *other = ws + ((tile * max_segs + o) * BN) * kTileN;
+                        float *other = ws + ((tile * max_segs + o) * BN) * kTileN;
 #pragma unroll
-                        for (int c = 0; c < kCols; ++c)
-                            tot[c] += (o == my_seg) ? acc[c] : __ldcg(other + (int64_t)(kq * kCols + c) * kTileN + r);
+                        for (int c = 0; c < kCols; ++c) {
+                            float *pv = other + (int64_t)(kq * kCols + c) * kTileN + r;
+                            tot[c] += (o == my_seg) ? acc[c] : __ldcg(pv);
+                            __stcg(pv, 0.0f);
+                        }
                     }
 #pragma unroll
                     for (int c = 0; c < kCols; ++c) acc[c] = tot[c];

@@ -562,10 +562,16 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
 #pragma unroll
                         for (int c = 0; c < 16; ++c) tot[c] = 0.0f;
                         float4 nxt[4];
+                        // each slot value read is cleared behind the read (and this segment's own slot too): the
+                        // workspace is left zero, as it was found (a later call of another shape may place its
+                        // arrival counters where these slots are)
                         auto fetch = [&](int64_t o) {
 #pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                nxt[q] = o == my_seg ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcg(seg_ptr(o, c0 / 4 + q));
+                            for (int q = 0; q < 4; ++q) {
+                                float4 *pq = seg_ptr(o, c0 / 4 + q);
+                                nxt[q] = o == my_seg ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcg(pq);
+                                __stcg(pq, make_float4(0.f, 0.f, 0.f, 0.f));
+                            }
                         };
                         fetch(0);
                         for (int64_t o = 0; o < nseg; ++o) {

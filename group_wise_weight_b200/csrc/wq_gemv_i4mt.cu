@@ -390,6 +390,15 @@ gemv_w4a16_i4mt_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_co
                             if (row + j < N) yr[row + j] = f32_to_bf16(v[j]);
                     }
                 }
+                // leave the slots zero, as the workspace was found: a later call of another shape may place
+                // its arrival counters where these slots are
+                for (int m = 0; m < M; ++m) {
+                    float4 *qz = reinterpret_cast<float4 *>(slots + (size_t)m * kTile + 8 * lane);
+                    for (int o = 0; o < nseg; ++o) {
+                        __stcg(qz + (size_t)o * sstride, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+                        __stcg(qz + (size_t)o * sstride + 1, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+                    }
+                }
                 __syncwarp();
                 if (lane == 0) atomicExch(cnt + tt, 0);
             }

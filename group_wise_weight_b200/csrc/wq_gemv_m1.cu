@@ -61,10 +61,16 @@
 //  * A tile split between CTAs leaves one binary32 partial per segment in the
 //    workspace.  The consumers never wait on global memory for this: each
 //    warp drops its 16 row sums into a double-buffered shared-memory tile and
-//    moves on, and a separate combiner warp copies the tile to the
-//    segment's slot, bumps the tile's arrival counter and, if it is the last
-//    to arrive, sums the slots in segment order, writes y and re-zeroes the
-//    counter -- a fixed order, so results do not depend on timing.
+//    moves on, and a separate combiner warp takes it from there.  The CTA
+//    holding the tile's first segment combines it: that segment is the end of
+//    its range, while the tile's last segment is the start of the next CTA's,
+//    so it is usually among the last to finish.  The other segments write
+//    their slots and bump the tile's arrival counter (a release add, no round
+//    trip); the first segment's combiner keeps its own sums in registers,
+//    waits (bounded) until the counter shows the others, adds their slots in
+//    segment order, clears them, writes y and re-zeroes the counter -- a
+//    fixed order, so results do not depend on timing, and the workspace is
+//    left zero, as it was found.
 //  * Launched with programmatic dependent launch: in a stream of linears the
 //    next kernel's CTAs start as SMs free up, initialise their barriers and
 //    load their first weight stages into shared memory while this one
@@ -178,13 +184,19 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// Device-scope add with acquire-release semantics: orders the writes that happen before it (this thread's,
-// and through the preceding CTA barrier the other consumers') before the add, and later reads after it.
-__device__ __forceinline__ int atom_add_acq_rel(int *p, int v)
+// Device-scope add with release semantics (no value returned): the writes that happen before it (this
+// thread's, and through the preceding warp barrier the other lanes') are visible before the add is.
+__device__ __forceinline__ void red_add_release(int *p, int v)
 {
-    int old;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Device-scope load with acquire semantics: later reads see what was written before the matching release.
+__device__ __forceinline__ int ld_acquire(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 // The CTA whose equal share [units * b / B, units * (b + 1) / B) holds unit u.
@@ -417,19 +429,38 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             const int c_first = cta_of(tt * P, units, B);
             const int nseg = cta_of(tt * P + P - 1, units, B) - c_first + 1;
             float *slots = ws + (size_t)tt * max_segs * kTile;
-            float4 *mine = reinterpret_cast<float4 *>(slots + (bid - c_first) * kTile + 8 * lane);
-            mine[0] = v0;
-            mine[1] = v1;
-            // the release of the add below covers every lane's slot writes (ordered by the warp barrier)
-            __syncwarp();
-            int last = 0;
-            if (lane == 0) last = (atom_add_acq_rel(cnt + tt, 1) + 1 == nseg) ? 1 : 0;
-            last = __shfl_sync(0xffffffffu, last, 0);
-            if (last) {
-                // sum the segments' slots in segment order (independent of which CTA arrived last)
-                float v[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+            if (bid != c_first) {
+                float4 *mine = reinterpret_cast<float4 *>(slots + (bid - c_first) * kTile + 8 * lane);
+                mine[0] = v0;
+                mine[1] = v1;
+                // the release of the add below covers every lane's slot writes (ordered by the warp barrier)
+                __syncwarp();
+                if (lane == 0) red_add_release(cnt + tt, 1);
+                continue;
+            }
+            // the tile's first segment: wait (bounded) for the other nseg - 1 to arrive
+            int arrived = 1;
+            if (lane == 0) {
+                const uint64_t t0 = global_ns();
+                while (ld_acquire(cnt + tt) != nseg - 1) {
+                    if (flags[0] != 0) { arrived = 0; break; }
+                    if (global_ns() - t0 > kWaitLimitNs) {
+                        record_timeout(status);
+                        flags[0] = 1;
+                        arrived = 0;
+                        break;
+                    }
+                }
+            }
+            // the other lanes read the slots after lane 0's acquire (ordered by the warp barrier)
+            if (!__shfl_sync(0xffffffffu, arrived, 0)) break;
+            {
+                // sum the segments in segment order, from 0: this CTA's own (segment 0, in registers), then the
+                // slots of the others
+                float v[8] = {0.0f + v0.x, 0.0f + v0.y, 0.0f + v0.z, 0.0f + v0.w,
+                              0.0f + v1.x, 0.0f + v1.y, 0.0f + v1.z, 0.0f + v1.w};
                 const float4 *q = reinterpret_cast<const float4 *>(slots + 8 * lane);
-                int o = 0;
+                int o = 1;
                 for (; o + 4 <= nseg; o += 4) {
                     float4 a[8];
 #pragma unroll
@@ -460,6 +491,15 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
                         if (row + j < N) y[row + j] = f32_to_bf16(v[j]);
+                }
+                // leave the slots zero, as the workspace was found: a later call of another shape may place
+                // its arrival counters where these slots are
+                {
+                    float4 *qz = reinterpret_cast<float4 *>(slots + 8 * lane);
+                    for (int o = 1; o < nseg; ++o) {  // segment 0's slot is never written
+                        __stcg(qz + (size_t)o * (kTile / 4), make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+                        __stcg(qz + (size_t)o * (kTile / 4) + 1, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) atomicExch(cnt + tt, 0);

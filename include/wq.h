@@ -156,11 +156,13 @@ int wq_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw
  * Bytes of device workspace wq_gemm_w4a16 (wbits = 4) or wq_gemm_w8a16
  * (wbits = 8) needs for this shape; 0 when the chosen kernel needs none.
  * The workspace holds binary32 partial sums of a K-split and per-tile
- * arrival counters; a call that completes normally leaves the counters
- * zeroed, so a workspace must be zero-filled once before its first use and
- * may then be reused by later calls on the same stream.  A call whose kernel
- * gave up on a bounded wait (wq_device_status returns WQ_ERR_DEVICE_TIMEOUT)
- * can leave counters of the tiles it did not finish non-zero: zero-fill the
+ * arrival counters, at offsets that depend on the shape; a call that
+ * completes normally leaves every byte it used zero again (partial sums and
+ * counters alike), so a workspace must be zero-filled once before its first
+ * use and may then be reused by later calls on the same stream, of this or
+ * any other shape and kernel, as long as it is large enough for each.  A call
+ * whose kernel gave up on a bounded wait (wq_device_status returns
+ * WQ_ERR_DEVICE_TIMEOUT) can leave non-zero bytes behind: zero-fill the
  * workspace again before reusing it after such a status.
  */
 size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits);
