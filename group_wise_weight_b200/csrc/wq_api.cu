@@ -558,16 +558,12 @@ int wq_gemm_w4a16_colscaled(const uint16_t *x, const float *col_scale, int64_t M
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (xb == 0)  // the M = 1 kernel divides x by the scales while it stages x
         return run_w4a16(what, x, M, N, K, qweight, scales, zeros, g, y, workspace, st, col_scale);
-    uint16_t *xs = static_cast<uint16_t *>(workspace);
+    // the matmul's workspace first (its counters at the front, as in every call), the scaled activations after it
+    uint16_t *xs = reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(workspace) + (need - xb));
     wq::launch_colscale_x(x, M, K, col_scale, xs, st);
     rc = check_launch(what);
     if (rc != WQ_OK) return rc;
-    rc = run_w4a16(what, xs, M, N, K, qweight, scales, zeros, g, y, static_cast<uint8_t *>(workspace) + xb, st,
-                   nullptr);
-    if (rc != WQ_OK) return rc;
-    // leave the staging area zero, as the workspace was found: a later call may place its counters there
-    if (cudaMemsetAsync(xs, 0, xb, st) != cudaSuccess) return fail(WQ_ERR_CUDA, "%s: clearing the staging area failed", what);
-    return WQ_OK;
+    return run_w4a16(what, xs, M, N, K, qweight, scales, zeros, g, y, workspace, st, nullptr);
 }
 
 int wq_awq_channel_magnitudes(const uint16_t *x, int64_t M, int64_t K, double *magnitudes, void *stream)

@@ -354,16 +354,12 @@ gemm_lowp_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant
                         float tot[32];
 #pragma unroll
                         for (int c = 0; c < 32; ++c) tot[c] = 0.0f;
-                        // each value read is cleared behind the read: the workspace is left zero, as it was found
-                        // (a later call of another shape may place its arrival counters where these slots are)
                         for (int64_t o = 0; o < nseg; ++o) {
-                            float *other = p.part + ((tile * p.max_segs + o) * BN) * kTileN;
+                            const float *other = p.part + ((tile * p.max_segs + o) * BN) * kTileN;
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) {
-                                float *pv = other + (int64_t)(c0 + c) * kTileN + r;
-                                tot[c] += (o == my_seg) ? __uint_as_float(v[c]) : __ldcg(pv);
-                                __stcg(pv, 0.0f);
-                            }
+                            for (int c = 0; c < 32; ++c)
+                                tot[c] += (o == my_seg) ? __uint_as_float(v[c])
+                                                        : __ldcg(other + (int64_t)(c0 + c) * kTileN + r);
                         }
                         if (n < N) {
 #pragma unroll
@@ -441,7 +437,7 @@ size_t workspace_bytes(int64_t M, int64_t N, int64_t kbytes, int bn)
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const Plan p = plan(M, N, kbytes, bn, sms);
-    return partials_bytes(p, bn) + ((size_t)p.tiles * sizeof(int) + 255) / 256 * 256;
+    return counter_region_bytes(p.tiles) + partials_bytes(p, bn);
 }
 
 template <int BN, int KIND>
@@ -458,8 +454,9 @@ int run(const uint8_t *x, const uint8_t *w, Args a, void *workspace, cudaStream_
     const int sms = sms_of_device();
     const Plan pl = plan(a.M, a.N, kbytes, BN, sms);
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
-    a.part = reinterpret_cast<float *>(w8);
-    a.counters = reinterpret_cast<int *>(w8 + partials_bytes(pl, BN));
+    a.counters = reinterpret_cast<int *>(w8);
+    a.part = reinterpret_cast<float *>(w8 + counter_region_bytes(pl.tiles));
+    if (clear_extra_counters(workspace, pl.tiles, st) != cudaSuccess) return -2;
     a.max_segs = (int)pl.max_segs;
     // at least 120 KB so that one CTA owns each SM (and its tensor memory)
     const size_t smem = std::max<size_t>(Cfg<BN, KIND>::kBytes + 1024, 120 * 1024);

@@ -557,16 +557,11 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     float tot[kCols];
 #pragma unroll
                     for (int c = 0; c < kCols; ++c) tot[c] = 0.0f;
-                    // each value read is cleared behind the read: the workspace is left zero, as it was found (a
-                    // later call of another shape may place its arrival counters where these slots are)
                     for (int64_t o = 0; o <= cta_last - cta_first; ++o) {
-                        float *other = ws + ((tile * max_segs + o) * BN) * kTileN;
+                        const float *other = ws + ((tile * max_segs + o) * BN) * kTileN;
 #pragma unroll
-                        for (int c = 0; c < kCols; ++c) {
-                            float *pv = other + (int64_t)(kq * kCols + c) * kTileN + r;
-                            tot[c] += (o == my_seg) ? acc[c] : __ldcg(pv);
-                            __stcg(pv, 0.0f);
-                        }
+                        for (int c = 0; c < kCols; ++c)
+                            tot[c] += (o == my_seg) ? acc[c] : __ldcg(other + (int64_t)(kq * kCols + c) * kTileN + r);
                     }
 #pragma unroll
                     for (int c = 0; c < kCols; ++c) acc[c] = tot[c];
@@ -633,8 +628,9 @@ int run(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, co
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(total, sms));
     const int max_segs = (int)gemm_tc_max_segments(total, grid, K / kStageK);
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
-    float *ws = reinterpret_cast<float *>(w8);
-    int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, BN));
+    int *counters = reinterpret_cast<int *>(w8);
+    float *ws = reinterpret_cast<float *>(w8 + counter_region_bytes(tiles));
+    if (clear_extra_counters(workspace, tiles, st) != cudaSuccess) return -2;
     kern<<<(unsigned)grid, kThreads, smem, st>>>(wmap, xmap, M, N, K, s, z, y, ws, counters, max_segs, status,
                                                   0x000F000Fu, 0x43004300u, W8 ? -1 : test_take_skip_unit(),
                                                   s_per_row);
@@ -700,7 +696,7 @@ size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
     if (!gemm_tc_eligible(M, N, K, g)) return 0;
     const int BN = gemm_tc_w4_bn(M, K, g);
     const int64_t tiles = ((N + kTileN - 1) / kTileN) * ((M + BN - 1) / BN);
-    return gemm_tc_partials_bytes(M, N, K, BN) + (sizeof(int) * (size_t)tiles + 255) / 256 * 256;
+    return counter_region_bytes(tiles) + gemm_tc_partials_bytes(M, N, K, BN);
 }
 
 int launch_gemm_w4a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
@@ -734,7 +730,7 @@ size_t gemm_tc_w8_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
     const int ge = w8_group(K, g);
     const int BN = gemm_tc_bn(M, ge);
     const int64_t tiles = ((N + kTileN - 1) / kTileN) * ((M + BN - 1) / BN);
-    return gemm_tc_partials_bytes(M, N, K, BN) + (sizeof(int) * (size_t)tiles + 255) / 256 * 256;
+    return counter_region_bytes(tiles) + gemm_tc_partials_bytes(M, N, K, BN);
 }
 
 int launch_gemm_w8a16_tc(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *q8, const uint16_t *s,

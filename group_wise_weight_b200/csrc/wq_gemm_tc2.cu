@@ -562,16 +562,10 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
 #pragma unroll
                         for (int c = 0; c < 16; ++c) tot[c] = 0.0f;
                         float4 nxt[4];
-                        // each slot value read is cleared behind the read (and this segment's own slot too): the
-                        // workspace is left zero, as it was found (a later call of another shape may place its
-                        // arrival counters where these slots are)
                         auto fetch = [&](int64_t o) {
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                float4 *pq = seg_ptr(o, c0 / 4 + q);
-                                nxt[q] = o == my_seg ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcg(pq);
-                                __stcg(pq, make_float4(0.f, 0.f, 0.f, 0.f));
-                            }
+                            for (int q = 0; q < 4; ++q)
+                                nxt[q] = o == my_seg ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcg(seg_ptr(o, c0 / 4 + q));
                         };
                         fetch(0);
                         for (int64_t o = 0; o < nseg; ++o) {
@@ -660,8 +654,9 @@ int launch_gemm_w4a16_tc2(const uint16_t *x, int64_t M, int64_t N, int64_t K, co
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(total, sms));
     const int max_segs = (int)gemm_tc_max_segments(total, grid, K / kStageK);
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
-    float *ws = reinterpret_cast<float *>(w8);
-    int *counters = reinterpret_cast<int *>(w8 + gemm_tc_partials_bytes(M, N, K, kBN));
+    int *counters = reinterpret_cast<int *>(w8);
+    float *ws = reinterpret_cast<float *>(w8 + counter_region_bytes(tiles));
+    if (clear_extra_counters(workspace, tiles, st) != cudaSuccess) return -2;
     // programmatic dependent launch: this grid may start while the previous kernel in the stream finishes;
     // it reads nothing that kernel may write, and writes nothing, before griddepcontrol.wait
     cudaLaunchConfig_t cfg = {};

@@ -390,15 +390,6 @@ gemv_w4a16_i4mt_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_co
                             if (row + j < N) yr[row + j] = f32_to_bf16(v[j]);
                     }
                 }
-                // leave the slots zero, as the workspace was found: a later call of another shape may place
-                // its arrival counters where these slots are
-                for (int m = 0; m < M; ++m) {
-                    float4 *qz = reinterpret_cast<float4 *>(slots + (size_t)m * kTile + 8 * lane);
-                    for (int o = 0; o < nseg; ++o) {
-                        __stcg(qz + (size_t)o * sstride, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
-                        __stcg(qz + (size_t)o * sstride + 1, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
-                    }
-                }
                 __syncwarp();
                 if (lane == 0) atomicExch(cnt + tt, 0);
             }
@@ -655,7 +646,7 @@ size_t gemv_i4mt_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
 {
     if (!gemv_i4mt_eligible(M, N, K, g)) return 0;
     const int64_t ntiles = (N + kTile - 1) / kTile;
-    return i4_slots_bytes(M, N, K, i4_config(M, N, K).grid) + ((size_t)ntiles * 4 + 255) / 256 * 256;
+    return counter_region_bytes(ntiles) + i4_slots_bytes(M, N, K, i4_config(M, N, K).grid);
 }
 
 int launch_gemv_w4a16_i4mt(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
@@ -688,9 +679,11 @@ int launch_gemv_w4a16_i4mt(const uint16_t *x, int64_t M, int64_t N, int64_t K, c
         return -1;
     const I4Config c = i4_config(M, N, K);
     const int max_segs = i4_max_segments(N, K, c.grid);
+    const int64_t ntiles = (N + kTile - 1) / kTile;
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
-    float *ws = reinterpret_cast<float *>(w8);
-    int *cnt = reinterpret_cast<int *>(w8 + i4_slots_bytes(M, N, K, c.grid));
+    int *cnt = reinterpret_cast<int *>(w8);
+    float *ws = reinterpret_cast<float *>(w8 + counter_region_bytes(ntiles));
+    if (clear_extra_counters(workspace, ntiles, st) != cudaSuccess) return -2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)c.grid);
     cfg.blockDim = dim3(kT);

@@ -68,9 +68,8 @@
 //    their slots and bump the tile's arrival counter (a release add, no round
 //    trip); the first segment's combiner keeps its own sums in registers,
 //    waits (bounded) until the counter shows the others, adds their slots in
-//    segment order, clears them, writes y and re-zeroes the counter -- a
-//    fixed order, so results do not depend on timing, and the workspace is
-//    left zero, as it was found.
+//    segment order, writes y and re-zeroes the counter -- a fixed order, so
+//    results do not depend on timing.
 //  * Launched with programmatic dependent launch: in a stream of linears the
 //    next kernel's CTAs start as SMs free up, initialise their barriers and
 //    load their first weight stages into shared memory while this one
@@ -492,15 +491,6 @@ gemv_w4a16_m1_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     for (int j = 0; j < 8; ++j)
                         if (row + j < N) y[row + j] = f32_to_bf16(v[j]);
                 }
-                // leave the slots zero, as the workspace was found: a later call of another shape may place
-                // its arrival counters where these slots are
-                {
-                    float4 *qz = reinterpret_cast<float4 *>(slots + 8 * lane);
-                    for (int o = 1; o < nseg; ++o) {  // segment 0's slot is never written
-                        __stcg(qz + (size_t)o * (kTile / 4), make_float4(0.0f, 0.0f, 0.0f, 0.0f));
-                        __stcg(qz + (size_t)o * (kTile / 4) + 1, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
-                    }
-                }
                 __syncwarp();
                 if (lane == 0) atomicExch(cnt + tt, 0);
             }
@@ -779,7 +769,7 @@ size_t gemv_m1_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
 {
     if (!gemv_m1_eligible(M, N, K, g)) return 0;
     const int64_t ntiles = (N + kTile - 1) / kTile;
-    return m1_slots_bytes(N, K, m1_config(N, K, g).grid) + ((size_t)ntiles * 4 + 255) / 256 * 256;
+    return counter_region_bytes(ntiles) + m1_slots_bytes(N, K, m1_config(N, K, g).grid);
 }
 
 int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
@@ -815,9 +805,11 @@ int launch_gemv_w4a16_m1(const uint16_t *x, int64_t N, int64_t K, const uint8_t 
     const M1Config c = m1_config(N, K, g);
     const int grid = c.grid;
     const int max_segs = m1_max_segments(N, K, grid);
+    const int64_t ntiles = (N + kTile - 1) / kTile;
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
-    float *ws = reinterpret_cast<float *>(w8);
-    int *cnt = reinterpret_cast<int *>(w8 + m1_slots_bytes(N, K, grid));
+    int *cnt = reinterpret_cast<int *>(w8);
+    float *ws = reinterpret_cast<float *>(w8 + counter_region_bytes(ntiles));
+    if (clear_extra_counters(workspace, ntiles, st) != cudaSuccess) return -2;
     // programmatic dependent launch: this grid may start while the previous kernel in the stream finishes;
     // the kernel reads nothing that kernel may write, and writes nothing, before griddepcontrol.wait
     cudaLaunchConfig_t cfg = {};

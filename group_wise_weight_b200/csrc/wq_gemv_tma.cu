@@ -506,7 +506,7 @@ size_t gemv_tma_workspace_bytes(int64_t M, int64_t N, int64_t K, int g)
 {
     if (!gemv_tma_eligible(M, N, K, g)) return 0;
     const int64_t tiles = (N + kTileRows - 1) / kTileRows;
-    return align_up(sizeof(float) * (size_t)(M * N), 256) + align_up(sizeof(int) * (size_t)tiles, 256);
+    return counter_region_bytes(tiles) + align_up(sizeof(float) * (size_t)(M * N), 256);
 }
 
 bool gemv_tma_eligible(int64_t M, int64_t N, int64_t K, int g)
@@ -515,12 +515,31 @@ bool gemv_tma_eligible(int64_t M, int64_t N, int64_t K, int g)
     return g == 128 && M >= 2 && M <= 16 && N >= kTileRows && K >= 256 && K / 128 <= 0x7fffffff / 64;
 }
 
-int launch_gemv_w4a16_tma(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
-                          const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st)
+size_t gemv_tma_compact_bytes(int64_t M, int64_t N, int64_t K, int g)
 {
-    float *ws = static_cast<float *>(workspace);
-    int *counters = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) +
-                                            align_up(sizeof(float) * (size_t)(M * N), 256));
+    if (!gemv_tma_eligible(M, N, K, g)) return 0;
+    const int64_t tiles = (N + kTileRows - 1) / kTileRows;
+    return align_up(sizeof(float) * (size_t)(M * N), 256) + align_up(sizeof(int) * (size_t)tiles, 256);
+}
+
+int launch_gemv_w4a16_tma(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
+                          const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st, bool compact)
+{
+    const int64_t tiles = (N + kTileRows - 1) / kTileRows;
+    uint8_t *w8 = static_cast<uint8_t *>(workspace);
+    int *counters;
+    float *ws;
+    if (compact) {  // a private scratch area cleared before every call: partial sums first, counters after
+        ws = reinterpret_cast<float *>(w8);
+        counters = reinterpret_cast<int *>(w8 + align_up(sizeof(float) * (size_t)(M * N), 256));
+    } else {
+        counters = reinterpret_cast<int *>(w8);
+        ws = reinterpret_cast<float *>(w8 + counter_region_bytes(tiles));
+        if (clear_extra_counters(workspace, tiles, st) != cudaSuccess) return -2;
+        // the partial sums meet in binary32 atomics, so they must start at zero; in a workspace shared with
+        // other shapes this region may hold their partial sums
+        if (cudaMemsetAsync(ws, 0, sizeof(float) * (size_t)(M * N), st) != cudaSuccess) return -2;
+    }
     const bool xsmem = (size_t)M * (size_t)K * 2 <= 32 * 1024;
     const bool even = ((K / 128) & 1) == 0;
 #define WQ_RUN(NT, XS, EV) return run<NT, XS, EV>(x, M, N, K, q, s, z, y, ws, counters, status, st)

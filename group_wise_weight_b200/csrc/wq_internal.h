@@ -6,6 +6,24 @@
 
 namespace wq {
 
+// Workspace layout of every kernel that splits tiles between CTAs: the per-tile arrival counters first, in a
+// region of counter_region_bytes(tiles) (4 bytes a tile, rounded up to 64 KB), then the binary32 partial sums.
+// A call that completes normally re-zeroes its counters and leaves its partial sums behind; since every shape
+// with up to 16,384 tiles keeps its counters below 64 KB and its partial sums above, one workspace can serve
+// calls of any shapes in turn.  A shape with more tiles has counters above 64 KB, where another shape's partial
+// sums may lie: clear_extra_counters() zeroes them on the stream before its launch.
+constexpr size_t kCounterRegion = 65536;
+inline size_t counter_region_bytes(int64_t tiles)
+{
+    return ((size_t)tiles * 4 + kCounterRegion - 1) / kCounterRegion * kCounterRegion;
+}
+inline cudaError_t clear_extra_counters(void *workspace, int64_t tiles, cudaStream_t st)
+{
+    const size_t region = counter_region_bytes(tiles);
+    if (region <= kCounterRegion) return cudaSuccess;
+    return cudaMemsetAsync(static_cast<uint8_t *>(workspace) + kCounterRegion, 0, region - kCounterRegion, st);
+}
+
 // y [M][N] bf16 overlaps x [M][K] bf16, the codes, the scales or the zero-points (wq_api.cu).
 bool output_overlaps_inputs(const void *x, int64_t M, int64_t N, int64_t K, const void *q, const void *s,
                             const void *z, int g, const void *y, bool int8);
@@ -75,13 +93,17 @@ int launch_gemv_w8a16_int(const uint16_t *x, int64_t M, int64_t N, int64_t K, co
                           uint16_t *y, void *workspace, int *status, cudaStream_t st);
 
 // TMA-pipelined W4A16 for group 128 and M <= 16 (wq_gemv_tma.cu).  Needs a
-// workspace of gemv_tma_workspace_bytes() (zero-filled before first use; the
-// kernel leaves it zeroed).  Returns 0, or -1 if the tensor map could not be
-// encoded.
+// workspace of gemv_tma_workspace_bytes() (counters first, zero-filled before
+// first use; the launcher clears the partial sums, which meet in atomics),
+// or, compact = true, a private scratch area of gemv_tma_compact_bytes()
+// cleared before every call (partial sums first).  Returns 0, -1 if the tensor map could not be
+// encoded, -2 if clearing counters failed.
 bool gemv_tma_eligible(int64_t M, int64_t N, int64_t K, int g);
 size_t gemv_tma_workspace_bytes(int64_t M, int64_t N, int64_t K, int g);
+size_t gemv_tma_compact_bytes(int64_t M, int64_t N, int64_t K, int g);
 int launch_gemv_w4a16_tma(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *q, const uint16_t *s,
-                          const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st);
+                          const uint16_t *z, uint16_t *y, void *workspace, int *status, cudaStream_t st,
+                          bool compact = false);
 
 // tcgen05 W4A16 for M > 16 (wq_gemm_tc.cu): N >= 128, K % 128 == 0.  Workspace
 // of gemm_tc_workspace_bytes(): per-segment binary32 partials and per-tile

@@ -73,7 +73,7 @@ extern "C" int wq_gemm_w4a16_noalloc(const uint16_t *x, int64_t M, int64_t N, in
         return wq::record_error(WQ_ERR_ALIGN, "wq_gemm_w4a16_noalloc: pointers must be 16-byte aligned");
     if (wq::output_overlaps_inputs(x, M, N, K, qweight, scales, zeros, g, y, false))
         return wq::record_error(WQ_ERR_ARG, "wq_gemm_w4a16_noalloc: y overlaps x, the codes, the scales or the zero-points");
-    const size_t need = wq::gemv_tma_workspace_bytes(M, N, K, g);
+    const size_t need = wq::gemv_tma_compact_bytes(M, N, K, g);
     if (need > kScratchBytes) {
         char msg[256];
         snprintf(msg, sizeof msg,
@@ -90,7 +90,7 @@ extern "C" int wq_gemm_w4a16_noalloc(const uint16_t *x, int64_t M, int64_t N, in
     // partial sums and tile counters must start at zero
     if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess)
         return wq::record_error(WQ_ERR_CUDA, "wq_gemm_w4a16_noalloc: clearing the scratch array failed");
-    if (wq::launch_gemv_w4a16_tma(x, M, N, K, qweight, scales, zeros, y, scratch, status, st) != 0)
+    if (wq::launch_gemv_w4a16_tma(x, M, N, K, qweight, scales, zeros, y, scratch, status, st, true) != 0)
         return wq::record_error(WQ_ERR_CUDA, "wq_gemm_w4a16_noalloc: tensor map encoding failed");
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {

@@ -155,15 +155,16 @@ int wq_quantize_int8(const void *w, int wtype, int64_t N, int64_t K, int64_t ldw
 /*
  * Bytes of device workspace wq_gemm_w4a16 (wbits = 4) or wq_gemm_w8a16
  * (wbits = 8) needs for this shape; 0 when the chosen kernel needs none.
- * The workspace holds binary32 partial sums of a K-split and per-tile
- * arrival counters, at offsets that depend on the shape; a call that
- * completes normally leaves every byte it used zero again (partial sums and
- * counters alike), so a workspace must be zero-filled once before its first
- * use and may then be reused by later calls on the same stream, of this or
- * any other shape and kernel, as long as it is large enough for each.  A call
- * whose kernel gave up on a bounded wait (wq_device_status returns
- * WQ_ERR_DEVICE_TIMEOUT) can leave non-zero bytes behind: zero-fill the
- * workspace again before reusing it after such a status.
+ * The workspace holds per-tile arrival counters, in its first 64 KB (a
+ * multiple of 64 KB for shapes of more than 16,384 tiles, whose counters
+ * above 64 KB the call clears first), and the binary32 partial sums of a
+ * K-split above them.  A call that completes normally re-zeroes its counters,
+ * so a workspace must be zero-filled once before its first use and may then
+ * be reused by later calls on the same stream, of this or any other shape and
+ * kernel, as long as it is large enough for each.  A call whose kernel gave
+ * up on a bounded wait (wq_device_status returns WQ_ERR_DEVICE_TIMEOUT) can
+ * leave counters non-zero: zero-fill the workspace again before reusing it
+ * after such a status.
  */
 size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits);
 
@@ -257,8 +258,8 @@ int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8
  * with the weights quantised by wq_quantize_int4_scaled with the same
  * col_scale (binary32 [K], device, 16-byte aligned) and x / col_scale an IEEE
  * binary32 quotient rounded to bf16.  The M = 1 decode kernel divides while
- * it stages x (no extra pass); other shapes write the scaled activations to
- * the front of the workspace first.  Arguments, accuracy and the rest of the
+ * it stages x (no extra pass); other shapes first write the scaled
+ * activations behind the matmul's part of the workspace.  Arguments, accuracy and the rest of the
  * contract as wq_gemm_w4a16, with a workspace of
  * wq_gemm_w4a16_colscaled_workspace_bytes(M, N, K, g) bytes that must not
  * overlap x or y.
