@@ -61,6 +61,21 @@ namespace wq {
 
 namespace {
 
+// Device-scope add with release semantics (no value returned): the writes that happen before it (this
+// thread's, and through the preceding CTA barrier and fences the other threads') are visible before the add.
+__device__ __forceinline__ void red_add_release(int *p, int v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Device-scope load with acquire semantics: later reads see what was written before the matching release.
+__device__ __forceinline__ int ld_acquire(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 constexpr int kTileN = 128;     // weight rows per tile (MMA M)
 constexpr int kBN = 128;        // activation rows per tile (MMA N)
 constexpr int kStageK = 128;    // k per stage = one group
@@ -541,20 +556,39 @@ gemm_w4a16_tc2_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_con
                     return reinterpret_cast<float4 *>(ws) +
                            ((tile * max_segs + o) * (kBN / 4) + ch * 16 + q) * kTileN + r;
                 };
+                // The CTA of the tile's first segment combines it: that segment ends its range, while the tile's
+                // last segment starts the next CTA's, so it is usually among the last to finish.  The others write
+                // their slots and add their stage counts with release semantics (no round trip); the first
+                // keeps its sums in registers and waits (bounded) until the counter shows every other stage.
+                if (my_seg != 0) {
 #pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    *seg_ptr(my_seg, q) = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
-                __threadfence();
-                named_bar_sync(1, kPrWarps * 32);
+                    for (int q = 0; q < 16; ++q)
+                        *seg_ptr(my_seg, q) = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+                    __threadfence();
+                    named_bar_sync(1, kPrWarps * 32);
+                    if (ptid == 0) red_add_release(counters + tile, ks1 - ks0);
+                    u += ks1 - ks0;
+                    continue;
+                }
                 if (ptid == 0) {
-                    const int add = ks1 - ks0;
-                    const int prev = atomicAdd(counters + tile, add);
-                    *last_flag = (prev + add == spt) ? 1 : 0;
+                    const int others = spt - (ks1 - ks0);
+                    int arrived = 1;
+                    const uint64_t t0 = global_ns();
+                    while (ld_acquire(counters + tile) != others) {
+                        if (*abort_flag) { arrived = 0; break; }
+                        if (global_ns() - t0 > kWaitLimitNs) {
+                            record_timeout(status);
+                            *abort_flag = 1;
+                            arrived = 0;
+                            break;
+                        }
+                    }
+                    *last_flag = arrived;
                 }
                 named_bar_sync(1, kPrWarps * 32);
                 if (*last_flag) {
-                    // sum the segments in segment order, whichever CTA finishes last; 16 columns at a time, the
-                    // next segment's values requested before the current ones are added
+                    // sum the segments in segment order (this CTA's own first, from registers); 16 columns at a
+                    // time, the next segment's values requested before the current ones are added
                     __threadfence();
 #pragma unroll
                     for (int c0 = 0; c0 < 64; c0 += 16) {
