@@ -99,11 +99,19 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-__device__ __forceinline__ int atom_add_acq_rel(int *p, int v)
+// Device-scope add with release semantics (no value returned): the writes that happen before it (this
+// thread's, and through the preceding warp barrier the other lanes') are visible before the add is.
+__device__ __forceinline__ void red_add_release(int *p, int v)
 {
-    int old;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Device-scope load with acquire semantics: later reads see what was written before the matching release.
+__device__ __forceinline__ int ld_acquire(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 __host__ __device__ __forceinline__ int cta_of(int64_t u, int64_t units, int64_t B)
@@ -258,28 +266,57 @@ gemv_w8a16_int_kernel(const __grid_constant__ CUtensorMap wmap, const uint16_t *
             const int c_first = cta_of(tt * G, units, B);
             const int nseg = cta_of(tt * G + G - 1, units, B) - c_first + 1;
             float *slots = ws + (size_t)tt * max_segs * M * kTile;  // [segment][m][256]
-            float *mine = slots + (size_t)(bid - c_first) * M * kTile + 8 * lane;
             const float *src = part + (size_t)b * M * kTile + 8 * lane;
-            for (int m = 0; m < M; ++m) {
-                const float4 v0 = *reinterpret_cast<const float4 *>(src + m * kTile);
-                const float4 v1 = *reinterpret_cast<const float4 *>(src + m * kTile + 4);
-                reinterpret_cast<float4 *>(mine + m * kTile)[0] = v0;
-                reinterpret_cast<float4 *>(mine + m * kTile)[1] = v1;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&pempty[b]);  // the shared tile is copied out: free it
             ++pseg;
-            int last = 0;
-            if (lane == 0) last = (atom_add_acq_rel(cnt + tt, 1) + 1 == nseg) ? 1 : 0;
-            last = __shfl_sync(0xffffffffu, last, 0);
-            if (last) {
-                // sum the segments' slots in segment order (independent of which CTA arrived last)
+            // The CTA of the tile's first segment combines it: that segment ends its range (so it is this CTA's
+            // last), while the tile's last segment starts the next CTA's.  The others copy their sums to their
+            // slots and publish them with a release add (no round trip); the first keeps its own in the shared
+            // tile and waits (bounded) until the counter shows the others.
+            if (bid != c_first) {
+                float *mine = slots + (size_t)(bid - c_first) * M * kTile + 8 * lane;
+                for (int m = 0; m < M; ++m) {
+                    const float4 v0 = *reinterpret_cast<const float4 *>(src + m * kTile);
+                    const float4 v1 = *reinterpret_cast<const float4 *>(src + m * kTile + 4);
+                    reinterpret_cast<float4 *>(mine + m * kTile)[0] = v0;
+                    reinterpret_cast<float4 *>(mine + m * kTile)[1] = v1;
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&pempty[b]);  // the shared tile is copied out: free it
+                    red_add_release(cnt + tt, 1);
+                }
+                continue;
+            }
+            int arrived = 1;
+            if (lane == 0) {
+                const uint64_t t0 = global_ns();
+                while (ld_acquire(cnt + tt) != nseg - 1) {
+                    if (flags[0] != 0) { arrived = 0; break; }
+                    if (global_ns() - t0 > kWaitLimitNs) {
+                        record_timeout(status);
+                        flags[0] = 1;
+                        arrived = 0;
+                        break;
+                    }
+                }
+            }
+            // the other lanes read the slots after lane 0's acquire (ordered by the warp barrier)
+            if (!__shfl_sync(0xffffffffu, arrived, 0)) {
+                if (lane == 0) mbar_arrive(&pempty[b]);
+                break;
+            }
+            {
+                // sum the segments in segment order, from 0: this CTA's own (segment 0, in the shared tile), then
+                // the slots of the others
                 const int64_t row = tt * kTile + 8 * lane;
                 const size_t sstride = (size_t)M * (kTile / 4);  // float4 between segments
                 for (int m = 0; m < M; ++m) {
-                    float v[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+                    const float4 s0 = *reinterpret_cast<const float4 *>(src + m * kTile);
+                    const float4 s1 = *reinterpret_cast<const float4 *>(src + m * kTile + 4);
+                    float v[8] = {0.0f + s0.x, 0.0f + s0.y, 0.0f + s0.z, 0.0f + s0.w,
+                                  0.0f + s1.x, 0.0f + s1.y, 0.0f + s1.z, 0.0f + s1.w};
                     const float4 *q = reinterpret_cast<const float4 *>(slots + (size_t)m * kTile + 8 * lane);
-                    int o = 0;
+                    int o = 1;
                     for (; o + 4 <= nseg; o += 4) {
                         float4 a[8];
 #pragma unroll
@@ -313,7 +350,10 @@ gemv_w8a16_int_kernel(const __grid_constant__ CUtensorMap wmap, const uint16_t *
                     }
                 }
                 __syncwarp();
-                if (lane == 0) atomicExch(cnt + tt, 0);
+                if (lane == 0) {
+                    mbar_arrive(&pempty[b]);  // the shared tile is summed: free it
+                    atomicExch(cnt + tt, 0);
+                }
             }
         }
         __syncthreads();
