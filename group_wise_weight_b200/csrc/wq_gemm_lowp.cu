@@ -50,6 +50,21 @@ namespace wq {
 
 namespace {
 
+// Device-scope add with release semantics (no value returned): the writes that happen before it (this
+// thread's, and through the preceding CTA barrier and fences the other threads') are visible before the add.
+__device__ __forceinline__ void red_add_release(int *p, int v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Device-scope load with acquire semantics: later reads see what was written before the matching release.
+__device__ __forceinline__ int ld_acquire(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 constexpr int kTileN = 128;     // weight rows per tile (MMA M)
 constexpr int kRowBytes = 128;  // bytes of K per row and stage (one 128-byte swizzle row)
 constexpr int kThreads = 192;   // warp 0: copies, warp 1: MMA, warps 2..5: epilogue
@@ -326,25 +341,43 @@ gemm_lowp_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant
                 const int64_t cta_first = sc.cta_of(tile * spt);
                 const int64_t my_seg = (int64_t)blockIdx.x - cta_first;
                 const int64_t nseg = sc.cta_of(tile * spt + spt - 1) - cta_first + 1;
-                float *slot = p.part + ((tile * p.max_segs + my_seg) * BN) * kTileN;
+                // The CTA of the tile's first segment combines it: that segment ends its range, while the tile's
+                // last segment starts the next CTA's, so it is usually among the last to finish.  The others
+                // write their slots and add their stage counts with release semantics (no round trip); the
+                // first keeps its sums in tensor memory and waits (bounded) until the counter shows every other
+                // stage.
+                if (my_seg != 0) {
+                    float *slot = p.part + ((tile * p.max_segs + my_seg) * BN) * kTileN;
 #pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(d_addr + (uint32_t)c0, v);
-                    tmem_wait_ld();
+                    for (int c0 = 0; c0 < BN; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(d_addr + (uint32_t)c0, v);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) slot[(int64_t)(c0 + c) * kTileN + r] = __uint_as_float(v[c]);
-                }
-                __threadfence();
-                named_bar_sync(1, 128);
+                        for (int c = 0; c < 32; ++c) slot[(int64_t)(c0 + c) * kTileN + r] = __uint_as_float(v[c]);
+                    }
+                    __threadfence();
+                    named_bar_sync(1, 128);
+                    if (tid == kEpiWarp0 * 32) red_add_release(p.counters + tile, ks1 - ks0);
+                } else {
                 if (tid == kEpiWarp0 * 32) {
-                    const int add = ks1 - ks0;
-                    const int prev = atomicAdd(p.counters + tile, add);
-                    *last_flag = (prev + add == spt) ? 1 : 0;
+                    const int others = spt - (ks1 - ks0);
+                    int arrived = 1;
+                    const uint64_t t0 = global_ns();
+                    while (ld_acquire(p.counters + tile) != others) {
+                        if (*abort_flag) { arrived = 0; break; }
+                        if (global_ns() - t0 > kWaitLimitNs) {
+                            record_timeout(status);
+                            *abort_flag = 1;
+                            arrived = 0;
+                            break;
+                        }
+                    }
+                    *last_flag = arrived;
                 }
                 named_bar_sync(1, 128);
                 if (*last_flag) {
-                    // sum the segments in segment order, whichever CTA arrives last
+                    // sum the segments in segment order (this CTA's own first, from tensor memory)
                     __threadfence();
 #pragma unroll 1
                     for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -369,6 +402,7 @@ gemm_lowp_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant
                     }
                     named_bar_sync(1, 128);
                     if (tid == kEpiWarp0 * 32) atomicExch(p.counters + tile, 0);
+                }
                 }
             }
             tc_fence_before();
