@@ -245,7 +245,9 @@ int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint
  * bf16, binary32 accumulation per group of g, or per 128 k for g = K, scaled
  * and summed in binary32); otherwise a CUDA-core kernel.  Workspace of
  * wq_gemm_workspace_bytes(M, N, K, g, 8) bytes.  Other arguments and
- * guarantees as wq_gemm_w4a16 (y is deterministic for every M here).
+ * guarantees as wq_gemm_w4a16 (y is deterministic for every M here), the
+ * integer kernel's split tiles combined by the CTA of their first segment as
+ * there.
  */
 int wq_gemm_w8a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const int8_t *qweight,
                   const uint16_t *scales, int g, uint16_t *y, void *workspace, size_t ws_bytes,
@@ -351,6 +353,8 @@ size_t wq_gemm_w8a8_fp8_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * Requirements: M, N >= 1; K >= 128, K % 128 == 0; xq, wq, wscales, y 16-byte
  * aligned, xscale 4-byte aligned; workspace of
  * wq_gemm_w8a8_fp8_workspace_bytes bytes; y must not overlap an input.
+ * Split tiles are combined by the CTA of their first segment, as described
+ * under wq_gemm_w4a16.
  */
 int wq_gemm_w8a8_fp8(const uint8_t *xq, const float *xscale, int64_t M, int64_t N, int64_t K, const uint8_t *wq,
                      const float *wscales, uint16_t *y, void *workspace, size_t ws_bytes, void *stream);
@@ -400,6 +404,8 @@ size_t wq_gemm_nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * Requirements: M, N >= 1; K >= 256, K % 256 == 0; every pointer 16-byte
  * aligned except the two tensor scales (4-byte); workspace of
  * wq_gemm_nvfp4_workspace_bytes bytes; y must not overlap an input.
+ * Split tiles are combined by the CTA of their first segment, as described
+ * under wq_gemm_w4a16.
  */
 int wq_gemm_nvfp4(const uint8_t *x_codes, const uint8_t *x_block_scales, const float *x_tensor_scale, int64_t M,
                   int64_t N, int64_t K, const uint8_t *w_codes, const uint8_t *w_block_scales,
