@@ -247,7 +247,8 @@ class Model:
         torch.cuda.empty_cache()
         self.quant_ms, self.quant_bytes = quant_ms, quant_bytes
         self.weights = sum(K * N for _, K, N, *_ in self.linears)
-        # one workspace serves every call: calls run in order on one stream and each leaves it zeroed
+        # one workspace serves every call: calls run in order on one stream, each re-zeroes its tile counters,
+        # and every kernel keeps those in the workspace's first 64 KB, below any partial sums
         need = max(wq.wq_gemm_workspace_bytes(M, N, K, G, 4) for M in (1, 128) for _, K, N, *_ in self.linears)
         self.ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=device)
 

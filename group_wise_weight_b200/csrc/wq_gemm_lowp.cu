@@ -36,9 +36,10 @@
 // MMAs, warps 2..5 read D back (one 32-lane quarter of tensor memory each),
 // scale it and write y.  Stream-K over (tile, stage) units gives every SM the
 // same number of stages; a tile split between CTAs leaves one binary32
-// partial per segment in the workspace, and the CTA that completes the tile
-// sums the segments in segment order (so results do not depend on timing)
-// and writes y.  Every barrier wait is bounded.
+// partial per segment in the workspace, and the CTA of the tile's first
+// segment waits (bounded) for the others, sums the segments in segment order
+// (so results do not depend on timing) and writes y.  Every barrier wait is
+// bounded.
 #include <algorithm>
 #include <map>
 #include <mutex>
@@ -337,7 +338,6 @@ gemm_lowp_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant
                     }
                 }
             } else {
-                // this segment's partial -> its workspace slot; the CTA that completes the tile sums them
                 const int64_t cta_first = sc.cta_of(tile * spt);
                 const int64_t my_seg = (int64_t)blockIdx.x - cta_first;
                 const int64_t nseg = sc.cta_of(tile * spt + spt - 1) - cta_first + 1;
