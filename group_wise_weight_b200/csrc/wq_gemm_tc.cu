@@ -56,6 +56,21 @@ namespace wq {
 
 namespace {
 
+// Device-scope add with release semantics (no value returned): the writes that happen before it (this
+// thread's, and through the preceding CTA barrier and fences the other threads') are visible before the add.
+__device__ __forceinline__ void red_add_release(int *p, int v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Device-scope load with acquire semantics: later reads see what was written before the matching release.
+__device__ __forceinline__ int ld_acquire(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 constexpr int kTileN = 128;         // weight rows per tile (MMA M)
 constexpr int kStageK = 128;        // k per stage
 constexpr int kWStages = 8;          // weight boxes in flight (released by the dequant warps)
@@ -535,24 +550,51 @@ gemm_w4a16_tc_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                         if (mbase + c < M) y[(mbase + c) * N + n] = f32_to_bf16(acc[c]);
                 }
             } else {
-                // partial of this segment -> workspace slot; the CTA that completes the tile sums them
+                // 32- and 64-column tiles: the CTA of the tile's first segment combines it (that segment ends its
+                // range, while the tile's last segment starts the next CTA's, so it is usually among the last to
+                // finish); the others write their slots and add their stage counts with release semantics, and
+                // the first keeps its sums in registers and waits (bounded) until the counter shows every other
+                // stage.  128-column tiles: the CTA that completes the tile combines it (the first-segment wait
+                // measured much slower in this form).
+                constexpr bool kFirstCombines = BN < 128;
                 const int64_t cta_first = S.cta_of(tile * spt);
                 const int64_t my_seg = (int64_t)blockIdx.x - cta_first;
                 const int64_t cta_last = S.cta_of(tile * spt + spt - 1);
-                float *slot = ws + ((tile * max_segs + my_seg) * BN) * kTileN;
+                if (!kFirstCombines || my_seg != 0) {
+                    float *slot = ws + ((tile * max_segs + my_seg) * BN) * kTileN;
 #pragma unroll
-                for (int c = 0; c < kCols; ++c) slot[(int64_t)(kq * kCols + c) * kTileN + r] = acc[c];
-                __threadfence();
-                named_bar_sync(1, kDequantWarps * 32);
-                if (tid == kFirstDequantWarp * 32) {
-                    const int add = ks1 - ks0;
-                    const int prev = atomicAdd(counters + tile, add);
-                    *last_flag = (prev + add == spt) ? 1 : 0;
+                    for (int c = 0; c < kCols; ++c) slot[(int64_t)(kq * kCols + c) * kTileN + r] = acc[c];
+                    __threadfence();
+                    named_bar_sync(1, kDequantWarps * 32);
+                    if (tid == kFirstDequantWarp * 32) {
+                        const int add = ks1 - ks0;
+                        if (kFirstCombines) {
+                            red_add_release(counters + tile, add);
+                            *last_flag = 0;
+                        } else {
+                            const int prev = atomicAdd(counters + tile, add);
+                            *last_flag = (prev + add == spt) ? 1 : 0;
+                        }
+                    }
+                } else if (tid == kFirstDequantWarp * 32) {
+                    const int others = spt - (ks1 - ks0);
+                    int arrived = 1;
+                    const uint64_t t0 = global_ns();
+                    while (ld_acquire(counters + tile) != others) {
+                        if (*abort_flag) { arrived = 0; break; }
+                        if (global_ns() - t0 > kWaitLimitNs) {
+                            record_timeout(status);
+                            *abort_flag = 1;
+                            arrived = 0;
+                            break;
+                        }
+                    }
+                    *last_flag = arrived;
                 }
                 named_bar_sync(1, kDequantWarps * 32);
                 if (*last_flag) {
-                    // sum the segments in segment order whichever CTA finishes last, so
-                    // repeated calls round identically
+                    // sum the segments in segment order (this CTA's own from registers), so repeated calls round
+                    // identically
                     __threadfence();
                     float tot[kCols];
 #pragma unroll
