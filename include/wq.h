@@ -221,11 +221,12 @@ size_t wq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int g, int wbits
  * those must not have been written by the kernel just before on the same
  * stream (the y or workspace of the previous call, or the quantiser that
  * produced them: put another operation or an event between).
- * The M = 1 kernel and the tensor-core kernel for M > 64, g = 128 run at most
- * one CTA per SM, and a tile split between CTAs is combined by the CTA of its
- * first segment, which waits for the others: a kernel on another stream that
- * holds SMs for good would make that wait run out (WQ_ERR_DEVICE_TIMEOUT
- * from wq_device_status after 1 s) rather than hang.
+ * The persistent M = 1 kernel and the tensor-core kernels (except the
+ * 128-column form of the one used for g = 32 or 64, or K % 1024 != 0) run at
+ * most one CTA per SM and have a tile split between CTAs combined by the CTA
+ * of its first segment, which waits for the others: a kernel on another
+ * stream that holds SMs for good would make that wait run out
+ * (WQ_ERR_DEVICE_TIMEOUT from wq_device_status after 1 s) rather than hang.
  */
 int wq_gemm_w4a16(const uint16_t *x, int64_t M, int64_t N, int64_t K, const uint8_t *qweight,
                   const uint16_t *scales, const uint16_t *zeros, int g, uint16_t *y,
