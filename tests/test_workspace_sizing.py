@@ -140,3 +140,25 @@ def _w8int_needed(M, N, K):
                                    (5, 8192, 8192), (8, 10240, 8192), (16, 8192, 8192), (16, 57344, 8192)])
 def test_w8int_workspace_covers_every_segment(M, N, K):
     assert wq.wq_gemm_workspace_bytes(M, N, K, K, 8) >= _w8int_needed(M, N, K)
+
+
+COUNTER_REGION = 65536
+
+
+@pytest.mark.parametrize("N,K", [(10240, 8192), (8192, 8192), (57344, 8192), (8192, 28672), (300000, 1024),
+                                 (4200000, 1024)])
+def test_tile_counters_sit_below_the_partial_sums(N, K):
+    """Every kernel that splits tiles keeps its arrival counters in the workspace's first 64 KB (more for a
+    shape of over 16,384 tiles) and its partial sums above them, so that one workspace can serve calls of any
+    shapes in turn (a call leaves its partial sums behind but re-zeroes its counters).  The size asked for is
+    therefore the counter region plus the partial sums: M = 1 INT4, M = 128 INT4 (128 x 128 tiles) and M = 1
+    W8A16 per channel."""
+    nt256 = math.ceil(N / 256)
+    region = max(COUNTER_REGION, math.ceil(nt256 * 4 / COUNTER_REGION) * COUNTER_REGION)
+    assert wq.wq_gemm_workspace_bytes(1, N, K, 128, 4) >= region + _m1_needed(N, K) - nt256 * 4
+    tiles128 = math.ceil(N / 128)
+    region128 = max(COUNTER_REGION, math.ceil(tiles128 * 4 / COUNTER_REGION) * COUNTER_REGION)
+    assert wq.wq_gemm_workspace_bytes(128, N, K, 128, 4) >= region128 + _tc_needed(128, N, K, 128) - tiles128 * 4
+    w8 = _w8int_needed(1, N, K)
+    if w8:
+        assert wq.wq_gemm_workspace_bytes(1, N, K, K, 8) >= region + w8 - nt256 * 4
