@@ -97,3 +97,35 @@ def test_one_workspace_serves_every_shape_and_kernel():
                 assert torch.equal(y.view(torch.int16), y2.view(torch.int16)), f"{name} (pass {rep}): y differs"
             else:
                 assert torch.allclose(y.float(), y2.float(), rtol=1e-2, atol=1e-2), f"{name} (pass {rep}): y differs"
+
+
+def test_more_than_16384_tiles_after_a_smaller_shape():
+    """A shape of more than 16,384 tiles keeps counters above 64 KB, where an earlier call's partial sums lie:
+    the library clears them before its launch.  M = 1, N = 4,325,376 (16,896 tiles of 256 rows), K = 1024,
+    with random codes, scales and zero-points (no quantiser pass over a 8.6 GB weight), after a smaller M = 1
+    call on the same workspace; y must equal the same call on a fresh workspace bit for bit."""
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(4242)
+    ntiles = 16896
+    N, K = 256 * ntiles, 1024
+    q = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g)
+    s = (0.001 + 0.01 * torch.rand((N, K // 128), device=dev, generator=g)).to(torch.bfloat16)
+    z = torch.randint(0, 16, (N, K // 128), device=dev, generator=g).to(torch.bfloat16)
+    x = wq_inputs.activations(1, K, 4243, device=dev)
+    need = wq.wq_gemm_workspace_bytes(1, N, K, 128, 4)
+    assert need > 2 * COUNTER_REGION  # the counter region reaches past 64 KB
+    qs, ss, zs = _w4(20000, 8192, 128, 4244, dev)
+    xs = wq_inputs.activations(1, 8192, 4245, device=dev)
+    small_need = wq.wq_gemm_workspace_bytes(1, 20000, 8192, 128, 4)
+    shared = torch.zeros(max(need, small_need) + 256, dtype=torch.uint8, device=dev)
+    wq.wq_gemm_w4a16(xs, qs, ss, zs, 128, workspace=shared)  # leaves partial sums above 64 KB
+    torch.cuda.synchronize()
+    # the big call's counters beyond 64 KB lie on the smaller call's partial sums
+    assert int(torch.count_nonzero(shared[COUNTER_REGION:ntiles * 4]).item()) > 0
+    y = wq.wq_gemm_w4a16(x, q, s, z, 128, workspace=shared)
+    torch.cuda.synchronize()
+    assert wq.wq_device_status() == wq.WQ_OK
+    fresh = torch.zeros(need, dtype=torch.uint8, device=dev)
+    y2 = wq.wq_gemm_w4a16(x, q, s, z, 128, workspace=fresh)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
